@@ -1,0 +1,549 @@
+// pi_host.cu -- host side of the C ABI declared in include/pi_ffn.h.
+//
+// Validates every call before enqueuing work, owns the per-layer device
+// memory (weights in neuron-table order) and the per-handle scratch, builds
+// the neuron tables, and launches the decode kernel (pi_decode.cu) and the
+// prefill kernels (pi_prefill.cu).
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <numeric>
+#include <vector>
+
+#include "../../include/pi_ffn.h"
+#include "pi_internal.h"
+#include "pi_prefill.h"
+
+namespace {
+
+thread_local char g_msg[512] = "no error";
+
+pi_status fail(pi_status st, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+pi_status cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(e == cudaErrorMemoryAllocation ? PI_ERR_OOM : PI_ERR_CUDA, "%s: %s (%s)", what,
+                cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+#define PI_CUDA(call, what)                                   \
+    do {                                                      \
+        cudaError_t e_ = (call);                              \
+        if (e_ != cudaSuccess) return cuda_fail(e_, what);    \
+    } while (0)
+
+int fmt_of(pi_dtype t)
+{
+    switch (t) {
+    case PI_F32: return pi::kF32;
+    case PI_F16: return pi::kF16;
+    case PI_BF16: return pi::kBF16;
+    case PI_INT4G32: return pi::kI4;
+    }
+    return -1;
+}
+
+int elem_bytes(pi_dtype t) { return t == PI_F32 ? 4 : 2; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+struct pi_ffn {
+    pi_ffn_desc desc{};
+    int S = 0;                       // strips = CTAs of the decode kernel
+    int wfmt = 0, pfmt = 0, gated = 0;
+    int vrow = 0, urow = 0, wrow = 0;
+    int np = 0, ng = 0;
+    size_t smem = 0;
+    std::vector<int32_t> strip_off;
+    std::vector<std::vector<int32_t>> perm;   // [layer * E + e]
+    std::vector<uint8_t *> mem;               // [layer * E + e]
+    std::vector<uint8_t *> router_mem;        // [layer]
+    std::vector<char> loaded;                 // [layer]
+    std::vector<pi::ExpertDev> h_ex;          // [layer * E]
+    pi::ExpertDev *d_ex = nullptr;
+    const uint8_t **d_router = nullptr;
+    int32_t *d_strip_off = nullptr;
+    // scratch
+    uint8_t *scratch = nullptr;
+    float *t_buf = nullptr, *partials = nullptr, *io = nullptr;
+    int32_t *lists = nullptr, *counts = nullptr;
+    unsigned *bar = nullptr;
+    int *err = nullptr;
+    long long wait_ns = 2000000000LL;
+    int debug_flags = 0;
+    pi::PrefillState *prefill = nullptr;
+};
+
+extern "C" {
+
+const char *pi_last_error(void) { return g_msg; }
+
+pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
+{
+    if (!desc || !out) return fail(PI_ERR_INVALID_ARG, "pi_ffn_create: null argument");
+    *out = nullptr;
+    const pi_ffn_desc &D = *desc;
+    if (D.n_layers < 1) return fail(PI_ERR_INVALID_ARG, "n_layers must be >= 1");
+    if (D.d_model < 256 || D.d_model % 256 != 0 || D.d_model > 8192)
+        return fail(PI_ERR_INVALID_ARG, "d_model must be a multiple of 256 in [256, 8192]");
+    if (D.w_dtype == PI_F32 && D.d_model > 4096)
+        return fail(PI_ERR_UNSUPPORTED, "F32 weights need d_model <= 4096");
+    if (D.d_ff < 1) return fail(PI_ERR_INVALID_ARG, "d_ff must be >= 1");
+    if (D.act < PI_ACT_RELU || D.act > PI_ACT_DRELU) return fail(PI_ERR_INVALID_ARG, "bad act");
+    if (fmt_of(D.w_dtype) < 0) return fail(PI_ERR_INVALID_ARG, "bad w_dtype");
+    if (D.pred_dtype != PI_F32 && D.pred_dtype != PI_F16 && D.pred_dtype != PI_BF16)
+        return fail(PI_ERR_INVALID_ARG, "pred_dtype must be F32, F16 or BF16");
+    const bool pair_ok = (D.w_dtype == PI_F32 && D.pred_dtype == PI_F32) ||
+                         (D.w_dtype == PI_F16 && D.pred_dtype == PI_F16) ||
+                         (D.w_dtype == PI_BF16 && D.pred_dtype == PI_BF16) ||
+                         (D.w_dtype == PI_INT4G32 && D.pred_dtype != PI_F32);
+    if (!pair_ok)
+        return fail(PI_ERR_UNSUPPORTED,
+                    "supported (w_dtype, pred_dtype): (F32,F32) (F16,F16) (BF16,BF16) "
+                    "(INT4G32,F16) (INT4G32,BF16)");
+    const int pb = elem_bytes(D.pred_dtype);
+    if (D.rank < 1 || (D.rank * pb) % 16 != 0 || D.rank > 128 * (16 / pb))
+        return fail(PI_ERR_INVALID_ARG, "rank*bytes must be a multiple of 16 and rank <= %d",
+                    128 * (16 / pb));
+    if (D.n_experts == 1) {
+        if (D.top_k != 1) return fail(PI_ERR_INVALID_ARG, "a dense FFN needs top_k = 1");
+    } else if (D.n_experts >= 2 && D.n_experts <= pi::kMaxExperts) {
+        if (D.top_k != 2) return fail(PI_ERR_UNSUPPORTED, "MoE supports top_k = 2");
+    } else {
+        return fail(PI_ERR_INVALID_ARG, "n_experts must be in [1, %d]", pi::kMaxExperts);
+    }
+    if (D.top_k * D.rank > pi::kMaxRankTotal)
+        return fail(PI_ERR_INVALID_ARG, "top_k * rank must be <= %d", pi::kMaxRankTotal);
+    if (!(D.eps > 0.f) || !std::isfinite(D.threshold))
+        return fail(PI_ERR_INVALID_ARG, "eps must be > 0 and threshold finite");
+
+    int ndev = 0;
+    PI_CUDA(cudaGetDeviceCount(&ndev), "cudaGetDeviceCount");
+    if (D.device < 0 || D.device >= ndev) return fail(PI_ERR_INVALID_ARG, "bad device %d", D.device);
+    PI_CUDA(cudaSetDevice(D.device), "cudaSetDevice");
+    cudaDeviceProp prop;
+    PI_CUDA(cudaGetDeviceProperties(&prop, D.device), "cudaGetDeviceProperties");
+    if (prop.major != 10)
+        return fail(PI_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a",
+                    D.device, prop.major, prop.minor);
+
+    pi_ffn *h = new (std::nothrow) pi_ffn;
+    if (!h) return fail(PI_ERR_OOM, "host allocation failed");
+    h->desc = D;
+    h->wfmt = fmt_of(D.w_dtype);
+    h->pfmt = fmt_of(D.pred_dtype);
+    h->gated = D.act != PI_ACT_RELU;
+    h->vrow = D.d_model * pb;
+    h->urow = D.rank * pb;
+    h->wrow = D.w_dtype == PI_INT4G32 ? D.d_model / 2 + D.d_model / 16
+                                      : D.d_model * elem_bytes(D.w_dtype);
+    h->S = D.n_strips > 0 ? D.n_strips : prop.multiProcessorCount;
+
+    // shared-memory rings: 6 predictor slots of 16 KB, gather slots fill the rest
+    const size_t budget = size_t(prop.sharedMemPerBlockOptin);
+    h->np = 6;
+    const size_t base = pi::decode_smem_bytes(h->np, 0, h->wrow);
+    int ng = base < budget ? int((budget - base) / size_t(h->wrow)) : 0;
+    ng = std::min(ng, pi::kMaxGSlots);
+    if (ng < 2) {
+        delete h;
+        return fail(PI_ERR_UNSUPPORTED, "shared memory too small for the gather ring");
+    }
+    h->ng = ng;
+    h->smem = pi::decode_smem_bytes(h->np, h->ng, h->wrow);
+    const int per_sm = pi::decode_max_blocks_per_sm(h->wfmt, h->pfmt, D.d_model, h->smem);
+    if (per_sm < 1 || h->S > per_sm * prop.multiProcessorCount) {
+        delete h;
+        return fail(PI_ERR_UNSUPPORTED, "n_strips %d exceeds co-resident CTAs (%d per SM x %d SMs)",
+                    D.n_strips, per_sm, prop.multiProcessorCount);
+    }
+    if (D.d_ff > pi::kMaxStrip * h->S) {
+        delete h;
+        return fail(PI_ERR_UNSUPPORTED, "d_ff %d exceeds %d neurons per strip x %d strips", D.d_ff,
+                    pi::kMaxStrip, h->S);
+    }
+    h->strip_off.resize(h->S + 1);
+    {
+        const int q = D.d_ff / h->S, rem = D.d_ff % h->S;
+        h->strip_off[0] = 0;
+        for (int b = 0; b < h->S; ++b) h->strip_off[b + 1] = h->strip_off[b] + q + (b < rem ? 1 : 0);
+    }
+    const int L = D.n_layers, E = D.n_experts;
+    h->perm.assign(size_t(L) * E, {});
+    h->mem.assign(size_t(L) * E, nullptr);
+    h->router_mem.assign(L, nullptr);
+    h->loaded.assign(L, 0);
+    h->h_ex.assign(size_t(L) * E, pi::ExpertDev{});
+
+    // scratch: t [2r] | partials [S d] | io [d] | lists [S kMaxStrip] | counts [S] | bar | err
+    const size_t o_t = 0;
+    const size_t o_part = up256(o_t + sizeof(float) * 2 * D.rank);
+    const size_t o_io = up256(o_part + sizeof(float) * size_t(h->S) * D.d_model);
+    const size_t o_lists = up256(o_io + sizeof(float) * D.d_model);
+    const size_t o_counts = up256(o_lists + sizeof(int32_t) * size_t(h->S) * pi::kMaxStrip);
+    const size_t o_bar = up256(o_counts + sizeof(int32_t) * h->S);
+    const size_t o_err = o_bar + 256;
+    const size_t total = o_err + 256;
+    cudaError_t e = cudaMalloc(&h->scratch, total);
+    if (e == cudaSuccess) e = cudaMemset(h->scratch, 0, total);
+    if (e == cudaSuccess) e = cudaMalloc(&h->d_ex, sizeof(pi::ExpertDev) * size_t(L) * E);
+    if (e == cudaSuccess) e = cudaMemset(h->d_ex, 0, sizeof(pi::ExpertDev) * size_t(L) * E);
+    if (e == cudaSuccess) e = cudaMalloc(&h->d_router, sizeof(uint8_t *) * size_t(L));
+    if (e == cudaSuccess) e = cudaMemset(h->d_router, 0, sizeof(uint8_t *) * size_t(L));
+    if (e == cudaSuccess) e = cudaMalloc(&h->d_strip_off, sizeof(int32_t) * (h->S + 1));
+    if (e == cudaSuccess)
+        e = cudaMemcpy(h->d_strip_off, h->strip_off.data(), sizeof(int32_t) * (h->S + 1),
+                       cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        pi_status st = cuda_fail(e, "pi_ffn_create: device allocation");
+        pi_ffn_destroy(h);
+        return st;
+    }
+    h->t_buf = reinterpret_cast<float *>(h->scratch + o_t);
+    h->partials = reinterpret_cast<float *>(h->scratch + o_part);
+    h->io = reinterpret_cast<float *>(h->scratch + o_io);
+    h->lists = reinterpret_cast<int32_t *>(h->scratch + o_lists);
+    h->counts = reinterpret_cast<int32_t *>(h->scratch + o_counts);
+    h->bar = reinterpret_cast<unsigned *>(h->scratch + o_bar);
+    h->err = reinterpret_cast<int *>(h->scratch + o_err);
+    *out = h;
+    return PI_OK;
+}
+
+void pi_ffn_destroy(pi_ffn_t h)
+{
+    if (!h) return;
+    cudaSetDevice(h->desc.device);
+    for (uint8_t *p : h->mem) cudaFree(p);
+    for (uint8_t *p : h->router_mem) cudaFree(p);
+    cudaFree(h->d_ex);
+    cudaFree(h->d_router);
+    cudaFree(h->d_strip_off);
+    cudaFree(h->scratch);
+    pi::prefill_destroy(h->prefill);
+    delete h;
+}
+
+pi_status pi_strip_offsets(pi_ffn_t h, int32_t *off_host, int *n_strips_out)
+{
+    if (!h) return fail(PI_ERR_INVALID_ARG, "null handle");
+    if (off_host) std::memcpy(off_host, h->strip_off.data(), sizeof(int32_t) * (h->S + 1));
+    if (n_strips_out) *n_strips_out = h->S;
+    return PI_OK;
+}
+
+// Neuron table: rank by descending frequency (ties: lower index first), deal
+// to the strips in snake order, each strip keeping its neurons hottest first.
+static void build_table(const float *freq, int F, const std::vector<int32_t> &off,
+                        std::vector<int32_t> &perm)
+{
+    perm.resize(F);
+    if (!freq) {
+        std::iota(perm.begin(), perm.end(), 0);
+        return;
+    }
+    std::vector<int32_t> order(F);
+    std::iota(order.begin(), order.end(), 0);
+    std::sort(order.begin(), order.end(), [&](int32_t a, int32_t b) {
+        if (freq[a] != freq[b]) return freq[a] > freq[b];
+        return a < b;
+    });
+    const int S = int(off.size()) - 1;
+    std::vector<int> fill(S, 0);
+    int next = 0;
+    for (int round = 0; next < F; ++round) {
+        for (int k = 0; k < S && next < F; ++k) {
+            const int b = (round & 1) ? S - 1 - k : k;
+            if (fill[b] < off[b + 1] - off[b]) perm[off[b] + fill[b]++] = order[next++];
+        }
+    }
+}
+
+pi_status pi_ffn_load_layer(pi_ffn_t h, int layer, const pi_expert_weights *experts,
+                            const void *router_dev, const float *freq_host, void *stream)
+{
+    if (!h || !experts) return fail(PI_ERR_INVALID_ARG, "pi_ffn_load_layer: null argument");
+    const pi_ffn_desc &D = h->desc;
+    if (layer < 0 || layer >= D.n_layers)
+        return fail(PI_ERR_INVALID_ARG, "layer %d out of range [0, %d)", layer, D.n_layers);
+    const int E = D.n_experts, F = D.d_ff, d = D.d_model, r = D.rank;
+    const bool int4 = D.w_dtype == PI_INT4G32;
+    for (int e = 0; e < E; ++e) {
+        const pi_expert_weights &w = experts[e];
+        if (!w.w_gate || !w.w_down || !w.bias || !w.U || !w.V)
+            return fail(PI_ERR_INVALID_ARG, "expert %d: w_gate, w_down, bias, U and V are required", e);
+        if (h->gated && !w.w_up) return fail(PI_ERR_INVALID_ARG, "expert %d: gated FFN needs w_up", e);
+        if (!h->gated && w.w_up) return fail(PI_ERR_INVALID_ARG, "expert %d: non-gated FFN takes no w_up", e);
+        if (int4 && (!w.s_gate || !w.s_down || (h->gated && !w.s_up)))
+            return fail(PI_ERR_INVALID_ARG, "expert %d: INT4 weights need scales", e);
+        const void *ptrs[] = {w.w_gate, w.w_up, w.w_down, w.s_gate, w.s_up, w.s_down, w.U, w.V};
+        for (const void *q : ptrs)
+            if (q && !aligned16(q))
+                return fail(PI_ERR_INVALID_ARG, "expert %d: weight pointers must be 16-byte aligned", e);
+    }
+    if (E > 1 && !router_dev) return fail(PI_ERR_INVALID_ARG, "MoE layer needs a router");
+    if (E == 1 && router_dev) return fail(PI_ERR_INVALID_ARG, "dense FFN takes no router");
+    if (freq_host)
+        for (size_t i = 0; i < size_t(E) * F; ++i)
+            if (!std::isfinite(freq_host[i]))
+                return fail(PI_ERR_INVALID_ARG, "freq[%zu] is not finite", i);
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    PI_CUDA(cudaSetDevice(D.device), "cudaSetDevice");
+    const size_t o_V = 0;
+    const size_t o_U = up256(o_V + size_t(r) * h->vrow);
+    const size_t o_c = up256(o_U + size_t(F) * h->urow);
+    const size_t o_g = up256(o_c + sizeof(float) * F);
+    const size_t o_u = up256(o_g + size_t(F) * h->wrow);
+    const size_t o_d = up256(o_u + (h->gated ? size_t(F) * h->wrow : 0));
+    const size_t total = up256(o_d + size_t(F) * h->wrow);
+    int32_t *d_perm = nullptr;
+    PI_CUDA(cudaMallocAsync(&d_perm, sizeof(int32_t) * F, st), "cudaMallocAsync(perm)");
+    for (int e = 0; e < E; ++e) {
+        const size_t idx = size_t(layer) * E + e;
+        const pi_expert_weights &w = experts[e];
+        build_table(freq_host ? freq_host + size_t(e) * F : nullptr, F, h->strip_off, h->perm[idx]);
+        if (!h->mem[idx]) PI_CUDA(cudaMalloc(&h->mem[idx], total), "cudaMalloc(layer)");
+        uint8_t *m = h->mem[idx];
+        PI_CUDA(cudaMemcpyAsync(d_perm, h->perm[idx].data(), sizeof(int32_t) * F,
+                                cudaMemcpyHostToDevice, st), "copy perm");
+        PI_CUDA(cudaMemcpyAsync(m + o_V, w.V, size_t(r) * h->vrow, cudaMemcpyDeviceToDevice, st), "copy V");
+        PI_CUDA(pi::repack_rows(static_cast<const uint8_t *>(w.U), m + o_U, d_perm, F, h->urow, nullptr, 0, st),
+                "repack U");
+        PI_CUDA(pi::repack_bias(w.bias, reinterpret_cast<float *>(m + o_c), d_perm, F, st), "repack c");
+        if (int4) {
+            const int qb = d / 2, sb = d / 16;
+            PI_CUDA(pi::repack_rows(static_cast<const uint8_t *>(w.w_gate), m + o_g, d_perm, F, qb,
+                                    static_cast<const uint8_t *>(w.s_gate), sb, st), "repack gate");
+            if (h->gated)
+                PI_CUDA(pi::repack_rows(static_cast<const uint8_t *>(w.w_up), m + o_u, d_perm, F, qb,
+                                        static_cast<const uint8_t *>(w.s_up), sb, st), "repack up");
+            PI_CUDA(pi::repack_rows(static_cast<const uint8_t *>(w.w_down), m + o_d, d_perm, F, qb,
+                                    static_cast<const uint8_t *>(w.s_down), sb, st), "repack down");
+        } else {
+            PI_CUDA(pi::repack_rows(static_cast<const uint8_t *>(w.w_gate), m + o_g, d_perm, F, h->wrow,
+                                    nullptr, 0, st), "repack gate");
+            if (h->gated)
+                PI_CUDA(pi::repack_rows(static_cast<const uint8_t *>(w.w_up), m + o_u, d_perm, F, h->wrow,
+                                        nullptr, 0, st), "repack up");
+            PI_CUDA(pi::repack_down_transpose(static_cast<const uint8_t *>(w.w_down), m + o_d, d_perm, d,
+                                              F, elem_bytes(D.w_dtype), st), "transpose down");
+        }
+        pi::ExpertDev &x = h->h_ex[idx];
+        x.V = m + o_V;
+        x.U = m + o_U;
+        x.c = reinterpret_cast<const float *>(m + o_c);
+        x.Wg = m + o_g;
+        x.Wu = h->gated ? m + o_u : nullptr;
+        x.Wd = m + o_d;
+        // the table is reused for the next expert: finish this one first
+        PI_CUDA(cudaStreamSynchronize(st), "load_layer sync");
+    }
+    PI_CUDA(cudaFreeAsync(d_perm, st), "cudaFreeAsync(perm)");
+    if (E > 1) {
+        if (!h->router_mem[layer])
+            PI_CUDA(cudaMalloc(&h->router_mem[layer], size_t(E) * d * 2), "cudaMalloc(router)");
+        PI_CUDA(cudaMemcpyAsync(h->router_mem[layer], router_dev, size_t(E) * d * 2,
+                                cudaMemcpyDeviceToDevice, st), "copy router");
+        const uint8_t *rp = h->router_mem[layer];
+        PI_CUDA(cudaMemcpyAsync(h->d_router + layer, &rp, sizeof(rp), cudaMemcpyHostToDevice, st),
+                "router table");
+    }
+    PI_CUDA(cudaMemcpyAsync(h->d_ex + size_t(layer) * E, h->h_ex.data() + size_t(layer) * E,
+                            sizeof(pi::ExpertDev) * E, cudaMemcpyHostToDevice, st), "expert table");
+    PI_CUDA(cudaStreamSynchronize(st), "load_layer sync");
+    h->loaded[layer] = 1;
+    if (h->prefill) pi::prefill_invalidate(h->prefill, layer);
+    return PI_OK;
+}
+
+pi_status pi_neuron_table(pi_ffn_t h, int layer, int expert, int32_t *perm_host)
+{
+    if (!h || !perm_host) return fail(PI_ERR_INVALID_ARG, "pi_neuron_table: null argument");
+    if (layer < 0 || layer >= h->desc.n_layers || expert < 0 || expert >= h->desc.n_experts)
+        return fail(PI_ERR_INVALID_ARG, "layer/expert out of range");
+    if (!h->loaded[layer]) return fail(PI_ERR_NOT_LOADED, "layer %d not loaded", layer);
+    const auto &v = h->perm[size_t(layer) * h->desc.n_experts + expert];
+    std::memcpy(perm_host, v.data(), sizeof(int32_t) * v.size());
+    return PI_OK;
+}
+
+static pi::DecodeParams base_params(pi_ffn_t h)
+{
+    pi::DecodeParams p{};
+    const pi_ffn_desc &D = h->desc;
+    p.ex = h->d_ex;
+    p.router = h->d_router;
+    p.strip_off = h->d_strip_off;
+    p.d = D.d_model;
+    p.F = D.d_ff;
+    p.r = D.rank;
+    p.E = D.n_experts;
+    p.top_k = D.top_k;
+    p.act = int(D.act);
+    p.gated = h->gated;
+    p.S = h->S;
+    p.threshold = D.threshold;
+    p.eps = D.eps;
+    p.vrow = h->vrow;
+    p.urow = h->urow;
+    p.wrow = h->wrow;
+    p.np_slots = h->np;
+    p.ng_slots = h->ng;
+    p.sg_bytes = h->wrow;
+    p.t_buf = h->t_buf;
+    p.partials = h->partials;
+    p.lists = h->lists;
+    p.counts = h->counts;
+    p.bar = h->bar;
+    p.err = h->err;
+    p.wait_ns = h->wait_ns;
+    p.debug_flags = h->debug_flags;
+    return p;
+}
+
+pi_status pi_predict(pi_ffn_t h, int layer, int expert, const float *x_dev, int32_t *idx_dev,
+                     int32_t *count_dev, float *z_dev, void *stream)
+{
+    if (!h || !x_dev || !idx_dev || !count_dev) return fail(PI_ERR_INVALID_ARG, "pi_predict: null argument");
+    const pi_ffn_desc &D = h->desc;
+    if (layer < 0 || layer >= D.n_layers || expert < 0 || expert >= D.n_experts)
+        return fail(PI_ERR_INVALID_ARG, "layer/expert out of range");
+    if (!h->loaded[layer]) return fail(PI_ERR_NOT_LOADED, "layer %d not loaded", layer);
+    if (!aligned16(x_dev)) return fail(PI_ERR_INVALID_ARG, "x_dev must be 16-byte aligned");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    PI_CUDA(cudaSetDevice(D.device), "cudaSetDevice");
+    pi::DecodeParams p = base_params(h);
+    p.mode = pi::kModePredict;
+    p.pred_expert = expert;
+    p.layer_begin = layer;
+    p.layer_end = layer + 1;
+    p.x_in = x_dev;
+    p.z_out = z_dev;
+    p.idx_out = idx_dev;
+    p.count_out = count_dev;
+    PI_CUDA(cudaMemsetAsync(h->bar, 0, sizeof(unsigned), st), "memset barrier");
+    PI_CUDA(pi::launch_decode(h->wfmt, h->pfmt, p, h->smem, st), "launch predict");
+    return PI_OK;
+}
+
+pi_status pi_sparse_ffn_decode(pi_ffn_t h, int layer_begin, int layer_end, float *resid_dev,
+                               float *trace_dev, int32_t *stats_dev, uint32_t *mask_dev, void *stream)
+{
+    if (!h || !resid_dev) return fail(PI_ERR_INVALID_ARG, "pi_sparse_ffn_decode: null argument");
+    const pi_ffn_desc &D = h->desc;
+    if (layer_begin < 0 || layer_end > D.n_layers || layer_begin >= layer_end)
+        return fail(PI_ERR_INVALID_ARG, "layer range [%d, %d) invalid for %d layers", layer_begin,
+                    layer_end, D.n_layers);
+    for (int l = layer_begin; l < layer_end; ++l)
+        if (!h->loaded[l]) return fail(PI_ERR_NOT_LOADED, "layer %d not loaded", l);
+    if (!aligned16(resid_dev) || (trace_dev && !aligned16(trace_dev)))
+        return fail(PI_ERR_INVALID_ARG, "resid_dev and trace_dev must be 16-byte aligned");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    PI_CUDA(cudaSetDevice(D.device), "cudaSetDevice");
+    const int nl = layer_end - layer_begin;
+    pi::DecodeParams p = base_params(h);
+    p.mode = pi::kModeDecode;
+    p.layer_begin = layer_begin;
+    p.layer_end = layer_end;
+    p.resid = resid_dev;
+    p.trace = trace_dev;
+    p.stats = stats_dev;
+    p.masks = mask_dev;
+    PI_CUDA(cudaMemsetAsync(h->bar, 0, sizeof(unsigned), st), "memset barrier");
+    if (stats_dev) PI_CUDA(cudaMemsetAsync(stats_dev, 0, sizeof(int32_t) * 4 * nl, st), "memset stats");
+    if (mask_dev)
+        PI_CUDA(cudaMemsetAsync(mask_dev, 0, sizeof(uint32_t) * size_t(nl) * D.top_k * ((D.d_ff + 31) / 32), st),
+                "memset masks");
+    PI_CUDA(pi::launch_decode(h->wfmt, h->pfmt, p, h->smem, st), "launch decode");
+    return PI_OK;
+}
+
+pi_status pi_sparse_ffn_decode_host(pi_ffn_t h, int layer_begin, int layer_end,
+                                    const float *resid_in_host, float *resid_out_host, void *stream)
+{
+    if (!h || !resid_in_host || !resid_out_host)
+        return fail(PI_ERR_INVALID_ARG, "pi_sparse_ffn_decode_host: null argument");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t bytes = sizeof(float) * h->desc.d_model;
+    PI_CUDA(cudaSetDevice(h->desc.device), "cudaSetDevice");
+    PI_CUDA(cudaMemcpyAsync(h->io, resid_in_host, bytes, cudaMemcpyHostToDevice, st), "copy in");
+    pi_status s = pi_sparse_ffn_decode(h, layer_begin, layer_end, h->io, nullptr, nullptr, nullptr, stream);
+    if (s != PI_OK) return s;
+    PI_CUDA(cudaMemcpyAsync(resid_out_host, h->io, bytes, cudaMemcpyDeviceToHost, st), "copy out");
+    PI_CUDA(cudaStreamSynchronize(st), "sync");
+    return PI_OK;
+}
+
+pi_status pi_sync(pi_ffn_t h, void *stream)
+{
+    if (!h) return fail(PI_ERR_INVALID_ARG, "null handle");
+    PI_CUDA(cudaSetDevice(h->desc.device), "cudaSetDevice");
+    PI_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)), "stream sync");
+    int err = 0;
+    PI_CUDA(cudaMemcpy(&err, h->err, sizeof(int), cudaMemcpyDeviceToHost), "read error word");
+    if (err == pi::kDevOk) return PI_OK;
+    PI_CUDA(cudaMemset(h->err, 0, sizeof(int)), "clear error word");
+    if (err == pi::kDevTimeout) return fail(PI_ERR_TIMEOUT, "a bounded device-side wait ran out");
+    return fail(PI_ERR_DEVICE_CHECK, "device-side check failed (code %d)", err);
+}
+
+pi_status pi_debug_set(pi_ffn_t h, int flags, double wait_limit_s)
+{
+    if (!h) return fail(PI_ERR_INVALID_ARG, "null handle");
+    if (!(wait_limit_s > 0.0) || wait_limit_s > 60.0)
+        return fail(PI_ERR_INVALID_ARG, "wait_limit_s must be in (0, 60]");
+    h->debug_flags = flags;
+    h->wait_ns = static_cast<long long>(wait_limit_s * 1e9);
+    return PI_OK;
+}
+
+pi_status pi_dense_ffn_prefill(pi_ffn_t h, int layer_begin, int layer_end, int n_tokens,
+                               float *resid_dev, void *stream)
+{
+    if (!h || !resid_dev) return fail(PI_ERR_INVALID_ARG, "pi_dense_ffn_prefill: null argument");
+    const pi_ffn_desc &D = h->desc;
+    if (layer_begin < 0 || layer_end > D.n_layers || layer_begin >= layer_end)
+        return fail(PI_ERR_INVALID_ARG, "layer range invalid");
+    if (n_tokens < 1) return fail(PI_ERR_INVALID_ARG, "n_tokens must be >= 1");
+    for (int l = layer_begin; l < layer_end; ++l)
+        if (!h->loaded[l]) return fail(PI_ERR_NOT_LOADED, "layer %d not loaded", l);
+    if (!aligned16(resid_dev)) return fail(PI_ERR_INVALID_ARG, "resid_dev must be 16-byte aligned");
+    PI_CUDA(cudaSetDevice(D.device), "cudaSetDevice");
+    pi::PrefillView v{};
+    v.d = D.d_model;
+    v.F = D.d_ff;
+    v.E = D.n_experts;
+    v.top_k = D.top_k;
+    v.act = int(D.act);
+    v.gated = h->gated;
+    v.wfmt = h->wfmt;
+    v.wrow = h->wrow;
+    v.eps = D.eps;
+    v.ex = h->h_ex.data();
+    v.router = h->router_mem.data();
+    v.perm = &h->perm;
+    char msg[256] = "";
+    const int rc = pi::prefill_run(&h->prefill, v, layer_begin, layer_end, n_tokens, resid_dev,
+                                   static_cast<cudaStream_t>(stream), msg, sizeof msg);
+    if (rc == 1) return fail(PI_ERR_UNSUPPORTED, "%s", msg);
+    if (rc == 2) return fail(PI_ERR_CUDA, "%s", msg);
+    if (rc == 3) return fail(PI_ERR_OOM, "%s", msg);
+    return PI_OK;
+}
+
+}  // extern "C"

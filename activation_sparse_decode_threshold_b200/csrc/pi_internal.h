@@ -1,0 +1,84 @@
+// pi_internal.h -- structures shared by the host side of the C ABI and the
+// sm_100a kernels.  Not part of the public interface.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace pi {
+
+// Decode kernel geometry: 8 consumer warps (256 threads) do the arithmetic,
+// warp 8 streams the input-independent predictor weights (V, U) into a
+// shared-memory ring, warp 9 streams the gathered neuron rows (W_gate / W_up /
+// W_down of active neurons) into a second ring.
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kPWarp = 8;
+constexpr int kGWarp = 9;
+constexpr int kThreads = 320;
+constexpr int kMaxStrip = 256;        // neurons per strip (per CTA) at most
+constexpr int kMaxTopK = 2;
+constexpr int kMaxExperts = 16;
+constexpr int kMaxPSlots = 16;
+constexpr int kMaxGSlots = 128;
+constexpr int kMaxRankTotal = 2048;   // top_k * rank
+constexpr int kPSlotBytes = 16384;
+
+enum Fmt { kF32 = 0, kF16 = 1, kBF16 = 2, kI4 = 3 };
+
+// One expert (or dense FFN) of one layer, in table order, library-owned.
+struct ExpertDev {
+    const uint8_t *V;    // r rows of vrow bytes (original order; rank is not permuted)
+    const uint8_t *U;    // F rows of urow bytes, table order
+    const float *c;      // F biases, table order
+    const uint8_t *Wg;   // F rows of wrow bytes (W_1 when non-gated)
+    const uint8_t *Wu;   // F rows of wrow bytes, or null when non-gated
+    const uint8_t *Wd;   // F rows of wrow bytes: W_down columns, neuron-major
+};
+
+enum Mode { kModeDecode = 0, kModePredict = 1 };
+
+struct DecodeParams {
+    const ExpertDev *ex;            // [n_layers * E]
+    const uint8_t *const *router;   // [n_layers] E x d fp16, or null entries
+    const int32_t *strip_off;       // [S + 1]
+    int d, F, r, E, top_k, act, gated, S;
+    int layer_begin, layer_end;
+    float threshold, eps;
+    int vrow, urow, wrow;           // row bytes: V (pred fmt), U (pred fmt), W (weight fmt)
+    int np_slots, ng_slots, sg_bytes;
+    int mode, pred_expert;
+    // inputs / outputs
+    float *resid;                   // [d] decode: in/out residual
+    const float *x_in;              // [d] predict: layer input
+    float *trace;                   // [(l1-l0) * d] or null
+    int32_t *stats;                 // [(l1-l0) * 4] or null (zeroed by the host)
+    uint32_t *masks;                // [(l1-l0) * top_k * ceil(F/32)] or null (zeroed)
+    float *z_out;                   // predict: [F] or null
+    int32_t *idx_out, *count_out;   // predict
+    // scratch (library-owned or caller-provided, see pi_host.cu)
+    float *t_buf;                   // [top_k * r]
+    float *partials;                // [S * d]
+    int32_t *lists;                 // [S * kMaxStrip]  (predict)
+    int32_t *counts;                // [S]              (predict)
+    unsigned *bar;                  // grid barrier counter, zeroed before launch
+    int *err;                       // device error word (0 = ok)
+    long long wait_ns;              // bound on every device-side wait
+    int debug_flags;
+};
+
+size_t decode_smem_bytes(int np_slots, int ng_slots, int sg_bytes);
+cudaError_t launch_decode(int wfmt, int pfmt, const DecodeParams &p, size_t smem,
+                          cudaStream_t stream);
+int decode_max_blocks_per_sm(int wfmt, int pfmt, int d, size_t smem);
+
+// Load-time repack kernels (pi_repack.cu).
+cudaError_t repack_rows(const uint8_t *src, uint8_t *dst, const int32_t *perm, int rows,
+                        int row_bytes, const uint8_t *src2, int row2_bytes, cudaStream_t s);
+cudaError_t repack_bias(const float *src, float *dst, const int32_t *perm, int n, cudaStream_t s);
+cudaError_t repack_down_transpose(const uint8_t *w_down, uint8_t *dst, const int32_t *perm,
+                                  int d, int F, int elem_bytes, cudaStream_t s);
+
+// Device error codes written into the error word.
+enum DevErr { kDevOk = 0, kDevTimeout = 1, kDevCheck = 2 };
+
+}  // namespace pi

@@ -1,0 +1,210 @@
+/*
+ * pi_ffn.h -- C ABI of the predictor-guided, neuron-aware sparse FFN library
+ * for NVIDIA B200 (sm_100a).
+ *
+ * What it computes (per decode token, per FFN layer), after the pages on
+ * PowerInfer and PowerInfer-2:
+ *   x = RMSNorm(r)                                   (no weight, eps)
+ *   [MoE] two experts from a softmax router           (TurboSparse-Mixtral-shaped layer)
+ *   t = V x ; z = U t - c ; neuron i active iff z_i > threshold
+ *        -- the online activation predictor: "PowerInfer: fast LLM serving
+ *           with a consumer-grade GPU" (unite.ai), sections "Online phase" and
+ *           "Adaptive sparse predictor"; nearauto.com PowerInfer article,
+ *           "PowerInfer architecture", Fig. 8.
+ *   for active i only: g = W_gate[i].x - c_i, u = W_up[i].x, h = act(g, u)
+ *   y = sum over active i with h_i != 0 of h_i * W_down[:, i]
+ *        -- neuron-aware operators over rows of the input matrices and
+ *           columns of the output matrix, no dense conversion: unite.ai,
+ *           "Neuron-aware operators".
+ *   r <- r + y
+ * Neurons are stored in neuron-table order ("Neuron placement and
+ * management", unite.ai): the table maps each stored position to the
+ * neuron's original index, and results are returned in original d_model order.
+ *
+ * Conventions for every call:
+ *  - Pointers marked _dev are CUDA device pointers owned by the caller; _host
+ *    are host pointers.  Nothing here takes or returns a torch type.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Device work is enqueued on it and the call returns without waiting,
+ *    unless the call says otherwise.
+ *  - Arguments are validated before any work is enqueued; on a bad argument
+ *    the call returns PI_ERR_INVALID_ARG (or PI_ERR_UNSUPPORTED) and enqueues
+ *    nothing.  pi_last_error() then describes the problem.
+ *  - Faults found on the device (a bounded wait that ran out, a bad index)
+ *    never trap: the kernel records an error word and returns; pi_sync()
+ *    reports it.  No call aborts, throws or exits the process.
+ *  - One handle may be used from one host thread at a time.  Calls that
+ *    overlap on the GPU (two streams, same handle) race on the handle's
+ *    scratch memory and must not be issued.
+ */
+#ifndef PI_FFN_H
+#define PI_FFN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PI_API __attribute__((visibility("default")))
+#else
+#define PI_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct pi_ffn *pi_ffn_t;
+
+typedef enum {
+    PI_OK = 0,
+    PI_ERR_INVALID_ARG = 1,   /* bad pointer, size, index or combination */
+    PI_ERR_UNSUPPORTED = 2,   /* valid but not implemented for this shape/format */
+    PI_ERR_OOM = 3,           /* device allocation failed */
+    PI_ERR_CUDA = 4,          /* a CUDA runtime call failed */
+    PI_ERR_TIMEOUT = 5,       /* a bounded device-side wait ran out */
+    PI_ERR_DEVICE_CHECK = 6,  /* a device-side consistency check failed */
+    PI_ERR_NOT_LOADED = 7     /* a layer in the range was never loaded */
+} pi_status;
+
+/* Activation of the FFN (h as a function of g = W_gate.x - c and u = W_up.x).
+ * RELU is non-gated: the layer has one input matrix, passed as w_gate
+ * (W_1), and h = max(g, 0).  REGLU: h = max(g, 0) * u.  DRELU: h = max(g, 0)
+ * * max(u, 0) (citnews.com.cn PowerInfer-2 article, dReLU replaces SwiGLU). */
+typedef enum { PI_ACT_RELU = 0, PI_ACT_REGLU = 1, PI_ACT_DRELU = 2 } pi_act;
+
+/* Stored formats.  INT4G32: symmetric 4-bit, value = s * (n - 8) with n the
+ * nibble (low nibble = even element) and s one fp16 scale per 32 consecutive
+ * elements of a neuron vector (a W_gate/W_up row or a W_down column). */
+typedef enum { PI_F32 = 0, PI_F16 = 1, PI_BF16 = 2, PI_INT4G32 = 3 } pi_dtype;
+
+typedef struct {
+    int n_layers;        /* layers in the stack, >= 1 */
+    int d_model;         /* d: multiple of 256, <= 8192 (<= 4096 for F32) */
+    int d_ff;            /* F: neurons per FFN (per expert), <= 256 * n_strips */
+    int rank;            /* predictor rank r: r * bytes(pred_dtype) a multiple of 16,
+                            r <= 1024 (<= 512 for F32) */
+    int n_experts;       /* 1 = dense FFN; 2..16 = MoE with top-2 routing */
+    int top_k;           /* 1 for a dense FFN, 2 for MoE */
+    pi_act act;
+    pi_dtype w_dtype;    /* F32, F16, BF16 or INT4G32 */
+    pi_dtype pred_dtype; /* F32, F16 or BF16 (F32 weights need F32 here) */
+    int n_strips;        /* neuron strips per FFN = CTAs of the decode kernel;
+                            0 = number of SMs of the device */
+    float threshold;     /* predictor threshold, normally 0 (active iff z > threshold) */
+    float eps;           /* RMSNorm epsilon, normally 1e-6 */
+    int device;          /* CUDA device ordinal */
+} pi_ffn_desc;
+
+/* Weights of one FFN or one MoE expert, in ORIGINAL neuron order, as device
+ * pointers (read during pi_ffn_load_layer only; the caller keeps ownership).
+ *   w_gate  F x d row-major (W_1 when non-gated)        [w_dtype]
+ *   w_up    F x d row-major, NULL when non-gated          [w_dtype]
+ *   w_down  float formats: d x F row-major (nn.Linear layout);
+ *           INT4G32: neuron-major F x d (row i = column i of W_down)
+ *   s_gate, s_up, s_down  INT4G32 only: F x d/32 fp16 scales (one per 32
+ *           consecutive elements of each neuron vector); NULL otherwise.
+ *           INT4 matrices are F x d/2 bytes of nibbles.
+ *   bias    c, F floats (the gate bias enters as -c)
+ *   U       F x r row-major [pred_dtype];  V  r x d row-major [pred_dtype]
+ */
+typedef struct {
+    const void *w_gate, *w_up, *w_down;
+    const void *s_gate, *s_up, *s_down;
+    const float *bias;
+    const void *U, *V;
+} pi_expert_weights;
+
+/* Create a handle: validates `desc`, reserves per-handle scratch on
+ * desc->device.  No weights yet.  Returns PI_OK and *out, or an error. */
+PI_API pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out);
+
+/* Load layer `layer` (0 <= layer < n_layers): builds each expert's neuron
+ * table from `freq_host` (n_experts x F profiled firing frequencies, NULL =
+ * identity table), then copies and repacks the weights into library-owned
+ * device memory in table order (rows of W_gate, W_up, U and c permuted;
+ * W_down transposed so each neuron's column is contiguous; INT4 scales stored
+ * after each neuron's nibbles).  `experts` has n_experts entries.  `router_dev`
+ * is the E x d fp16 router for MoE (NULL for a dense FFN).  Work runs on
+ * `stream`; the call synchronises it before returning, so the caller's
+ * buffers may be freed afterwards.  Reloading a layer replaces it. */
+PI_API pi_status pi_ffn_load_layer(pi_ffn_t h, int layer, const pi_expert_weights *experts,
+                            const void *router_dev, const float *freq_host, void *stream);
+
+/* Neuron table of (layer, expert): perm_host[p] = original index of the
+ * neuron stored at table position p (F entries).  Strip b of the table holds
+ * positions [off[b], off[b+1]) with off from pi_strip_offsets.  Table rule:
+ * neurons ranked by descending frequency (ties: lower index first), dealt to
+ * the strips in snake order (round j ascending for even j, descending for odd
+ * j; a full strip is skipped); a strip keeps its neurons hottest first. */
+PI_API pi_status pi_neuron_table(pi_ffn_t h, int layer, int expert, int32_t *perm_host);
+
+/* Strip offsets (n_strips + 1 entries): strip b holds floor(F/S) + (b < F mod S)
+ * neurons.  n_strips is also returned through *n_strips_out when non-NULL. */
+PI_API pi_status pi_strip_offsets(pi_ffn_t h, int32_t *off_host, int *n_strips_out);
+
+/* Predictor alone for (layer, expert) on a given layer input x (already
+ * normalised, d floats):
+ *   idx_dev    [F] int32: the active neurons' TABLE positions, ascending
+ *              (map back with pi_neuron_table); entries past *count unspecified
+ *   count_dev  [1] int32: number of active neurons
+ *   z_dev      [F] float or NULL: predictor logits z in table order
+ * Uses the same device code as the predictor inside pi_sparse_ffn_decode. */
+PI_API pi_status pi_predict(pi_ffn_t h, int layer, int expert, const float *x_dev,
+                     int32_t *idx_dev, int32_t *count_dev, float *z_dev, void *stream);
+
+/* Batch-1 sparse decode of layers [layer_begin, layer_end) on one token.
+ *   resid_dev   [d] float, in/out: the residual stream r; on return r after
+ *               the last layer.
+ *   trace_dev   [(l1-l0) x d] float or NULL: the residual entering each layer.
+ *   stats_dev   [(l1-l0) x 4] int32 or NULL: per layer {predicted-active
+ *               neurons, neurons with h != 0, first expert, second expert}
+ *               (counts summed over the used experts; experts -1 if dense).
+ *   mask_dev    [(l1-l0) x top_k x ceil(F/32)] uint32 or NULL: predicted-active
+ *               bits in table order (bit p%32 of word p/32), per used expert
+ *               in ascending expert index.
+ * All layers run in one persistent kernel with one CTA per strip.  The result
+ * is deterministic: the same inputs give bit-identical outputs, and splitting
+ * the range into several calls gives the same bits as one call. */
+PI_API pi_status pi_sparse_ffn_decode(pi_ffn_t h, int layer_begin, int layer_end, float *resid_dev,
+                               float *trace_dev, int32_t *stats_dev, uint32_t *mask_dev,
+                               void *stream);
+
+/* Same as pi_sparse_ffn_decode on HOST buffers: copies resid_in_host (d
+ * floats) to the device, decodes, copies the result to resid_out_host, and
+ * synchronises `stream` before returning.  Host buffers should be pinned for
+ * the copies to run at full speed.  The two may alias. */
+PI_API pi_status pi_sparse_ffn_decode_host(pi_ffn_t h, int layer_begin, int layer_end,
+                                    const float *resid_in_host, float *resid_out_host,
+                                    void *stream);
+
+/* Dense multi-token prefill of layers [layer_begin, layer_end) on the tensor
+ * cores (PowerInfer-2: prefill activates almost every neuron and runs as large
+ * dense clusters; citnews.com.cn article, "Neuron-cluster heterogeneous
+ * computing").  resid_dev is n_tokens x d float, in/out.  Per layer every
+ * token is normalised, routed (MoE), and passed through the full FFN of its
+ * expert(s) with no predictor; outputs are combined in ascending expert index
+ * and added to the residual. */
+PI_API pi_status pi_dense_ffn_prefill(pi_ffn_t h, int layer_begin, int layer_end, int n_tokens,
+                               float *resid_dev, void *stream);
+
+/* Wait for `stream` and report (then clear) the handle's device error word:
+ * PI_OK, PI_ERR_TIMEOUT or PI_ERR_DEVICE_CHECK. */
+PI_API pi_status pi_sync(pi_ffn_t h, void *stream);
+
+/* Message for the last non-OK status returned on this host thread. */
+PI_API const char *pi_last_error(void);
+
+/* Release the handle and all device memory it owns (after its work is done). */
+PI_API void pi_ffn_destroy(pi_ffn_t h);
+
+/* Testing aid: bound every device-side wait of this handle by `wait_limit_s`
+ * seconds (default 2.0) and, with flags & PI_DEBUG_STALL_BARRIER, make the
+ * decode kernel's first grid barrier wait for one arrival that never comes,
+ * so that the bounded wait runs out and pi_sync reports PI_ERR_TIMEOUT. */
+#define PI_DEBUG_STALL_BARRIER 1
+PI_API pi_status pi_debug_set(pi_ffn_t h, int flags, double wait_limit_s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PI_FFN_H */

@@ -1,0 +1,222 @@
+"""GPU parity of the CUDA path against the fp64 oracle, through the C ABI.
+
+Small cases (the oracle finishes in seconds) span several strips and ragged
+strip tails; full-size cases run the workloads at their real shapes in the
+launch configuration the benchmark uses (one CTA per SM) and check sampled
+layers teacher-forced on the GPU's own trace."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from activation_sparse_decode_threshold_b200 import binding as B
+from activation_sparse_decode_threshold_b200 import synth
+import gpu_util as G
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    # name: (config, strips)
+    "reglu-f16": synth.small(synth.CONFIGS["llama7b"], n_layers=3, d=512, F=1000, rank=64),
+    "drelu-bf16": synth.small(synth.CONFIGS["mistral7b"], n_layers=3, d=768, F=2100, rank=128),
+    "relu-f16-nongated": synth.small(synth.CONFIGS["falcon40b"], n_layers=2, d=1024, F=4100, rank=256),
+    "reglu-f32": synth.small(synth.CONFIGS["relu1"], n_layers=2, d=256, F=333, rank=32),
+    "moe-int4-drelu": synth.small(synth.CONFIGS["mixtral47b"], n_layers=2, d=512, F=1024, rank=64,
+                                  n_experts=4),
+    "fewer-neurons-than-strips": synth.small(synth.CONFIGS["llama7b"], n_layers=2, d=256, F=100,
+                                             rank=32),
+}
+
+
+@pytest.fixture
+def handles():
+    hs = []
+    yield hs
+    torch.cuda.synchronize()
+    for h in hs:
+        B.pi_ffn_destroy(h)
+
+
+def _build(cfg, handles, n_strips=0, threshold=0.0, use_freq=True, n_layers=None):
+    L = n_layers or cfg.n_layers
+    h = G.create(cfg, L, n_strips, threshold)
+    handles.append(h)
+    lws = [synth.make_layer(cfg, l, "cuda") for l in range(L)]
+    for l, lw in enumerate(lws):
+        G.load(h, l, lw, use_freq)
+    return h, lws
+
+
+# ---------------------------------------------------------------------------
+def test_neuron_table_and_strips_match_oracle(handles):
+    cfg = SMALL["reglu-f16"]
+    h, lws = _build(cfg, handles, n_layers=1)
+    off = B.pi_strip_offsets(h)
+    S = len(off) - 1
+    assert np.array_equal(off, oracle.strip_offsets(cfg.F, S))
+    freq32 = G.freq_of(lws[0])[0]
+    perm = B.pi_neuron_table(h, 0, 0, cfg.F)
+    assert np.array_equal(perm, oracle.neuron_table(cfg.F, S, freq32.astype(np.float64)))
+
+
+def test_predict_parity_single_layer_fp32(handles):
+    """64 tokens of the single-layer fp32 workload: predicted sets and logits."""
+    cfg = synth.CONFIGS["relu1"]
+    h, lws = _build(cfg, handles)
+    ex, _ = G.oracle_layer(cfg, lws[0])
+    perm = B.pi_neuron_table(h, 0, 0, cfg.F)
+    idx = torch.empty(cfg.F, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(1, dtype=torch.int32, device="cuda")
+    z = torch.empty(cfg.F, dtype=torch.float32, device="cuda")
+    band = 0
+    for t in range(cfg.n_tokens):
+        x32 = oracle.rmsnorm(synth.token_input(cfg, t).double().numpy()).astype(np.float32)
+        B.pi_predict(h, 0, 0, torch.from_numpy(x32).cuda(), idx, cnt, z)
+        assert B.pi_sync(h) == B.PI_OK
+        n = int(cnt.item())
+        got = idx[:n].cpu().numpy()
+        assert np.all(np.diff(got) > 0), "table positions must be ascending"
+        gm = np.zeros(cfg.F, bool)
+        gm[perm[got]] = True
+        _, z_or, _ = oracle.predict(x32.astype(np.float64), ex[0].V, ex[0].U, ex[0].c, "f32")
+        band += G.check_active_set(gm, z_or)
+        z_gpu = np.empty(cfg.F)
+        z_gpu[perm] = z.cpu().double().numpy()
+        assert np.max(np.abs(z_gpu - z_or)) <= 1e-4 + 1e-5 * np.max(np.abs(z_or))
+    assert band <= 2
+
+
+def test_decode_single_layer_fp32_all_tokens(handles):
+    cfg = synth.CONFIGS["relu1"]
+    h, lws = _build(cfg, handles)
+    ex, router = G.oracle_layer(cfg, lws[0])
+    perms = G.tables(h, lws[0], 0, cfg.F)
+    for t in range(cfg.n_tokens):
+        r0 = synth.token_input(cfg, t)
+        r1, trace, stats, masks = G.decode_traced(h, cfg, 0, 1, r0)
+        assert np.array_equal(trace[0], r0.double().numpy())
+        G.check_layer(cfg, ex, router, perms, trace[0], r1, stats[0], masks[0])
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_decode_stack_small(handles, name):
+    cfg = SMALL[name]
+    h, lws = _build(cfg, handles)
+    olayers = [G.oracle_layer(cfg, lw) for lw in lws]
+    perms = [G.tables(h, lw, l, cfg.F) for l, lw in enumerate(lws)]
+    for t in range(4):
+        r0 = synth.token_input(cfg, t)
+        rL, trace, stats, masks = G.decode_traced(h, cfg, 0, cfg.n_layers, r0)
+        outs = list(trace[1:]) + [rL]
+        for l in range(cfg.n_layers):
+            ex, router = olayers[l]
+            G.check_layer(cfg, ex, router, perms[l], trace[l], outs[l], stats[l], masks[l])
+
+
+def test_decode_is_deterministic_and_splits_agree(handles):
+    cfg = SMALL["drelu-bf16"]
+    h, _ = _build(cfg, handles)
+    r0 = synth.token_input(cfg, 5).cuda()
+    outs = []
+    for _ in range(2):
+        r = r0.clone()
+        B.pi_sparse_ffn_decode(h, 0, cfg.n_layers, r)
+        outs.append(r.clone())
+    r = r0.clone()
+    for l in range(cfg.n_layers):
+        B.pi_sparse_ffn_decode(h, l, l + 1, r)
+    outs.append(r)
+    assert B.pi_sync(h) == B.PI_OK
+    assert torch.equal(outs[0], outs[1])
+    assert torch.equal(outs[0], outs[2])
+
+
+def test_host_buffer_entry_point_matches_device_call(handles):
+    cfg = SMALL["reglu-f16"]
+    h, _ = _build(cfg, handles)
+    r0 = synth.token_input(cfg, 1)
+    rin = r0.clone().pin_memory()
+    rout = torch.empty_like(rin).pin_memory()
+    B.pi_sparse_ffn_decode_host(h, 0, cfg.n_layers, rin, rout)
+    rd = r0.clone().cuda()
+    B.pi_sparse_ffn_decode(h, 0, cfg.n_layers, rd)
+    assert B.pi_sync(h) == B.PI_OK
+    assert torch.equal(rout, rd.cpu())
+
+
+def test_threshold_extremes_empty_and_dense(handles):
+    cfg = SMALL["reglu-f16"]
+    lw = synth.make_layer(cfg, 0, "cuda")
+    ex, _ = G.oracle_layer(cfg, lw)
+    r0 = synth.token_input(cfg, 2)
+    # nothing predicted active: the layer adds exactly zero
+    h = G.create(cfg, 1, threshold=1e30)
+    handles.append(h)
+    G.load(h, 0, lw)
+    r1, _, stats, _ = G.decode_traced(h, cfg, 0, 1, r0)
+    assert stats[0][0] == 0 and np.array_equal(r1, r0.double().numpy())
+    # everything active: the dense FFN
+    h2 = G.create(cfg, 1, threshold=-1e30)
+    handles.append(h2)
+    G.load(h2, 0, lw)
+    r1, _, stats, _ = G.decode_traced(h2, cfg, 0, 1, r0)
+    assert stats[0][0] == cfg.F
+    x = oracle.rmsnorm(r0.double().numpy())
+    _, y = oracle.ffn_masked(ex[0], x)
+    G.check_output(r1 - r0.double().numpy(), y)
+
+
+def test_identity_table_gives_same_result_within_rounding(handles):
+    cfg = SMALL["reglu-f16"]
+    h1, _ = _build(cfg, handles, use_freq=True, n_layers=1)
+    h2, _ = _build(cfg, handles, use_freq=False, n_layers=1)
+    assert np.array_equal(B.pi_neuron_table(h2, 0, 0, cfg.F), np.arange(cfg.F))
+    r0 = synth.token_input(cfg, 3)
+    a, _, sa, _ = G.decode_traced(h1, cfg, 0, 1, r0)
+    b, _, sb, _ = G.decode_traced(h2, cfg, 0, 1, r0)
+    assert abs(int(sa[0][0]) - int(sb[0][0])) <= 1
+    G.check_output(a - r0.double().numpy(), b - r0.double().numpy())
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(handles):
+    cfg = SMALL["reglu-f16"]
+    h, _ = _build(cfg, handles, n_layers=1)
+    r = synth.token_input(cfg, 0).cuda()
+    B.pi_debug_set(h, B.PI_DEBUG_STALL_BARRIER, 0.05)
+    B.pi_sparse_ffn_decode(h, 0, 1, r.clone())
+    assert B.pi_sync(h) == B.PI_ERR_TIMEOUT
+    B.pi_debug_set(h, 0, 2.0)
+    r2 = r.clone()
+    B.pi_sparse_ffn_decode(h, 0, 1, r2)
+    assert B.pi_sync(h) == B.PI_OK
+    assert torch.isfinite(r2).all() and not torch.equal(r2, r)
+
+
+# ---------------------------------------------------------------------------
+# Full-size workloads (launch configuration of the benchmark: one CTA per SM)
+# ---------------------------------------------------------------------------
+FULL = ["llama7b", "mistral7b", "falcon40b", "mixtral47b"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled_layers(handles, name):
+    cfg = synth.CONFIGS[name]
+    h = G.create(cfg)
+    handles.append(h)
+    for l in range(cfg.n_layers):
+        G.load(h, l, synth.make_layer(cfg, l, "cuda"))
+    torch.cuda.empty_cache()
+    sample = sorted({0, cfg.n_layers // 2, cfg.n_layers - 1})
+    for t in (0, 1):
+        r0 = synth.token_input(cfg, t)
+        rL, trace, stats, masks = G.decode_traced(h, cfg, 0, cfg.n_layers, r0)
+        assert np.all(np.isfinite(rL))
+        outs = list(trace[1:]) + [rL]
+        for l in sample:
+            lw = synth.make_layer(cfg, l, "cuda")
+            ex, router = G.oracle_layer(cfg, lw)
+            perms = G.tables(h, lw, l, cfg.F)
+            del lw
+            G.check_layer(cfg, ex, router, perms, trace[l], outs[l], stats[l], masks[l])
+        frac = stats[:, 0].mean() / (cfg.F * cfg.top_k)
+        assert abs(frac - cfg.mean_active) < 0.05, f"predicted active fraction {frac:.3f}"
