@@ -68,6 +68,7 @@ def lib() -> ctypes.CDLL:
             "pi_dense_ffn_prefill": [vp, ip, ip, ip, vp, vp],
             "pi_sync": [vp, vp],
             "pi_debug_set": [vp, ip, ctypes.c_double],
+            "pi_debug_phase_times": [vp, vp],
         }
         for name, args in sigs.items():
             f = getattr(L, name)
@@ -195,3 +196,7 @@ def pi_sync(h, stream=None) -> int:
 
 def pi_debug_set(h, flags: int, wait_limit_s: float):
     _check(lib().pi_debug_set(h, flags, wait_limit_s), "pi_debug_set")
+
+
+def pi_debug_phase_times(h, times=None):
+    _check(lib().pi_debug_phase_times(h, _ptr(times)), "pi_debug_phase_times")

@@ -86,6 +86,15 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         "l"(src), "r"(bytes), "r"(s2u(bar)), "l"(pol)
         : "memory");
 }
+// Bulk prefetch of a global range into L2 (fire and forget), in 32 KB pieces.
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes)
+{
+    const uint8_t *p = static_cast<const uint8_t *>(src);
+    for (uint32_t o = 0; o < bytes; o += 32768u) {
+        const uint32_t n = bytes - o < 32768u ? bytes - o : 32768u;
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p + o), "r"(n) : "memory");
+    }
+}
 __device__ __forceinline__ long long gtimer()
 {
     long long t;
@@ -110,9 +119,15 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p)
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
-__device__ __forceinline__ void red_release_gpu(unsigned *p, unsigned v)
+__device__ __forceinline__ unsigned atom_add_acqrel_gpu(unsigned *p, unsigned v)
 {
-    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+__device__ __forceinline__ void st_release_gpu(unsigned *p, unsigned v)
+{
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -237,7 +252,7 @@ __device__ __forceinline__ float act_h(int act, float g, float u)
 // ---------------------------------------------------------------------------
 // Shared-memory control block
 // ---------------------------------------------------------------------------
-enum GType { kGate = 0, kUp = 1, kDown = 2 };
+enum GType { kGU = 0, kDown = 2 };   // a neuron's input record, or its W_down row
 struct GDesc {
     int type, e, k;
     float h;
@@ -296,6 +311,17 @@ __device__ __forceinline__ int make_pieces(int r, int ntop, int a0, int a1, int 
     return n;
 }
 
+__device__ __forceinline__ void prof_mark(const DecodeParams &p, int li, int point)
+{
+    if (p.prof && threadIdx.x == 0)
+        p.prof[(size_t(li) * kProfPoints + point) * gridDim.x + blockIdx.x] = gtimer();
+}
+__device__ __forceinline__ void prof_put(const DecodeParams &p, int li, int point, long long v)
+{
+    if (p.prof && threadIdx.x == 0)
+        p.prof[(size_t(li) * kProfPoints + point) * gridDim.x + blockIdx.x] = v;
+}
+
 __device__ void set_error(int *err, int code)
 {
     atomicCAS(err, 0, code);
@@ -323,9 +349,13 @@ __device__ bool wait_phase(uint64_t *bar, uint32_t parity, Ctl *ctl, const Decod
 // Collective wait of the 256 consumer threads: thread 0 waits (bounded) and
 // broadcasts the outcome, so every consumer thread takes the same branch.
 __device__ __forceinline__ bool cwait(uint64_t *bar, uint32_t parity, Ctl *ctl,
-                                      const DecodeParams &p, int &bci)
+                                      const DecodeParams &p, int &bci, long long *wait_cyc = nullptr)
 {
-    if (threadIdx.x == 0) st_vol(&ctl->bc[bci], wait_phase(bar, parity, ctl, p) ? 1 : 0);
+    if (threadIdx.x == 0) {
+        const long long c0 = clock64();
+        st_vol(&ctl->bc[bci], wait_phase(bar, parity, ctl, p) ? 1 : 0);
+        if (wait_cyc) *wait_cyc += clock64() - c0;
+    }
     cons_sync();
     const bool ok = ld_vol(&ctl->bc[bci]) != 0;
     bci ^= 1;
@@ -334,34 +364,43 @@ __device__ __forceinline__ bool cwait(uint64_t *bar, uint32_t parity, Ctl *ctl,
 }
 
 // Grid-wide barrier of the consumer warps of all CTAs (one cooperative launch).
-__device__ bool grid_sync(Ctl *ctl, const DecodeParams &p, unsigned &epoch, int &bci)
+// bar[0] counts arrivals (never reset within a launch); the CTA whose arrival
+// completes barrier `epoch` publishes it in bar[1]; the others wait for that
+// generation word, so the waiting CTAs poll a line that changes once.
+__device__ bool grid_sync(Ctl *ctl, const DecodeParams &p, unsigned &epoch, int &bci,
+                          long long *wait_cyc = nullptr)
 {
     cons_sync();
+    const long long c0 = clock64();
     if (threadIdx.x == 0) {
         bool ok = ld_vol(&ctl->abort_flag) == 0;
         epoch += 1;
         if (ok) {
-            unsigned target = epoch * gridDim.x;
-            if ((p.debug_flags & 1) && epoch == 1) target += 1;   // PI_DEBUG_STALL_BARRIER
+            unsigned last = epoch * gridDim.x - 1;
+            if ((p.debug_flags & 1) && epoch == 1) last += 1;   // PI_DEBUG_STALL_BARRIER
             __threadfence();
-            red_release_gpu(p.bar, 1u);
-            const long long t0 = gtimer();
-            unsigned it = 0;
-            while (ld_acquire_gpu(p.bar) < target) {
-                __nanosleep(32);
-                if ((++it & 63) == 0) {
-                    if (ld_vol(&ctl->abort_flag)) { ok = false; break; }
-                    if (gtimer() - t0 > p.wait_ns) {
-                        st_vol(&ctl->abort_flag, 1);
-                        set_error(p.err, kDevTimeout);
-                        ok = false;
-                        break;
+            const unsigned old = atom_add_acqrel_gpu(p.bar, 1u);
+            if (old == last) {
+                st_release_gpu(p.bar + 1, epoch);
+            } else {
+                const long long t0 = gtimer();
+                unsigned it = 0;
+                while (ld_acquire_gpu(p.bar + 1) < epoch) {
+                    if ((++it & 31) == 0) {
+                        if (ld_vol(&ctl->abort_flag)) { ok = false; break; }
+                        if (gtimer() - t0 > p.wait_ns) {
+                            st_vol(&ctl->abort_flag, 1);
+                            set_error(p.err, kDevTimeout);
+                            ok = false;
+                            break;
+                        }
                     }
                 }
             }
             __threadfence();
         }
         st_vol(&ctl->bc[bci], ok ? 1 : 0);
+        if (wait_cyc) *wait_cyc += clock64() - c0;
     }
     cons_sync();
     const bool ok = ld_vol(&ctl->bc[bci]) != 0;
@@ -444,15 +483,33 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         const uint64_t pol = policy_evict_first();
         int pi = 0;
         bool ok = true;
+        // L2 prefetch of all predictor bytes a layer will stream into this CTA
+        auto prefetch_layer = [&](int l, const int *experts) {
+            Piece pc[2 * kMaxTopK];
+            const int npc = make_pieces(r, ntop, a0, a1, s0, ns, pc);
+            for (int q = 0; q < npc; ++q) {
+                const ExpertDev &ex = p.ex[size_t(l) * p.E + experts[pc[q].slot]];
+                const int rowb = pc[q].kind == 0 ? p.vrow : p.urow;
+                const uint8_t *base = pc[q].kind == 0 ? ex.V : ex.U;
+                prefetch_l2(base + size_t(pc[q].row0) * rowb, uint32_t(pc[q].nrows) * rowb);
+            }
+        };
+        const bool dense_ahead = !predict && p.E == 1;   // experts known ahead of time
+        if (dense_ahead) {
+            const int e0[kMaxTopK] = {0, 0};
+            prefetch_layer(l0, e0);
+        }
         for (int l = l0; l < l1 && ok; ++l) {
             const int lp = (l - l0) & 1;
             int experts[kMaxTopK] = {0, 0};
             if (predict) {
                 experts[0] = p.pred_expert;
+                prefetch_layer(l, experts);
             } else if (p.E > 1) {
                 if (!wait_phase(&ctl->route_ready, (l - l0) & 1, ctl, p)) { ok = false; break; }
                 experts[0] = ctl->route_e[lp][0];
                 experts[1] = ctl->route_e[lp][1];
+                prefetch_layer(l, experts);
             }
             Piece pc[2 * kMaxTopK];
             const int npc = make_pieces(r, ntop, a0, a1, s0, ns, pc);
@@ -472,6 +529,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     ++pi;
                 }
             }
+            if (ok && dense_ahead && l + 1 < l1) {
+                const int e0[kMaxTopK] = {0, 0};
+                prefetch_layer(l + 1, e0);
+            }
         }
         if (!ok) drain_ring(ctl->p_full, NP, pi, p.wait_ns);
         return;
@@ -485,12 +546,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         const uint64_t pol = policy_evict_first();
         int gi = 0, rep_base = 0, dq_head = 0;
         bool ok = true;
-        auto issue = [&](int type, int e, int k, float h, const uint8_t *src) -> bool {
+        auto issue = [&](int type, int e, int k, float h, const uint8_t *src, int bytes) -> bool {
             const int s = gi % NG;
             if (!wait_phase(&ctl->g_empty[s], ((gi / NG) & 1) ^ 1, ctl, p)) return false;
             ctl->gdesc[s] = GDesc{type, e, k, h};
-            mbar_arrive_tx(&ctl->g_full[s], uint32_t(p.wrow));
-            bulk_g2s(gring + size_t(s) * SG, src, uint32_t(p.wrow), &ctl->g_full[s], pol);
+            mbar_arrive_tx(&ctl->g_full[s], uint32_t(bytes));
+            bulk_g2s(gring + size_t(s) * SG, src, uint32_t(bytes), &ctl->g_full[s], pol);
             ++gi;
             return true;
         };
@@ -502,10 +563,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             const int ex0 = p.E > 1 ? ctl->route_e[lp][0] : 0;
             const int ex1 = p.E > 1 ? ctl->route_e[lp][1] : 0;
             const ExpertDev *exs[2] = {&p.ex[size_t(l) * p.E + ex0], &p.ex[size_t(l) * p.E + ex1]};
+            // every row this CTA may need this layer starts moving towards L2 now
+            for (int j = 0; j < m; ++j) {
+                const int e = j < m0 ? 0 : 1;
+                const int k = ctl->lst[lp][e][j < m0 ? j : j - m0];
+                prefetch_l2(exs[e]->Wgu + size_t(s0 + k) * p.gu_bytes, uint32_t(p.gu_bytes));
+                if (p.spec_down)
+                    prefetch_l2(exs[e]->Wd + size_t(s0 + k) * p.wrow, uint32_t(p.wrow));
+            }
             const int rep_target = rep_base + m;
             int gu = 0;
-            const long long t_idle0 = gtimer();
-            long long idle_since = t_idle0;
+            long long idle_since = gtimer();
             while (ok) {
                 const int tail = ld_vol(&ctl->dq_tail);
                 if (dq_head < tail) {
@@ -514,15 +582,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     const float h = *reinterpret_cast<volatile float *>(&ctl->dqh[q]);
                     ++dq_head;
                     const int e = ent >> 16, k = ent & 0xffff;
-                    ok = issue(kDown, e, k, h, exs[e]->Wd + size_t(s0 + k) * p.wrow);
+                    ok = issue(kDown, e, k, h, exs[e]->Wd + size_t(s0 + k) * p.wrow, p.wrow);
                     idle_since = gtimer();
                 } else if (gu < m) {
                     const int e = gu < m0 ? 0 : 1;
                     const int k = ctl->lst[lp][e][gu < m0 ? gu : gu - m0];
                     ++gu;
-                    ok = issue(kGate, e, k, 0.f, exs[e]->Wg + size_t(s0 + k) * p.wrow);
-                    if (ok && p.gated)
-                        ok = issue(kUp, e, k, 0.f, exs[e]->Wu + size_t(s0 + k) * p.wrow);
+                    ok = issue(kGU, e, k, 0.f, exs[e]->Wgu + size_t(s0 + k) * p.gu_bytes, p.gu_bytes);
                     idle_since = gtimer();
                 } else {
                     if (ld_vol(&ctl->h_rep) >= rep_target) {
@@ -559,16 +625,50 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         const int li = l - l0;
 
         // ---------------- phase A: layer input, routing, t = V x ----------
+        prof_mark(p, li, 0);
+        long long wc_a = 0, wc_b = 0, wc_c = 0, wc_bar = 0;
         float inv = 1.f;
         const float *src = predict ? p.x_in : p.resid;
+        // one round trip to L2: this thread's columns in both row formats
+#pragma unroll
+        for (int k = 0; k < MAXVW; ++k) {
+            const int v = tid + kConsumers * k;
+#pragma unroll
+            for (int i = 0; i < EPVW; i += 4) {
+                float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (v < nvecW) q = __ldcg(reinterpret_cast<const float4 *>(src + v * EPVW + i));
+                xw[k * EPVW + i] = q.x; xw[k * EPVW + i + 1] = q.y;
+                xw[k * EPVW + i + 2] = q.z; xw[k * EPVW + i + 3] = q.w;
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < MAXVP; ++k) {
+            const int v = tid + kConsumers * k;
+#pragma unroll
+            for (int i = 0; i < EPVP; i += 4) {
+                float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (v < nvecP) q = __ldcg(reinterpret_cast<const float4 *>(src + v * EPVP + i));
+                xp[k * EPVP + i] = q.x; xp[k * EPVP + i + 1] = q.y;
+                xp[k * EPVP + i + 2] = q.z; xp[k * EPVP + i + 3] = q.w;
+            }
+        }
         if (!predict) {
+            // x = r / sqrt(mean(r^2) + eps); the W-format columns cover d once
             float ss = 0.f;
-            for (int j = tid * 4; j < d; j += kConsumers * 4) {
-                const float4 v = __ldcg(reinterpret_cast<const float4 *>(src + j));
-                ss = fmaf(v.x, v.x, ss); ss = fmaf(v.y, v.y, ss);
-                ss = fmaf(v.z, v.z, ss); ss = fmaf(v.w, v.w, ss);
-                if (p.trace && b == 0)
-                    __stcg(reinterpret_cast<float4 *>(p.trace + size_t(li) * d + j), v);
+#pragma unroll
+            for (int k = 0; k < MAXVW; ++k) {
+                const int v = tid + kConsumers * k;
+                if (v < nvecW) {
+#pragma unroll
+                    for (int i = 0; i < EPVW; ++i) ss = fmaf(xw[k * EPVW + i], xw[k * EPVW + i], ss);
+                    if (p.trace && b == 0) {
+#pragma unroll
+                        for (int i = 0; i < EPVW; i += 4)
+                            __stcg(reinterpret_cast<float4 *>(p.trace + size_t(li) * d + v * EPVW + i),
+                                   make_float4(xw[k * EPVW + i], xw[k * EPVW + i + 1],
+                                               xw[k * EPVW + i + 2], xw[k * EPVW + i + 3]));
+                    }
+                }
             }
             ss = warp_sum(ss);
             if (lane == 0) ctl->red[rb][warp][16] = ss;
@@ -581,28 +681,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             cons_sync();
             inv = ctl->inv_rms;
             rb ^= 1;
-        }
 #pragma unroll
-        for (int k = 0; k < MAXVW; ++k) {
-            const int v = tid + kConsumers * k;
+            for (int i = 0; i < MAXVW * EPVW; ++i) xw[i] *= inv;
 #pragma unroll
-            for (int i = 0; i < EPVW; i += 4) {
-                float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (v < nvecW) q = __ldcg(reinterpret_cast<const float4 *>(src + v * EPVW + i));
-                xw[k * EPVW + i] = q.x * inv; xw[k * EPVW + i + 1] = q.y * inv;
-                xw[k * EPVW + i + 2] = q.z * inv; xw[k * EPVW + i + 3] = q.w * inv;
-            }
-        }
-#pragma unroll
-        for (int k = 0; k < MAXVP; ++k) {
-            const int v = tid + kConsumers * k;
-#pragma unroll
-            for (int i = 0; i < EPVP; i += 4) {
-                float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (v < nvecP) q = __ldcg(reinterpret_cast<const float4 *>(src + v * EPVP + i));
-                xp[k * EPVP + i] = q.x * inv; xp[k * EPVP + i + 1] = q.y * inv;
-                xp[k * EPVP + i + 2] = q.z * inv; xp[k * EPVP + i + 3] = q.w * inv;
-            }
+            for (int i = 0; i < MAXVP * EPVP; ++i) xp[i] *= inv;
         }
 
         // MoE routing, computed identically by every CTA: logits of the E
@@ -659,6 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
 
         // t rows [a0, a1): consume the V chunks of the P ring
+        prof_mark(p, li, 1);
         bool alive = true;
         {
             Piece pc[2 * kMaxTopK];
@@ -668,7 +751,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 for (int row = 0; row < pc[q].nrows; row += RV) {
                     const int n = min(RV, pc[q].nrows - row);
                     const int s = pc_i % NP;
-                    if (!cwait(&ctl->p_full[s], (pc_i / NP) & 1, ctl, p, bci)) { alive = false; break; }
+                    if (!cwait(&ctl->p_full[s], (pc_i / NP) & 1, ctl, p, bci, &wc_a)) { alive = false; break; }
                     const uint8_t *slot = pring + size_t(s) * kPSlotBytes;
                     float part[MAXRV];
 #pragma unroll
@@ -693,7 +776,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 }
             }
         }
-        if (!alive || !grid_sync(ctl, p, epoch, bci)) break;
+        prof_mark(p, li, 2);
+        if (!alive || !grid_sync(ctl, p, epoch, bci, &wc_bar)) break;
+        prof_mark(p, li, 3);
 
         // ---------------- phase B: z = U t - c, threshold, compaction -----
         for (int i = tid; i < ntop * r; i += kConsumers) ctl->tsm[i] = __ldcg(p.t_buf + i);
@@ -714,7 +799,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             for (int row = 0; row < ns; row += RU) {
                 const int n = min(RU, ns - row);
                 const int s = pc_i % NP;
-                if (!cwait(&ctl->p_full[s], (pc_i / NP) & 1, ctl, p, bci)) { alive = false; break; }
+                if (!cwait(&ctl->p_full[s], (pc_i / NP) & 1, ctl, p, bci, &wc_b)) { alive = false; break; }
                 const uint8_t *slot = pring + size_t(s) * kPSlotBytes;
                 for (int rr = warp; rr < n; rr += kConsumerWarps) {
                     const uint8_t *urow = slot + size_t(rr) * p.urow;
@@ -744,6 +829,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
         if (!alive) break;
         cons_sync();
+        prof_mark(p, li, 4);
         // compaction in ascending strip order: warp e builds expert slot e's list
         if (warp < ntop) {
             const int e = warp;
@@ -790,6 +876,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
 
         if (tid == 0) mbar_arrive(&ctl->list_ready);
+        prof_mark(p, li, 5);
 
         // ---------------- phase C: gather rows of active neurons ----------
         float acc[MAXVW * EPVW];
@@ -801,7 +888,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             int gu_done = 0, dn_done = 0, nnz = 0;
             for (int iter = 0; (gu_done < m || dn_done < nnz) && iter < cap; ++iter) {
                 const int s = gs % NG;
-                if (!cwait(&ctl->g_full[s], (gs / NG) & 1, ctl, p, bci)) { alive = false; break; }
+                if (!cwait(&ctl->g_full[s], (gs / NG) & 1, ctl, p, bci, &wc_c)) { alive = false; break; }
                 const GDesc dsc = ctl->gdesc[s];
                 const uint8_t *row = gring + size_t(s) * SG;
                 if (dsc.type == kDown) {
@@ -812,20 +899,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     ++dn_done;
                     continue;
                 }
-                // gate (or W_1) row, then the up row when gated
+                // the neuron's input record: gate (or W_1) row, then its up row
                 float pg = dot_row<WF, MAXVW>(row, xw, nvecW, d);
+                float pu = 0.f;
+                if (p.gated) pu = dot_row<WF, MAXVW>(row + p.wrow, xw, nvecW, d);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ctl->g_empty[s]);
                 ++gs;
-                float pu = 0.f;
-                if (p.gated) {
-                    const int s2 = gs % NG;
-                    if (!cwait(&ctl->g_full[s2], (gs / NG) & 1, ctl, p, bci)) { alive = false; break; }
-                    pu = dot_row<WF, MAXVW>(gring + size_t(s2) * SG, xw, nvecW, d);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&ctl->g_empty[s2]);
-                    ++gs;
-                }
                 pg = warp_sum(pg);
                 pu = warp_sum(pu);
                 if (lane == 0) {
@@ -861,6 +941,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             if (tid == 0 && p.stats) atomicAdd(p.stats + li * 4 + 1, nnz);
         }
         if (!alive) break;
+        prof_mark(p, li, 6);
         // per-CTA partial of y
 #pragma unroll
         for (int k = 0; k < MAXVW; ++k) {
@@ -873,7 +954,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                                        acc[k * EPVW + i + 2], acc[k * EPVW + i + 3]));
             }
         }
-        if (!grid_sync(ctl, p, epoch, bci)) break;
+        if (!grid_sync(ctl, p, epoch, bci, &wc_bar)) break;
+        prof_mark(p, li, 7);
 
         // ---------------- phase D: r += sum of partials (fixed order) -----
         {
@@ -894,7 +976,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 }
             }
         }
-        if (!grid_sync(ctl, p, epoch, bci)) break;
+        prof_mark(p, li, 8);
+        if (!grid_sync(ctl, p, epoch, bci, &wc_bar)) break;
+        prof_mark(p, li, 9);
+        prof_put(p, li, 10, wc_a);
+        prof_put(p, li, 11, wc_b);
+        prof_put(p, li, 12, wc_c);
+        prof_put(p, li, 13, wc_bar);
     }
 }
 

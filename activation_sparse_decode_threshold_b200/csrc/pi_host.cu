@@ -85,6 +85,7 @@ struct pi_ffn {
     int *err = nullptr;
     long long wait_ns = 2000000000LL;
     int debug_flags = 0;
+    long long *prof = nullptr;
     pi::PrefillState *prefill = nullptr;
 };
 
@@ -156,15 +157,16 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
     // shared-memory rings: 6 predictor slots of 16 KB, gather slots fill the rest
     const size_t budget = size_t(prop.sharedMemPerBlockOptin);
     h->np = 6;
-    const size_t base = pi::decode_smem_bytes(h->np, 0, h->wrow);
-    int ng = base < budget ? int((budget - base) / size_t(h->wrow)) : 0;
+    const int sg = (h->gated ? 2 : 1) * h->wrow;   // a gather slot holds one input record
+    const size_t base = pi::decode_smem_bytes(h->np, 0, sg);
+    int ng = base < budget ? int((budget - base) / size_t(sg)) : 0;
     ng = std::min(ng, pi::kMaxGSlots);
     if (ng < 2) {
         delete h;
         return fail(PI_ERR_UNSUPPORTED, "shared memory too small for the gather ring");
     }
     h->ng = ng;
-    h->smem = pi::decode_smem_bytes(h->np, h->ng, h->wrow);
+    h->smem = pi::decode_smem_bytes(h->np, h->ng, sg);
     const int per_sm = pi::decode_max_blocks_per_sm(h->wfmt, h->pfmt, D.d_model, h->smem);
     if (per_sm < 1 || h->S > per_sm * prop.multiProcessorCount) {
         delete h;
@@ -304,12 +306,12 @@ pi_status pi_ffn_load_layer(pi_ffn_t h, int layer, const pi_expert_weights *expe
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     PI_CUDA(cudaSetDevice(D.device), "cudaSetDevice");
+    const int gu_bytes = (h->gated ? 2 : 1) * h->wrow;
     const size_t o_V = 0;
     const size_t o_U = up256(o_V + size_t(r) * h->vrow);
     const size_t o_c = up256(o_U + size_t(F) * h->urow);
     const size_t o_g = up256(o_c + sizeof(float) * F);
-    const size_t o_u = up256(o_g + size_t(F) * h->wrow);
-    const size_t o_d = up256(o_u + (h->gated ? size_t(F) * h->wrow : 0));
+    const size_t o_d = up256(o_g + size_t(F) * gu_bytes);
     const size_t total = up256(o_d + size_t(F) * h->wrow);
     int32_t *d_perm = nullptr;
     PI_CUDA(cudaMallocAsync(&d_perm, sizeof(int32_t) * F, st), "cudaMallocAsync(perm)");
@@ -322,24 +324,29 @@ pi_status pi_ffn_load_layer(pi_ffn_t h, int layer, const pi_expert_weights *expe
         PI_CUDA(cudaMemcpyAsync(d_perm, h->perm[idx].data(), sizeof(int32_t) * F,
                                 cudaMemcpyHostToDevice, st), "copy perm");
         PI_CUDA(cudaMemcpyAsync(m + o_V, w.V, size_t(r) * h->vrow, cudaMemcpyDeviceToDevice, st), "copy V");
-        PI_CUDA(pi::repack_rows(static_cast<const uint8_t *>(w.U), m + o_U, d_perm, F, h->urow, nullptr, 0, st),
-                "repack U");
+        {
+            const uint8_t *src[1] = {static_cast<const uint8_t *>(w.U)};
+            const int rb[1] = {h->urow};
+            PI_CUDA(pi::repack_rows(m + o_U, d_perm, F, 1, src, rb, st), "repack U");
+        }
         PI_CUDA(pi::repack_bias(w.bias, reinterpret_cast<float *>(m + o_c), d_perm, F, st), "repack c");
+        const uint8_t *g8 = static_cast<const uint8_t *>(w.w_gate);
+        const uint8_t *u8 = static_cast<const uint8_t *>(w.w_up);
         if (int4) {
             const int qb = d / 2, sb = d / 16;
-            PI_CUDA(pi::repack_rows(static_cast<const uint8_t *>(w.w_gate), m + o_g, d_perm, F, qb,
-                                    static_cast<const uint8_t *>(w.s_gate), sb, st), "repack gate");
-            if (h->gated)
-                PI_CUDA(pi::repack_rows(static_cast<const uint8_t *>(w.w_up), m + o_u, d_perm, F, qb,
-                                        static_cast<const uint8_t *>(w.s_up), sb, st), "repack up");
-            PI_CUDA(pi::repack_rows(static_cast<const uint8_t *>(w.w_down), m + o_d, d_perm, F, qb,
-                                    static_cast<const uint8_t *>(w.s_down), sb, st), "repack down");
+            const uint8_t *sg8 = static_cast<const uint8_t *>(w.s_gate);
+            const uint8_t *su8 = static_cast<const uint8_t *>(w.s_up);
+            const uint8_t *src[4] = {g8, sg8, u8, su8};
+            const int rb[4] = {qb, sb, qb, sb};
+            PI_CUDA(pi::repack_rows(m + o_g, d_perm, F, h->gated ? 4 : 2, src, rb, st), "repack gate/up");
+            const uint8_t *dsrc[2] = {static_cast<const uint8_t *>(w.w_down),
+                                      static_cast<const uint8_t *>(w.s_down)};
+            const int drb[2] = {qb, sb};
+            PI_CUDA(pi::repack_rows(m + o_d, d_perm, F, 2, dsrc, drb, st), "repack down");
         } else {
-            PI_CUDA(pi::repack_rows(static_cast<const uint8_t *>(w.w_gate), m + o_g, d_perm, F, h->wrow,
-                                    nullptr, 0, st), "repack gate");
-            if (h->gated)
-                PI_CUDA(pi::repack_rows(static_cast<const uint8_t *>(w.w_up), m + o_u, d_perm, F, h->wrow,
-                                        nullptr, 0, st), "repack up");
+            const uint8_t *src[2] = {g8, u8};
+            const int rb[2] = {h->wrow, h->wrow};
+            PI_CUDA(pi::repack_rows(m + o_g, d_perm, F, h->gated ? 2 : 1, src, rb, st), "repack gate/up");
             PI_CUDA(pi::repack_down_transpose(static_cast<const uint8_t *>(w.w_down), m + o_d, d_perm, d,
                                               F, elem_bytes(D.w_dtype), st), "transpose down");
         }
@@ -347,8 +354,7 @@ pi_status pi_ffn_load_layer(pi_ffn_t h, int layer, const pi_expert_weights *expe
         x.V = m + o_V;
         x.U = m + o_U;
         x.c = reinterpret_cast<const float *>(m + o_c);
-        x.Wg = m + o_g;
-        x.Wu = h->gated ? m + o_u : nullptr;
+        x.Wgu = m + o_g;
         x.Wd = m + o_d;
         // the table is reused for the next expert: finish this one first
         PI_CUDA(cudaStreamSynchronize(st), "load_layer sync");
@@ -402,9 +408,11 @@ static pi::DecodeParams base_params(pi_ffn_t h)
     p.vrow = h->vrow;
     p.urow = h->urow;
     p.wrow = h->wrow;
+    p.gu_bytes = (h->gated ? 2 : 1) * h->wrow;
+    p.spec_down = D.act != PI_ACT_DRELU;
     p.np_slots = h->np;
     p.ng_slots = h->ng;
-    p.sg_bytes = h->wrow;
+    p.sg_bytes = p.gu_bytes;
     p.t_buf = h->t_buf;
     p.partials = h->partials;
     p.lists = h->lists;
@@ -413,6 +421,7 @@ static pi::DecodeParams base_params(pi_ffn_t h)
     p.err = h->err;
     p.wait_ns = h->wait_ns;
     p.debug_flags = h->debug_flags;
+    p.prof = h->prof;
     return p;
 }
 
@@ -436,7 +445,7 @@ pi_status pi_predict(pi_ffn_t h, int layer, int expert, const float *x_dev, int3
     p.z_out = z_dev;
     p.idx_out = idx_dev;
     p.count_out = count_dev;
-    PI_CUDA(cudaMemsetAsync(h->bar, 0, sizeof(unsigned), st), "memset barrier");
+    PI_CUDA(cudaMemsetAsync(h->bar, 0, 2 * sizeof(unsigned), st), "memset barrier");
     PI_CUDA(pi::launch_decode(h->wfmt, h->pfmt, p, h->smem, st), "launch predict");
     return PI_OK;
 }
@@ -464,7 +473,7 @@ pi_status pi_sparse_ffn_decode(pi_ffn_t h, int layer_begin, int layer_end, float
     p.trace = trace_dev;
     p.stats = stats_dev;
     p.masks = mask_dev;
-    PI_CUDA(cudaMemsetAsync(h->bar, 0, sizeof(unsigned), st), "memset barrier");
+    PI_CUDA(cudaMemsetAsync(h->bar, 0, 2 * sizeof(unsigned), st), "memset barrier");
     if (stats_dev) PI_CUDA(cudaMemsetAsync(stats_dev, 0, sizeof(int32_t) * 4 * nl, st), "memset stats");
     if (mask_dev)
         PI_CUDA(cudaMemsetAsync(mask_dev, 0, sizeof(uint32_t) * size_t(nl) * D.top_k * ((D.d_ff + 31) / 32), st),
@@ -509,6 +518,15 @@ pi_status pi_debug_set(pi_ffn_t h, int flags, double wait_limit_s)
         return fail(PI_ERR_INVALID_ARG, "wait_limit_s must be in (0, 60]");
     h->debug_flags = flags;
     h->wait_ns = static_cast<long long>(wait_limit_s * 1e9);
+    return PI_OK;
+}
+
+pi_status pi_debug_phase_times(pi_ffn_t h, long long *times_dev)
+{
+    if (!h) return fail(PI_ERR_INVALID_ARG, "null handle");
+    if (times_dev && (reinterpret_cast<uintptr_t>(times_dev) & 7u))
+        return fail(PI_ERR_INVALID_ARG, "times_dev must be 8-byte aligned");
+    h->prof = times_dev;
     return PI_OK;
 }
 

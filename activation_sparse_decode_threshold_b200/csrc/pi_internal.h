@@ -26,12 +26,15 @@ constexpr int kPSlotBytes = 16384;
 enum Fmt { kF32 = 0, kF16 = 1, kBF16 = 2, kI4 = 3 };
 
 // One expert (or dense FFN) of one layer, in table order, library-owned.
+// A neuron's input record holds its W_gate row followed by its W_up row when
+// gated (2 * wrow bytes), or its W_1 row when non-gated (wrow bytes), so one
+// bulk copy brings everything the neuron's activation needs.  An INT4 row is
+// its d/2 nibble bytes followed by its d/32 fp16 scales.
 struct ExpertDev {
     const uint8_t *V;    // r rows of vrow bytes (original order; rank is not permuted)
     const uint8_t *U;    // F rows of urow bytes, table order
     const float *c;      // F biases, table order
-    const uint8_t *Wg;   // F rows of wrow bytes (W_1 when non-gated)
-    const uint8_t *Wu;   // F rows of wrow bytes, or null when non-gated
+    const uint8_t *Wgu;  // F input records of gu_bytes, table order
     const uint8_t *Wd;   // F rows of wrow bytes: W_down columns, neuron-major
 };
 
@@ -45,6 +48,8 @@ struct DecodeParams {
     int layer_begin, layer_end;
     float threshold, eps;
     int vrow, urow, wrow;           // row bytes: V (pred fmt), U (pred fmt), W (weight fmt)
+    int gu_bytes;                   // bytes of a neuron's input record (2 * wrow gated)
+    int spec_down;                  // prefetch down rows of all predicted-active neurons
     int np_slots, ng_slots, sg_bytes;
     int mode, pred_expert;
     // inputs / outputs
@@ -60,20 +65,27 @@ struct DecodeParams {
     float *partials;                // [S * d]
     int32_t *lists;                 // [S * kMaxStrip]  (predict)
     int32_t *counts;                // [S]              (predict)
-    unsigned *bar;                  // grid barrier counter, zeroed before launch
+    unsigned *bar;                  // [2] grid barrier: arrivals, generation; zeroed before launch
     int *err;                       // device error word (0 = ok)
     long long wait_ns;              // bound on every device-side wait
     int debug_flags;
+    long long *prof;                // [(l1-l0) * kProfPoints * S] phase timestamps, or null
 };
+
+// Phase timestamps recorded per layer and CTA when DecodeParams::prof is set.
+constexpr int kProfPoints = 14;   // 10 timestamps + 4 cycle counters
 
 size_t decode_smem_bytes(int np_slots, int ng_slots, int sg_bytes);
 cudaError_t launch_decode(int wfmt, int pfmt, const DecodeParams &p, size_t smem,
                           cudaStream_t stream);
 int decode_max_blocks_per_sm(int wfmt, int pfmt, int d, size_t smem);
 
-// Load-time repack kernels (pi_repack.cu).
-cudaError_t repack_rows(const uint8_t *src, uint8_t *dst, const int32_t *perm, int rows,
-                        int row_bytes, const uint8_t *src2, int row2_bytes, cudaStream_t s);
+// Load-time repack kernels (pi_repack.cu).  repack_rows: dst record p is the
+// concatenation of row perm[p] of each of the n_src sources (row bytes each a
+// multiple of 16).
+constexpr int kMaxRepackSrc = 4;
+cudaError_t repack_rows(uint8_t *dst, const int32_t *perm, int rows, int n_src,
+                        const uint8_t *const *src, const int *row_bytes, cudaStream_t s);
 cudaError_t repack_bias(const float *src, float *dst, const int32_t *perm, int n, cudaStream_t s);
 cudaError_t repack_down_transpose(const uint8_t *w_down, uint8_t *dst, const int32_t *perm,
                                   int d, int F, int elem_bytes, cudaStream_t s);

@@ -2,9 +2,9 @@
 // table order (PowerInfer (unite.ai), "Neuron placement and management": a
 // table maps each stored neuron to its original position in the matrix).
 //
-//   repack_rows:  dst row p = src row perm[p] (optionally followed by the
-//                 matching row of a second matrix, used to keep each INT4
-//                 neuron's nibbles and scales in one contiguous record)
+//   repack_rows:  dst record p = row perm[p] of each source, concatenated
+//                 (a neuron's gate and up rows, and for INT4 their nibbles
+//                 and scales, become one contiguous record)
 //   repack_bias:  dst[p] = src[perm[p]]
 //   repack_down_transpose: W_down (d x F, output-major) -> neuron-major rows,
 //                 row p = column perm[p]; tiled through shared memory, reading
@@ -15,21 +15,26 @@
 namespace pi {
 namespace {
 
-__global__ void k_repack_rows(const uint8_t *__restrict__ src, uint8_t *__restrict__ dst,
-                              const int32_t *__restrict__ perm, int rows, int rb,
-                              const uint8_t *__restrict__ src2, int rb2)
+struct RepackSrc {
+    const uint8_t *src[kMaxRepackSrc];
+    int bytes[kMaxRepackSrc];
+    int n;
+};
+
+__global__ void k_repack_rows(uint8_t *__restrict__ dst, const int32_t *__restrict__ perm, int rows,
+                              RepackSrc rs)
 {
     const int p = blockIdx.x;
     if (p >= rows) return;
     const long long o = perm[p];
-    const int out_rb = rb + rb2;
-    const uint4 *s = reinterpret_cast<const uint4 *>(src + o * rb);
-    uint4 *t = reinterpret_cast<uint4 *>(dst + (long long)p * out_rb);
-    for (int i = threadIdx.x; i < rb / 16; i += blockDim.x) t[i] = s[i];
-    if (src2) {
-        const uint4 *s2 = reinterpret_cast<const uint4 *>(src2 + o * rb2);
-        uint4 *t2 = reinterpret_cast<uint4 *>(dst + (long long)p * out_rb + rb);
-        for (int i = threadIdx.x; i < rb2 / 16; i += blockDim.x) t2[i] = s2[i];
+    int out_rb = 0;
+    for (int i = 0; i < rs.n; ++i) out_rb += rs.bytes[i];
+    uint8_t *t = dst + (long long)p * out_rb;
+    for (int i = 0; i < rs.n; ++i) {
+        const uint4 *s = reinterpret_cast<const uint4 *>(rs.src[i] + o * rs.bytes[i]);
+        uint4 *tt = reinterpret_cast<uint4 *>(t);
+        for (int j = threadIdx.x; j < rs.bytes[i] / 16; j += blockDim.x) tt[j] = s[j];
+        t += rs.bytes[i];
     }
 }
 
@@ -66,11 +71,18 @@ __global__ void k_invert(const int32_t *__restrict__ perm, int32_t *__restrict__
 
 }  // namespace
 
-cudaError_t repack_rows(const uint8_t *src, uint8_t *dst, const int32_t *perm, int rows,
-                        int row_bytes, const uint8_t *src2, int row2_bytes, cudaStream_t s)
+cudaError_t repack_rows(uint8_t *dst, const int32_t *perm, int rows, int n_src,
+                        const uint8_t *const *src, const int *row_bytes, cudaStream_t s)
 {
     if (rows <= 0) return cudaSuccess;
-    k_repack_rows<<<rows, 128, 0, s>>>(src, dst, perm, rows, row_bytes, src2, src2 ? row2_bytes : 0);
+    if (n_src < 1 || n_src > kMaxRepackSrc) return cudaErrorInvalidValue;
+    RepackSrc rs{};
+    rs.n = n_src;
+    for (int i = 0; i < n_src; ++i) {
+        rs.src[i] = src[i];
+        rs.bytes[i] = row_bytes[i];
+    }
+    k_repack_rows<<<rows, 128, 0, s>>>(dst, perm, rows, rs);
     return cudaGetLastError();
 }
 

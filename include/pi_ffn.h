@@ -204,6 +204,17 @@ PI_API void pi_ffn_destroy(pi_ffn_t h);
 #define PI_DEBUG_STALL_BARRIER 1
 PI_API pi_status pi_debug_set(pi_ffn_t h, int flags, double wait_limit_s);
 
+/* Testing aid: when `times_dev` is non-NULL, each later pi_sparse_ffn_decode
+ * call records %globaltimer (ns) at ten points of every layer in every CTA:
+ * times_dev[((l - layer_begin) * 14 + k) * n_strips + cta], k = 0 layer start,
+ * 1 input ready, 2 t rows done, 3 after barrier 1, 4 logits done, 5 active
+ * list published, 6 gather done, 7 after barrier 2, 8 reduction done,
+ * 9 after barrier 3; k = 10..13 hold clock cycles thread 0 spent waiting for
+ * predictor data, logit data, gathered rows and grid barriers.  The buffer
+ * (caller-owned, device, 8-byte aligned) must
+ * hold (l1 - l0) * 14 * n_strips values.  NULL turns recording off. */
+PI_API pi_status pi_debug_phase_times(pi_ffn_t h, long long *times_dev);
+
 #ifdef __cplusplus
 }
 #endif
