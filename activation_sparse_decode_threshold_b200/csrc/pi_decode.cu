@@ -2,34 +2,37 @@
 //
 // One cooperative launch runs a range of layers for one token.  Each CTA owns
 // one strip of the neuron table (a contiguous run of table positions holding
-// a balanced share of hot neurons, hottest first).  Per layer:
+// a balanced share of hot neurons, hottest first) and a slice of the rows of
+// t = V x.  Per layer:
 //
 //   phase A  x = RMSNorm(r) (every CTA, identical arithmetic); [MoE] router +
-//            top-2 (every CTA, identical); rows [a0, a1) of t = V x.
+//            top-2 (every CTA, identical); the CTA's rows of t = V x.
 //   --- grid barrier ---
-//   phase B  z = U t - c for the CTA's strip; active iff z > threshold; the
-//            active list is compacted in ascending table order with warp
-//            ballots (PowerInfer (unite.ai), "Adaptive sparse predictor").
-//   phase C  for active neurons only: rows of W_gate / W_up -> h = act(g, u);
-//            for h != 0: the neuron's W_down column (stored as a row) is
+//   phase B  z = U t - c over the strip; active iff z > threshold; the active
+//            list is compacted in ascending table order with warp ballots
+//            (PowerInfer (unite.ai), "Adaptive sparse predictor").
+//   phase C  for active neurons only: the neuron's W_gate / W_up rows ->
+//            h = act(g, u); for h != 0 its W_down column (stored as a row) is
 //            accumulated into a per-CTA fp32 partial of y ("Neuron-aware
 //            operators": rows of the input matrices, columns of the output).
 //   --- grid barrier ---
-//   phase D  r <- r + sum of the per-CTA partials, in fixed CTA order, by
-//            column slices (deterministic; no atomics).  This is the merge of
-//            the per-processor partial results (nearauto.com PowerInfer
-//            article, Fig. 8), done in HBM-resident fp32 on one GPU.
+//   phase D  r <- r + sum of the per-CTA partials in fixed CTA order, by
+//            column slices (deterministic, no atomics): the merge of partial
+//            results (nearauto.com PowerInfer article, Fig. 8).
 //   --- grid barrier ---
 //
-// Warp roles: warps 0-7 compute.  Warp 8 streams the predictor weights (V rows
-// of the CTA's t slice, U rows of its strip), which do not depend on the
-// input, into a ring of 16 KB shared-memory slots with cp.async.bulk, running
-// ahead across layers as far as the ring allows.  Warp 9 streams the rows of
-// active neurons into a second ring: the gate/up rows as soon as the active
-// list is known, each down row as soon as its h is known to be non-zero.
-// Every slot carries a descriptor so consumers process the ring in issue
-// order.  All waits are bounded (%globaltimer); a wait that runs out records
-// an error word and every thread of the grid returns.
+// Memory strategy: every weight byte is first pulled into L2 with
+// cp.async.bulk.prefetch.L2 as early as its address is known -- the next
+// layer's predictor slice (V rows, U strip) while the current layer gathers,
+// a strip's active neuron records the moment its active list exists (and,
+// for ReLU / ReGLU, where h != 0 almost always follows z > 0, their W_down
+// rows too) -- and the 16 warps then read it with batched 128-bit loads:
+// many rows in flight per thread and one cross-warp reduction per batch.
+// The gather is software-pipelined: the W_down rows of batch i and the
+// W_gate/W_up records of batch i+1 are loaded together.  HBM traffic is the
+// algorithmic bytes (plus the speculative W_down rows whose h turns out 0).
+// All waits are bounded (%globaltimer); a wait that runs out records an
+// error word and every thread of the grid returns.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -41,6 +44,30 @@ namespace {
 // ---------------------------------------------------------------------------
 // PTX helpers
 // ---------------------------------------------------------------------------
+// Bulk prefetch of a global range into L2 (fire and forget), 32 KB pieces.
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes)
+{
+    const uint8_t *p = static_cast<const uint8_t *>(src);
+    for (uint32_t o = 0; o < bytes; o += 32768u) {
+        const uint32_t n = bytes - o < 32768u ? bytes - o : 32768u;
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p + o), "r"(n) : "memory");
+    }
+}
+// Read-only weight loads that do not allocate in L1.
+__device__ __forceinline__ uint4 ldw4(const uint8_t *p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint2 ldw2(const uint8_t *p)
+{
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
 __device__ __forceinline__ uint32_t s2u(const void *p)
 {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -48,10 +75,6 @@ __device__ __forceinline__ uint32_t s2u(const void *p)
 __device__ __forceinline__ void mbar_init(uint64_t *b, unsigned count)
 {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(s2u(b)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t *b)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(s2u(b)) : "memory");
 }
 __device__ __forceinline__ void mbar_arrive_tx(uint64_t *b, uint32_t bytes)
 {
@@ -70,30 +93,13 @@ __device__ __forceinline__ bool mbar_test(uint64_t *b, uint32_t parity)
         : "memory");
     return ok != 0;
 }
-__device__ __forceinline__ uint64_t policy_evict_first()
-{
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
 // 1-D bulk copy global -> this CTA's shared memory, completion on `bar`.
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
-                                         uint64_t *bar, uint64_t pol)
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
 {
     asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1], %2, [%3], %4;" ::"r"(s2u(dst)),
-        "l"(src), "r"(bytes), "r"(s2u(bar)), "l"(pol)
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(s2u(dst)), "l"(src), "r"(bytes), "r"(s2u(bar))
         : "memory");
-}
-// Bulk prefetch of a global range into L2 (fire and forget), in 32 KB pieces.
-__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes)
-{
-    const uint8_t *p = static_cast<const uint8_t *>(src);
-    for (uint32_t o = 0; o < bytes; o += 32768u) {
-        const uint32_t n = bytes - o < 32768u ? bytes - o : 32768u;
-        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p + o), "r"(n) : "memory");
-    }
 }
 __device__ __forceinline__ long long gtimer()
 {
@@ -101,9 +107,19 @@ __device__ __forceinline__ long long gtimer()
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-__device__ __forceinline__ void cons_sync()
+__device__ __forceinline__ void cta_sync()
 {
-    asm volatile("bar.sync 1, 256;" ::: "memory");
+    asm volatile("bar.sync 0;" ::: "memory");
+}
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p)
+{
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void red_release_gpu(unsigned *p, unsigned v)
+{
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 __device__ __forceinline__ int ld_vol(const int *p)
 {
@@ -113,50 +129,39 @@ __device__ __forceinline__ void st_vol(int *p, int v)
 {
     *reinterpret_cast<volatile int *>(p) = v;
 }
-__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p)
-{
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ unsigned atom_add_acqrel_gpu(unsigned *p, unsigned v)
-{
-    unsigned old;
-    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-    return old;
-}
-__device__ __forceinline__ void st_release_gpu(unsigned *p, unsigned v)
-{
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
 
 // ---------------------------------------------------------------------------
-// Stored formats: one vector = 16 bytes (8 bytes for INT4) of a row.
+// Stored formats.  A vector is 16 bytes of a row (8 bytes for INT4: 16
+// nibbles, half of a 32-element scale group).
 // ---------------------------------------------------------------------------
 template <int F> struct Fm;
-template <> struct Fm<kF32>  { static constexpr int VB = 16, EPV = 4; };
-template <> struct Fm<kF16>  { static constexpr int VB = 16, EPV = 8; };
-template <> struct Fm<kBF16> { static constexpr int VB = 16, EPV = 8; };
-template <> struct Fm<kI4>   { static constexpr int VB = 8, EPV = 16; };
+template <> struct Fm<kF32>  { static constexpr int VB = 16, EPV = 4;  using V = uint4; };
+template <> struct Fm<kF16>  { static constexpr int VB = 16, EPV = 8;  using V = uint4; };
+template <> struct Fm<kBF16> { static constexpr int VB = 16, EPV = 8;  using V = uint4; };
+template <> struct Fm<kI4>   { static constexpr int VB = 8,  EPV = 16; using V = uint2; };
 
 template <int F>
-__device__ __forceinline__ void load_vec(const uint8_t *p, float *o)
+__device__ __forceinline__ typename Fm<F>::V ldvec(const uint8_t *p)
+{
+    if constexpr (F == kI4) return ldw2(p);
+    else return ldw4(p);
+}
+
+template <int F>
+__device__ __forceinline__ void cvt(const typename Fm<F>::V &v, float *o)
 {
     if constexpr (F == kF32) {
-        float4 v = *reinterpret_cast<const float4 *>(p);
-        o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+        o[0] = __uint_as_float(v.x); o[1] = __uint_as_float(v.y);
+        o[2] = __uint_as_float(v.z); o[3] = __uint_as_float(v.w);
     } else if constexpr (F == kF16) {
-        uint4 v = *reinterpret_cast<const uint4 *>(p);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            __half2 h2 = *reinterpret_cast<const __half2 *>(&w[i]);
-            float2 f = __half22float2(h2);
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
             o[2 * i] = f.x;
             o[2 * i + 1] = f.y;
         }
     } else if constexpr (F == kBF16) {
-        uint4 v = *reinterpret_cast<const uint4 *>(p);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -164,260 +169,140 @@ __device__ __forceinline__ void load_vec(const uint8_t *p, float *o)
             o[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
         }
     } else {
-        // 16 nibbles, element 2j in the low nibble of byte j.  n - 8 is formed
-        // exactly by placing n in the mantissa of 2^23 and subtracting 2^23 + 8.
-        uint2 v = *reinterpret_cast<const uint2 *>(p);
+        // element 2j sits in the low nibble of byte j; n - 8 is formed exactly
+        // by placing n in the mantissa of 2^23 and subtracting 2^23 + 8
         const uint32_t w[2] = {v.x, v.y};
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < 2; ++i)
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                uint32_t n = (w[i] >> (4 * j)) & 0xfu;
-                o[8 * i + j] = __uint_as_float(0x4b000000u | n) - 8388616.0f;
-            }
-        }
+            for (int j = 0; j < 8; ++j)
+                o[8 * i + j] = __uint_as_float(0x4b000000u | ((w[i] >> (4 * j)) & 0xfu)) - 8388616.0f;
     }
 }
 
-// Scale of the group holding vector v of an INT4 row record (nibbles, then
-// one fp16 scale per 32 elements).
+// Scale of the 32-element group holding INT4 vector v of a row record
+// (d/2 nibble bytes, then one fp16 scale per 32 elements).
 __device__ __forceinline__ float i4_scale(const uint8_t *row, int d, int v)
 {
-    return __half2float(*reinterpret_cast<const __half *>(row + d / 2 + (v >> 1) * 2));
-}
-
-// Partial dot product of a row (in shared memory) with this thread's cached
-// x values.  Thread t owns vectors t, t + 256, ... of the row.
-template <int F, int MAXV>
-__device__ __forceinline__ float dot_row(const uint8_t *row, const float *xc, int nvec, int d)
-{
-    constexpr int EPV = Fm<F>::EPV, VB = Fm<F>::VB;
-    float acc = 0.f;
-#pragma unroll
-    for (int k = 0; k < MAXV; ++k) {
-        const int v = threadIdx.x + kConsumers * k;
-        if (v < nvec) {
-            float w[EPV];
-            load_vec<F>(row + v * VB, w);
-            float a = 0.f;
-#pragma unroll
-            for (int i = 0; i < EPV; ++i)
-                a = fmaf(w[i], xc[k * EPV + i], a);
-            if constexpr (F == kI4)
-                acc = fmaf(i4_scale(row, d, v), a, acc);
-            else
-                acc += a;
-        }
-    }
-    return acc;
-}
-
-// acc[owned columns] += h * row[owned columns]
-template <int F, int MAXV>
-__device__ __forceinline__ void axpy_row(const uint8_t *row, float h, float *acc, int nvec, int d)
-{
-    constexpr int EPV = Fm<F>::EPV, VB = Fm<F>::VB;
-#pragma unroll
-    for (int k = 0; k < MAXV; ++k) {
-        const int v = threadIdx.x + kConsumers * k;
-        if (v < nvec) {
-            float w[EPV];
-            load_vec<F>(row + v * VB, w);
-            float hs = h;
-            if constexpr (F == kI4)
-                hs = h * i4_scale(row, d, v);
-#pragma unroll
-            for (int i = 0; i < EPV; ++i)
-                acc[k * EPV + i] = fmaf(hs, w[i], acc[k * EPV + i]);
-        }
-    }
+    const unsigned short s = __ldg(reinterpret_cast<const unsigned short *>(row + d / 2) + (v >> 1));
+    return __half2float(__ushort_as_half(s));
 }
 
 __device__ __forceinline__ float warp_sum(float v)
 {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        v += __shfl_xor_sync(0xffffffffu, v, o);
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
 }
 
 __device__ __forceinline__ float act_h(int act, float g, float u)
 {
     const float gp = g > 0.f ? g : 0.f;
-    if (act == 0) return gp;              // ReLU (non-gated)
-    if (act == 1) return gp * u;          // ReGLU
-    return gp * (u > 0.f ? u : 0.f);      // dReLU
+    if (act == 0) return gp;               // ReLU (non-gated)
+    if (act == 1) return gp * u;           // ReGLU
+    return gp * (u > 0.f ? u : 0.f);       // dReLU
 }
 
-// ---------------------------------------------------------------------------
-// Shared-memory control block
-// ---------------------------------------------------------------------------
-enum GType { kGU = 0, kDown = 2 };   // a neuron's input record, or its W_down row
-struct GDesc {
-    int type, e, k;
-    float h;
-};
-constexpr int kQueue = kMaxTopK * kMaxStrip;  // down-row request queue
+constexpr int kNB = 4;            // neurons per gather batch
+constexpr int kRA = 16;           // V rows per staging round at most
+constexpr int kMaxU = 4;          // U vectors per lane (rank <= 128 * EPV)
+constexpr int kRed = 2 * kNB > kRA ? 2 * kNB : kRA;
 
-struct Ctl {
-    uint64_t p_full[kMaxPSlots], p_empty[kMaxPSlots];
-    uint64_t g_full[kMaxGSlots], g_empty[kMaxGSlots];
-    uint64_t route_ready, list_ready;
-    GDesc gdesc[kMaxGSlots];
-    int abort_flag;
-    int bc[2];                                   // broadcast of collective decisions
-    int route_e[2][kMaxTopK];                    // [layer parity][slot] expert id
-    float route_w[2][kMaxTopK];
-    int lst_n[2][kMaxTopK];
-    int16_t lst[2][kMaxTopK][kMaxStrip];         // active strip-local indices, ascending
-    int dq[kQueue];                              // down-row requests: (slot << 16) | k
-    float dqh[kQueue];
-    int dq_tail, h_rep;                          // cumulative counters (consumer thread 0)
-    float zbuf[kMaxTopK][kMaxStrip];
+struct Smem {
+    float red[2][kConsumerWarps][kRed];
+    alignas(16) float tsm[kMaxRankTotal];
     float cbuf[kMaxTopK][kMaxStrip];
-    float tsm[kMaxRankTotal];
-    float red[2][kConsumerWarps][17];
+    float zbuf[kMaxTopK][kMaxStrip];
+    int16_t lst[kMaxTopK * kMaxStrip];     // active neurons: (slot << 12) | local
+    int lst_n[kMaxTopK];
+    int16_t nz[kMaxTopK * kMaxStrip];      // neurons with h != 0, same encoding
+    float hz[kMaxTopK * kMaxStrip];        // their h (routing weight folded in)
+    int nz_n;
+    int route_e[kMaxTopK];
+    float route_w[kMaxTopK];
+    float lg[kConsumerWarps][kMaxExperts];
     float inv_rms;
-    float logits[kMaxExperts];
+    int bc[2];
+    uint64_t stage_bar;                    // completion of a staging round
 };
-
-}  // namespace
-
-size_t decode_smem_bytes(int np_slots, int ng_slots, int sg_bytes)
-{
-    size_t ctl = (sizeof(Ctl) + 127) & ~size_t(127);
-    return ctl + size_t(np_slots) * kPSlotBytes + size_t(ng_slots) * sg_bytes + 128;
-}
-
-namespace {
-
-struct Piece {
-    int kind;   // 0: V rows, 1: U rows
-    int slot;   // expert slot (0 .. top_k-1)
-    int row0;   // first row (V: within the expert's V; U: table position)
-    int nrows;
-};
-
-__device__ __forceinline__ int make_pieces(int r, int ntop, int a0, int a1, int s0, int ns,
-                                           Piece *pc)
-{
-    int n = 0;
-    for (int e = 0; e < ntop; ++e) {
-        const int lo = max(a0, e * r), hi = min(a1, (e + 1) * r);
-        if (hi > lo) pc[n++] = Piece{0, e, lo - e * r, hi - lo};
-    }
-    for (int e = 0; e < ntop; ++e)
-        if (ns > 0) pc[n++] = Piece{1, e, s0, ns};
-    return n;
-}
-
-__device__ __forceinline__ void prof_mark(const DecodeParams &p, int li, int point)
-{
-    if (p.prof && threadIdx.x == 0)
-        p.prof[(size_t(li) * kProfPoints + point) * gridDim.x + blockIdx.x] = gtimer();
-}
-__device__ __forceinline__ void prof_put(const DecodeParams &p, int li, int point, long long v)
-{
-    if (p.prof && threadIdx.x == 0)
-        p.prof[(size_t(li) * kProfPoints + point) * gridDim.x + blockIdx.x] = v;
-}
 
 __device__ void set_error(int *err, int code)
 {
     atomicCAS(err, 0, code);
 }
 
-// Bounded wait on an mbarrier phase by a single thread.  Returns false when
-// the CTA is aborting or the wait ran out (which starts the abort).
-__device__ bool wait_phase(uint64_t *bar, uint32_t parity, Ctl *ctl, const DecodeParams &p)
+__device__ __forceinline__ void prof_put(const DecodeParams &p, int li, int point, long long v)
 {
-    if (mbar_test(bar, parity)) return true;
-    const long long t0 = gtimer();
-    for (unsigned it = 1;; ++it) {
-        if (mbar_test(bar, parity)) return true;
-        if ((it & 15) == 0) {
-            if (ld_vol(&ctl->abort_flag)) return false;
-            if (gtimer() - t0 > p.wait_ns) {
-                st_vol(&ctl->abort_flag, 1);
-                set_error(p.err, kDevTimeout);
-                return false;
-            }
-        }
-    }
+    if (p.prof && threadIdx.x == 0)
+        p.prof[(size_t(li) * kProfPoints + point) * gridDim.x + blockIdx.x] = v;
 }
 
-// Collective wait of the 256 consumer threads: thread 0 waits (bounded) and
-// broadcasts the outcome, so every consumer thread takes the same branch.
-__device__ __forceinline__ bool cwait(uint64_t *bar, uint32_t parity, Ctl *ctl,
-                                      const DecodeParams &p, int &bci, long long *wait_cyc = nullptr)
+// Grid-wide barrier of all CTAs of the cooperative launch: arrivals are
+// fire-and-forget releases on one counter (never reset within a launch);
+// thread 0 of each CTA polls it with acquire loads, bounded by wait_ns.  The
+// outcome is broadcast through shared memory so the whole CTA agrees.
+__device__ bool grid_sync(Smem *sm, const DecodeParams &p, unsigned &epoch, int &bci, long long *cyc)
 {
+    cta_sync();
     if (threadIdx.x == 0) {
         const long long c0 = clock64();
-        st_vol(&ctl->bc[bci], wait_phase(bar, parity, ctl, p) ? 1 : 0);
-        if (wait_cyc) *wait_cyc += clock64() - c0;
+        bool ok = true;
+        epoch += 1;
+        unsigned target = epoch * gridDim.x;
+        if ((p.debug_flags & 1) && epoch == 1) target += 1;   // PI_DEBUG_STALL_BARRIER
+        __threadfence();
+        red_release_gpu(p.bar, 1u);
+        const long long t0 = gtimer();
+        unsigned it = 0;
+        while (ld_acquire_gpu(p.bar) < target) {
+            if ((++it & 31) == 0 && gtimer() - t0 > p.wait_ns) {
+                set_error(p.err, kDevTimeout);
+                ok = false;
+                break;
+            }
+        }
+        __threadfence();
+        st_vol(&sm->bc[bci], ok ? 1 : 0);
+        if (cyc) *cyc += clock64() - c0;
     }
-    cons_sync();
-    const bool ok = ld_vol(&ctl->bc[bci]) != 0;
+    cta_sync();
+    const bool ok = ld_vol(&sm->bc[bci]) != 0;
     bci ^= 1;
-    if (ok) mbar_test(bar, parity);   // acquire for this thread (phase already complete)
     return ok;
 }
 
-// Grid-wide barrier of the consumer warps of all CTAs (one cooperative launch).
-// bar[0] counts arrivals (never reset within a launch); the CTA whose arrival
-// completes barrier `epoch` publishes it in bar[1]; the others wait for that
-// generation word, so the waiting CTAs poll a line that changes once.
-__device__ bool grid_sync(Ctl *ctl, const DecodeParams &p, unsigned &epoch, int &bci,
-                          long long *wait_cyc = nullptr)
+// Staging round: thread 0 has issued bulk copies of `bytes` in total onto
+// sm->stage_bar; it waits (bounded) and the whole CTA adopts its verdict.
+__device__ bool stage_wait(Smem *sm, const DecodeParams &p, uint32_t &par, int &bci)
 {
-    cons_sync();
-    const long long c0 = clock64();
     if (threadIdx.x == 0) {
-        bool ok = ld_vol(&ctl->abort_flag) == 0;
-        epoch += 1;
-        if (ok) {
-            unsigned last = epoch * gridDim.x - 1;
-            if ((p.debug_flags & 1) && epoch == 1) last += 1;   // PI_DEBUG_STALL_BARRIER
-            __threadfence();
-            const unsigned old = atom_add_acqrel_gpu(p.bar, 1u);
-            if (old == last) {
-                st_release_gpu(p.bar + 1, epoch);
-            } else {
-                const long long t0 = gtimer();
-                unsigned it = 0;
-                while (ld_acquire_gpu(p.bar + 1) < epoch) {
-                    if ((++it & 31) == 0) {
-                        if (ld_vol(&ctl->abort_flag)) { ok = false; break; }
-                        if (gtimer() - t0 > p.wait_ns) {
-                            st_vol(&ctl->abort_flag, 1);
-                            set_error(p.err, kDevTimeout);
-                            ok = false;
-                            break;
-                        }
-                    }
+        bool ok = mbar_test(&sm->stage_bar, par);
+        if (!ok) {
+            const long long t0 = gtimer();
+            for (unsigned it = 1; !ok; ++it) {
+                ok = mbar_test(&sm->stage_bar, par);
+                if (!ok && (it & 15) == 0 && gtimer() - t0 > p.wait_ns) {
+                    set_error(p.err, kDevTimeout);
+                    break;
                 }
             }
-            __threadfence();
         }
-        st_vol(&ctl->bc[bci], ok ? 1 : 0);
-        if (wait_cyc) *wait_cyc += clock64() - c0;
+        st_vol(&sm->bc[bci], ok ? 1 : 0);
     }
-    cons_sync();
-    const bool ok = ld_vol(&ctl->bc[bci]) != 0;
+    cta_sync();
+    const bool ok = ld_vol(&sm->bc[bci]) != 0;
     bci ^= 1;
+    if (ok) mbar_test(&sm->stage_bar, par);   // acquire for this thread (phase complete)
+    par ^= 1;
     return ok;
 }
 
-// Wait for every bulk copy this producer issued into a ring (used when the
-// CTA aborts, so no copy is in flight when the CTA exits).
-__device__ void drain_ring(uint64_t *full, int nslots, int issued, long long wait_ns)
+// Issue bulk copies of [src, src + bytes) into dst in pieces of <= 32 KB.
+__device__ __forceinline__ void stage_copy(uint8_t *dst, const uint8_t *src, uint32_t bytes, uint64_t *bar)
 {
-    for (int s = 0; s < nslots && s < issued; ++s) {
-        const int uses = (issued - 1 - s) / nslots + 1;
-        const uint32_t par = (uses - 1) & 1;
-        const long long t0 = gtimer();
-        while (!mbar_test(&full[s], par))
-            if (gtimer() - t0 > wait_ns) break;
+    for (uint32_t o = 0; o < bytes; o += 32768u) {
+        const uint32_t n = bytes - o < 32768u ? bytes - o : 32768u;
+        bulk_g2s(dst + o, src + o, n, bar);
     }
 }
 
@@ -427,212 +312,78 @@ __device__ void drain_ring(uint64_t *full, int nslots, int issued, long long wai
 template <int WF, int PF, int DMAX>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p)
 {
-    constexpr int EPVW = Fm<WF>::EPV, EPVP = Fm<PF>::EPV;
-    constexpr int MAXVW = (DMAX / EPVW + kConsumers - 1) / kConsumers;
-    constexpr int MAXVP = (DMAX / EPVP + kConsumers - 1) / kConsumers;
-    constexpr int MAXU = 4;                    // U vectors per lane (rank <= 128 * EPVP)
-    // V rows per P slot at most: rows are >= 512 B below d = 2048, >= 4.5 KB up
-    // to 4096 and >= 8.5 KB above
-    constexpr int MAXRV = DMAX == 2048 ? 16 : (DMAX == 4096 ? 4 : 2);
+    constexpr int EPVW = Fm<WF>::EPV, EPVP = Fm<PF>::EPV, VBW = Fm<WF>::VB, VBP = Fm<PF>::VB;
+    constexpr int MAXVW = (DMAX / EPVW + kThreads - 1) / kThreads;
+    constexpr int MAXVP = (DMAX / EPVP + kThreads - 1) / kThreads;
+    // neurons per gather batch: fewer when a row takes several vectors per thread
+    constexpr int NB = MAXVW >= 2 ? kNB / 2 : kNB;
+    // when both formats share the vector layout, x is cached once
+    constexpr bool kSameX = (WF == PF);
+    using VW = typename Fm<WF>::V;
+    using VP = typename Fm<PF>::V;
 
-    extern __shared__ __align__(128) uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
-                                                ~uintptr_t(127));
-    Ctl *ctl = reinterpret_cast<Ctl *>(smem);
-    uint8_t *pring = smem + ((sizeof(Ctl) + 127) & ~size_t(127));
-    uint8_t *gring = pring + size_t(p.np_slots) * kPSlotBytes;
-
+    __shared__ Smem sm;
+    extern __shared__ __align__(128) uint8_t stg[];   // kStageBytes staging buffer
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = blockIdx.x, S = gridDim.x;
-    const int d = p.d, r = p.r, NP = p.np_slots, NG = p.ng_slots, SG = p.sg_bytes;
+    const int d = p.d, r = p.r;
     const int s0 = p.strip_off[b], ns = p.strip_off[b + 1] - s0;
     const bool predict = p.mode == kModePredict;
     const int ntop = predict ? 1 : p.top_k;
     const int rows_total = ntop * r;
     const int a0 = int((long long)b * rows_total / S), a1 = int((long long)(b + 1) * rows_total / S);
-    const int RV = min(MAXRV, kPSlotBytes / p.vrow), RU = kPSlotBytes / p.urow;
-    const int nvecW = (WF == kI4 ? d / 2 : d * (WF == kF32 ? 4 : 2)) / Fm<WF>::VB;
-    const int nvecP = p.vrow / Fm<PF>::VB;
-    const int nvecU = p.urow / Fm<PF>::VB;
-    const int l0 = predict ? p.layer_begin : p.layer_begin;
+    const int nvecW = (WF == kI4 ? d / 2 : d * (WF == kF32 ? 4 : 2)) / VBW;
+    const int nvecP = p.vrow / VBP;
+    const int nvecU = p.urow / VBP;
+    const int l0 = p.layer_begin;
     const int l1 = predict ? p.layer_begin + 1 : p.layer_end;
+    const bool dense_ahead = !predict && p.E == 1;
+
+    // L2 prefetch of a layer's predictor slice of this CTA: V rows [a0, a1)
+    // of the concatenated experts and the U strip of each expert.
+    auto prefetch_pred = [&](int l, const int *experts, bool want_v, bool want_u) {
+        for (int e = 0; e < ntop; ++e) {
+            const ExpertDev &ex = p.ex[size_t(l) * p.E + experts[e]];
+            const int lo = max(a0, e * r), hi = min(a1, (e + 1) * r);
+            if (want_v && hi > lo)
+                prefetch_l2(ex.V + size_t(lo - e * r) * p.vrow, uint32_t(hi - lo) * p.vrow);
+            if (want_u && ns > 0)
+                prefetch_l2(ex.U + size_t(s0) * p.urow, uint32_t(ns) * p.urow);
+        }
+    };
 
     if (tid == 0) {
-        for (int i = 0; i < NP; ++i) {
-            mbar_init(&ctl->p_full[i], 1);
-            mbar_init(&ctl->p_empty[i], kConsumerWarps);
-        }
-        for (int i = 0; i < NG; ++i) {
-            mbar_init(&ctl->g_full[i], 1);
-            mbar_init(&ctl->g_empty[i], kConsumerWarps);
-        }
-        mbar_init(&ctl->route_ready, 1);
-        mbar_init(&ctl->list_ready, 1);
-        ctl->abort_flag = 0;
-        ctl->dq_tail = 0;
-        ctl->h_rep = 0;
+        mbar_init(&sm.stage_bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncthreads();
-
-    // =====================================================================
-    // Warp 8: predictor stream (V rows of the t slice, U rows of the strip)
-    // =====================================================================
-    if (warp == kPWarp) {
-        if (lane != 0) return;
-        const uint64_t pol = policy_evict_first();
-        int pi = 0;
-        bool ok = true;
-        // L2 prefetch of all predictor bytes a layer will stream into this CTA
-        auto prefetch_layer = [&](int l, const int *experts) {
-            Piece pc[2 * kMaxTopK];
-            const int npc = make_pieces(r, ntop, a0, a1, s0, ns, pc);
-            for (int q = 0; q < npc; ++q) {
-                const ExpertDev &ex = p.ex[size_t(l) * p.E + experts[pc[q].slot]];
-                const int rowb = pc[q].kind == 0 ? p.vrow : p.urow;
-                const uint8_t *base = pc[q].kind == 0 ? ex.V : ex.U;
-                prefetch_l2(base + size_t(pc[q].row0) * rowb, uint32_t(pc[q].nrows) * rowb);
-            }
-        };
-        const bool dense_ahead = !predict && p.E == 1;   // experts known ahead of time
-        if (dense_ahead) {
-            const int e0[kMaxTopK] = {0, 0};
-            prefetch_layer(l0, e0);
+        if (predict) {
+            const int ex[kMaxTopK] = {p.pred_expert, 0};
+            prefetch_pred(l0, ex, true, true);
+        } else if (dense_ahead) {
+            const int ex[kMaxTopK] = {0, 0};
+            prefetch_pred(l0, ex, true, true);
         }
-        for (int l = l0; l < l1 && ok; ++l) {
-            const int lp = (l - l0) & 1;
-            int experts[kMaxTopK] = {0, 0};
-            if (predict) {
-                experts[0] = p.pred_expert;
-                prefetch_layer(l, experts);
-            } else if (p.E > 1) {
-                if (!wait_phase(&ctl->route_ready, (l - l0) & 1, ctl, p)) { ok = false; break; }
-                experts[0] = ctl->route_e[lp][0];
-                experts[1] = ctl->route_e[lp][1];
-                prefetch_layer(l, experts);
-            }
-            Piece pc[2 * kMaxTopK];
-            const int npc = make_pieces(r, ntop, a0, a1, s0, ns, pc);
-            for (int q = 0; q < npc && ok; ++q) {
-                const ExpertDev &ex = p.ex[size_t(l) * p.E + experts[pc[q].slot]];
-                const int rowb = pc[q].kind == 0 ? p.vrow : p.urow;
-                const int per = pc[q].kind == 0 ? RV : RU;
-                const uint8_t *base = pc[q].kind == 0 ? ex.V : ex.U;
-                for (int row = 0; row < pc[q].nrows; row += per) {
-                    const int n = min(per, pc[q].nrows - row);
-                    const int s = pi % NP;
-                    if (!wait_phase(&ctl->p_empty[s], ((pi / NP) & 1) ^ 1, ctl, p)) { ok = false; break; }
-                    const uint32_t bytes = uint32_t(n) * rowb;
-                    mbar_arrive_tx(&ctl->p_full[s], bytes);
-                    bulk_g2s(pring + size_t(s) * kPSlotBytes,
-                             base + size_t(pc[q].row0 + row) * rowb, bytes, &ctl->p_full[s], pol);
-                    ++pi;
-                }
-            }
-            if (ok && dense_ahead && l + 1 < l1) {
-                const int e0[kMaxTopK] = {0, 0};
-                prefetch_layer(l + 1, e0);
-            }
-        }
-        if (!ok) drain_ring(ctl->p_full, NP, pi, p.wait_ns);
-        return;
     }
 
-    // =====================================================================
-    // Warp 9: gather stream (rows of active neurons)
-    // =====================================================================
-    if (warp == kGWarp) {
-        if (lane != 0 || predict) return;
-        const uint64_t pol = policy_evict_first();
-        int gi = 0, rep_base = 0, dq_head = 0;
-        bool ok = true;
-        auto issue = [&](int type, int e, int k, float h, const uint8_t *src, int bytes) -> bool {
-            const int s = gi % NG;
-            if (!wait_phase(&ctl->g_empty[s], ((gi / NG) & 1) ^ 1, ctl, p)) return false;
-            ctl->gdesc[s] = GDesc{type, e, k, h};
-            mbar_arrive_tx(&ctl->g_full[s], uint32_t(bytes));
-            bulk_g2s(gring + size_t(s) * SG, src, uint32_t(bytes), &ctl->g_full[s], pol);
-            ++gi;
-            return true;
-        };
-        for (int l = l0; l < l1 && ok; ++l) {
-            const int lp = (l - l0) & 1;
-            if (!wait_phase(&ctl->list_ready, (l - l0) & 1, ctl, p)) { ok = false; break; }
-            const int m0 = ctl->lst_n[lp][0];
-            const int m = m0 + (ntop > 1 ? ctl->lst_n[lp][1] : 0);
-            const int ex0 = p.E > 1 ? ctl->route_e[lp][0] : 0;
-            const int ex1 = p.E > 1 ? ctl->route_e[lp][1] : 0;
-            const ExpertDev *exs[2] = {&p.ex[size_t(l) * p.E + ex0], &p.ex[size_t(l) * p.E + ex1]};
-            // every row this CTA may need this layer starts moving towards L2 now
-            for (int j = 0; j < m; ++j) {
-                const int e = j < m0 ? 0 : 1;
-                const int k = ctl->lst[lp][e][j < m0 ? j : j - m0];
-                prefetch_l2(exs[e]->Wgu + size_t(s0 + k) * p.gu_bytes, uint32_t(p.gu_bytes));
-                if (p.spec_down)
-                    prefetch_l2(exs[e]->Wd + size_t(s0 + k) * p.wrow, uint32_t(p.wrow));
-            }
-            const int rep_target = rep_base + m;
-            int gu = 0;
-            long long idle_since = gtimer();
-            while (ok) {
-                const int tail = ld_vol(&ctl->dq_tail);
-                if (dq_head < tail) {
-                    const int q = dq_head % kQueue;
-                    const int ent = ld_vol(&ctl->dq[q]);
-                    const float h = *reinterpret_cast<volatile float *>(&ctl->dqh[q]);
-                    ++dq_head;
-                    const int e = ent >> 16, k = ent & 0xffff;
-                    ok = issue(kDown, e, k, h, exs[e]->Wd + size_t(s0 + k) * p.wrow, p.wrow);
-                    idle_since = gtimer();
-                } else if (gu < m) {
-                    const int e = gu < m0 ? 0 : 1;
-                    const int k = ctl->lst[lp][e][gu < m0 ? gu : gu - m0];
-                    ++gu;
-                    ok = issue(kGU, e, k, 0.f, exs[e]->Wgu + size_t(s0 + k) * p.gu_bytes, p.gu_bytes);
-                    idle_since = gtimer();
-                } else {
-                    if (ld_vol(&ctl->h_rep) >= rep_target) {
-                        __threadfence_block();
-                        if (dq_head >= ld_vol(&ctl->dq_tail)) break;
-                        continue;
-                    }
-                    if (ld_vol(&ctl->abort_flag)) { ok = false; break; }
-                    if (gtimer() - idle_since > p.wait_ns) {
-                        st_vol(&ctl->abort_flag, 1);
-                        set_error(p.err, kDevTimeout);
-                        ok = false;
-                        break;
-                    }
-                }
-            }
-            rep_base = rep_target;
-        }
-        if (!ok) drain_ring(ctl->g_full, NG, gi, p.wait_ns);
-        return;
-    }
-
-    // =====================================================================
-    // Warps 0-7: arithmetic
-    // =====================================================================
+    cta_sync();
     unsigned epoch = 0;
-    int bci = 0, pc_i = 0, gs = 0, rb = 0;
-    int rep_count = 0, q_tail = 0;                 // thread 0's cumulative counters
+    uint32_t spar = 0;
+    int bci = 0;
     float xw[MAXVW * EPVW];
-    float xp[MAXVP * EPVP];
+    float xp_own[kSameX ? 1 : MAXVP * EPVP];
+#define XP(i) (kSameX ? xw[(i)] : xp_own[(i)])
+    int rb = 0;
 
     for (int l = l0; l < l1; ++l) {
-        const int lp = (l - l0) & 1;
         const int li = l - l0;
+        long long cyc_a = 0, cyc_b = 0, cyc_c = 0, cyc_bar = 0;
+        prof_put(p, li, 0, gtimer());
+        const long long ca0 = clock64();
 
-        // ---------------- phase A: layer input, routing, t = V x ----------
-        prof_mark(p, li, 0);
-        long long wc_a = 0, wc_b = 0, wc_c = 0, wc_bar = 0;
-        float inv = 1.f;
+        // ---------------- phase A: layer input ------------------------------
         const float *src = predict ? p.x_in : p.resid;
-        // one round trip to L2: this thread's columns in both row formats
 #pragma unroll
         for (int k = 0; k < MAXVW; ++k) {
-            const int v = tid + kConsumers * k;
+            const int v = tid + kThreads * k;
 #pragma unroll
             for (int i = 0; i < EPVW; i += 4) {
                 float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -641,15 +392,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 xw[k * EPVW + i + 2] = q.z; xw[k * EPVW + i + 3] = q.w;
             }
         }
+        if constexpr (!kSameX) {
 #pragma unroll
-        for (int k = 0; k < MAXVP; ++k) {
-            const int v = tid + kConsumers * k;
+            for (int k = 0; k < MAXVP; ++k) {
+                const int v = tid + kThreads * k;
 #pragma unroll
-            for (int i = 0; i < EPVP; i += 4) {
-                float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (v < nvecP) q = __ldcg(reinterpret_cast<const float4 *>(src + v * EPVP + i));
-                xp[k * EPVP + i] = q.x; xp[k * EPVP + i + 1] = q.y;
-                xp[k * EPVP + i + 2] = q.z; xp[k * EPVP + i + 3] = q.w;
+                for (int i = 0; i < EPVP; i += 4) {
+                    float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (v < nvecP) q = __ldcg(reinterpret_cast<const float4 *>(src + v * EPVP + i));
+                    xp_own[k * EPVP + i] = q.x; xp_own[k * EPVP + i + 1] = q.y;
+                    xp_own[k * EPVP + i + 2] = q.z; xp_own[k * EPVP + i + 3] = q.w;
+                }
             }
         }
         if (!predict) {
@@ -657,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             float ss = 0.f;
 #pragma unroll
             for (int k = 0; k < MAXVW; ++k) {
-                const int v = tid + kConsumers * k;
+                const int v = tid + kThreads * k;
                 if (v < nvecW) {
 #pragma unroll
                     for (int i = 0; i < EPVW; ++i) ss = fmaf(xw[k * EPVW + i], xw[k * EPVW + i], ss);
@@ -671,176 +424,238 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 }
             }
             ss = warp_sum(ss);
-            if (lane == 0) ctl->red[rb][warp][16] = ss;
-            cons_sync();
+            if (lane == 0) sm.red[rb][warp][0] = ss;
+            cta_sync();
             if (tid == 0) {
                 float tot = 0.f;
-                for (int w = 0; w < kConsumerWarps; ++w) tot += ctl->red[rb][w][16];
-                ctl->inv_rms = 1.f / sqrtf(tot / float(d) + p.eps);
+                for (int w = 0; w < kConsumerWarps; ++w) tot += sm.red[rb][w][0];
+                sm.inv_rms = 1.f / sqrtf(tot / float(d) + p.eps);
             }
-            cons_sync();
-            inv = ctl->inv_rms;
+            cta_sync();
             rb ^= 1;
+            const float inv = sm.inv_rms;
 #pragma unroll
             for (int i = 0; i < MAXVW * EPVW; ++i) xw[i] *= inv;
+            if constexpr (!kSameX) {
 #pragma unroll
-            for (int i = 0; i < MAXVP * EPVP; ++i) xp[i] *= inv;
+                for (int i = 0; i < MAXVP * EPVP; ++i) xp_own[i] *= inv;
+            }
         }
+        prof_put(p, li, 1, gtimer());
 
         // MoE routing, computed identically by every CTA: logits of the E
-        // experts (fp16 router), softmax, two largest (ties: lower index),
-        // weights renormalised over the two, experts in ascending index.
+        // experts (fp16 router, 8-element vectors like the predictor format),
+        // softmax, two largest (ties: lower index), weights renormalised over
+        // the two, experts in ascending index.
         if (!predict && p.E > 1) {
-            const __half *R = reinterpret_cast<const __half *>(p.router[l]);
-            for (int e = 0; e < p.E; ++e) {
-                float a = 0.f;
-                for (int j = tid; j < d; j += kConsumers)
-                    a = fmaf(__half2float(R[size_t(e) * d + j]), __ldcg(src + j) * inv, a);
-                a = warp_sum(a);
-                if (lane == 0) ctl->red[rb][warp][e] = a;
+            const uint8_t *R = p.router[l];
+            float lg[kMaxExperts];
+#pragma unroll
+            for (int e = 0; e < kMaxExperts; ++e) {
+                lg[e] = 0.f;
+                if (e < p.E) {
+#pragma unroll
+                    for (int k = 0; k < MAXVP; ++k) {
+                        const int v = tid + kThreads * k;
+                        if (v < nvecP) {
+                            float w[8];
+                            cvt<kF16>(ldw4(R + (size_t(e) * nvecP + v) * 16), w);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) lg[e] = fmaf(w[i], XP(k * EPVP + i), lg[e]);
+                        }
+                    }
+                }
             }
-            cons_sync();
+#pragma unroll
+            for (int e = 0; e < kMaxExperts; ++e) {
+                if (e < p.E) {
+                    const float v = warp_sum(lg[e]);
+                    if (lane == 0) sm.lg[warp][e] = v;
+                }
+            }
+            cta_sync();
             if (tid == 0) {
+                float logit[kMaxExperts];
                 float mx = -INFINITY;
                 for (int e = 0; e < p.E; ++e) {
                     float s = 0.f;
-                    for (int w = 0; w < kConsumerWarps; ++w) s += ctl->red[rb][w][e];
-                    ctl->logits[e] = s;
+                    for (int w = 0; w < kConsumerWarps; ++w) s += sm.lg[w][e];
+                    logit[e] = s;
                     mx = fmaxf(mx, s);
                 }
                 float pr[kMaxExperts];
                 float den = 0.f;
-                for (int e = 0; e < p.E; ++e) { pr[e] = expf(ctl->logits[e] - mx); den += pr[e]; }
+                for (int e = 0; e < p.E; ++e) { pr[e] = expf(logit[e] - mx); den += pr[e]; }
                 for (int e = 0; e < p.E; ++e) pr[e] /= den;
                 int ea = 0;
                 for (int e = 1; e < p.E; ++e) if (pr[e] > pr[ea]) ea = e;
                 int eb = ea == 0 ? 1 : 0;
                 for (int e = 0; e < p.E; ++e) if (e != ea && pr[e] > pr[eb]) eb = e;
                 const int lo = min(ea, eb), hi = max(ea, eb);
-                ctl->route_e[lp][0] = lo;
-                ctl->route_e[lp][1] = hi;
-                ctl->route_w[lp][0] = pr[lo] / (pr[lo] + pr[hi]);
-                ctl->route_w[lp][1] = pr[hi] / (pr[lo] + pr[hi]);
+                sm.route_e[0] = lo;
+                sm.route_e[1] = hi;
+                sm.route_w[0] = pr[lo] / (pr[lo] + pr[hi]);
+                sm.route_w[1] = pr[hi] / (pr[lo] + pr[hi]);
                 if (p.stats && b == 0) {
                     p.stats[li * 4 + 2] = lo;
                     p.stats[li * 4 + 3] = hi;
                 }
-                mbar_arrive(&ctl->route_ready);
+                // the two experts' predictor slices start moving now
+                prefetch_pred(l, sm.route_e, true, true);
             }
-            cons_sync();
-            rb ^= 1;
         } else if (tid == 0) {
-            ctl->route_e[lp][0] = predict ? p.pred_expert : 0;
-            ctl->route_e[lp][1] = 0;
-            ctl->route_w[lp][0] = 1.f;
-            ctl->route_w[lp][1] = 0.f;
+            sm.route_e[0] = predict ? p.pred_expert : 0;
+            sm.route_e[1] = 0;
+            sm.route_w[0] = 1.f;
+            sm.route_w[1] = 0.f;
             if (p.stats && b == 0 && !predict) {
                 p.stats[li * 4 + 2] = -1;
                 p.stats[li * 4 + 3] = -1;
             }
         }
+        cta_sync();
 
-        // t rows [a0, a1): consume the V chunks of the P ring
-        prof_mark(p, li, 1);
-        bool alive = true;
+        // ---------------- phase A: t rows [a0, a1) ---------------------------
+        // staged through shared memory in rounds of up to kRA rows
         {
-            Piece pc[2 * kMaxTopK];
-            const int npc = make_pieces(r, ntop, a0, a1, s0, ns, pc);
-            for (int q = 0; q < npc && alive; ++q) {
-                if (pc[q].kind != 0) continue;
-                for (int row = 0; row < pc[q].nrows; row += RV) {
-                    const int n = min(RV, pc[q].nrows - row);
-                    const int s = pc_i % NP;
-                    if (!cwait(&ctl->p_full[s], (pc_i / NP) & 1, ctl, p, bci, &wc_a)) { alive = false; break; }
-                    const uint8_t *slot = pring + size_t(s) * kPSlotBytes;
-                    float part[MAXRV];
+            const int per = min(kRA, kStageBytes / p.vrow);
+            bool ok = true;
+            for (int row0 = a0; row0 < a1 && ok; row0 += per) {
+                const int n = min(per, a1 - row0);
+                if (tid == 0) {
+                    mbar_arrive_tx(&sm.stage_bar, uint32_t(n) * p.vrow);
+                    // the rows of one round lie in at most two experts' V
+                    for (int rr = 0; rr < n;) {
+                        const int row = row0 + rr, e = row / r;
+                        const int cnt = min(n - rr, (e + 1) * r - row);
+                        const uint8_t *vrow =
+                            p.ex[size_t(l) * p.E + sm.route_e[e]].V + size_t(row - e * r) * p.vrow;
+                        stage_copy(stg + size_t(rr) * p.vrow, vrow, uint32_t(cnt) * p.vrow, &sm.stage_bar);
+                        rr += cnt;
+                    }
+                }
+                if (!stage_wait(&sm, p, spar, bci)) { ok = false; break; }
+                float part[kRA];
 #pragma unroll
-                    for (int rr = 0; rr < MAXRV; ++rr)
-                        part[rr] = rr < n ? dot_row<PF, MAXVP>(slot + rr * p.vrow, xp, nvecP, d) : 0.f;
+                for (int rr = 0; rr < kRA; ++rr) {
+                    part[rr] = 0.f;
+                    if (rr < n) {
 #pragma unroll
-                    for (int rr = 0; rr < MAXRV; ++rr) {
-                        if (rr < n) {
-                            const float v = warp_sum(part[rr]);
-                            if (lane == 0) ctl->red[rb][warp][rr] = v;
+                        for (int k = 0; k < MAXVP; ++k) {
+                            const int v = tid + kThreads * k;
+                            if (v < nvecP) {
+                                float w[EPVP];
+                                cvt<PF>(*reinterpret_cast<const VP *>(stg + size_t(rr) * p.vrow + v * VBP), w);
+#pragma unroll
+                                for (int i = 0; i < EPVP; ++i) part[rr] = fmaf(w[i], XP(k * EPVP + i), part[rr]);
+                            }
                         }
                     }
-                    cons_sync();
-                    if (lane == 0) mbar_arrive(&ctl->p_empty[s]);
-                    if (tid < n) {
-                        float t = 0.f;
-                        for (int w = 0; w < kConsumerWarps; ++w) t += ctl->red[rb][w][tid];
-                        __stcg(p.t_buf + pc[q].slot * r + pc[q].row0 + row + tid, t);
-                    }
-                    rb ^= 1;
-                    ++pc_i;
                 }
+#pragma unroll
+                for (int rr = 0; rr < kRA; ++rr) {
+                    if (rr < n) {
+                        const float v = warp_sum(part[rr]);
+                        if (lane == 0) sm.red[rb][warp][rr] = v;
+                    }
+                }
+                cta_sync();
+                if (tid < n) {
+                    float t = 0.f;
+                    for (int w = 0; w < kConsumerWarps; ++w) t += sm.red[rb][w][tid];
+                    __stcg(p.t_buf + row0 + tid, t);
+                }
+                rb ^= 1;
             }
+            if (!ok) break;
         }
-        prof_mark(p, li, 2);
-        if (!alive || !grid_sync(ctl, p, epoch, bci, &wc_bar)) break;
-        prof_mark(p, li, 3);
+        cyc_a = clock64() - ca0;
+        prof_put(p, li, 2, gtimer());
+        if (!grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
+        prof_put(p, li, 3, gtimer());
 
-        // ---------------- phase B: z = U t - c, threshold, compaction -----
-        for (int i = tid; i < ntop * r; i += kConsumers) ctl->tsm[i] = __ldcg(p.t_buf + i);
-        for (int e = 0; e < ntop; ++e) {
-            const ExpertDev &ex = p.ex[size_t(l) * p.E + ctl->route_e[lp][e]];
-            for (int i = tid; i < ns; i += kConsumers) ctl->cbuf[e][i] = __ldg(ex.c + s0 + i);
-        }
-        cons_sync();
-        for (int e = 0; e < ntop && alive; ++e) {
-            float tu[MAXU * EPVP];
+        // ---------------- phase B: z = U t - c, threshold, compaction --------
+        const long long cb0 = clock64();
+        {
+            constexpr int kTV = kMaxRankTotal / kThreads;
+            float tv[kTV];
 #pragma unroll
-            for (int k = 0; k < MAXU; ++k) {
-                const int v = lane + 32 * k;
-#pragma unroll
-                for (int i = 0; i < EPVP; ++i)
-                    tu[k * EPVP + i] = v < nvecU ? ctl->tsm[e * r + v * EPVP + i] : 0.f;
+            for (int k = 0; k < kTV; ++k) {
+                const int i = tid + kThreads * k;
+                tv[k] = i < ntop * r ? __ldcg(p.t_buf + i) : 0.f;
             }
-            for (int row = 0; row < ns; row += RU) {
-                const int n = min(RU, ns - row);
-                const int s = pc_i % NP;
-                if (!cwait(&ctl->p_full[s], (pc_i / NP) & 1, ctl, p, bci, &wc_b)) { alive = false; break; }
-                const uint8_t *slot = pring + size_t(s) * kPSlotBytes;
-                for (int rr = warp; rr < n; rr += kConsumerWarps) {
-                    const uint8_t *urow = slot + size_t(rr) * p.urow;
-                    float a = 0.f;
+            float cv[kMaxTopK];
 #pragma unroll
-                    for (int k = 0; k < MAXU; ++k) {
-                        const int v = lane + 32 * k;
-                        if (v < nvecU) {
-                            float w[EPVP];
-                            load_vec<PF>(urow + v * Fm<PF>::VB, w);
+            for (int e = 0; e < kMaxTopK; ++e)
+                cv[e] = (e < ntop && tid < ns) ? __ldg(p.ex[size_t(l) * p.E + sm.route_e[e]].c + s0 + tid)
+                                               : 0.f;
 #pragma unroll
-                            for (int i = 0; i < EPVP; ++i) a = fmaf(w[i], tu[k * EPVP + i], a);
+            for (int k = 0; k < kTV; ++k) {
+                const int i = tid + kThreads * k;
+                if (i < ntop * r) sm.tsm[i] = tv[k];
+            }
+#pragma unroll
+            for (int e = 0; e < kMaxTopK; ++e)
+                if (e < ntop && tid < ns) sm.cbuf[e][tid] = cv[e];
+        }
+        cta_sync();
+        {
+            bool ok = true;
+            const int per = kStageBytes / p.urow;   // U rows per staging round
+            for (int e = 0; e < ntop && ok; ++e) {
+                const float *te = sm.tsm + e * r;
+                const uint8_t *U = p.ex[size_t(l) * p.E + sm.route_e[e]].U + size_t(s0) * p.urow;
+                for (int row0 = 0; row0 < ns && ok; row0 += per) {
+                    const int n = min(per, ns - row0);
+                    if (tid == 0) {
+                        mbar_arrive_tx(&sm.stage_bar, uint32_t(n) * p.urow);
+                        stage_copy(stg, U + size_t(row0) * p.urow, uint32_t(n) * p.urow, &sm.stage_bar);
+                    }
+                    if (!stage_wait(&sm, p, spar, bci)) { ok = false; break; }
+                    for (int rr = warp; rr < n; rr += kConsumerWarps) {
+                        const uint8_t *urow = stg + size_t(rr) * p.urow;
+                        float a = 0.f;
+#pragma unroll
+                        for (int k = 0; k < kMaxU; ++k) {
+                            const int v = lane + 32 * k;
+                            if (v < nvecU) {
+                                float w[EPVP];
+                                cvt<PF>(*reinterpret_cast<const VP *>(urow + v * VBP), w);
+#pragma unroll
+                                for (int i = 0; i < EPVP; i += 4) {
+                                    const float4 tq = *reinterpret_cast<const float4 *>(te + v * EPVP + i);
+                                    a = fmaf(w[i], tq.x, a);
+                                    a = fmaf(w[i + 1], tq.y, a);
+                                    a = fmaf(w[i + 2], tq.z, a);
+                                    a = fmaf(w[i + 3], tq.w, a);
+                                }
+                            }
+                        }
+                        a = warp_sum(a);
+                        if (lane == 0) {
+                            const int loc = row0 + rr;
+                            const float z = a - sm.cbuf[e][loc];
+                            sm.zbuf[e][loc] = z;
+                            if (predict && p.z_out) p.z_out[s0 + loc] = z;
                         }
                     }
-                    a = warp_sum(a);
-                    if (lane == 0) {
-                        const int loc = row + rr;
-                        const float z = a - ctl->cbuf[e][loc];
-                        ctl->zbuf[e][loc] = z;
-                        if (predict && p.z_out) p.z_out[s0 + loc] = z;
-                    }
+                    cta_sync();   // the staging buffer is reused by the next round
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&ctl->p_empty[s]);
-                ++pc_i;
             }
+            if (!ok) break;
         }
-        if (!alive) break;
-        cons_sync();
-        prof_mark(p, li, 4);
         // compaction in ascending strip order: warp e builds expert slot e's list
         if (warp < ntop) {
             const int e = warp;
             int cnt = 0;
+            const int off = e == 0 ? 0 : kMaxStrip;
             for (int base = 0; base < ns; base += 32) {
                 const int loc = base + lane;
-                const bool act = loc < ns && ctl->zbuf[e][loc] > p.threshold;
-                const unsigned m = __ballot_sync(0xffffffffu, act);
+                const bool act = loc < ns && sm.zbuf[e][loc] > p.threshold;
+                const unsigned msk = __ballot_sync(0xffffffffu, act);
                 if (act) {
-                    const int pos = cnt + __popc(m & ((1u << lane) - 1u));
-                    ctl->lst[lp][e][pos] = int16_t(loc);
+                    const int pos = cnt + __popc(msk & ((1u << lane) - 1u));
+                    sm.lst[off + pos] = int16_t((e << 12) | loc);
                     if (predict) p.lists[size_t(b) * kMaxStrip + pos] = s0 + loc;
                     if (p.masks) {
                         const int gp = s0 + loc;
@@ -848,104 +663,213 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                         atomicOr(p.masks + (size_t(li) * ntop + e) * words + (gp >> 5), 1u << (gp & 31));
                     }
                 }
-                cnt += __popc(m);
+                cnt += __popc(msk);
             }
             if (lane == 0) {
-                ctl->lst_n[lp][e] = cnt;
+                sm.lst_n[e] = cnt;
                 if (predict) p.counts[b] = cnt;
                 if (p.stats && !predict) atomicAdd(p.stats + li * 4 + 0, cnt);
             }
         }
-        cons_sync();
+        if (tid == 0) sm.nz_n = 0;
+        cta_sync();
+        cyc_b = clock64() - cb0;
+        prof_put(p, li, 4, gtimer());
 
         if (predict) {
             // global ascending list: prefix of the strip counts, then copy
-            if (!grid_sync(ctl, p, epoch, bci)) break;
+            if (!grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
             int pre = 0;
-            for (int i = tid; i < b; i += kConsumers) pre += __ldcg(p.counts + i);
+            for (int i = tid; i < b; i += kThreads) pre += __ldcg(p.counts + i);
             pre = __reduce_add_sync(0xffffffffu, pre);
-            if (lane == 0) ctl->red[rb][warp][0] = __int_as_float(pre);
-            cons_sync();
+            if (lane == 0) sm.red[rb][warp][0] = __int_as_float(pre);
+            cta_sync();
             int base = 0;
-            for (int w = 0; w < kConsumerWarps; ++w) base += __float_as_int(ctl->red[rb][w][0]);
-            const int cnt = ctl->lst_n[lp][0];
-            for (int i = tid; i < cnt; i += kConsumers)
-                p.idx_out[base + i] = s0 + ctl->lst[lp][0][i];
+            for (int w = 0; w < kConsumerWarps; ++w) base += __float_as_int(sm.red[rb][w][0]);
+            const int cnt = sm.lst_n[0];
+            for (int i = tid; i < cnt; i += kThreads) p.idx_out[base + i] = s0 + (sm.lst[i] & 0xfff);
             if (b == S - 1 && tid == 0) p.count_out[0] = base + cnt;
             break;
         }
 
-        if (tid == 0) mbar_arrive(&ctl->list_ready);
-        prof_mark(p, li, 5);
+        // ---------------- phase C: gather rows of active neurons -------------
+        const long long cc0 = clock64();
+        const int m0 = sm.lst_n[0];
+        const int m = m0 + (ntop > 1 ? sm.lst_n[1] : 0);
+        // list index j -> (slot << 12 | local): slot 0 entries, then slot 1
+        auto entry = [&](int j) -> int { return j < m0 ? sm.lst[j] : sm.lst[kMaxStrip + (j - m0)]; };
+        const ExpertDev *exs[kMaxTopK] = {&p.ex[size_t(l) * p.E + sm.route_e[0]],
+                                          &p.ex[size_t(l) * p.E + sm.route_e[ntop > 1 ? 1 : 0]]};
+        for (int j = tid; j < m; j += kThreads) {
+            const int en = entry(j), e = en >> 12, loc = en & 0xfff;
+            prefetch_l2(exs[e]->Wgu + size_t(s0 + loc) * p.gu_bytes, uint32_t(p.gu_bytes));
+            if (p.spec_down) prefetch_l2(exs[e]->Wd + size_t(s0 + loc) * p.wrow, uint32_t(p.wrow));
+        }
+        if (tid == kThreads - 1 && dense_ahead && l + 1 < l1) {
+            const int ex[kMaxTopK] = {0, 0};
+            prefetch_pred(l + 1, ex, true, true);
+        }
 
-        // ---------------- phase C: gather rows of active neurons ----------
         float acc[MAXVW * EPVW];
 #pragma unroll
         for (int i = 0; i < MAXVW * EPVW; ++i) acc[i] = 0.f;
-        {
-            const int m = ctl->lst_n[lp][0] + (ntop > 1 ? ctl->lst_n[lp][1] : 0);
-            const int cap = (p.gated ? 3 : 2) * m + 1;   // slots this layer can hold at most
-            int gu_done = 0, dn_done = 0, nnz = 0;
-            for (int iter = 0; (gu_done < m || dn_done < nnz) && iter < cap; ++iter) {
-                const int s = gs % NG;
-                if (!cwait(&ctl->g_full[s], (gs / NG) & 1, ctl, p, bci, &wc_c)) { alive = false; break; }
-                const GDesc dsc = ctl->gdesc[s];
-                const uint8_t *row = gring + size_t(s) * SG;
-                if (dsc.type == kDown) {
-                    axpy_row<WF, MAXVW>(row, dsc.h, acc, nvecW, d);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&ctl->g_empty[s]);
-                    ++gs;
-                    ++dn_done;
-                    continue;
-                }
-                // the neuron's input record: gate (or W_1) row, then its up row
-                float pg = dot_row<WF, MAXVW>(row, xw, nvecW, d);
-                float pu = 0.f;
-                if (p.gated) pu = dot_row<WF, MAXVW>(row + p.wrow, xw, nvecW, d);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&ctl->g_empty[s]);
-                ++gs;
-                pg = warp_sum(pg);
-                pu = warp_sum(pu);
-                if (lane == 0) {
-                    ctl->red[rb][warp][0] = pg;
-                    ctl->red[rb][warp][1] = pu;
-                }
-                cons_sync();
-                float G = 0.f, Uv = 0.f;
-                for (int w = 0; w < kConsumerWarps; ++w) {
-                    G += ctl->red[rb][w][0];
-                    Uv += ctl->red[rb][w][1];
-                }
-                rb ^= 1;
-                const int e = dsc.e & 1, k = dsc.k;
-                const float g = G - ctl->cbuf[e][k];
-                const float h = act_h(p.act, g, Uv) * ctl->route_w[lp][e];
-                if (h != 0.f) ++nnz;
-                if (tid == 0) {
-                    if (h != 0.f) {
-                        const int q = q_tail % kQueue;
-                        ctl->dq[q] = (e << 16) | k;
-                        ctl->dqh[q] = h;
-                        __threadfence_block();
-                        ++q_tail;
-                        st_vol(&ctl->dq_tail, q_tail);
+
+        const int nbat = (m + NB - 1) / NB;
+        VW gv[NB][2][MAXVW];      // input records of the batch being loaded
+        VW dv[NB][MAXVW];         // W_down rows being accumulated
+
+        auto load_gu = [&](int bt) {
+#pragma unroll
+            for (int n = 0; n < NB; ++n) {
+                const int j = bt * NB + n;
+                if (j < m) {
+                    const int en = entry(j), e = en >> 12, loc = en & 0xfff;
+                    const uint8_t *rec = exs[e]->Wgu + size_t(s0 + loc) * p.gu_bytes;
+#pragma unroll
+                    for (int k = 0; k < MAXVW; ++k) {
+                        const int v = tid + kThreads * k;
+                        if (v < nvecW) {
+                            gv[n][0][k] = ldvec<WF>(rec + v * VBW);
+                            if (p.gated) gv[n][1][k] = ldvec<WF>(rec + p.wrow + v * VBW);
+                        }
                     }
-                    __threadfence_block();
-                    ++rep_count;
-                    st_vol(&ctl->h_rep, rep_count);
                 }
-                ++gu_done;
             }
-            if (tid == 0 && p.stats) atomicAdd(p.stats + li * 4 + 1, nnz);
+        };
+        // dots of batch bt's records (in registers), reduced across the CTA;
+        // neurons with h != 0 are appended to sm.nz in list order
+        auto finish_gu = [&](int bt) {
+            float pg[NB], pu[NB];
+#pragma unroll
+            for (int n = 0; n < NB; ++n) {
+                pg[n] = 0.f;
+                pu[n] = 0.f;
+                const int j = bt * NB + n;
+                if (j < m) {
+                    const int en = entry(j), e = en >> 12, loc = en & 0xfff;
+                    const uint8_t *rec = exs[e]->Wgu + size_t(s0 + loc) * p.gu_bytes;
+#pragma unroll
+                    for (int k = 0; k < MAXVW; ++k) {
+                        const int v = tid + kThreads * k;
+                        if (v < nvecW) {
+                            float w[EPVW];
+                            float a = 0.f;
+                            cvt<WF>(gv[n][0][k], w);
+#pragma unroll
+                            for (int i = 0; i < EPVW; ++i) a = fmaf(w[i], xw[k * EPVW + i], a);
+                            if constexpr (WF == kI4) a *= i4_scale(rec, d, v);
+                            pg[n] += a;
+                            if (p.gated) {
+                                float c = 0.f;
+                                cvt<WF>(gv[n][1][k], w);
+#pragma unroll
+                                for (int i = 0; i < EPVW; ++i) c = fmaf(w[i], xw[k * EPVW + i], c);
+                                if constexpr (WF == kI4) c *= i4_scale(rec + p.wrow, d, v);
+                                pu[n] += c;
+                            }
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int n = 0; n < NB; ++n) {
+                const float a = warp_sum(pg[n]);
+                const float c = warp_sum(pu[n]);
+                if (lane == 0) {
+                    sm.red[rb][warp][2 * n] = a;
+                    sm.red[rb][warp][2 * n + 1] = c;
+                }
+            }
+            cta_sync();
+            if (tid == 0) {
+                int nzn = sm.nz_n;
+                for (int n = 0; n < NB; ++n) {
+                    const int j = bt * NB + n;
+                    if (j >= m) break;
+                    float G = 0.f, Uv = 0.f;
+                    for (int w = 0; w < kConsumerWarps; ++w) {
+                        G += sm.red[rb][w][2 * n];
+                        Uv += sm.red[rb][w][2 * n + 1];
+                    }
+                    const int en = entry(j), e = en >> 12, loc = en & 0xfff;
+                    const float h = act_h(p.act, G - sm.cbuf[e][loc], Uv) * sm.route_w[e];
+                    if (h != 0.f) {
+                        sm.nz[nzn] = int16_t(en);
+                        sm.hz[nzn] = h;
+                        ++nzn;
+                    }
+                }
+                sm.nz_n = nzn;
+            }
+            cta_sync();
+            rb ^= 1;
+        };
+        // W_down rows of sm.nz[q0, q1) into registers / into acc
+        auto load_dn = [&](int q0, int q1) {
+#pragma unroll
+            for (int n = 0; n < NB; ++n) {
+                const int q = q0 + n;
+                if (q < q1) {
+                    const int en = sm.nz[q], e = en >> 12, loc = en & 0xfff;
+                    const uint8_t *row = exs[e]->Wd + size_t(s0 + loc) * p.wrow;
+#pragma unroll
+                    for (int k = 0; k < MAXVW; ++k) {
+                        const int v = tid + kThreads * k;
+                        if (v < nvecW) dv[n][k] = ldvec<WF>(row + v * VBW);
+                    }
+                }
+            }
+        };
+        auto axpy_dn = [&](int q0, int q1) {
+#pragma unroll
+            for (int n = 0; n < NB; ++n) {
+                const int q = q0 + n;
+                if (q < q1) {
+                    const int en = sm.nz[q], e = en >> 12, loc = en & 0xfff;
+                    const uint8_t *row = exs[e]->Wd + size_t(s0 + loc) * p.wrow;
+                    const float h = sm.hz[q];
+#pragma unroll
+                    for (int k = 0; k < MAXVW; ++k) {
+                        const int v = tid + kThreads * k;
+                        if (v < nvecW) {
+                            float w[EPVW];
+                            cvt<WF>(dv[n][k], w);
+                            float hs = h;
+                            if constexpr (WF == kI4) hs = h * i4_scale(row, d, v);
+#pragma unroll
+                            for (int i = 0; i < EPVW; ++i) acc[k * EPVW + i] = fmaf(hs, w[i], acc[k * EPVW + i]);
+                        }
+                    }
+                }
+            }
+        };
+
+        int dn_done = 0;   // entries of sm.nz already accumulated
+        if (nbat > 0) {
+            load_gu(0);
+            finish_gu(0);
         }
-        if (!alive) break;
-        prof_mark(p, li, 6);
+        for (int bt = 0; bt < nbat; ++bt) {
+            // W_down rows found so far + the records of batch bt + 1, together
+            const int dn_hi = min(sm.nz_n, dn_done + NB);
+            load_dn(dn_done, dn_hi);
+            if (bt + 1 < nbat) load_gu(bt + 1);
+            axpy_dn(dn_done, dn_hi);
+            dn_done = dn_hi;
+            if (bt + 1 < nbat) finish_gu(bt + 1);
+        }
+        const int nz_total = sm.nz_n;
+        while (dn_done < nz_total) {
+            const int dn_hi = min(nz_total, dn_done + NB);
+            load_dn(dn_done, dn_hi);
+            axpy_dn(dn_done, dn_hi);
+            dn_done = dn_hi;
+        }
+        if (tid == 0 && p.stats) atomicAdd(p.stats + li * 4 + 1, nz_total);
         // per-CTA partial of y
 #pragma unroll
         for (int k = 0; k < MAXVW; ++k) {
-            const int v = tid + kConsumers * k;
+            const int v = tid + kThreads * k;
             if (v < nvecW) {
 #pragma unroll
                 for (int i = 0; i < EPVW; i += 4)
@@ -954,18 +878,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                                        acc[k * EPVW + i + 2], acc[k * EPVW + i + 3]));
             }
         }
-        if (!grid_sync(ctl, p, epoch, bci, &wc_bar)) break;
-        prof_mark(p, li, 7);
+        cyc_c = clock64() - cc0;
+        prof_put(p, li, 5, gtimer());
+        prof_put(p, li, 6, gtimer());
+        if (!grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
+        prof_put(p, li, 7, gtimer());
 
-        // ---------------- phase D: r += sum of partials (fixed order) -----
+        // ---------------- phase D: r += sum of partials (fixed order) --------
         {
+            constexpr int kParts = kMaxStrips / 32;   // partial rows per lane
             const int nq = d / 4;
             const int q0 = int((long long)b * nq / S), q1 = int((long long)(b + 1) * nq / S);
             for (int q = q0 + warp; q < q1; q += kConsumerWarps) {
+                float4 pv[kParts];
+#pragma unroll
+                for (int j = 0; j < kParts; ++j) {
+                    const int c = lane + 32 * j;
+                    pv[j] = c < S ? __ldcg(reinterpret_cast<const float4 *>(p.partials + size_t(c) * d) + q)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
                 float4 sacc = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int c = lane; c < S; c += 32) {
-                    const float4 v = __ldcg(reinterpret_cast<const float4 *>(p.partials + size_t(c) * d) + q);
-                    sacc.x += v.x; sacc.y += v.y; sacc.z += v.z; sacc.w += v.w;
+#pragma unroll
+                for (int j = 0; j < kParts; ++j) {
+                    sacc.x += pv[j].x; sacc.y += pv[j].y; sacc.z += pv[j].z; sacc.w += pv[j].w;
                 }
                 sacc.x = warp_sum(sacc.x); sacc.y = warp_sum(sacc.y);
                 sacc.z = warp_sum(sacc.z); sacc.w = warp_sum(sacc.w);
@@ -976,19 +911,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 }
             }
         }
-        prof_mark(p, li, 8);
-        if (!grid_sync(ctl, p, epoch, bci, &wc_bar)) break;
-        prof_mark(p, li, 9);
-        prof_put(p, li, 10, wc_a);
-        prof_put(p, li, 11, wc_b);
-        prof_put(p, li, 12, wc_c);
-        prof_put(p, li, 13, wc_bar);
+        prof_put(p, li, 8, gtimer());
+        if (!grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
+        prof_put(p, li, 9, gtimer());
+        prof_put(p, li, 10, cyc_a);
+        prof_put(p, li, 11, cyc_b);
+        prof_put(p, li, 12, cyc_c);
+        prof_put(p, li, 13, cyc_bar);
     }
 }
 
 template <int WF, int PF>
-cudaError_t launch_t(int dmax_cls, const DecodeParams &p, size_t smem, cudaStream_t st,
-                     bool query, int *blocks)
+cudaError_t launch_t(int dmax_cls, const DecodeParams &p, cudaStream_t st, bool query, int *blocks)
 {
     void *fn = nullptr;
     switch (dmax_cls) {
@@ -999,38 +933,38 @@ cudaError_t launch_t(int dmax_cls, const DecodeParams &p, size_t smem, cudaStrea
         else fn = (void *)decode_kernel<WF, PF, 8192>;
         break;
     }
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kStageBytes);
     if (e != cudaSuccess) return e;
-    if (query) return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, fn, kThreads, smem);
+    if (query) return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, fn, kThreads, kStageBytes);
     void *args[] = {const_cast<DecodeParams *>(&p)};
-    return cudaLaunchCooperativeKernel(fn, dim3(p.S), dim3(kThreads), args, smem, st);
+    return cudaLaunchCooperativeKernel(fn, dim3(p.S), dim3(kThreads), args, kStageBytes, st);
 }
 
-cudaError_t dispatch(int wfmt, int pfmt, int d, const DecodeParams *p, size_t smem,
-                     cudaStream_t st, bool query, int *blocks)
+cudaError_t dispatch(int wfmt, int pfmt, int d, const DecodeParams *p, cudaStream_t st, bool query,
+                     int *blocks)
 {
     const int cls = d <= 2048 ? 0 : (d <= 4096 ? 1 : 2);
     static const DecodeParams dummy{};
     const DecodeParams &pp = p ? *p : dummy;
-    if (wfmt == kF32 && pfmt == kF32) return launch_t<kF32, kF32>(cls, pp, smem, st, query, blocks);
-    if (wfmt == kF16 && pfmt == kF16) return launch_t<kF16, kF16>(cls, pp, smem, st, query, blocks);
-    if (wfmt == kBF16 && pfmt == kBF16) return launch_t<kBF16, kBF16>(cls, pp, smem, st, query, blocks);
-    if (wfmt == kI4 && pfmt == kF16) return launch_t<kI4, kF16>(cls, pp, smem, st, query, blocks);
-    if (wfmt == kI4 && pfmt == kBF16) return launch_t<kI4, kBF16>(cls, pp, smem, st, query, blocks);
+    if (wfmt == kF32 && pfmt == kF32) return launch_t<kF32, kF32>(cls, pp, st, query, blocks);
+    if (wfmt == kF16 && pfmt == kF16) return launch_t<kF16, kF16>(cls, pp, st, query, blocks);
+    if (wfmt == kBF16 && pfmt == kBF16) return launch_t<kBF16, kBF16>(cls, pp, st, query, blocks);
+    if (wfmt == kI4 && pfmt == kF16) return launch_t<kI4, kF16>(cls, pp, st, query, blocks);
+    if (wfmt == kI4 && pfmt == kBF16) return launch_t<kI4, kBF16>(cls, pp, st, query, blocks);
     return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-cudaError_t launch_decode(int wfmt, int pfmt, const DecodeParams &p, size_t smem, cudaStream_t stream)
+cudaError_t launch_decode(int wfmt, int pfmt, const DecodeParams &p, cudaStream_t stream)
 {
-    return dispatch(wfmt, pfmt, p.d, &p, smem, stream, false, nullptr);
+    return dispatch(wfmt, pfmt, p.d, &p, stream, false, nullptr);
 }
 
-int decode_max_blocks_per_sm(int wfmt, int pfmt, int d, size_t smem)
+int decode_max_blocks_per_sm(int wfmt, int pfmt, int d)
 {
     int blocks = 0;
-    if (dispatch(wfmt, pfmt, d, nullptr, smem, nullptr, true, &blocks) != cudaSuccess) return 0;
+    if (dispatch(wfmt, pfmt, d, nullptr, nullptr, true, &blocks) != cudaSuccess) return 0;
     return blocks;
 }
 

@@ -66,8 +66,6 @@ struct pi_ffn {
     int S = 0;                       // strips = CTAs of the decode kernel
     int wfmt = 0, pfmt = 0, gated = 0;
     int vrow = 0, urow = 0, wrow = 0;
-    int np = 0, ng = 0;
-    size_t smem = 0;
     std::vector<int32_t> strip_off;
     std::vector<std::vector<int32_t>> perm;   // [layer * E + e]
     std::vector<uint8_t *> mem;               // [layer * E + e]
@@ -127,6 +125,8 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
     } else {
         return fail(PI_ERR_INVALID_ARG, "n_experts must be in [1, %d]", pi::kMaxExperts);
     }
+    if (D.n_experts > 1 && D.pred_dtype == PI_F32)
+        return fail(PI_ERR_UNSUPPORTED, "MoE needs an F16 or BF16 predictor");
     if (D.top_k * D.rank > pi::kMaxRankTotal)
         return fail(PI_ERR_INVALID_ARG, "top_k * rank must be <= %d", pi::kMaxRankTotal);
     if (!(D.eps > 0.f) || !std::isfinite(D.threshold))
@@ -154,24 +154,15 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
                                       : D.d_model * elem_bytes(D.w_dtype);
     h->S = D.n_strips > 0 ? D.n_strips : prop.multiProcessorCount;
 
-    // shared-memory rings: 6 predictor slots of 16 KB, gather slots fill the rest
-    const size_t budget = size_t(prop.sharedMemPerBlockOptin);
-    h->np = 6;
-    const int sg = (h->gated ? 2 : 1) * h->wrow;   // a gather slot holds one input record
-    const size_t base = pi::decode_smem_bytes(h->np, 0, sg);
-    int ng = base < budget ? int((budget - base) / size_t(sg)) : 0;
-    ng = std::min(ng, pi::kMaxGSlots);
-    if (ng < 2) {
+    if (h->S > pi::kMaxStrips) {
         delete h;
-        return fail(PI_ERR_UNSUPPORTED, "shared memory too small for the gather ring");
+        return fail(PI_ERR_UNSUPPORTED, "n_strips %d exceeds %d", h->S, pi::kMaxStrips);
     }
-    h->ng = ng;
-    h->smem = pi::decode_smem_bytes(h->np, h->ng, sg);
-    const int per_sm = pi::decode_max_blocks_per_sm(h->wfmt, h->pfmt, D.d_model, h->smem);
+    const int per_sm = pi::decode_max_blocks_per_sm(h->wfmt, h->pfmt, D.d_model);
     if (per_sm < 1 || h->S > per_sm * prop.multiProcessorCount) {
         delete h;
         return fail(PI_ERR_UNSUPPORTED, "n_strips %d exceeds co-resident CTAs (%d per SM x %d SMs)",
-                    D.n_strips, per_sm, prop.multiProcessorCount);
+                    h->S, per_sm, prop.multiProcessorCount);
     }
     if (D.d_ff > pi::kMaxStrip * h->S) {
         delete h;
@@ -410,9 +401,6 @@ static pi::DecodeParams base_params(pi_ffn_t h)
     p.wrow = h->wrow;
     p.gu_bytes = (h->gated ? 2 : 1) * h->wrow;
     p.spec_down = D.act != PI_ACT_DRELU;
-    p.np_slots = h->np;
-    p.ng_slots = h->ng;
-    p.sg_bytes = p.gu_bytes;
     p.t_buf = h->t_buf;
     p.partials = h->partials;
     p.lists = h->lists;
@@ -446,7 +434,7 @@ pi_status pi_predict(pi_ffn_t h, int layer, int expert, const float *x_dev, int3
     p.idx_out = idx_dev;
     p.count_out = count_dev;
     PI_CUDA(cudaMemsetAsync(h->bar, 0, 2 * sizeof(unsigned), st), "memset barrier");
-    PI_CUDA(pi::launch_decode(h->wfmt, h->pfmt, p, h->smem, st), "launch predict");
+    PI_CUDA(pi::launch_decode(h->wfmt, h->pfmt, p, st), "launch predict");
     return PI_OK;
 }
 
@@ -478,7 +466,7 @@ pi_status pi_sparse_ffn_decode(pi_ffn_t h, int layer_begin, int layer_end, float
     if (mask_dev)
         PI_CUDA(cudaMemsetAsync(mask_dev, 0, sizeof(uint32_t) * size_t(nl) * D.top_k * ((D.d_ff + 31) / 32), st),
                 "memset masks");
-    PI_CUDA(pi::launch_decode(h->wfmt, h->pfmt, p, h->smem, st), "launch decode");
+    PI_CUDA(pi::launch_decode(h->wfmt, h->pfmt, p, st), "launch decode");
     return PI_OK;
 }
 

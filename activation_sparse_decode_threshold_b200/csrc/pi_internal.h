@@ -6,22 +6,17 @@
 
 namespace pi {
 
-// Decode kernel geometry: 8 consumer warps (256 threads) do the arithmetic,
-// warp 8 streams the input-independent predictor weights (V, U) into a
-// shared-memory ring, warp 9 streams the gathered neuron rows (W_gate / W_up /
-// W_down of active neurons) into a second ring.
-constexpr int kConsumerWarps = 8;
-constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kPWarp = 8;
-constexpr int kGWarp = 9;
-constexpr int kThreads = 320;
+// Decode kernel geometry: one CTA of 16 warps per neuron strip, one strip per
+// SM; every warp computes (weights reach the SM through L2 prefetches and
+// batched 128-bit loads).
+constexpr int kConsumerWarps = 16;
+constexpr int kThreads = kConsumerWarps * 32;
 constexpr int kMaxStrip = 256;        // neurons per strip (per CTA) at most
+constexpr int kMaxStrips = 256;       // strips (CTAs) at most
 constexpr int kMaxTopK = 2;
 constexpr int kMaxExperts = 16;
-constexpr int kMaxPSlots = 16;
-constexpr int kMaxGSlots = 128;
 constexpr int kMaxRankTotal = 2048;   // top_k * rank
-constexpr int kPSlotBytes = 16384;
+constexpr int kStageBytes = 192 * 1024;   // shared-memory staging of V rows / U strips
 
 enum Fmt { kF32 = 0, kF16 = 1, kBF16 = 2, kI4 = 3 };
 
@@ -50,7 +45,6 @@ struct DecodeParams {
     int vrow, urow, wrow;           // row bytes: V (pred fmt), U (pred fmt), W (weight fmt)
     int gu_bytes;                   // bytes of a neuron's input record (2 * wrow gated)
     int spec_down;                  // prefetch down rows of all predicted-active neurons
-    int np_slots, ng_slots, sg_bytes;
     int mode, pred_expert;
     // inputs / outputs
     float *resid;                   // [d] decode: in/out residual
@@ -75,10 +69,8 @@ struct DecodeParams {
 // Phase timestamps recorded per layer and CTA when DecodeParams::prof is set.
 constexpr int kProfPoints = 14;   // 10 timestamps + 4 cycle counters
 
-size_t decode_smem_bytes(int np_slots, int ng_slots, int sg_bytes);
-cudaError_t launch_decode(int wfmt, int pfmt, const DecodeParams &p, size_t smem,
-                          cudaStream_t stream);
-int decode_max_blocks_per_sm(int wfmt, int pfmt, int d, size_t smem);
+cudaError_t launch_decode(int wfmt, int pfmt, const DecodeParams &p, cudaStream_t stream);
+int decode_max_blocks_per_sm(int wfmt, int pfmt, int d);
 
 // Load-time repack kernels (pi_repack.cu).  repack_rows: dst record p is the
 // concatenation of row perm[p] of each of the n_src sources (row bytes each a
