@@ -2,37 +2,38 @@
 //
 // One cooperative launch runs a range of layers for one token.  Each CTA owns
 // one strip of the neuron table (a contiguous run of table positions holding
-// a balanced share of hot neurons, hottest first) and a slice of the rows of
-// t = V x.  Per layer:
+// a balanced share of hot neurons, hottest first) and one slice of the d_model
+// columns.  Per layer l (dense FFN):
 //
-//   phase A  x = RMSNorm(r) (every CTA, identical arithmetic); [MoE] router +
-//            top-2 (every CTA, identical); the CTA's rows of t = V x.
+//   [B] t = V x (from the column phase below), x = RMSNorm(r);
+//       z = U t - c over the strip, active iff z > threshold, the active list
+//       compacted in ascending table order with warp ballots (PowerInfer
+//       (unite.ai), "Adaptive sparse predictor").
+//   [C] for active neurons only: the neuron's W_gate / W_up rows -> h =
+//       act(g, u); for h != 0 its W_down column (stored as a row) accumulates
+//       into a per-CTA fp32 partial of y ("Neuron-aware operators": rows of
+//       the input matrices, columns of the output matrix).
 //   --- grid barrier ---
-//   phase B  z = U t - c over the strip; active iff z > threshold; the active
-//            list is compacted in ascending table order with warp ballots
-//            (PowerInfer (unite.ai), "Adaptive sparse predictor").
-//   phase C  for active neurons only: the neuron's W_gate / W_up rows ->
-//            h = act(g, u); for h != 0 its W_down column (stored as a row) is
-//            accumulated into a per-CTA fp32 partial of y ("Neuron-aware
-//            operators": rows of the input matrices, columns of the output).
-//   --- grid barrier ---
-//   phase D  r <- r + sum of the per-CTA partials in fixed CTA order, by
-//            column slices (deterministic, no atomics): the merge of partial
-//            results (nearauto.com PowerInfer article, Fig. 8).
+//   [column phase] r <- r + sum of the per-CTA partials, for this CTA's
+//       columns, in fixed CTA order (the merge of partial results, nearauto.com
+//       PowerInfer article, Fig. 8); then, for layer l + 1, this CTA's share of
+//       sum(r^2) and of t = V r (V stored column-blocked per CTA), added in
+//       64-bit fixed point so the totals do not depend on arrival order.
 //   --- grid barrier ---
 //
-// Memory strategy: every weight byte is first pulled into L2 with
-// cp.async.bulk.prefetch.L2 as early as its address is known -- the next
-// layer's predictor slice (V rows, U strip) while the current layer gathers,
-// a strip's active neuron records the moment its active list exists (and,
-// for ReLU / ReGLU, where h != 0 almost always follows z > 0, their W_down
-// rows too) -- and the 16 warps then read it with batched 128-bit loads:
-// many rows in flight per thread and one cross-warp reduction per batch.
-// The gather is software-pipelined: the W_down rows of batch i and the
-// W_gate/W_up records of batch i+1 are loaded together.  HBM traffic is the
-// algorithmic bytes (plus the speculative W_down rows whose h turns out 0).
-// All waits are bounded (%globaltimer); a wait that runs out records an
-// error word and every thread of the grid returns.
+// Two grid barriers per layer.  The MoE layer adds routing (from fixed-point
+// router logits, identical in every CTA), t computed by rows of the two
+// chosen experts, and a third barrier.
+//
+// Memory: weight bytes are pulled towards the SM as soon as their addresses
+// are known -- the next layer's U strip is bulk-copied straight into shared
+// memory when the gather ends (it lands during the barriers), its V block is
+// prefetched into L2, and a strip's active neuron records (plus, for ReLU /
+// ReGLU, where h != 0 almost always follows z > 0, their W_down rows) are
+// prefetched into L2 the moment the active list exists; the 16 warps read
+// them with batched 128-bit loads, the W_down rows of one batch together with
+// the W_gate/W_up records of the next.  All waits are bounded (%globaltimer);
+// a wait that runs out records an error word and every CTA returns.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -211,6 +212,7 @@ constexpr int kRed = 2 * kNB > kRA ? 2 * kNB : kRA;
 struct Smem {
     float red[2][kConsumerWarps][kRed];
     alignas(16) float tsm[kMaxRankTotal];
+    alignas(16) float rsl[kMaxSliceCols];  // this CTA's columns of the new residual
     float cbuf[kMaxTopK][kMaxStrip];
     float zbuf[kMaxTopK][kMaxStrip];
     int16_t lst[kMaxTopK * kMaxStrip];     // active neurons: (slot << 12) | local
@@ -220,7 +222,6 @@ struct Smem {
     int nz_n;
     int route_e[kMaxTopK];
     float route_w[kMaxTopK];
-    float lg[kConsumerWarps][kMaxExperts];
     float inv_rms;
     int bc[2];
     uint64_t stage_bar;                    // completion of a staging round
@@ -236,6 +237,17 @@ __device__ __forceinline__ void prof_put(const DecodeParams &p, int li, int poin
     if (p.prof && threadIdx.x == 0)
         p.prof[(size_t(li) * kProfPoints + point) * gridDim.x + blockIdx.x] = v;
 }
+
+// Fixed-point accumulation (exact, so the result does not depend on the
+// order in which CTAs arrive): values are rounded to multiples of 2^-32 (2^-24
+// for sums of squares) and added as 64-bit integers.
+__device__ __forceinline__ void fix_add(long long *dst, float v, float scale)
+{
+    const long long q = __float2ll_rn(v * scale);
+    atomicAdd(reinterpret_cast<unsigned long long *>(dst), static_cast<unsigned long long>(q));
+}
+constexpr float kFixT = 4294967296.0f;    // 2^32
+constexpr float kFixSS = 16777216.0f;     // 2^24
 
 // Grid-wide barrier of all CTAs of the cooperative launch: arrivals are
 // fire-and-forget releases on one counter (never reset within a launch);
@@ -271,8 +283,8 @@ __device__ bool grid_sync(Smem *sm, const DecodeParams &p, unsigned &epoch, int 
     return ok;
 }
 
-// Staging round: thread 0 has issued bulk copies of `bytes` in total onto
-// sm->stage_bar; it waits (bounded) and the whole CTA adopts its verdict.
+// Staging round: thread 0 has issued bulk copies onto sm->stage_bar; it waits
+// (bounded) and the whole CTA adopts its verdict.
 __device__ bool stage_wait(Smem *sm, const DecodeParams &p, uint32_t &par, int &bci)
 {
     if (threadIdx.x == 0) {
@@ -292,8 +304,10 @@ __device__ bool stage_wait(Smem *sm, const DecodeParams &p, uint32_t &par, int &
     cta_sync();
     const bool ok = ld_vol(&sm->bc[bci]) != 0;
     bci ^= 1;
-    if (ok) mbar_test(&sm->stage_bar, par);   // acquire for this thread (phase complete)
-    par ^= 1;
+    if (ok) {
+        mbar_test(&sm->stage_bar, par);   // acquire for this thread (phase complete)
+        par ^= 1;                         // a failed round keeps its phase for the drain
+    }
     return ok;
 }
 
@@ -329,58 +343,149 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     const int d = p.d, r = p.r;
     const int s0 = p.strip_off[b], ns = p.strip_off[b + 1] - s0;
     const bool predict = p.mode == kModePredict;
+    const bool moe = p.E > 1;
     const int ntop = predict ? 1 : p.top_k;
-    const int rows_total = ntop * r;
-    const int a0 = int((long long)b * rows_total / S), a1 = int((long long)(b + 1) * rows_total / S);
     const int nvecW = (WF == kI4 ? d / 2 : d * (WF == kF32 ? 4 : 2)) / VBW;
     const int nvecP = p.vrow / VBP;
     const int nvecU = p.urow / VBP;
     const int l0 = p.layer_begin;
     const int l1 = predict ? p.layer_begin + 1 : p.layer_end;
-    const bool dense_ahead = !predict && p.E == 1;
+    // this CTA's columns of the residual (8-column groups)
+    const int c0 = 8 * p.grp_off[b], ncol = 8 * (p.grp_off[b + 1] - p.grp_off[b]);
+    // this CTA's rows of t (row-split form, MoE)
+    const int rows_total = ntop * r;
+    const int a0 = int((long long)b * rows_total / S), a1 = int((long long)(b + 1) * rows_total / S);
+    const int ucap = kStageBytes / p.urow;   // U rows per staging round
 
-    // L2 prefetch of a layer's predictor slice of this CTA: V rows [a0, a1)
-    // of the concatenated experts and the U strip of each expert.
-    auto prefetch_pred = [&](int l, const int *experts, bool want_v, bool want_u) {
-        for (int e = 0; e < ntop; ++e) {
-            const ExpertDev &ex = p.ex[size_t(l) * p.E + experts[e]];
-            const int lo = max(a0, e * r), hi = min(a1, (e + 1) * r);
-            if (want_v && hi > lo)
-                prefetch_l2(ex.V + size_t(lo - e * r) * p.vrow, uint32_t(hi - lo) * p.vrow);
-            if (want_u && ns > 0)
-                prefetch_l2(ex.U + size_t(s0) * p.urow, uint32_t(ns) * p.urow);
-        }
+    // V block of this CTA (dense): rows of t restricted to this CTA's columns
+    auto vblk = [&](int l) -> const uint8_t * {
+        return p.ex[size_t(l) * p.E].V + size_t(r) * c0 * (p.vrow / d);
+    };
+    const int vbrow = ncol * (p.vrow / d);   // bytes of one V-block row
+
+    unsigned epoch = 0;
+    uint32_t spar = 0;
+    int bci = 0, rb = 0;
+    bool staged_early = false;   // round 0 of the next U strip is already in flight
+    bool pending = false;        // a staging round was issued and not yet waited for
+
+    // stage rows [0, n) of expert slot e's U strip (thread 0)
+    auto stage_u = [&](int l, int expert, int row0, int n) {
+        const uint8_t *U = p.ex[size_t(l) * p.E + expert].U + size_t(s0 + row0) * p.urow;
+        mbar_arrive_tx(&sm.stage_bar, uint32_t(n) * p.urow);
+        stage_copy(stg, U, uint32_t(n) * p.urow, &sm.stage_bar);
     };
 
     if (tid == 0) {
         mbar_init(&sm.stage_bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        if (predict) {
-            const int ex[kMaxTopK] = {p.pred_expert, 0};
-            prefetch_pred(l0, ex, true, true);
-        } else if (dense_ahead) {
-            const int ex[kMaxTopK] = {0, 0};
-            prefetch_pred(l0, ex, true, true);
+        if (!moe && ns > 0) {
+            stage_u(l0, 0, 0, min(ns, ucap));
+            if (ns > ucap) prefetch_l2(p.ex[size_t(l0) * p.E].U + size_t(s0 + ucap) * p.urow,
+                                       uint32_t(ns - ucap) * p.urow);
         }
     }
-
+    if (!moe && ns > 0) staged_early = pending = true;
     cta_sync();
-    unsigned epoch = 0;
-    uint32_t spar = 0;
-    int bci = 0;
+
+    // -----------------------------------------------------------------------
+    // Column phase: this CTA's columns of r (the layer input `li_in`), its
+    // sum of squares, and its partial products for the next layer: the t
+    // partial V[:, cols] r[cols] (dense) or the router logit partials (MoE),
+    // all added in fixed point.  `from_partials`: r = r_old + sum of the
+    // per-CTA partials of y in fixed CTA order; otherwise r is the input.
+    // -----------------------------------------------------------------------
+    auto column_phase = [&](int li_in, bool from_partials, bool next_exists, int l_next) {
+        const float *src = predict ? p.x_in : p.resid;
+        long long *fx = p.fix + size_t(li_in & 1) * kFixStride;
+        if (from_partials) {
+            const int q0 = c0 / 4, nq = ncol / 4;
+            for (int qq = warp; qq < nq; qq += kConsumerWarps) {
+                const int q = q0 + qq;
+                float4 pv[kMaxStrips / 32];
+#pragma unroll
+                for (int j = 0; j < kMaxStrips / 32; ++j) {
+                    const int c = lane + 32 * j;
+                    pv[j] = c < S ? __ldcg(reinterpret_cast<const float4 *>(p.partials + size_t(c) * d) + q)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+                float4 sacc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int j = 0; j < kMaxStrips / 32; ++j) {
+                    sacc.x += pv[j].x; sacc.y += pv[j].y; sacc.z += pv[j].z; sacc.w += pv[j].w;
+                }
+                sacc.x = warp_sum(sacc.x); sacc.y = warp_sum(sacc.y);
+                sacc.z = warp_sum(sacc.z); sacc.w = warp_sum(sacc.w);
+                if (lane == 0) {
+                    float4 rv = __ldcg(reinterpret_cast<const float4 *>(p.resid) + q);
+                    rv.x += sacc.x; rv.y += sacc.y; rv.z += sacc.z; rv.w += sacc.w;
+                    __stcg(reinterpret_cast<float4 *>(p.resid) + q, rv);
+                    *reinterpret_cast<float4 *>(sm.rsl + 4 * qq) = rv;
+                }
+            }
+        } else {
+            for (int j = tid; j < ncol; j += kThreads) sm.rsl[j] = __ldcg(src + c0 + j);
+        }
+        cta_sync();
+        if (!predict && p.trace && li_in < l1 - l0)
+            for (int j = tid; j < ncol; j += kThreads) __stcg(p.trace + size_t(li_in) * d + c0 + j, sm.rsl[j]);
+        if (!next_exists) return;
+        // sum of squares of this CTA's columns (fixed order: lanes, then tree)
+        if (warp == 0 && !predict) {
+            float ss = 0.f;
+            for (int j = lane; j < ncol; j += 32) ss = fmaf(sm.rsl[j], sm.rsl[j], ss);
+            ss = warp_sum(ss);
+            if (lane == 0 && ncol > 0) fix_add(fx + kMaxRankTotal, ss, kFixSS);
+        }
+        if (!moe) {
+            // t partial: row k of the V block dotted with this CTA's columns
+            const uint8_t *vb = vblk(l_next);
+            const int nv = vbrow / VBP;
+            for (int k = tid; k < r; k += kThreads) {
+                float a = 0.f;
+                const uint8_t *row = vb + size_t(k) * vbrow;
+                for (int v = 0; v < nv; ++v) {
+                    float w[EPVP];
+                    cvt<PF>(ldvec<PF>(row + v * VBP), w);
+#pragma unroll
+                    for (int i = 0; i < EPVP; ++i) a = fmaf(w[i], sm.rsl[v * EPVP + i], a);
+                }
+                if (ncol > 0) fix_add(fx + k, a, kFixT);
+            }
+        } else if (!predict) {
+            // router logit partials: W_r[e, cols] . r[cols]
+            const __half *R = reinterpret_cast<const __half *>(p.router[l_next]);
+            if (tid < p.E && ncol > 0) {
+                float a = 0.f;
+                for (int j = 0; j < ncol; ++j) a = fmaf(__half2float(R[size_t(tid) * d + c0 + j]), sm.rsl[j], a);
+                fix_add(fx + kMaxRankTotal + 1 + tid, a, kFixT);
+            }
+        }
+    };
+
     float xw[MAXVW * EPVW];
     float xp_own[kSameX ? 1 : MAXVP * EPVP];
 #define XP(i) (kSameX ? xw[(i)] : xp_own[(i)])
-    int rb = 0;
 
-    for (int l = l0; l < l1; ++l) {
+    // prologue: the first layer's input columns
+    column_phase(0, false, true, l0);
+    long long cyc0 = 0;
+    const bool started = grid_sync(&sm, p, epoch, bci, &cyc0);
+
+    for (int l = l0; started && l < l1; ++l) {
         const int li = l - l0;
         long long cyc_a = 0, cyc_b = 0, cyc_c = 0, cyc_bar = 0;
         prof_put(p, li, 0, gtimer());
         const long long ca0 = clock64();
+        const long long *fx = p.fix + size_t(li & 1) * kFixStride;
 
-        // ---------------- phase A: layer input ------------------------------
+        // ---------------- layer input x, [MoE] routing and t rows ------------
         const float *src = predict ? p.x_in : p.resid;
+        float inv = 1.f;
+        if (!predict) {
+            const long long ssq = __ldcg(fx + kMaxRankTotal);
+            inv = 1.f / sqrtf(float(double(ssq) * (1.0 / 16777216.0)) / float(d) + p.eps);
+        }
 #pragma unroll
         for (int k = 0; k < MAXVW; ++k) {
             const int v = tid + kThreads * k;
@@ -388,8 +493,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             for (int i = 0; i < EPVW; i += 4) {
                 float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (v < nvecW) q = __ldcg(reinterpret_cast<const float4 *>(src + v * EPVW + i));
-                xw[k * EPVW + i] = q.x; xw[k * EPVW + i + 1] = q.y;
-                xw[k * EPVW + i + 2] = q.z; xw[k * EPVW + i + 3] = q.w;
+                xw[k * EPVW + i] = q.x * inv; xw[k * EPVW + i + 1] = q.y * inv;
+                xw[k * EPVW + i + 2] = q.z * inv; xw[k * EPVW + i + 3] = q.w * inv;
             }
         }
         if constexpr (!kSameX) {
@@ -400,131 +505,76 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 for (int i = 0; i < EPVP; i += 4) {
                     float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
                     if (v < nvecP) q = __ldcg(reinterpret_cast<const float4 *>(src + v * EPVP + i));
-                    xp_own[k * EPVP + i] = q.x; xp_own[k * EPVP + i + 1] = q.y;
-                    xp_own[k * EPVP + i + 2] = q.z; xp_own[k * EPVP + i + 3] = q.w;
+                    xp_own[k * EPVP + i] = q.x * inv; xp_own[k * EPVP + i + 1] = q.y * inv;
+                    xp_own[k * EPVP + i + 2] = q.z * inv; xp_own[k * EPVP + i + 3] = q.w * inv;
                 }
             }
         }
-        if (!predict) {
-            // x = r / sqrt(mean(r^2) + eps); the W-format columns cover d once
-            float ss = 0.f;
-#pragma unroll
-            for (int k = 0; k < MAXVW; ++k) {
-                const int v = tid + kThreads * k;
-                if (v < nvecW) {
-#pragma unroll
-                    for (int i = 0; i < EPVW; ++i) ss = fmaf(xw[k * EPVW + i], xw[k * EPVW + i], ss);
-                    if (p.trace && b == 0) {
-#pragma unroll
-                        for (int i = 0; i < EPVW; i += 4)
-                            __stcg(reinterpret_cast<float4 *>(p.trace + size_t(li) * d + v * EPVW + i),
-                                   make_float4(xw[k * EPVW + i], xw[k * EPVW + i + 1],
-                                               xw[k * EPVW + i + 2], xw[k * EPVW + i + 3]));
+        if (!moe) {
+            // t from the fixed-point column partials
+            for (int k = tid; k < r; k += kThreads)
+                sm.tsm[k] = float(double(__ldcg(fx + k)) * (1.0 / 4294967296.0)) * inv;
+            if (tid == 0) {
+                sm.route_e[0] = predict ? p.pred_expert : 0;
+                sm.route_e[1] = 0;
+                sm.route_w[0] = 1.f;
+                sm.route_w[1] = 0.f;
+                if (p.stats && b == 0 && !predict) {
+                    p.stats[li * 4 + 2] = -1;
+                    p.stats[li * 4 + 3] = -1;
+                }
+            }
+            cta_sync();
+        } else {
+            // routing from the fixed-point logits, identical in every CTA:
+            // softmax over E, two largest (ties: lower index), renormalised
+            if (tid == 0) {
+                int lo = p.pred_expert, hi = 0;
+                float wlo = 1.f, whi = 0.f;
+                if (!predict) {
+                    float logit[kMaxExperts], pr[kMaxExperts];
+                    float mx = -INFINITY;
+                    for (int e = 0; e < p.E; ++e) {
+                        logit[e] = float(double(__ldcg(fx + kMaxRankTotal + 1 + e)) * (1.0 / 4294967296.0)) * inv;
+                        mx = fmaxf(mx, logit[e]);
+                    }
+                    float den = 0.f;
+                    for (int e = 0; e < p.E; ++e) { pr[e] = expf(logit[e] - mx); den += pr[e]; }
+                    for (int e = 0; e < p.E; ++e) pr[e] /= den;
+                    int ea = 0;
+                    for (int e = 1; e < p.E; ++e) if (pr[e] > pr[ea]) ea = e;
+                    int eb = ea == 0 ? 1 : 0;
+                    for (int e = 0; e < p.E; ++e) if (e != ea && pr[e] > pr[eb]) eb = e;
+                    lo = min(ea, eb);
+                    hi = max(ea, eb);
+                    wlo = pr[lo] / (pr[lo] + pr[hi]);
+                    whi = pr[hi] / (pr[lo] + pr[hi]);
+                    if (p.stats && b == 0) {
+                        p.stats[li * 4 + 2] = lo;
+                        p.stats[li * 4 + 3] = hi;
                     }
                 }
-            }
-            ss = warp_sum(ss);
-            if (lane == 0) sm.red[rb][warp][0] = ss;
-            cta_sync();
-            if (tid == 0) {
-                float tot = 0.f;
-                for (int w = 0; w < kConsumerWarps; ++w) tot += sm.red[rb][w][0];
-                sm.inv_rms = 1.f / sqrtf(tot / float(d) + p.eps);
-            }
-            cta_sync();
-            rb ^= 1;
-            const float inv = sm.inv_rms;
-#pragma unroll
-            for (int i = 0; i < MAXVW * EPVW; ++i) xw[i] *= inv;
-            if constexpr (!kSameX) {
-#pragma unroll
-                for (int i = 0; i < MAXVP * EPVP; ++i) xp_own[i] *= inv;
-            }
-        }
-        prof_put(p, li, 1, gtimer());
-
-        // MoE routing, computed identically by every CTA: logits of the E
-        // experts (fp16 router, 8-element vectors like the predictor format),
-        // softmax, two largest (ties: lower index), weights renormalised over
-        // the two, experts in ascending index.
-        if (!predict && p.E > 1) {
-            const uint8_t *R = p.router[l];
-            float lg[kMaxExperts];
-#pragma unroll
-            for (int e = 0; e < kMaxExperts; ++e) {
-                lg[e] = 0.f;
-                if (e < p.E) {
-#pragma unroll
-                    for (int k = 0; k < MAXVP; ++k) {
-                        const int v = tid + kThreads * k;
-                        if (v < nvecP) {
-                            float w[8];
-                            cvt<kF16>(ldw4(R + (size_t(e) * nvecP + v) * 16), w);
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) lg[e] = fmaf(w[i], XP(k * EPVP + i), lg[e]);
-                        }
-                    }
-                }
-            }
-#pragma unroll
-            for (int e = 0; e < kMaxExperts; ++e) {
-                if (e < p.E) {
-                    const float v = warp_sum(lg[e]);
-                    if (lane == 0) sm.lg[warp][e] = v;
-                }
-            }
-            cta_sync();
-            if (tid == 0) {
-                float logit[kMaxExperts];
-                float mx = -INFINITY;
-                for (int e = 0; e < p.E; ++e) {
-                    float s = 0.f;
-                    for (int w = 0; w < kConsumerWarps; ++w) s += sm.lg[w][e];
-                    logit[e] = s;
-                    mx = fmaxf(mx, s);
-                }
-                float pr[kMaxExperts];
-                float den = 0.f;
-                for (int e = 0; e < p.E; ++e) { pr[e] = expf(logit[e] - mx); den += pr[e]; }
-                for (int e = 0; e < p.E; ++e) pr[e] /= den;
-                int ea = 0;
-                for (int e = 1; e < p.E; ++e) if (pr[e] > pr[ea]) ea = e;
-                int eb = ea == 0 ? 1 : 0;
-                for (int e = 0; e < p.E; ++e) if (e != ea && pr[e] > pr[eb]) eb = e;
-                const int lo = min(ea, eb), hi = max(ea, eb);
                 sm.route_e[0] = lo;
                 sm.route_e[1] = hi;
-                sm.route_w[0] = pr[lo] / (pr[lo] + pr[hi]);
-                sm.route_w[1] = pr[hi] / (pr[lo] + pr[hi]);
-                if (p.stats && b == 0) {
-                    p.stats[li * 4 + 2] = lo;
-                    p.stats[li * 4 + 3] = hi;
+                sm.route_w[0] = wlo;
+                sm.route_w[1] = whi;
+                // the experts' V rows and U strips start moving now
+                for (int e = 0; e < ntop; ++e) {
+                    const ExpertDev &ex = p.ex[size_t(l) * p.E + (e == 0 ? lo : hi)];
+                    const int lo_r = max(a0, e * r), hi_r = min(a1, (e + 1) * r);
+                    if (hi_r > lo_r)
+                        prefetch_l2(ex.V + size_t(lo_r - e * r) * p.vrow, uint32_t(hi_r - lo_r) * p.vrow);
+                    if (ns > 0) prefetch_l2(ex.U + size_t(s0) * p.urow, uint32_t(ns) * p.urow);
                 }
-                // the two experts' predictor slices start moving now
-                prefetch_pred(l, sm.route_e, true, true);
             }
-        } else if (tid == 0) {
-            sm.route_e[0] = predict ? p.pred_expert : 0;
-            sm.route_e[1] = 0;
-            sm.route_w[0] = 1.f;
-            sm.route_w[1] = 0.f;
-            if (p.stats && b == 0 && !predict) {
-                p.stats[li * 4 + 2] = -1;
-                p.stats[li * 4 + 3] = -1;
-            }
-        }
-        cta_sync();
-
-        // ---------------- phase A: t rows [a0, a1) ---------------------------
-        // staged through shared memory in rounds of up to kRA rows
-        {
+            cta_sync();
+            // t rows [a0, a1) of the two experts, staged in rounds of kRA rows
             const int per = min(kRA, kStageBytes / p.vrow);
             bool ok = true;
             for (int row0 = a0; row0 < a1 && ok; row0 += per) {
                 const int n = min(per, a1 - row0);
                 if (tid == 0) {
                     mbar_arrive_tx(&sm.stage_bar, uint32_t(n) * p.vrow);
-                    // the rows of one round lie in at most two experts' V
                     for (int rr = 0; rr < n;) {
                         const int row = row0 + rr, e = row / r;
                         const int cnt = min(n - rr, (e + 1) * r - row);
@@ -534,7 +584,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                         rr += cnt;
                     }
                 }
+                pending = true;
                 if (!stage_wait(&sm, p, spar, bci)) { ok = false; break; }
+                pending = false;
                 float part[kRA];
 #pragma unroll
                 for (int rr = 0; rr < kRA; ++rr) {
@@ -568,50 +620,34 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 rb ^= 1;
             }
             if (!ok) break;
+            // round 0 of the first expert's U strip lands during the barrier
+            if (tid == 0 && ns > 0) stage_u(l, sm.route_e[0], 0, min(ns, ucap));
+            staged_early = pending = ns > 0;
+            if (!grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
+            for (int k = tid; k < ntop * r; k += kThreads) sm.tsm[k] = __ldcg(p.t_buf + k);
         }
+        for (int e = 0; e < ntop; ++e)
+            for (int i = tid; i < ns; i += kThreads)
+                sm.cbuf[e][i] = __ldg(p.ex[size_t(l) * p.E + sm.route_e[e]].c + s0 + i);
+        cta_sync();
         cyc_a = clock64() - ca0;
-        prof_put(p, li, 2, gtimer());
-        if (!grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
-        prof_put(p, li, 3, gtimer());
+        prof_put(p, li, 1, gtimer());
 
-        // ---------------- phase B: z = U t - c, threshold, compaction --------
+        // ---------------- z = U t - c over the strip, compaction -------------
         const long long cb0 = clock64();
         {
-            constexpr int kTV = kMaxRankTotal / kThreads;
-            float tv[kTV];
-#pragma unroll
-            for (int k = 0; k < kTV; ++k) {
-                const int i = tid + kThreads * k;
-                tv[k] = i < ntop * r ? __ldcg(p.t_buf + i) : 0.f;
-            }
-            float cv[kMaxTopK];
-#pragma unroll
-            for (int e = 0; e < kMaxTopK; ++e)
-                cv[e] = (e < ntop && tid < ns) ? __ldg(p.ex[size_t(l) * p.E + sm.route_e[e]].c + s0 + tid)
-                                               : 0.f;
-#pragma unroll
-            for (int k = 0; k < kTV; ++k) {
-                const int i = tid + kThreads * k;
-                if (i < ntop * r) sm.tsm[i] = tv[k];
-            }
-#pragma unroll
-            for (int e = 0; e < kMaxTopK; ++e)
-                if (e < ntop && tid < ns) sm.cbuf[e][tid] = cv[e];
-        }
-        cta_sync();
-        {
             bool ok = true;
-            const int per = kStageBytes / p.urow;   // U rows per staging round
             for (int e = 0; e < ntop && ok; ++e) {
                 const float *te = sm.tsm + e * r;
-                const uint8_t *U = p.ex[size_t(l) * p.E + sm.route_e[e]].U + size_t(s0) * p.urow;
-                for (int row0 = 0; row0 < ns && ok; row0 += per) {
-                    const int n = min(per, ns - row0);
-                    if (tid == 0) {
-                        mbar_arrive_tx(&sm.stage_bar, uint32_t(n) * p.urow);
-                        stage_copy(stg, U + size_t(row0) * p.urow, uint32_t(n) * p.urow, &sm.stage_bar);
+                for (int row0 = 0; row0 < ns && ok; row0 += ucap) {
+                    const int n = min(ucap, ns - row0);
+                    if (!(staged_early && row0 == 0)) {
+                        if (tid == 0) stage_u(l, sm.route_e[e], row0, n);
                     }
+                    staged_early = false;
+                    pending = true;
                     if (!stage_wait(&sm, p, spar, bci)) { ok = false; break; }
+                    pending = false;
                     for (int rr = warp; rr < n; rr += kConsumerWarps) {
                         const uint8_t *urow = stg + size_t(rr) * p.urow;
                         float a = 0.f;
@@ -674,7 +710,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         if (tid == 0) sm.nz_n = 0;
         cta_sync();
         cyc_b = clock64() - cb0;
-        prof_put(p, li, 4, gtimer());
+        prof_put(p, li, 2, gtimer());
 
         if (predict) {
             // global ascending list: prefix of the strip counts, then copy
@@ -692,11 +728,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             break;
         }
 
-        // ---------------- phase C: gather rows of active neurons -------------
+        // ---------------- gather rows of active neurons ----------------------
         const long long cc0 = clock64();
         const int m0 = sm.lst_n[0];
         const int m = m0 + (ntop > 1 ? sm.lst_n[1] : 0);
-        // list index j -> (slot << 12 | local): slot 0 entries, then slot 1
         auto entry = [&](int j) -> int { return j < m0 ? sm.lst[j] : sm.lst[kMaxStrip + (j - m0)]; };
         const ExpertDev *exs[kMaxTopK] = {&p.ex[size_t(l) * p.E + sm.route_e[0]],
                                           &p.ex[size_t(l) * p.E + sm.route_e[ntop > 1 ? 1 : 0]]};
@@ -704,10 +739,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             const int en = entry(j), e = en >> 12, loc = en & 0xfff;
             prefetch_l2(exs[e]->Wgu + size_t(s0 + loc) * p.gu_bytes, uint32_t(p.gu_bytes));
             if (p.spec_down) prefetch_l2(exs[e]->Wd + size_t(s0 + loc) * p.wrow, uint32_t(p.wrow));
-        }
-        if (tid == kThreads - 1 && dense_ahead && l + 1 < l1) {
-            const int ex[kMaxTopK] = {0, 0};
-            prefetch_pred(l + 1, ex, true, true);
         }
 
         float acc[MAXVW * EPVW];
@@ -804,7 +835,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             cta_sync();
             rb ^= 1;
         };
-        // W_down rows of sm.nz[q0, q1) into registers / into acc
         auto load_dn = [&](int q0, int q1) {
 #pragma unroll
             for (int n = 0; n < NB; ++n) {
@@ -850,7 +880,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             finish_gu(0);
         }
         for (int bt = 0; bt < nbat; ++bt) {
-            // W_down rows found so far + the records of batch bt + 1, together
+            // W_down rows found so far together with the records of batch bt + 1
             const int dn_hi = min(sm.nz_n, dn_done + NB);
             load_dn(dn_done, dn_hi);
             if (bt + 1 < nbat) load_gu(bt + 1);
@@ -865,7 +895,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             axpy_dn(dn_done, dn_hi);
             dn_done = dn_hi;
         }
-        if (tid == 0 && p.stats) atomicAdd(p.stats + li * 4 + 1, nz_total);
+        if (tid == 0) {
+            if (p.stats) atomicAdd(p.stats + li * 4 + 1, nz_total);
+            // the next layer's predictor slice starts moving: U strip straight
+            // into shared memory (free until then), V block into L2
+            if (!moe && l + 1 < l1) {
+                if (ns > 0) {
+                    stage_u(l + 1, 0, 0, min(ns, ucap));
+                    if (ns > ucap)
+                        prefetch_l2(p.ex[size_t(l + 1) * p.E].U + size_t(s0 + ucap) * p.urow,
+                                    uint32_t(ns - ucap) * p.urow);
+                }
+                if (ncol > 0) prefetch_l2(vblk(l + 1), uint32_t(r) * vbrow);
+            }
+        }
+        staged_early = !moe && l + 1 < l1 && ns > 0;
+        if (staged_early) pending = true;
+        // the fixed-point buffer of layer l - 1 (read before two barriers ago)
+        // is cleared for layer l + 1
+        if (b == S - 1) {
+            long long *fz = p.fix + size_t((li + 1) & 1) * kFixStride;
+            for (int i = tid; i < kFixStride; i += kThreads) fz[i] = 0;
+        }
         // per-CTA partial of y
 #pragma unroll
         for (int k = 0; k < MAXVW; ++k) {
@@ -879,46 +930,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             }
         }
         cyc_c = clock64() - cc0;
-        prof_put(p, li, 5, gtimer());
-        prof_put(p, li, 6, gtimer());
+        prof_put(p, li, 3, gtimer());
         if (!grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
-        prof_put(p, li, 7, gtimer());
+        prof_put(p, li, 4, gtimer());
 
-        // ---------------- phase D: r += sum of partials (fixed order) --------
-        {
-            constexpr int kParts = kMaxStrips / 32;   // partial rows per lane
-            const int nq = d / 4;
-            const int q0 = int((long long)b * nq / S), q1 = int((long long)(b + 1) * nq / S);
-            for (int q = q0 + warp; q < q1; q += kConsumerWarps) {
-                float4 pv[kParts];
-#pragma unroll
-                for (int j = 0; j < kParts; ++j) {
-                    const int c = lane + 32 * j;
-                    pv[j] = c < S ? __ldcg(reinterpret_cast<const float4 *>(p.partials + size_t(c) * d) + q)
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-                float4 sacc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int j = 0; j < kParts; ++j) {
-                    sacc.x += pv[j].x; sacc.y += pv[j].y; sacc.z += pv[j].z; sacc.w += pv[j].w;
-                }
-                sacc.x = warp_sum(sacc.x); sacc.y = warp_sum(sacc.y);
-                sacc.z = warp_sum(sacc.z); sacc.w = warp_sum(sacc.w);
-                if (lane == 0) {
-                    float4 rv = __ldcg(reinterpret_cast<const float4 *>(p.resid) + q);
-                    rv.x += sacc.x; rv.y += sacc.y; rv.z += sacc.z; rv.w += sacc.w;
-                    __stcg(reinterpret_cast<float4 *>(p.resid) + q, rv);
-                }
-            }
-        }
-        prof_put(p, li, 8, gtimer());
-        if (!grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
-        prof_put(p, li, 9, gtimer());
+        // ---------------- reduction + next layer's column products -----------
+        const bool next = l + 1 < l1;
+        column_phase(li + 1, true, next, l + 1);
+        prof_put(p, li, 5, gtimer());
+        if (next && !grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
+        prof_put(p, li, 6, gtimer());
         prof_put(p, li, 10, cyc_a);
         prof_put(p, li, 11, cyc_b);
         prof_put(p, li, 12, cyc_c);
         prof_put(p, li, 13, cyc_bar);
     }
+    // an early exit may leave one staging round in flight: let it land
+    // (bounded) so no bulk copy writes this CTA's shared memory after exit
+    if (pending && tid == 0) {
+        const long long t0 = gtimer();
+        while (!mbar_test(&sm.stage_bar, spar) && gtimer() - t0 < p.wait_ns) {
+        }
+    }
+#undef XP
 }
 
 template <int WF, int PF>

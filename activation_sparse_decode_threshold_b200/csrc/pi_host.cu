@@ -67,6 +67,7 @@ struct pi_ffn {
     int wfmt = 0, pfmt = 0, gated = 0;
     int vrow = 0, urow = 0, wrow = 0;
     std::vector<int32_t> strip_off;
+    std::vector<int32_t> grp_off;              // column slices in 8-column groups
     std::vector<std::vector<int32_t>> perm;   // [layer * E + e]
     std::vector<uint8_t *> mem;               // [layer * E + e]
     std::vector<uint8_t *> router_mem;        // [layer]
@@ -75,6 +76,8 @@ struct pi_ffn {
     pi::ExpertDev *d_ex = nullptr;
     const uint8_t **d_router = nullptr;
     int32_t *d_strip_off = nullptr;
+    int32_t *d_grp_off = nullptr;
+    long long *fix = nullptr;
     // scratch
     uint8_t *scratch = nullptr;
     float *t_buf = nullptr, *partials = nullptr, *io = nullptr;
@@ -169,6 +172,16 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
         return fail(PI_ERR_UNSUPPORTED, "d_ff %d exceeds %d neurons per strip x %d strips", D.d_ff,
                     pi::kMaxStrip, h->S);
     }
+    {
+        const int ng = D.d_model / 8;
+        h->grp_off.resize(h->S + 1);
+        for (int b = 0; b <= h->S; ++b) h->grp_off[b] = int((long long)b * ng / h->S);
+        if ((ng + h->S - 1) / h->S * 8 > pi::kMaxSliceCols) {
+            delete h;
+            return fail(PI_ERR_UNSUPPORTED, "d_model / n_strips exceeds %d columns per strip",
+                        pi::kMaxSliceCols);
+        }
+    }
     h->strip_off.resize(h->S + 1);
     {
         const int q = D.d_ff / h->S, rem = D.d_ff % h->S;
@@ -190,13 +203,17 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
     const size_t o_counts = up256(o_lists + sizeof(int32_t) * size_t(h->S) * pi::kMaxStrip);
     const size_t o_bar = up256(o_counts + sizeof(int32_t) * h->S);
     const size_t o_err = o_bar + 256;
-    const size_t total = o_err + 256;
+    const size_t o_fix = o_err + 256;
+    const size_t total = up256(o_fix + sizeof(long long) * 2 * pi::kFixStride);
     cudaError_t e = cudaMalloc(&h->scratch, total);
     if (e == cudaSuccess) e = cudaMemset(h->scratch, 0, total);
     if (e == cudaSuccess) e = cudaMalloc(&h->d_ex, sizeof(pi::ExpertDev) * size_t(L) * E);
     if (e == cudaSuccess) e = cudaMemset(h->d_ex, 0, sizeof(pi::ExpertDev) * size_t(L) * E);
     if (e == cudaSuccess) e = cudaMalloc(&h->d_router, sizeof(uint8_t *) * size_t(L));
     if (e == cudaSuccess) e = cudaMemset(h->d_router, 0, sizeof(uint8_t *) * size_t(L));
+    if (e == cudaSuccess) e = cudaMalloc(&h->d_grp_off, sizeof(int32_t) * (h->S + 1));
+    if (e == cudaSuccess)
+        e = cudaMemcpy(h->d_grp_off, h->grp_off.data(), sizeof(int32_t) * (h->S + 1), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMalloc(&h->d_strip_off, sizeof(int32_t) * (h->S + 1));
     if (e == cudaSuccess)
         e = cudaMemcpy(h->d_strip_off, h->strip_off.data(), sizeof(int32_t) * (h->S + 1),
@@ -213,6 +230,7 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
     h->counts = reinterpret_cast<int32_t *>(h->scratch + o_counts);
     h->bar = reinterpret_cast<unsigned *>(h->scratch + o_bar);
     h->err = reinterpret_cast<int *>(h->scratch + o_err);
+    h->fix = reinterpret_cast<long long *>(h->scratch + o_fix);
     *out = h;
     return PI_OK;
 }
@@ -226,6 +244,7 @@ void pi_ffn_destroy(pi_ffn_t h)
     cudaFree(h->d_ex);
     cudaFree(h->d_router);
     cudaFree(h->d_strip_off);
+    cudaFree(h->d_grp_off);
     cudaFree(h->scratch);
     pi::prefill_destroy(h->prefill);
     delete h;
@@ -314,7 +333,11 @@ pi_status pi_ffn_load_layer(pi_ffn_t h, int layer, const pi_expert_weights *expe
         uint8_t *m = h->mem[idx];
         PI_CUDA(cudaMemcpyAsync(d_perm, h->perm[idx].data(), sizeof(int32_t) * F,
                                 cudaMemcpyHostToDevice, st), "copy perm");
-        PI_CUDA(cudaMemcpyAsync(m + o_V, w.V, size_t(r) * h->vrow, cudaMemcpyDeviceToDevice, st), "copy V");
+        if (E == 1)   // dense: column blocks, one per strip (see pi_decode.cu)
+            PI_CUDA(pi::repack_v_blocks(static_cast<const uint8_t *>(w.V), m + o_V, h->d_grp_off, h->S, r, d,
+                                        elem_bytes(D.pred_dtype), st), "repack V");
+        else
+            PI_CUDA(cudaMemcpyAsync(m + o_V, w.V, size_t(r) * h->vrow, cudaMemcpyDeviceToDevice, st), "copy V");
         {
             const uint8_t *src[1] = {static_cast<const uint8_t *>(w.U)};
             const int rb[1] = {h->urow};
@@ -386,6 +409,8 @@ static pi::DecodeParams base_params(pi_ffn_t h)
     p.ex = h->d_ex;
     p.router = h->d_router;
     p.strip_off = h->d_strip_off;
+    p.grp_off = h->d_grp_off;
+    p.fix = h->fix;
     p.d = D.d_model;
     p.F = D.d_ff;
     p.r = D.rank;
@@ -434,6 +459,7 @@ pi_status pi_predict(pi_ffn_t h, int layer, int expert, const float *x_dev, int3
     p.idx_out = idx_dev;
     p.count_out = count_dev;
     PI_CUDA(cudaMemsetAsync(h->bar, 0, 2 * sizeof(unsigned), st), "memset barrier");
+    PI_CUDA(cudaMemsetAsync(h->fix, 0, sizeof(long long) * 2 * pi::kFixStride, st), "memset accumulators");
     PI_CUDA(pi::launch_decode(h->wfmt, h->pfmt, p, st), "launch predict");
     return PI_OK;
 }
@@ -462,6 +488,7 @@ pi_status pi_sparse_ffn_decode(pi_ffn_t h, int layer_begin, int layer_end, float
     p.stats = stats_dev;
     p.masks = mask_dev;
     PI_CUDA(cudaMemsetAsync(h->bar, 0, 2 * sizeof(unsigned), st), "memset barrier");
+    PI_CUDA(cudaMemsetAsync(h->fix, 0, sizeof(long long) * 2 * pi::kFixStride, st), "memset accumulators");
     if (stats_dev) PI_CUDA(cudaMemsetAsync(stats_dev, 0, sizeof(int32_t) * 4 * nl, st), "memset stats");
     if (mask_dev)
         PI_CUDA(cudaMemsetAsync(mask_dev, 0, sizeof(uint32_t) * size_t(nl) * D.top_k * ((D.d_ff + 31) / 32), st),

@@ -17,6 +17,8 @@ constexpr int kMaxTopK = 2;
 constexpr int kMaxExperts = 16;
 constexpr int kMaxRankTotal = 2048;   // top_k * rank
 constexpr int kStageBytes = 192 * 1024;   // shared-memory staging of V rows / U strips
+constexpr int kMaxSliceCols = 1024;       // residual columns per CTA at most
+constexpr int kFixStride = kMaxRankTotal + 1 + kMaxExperts;   // t, sum r^2, logits
 
 enum Fmt { kF32 = 0, kF16 = 1, kBF16 = 2, kI4 = 3 };
 
@@ -26,7 +28,8 @@ enum Fmt { kF32 = 0, kF16 = 1, kBF16 = 2, kI4 = 3 };
 // bulk copy brings everything the neuron's activation needs.  An INT4 row is
 // its d/2 nibble bytes followed by its d/32 fp16 scales.
 struct ExpertDev {
-    const uint8_t *V;    // r rows of vrow bytes (original order; rank is not permuted)
+    const uint8_t *V;    // dense: column blocks, one per CTA (block b: r rows of its
+                         // columns); MoE: r rows of vrow bytes (rank is not permuted)
     const uint8_t *U;    // F rows of urow bytes, table order
     const float *c;      // F biases, table order
     const uint8_t *Wgu;  // F input records of gu_bytes, table order
@@ -39,6 +42,7 @@ struct DecodeParams {
     const ExpertDev *ex;            // [n_layers * E]
     const uint8_t *const *router;   // [n_layers] E x d fp16, or null entries
     const int32_t *strip_off;       // [S + 1]
+    const int32_t *grp_off;         // [S + 1] column slices, in 8-column groups
     int d, F, r, E, top_k, act, gated, S;
     int layer_begin, layer_end;
     float threshold, eps;
@@ -56,6 +60,7 @@ struct DecodeParams {
     int32_t *idx_out, *count_out;   // predict
     // scratch (library-owned or caller-provided, see pi_host.cu)
     float *t_buf;                   // [top_k * r]
+    long long *fix;                 // [2 * kFixStride] fixed-point accumulators, zeroed
     float *partials;                // [S * d]
     int32_t *lists;                 // [S * kMaxStrip]  (predict)
     int32_t *counts;                // [S]              (predict)
@@ -67,7 +72,7 @@ struct DecodeParams {
 };
 
 // Phase timestamps recorded per layer and CTA when DecodeParams::prof is set.
-constexpr int kProfPoints = 14;   // 10 timestamps + 4 cycle counters
+constexpr int kProfPoints = 14;   // 7 timestamps, 3 unused, 4 cycle counters
 
 cudaError_t launch_decode(int wfmt, int pfmt, const DecodeParams &p, cudaStream_t stream);
 int decode_max_blocks_per_sm(int wfmt, int pfmt, int d);
@@ -78,6 +83,8 @@ int decode_max_blocks_per_sm(int wfmt, int pfmt, int d);
 constexpr int kMaxRepackSrc = 4;
 cudaError_t repack_rows(uint8_t *dst, const int32_t *perm, int rows, int n_src,
                         const uint8_t *const *src, const int *row_bytes, cudaStream_t s);
+cudaError_t repack_v_blocks(const uint8_t *V, uint8_t *dst, const int32_t *grp_off, int S, int r,
+                            int d, int elem_bytes, cudaStream_t s);
 cudaError_t repack_bias(const float *src, float *dst, const int32_t *perm, int n, cudaStream_t s);
 cudaError_t repack_down_transpose(const uint8_t *w_down, uint8_t *dst, const int32_t *perm,
                                   int d, int F, int elem_bytes, cudaStream_t s);
