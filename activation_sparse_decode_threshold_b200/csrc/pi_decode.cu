@@ -196,6 +196,25 @@ __device__ __forceinline__ float warp_sum(float v)
     return v;
 }
 
+// Warp reduction of 32 values per lane in 31 shuffles: after it, lane L holds
+// the warp-wide sum of value L.  (At each stage a lane keeps one half of its
+// values, chosen by its lane bit, and adds the partner's copy of that half.)
+__device__ __forceinline__ float warp_transpose_sum32(float (&v)[32])
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 16, n = 32; o >= 1; o >>= 1, n >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+            const float send = upper ? v[i] : v[i + n / 2];
+            const float keep = upper ? v[i + n / 2] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+    return v[0];
+}
+
 __device__ __forceinline__ float act_h(int act, float g, float u)
 {
     const float gp = g > 0.f ? g : 0.f;
@@ -204,10 +223,10 @@ __device__ __forceinline__ float act_h(int act, float g, float u)
     return gp * (u > 0.f ? u : 0.f);       // dReLU
 }
 
-constexpr int kNB = 4;            // neurons per gather batch
 constexpr int kRA = 16;           // V rows per staging round at most
 constexpr int kMaxU = 4;          // U vectors per lane (rank <= 128 * EPV)
-constexpr int kRed = 2 * kNB > kRA ? 2 * kNB : kRA;
+constexpr int kRound = 16;        // neurons per gather round at most
+constexpr int kRed = 2 * kRound;  // values reduced per warp at most
 
 struct Smem {
     float red[2][kConsumerWarps][kRed];
@@ -220,6 +239,8 @@ struct Smem {
     int16_t nz[kMaxTopK * kMaxStrip];      // neurons with h != 0, same encoding
     float hz[kMaxTopK * kMaxStrip];        // their h (routing weight folded in)
     int nz_n;
+    float rsum[kRed];                      // CTA-wide dot products of a gather round
+    float rh[kRound];                      // h of each neuron of a gather round
     int route_e[kMaxTopK];
     float route_w[kMaxTopK];
     float inv_rms;
@@ -285,9 +306,11 @@ __device__ bool grid_sync(Smem *sm, const DecodeParams &p, unsigned &epoch, int 
 
 // Staging round: thread 0 has issued bulk copies onto sm->stage_bar; it waits
 // (bounded) and the whole CTA adopts its verdict.
-__device__ bool stage_wait(Smem *sm, const DecodeParams &p, uint32_t &par, int &bci)
+__device__ bool stage_wait(Smem *sm, const DecodeParams &p, uint32_t &par, int &bci,
+                           long long *cyc = nullptr)
 {
     if (threadIdx.x == 0) {
+        const long long c0 = clock64();
         bool ok = mbar_test(&sm->stage_bar, par);
         if (!ok) {
             const long long t0 = gtimer();
@@ -300,6 +323,7 @@ __device__ bool stage_wait(Smem *sm, const DecodeParams &p, uint32_t &par, int &
             }
         }
         st_vol(&sm->bc[bci], ok ? 1 : 0);
+        if (cyc) *cyc += clock64() - c0;
     }
     cta_sync();
     const bool ok = ld_vol(&sm->bc[bci]) != 0;
@@ -329,8 +353,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     constexpr int EPVW = Fm<WF>::EPV, EPVP = Fm<PF>::EPV, VBW = Fm<WF>::VB, VBP = Fm<PF>::VB;
     constexpr int MAXVW = (DMAX / EPVW + kThreads - 1) / kThreads;
     constexpr int MAXVP = (DMAX / EPVP + kThreads - 1) / kThreads;
-    // neurons per gather batch: fewer when a row takes several vectors per thread
-    constexpr int NB = MAXVW >= 2 ? kNB / 2 : kNB;
     // when both formats share the vector layout, x is cached once
     constexpr bool kSameX = (WF == PF);
     using VW = typename Fm<WF>::V;
@@ -395,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // all added in fixed point.  `from_partials`: r = r_old + sum of the
     // per-CTA partials of y in fixed CTA order; otherwise r is the input.
     // -----------------------------------------------------------------------
-    auto column_phase = [&](int li_in, bool from_partials, bool next_exists, int l_next) {
+    auto column_phase = [&](int li_in, bool from_partials, bool next_exists, int l_next, int prow) {
         const float *src = predict ? p.x_in : p.resid;
         long long *fx = p.fix + size_t(li_in & 1) * kFixStride;
         if (from_partials) {
@@ -409,15 +431,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     pv[j] = c < S ? __ldcg(reinterpret_cast<const float4 *>(p.partials + size_t(c) * d) + q)
                                   : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
+                float4 rv = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (lane == 0) rv = __ldcg(reinterpret_cast<const float4 *>(p.resid) + q);
                 float4 sacc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                 for (int j = 0; j < kMaxStrips / 32; ++j) {
                     sacc.x += pv[j].x; sacc.y += pv[j].y; sacc.z += pv[j].z; sacc.w += pv[j].w;
                 }
-                sacc.x = warp_sum(sacc.x); sacc.y = warp_sum(sacc.y);
-                sacc.z = warp_sum(sacc.z); sacc.w = warp_sum(sacc.w);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    sacc.x += __shfl_xor_sync(0xffffffffu, sacc.x, o);
+                    sacc.y += __shfl_xor_sync(0xffffffffu, sacc.y, o);
+                    sacc.z += __shfl_xor_sync(0xffffffffu, sacc.z, o);
+                    sacc.w += __shfl_xor_sync(0xffffffffu, sacc.w, o);
+                }
                 if (lane == 0) {
-                    float4 rv = __ldcg(reinterpret_cast<const float4 *>(p.resid) + q);
                     rv.x += sacc.x; rv.y += sacc.y; rv.z += sacc.z; rv.w += sacc.w;
                     __stcg(reinterpret_cast<float4 *>(p.resid) + q, rv);
                     *reinterpret_cast<float4 *>(sm.rsl + 4 * qq) = rv;
@@ -427,6 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             for (int j = tid; j < ncol; j += kThreads) sm.rsl[j] = __ldcg(src + c0 + j);
         }
         cta_sync();
+        if (prow >= 0) prof_put(p, prow, 7, gtimer());
         if (!predict && p.trace && li_in < l1 - l0)
             for (int j = tid; j < ncol; j += kThreads) __stcg(p.trace + size_t(li_in) * d + c0 + j, sm.rsl[j]);
         if (!next_exists) return;
@@ -441,16 +470,40 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             // t partial: row k of the V block dotted with this CTA's columns
             const uint8_t *vb = vblk(l_next);
             const int nv = vbrow / VBP;
-            for (int k = tid; k < r; k += kThreads) {
-                float a = 0.f;
-                const uint8_t *row = vb + size_t(k) * vbrow;
-                for (int v = 0; v < nv; ++v) {
-                    float w[EPVP];
-                    cvt<PF>(ldvec<PF>(row + v * VBP), w);
+            // rows k and k + 512 together; four vectors of each in flight
+            for (int k = tid; k < r && ncol > 0; k += 2 * kThreads) {
+                const bool two = k + kThreads < r;
+                const uint8_t *row0 = vb + size_t(k) * vbrow;
+                const uint8_t *row1 = vb + size_t(two ? k + kThreads : k) * vbrow;
+                float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+                for (int v0 = 0; v0 < nv; v0 += 4) {
+                    VP q0[4], q1[4];
 #pragma unroll
-                    for (int i = 0; i < EPVP; ++i) a = fmaf(w[i], sm.rsl[v * EPVP + i], a);
+                    for (int j = 0; j < 4; ++j) {
+                        if (v0 + j < nv) {
+                            q0[j] = ldvec<PF>(row0 + (v0 + j) * VBP);
+                            q1[j] = ldvec<PF>(row1 + (v0 + j) * VBP);
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        if (v0 + j < nv) {
+                            float w0[EPVP], w1[EPVP];
+                            cvt<PF>(q0[j], w0);
+                            cvt<PF>(q1[j], w1);
+#pragma unroll
+                            for (int i = 0; i < EPVP; i += 2) {
+                                const float x0 = sm.rsl[(v0 + j) * EPVP + i], x1 = sm.rsl[(v0 + j) * EPVP + i + 1];
+                                a0 = fmaf(w0[i], x0, a0);
+                                a1 = fmaf(w0[i + 1], x1, a1);
+                                b0 = fmaf(w1[i], x0, b0);
+                                b1 = fmaf(w1[i + 1], x1, b1);
+                            }
+                        }
+                    }
                 }
-                if (ncol > 0) fix_add(fx + k, a, kFixT);
+                fix_add(fx + k, a0 + a1, kFixT);
+                if (two) fix_add(fx + k + kThreads, b0 + b1, kFixT);
             }
         } else if (!predict) {
             // router logit partials: W_r[e, cols] . r[cols]
@@ -468,7 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 #define XP(i) (kSameX ? xw[(i)] : xp_own[(i)])
 
     // prologue: the first layer's input columns
-    column_phase(0, false, true, l0);
+    column_phase(0, false, true, l0, -1);
     long long cyc0 = 0;
     const bool started = grid_sync(&sm, p, epoch, bci, &cyc0);
 
@@ -512,8 +565,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
         if (!moe) {
             // t from the fixed-point column partials
-            for (int k = tid; k < r; k += kThreads)
-                sm.tsm[k] = float(double(__ldcg(fx + k)) * (1.0 / 4294967296.0)) * inv;
+            {
+                long long tq[kMaxRankTotal / kThreads];
+#pragma unroll
+                for (int j = 0; j < kMaxRankTotal / kThreads; ++j) {
+                    const int k = tid + kThreads * j;
+                    tq[j] = k < r ? __ldcg(fx + k) : 0;
+                }
+#pragma unroll
+                for (int j = 0; j < kMaxRankTotal / kThreads; ++j) {
+                    const int k = tid + kThreads * j;
+                    if (k < r) sm.tsm[k] = float(double(tq[j]) * (1.0 / 4294967296.0)) * inv;
+                }
+            }
             if (tid == 0) {
                 sm.route_e[0] = predict ? p.pred_expert : 0;
                 sm.route_e[1] = 0;
@@ -638,7 +702,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         {
             bool ok = true;
             for (int e = 0; e < ntop && ok; ++e) {
-                const float *te = sm.tsm + e * r;
+                // this lane's t values (the columns of its U vectors)
+                float tu[kMaxU * EPVP];
+#pragma unroll
+                for (int k = 0; k < kMaxU; ++k) {
+                    const int v = lane + 32 * k;
+#pragma unroll
+                    for (int i = 0; i < EPVP; i += 4) {
+                        float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (v < nvecU) q = *reinterpret_cast<const float4 *>(sm.tsm + e * r + v * EPVP + i);
+                        tu[k * EPVP + i] = q.x; tu[k * EPVP + i + 1] = q.y;
+                        tu[k * EPVP + i + 2] = q.z; tu[k * EPVP + i + 3] = q.w;
+                    }
+                }
                 for (int row0 = 0; row0 < ns && ok; row0 += ucap) {
                     const int n = min(ucap, ns - row0);
                     if (!(staged_early && row0 == 0)) {
@@ -646,33 +722,51 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     }
                     staged_early = false;
                     pending = true;
-                    if (!stage_wait(&sm, p, spar, bci)) { ok = false; break; }
+                    if (!stage_wait(&sm, p, spar, bci, &cyc_b)) { ok = false; break; }
                     pending = false;
-                    for (int rr = warp; rr < n; rr += kConsumerWarps) {
-                        const uint8_t *urow = stg + size_t(rr) * p.urow;
-                        float a = 0.f;
+                    // each warp takes rows warp, warp + 16, ...; four rows at a time,
+                    // each with its own accumulators, to keep the dependent FMA and
+                    // shuffle chains of different rows overlapped
+                    constexpr int kZR = 4;
+                    for (int rr0 = warp; rr0 < n; rr0 += kConsumerWarps * kZR) {
+                        float a[kZR][2];
 #pragma unroll
-                        for (int k = 0; k < kMaxU; ++k) {
-                            const int v = lane + 32 * k;
-                            if (v < nvecU) {
-                                float w[EPVP];
-                                cvt<PF>(*reinterpret_cast<const VP *>(urow + v * VBP), w);
+                        for (int j = 0; j < kZR; ++j) {
+                            a[j][0] = 0.f;
+                            a[j][1] = 0.f;
+                            const int rr = rr0 + j * kConsumerWarps;
+                            if (rr < n) {
+                                const uint8_t *urow = stg + size_t(rr) * p.urow;
 #pragma unroll
-                                for (int i = 0; i < EPVP; i += 4) {
-                                    const float4 tq = *reinterpret_cast<const float4 *>(te + v * EPVP + i);
-                                    a = fmaf(w[i], tq.x, a);
-                                    a = fmaf(w[i + 1], tq.y, a);
-                                    a = fmaf(w[i + 2], tq.z, a);
-                                    a = fmaf(w[i + 3], tq.w, a);
+                                for (int k = 0; k < kMaxU; ++k) {
+                                    const int v = lane + 32 * k;
+                                    if (v < nvecU) {
+                                        float w[EPVP];
+                                        cvt<PF>(*reinterpret_cast<const VP *>(urow + v * VBP), w);
+#pragma unroll
+                                        for (int i = 0; i < EPVP; ++i)
+                                            a[j][i & 1] = fmaf(w[i], tu[k * EPVP + i], a[j][i & 1]);
+                                    }
                                 }
                             }
                         }
-                        a = warp_sum(a);
+#pragma unroll
+                        for (int j = 0; j < kZR; ++j) a[j][0] += a[j][1];
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                            for (int j = 0; j < kZR; ++j) a[j][0] += __shfl_xor_sync(0xffffffffu, a[j][0], o);
                         if (lane == 0) {
-                            const int loc = row0 + rr;
-                            const float z = a - sm.cbuf[e][loc];
-                            sm.zbuf[e][loc] = z;
-                            if (predict && p.z_out) p.z_out[s0 + loc] = z;
+#pragma unroll
+                            for (int j = 0; j < kZR; ++j) {
+                                const int rr = rr0 + j * kConsumerWarps;
+                                if (rr < n) {
+                                    const int loc = row0 + rr;
+                                    const float z = a[j][0] - sm.cbuf[e][loc];
+                                    sm.zbuf[e][loc] = z;
+                                    if (predict && p.z_out) p.z_out[s0 + loc] = z;
+                                }
+                            }
                         }
                     }
                     cta_sync();   // the staging buffer is reused by the next round
@@ -680,6 +774,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             }
             if (!ok) break;
         }
+        prof_put(p, li, 9, gtimer());
         // compaction in ascending strip order: warp e builds expert slot e's list
         if (warp < ntop) {
             const int e = warp;
@@ -709,7 +804,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
         if (tid == 0) sm.nz_n = 0;
         cta_sync();
-        cyc_b = clock64() - cb0;
+        (void)cb0;
         prof_put(p, li, 2, gtimer());
 
         if (predict) {
@@ -729,172 +824,155 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
 
         // ---------------- gather rows of active neurons ----------------------
+        // Rounds of up to kRound neurons: one bulk-copy round brings their
+        // W_gate/W_up records (and, when speculative, their W_down rows) into
+        // shared memory; the dots of all of them are reduced at once.
         const long long cc0 = clock64();
         const int m0 = sm.lst_n[0];
         const int m = m0 + (ntop > 1 ? sm.lst_n[1] : 0);
         auto entry = [&](int j) -> int { return j < m0 ? sm.lst[j] : sm.lst[kMaxStrip + (j - m0)]; };
         const ExpertDev *exs[kMaxTopK] = {&p.ex[size_t(l) * p.E + sm.route_e[0]],
                                           &p.ex[size_t(l) * p.E + sm.route_e[ntop > 1 ? 1 : 0]]};
-        for (int j = tid; j < m; j += kThreads) {
+        const int per_n = p.gu_bytes + (p.spec_down ? p.wrow : 0);   // bytes per neuron in a round
+        const int cap_n = min(kRound, kStageBytes / per_n);
+        // rows beyond the first round, and the next layer's V block and
+        // biases, start moving towards L2 now
+        for (int j = cap_n + tid; j < m; j += kThreads) {
             const int en = entry(j), e = en >> 12, loc = en & 0xfff;
             prefetch_l2(exs[e]->Wgu + size_t(s0 + loc) * p.gu_bytes, uint32_t(p.gu_bytes));
             if (p.spec_down) prefetch_l2(exs[e]->Wd + size_t(s0 + loc) * p.wrow, uint32_t(p.wrow));
+        }
+        if (tid == kThreads - 1 && !moe && l + 1 < l1) {
+            if (ncol > 0) prefetch_l2(vblk(l + 1), uint32_t(r) * vbrow);
+            if (ns > 0) {
+                const int c_lo = s0 & ~3, c_hi = (s0 + ns + 3) & ~3;   // 16-byte aligned, padded
+                prefetch_l2(p.ex[size_t(l + 1) * p.E].c + c_lo, uint32_t(c_hi - c_lo) * 4);
+            }
         }
 
         float acc[MAXVW * EPVW];
 #pragma unroll
         for (int i = 0; i < MAXVW * EPVW; ++i) acc[i] = 0.f;
-
-        const int nbat = (m + NB - 1) / NB;
-        VW gv[NB][2][MAXVW];      // input records of the batch being loaded
-        VW dv[NB][MAXVW];         // W_down rows being accumulated
-
-        auto load_gu = [&](int bt) {
+        // acc += h * (a W_down row in shared memory)
+        auto axpy_smem = [&](const uint8_t *row, float h) {
 #pragma unroll
-            for (int n = 0; n < NB; ++n) {
-                const int j = bt * NB + n;
-                if (j < m) {
-                    const int en = entry(j), e = en >> 12, loc = en & 0xfff;
-                    const uint8_t *rec = exs[e]->Wgu + size_t(s0 + loc) * p.gu_bytes;
+            for (int k = 0; k < MAXVW; ++k) {
+                const int v = tid + kThreads * k;
+                if (v < nvecW) {
+                    float w[EPVW];
+                    cvt<WF>(*reinterpret_cast<const VW *>(row + v * VBW), w);
+                    float hs = h;
+                    if constexpr (WF == kI4) hs = h * __half2float(*reinterpret_cast<const __half *>(row + d / 2 + (v >> 1) * 2));
 #pragma unroll
-                    for (int k = 0; k < MAXVW; ++k) {
-                        const int v = tid + kThreads * k;
-                        if (v < nvecW) {
-                            gv[n][0][k] = ldvec<WF>(rec + v * VBW);
-                            if (p.gated) gv[n][1][k] = ldvec<WF>(rec + p.wrow + v * VBW);
-                        }
-                    }
+                    for (int i = 0; i < EPVW; ++i) acc[k * EPVW + i] = fmaf(hs, w[i], acc[k * EPVW + i]);
                 }
             }
         };
-        // dots of batch bt's records (in registers), reduced across the CTA;
-        // neurons with h != 0 are appended to sm.nz in list order
-        auto finish_gu = [&](int bt) {
-            float pg[NB], pu[NB];
+        // dot of a row in shared memory with this thread's x columns
+        auto dot_smem = [&](const uint8_t *row) -> float {
+            float a = 0.f;
 #pragma unroll
-            for (int n = 0; n < NB; ++n) {
-                pg[n] = 0.f;
-                pu[n] = 0.f;
-                const int j = bt * NB + n;
-                if (j < m) {
-                    const int en = entry(j), e = en >> 12, loc = en & 0xfff;
-                    const uint8_t *rec = exs[e]->Wgu + size_t(s0 + loc) * p.gu_bytes;
+            for (int k = 0; k < MAXVW; ++k) {
+                const int v = tid + kThreads * k;
+                if (v < nvecW) {
+                    float w[EPVW];
+                    cvt<WF>(*reinterpret_cast<const VW *>(row + v * VBW), w);
+                    float c = 0.f;
 #pragma unroll
-                    for (int k = 0; k < MAXVW; ++k) {
-                        const int v = tid + kThreads * k;
-                        if (v < nvecW) {
-                            float w[EPVW];
-                            float a = 0.f;
-                            cvt<WF>(gv[n][0][k], w);
-#pragma unroll
-                            for (int i = 0; i < EPVW; ++i) a = fmaf(w[i], xw[k * EPVW + i], a);
-                            if constexpr (WF == kI4) a *= i4_scale(rec, d, v);
-                            pg[n] += a;
-                            if (p.gated) {
-                                float c = 0.f;
-                                cvt<WF>(gv[n][1][k], w);
-#pragma unroll
-                                for (int i = 0; i < EPVW; ++i) c = fmaf(w[i], xw[k * EPVW + i], c);
-                                if constexpr (WF == kI4) c *= i4_scale(rec + p.wrow, d, v);
-                                pu[n] += c;
-                            }
-                        }
-                    }
+                    for (int i = 0; i < EPVW; ++i) c = fmaf(w[i], xw[k * EPVW + i], c);
+                    if constexpr (WF == kI4) c *= __half2float(*reinterpret_cast<const __half *>(row + d / 2 + (v >> 1) * 2));
+                    a += c;
                 }
             }
-#pragma unroll
-            for (int n = 0; n < NB; ++n) {
-                const float a = warp_sum(pg[n]);
-                const float c = warp_sum(pu[n]);
-                if (lane == 0) {
-                    sm.red[rb][warp][2 * n] = a;
-                    sm.red[rb][warp][2 * n + 1] = c;
+            return a;
+        };
+
+        bool gok = true;
+        int nz_total = 0;            // neurons with h != 0 so far (list order)
+        for (int j0 = 0; j0 < m && gok; j0 += cap_n) {
+            const int k = min(cap_n, m - j0);
+            if (warp == 0) {
+                // lane 0 announces the round's bytes, then lane n copies neuron n
+                if (lane == 0) mbar_arrive_tx(&sm.stage_bar, uint32_t(k) * per_n);
+                __syncwarp();
+                if (lane < k) {
+                    const int en = entry(j0 + lane), e = en >> 12, loc = en & 0xfff;
+                    uint8_t *slot = stg + size_t(lane) * per_n;
+                    stage_copy(slot, exs[e]->Wgu + size_t(s0 + loc) * p.gu_bytes, uint32_t(p.gu_bytes),
+                               &sm.stage_bar);
+                    if (p.spec_down)
+                        stage_copy(slot + p.gu_bytes, exs[e]->Wd + size_t(s0 + loc) * p.wrow, uint32_t(p.wrow),
+                                   &sm.stage_bar);
                 }
             }
+            pending = true;
+            if (!stage_wait(&sm, p, spar, bci, &cyc_c)) { gok = false; break; }
+            pending = false;
+            // dots of every neuron of the round: values 2n (gate) and 2n + 1 (up)
+            float v[32];
+#pragma unroll
+            for (int n = 0; n < kRound; ++n) {
+                v[2 * n] = 0.f;
+                v[2 * n + 1] = 0.f;
+                if (n < k) {
+                    const uint8_t *slot = stg + size_t(n) * per_n;
+                    v[2 * n] = dot_smem(slot);
+                    if (p.gated) v[2 * n + 1] = dot_smem(slot + p.wrow);
+                }
+            }
+            const float ws = warp_transpose_sum32(v);
+            if (lane < 2 * k) sm.red[rb][warp][lane] = ws;
             cta_sync();
-            if (tid == 0) {
-                int nzn = sm.nz_n;
-                for (int n = 0; n < NB; ++n) {
-                    const int j = bt * NB + n;
-                    if (j >= m) break;
-                    float G = 0.f, Uv = 0.f;
-                    for (int w = 0; w < kConsumerWarps; ++w) {
-                        G += sm.red[rb][w][2 * n];
-                        Uv += sm.red[rb][w][2 * n + 1];
-                    }
-                    const int en = entry(j), e = en >> 12, loc = en & 0xfff;
-                    const float h = act_h(p.act, G - sm.cbuf[e][loc], Uv) * sm.route_w[e];
-                    if (h != 0.f) {
-                        sm.nz[nzn] = int16_t(en);
-                        sm.hz[nzn] = h;
-                        ++nzn;
-                    }
-                }
-                sm.nz_n = nzn;
+            if (tid < 2 * k) {
+                float a = 0.f;
+                for (int w = 0; w < kConsumerWarps; ++w) a += sm.red[rb][w][tid];
+                sm.rsum[tid] = a;
             }
-            cta_sync();
             rb ^= 1;
-        };
-        auto load_dn = [&](int q0, int q1) {
-#pragma unroll
-            for (int n = 0; n < NB; ++n) {
-                const int q = q0 + n;
-                if (q < q1) {
-                    const int en = sm.nz[q], e = en >> 12, loc = en & 0xfff;
-                    const uint8_t *row = exs[e]->Wd + size_t(s0 + loc) * p.wrow;
-#pragma unroll
-                    for (int k = 0; k < MAXVW; ++k) {
-                        const int v = tid + kThreads * k;
-                        if (v < nvecW) dv[n][k] = ldvec<WF>(row + v * VBW);
+            cta_sync();
+            if (tid < k) {
+                const int en = entry(j0 + tid), e = en >> 12, loc = en & 0xfff;
+                sm.rh[tid] = act_h(p.act, sm.rsum[2 * tid] - sm.cbuf[e][loc], sm.rsum[2 * tid + 1]) *
+                             sm.route_w[e];
+            }
+            cta_sync();
+            // neurons with h != 0, in list order
+            int nz_round = 0;
+            for (int n = 0; n < k; ++n) {
+                const float h = sm.rh[n];
+                if (h == 0.f) continue;
+                if (tid == 0) {
+                    sm.nz[nz_total + nz_round] = int16_t(entry(j0 + n));
+                    sm.hz[nz_total + nz_round] = h;
+                }
+                ++nz_round;
+                if (p.spec_down) axpy_smem(stg + size_t(n) * per_n + p.gu_bytes, h);
+            }
+            nz_total += nz_round;
+            cta_sync();   // the staging buffer is reused by the next round
+        }
+        // not speculative: the W_down rows of the neurons with h != 0, in rounds
+        if (gok && !p.spec_down) {
+            const int cap_d = min(kMaxTopK * kMaxStrip, kStageBytes / p.wrow);
+            for (int q0 = 0; q0 < nz_total && gok; q0 += cap_d) {
+                const int k = min(cap_d, nz_total - q0);
+                if (warp == 0) {
+                    if (lane == 0) mbar_arrive_tx(&sm.stage_bar, uint32_t(k) * p.wrow);
+                    __syncwarp();
+                    for (int n = lane; n < k; n += 32) {
+                        const int en = sm.nz[q0 + n], e = en >> 12, loc = en & 0xfff;
+                        stage_copy(stg + size_t(n) * p.wrow, exs[e]->Wd + size_t(s0 + loc) * p.wrow,
+                                   uint32_t(p.wrow), &sm.stage_bar);
                     }
                 }
+                pending = true;
+                if (!stage_wait(&sm, p, spar, bci, &cyc_c)) { gok = false; break; }
+                pending = false;
+                for (int n = 0; n < k; ++n) axpy_smem(stg + size_t(n) * p.wrow, sm.hz[q0 + n]);
+                cta_sync();
             }
-        };
-        auto axpy_dn = [&](int q0, int q1) {
-#pragma unroll
-            for (int n = 0; n < NB; ++n) {
-                const int q = q0 + n;
-                if (q < q1) {
-                    const int en = sm.nz[q], e = en >> 12, loc = en & 0xfff;
-                    const uint8_t *row = exs[e]->Wd + size_t(s0 + loc) * p.wrow;
-                    const float h = sm.hz[q];
-#pragma unroll
-                    for (int k = 0; k < MAXVW; ++k) {
-                        const int v = tid + kThreads * k;
-                        if (v < nvecW) {
-                            float w[EPVW];
-                            cvt<WF>(dv[n][k], w);
-                            float hs = h;
-                            if constexpr (WF == kI4) hs = h * i4_scale(row, d, v);
-#pragma unroll
-                            for (int i = 0; i < EPVW; ++i) acc[k * EPVW + i] = fmaf(hs, w[i], acc[k * EPVW + i]);
-                        }
-                    }
-                }
-            }
-        };
-
-        int dn_done = 0;   // entries of sm.nz already accumulated
-        if (nbat > 0) {
-            load_gu(0);
-            finish_gu(0);
         }
-        for (int bt = 0; bt < nbat; ++bt) {
-            // W_down rows found so far together with the records of batch bt + 1
-            const int dn_hi = min(sm.nz_n, dn_done + NB);
-            load_dn(dn_done, dn_hi);
-            if (bt + 1 < nbat) load_gu(bt + 1);
-            axpy_dn(dn_done, dn_hi);
-            dn_done = dn_hi;
-            if (bt + 1 < nbat) finish_gu(bt + 1);
-        }
-        const int nz_total = sm.nz_n;
-        while (dn_done < nz_total) {
-            const int dn_hi = min(nz_total, dn_done + NB);
-            load_dn(dn_done, dn_hi);
-            axpy_dn(dn_done, dn_hi);
-            dn_done = dn_hi;
-        }
+        if (!gok) break;
         if (tid == 0) {
             if (p.stats) atomicAdd(p.stats + li * 4 + 1, nz_total);
             // the next layer's predictor slice starts moving: U strip straight
@@ -906,7 +984,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                         prefetch_l2(p.ex[size_t(l + 1) * p.E].U + size_t(s0 + ucap) * p.urow,
                                     uint32_t(ns - ucap) * p.urow);
                 }
-                if (ncol > 0) prefetch_l2(vblk(l + 1), uint32_t(r) * vbrow);
             }
         }
         staged_early = !moe && l + 1 < l1 && ns > 0;
@@ -929,14 +1006,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                                        acc[k * EPVW + i + 2], acc[k * EPVW + i + 3]));
             }
         }
-        cyc_c = clock64() - cc0;
+        (void)cc0;
         prof_put(p, li, 3, gtimer());
         if (!grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
         prof_put(p, li, 4, gtimer());
 
         // ---------------- reduction + next layer's column products -----------
         const bool next = l + 1 < l1;
-        column_phase(li + 1, true, next, l + 1);
+        column_phase(li + 1, true, next, l + 1, li);
         prof_put(p, li, 5, gtimer());
         if (next && !grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
         prof_put(p, li, 6, gtimer());
