@@ -69,6 +69,7 @@ def lib() -> ctypes.CDLL:
             "pi_sync": [vp, vp],
             "pi_debug_set": [vp, ip, ctypes.c_double],
             "pi_debug_phase_times": [vp, vp],
+            "pi_predict_noalloc": [ip, ip, ip, ip, ctypes.c_float, vp, vp, vp, vp, vp, vp, vp, vp],
         }
         for name, args in sigs.items():
             f = getattr(L, name)
@@ -200,3 +201,11 @@ def pi_debug_set(h, flags: int, wait_limit_s: float):
 
 def pi_debug_phase_times(h, times=None):
     _check(lib().pi_debug_phase_times(h, _ptr(times)), "pi_debug_phase_times")
+
+
+def pi_predict_noalloc(d_model, d_ff, rank, pred_dtype, threshold, V, U, bias, x, idx, count, z=None,
+                       stream=None):
+    """Predictor on caller-owned weights (original order) with no device allocation."""
+    _check(lib().pi_predict_noalloc(d_model, d_ff, rank, DTYPE[pred_dtype], threshold, _ptr(V), _ptr(U),
+                                    _ptr(bias), _ptr(x), _ptr(idx), _ptr(count), _ptr(z), _stream(stream)),
+           "pi_predict_noalloc")

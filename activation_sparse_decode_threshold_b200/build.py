@@ -15,7 +15,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libpi_ffn.so")
 OBJ = os.path.join(ROOT, "_build")
-SOURCES = ["pi_host.cu", "pi_decode.cu", "pi_repack.cu", "pi_prefill.cu"]
+SOURCES = ["pi_host.cu", "pi_decode.cu", "pi_repack.cu", "pi_prefill.cu", "pi_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-Xcompiler", "-fvisibility=hidden"]

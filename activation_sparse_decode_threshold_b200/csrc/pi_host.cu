@@ -61,6 +61,11 @@ size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
+void pi::set_last_error(const char *msg)
+{
+    snprintf(g_msg, sizeof g_msg, "%s", msg);
+}
+
 struct pi_ffn {
     pi_ffn_desc desc{};
     int S = 0;                       // strips = CTAs of the decode kernel

@@ -89,6 +89,9 @@ cudaError_t repack_bias(const float *src, float *dst, const int32_t *perm, int n
 cudaError_t repack_down_transpose(const uint8_t *w_down, uint8_t *dst, const int32_t *perm,
                                   int d, int F, int elem_bytes, cudaStream_t s);
 
+// Sets the message returned by pi_last_error on this host thread.
+void set_last_error(const char *msg);
+
 // Device error codes written into the error word.
 enum DevErr { kDevOk = 0, kDevTimeout = 1, kDevCheck = 2 };
 

@@ -215,6 +215,32 @@ PI_API pi_status pi_debug_set(pi_ffn_t h, int flags, double wait_limit_s);
  * hold (l1 - l0) * 14 * n_strips values.  NULL turns recording off. */
 PI_API pi_status pi_debug_phase_times(pi_ffn_t h, long long *times_dev);
 
+/* The low-rank predictor on caller-owned weights, with no device allocation
+ * (no counterpart in the pages: it exists for callers that cannot call
+ * cudaMalloc where they predict -- a serving loop whose device memory is fully
+ * committed at start-up, a host runtime that owns the allocator, or code with
+ * no pi_ffn handle, whose creation allocates).
+ *   V_dev r x d, U_dev F x r (row-major, ORIGINAL neuron order, pred_dtype),
+ *   bias_dev F floats, x_dev d floats (the layer input, already normalised);
+ *   V, U and x 16-byte aligned.  Outputs as pi_predict, with table position =
+ *   original index: idx_dev [F] active neurons ascending, count_dev [1],
+ *   z_dev [F] logits or NULL.
+ * Limits: d_model a multiple of 256, <= 8192 (<= 4096 for F32); rank as in
+ * pi_ffn_desc; d_ff <= 256 * min(SM count, 256); larger sizes return
+ * PI_ERR_INVALID_ARG.  Scratch: one file-scope __device__ array of about 300 KB
+ * that every device loading the library holds until exit.
+ * Runs on the current device.  Its first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) and must come before any
+ * stream capture on that device.  Every call shares the array and leaves its
+ * contents behind (each call clears what must start at zero), so calls that
+ * overlap on the GPU -- on two streams, or from two threads -- race and must
+ * not be issued.  *count_dev reads -1 if the kernel gave up on a bounded wait.
+ * Asynchronous on `stream`. */
+PI_API pi_status pi_predict_noalloc(int d_model, int d_ff, int rank, pi_dtype pred_dtype,
+                                    float threshold, const void *V_dev, const void *U_dev,
+                                    const float *bias_dev, const float *x_dev, int32_t *idx_dev,
+                                    int32_t *count_dev, float *z_dev, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
