@@ -575,6 +575,7 @@ pi_status pi_dense_ffn_prefill(pi_ffn_t h, int layer_begin, int layer_end, int n
     v.ex = h->h_ex.data();
     v.router = h->router_mem.data();
     v.perm = &h->perm;
+    v.err = h->err;
     char msg[256] = "";
     const int rc = pi::prefill_run(&h->prefill, v, layer_begin, layer_end, n_tokens, resid_dev,
                                    static_cast<cudaStream_t>(stream), msg, sizeof msg);

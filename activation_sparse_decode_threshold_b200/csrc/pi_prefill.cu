@@ -1,24 +1,700 @@
-// pi_prefill.cu -- dense multi-token prefill on the tensor cores.
+// pi_prefill.cu -- dense multi-token prefill on the sm_100a tensor cores.
+//
+// PowerInfer-2 runs prefill as large dense neuron clusters ("Neuron-cluster
+// heterogeneous computing", citnews.com.cn article): with many tokens almost
+// every neuron fires, so the FFN is a real dense contraction and goes to the
+// tensor cores.  Per layer:
+//
+//   k_norm_route   x = RMSNorm(r) per token (fp32), an fp16 copy for the MMA,
+//                  MoE router logits (fp32) and top-2 with renormalised weights
+//   k_sort         tokens grouped by expert (counting sort, ascending token
+//                  order inside each expert: deterministic)
+//   k_gemm<GU>     per expert: [tokens x d] x [d x 2F] -> gate and up for 128
+//                  neurons per CTA tile (their rows interleaved so one TMEM
+//                  column pair holds a neuron's g and u), activation fused in
+//                  the epilogue: H = act(g - c, u) (fp16)
+//   k_gemm<DOWN>   per expert: H [tokens x F] x W_down^T [F x d], split over
+//                  K into fp32 partials (W_down stored neuron-major is the
+//                  MN-major operand)
+//   k_combine      y = sum over the token's experts in ascending expert index
+//                  of w * (sum of the K-split partials, fixed order); r += y
+//
+// GEMM tiles: 128 x 256 x 64; operands are written into shared memory by the
+// CTA's threads in the canonical no-swizzle core-matrix layout (8 rows x 16
+// bytes per core matrix; INT4 weights are dequantised to fp16 on the way),
+// one elected thread issues tcgen05.mma (kind::f16, fp32 accumulators in
+// TMEM) four K=16 steps per stage, and tcgen05.commit on a per-stage
+// mbarrier frees the stage.  Three stages.  Every wait is bounded.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
 #include <cstdio>
+#include <cstring>
+#include <vector>
 
 #include "pi_prefill.h"
 
 namespace pi {
+namespace {
 
-struct PrefillState {
-    int dummy;
+constexpr int BM = 128, BN = 256, BK = 64, NSTAGE = 3;
+constexpr int kGemmThreads = 256;
+constexpr int kATileBytes = BM * BK * 2;          // 16 KB
+constexpr int kBTileBytes = BN * BK * 2;          // 32 KB
+constexpr int kStageBytes = kATileBytes + kBTileBytes;
+constexpr int kGemmSmem = NSTAGE * kStageBytes + 1024;
+constexpr int kSplitK = 4;                        // K splits of the down GEMM
+constexpr long long kWaitNs = 2000000000LL;
+
+enum GemmKind { kGU = 0, kDOWN = 1 };
+
+struct PrefillExpert {
+    const uint8_t *Wgu;   // F records of gu_bytes (gate row, then up row when gated)
+    const uint8_t *Wd;    // F rows of wrow bytes (W_down columns)
+    const float *c;       // F biases
 };
+
+struct GemmParams {
+    PrefillExpert ex[kMaxExperts];
+    int E, d, F, gated, act, wrow, gu_bytes;
+    const int32_t *e_off;     // [E + 1] first list position of each expert
+    const int32_t *e_tok;     // [2T] token of each list position
+    const void *X16;          // [T x d] normalised inputs (element type of the MMA)
+    void *H;                  // [2T x F] activations per list position (same type)
+    float *Ypart;             // [kSplitK x 2T x d] down partials
+    int rows_cap;             // 2T
+    int *err;
+};
+
+// ---------------------------------------------------------------------------
+// PTX helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t s2u(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t *b, unsigned count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(s2u(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint64_t *b, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(s2u(b)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ long long gtimer()
+{
+    long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// bounded wait; false (and the error word set) when it runs out
+__device__ bool mbar_wait(uint64_t *b, uint32_t parity, int *err)
+{
+    if (mbar_test(b, parity)) return true;
+    const long long t0 = gtimer();
+    for (unsigned it = 1;; ++it) {
+        if (mbar_test(b, parity)) return true;
+        if ((it & 15) == 0 && gtimer() - t0 > kWaitNs) {
+            atomicCAS(err, 0, int(kDevTimeout));
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, bool pred)
+{
+    const int n = pred ? 16 : 0;   // zero-fill when out of range
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(s2u(dst)), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// shared-memory matrix descriptor: canonical layout without swizzle; start,
+// leading (K direction) and stride (M/N direction) byte offsets in 16-byte
+// units; descriptor version 1
+__device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    uint64_t d = 0;
+    d |= uint64_t((saddr >> 4) & 0x3fff);
+    d |= uint64_t((lbo >> 4) & 0x3fff) << 16;
+    d |= uint64_t((sbo >> 4) & 0x3fff) << 32;
+    d |= uint64_t(1) << 46;
+    return d;
+}
+// instruction descriptor: f16 A and B, f32 accumulate, M = 128, N = 256
+__device__ __forceinline__ uint32_t make_idesc(bool b_mn_major, bool bf16)
+{
+    uint32_t i = 0;
+    i |= 1u << 4;                        // D format: f32
+    i |= (bf16 ? 1u : 0u) << 7;          // A: f16 / bf16
+    i |= (bf16 ? 1u : 0u) << 10;         // B: same type as A
+    i |= 0u << 15;                       // A K-major
+    i |= (b_mn_major ? 1u : 0u) << 16;   // B K-major / MN-major
+    i |= uint32_t(BN >> 3) << 17;
+    i |= uint32_t(BM >> 4) << 24;
+    return i;
+}
+__device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, bool acc)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc ? 1u : 0u)
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(s2u(bar)) : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v)
+{
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// byte offset of element (row, k) of a K-major tile with BK columns
+__device__ __forceinline__ uint32_t kmaj_off(int row, int kchunk)
+{
+    return uint32_t((row >> 3) * (BK / 8 * 128) + kchunk * 128 + (row & 7) * 16);
+}
+// byte offset of the 16-byte chunk holding n = 8*ng .. 8*ng+7 of k-row `k`
+// in an MN-major tile (core matrices: 8 k-rows x 8 n-values)
+__device__ __forceinline__ uint32_t mnmaj_off(int ng, int k)
+{
+    return uint32_t(ng * (BK / 8 * 128) + (k >> 3) * 128 + (k & 7) * 16);
+}
+
+// 16 INT4 weights (8 bytes of nibbles, one group scale) -> 16 fp16 values
+__device__ __forceinline__ void dequant16(uint2 q, float s, uint4 &lo, uint4 &hi)
+{
+    __half2 h[8];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const uint32_t w = i == 0 ? q.x : q.y;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float a = float(int((w >> (8 * j)) & 0xf) - 8) * s;
+            const float b = float(int((w >> (8 * j + 4)) & 0xf) - 8) * s;
+            h[4 * i + j] = __floats2half2_rn(a, b);
+        }
+    }
+    lo = *reinterpret_cast<uint4 *>(&h[0]);
+    hi = *reinterpret_cast<uint4 *>(&h[4]);
+}
+
+// ---------------------------------------------------------------------------
+// GEMM kernel
+// ---------------------------------------------------------------------------
+template <int W> struct Elem { using T = __half; };
+template <> struct Elem<1> { using T = __nv_bfloat16; };
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ __half from_f<__half>(float x) { return __float2half_rn(x); }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+template <int KIND, int W>
+__global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant__ GemmParams p)
+{
+    constexpr bool I4 = W == 2;
+    using AT = typename Elem<W>::T;
+    const AT *X16 = reinterpret_cast<const AT *>(p.X16);
+    AT *Hbuf = reinterpret_cast<AT *>(p.H);
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t bars[NSTAGE];
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int d = p.d, F = p.F;
+    // tile coordinates: blockIdx.x = N tile, blockIdx.y = M tile over all experts,
+    // blockIdx.z = K split (down GEMM)
+    int e = -1, mrow0 = 0;
+    {
+        int acc = 0;
+        for (int x = 0; x < p.E; ++x) {
+            const int cnt = p.e_off[x + 1] - p.e_off[x];
+            const int tiles = (cnt + BM - 1) / BM;
+            if (int(blockIdx.y) < acc + tiles) {
+                e = x;
+                mrow0 = p.e_off[x] + (int(blockIdx.y) - acc) * BM;
+                break;
+            }
+            acc += tiles;
+        }
+    }
+    if (e < 0) return;   // uniform: no tile for this CTA
+    const int mrow_end = p.e_off[e + 1];
+    const PrefillExpert ex = p.ex[e];
+    const int K = KIND == kGU ? d : F;
+    const int nk_all = K / BK;
+    const int ksplit = KIND == kGU ? 1 : kSplitK;
+    const int kt0 = int((long long)blockIdx.z * nk_all / ksplit), kt1 = int((long long)(blockIdx.z + 1) * nk_all / ksplit);
+    const int n0 = blockIdx.x * BN;   // GU: B-row 2j/2j+1 = gate/up of neuron n0/2 + j
+
+    if (tid == 0) {
+        for (int s = 0; s < NSTAGE; ++s) mbar_init(&bars[s], 1);
+        abort_sh = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(s2u(&tmem_base_sh)), "r"(BN) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = tmem_base_sh;
+
+    // ---- stage loader: A (activations, K-major) and B (weights) ------------
+    auto load_stage = [&](int kt, int s) {
+        uint8_t *A = smem + s * kStageBytes;
+        uint8_t *B = A + kATileBytes;
+        const int k0 = kt * BK;
+        // A: 128 rows x 8 chunks of 16 bytes
+        for (int c = tid; c < BM * (BK / 8); c += kGemmThreads) {
+            const int row = c >> 3, kc = c & 7;
+            const int lr = mrow0 + row;
+            const bool ok = lr < mrow_end;
+            const AT *src;
+            if (KIND == kGU) src = X16 + size_t(ok ? p.e_tok[lr] : 0) * d + k0 + kc * 8;
+            else src = Hbuf + size_t(ok ? lr : 0) * F + k0 + kc * 8;
+            cp_async16(A + kmaj_off(row, kc), src, ok);
+        }
+        if constexpr (KIND == kGU) {
+            // B: 256 rows (neuron n0/2 + row/2; gate for even rows, up for odd) x 64 k, K-major
+            if constexpr (!I4) {
+                for (int c = tid; c < BN * (BK / 8); c += kGemmThreads) {
+                    const int row = c >> 3, kc = c & 7;
+                    const int nn = n0 / 2 + (row >> 1);
+                    const bool ok = nn < F && (p.gated || (row & 1) == 0);
+                    const uint8_t *rec = ex.Wgu + size_t(ok ? nn : 0) * p.gu_bytes + ((row & 1) ? p.wrow : 0);
+                    cp_async16(B + kmaj_off(row, kc), rec + (k0 + kc * 8) * 2, ok);
+                }
+            } else {
+                // one thread per (row, 16-element half of the 64-wide stage)... 4 per row
+                for (int c = tid; c < BN * 4; c += kGemmThreads) {
+                    const int row = c >> 2, q16 = c & 3;       // elements k0 + 16 q16 .. +15
+                    const int nn = n0 / 2 + (row >> 1);
+                    const bool ok = nn < F && (p.gated || (row & 1) == 0);
+                    uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
+                    if (ok) {
+                        const uint8_t *rec = ex.Wgu + size_t(nn) * p.gu_bytes + ((row & 1) ? p.wrow : 0);
+                        const int kk = k0 + 16 * q16;
+                        const uint2 q = *reinterpret_cast<const uint2 *>(rec + kk / 2);
+                        const float sc = __half2float(*reinterpret_cast<const __half *>(rec + d / 2 + (kk / 32) * 2));
+                        dequant16(q, sc, lo, hi);
+                    }
+                    *reinterpret_cast<uint4 *>(B + kmaj_off(row, 2 * q16)) = lo;
+                    *reinterpret_cast<uint4 *>(B + kmaj_off(row, 2 * q16 + 1)) = hi;
+                }
+            }
+        } else {
+            // B (down): n = output column j in [n0, n0 + 256), k = neuron i in [k0, k0 + 64):
+            // W_down neuron-major rows give 8 consecutive n per 16 bytes (MN-major)
+            if constexpr (!I4) {
+                for (int c = tid; c < BK * (BN / 8); c += kGemmThreads) {
+                    const int k = c / (BN / 8), ng = c % (BN / 8);
+                    const uint8_t *row = ex.Wd + size_t(k0 + k) * p.wrow + (n0 + ng * 8) * 2;
+                    cp_async16(B + mnmaj_off(ng, k), row, true);
+                }
+            } else {
+                for (int c = tid; c < BK * (BN / 16); c += kGemmThreads) {
+                    const int k = c / (BN / 16), g16 = c % (BN / 16);   // 16 n-values
+                    const uint8_t *row = ex.Wd + size_t(k0 + k) * p.wrow;
+                    const int nn = n0 + 16 * g16;
+                    const uint2 q = *reinterpret_cast<const uint2 *>(row + nn / 2);
+                    const float sc = __half2float(*reinterpret_cast<const __half *>(row + d / 2 + (nn / 32) * 2));
+                    uint4 lo, hi;
+                    dequant16(q, sc, lo, hi);
+                    *reinterpret_cast<uint4 *>(B + mnmaj_off(2 * g16, k)) = lo;
+                    *reinterpret_cast<uint4 *>(B + mnmaj_off(2 * g16 + 1, k)) = hi;
+                }
+            }
+        }
+        cp_async_commit();
+    };
+
+    const uint32_t idesc = make_idesc(KIND == kDOWN, W == 1);
+    const int nk = kt1 - kt0;
+    bool ok = true;
+    int j_issued = 0;   // last step whose MMAs were issued and committed
+    // prologue: stages 0 and 1 in flight
+    for (int j = 0; j < 2 && j < nk; ++j) load_stage(kt0 + j, j);
+    for (int j = 0; j < nk; ++j) {
+        const int s = j % NSTAGE;
+        if (j + 1 < nk) cp_async_wait<1>();
+        else cp_async_wait<0>();
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncthreads();
+        if (tid == 0) {
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const uint32_t a0 = s2u(smem + s * kStageBytes), b0 = a0 + kATileBytes;
+#pragma unroll
+            for (int ks = 0; ks < BK / 16; ++ks) {
+                const uint64_t ad = make_sdesc(a0 + ks * 256, 128, BK / 8 * 128);
+                const uint64_t bd = make_sdesc(b0 + ks * 256, 128, BK / 8 * 128);
+                umma(tmem, ad, bd, idesc, j > 0 || ks > 0);
+            }
+            umma_commit(&bars[s]);
+        }
+        j_issued = j;
+        // refill the stage freed by the MMAs of step j - 1
+        if (j + 2 < nk) {
+            const int sn = (j + 2) % NSTAGE;
+            if (j + 2 >= NSTAGE) {
+                // that stage was last read by the MMAs of step j + 2 - NSTAGE
+                const uint32_t par = uint32_t(((j + 2 - NSTAGE) / NSTAGE) & 1);
+                if (tid == 0 && !mbar_wait(&bars[sn], par, p.err)) abort_sh = 1;
+                __syncthreads();
+                if (abort_sh) { ok = false; break; }
+            }
+            load_stage(kt0 + j + 2, sn);
+        }
+    }
+    // all MMAs done: the last commit covers every earlier MMA of this thread.
+    // After a timed-out wait this is the (again bounded) drain of the MMAs in
+    // flight before TMEM is released.
+    cp_async_wait<0>();
+    if (nk > 0 && tid == 0) {
+        const int last = ok ? nk - 1 : j_issued;
+        if (!mbar_wait(&bars[last % NSTAGE], uint32_t((last / NSTAGE) & 1), p.err)) abort_sh = 1;
+    }
+    __syncthreads();
+    ok = ok && !abort_sh;
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+
+    // ---- epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31, columns half (w / 4)
+    if (ok && nk > 0) {
+        const int row = 32 * (warp & 3) + lane;
+        const int lr = mrow0 + row;
+        const bool valid = lr < mrow_end;
+        const int col0 = 128 * (warp >> 2);
+        for (int cc = 0; cc < 128; cc += 16) {
+            float v[16];
+            tmem_ld16(tmem + (uint32_t(32 * (warp & 3)) << 16) + uint32_t(col0 + cc), v);
+            if (!valid) continue;
+            if constexpr (KIND == kGU) {
+                // columns 2j, 2j+1 = gate, up of neuron n0/2 + (col0 + cc)/2 + j
+                const int nb = n0 / 2 + (col0 + cc) / 2;
+                AT hv[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int nn = nb + j;
+                    float g = v[2 * j] - (nn < F ? __ldg(ex.c + nn) : 0.f);
+                    float u = v[2 * j + 1];
+                    const float gp = g > 0.f ? g : 0.f;
+                    float h = p.act == 0 ? gp : (p.act == 1 ? gp * u : gp * (u > 0.f ? u : 0.f));
+                    hv[j] = from_f<AT>(h);
+                }
+                if (nb + 8 <= F)
+                    *reinterpret_cast<uint4 *>(Hbuf + size_t(lr) * F + nb) = *reinterpret_cast<uint4 *>(hv);
+            } else {
+                float *dst = p.Ypart + (size_t(blockIdx.z) * p.rows_cap + lr) * d + n0 + col0 + cc;
+#pragma unroll
+                for (int j = 0; j < 16; j += 4)
+                    *reinterpret_cast<float4 *>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+            }
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BN) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Per-token kernels
+// ---------------------------------------------------------------------------
+struct TokenParams {
+    float *resid;             // [T x d]
+    void *X16;                // [T x d], fp16 or bf16 (x_bf16)
+    int x_bf16;
+    const __half *router;     // [E x d] or null
+    int d, E, T, top_k;
+    float eps;
+    int32_t *route_e;         // [T x 2]
+    float *route_w;           // [T x 2]
+    int32_t *e_off;           // [E + 1]
+    int32_t *e_tok;           // [2T]
+    int32_t *pos;             // [T x 2] list position of (token, k)
+    const float *Ypart;       // [kSplitK x 2T x d]
+    int rows_cap;
+};
+
+__global__ void k_norm_route(TokenParams p)
+{
+    const int t = blockIdx.x, tid = threadIdx.x;
+    const float *r = p.resid + size_t(t) * p.d;
+    __shared__ float red[32];
+    __shared__ float lg[kMaxExperts];
+    float ss = 0.f;
+    for (int j = tid; j < p.d; j += blockDim.x) ss = fmaf(r[j], r[j], ss);
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if ((tid & 31) == 0) red[tid >> 5] = ss;
+    __syncthreads();
+    if (tid == 0) {
+        float a = 0.f;
+        for (int w = 0; w < int(blockDim.x >> 5); ++w) a += red[w];
+        red[31] = 1.f / sqrtf(a / float(p.d) + p.eps);
+    }
+    __syncthreads();
+    const float inv = red[31];
+    for (int j = tid; j < p.d; j += blockDim.x) {
+        if (p.x_bf16) reinterpret_cast<__nv_bfloat16 *>(p.X16)[size_t(t) * p.d + j] = __float2bfloat16_rn(r[j] * inv);
+        else reinterpret_cast<__half *>(p.X16)[size_t(t) * p.d + j] = __float2half_rn(r[j] * inv);
+    }
+    if (p.E > 1) {
+        // router logits in fp32 from the fp32 input
+        for (int e = 0; e < p.E; ++e) {
+            float a = 0.f;
+            for (int j = tid; j < p.d; j += blockDim.x)
+                a = fmaf(__half2float(p.router[size_t(e) * p.d + j]), r[j] * inv, a);
+            for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+            __syncthreads();
+            if ((tid & 31) == 0) red[tid >> 5] = a;
+            __syncthreads();
+            if (tid == 0) {
+                float s = 0.f;
+                for (int w = 0; w < int(blockDim.x >> 5); ++w) s += red[w];
+                lg[e] = s;
+            }
+        }
+        __syncthreads();
+        if (tid == 0) {
+            float mx = -INFINITY, pr[kMaxExperts], den = 0.f;
+            for (int e = 0; e < p.E; ++e) mx = fmaxf(mx, lg[e]);
+            for (int e = 0; e < p.E; ++e) { pr[e] = expf(lg[e] - mx); den += pr[e]; }
+            for (int e = 0; e < p.E; ++e) pr[e] /= den;
+            int ea = 0;
+            for (int e = 1; e < p.E; ++e) if (pr[e] > pr[ea]) ea = e;
+            int eb = ea == 0 ? 1 : 0;
+            for (int e = 0; e < p.E; ++e) if (e != ea && pr[e] > pr[eb]) eb = e;
+            const int lo = min(ea, eb), hi = max(ea, eb);
+            p.route_e[2 * t] = lo;
+            p.route_e[2 * t + 1] = hi;
+            p.route_w[2 * t] = pr[lo] / (pr[lo] + pr[hi]);
+            p.route_w[2 * t + 1] = pr[hi] / (pr[lo] + pr[hi]);
+        }
+    } else if (tid == 0) {
+        p.route_e[2 * t] = 0;
+        p.route_e[2 * t + 1] = -1;
+        p.route_w[2 * t] = 1.f;
+        p.route_w[2 * t + 1] = 0.f;
+    }
+}
+
+// Counting sort of the (token, slot) items by expert, items taken in
+// ascending (token, slot) order so each expert's list is in ascending token
+// order: deterministic.  One CTA of 1024 threads; per chunk of 1024 items,
+// warp ballots give each item its rank among the chunk's items of the same
+// expert before it.
+constexpr int kSortThreads = 1024;
+__global__ void __launch_bounds__(kSortThreads) k_sort(TokenParams p)
+{
+    __shared__ int tot[kMaxExperts];
+    __shared__ int base[kMaxExperts];
+    __shared__ int wcnt[kSortThreads / 32][kMaxExperts];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n = p.T * p.top_k;
+    if (tid < kMaxExperts) tot[tid] = 0;
+    __syncthreads();
+    for (int i = tid; i < n; i += kSortThreads) atomicAdd(&tot[p.route_e[2 * (i / p.top_k) + i % p.top_k]], 1);
+    __syncthreads();
+    if (tid == 0) {
+        int acc = 0;
+        for (int e = 0; e < p.E; ++e) {
+            p.e_off[e] = acc;
+            base[e] = acc;
+            acc += tot[e];
+        }
+        p.e_off[p.E] = acc;
+    }
+    __syncthreads();
+    const unsigned lt = (1u << lane) - 1u;
+    for (int c0 = 0; c0 < n; c0 += kSortThreads) {
+        const int i = c0 + tid;
+        const int t = i / p.top_k, k = i % p.top_k;
+        const int e = i < n ? p.route_e[2 * t + k] : -1;
+        int rank = 0;
+        for (int x = 0; x < p.E; ++x) {
+            const unsigned m = __ballot_sync(0xffffffffu, e == x);
+            if (e == x) rank = __popc(m & lt);
+            if (lane == 0) wcnt[warp][x] = __popc(m);
+        }
+        __syncthreads();
+        if (e >= 0) {
+            int q = base[e] + rank;
+            for (int w = 0; w < warp; ++w) q += wcnt[w][e];
+            p.e_tok[q] = t;
+            p.pos[2 * t + k] = q;
+        }
+        __syncthreads();
+        if (tid < p.E) {
+            int s = 0;
+            for (int w = 0; w < kSortThreads / 32; ++w) s += wcnt[w][tid];
+            base[tid] += s;
+        }
+        __syncthreads();
+    }
+}
+
+// r += sum over the token's experts (ascending index) of w * (sum of the
+// K-split partials in split order)
+__global__ void k_combine(TokenParams p)
+{
+    const int t = blockIdx.x;
+    for (int j = threadIdx.x; j < p.d; j += blockDim.x) {
+        float y = 0.f;
+        for (int k = 0; k < p.top_k; ++k) {
+            const int q = p.pos[2 * t + k];
+            float s = 0.f;
+            for (int sp = 0; sp < kSplitK; ++sp) s += p.Ypart[(size_t(sp) * p.rows_cap + q) * p.d + j];
+            y = fmaf(p.route_w[2 * t + k], s, y);
+        }
+        p.resid[size_t(t) * p.d + j] += y;
+    }
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Host
+// ---------------------------------------------------------------------------
+struct PrefillState {
+    int T = 0, d = 0, F = 0;
+    uint8_t *buf = nullptr;
+    size_t bytes = 0;
+};
+
+static size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
 int prefill_run(PrefillState **state, const PrefillView &v, int l0, int l1, int T, float *resid,
                 cudaStream_t stream, char *msg, int msg_len)
 {
-    (void)state; (void)v; (void)l0; (void)l1; (void)T; (void)resid; (void)stream;
-    snprintf(msg, msg_len, "dense prefill is not available in this build");
-    return 1;
+    if (v.wfmt != kF16 && v.wfmt != kBF16 && v.wfmt != kI4) {
+        snprintf(msg, msg_len, "dense prefill supports F16, BF16 and INT4G32 weights");
+        return 1;
+    }
+    if (v.d % BN != 0 || v.F % (BN / 2) != 0 || v.F % BK != 0 || v.d % BK != 0) {
+        snprintf(msg, msg_len, "dense prefill needs d_model %% 256 == 0 and d_ff %% 128 == 0");
+        return 1;
+    }
+    const int rows_cap = 2 * T;
+    const size_t o_x16 = 0;
+    const size_t o_h = up256(o_x16 + sizeof(__half) * size_t(T) * v.d);
+    const size_t o_y = up256(o_h + sizeof(__half) * size_t(rows_cap) * v.F);
+    const size_t o_re = up256(o_y + sizeof(float) * size_t(kSplitK) * rows_cap * v.d);
+    const size_t o_rw = up256(o_re + sizeof(int32_t) * 2 * T);
+    const size_t o_eo = up256(o_rw + sizeof(float) * 2 * T);
+    const size_t o_et = up256(o_eo + sizeof(int32_t) * (kMaxExperts + 1));
+    const size_t o_pos = up256(o_et + sizeof(int32_t) * rows_cap);
+    const size_t total = up256(o_pos + sizeof(int32_t) * 2 * T);
+    PrefillState *st = *state;
+    if (!st || st->bytes < total) {
+        if (st) cudaFree(st->buf);
+        if (!st) st = new PrefillState;
+        *state = st;
+        st->buf = nullptr;
+        st->bytes = 0;
+        if (cudaMalloc(&st->buf, total) != cudaSuccess) {
+            snprintf(msg, msg_len, "prefill workspace allocation of %zu bytes failed", total);
+            return 3;
+        }
+        st->bytes = total;
+    }
+    uint8_t *B = st->buf;
+    // element type of the MMA operands: 0 f16, 1 bf16, 2 INT4 dequantised to f16
+    const int W = v.wfmt == kBF16 ? 1 : (v.wfmt == kI4 ? 2 : 0);
+    void (*gu)(GemmParams) = W == 0 ? k_gemm<kGU, 0> : (W == 1 ? k_gemm<kGU, 1> : k_gemm<kGU, 2>);
+    void (*dn)(GemmParams) = W == 0 ? k_gemm<kDOWN, 0> : (W == 1 ? k_gemm<kDOWN, 1> : k_gemm<kDOWN, 2>);
+    // per device and kernel; cheap enough to repeat per call
+    if (cudaFuncSetAttribute(gu, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) != cudaSuccess ||
+        cudaFuncSetAttribute(dn, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) != cudaSuccess) {
+        snprintf(msg, msg_len, "prefill: cudaFuncSetAttribute: %s", cudaGetErrorString(cudaGetLastError()));
+        return 2;
+    }
+
+    TokenParams tp{};
+    tp.resid = resid;
+    tp.X16 = B + o_x16;
+    tp.x_bf16 = W == 1;
+    tp.d = v.d;
+    tp.E = v.E;
+    tp.T = T;
+    tp.top_k = v.top_k;
+    tp.eps = v.eps;
+    tp.route_e = reinterpret_cast<int32_t *>(B + o_re);
+    tp.route_w = reinterpret_cast<float *>(B + o_rw);
+    tp.e_off = reinterpret_cast<int32_t *>(B + o_eo);
+    tp.e_tok = reinterpret_cast<int32_t *>(B + o_et);
+    tp.pos = reinterpret_cast<int32_t *>(B + o_pos);
+    tp.Ypart = reinterpret_cast<const float *>(B + o_y);
+    tp.rows_cap = rows_cap;
+
+    GemmParams gp{};
+    gp.E = v.E;
+    gp.d = v.d;
+    gp.F = v.F;
+    gp.gated = v.gated;
+    gp.act = v.act;
+    gp.wrow = v.wrow;
+    gp.gu_bytes = (v.gated ? 2 : 1) * v.wrow;
+    gp.e_off = tp.e_off;
+    gp.e_tok = tp.e_tok;
+    gp.X16 = tp.X16;
+    gp.H = B + o_h;
+    gp.Ypart = reinterpret_cast<float *>(B + o_y);
+    gp.rows_cap = rows_cap;
+    gp.err = v.err;
+    const int mtiles = (rows_cap + BM - 1) / BM + v.E;   // upper bound over experts
+
+    for (int l = l0; l < l1; ++l) {
+        tp.router = v.E > 1 ? reinterpret_cast<const __half *>(v.router[l]) : nullptr;
+        for (int e = 0; e < v.E; ++e) {
+            const ExpertDev &x = v.ex[size_t(l) * v.E + e];
+            gp.ex[e] = PrefillExpert{x.Wgu, x.Wd, x.c};
+        }
+        k_norm_route<<<T, 256, 0, stream>>>(tp);
+        k_sort<<<1, kSortThreads, 0, stream>>>(tp);
+        dim3 g1(2 * v.F / BN, mtiles, 1);
+        gu<<<g1, kGemmThreads, kGemmSmem, stream>>>(gp);
+        dim3 g2(v.d / BN, mtiles, kSplitK);
+        dn<<<g2, kGemmThreads, kGemmSmem, stream>>>(gp);
+        k_combine<<<T, 256, 0, stream>>>(tp);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) {
+            snprintf(msg, msg_len, "prefill launch: %s", cudaGetErrorString(e));
+            return 2;
+        }
+    }
+    return 0;
 }
 
 void prefill_invalidate(PrefillState *, int) {}
 
-void prefill_destroy(PrefillState *state) { delete state; }
+void prefill_destroy(PrefillState *state)
+{
+    if (!state) return;
+    cudaFree(state->buf);
+    delete state;
+}
 
 }  // namespace pi

@@ -17,6 +17,7 @@ struct PrefillView {
     const ExpertDev *ex;                        // host copy [n_layers * E]
     uint8_t *const *router;                     // host copy [n_layers] device pointers
     const std::vector<std::vector<int32_t>> *perm;
+    int *err;                                   // the handle's device error word
 };
 
 // Returns 0 on success, 1 unsupported, 2 CUDA error, 3 out of memory; `msg`

@@ -260,3 +260,43 @@ def decode_stack(r, layers: list, routers=None, threshold: float = 0.0):
         out.append(res)
         r = res.r_out
     return r, out
+
+
+@dataclass
+class PrefillResult:
+    x: np.ndarray            # T x d normalised inputs
+    y: np.ndarray            # T x d FFN outputs
+    r_out: np.ndarray        # T x d residual after the layer
+    experts: np.ndarray      # T x 2 experts used (-1 unused), ascending
+    weights: np.ndarray      # T x 2 their combine weights
+    logits: np.ndarray | None
+
+
+def prefill_layer(R, experts: list, router=None, eps: float = EPS) -> PrefillResult:
+    """One layer of dense multi-token prefill: every token row of R is
+    normalised, routed (MoE) and passed through the full FFN of its expert(s)
+    with no predictor (PowerInfer-2, "Neuron-cluster heterogeneous computing":
+    prefill activates almost every neuron and runs dense).  Rows are
+    independent; each is the decode layer with every neuron active."""
+    R = np.atleast_2d(_c(R, np.float64))
+    T, d = R.shape
+    X = np.empty_like(R)
+    Y = np.zeros_like(R)
+    used = np.full((T, 2), -1, np.int32)
+    wts = np.zeros((T, 2), np.float64)
+    L = None if router is None else np.empty((T, router.shape[0]), np.float64)
+    for t in range(T):
+        x = rmsnorm(R[t], eps)
+        X[t] = x
+        if router is None:
+            use, w = [0], [1.0]
+        else:
+            lg, ex, w2 = route_top2(x, router)
+            L[t] = lg
+            use, w = [int(ex[0]), int(ex[1])], [float(w2[0]), float(w2[1])]
+        for k, (e_id, w_e) in enumerate(zip(use, w)):
+            _, y_e = ffn_masked(experts[e_id], x, None)
+            Y[t] = y_e if router is None else Y[t] + w_e * y_e
+            used[t, k] = e_id
+            wts[t, k] = w_e
+    return PrefillResult(x=X, y=Y, r_out=R + Y, experts=used, weights=wts, logits=L)

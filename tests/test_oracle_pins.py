@@ -428,3 +428,57 @@ def test_stack_is_residual_composition(oracle_mod):
         assert np.allclose(res[l].x, x, rtol=1e-14, atol=1e-14)
         r = r + res[l].y
     assert np.allclose(r_final, r, rtol=1e-14, atol=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# Dense prefill (PowerInfer-2, "Neuron-cluster heterogeneous computing")
+# ---------------------------------------------------------------------------
+def test_prefill_equals_matrix_form(oracle_mod):
+    """T tokens through a dense ReGLU FFN equal the matrix form of the layer,
+    Y = (relu(X Wg^T - c) * (X Wu^T)) Wd^T with X the row-wise RMSNorm of R,
+    written with numpy matmuls."""
+    rng = np.random.default_rng(21)
+    T, d, F = 7, 16, 40
+    wg, wu = rng.standard_normal((F, d)), rng.standard_normal((F, d))
+    wd, c = rng.standard_normal((d, F)), rng.standard_normal(F)
+    e = expert_from(oracle_mod, "reglu", wg, wu, wd, c)
+    R = rng.standard_normal((T, d))
+    res = oracle_mod.prefill_layer(R, [e])
+    X = R / np.sqrt((R * R).mean(axis=1, keepdims=True) + 1e-6)
+    wg32, wu32, wd32, c32 = (f32(a).astype(np.float64) for a in (wg, wu, wd, c))
+    H = np.maximum(X @ wg32.T - c32, 0) * (X @ wu32.T)
+    assert np.allclose(res.x, X, rtol=1e-14, atol=1e-14)
+    assert np.allclose(res.y, H @ wd32.T, rtol=1e-12, atol=1e-12)
+    assert np.array_equal(res.r_out, R + res.y)
+
+
+def test_prefill_rows_are_decode_with_every_neuron_active(oracle_mod):
+    """Each prefill row is the decode layer of that token with threshold -inf
+    (every neuron active), for an INT4 dReLU MoE; routing per token."""
+    from activation_sparse_decode_threshold_b200.synth import quantize_int4_g32
+    rng = np.random.default_rng(22)
+    T, d, F, E = 5, 64, 32, 4
+    experts = []
+
+    def q4(shape):
+        q, s = quantize_int4_g32(torch.from_numpy(rng.standard_normal(shape).astype(np.float32)))
+        return q.numpy(), s.numpy()
+    for _ in range(E):
+        qg, sg = q4((F, d))
+        qu, su = q4((F, d))
+        qd, sd = q4((F, d))
+        experts.append(oracle_mod.Expert(
+            act="drelu", wdtype="int4g32", pdtype="f16", w_gate=qg, w_up=qu, w_down=qd,
+            c=f32(rng.standard_normal(F) * 0.1), U=rng.standard_normal((F, 8)).astype(np.float16),
+            V=rng.standard_normal((8, d)).astype(np.float16), s_gate=sg, s_up=su, s_down=sd))
+    router = rng.standard_normal((E, d)).astype(np.float16)
+    R = rng.standard_normal((T, d))
+    res = oracle_mod.prefill_layer(R, experts, router)
+    for t in range(T):
+        ref = oracle_mod.decode_layer(R[t], experts, router, threshold=-np.inf)
+        assert all(m.all() for m in ref.mask)
+        assert res.experts[t].tolist() == ref.experts
+        assert np.array_equal(res.y[t], ref.y)
+    # token order does not matter: a permutation of the rows permutes the results
+    p = rng.permutation(T)
+    assert np.array_equal(oracle_mod.prefill_layer(R[p], experts, router).y, res.y[p])
