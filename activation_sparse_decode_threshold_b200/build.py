@@ -15,7 +15,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libpi_ffn.so")
 OBJ = os.path.join(ROOT, "_build")
-SOURCES = ["pi_host.cu", "pi_decode.cu", "pi_repack.cu", "pi_prefill.cu", "pi_noalloc.cu"]
+SOURCES = ["pi_decode_f16.cu", "pi_decode_bf16.cu", "pi_decode_i4f16.cu", "pi_decode_i4bf16.cu",
+           "pi_decode_f32.cu", "pi_host.cu", "pi_decode.cu", "pi_repack.cu", "pi_prefill.cu", "pi_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-Xcompiler", "-fvisibility=hidden"]
@@ -64,7 +65,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed: {' '.join(cmd)}")
 
-    with ThreadPoolExecutor(max_workers=min(4, max(1, len(jobs)))) as ex:
+    with ThreadPoolExecutor(max_workers=min(os.cpu_count() or 4, max(1, len(jobs)))) as ex:
         list(ex.map(run, jobs))
     if force or jobs or not os.path.exists(OUT):
         cmd = [nvcc, *ARCH, "-shared", "-o", OUT + ".tmp", *objs, "-lcudart", "-lcuda"]

@@ -1,0 +1,1214 @@
+// pi_decode_kernel.cuh -- persistent sparse-FFN decode kernel for sm_100a.
+//
+// One cooperative launch runs a range of layers for one token.  Each CTA owns
+// one strip of the neuron table (a contiguous run of table positions holding
+// a balanced share of hot neurons, hottest first) and one slice of the d_model
+// columns.  Per layer l (dense FFN):
+//
+//   [B] t = V x (from the column phase below), x = RMSNorm(r);
+//       z = U t - c over the strip, active iff z > threshold, the active list
+//       compacted in ascending table order with warp ballots (PowerInfer
+//       (unite.ai), "Adaptive sparse predictor").
+//   [C] for active neurons only: the neuron's W_gate / W_up rows -> h =
+//       act(g, u); for h != 0 its W_down column (stored as a row) accumulates
+//       into a per-CTA fp32 partial of y ("Neuron-aware operators": rows of
+//       the input matrices, columns of the output matrix).
+//   --- grid barrier ---
+//   [column phase] r <- r + sum of the per-CTA partials, for this CTA's
+//       columns, in fixed CTA order (the merge of partial results, nearauto.com
+//       PowerInfer article, Fig. 8); then, for layer l + 1, this CTA's share of
+//       sum(r^2) and of t = V r (V stored column-blocked per CTA), added in
+//       64-bit fixed point so the totals do not depend on arrival order.
+//   --- grid barrier ---
+//
+// Two grid barriers per layer.  The MoE layer adds routing (from fixed-point
+// router logits, identical in every CTA), t computed by rows of the two
+// chosen experts, and a third barrier.
+//
+// Memory: weight bytes are pulled towards the SM as soon as their addresses
+// are known -- the next layer's U strip is bulk-copied straight into shared
+// memory when the gather ends (it lands during the barriers), its V block is
+// prefetched into L2, and a strip's active neuron records (plus, for ReLU /
+// ReGLU, where h != 0 almost always follows z > 0, their W_down rows) are
+// prefetched into L2 the moment the active list exists; the 16 warps read
+// them with batched 128-bit loads, the W_down rows of one batch together with
+// the W_gate/W_up records of the next.  All waits are bounded (%globaltimer);
+// a wait that runs out records an error word and every CTA returns.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#pragma once
+#include "pi_internal.h"
+
+namespace pi {
+namespace {
+
+// ---------------------------------------------------------------------------
+// PTX helpers
+// ---------------------------------------------------------------------------
+// Bulk prefetch of a global range into L2 (fire and forget), 32 KB pieces.
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes)
+{
+    const uint8_t *p = static_cast<const uint8_t *>(src);
+    for (uint32_t o = 0; o < bytes; o += 32768u) {
+        const uint32_t n = bytes - o < 32768u ? bytes - o : 32768u;
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p + o), "r"(n) : "memory");
+    }
+}
+// Read-only weight loads that do not allocate in L1.
+__device__ __forceinline__ uint4 ldw4(const uint8_t *p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint2 ldw2(const uint8_t *p)
+{
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint32_t s2u(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t *b, unsigned count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(s2u(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_tx(uint64_t *b, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(s2u(b)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint64_t *b, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(s2u(b)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// 1-D bulk copy global -> this CTA's shared memory, completion on `bar`.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(s2u(dst)), "l"(src), "r"(bytes), "r"(s2u(bar))
+        : "memory");
+}
+__device__ __forceinline__ long long gtimer()
+{
+    long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void cta_sync()
+{
+    asm volatile("bar.sync 0;" ::: "memory");
+}
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p)
+{
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void red_release_gpu(unsigned *p, unsigned v)
+{
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_vol(const int *p)
+{
+    return *reinterpret_cast<const volatile int *>(p);
+}
+__device__ __forceinline__ void st_vol(int *p, int v)
+{
+    *reinterpret_cast<volatile int *>(p) = v;
+}
+
+// ---------------------------------------------------------------------------
+// Stored formats.  A vector is 16 bytes of a row (8 bytes for INT4: 16
+// nibbles, half of a 32-element scale group).
+// ---------------------------------------------------------------------------
+template <int F> struct Fm;
+template <> struct Fm<kF32>  { static constexpr int VB = 16, EPV = 4;  using V = uint4; };
+template <> struct Fm<kF16>  { static constexpr int VB = 16, EPV = 8;  using V = uint4; };
+template <> struct Fm<kBF16> { static constexpr int VB = 16, EPV = 8;  using V = uint4; };
+template <> struct Fm<kI4>   { static constexpr int VB = 8,  EPV = 16; using V = uint2; };
+
+template <int F>
+__device__ __forceinline__ typename Fm<F>::V ldvec(const uint8_t *p)
+{
+    if constexpr (F == kI4) return ldw2(p);
+    else return ldw4(p);
+}
+
+template <int F>
+__device__ __forceinline__ void cvt(const typename Fm<F>::V &v, float *o)
+{
+    if constexpr (F == kF32) {
+        o[0] = __uint_as_float(v.x); o[1] = __uint_as_float(v.y);
+        o[2] = __uint_as_float(v.z); o[3] = __uint_as_float(v.w);
+    } else if constexpr (F == kF16) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
+            o[2 * i] = f.x;
+            o[2 * i + 1] = f.y;
+        }
+    } else if constexpr (F == kBF16) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            o[2 * i] = __uint_as_float(w[i] << 16);
+            o[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    } else {
+        // element 2j sits in the low nibble of byte j; n - 8 is formed exactly
+        // by placing n in the mantissa of 2^23 and subtracting 2^23 + 8
+        const uint32_t w[2] = {v.x, v.y};
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                o[8 * i + j] = __uint_as_float(0x4b000000u | ((w[i] >> (4 * j)) & 0xfu)) - 8388616.0f;
+    }
+}
+
+__device__ __forceinline__ float warp_sum(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Warp reduction of N values per lane (N a power of two <= 32): after it,
+// lane L holds the warp-wide sum of value L / (32 / N).  At each of the first
+// log2(N) stages a lane keeps one half of its values, chosen by its lane bit,
+// and adds the partner's copy of that half; the lanes left sharing a value
+// finish with a plain butterfly.  N - 1 + log2(32 / N) shuffles.
+template <int N>
+__device__ __forceinline__ float warp_transpose_sum(float (&v)[N])
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 16, n = N; n > 1; o >>= 1, n >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+            const float send = upper ? v[i] : v[i + n / 2];
+            const float keep = upper ? v[i + n / 2] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+#pragma unroll
+    for (int o = 32 / N / 2; o >= 1; o >>= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+    return v[0];
+}
+
+// Four 8x8 b16 matrices from shared memory (lane L gives the address of row
+// L % 8 of matrix L / 8).
+__device__ __forceinline__ void ldsm_x4(const void *p, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(s2u(p)));
+}
+// D += A (16x16, row) * B (16x8, col), 16-bit inputs of format F, fp32 accumulate.
+template <int F>
+__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1)
+{
+    if constexpr (F == kBF16)
+        asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                     "{%8, %9}, {%0, %1, %2, %3};"
+                     : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                     : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    else
+        asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                     "{%8, %9}, {%0, %1, %2, %3};"
+                     : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                     : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// An fp32 value as an unevaluated sum of 16-bit values of format F: two fp16
+// parts (22 significant bits) or up to three bf16 parts (24 bits; two, 16
+// bits, where shared memory holds only two per value).  Multiplying a 16-bit
+// weight by each part is exact in fp32, so a tensor-core dot with the parts as
+// columns of B, summed over the columns, carries the fp32 operand rather than
+// a 16-bit rounding of it.  Part p of value k is written at out[p * stride + k].
+template <int F>
+__device__ __forceinline__ void split_parts(float x, int nparts, uint16_t *out, int stride)
+{
+    if constexpr (F == kBF16) {
+        const __nv_bfloat16 h = __float2bfloat16_rn(x);
+        const float r1 = x - __bfloat162float(h);
+        const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+        out[0] = __bfloat16_as_ushort(h);
+        out[stride] = __bfloat16_as_ushort(m);
+        if (nparts > 2) out[2 * stride] = __bfloat16_as_ushort(__float2bfloat16_rn(r1 - __bfloat162float(m)));
+    } else {
+        const __half h = __float2half_rn(x);
+        out[0] = __half_as_ushort(h);
+        out[stride] = __half_as_ushort(__float2half_rn(x - __half2float(h)));
+    }
+}
+
+__device__ __forceinline__ float act_h(int act, float g, float u)
+{
+    const float gp = g > 0.f ? g : 0.f;
+    if (act == 0) return gp;               // ReLU (non-gated)
+    if (act == 1) return gp * u;           // ReGLU
+    return gp * (u > 0.f ? u : 0.f);       // dReLU
+}
+
+constexpr int kRA = 16;           // V rows per staging round at most
+constexpr int kZRows = 96;        // U rows per staging round at most (a multiple of 16)
+constexpr int kMaxU = 4;          // U vectors per lane (rank <= 128 * EPV)
+constexpr int kRound = 16;        // neurons per gather round at most
+constexpr int kRed = 2 * kRound;  // values reduced per warp at most
+
+struct Smem {
+    float red[2][kConsumerWarps][kRed];
+    float zred[kConsumerWarps][kZRows];    // per-warp partial logits of a U round
+    alignas(16) float tsm[kMaxRankTotal];  // t (fp32 predictor) or its 16-bit parts (split_parts)
+    alignas(16) float rsl[kMaxSliceCols];  // this CTA's columns of the new residual
+    float cbuf[kMaxTopK][kMaxStrip];
+    float zbuf[kMaxTopK][kMaxStrip];
+    ExpertDev exl[2][kMaxTopK];            // weight pointers of the layer's expert slots, by layer parity
+    int16_t lst[kMaxTopK * kMaxStrip];     // active neurons: (slot << 12) | local
+    int lst_n[kMaxTopK];
+    int16_t nz[kMaxTopK * kMaxStrip];      // neurons with h != 0, same encoding
+    float hz[kMaxTopK * kMaxStrip];        // their h (routing weight folded in)
+    int nz_n;
+    float rsum[kRed];                      // CTA-wide dot products of a gather round
+    float rh[kRound];                      // h of each neuron of a gather round
+    int route_e[kMaxTopK];
+    float route_w[kMaxTopK];
+    float inv_rms;
+    int bc[2];
+    uint64_t stage_bar;                    // completion of a staging round
+};
+
+__device__ void set_error(int *err, int code)
+{
+    atomicCAS(err, 0, code);
+}
+
+__device__ __forceinline__ void prof_put(const DecodeParams &p, int li, int point, long long v)
+{
+    if (p.prof && threadIdx.x == 0)
+        p.prof[(size_t(li) * kProfPoints + point) * gridDim.x + blockIdx.x] = v;
+}
+
+// Fixed-point accumulation (exact, so the result does not depend on the
+// order in which CTAs arrive): values are rounded to multiples of 2^-32 (2^-24
+// for sums of squares) and added as 64-bit integers.
+__device__ __forceinline__ void fix_add(long long *dst, float v, float scale)
+{
+    const long long q = __float2ll_rn(v * scale);
+    atomicAdd(reinterpret_cast<unsigned long long *>(dst), static_cast<unsigned long long>(q));
+}
+constexpr float kFixT = 4294967296.0f;    // 2^32
+constexpr float kFixSS = 16777216.0f;     // 2^24
+
+// Grid-wide barrier of all CTAs of the cooperative launch: arrivals are
+// fire-and-forget releases on one counter (never reset within a launch);
+// thread 0 of each CTA polls it with acquire loads, bounded by wait_ns.  The
+// outcome is broadcast through shared memory so the whole CTA agrees.
+__device__ bool grid_sync(Smem *sm, const DecodeParams &p, unsigned &epoch, int &bci, long long *cyc)
+{
+    cta_sync();
+    if (threadIdx.x == 0) {
+        const long long c0 = clock64();
+        bool ok = true;
+        epoch += 1;
+        unsigned target = epoch * gridDim.x;
+        if ((p.debug_flags & 1) && epoch == 1) target += 1;   // PI_DEBUG_STALL_BARRIER
+        __threadfence();
+        red_release_gpu(p.bar, 1u);
+        const long long t0 = gtimer();
+        unsigned it = 0;
+        while (ld_acquire_gpu(p.bar) < target) {
+            if ((++it & 31) == 0 && gtimer() - t0 > p.wait_ns) {
+                set_error(p.err, kDevTimeout);
+                ok = false;
+                break;
+            }
+        }
+        __threadfence();
+        st_vol(&sm->bc[bci], ok ? 1 : 0);
+        if (cyc) *cyc += clock64() - c0;
+    }
+    cta_sync();
+    const bool ok = ld_vol(&sm->bc[bci]) != 0;
+    bci ^= 1;
+    return ok;
+}
+
+// Staging round: thread 0 has issued bulk copies onto sm->stage_bar; it waits
+// (bounded) and the whole CTA adopts its verdict.
+__device__ bool stage_wait(Smem *sm, const DecodeParams &p, uint32_t &par, int &bci,
+                           long long *cyc = nullptr)
+{
+    if (threadIdx.x == 0) {
+        const long long c0 = clock64();
+        bool ok = mbar_test(&sm->stage_bar, par);
+        if (!ok) {
+            const long long t0 = gtimer();
+            for (unsigned it = 1; !ok; ++it) {
+                ok = mbar_test(&sm->stage_bar, par);
+                if (!ok && (it & 15) == 0 && gtimer() - t0 > p.wait_ns) {
+                    set_error(p.err, kDevTimeout);
+                    break;
+                }
+            }
+        }
+        st_vol(&sm->bc[bci], ok ? 1 : 0);
+        if (cyc) *cyc += clock64() - c0;
+    }
+    cta_sync();
+    const bool ok = ld_vol(&sm->bc[bci]) != 0;
+    bci ^= 1;
+    if (ok) {
+        mbar_test(&sm->stage_bar, par);   // acquire for this thread (phase complete)
+        par ^= 1;                         // a failed round keeps its phase for the drain
+    }
+    return ok;
+}
+
+// Issue bulk copies of [src, src + bytes) into dst in pieces of <= 32 KB.
+__device__ __forceinline__ void stage_copy(uint8_t *dst, const uint8_t *src, uint32_t bytes, uint64_t *bar)
+{
+    for (uint32_t o = 0; o < bytes; o += 32768u) {
+        const uint32_t n = bytes - o < 32768u ? bytes - o : 32768u;
+        bulk_g2s(dst + o, src + o, n, bar);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// The kernel
+// ---------------------------------------------------------------------------
+template <int WF, int PF, int DMAX, int MODE>
+__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p)
+{
+    constexpr int EPVW = Fm<WF>::EPV, EPVP = Fm<PF>::EPV, VBW = Fm<WF>::VB, VBP = Fm<PF>::VB;
+    constexpr int MAXVW = (DMAX / EPVW + kThreads - 1) / kThreads;
+    constexpr int MAXVP = (DMAX / EPVP + kThreads - 1) / kThreads;
+    // when both formats share the vector layout, x is cached once
+    constexpr bool kSameX = (WF == PF);
+    using VW = typename Fm<WF>::V;
+    using VP = typename Fm<PF>::V;
+
+    __shared__ Smem sm;
+    extern __shared__ __align__(128) uint8_t stg[];   // kStageBytes staging buffer
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int b = blockIdx.x, S = gridDim.x;
+    const int d = p.d, r = p.r;
+    const int s0 = p.strip_off[b], ns = p.strip_off[b + 1] - s0;
+    const bool predict = p.mode == kModePredict;
+    // layer kind, fixed per instantiation so each kernel holds only its path
+    constexpr bool moe = (MODE & kModeMoE) != 0;
+    constexpr bool kGated = (MODE & kModeGated) != 0;
+    constexpr bool kSpec = (MODE & kModeSpec) != 0;
+    const int ntop = predict ? 1 : p.top_k;
+    const int nvecW = (WF == kI4 ? d / 2 : d * (WF == kF32 ? 4 : 2)) / VBW;
+    const int nvecP = p.vrow / VBP;
+    const int nvecU = p.urow / VBP;
+    const int l0 = p.layer_begin;
+    const int l1 = predict ? p.layer_begin + 1 : p.layer_end;
+    // this CTA's columns of the residual (8-column groups)
+    const int c0 = 8 * p.grp_off[b], ncol = 8 * (p.grp_off[b + 1] - p.grp_off[b]);
+    // this CTA's rows of t (row-split form, MoE)
+    const int rows_total = ntop * r;
+    const int a0 = int((long long)b * rows_total / S), a1 = int((long long)(b + 1) * rows_total / S);
+    const int ucap = min(kZRows, kStageBytes / p.urow) & ~15;   // U rows per staging round (a multiple of 16)
+
+    // V block of this CTA (dense): rows of t restricted to this CTA's columns
+    auto vblk = [&](int l) -> const uint8_t * {
+        return sm.exl[l & 1][0].V + size_t(r) * c0 * (p.vrow / d);
+    };
+    const int vbrow = ncol * (p.vrow / d);   // bytes of one V-block row
+
+    unsigned epoch = 0;
+    uint32_t spar = 0;
+    int bci = 0, rb = 0;
+    bool staged_early = false;   // round 0 of the next U strip is already in flight
+    bool pending = false;        // a staging round was issued and not yet waited for
+
+    // stage rows [row0, row0 + n) of an expert's U strip, contiguous (lane 0
+    // of warp 0 issues the copies)
+    auto stage_u = [&](const ExpertDev &ex, int row0, int n) {
+        if (lane == 0) {
+            mbar_arrive_tx(&sm.stage_bar, uint32_t(n) * p.urow);
+            stage_copy(stg, ex.U + size_t(s0 + row0) * p.urow, uint32_t(n) * p.urow, &sm.stage_bar);
+        }
+    };
+
+    if (tid == 0) {
+        mbar_init(&sm.stage_bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        if (!moe) sm.exl[l0 & 1][0] = p.ex[size_t(l0) * p.E];
+    }
+    __syncwarp();
+    if (!moe && warp == 0 && ns > 0) {
+        const ExpertDev ex0 = sm.exl[l0 & 1][0];
+        stage_u(ex0, 0, min(ns, ucap));
+        if (lane == 0 && ns > ucap) prefetch_l2(ex0.U + size_t(s0 + ucap) * p.urow, uint32_t(ns - ucap) * p.urow);
+    }
+    if (!moe && ns > 0) staged_early = pending = true;
+    cta_sync();
+
+    // t value k of `ntr` (the layer's experts' ranks together) into shared memory
+    uint16_t *const tpart = reinterpret_cast<uint16_t *>(sm.tsm);
+    auto put_t = [&](int k, float tv, int ntr) {
+        if constexpr (PF == kF32) sm.tsm[k] = tv;
+        else split_parts<PF>(tv, (PF == kBF16 && 3 * ntr <= 2 * kMaxRankTotal) ? 3 : 2, tpart + k, ntr);
+    };
+
+    // -----------------------------------------------------------------------
+    // Column phase: this CTA's columns of r (the layer input `li_in`), its
+    // sum of squares, and its partial products for the next layer: the t
+    // partial V[:, cols] r[cols] (dense) or the router logit partials (MoE),
+    // all added in fixed point.  `from_partials`: r = r_old + sum of the
+    // per-CTA partials of y in fixed CTA order; otherwise r is the input.
+    // -----------------------------------------------------------------------
+    auto column_phase = [&](int li_in, bool from_partials, bool next_exists, int l_next, int prow) {
+        const float *src = predict ? p.x_in : p.resid;
+        long long *fx = p.fix + size_t(li_in & 1) * kFixStride;
+        if (from_partials) {
+            const int q0 = c0 / 4, nq = ncol / 4;
+            for (int qq = warp; qq < nq; qq += kConsumerWarps) {
+                const int q = q0 + qq;
+                float4 pv[kMaxStrips / 32];
+#pragma unroll
+                for (int j = 0; j < kMaxStrips / 32; ++j) {
+                    const int c = lane + 32 * j;
+                    pv[j] = c < S ? __ldcg(reinterpret_cast<const float4 *>(p.partials + size_t(c) * d) + q)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+                float4 rv = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (lane == 0) rv = __ldcg(reinterpret_cast<const float4 *>(p.resid) + q);
+                float4 sacc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int j = 0; j < kMaxStrips / 32; ++j) {
+                    sacc.x += pv[j].x; sacc.y += pv[j].y; sacc.z += pv[j].z; sacc.w += pv[j].w;
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    sacc.x += __shfl_xor_sync(0xffffffffu, sacc.x, o);
+                    sacc.y += __shfl_xor_sync(0xffffffffu, sacc.y, o);
+                    sacc.z += __shfl_xor_sync(0xffffffffu, sacc.z, o);
+                    sacc.w += __shfl_xor_sync(0xffffffffu, sacc.w, o);
+                }
+                if (lane == 0) {
+                    rv.x += sacc.x; rv.y += sacc.y; rv.z += sacc.z; rv.w += sacc.w;
+                    __stcg(reinterpret_cast<float4 *>(p.resid) + q, rv);
+                    *reinterpret_cast<float4 *>(sm.rsl + 4 * qq) = rv;
+                }
+            }
+        } else {
+            for (int j = tid; j < ncol; j += kThreads) sm.rsl[j] = __ldcg(src + c0 + j);
+        }
+        cta_sync();
+        if (prow >= 0) prof_put(p, prow, 7, gtimer());
+        if (!predict && p.trace && li_in < l1 - l0)
+            for (int j = tid; j < ncol; j += kThreads) __stcg(p.trace + size_t(li_in) * d + c0 + j, sm.rsl[j]);
+        if (!next_exists) return;
+        // sum of squares of this CTA's columns (fixed order: lanes, then tree)
+        if (warp == 0 && !predict) {
+            float ss = 0.f;
+            for (int j = lane; j < ncol; j += 32) ss = fmaf(sm.rsl[j], sm.rsl[j], ss);
+            ss = warp_sum(ss);
+            if (lane == 0 && ncol > 0) fix_add(fx + kMaxRankTotal, ss, kFixSS);
+        }
+        if (!moe) {
+            // t partial: row k of the V block dotted with this CTA's columns
+            const uint8_t *vb = vblk(l_next);
+            const int nv = vbrow / VBP;
+            // rows k and k + 512 together; four vectors of each in flight
+            for (int k = tid; k < r && ncol > 0; k += 2 * kThreads) {
+                const bool two = k + kThreads < r;
+                const uint8_t *row0 = vb + size_t(k) * vbrow;
+                const uint8_t *row1 = vb + size_t(two ? k + kThreads : k) * vbrow;
+                float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+                for (int v0 = 0; v0 < nv; v0 += 4) {
+                    VP q0[4], q1[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        if (v0 + j < nv) {
+                            q0[j] = ldvec<PF>(row0 + (v0 + j) * VBP);
+                            q1[j] = ldvec<PF>(row1 + (v0 + j) * VBP);
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        if (v0 + j < nv) {
+                            float w0[EPVP], w1[EPVP];
+                            cvt<PF>(q0[j], w0);
+                            cvt<PF>(q1[j], w1);
+#pragma unroll
+                            for (int i = 0; i < EPVP; i += 2) {
+                                const float x0 = sm.rsl[(v0 + j) * EPVP + i], x1 = sm.rsl[(v0 + j) * EPVP + i + 1];
+                                a0 = fmaf(w0[i], x0, a0);
+                                a1 = fmaf(w0[i + 1], x1, a1);
+                                b0 = fmaf(w1[i], x0, b0);
+                                b1 = fmaf(w1[i + 1], x1, b1);
+                            }
+                        }
+                    }
+                }
+                fix_add(fx + k, a0 + a1, kFixT);
+                if (two) fix_add(fx + k + kThreads, b0 + b1, kFixT);
+            }
+        } else if (!predict) {
+            // router logit partials: W_r[e, cols] . r[cols]
+            const __half *R = reinterpret_cast<const __half *>(p.router[l_next]);
+            if (tid < p.E && ncol > 0) {
+                float a = 0.f;
+                for (int j = 0; j < ncol; ++j) a = fmaf(__half2float(R[size_t(tid) * d + c0 + j]), sm.rsl[j], a);
+                fix_add(fx + kMaxRankTotal + 1 + tid, a, kFixT);
+            }
+        }
+    };
+
+    float xw[MAXVW * EPVW];
+    float xp_own[kSameX ? 1 : MAXVP * EPVP];
+#define XP(i) (kSameX ? xw[(i)] : xp_own[(i)])
+
+    // prologue: the first layer's input columns
+    column_phase(0, false, true, l0, -1);
+    long long cyc0 = 0;
+    const bool started = grid_sync(&sm, p, epoch, bci, &cyc0);
+
+    for (int l = l0; started && l < l1; ++l) {
+        const int li = l - l0;
+        long long cyc_a = 0, cyc_b = 0, cyc_c = 0, cyc_bar = 0;
+        prof_put(p, li, 0, gtimer());
+        const long long ca0 = clock64();
+        const long long *fx = p.fix + size_t(li & 1) * kFixStride;
+
+        // ---------------- layer input x, [MoE] routing and t rows ------------
+        const float *src = predict ? p.x_in : p.resid;
+        float inv = 1.f;
+        if (!predict) {
+            const long long ssq = __ldcg(fx + kMaxRankTotal);
+            inv = 1.f / sqrtf(float(double(ssq) * (1.0 / 16777216.0)) / float(d) + p.eps);
+        }
+#pragma unroll
+        for (int k = 0; k < MAXVW; ++k) {
+            const int v = tid + kThreads * k;
+#pragma unroll
+            for (int i = 0; i < EPVW; i += 4) {
+                float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (v < nvecW) q = __ldcg(reinterpret_cast<const float4 *>(src + v * EPVW + i));
+                xw[k * EPVW + i] = q.x * inv; xw[k * EPVW + i + 1] = q.y * inv;
+                xw[k * EPVW + i + 2] = q.z * inv; xw[k * EPVW + i + 3] = q.w * inv;
+            }
+        }
+        if constexpr (!kSameX) {
+#pragma unroll
+            for (int k = 0; k < MAXVP; ++k) {
+                const int v = tid + kThreads * k;
+#pragma unroll
+                for (int i = 0; i < EPVP; i += 4) {
+                    float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (v < nvecP) q = __ldcg(reinterpret_cast<const float4 *>(src + v * EPVP + i));
+                    xp_own[k * EPVP + i] = q.x * inv; xp_own[k * EPVP + i + 1] = q.y * inv;
+                    xp_own[k * EPVP + i + 2] = q.z * inv; xp_own[k * EPVP + i + 3] = q.w * inv;
+                }
+            }
+        }
+        if (!moe) {
+            // t from the fixed-point column partials
+            {
+                long long tq[kMaxRankTotal / kThreads];
+#pragma unroll
+                for (int j = 0; j < kMaxRankTotal / kThreads; ++j) {
+                    const int k = tid + kThreads * j;
+                    tq[j] = k < r ? __ldcg(fx + k) : 0;
+                }
+#pragma unroll
+                for (int j = 0; j < kMaxRankTotal / kThreads; ++j) {
+                    const int k = tid + kThreads * j;
+                    if (k < r) put_t(k, float(double(tq[j]) * (1.0 / 4294967296.0)) * inv, r);
+                }
+            }
+            // the next layer's weight pointers, for its prefetches during this layer
+            if (tid == kThreads - 1 && l + 1 < l1) sm.exl[(l + 1) & 1][0] = p.ex[size_t(l + 1) * p.E];
+            if (tid == 0) {
+                sm.route_e[0] = predict ? p.pred_expert : 0;
+                sm.route_e[1] = 0;
+                sm.route_w[0] = 1.f;
+                sm.route_w[1] = 0.f;
+                if (p.stats && b == 0 && !predict) {
+                    p.stats[li * 4 + 2] = -1;
+                    p.stats[li * 4 + 3] = -1;
+                }
+            }
+            cta_sync();
+        } else {
+            // routing from the fixed-point logits, identical in every CTA:
+            // softmax over E, two largest (ties: lower index), renormalised
+            if (tid == 0) {
+                int lo = p.pred_expert, hi = 0;
+                float wlo = 1.f, whi = 0.f;
+                if (!predict) {
+                    float logit[kMaxExperts], pr[kMaxExperts];
+                    float mx = -INFINITY;
+                    for (int e = 0; e < p.E; ++e) {
+                        logit[e] = float(double(__ldcg(fx + kMaxRankTotal + 1 + e)) * (1.0 / 4294967296.0)) * inv;
+                        mx = fmaxf(mx, logit[e]);
+                    }
+                    float den = 0.f;
+                    for (int e = 0; e < p.E; ++e) { pr[e] = expf(logit[e] - mx); den += pr[e]; }
+                    for (int e = 0; e < p.E; ++e) pr[e] /= den;
+                    int ea = 0;
+                    for (int e = 1; e < p.E; ++e) if (pr[e] > pr[ea]) ea = e;
+                    int eb = ea == 0 ? 1 : 0;
+                    for (int e = 0; e < p.E; ++e) if (e != ea && pr[e] > pr[eb]) eb = e;
+                    lo = min(ea, eb);
+                    hi = max(ea, eb);
+                    wlo = pr[lo] / (pr[lo] + pr[hi]);
+                    whi = pr[hi] / (pr[lo] + pr[hi]);
+                    if (p.stats && b == 0) {
+                        p.stats[li * 4 + 2] = lo;
+                        p.stats[li * 4 + 3] = hi;
+                    }
+                }
+                sm.route_e[0] = lo;
+                sm.route_e[1] = hi;
+                sm.route_w[0] = wlo;
+                sm.route_w[1] = whi;
+                // the experts' V rows and U strips start moving now
+                for (int e = 0; e < ntop; ++e) {
+                    const ExpertDev ex = p.ex[size_t(l) * p.E + (e == 0 ? lo : hi)];
+                    sm.exl[l & 1][e] = ex;
+                    const int lo_r = max(a0, e * r), hi_r = min(a1, (e + 1) * r);
+                    if (hi_r > lo_r)
+                        prefetch_l2(ex.V + size_t(lo_r - e * r) * p.vrow, uint32_t(hi_r - lo_r) * p.vrow);
+                    if (ns > 0) prefetch_l2(ex.U + size_t(s0) * p.urow, uint32_t(ns) * p.urow);
+                }
+            }
+            cta_sync();
+            // t rows [a0, a1) of the two experts, staged in rounds of kRA rows
+            const int per = min(kRA, kStageBytes / p.vrow);
+            bool ok = true;
+            for (int row0 = a0; row0 < a1 && ok; row0 += per) {
+                const int n = min(per, a1 - row0);
+                if (tid == 0) {
+                    mbar_arrive_tx(&sm.stage_bar, uint32_t(n) * p.vrow);
+                    for (int rr = 0; rr < n;) {
+                        const int row = row0 + rr, e = row / r;
+                        const int cnt = min(n - rr, (e + 1) * r - row);
+                        const uint8_t *vrow = sm.exl[l & 1][e].V + size_t(row - e * r) * p.vrow;
+                        stage_copy(stg + size_t(rr) * p.vrow, vrow, uint32_t(cnt) * p.vrow, &sm.stage_bar);
+                        rr += cnt;
+                    }
+                }
+                pending = true;
+                if (!stage_wait(&sm, p, spar, bci)) { ok = false; break; }
+                pending = false;
+                float part[kRA];
+#pragma unroll
+                for (int rr = 0; rr < kRA; ++rr) {
+                    part[rr] = 0.f;
+                    if (rr < n) {
+#pragma unroll
+                        for (int k = 0; k < MAXVP; ++k) {
+                            const int v = tid + kThreads * k;
+                            if (v < nvecP) {
+                                float w[EPVP];
+                                cvt<PF>(*reinterpret_cast<const VP *>(stg + size_t(rr) * p.vrow + v * VBP), w);
+#pragma unroll
+                                for (int i = 0; i < EPVP; ++i) part[rr] = fmaf(w[i], XP(k * EPVP + i), part[rr]);
+                            }
+                        }
+                    }
+                }
+#pragma unroll
+                for (int rr = 0; rr < kRA; ++rr) {
+                    if (rr < n) {
+                        const float v = warp_sum(part[rr]);
+                        if (lane == 0) sm.red[rb][warp][rr] = v;
+                    }
+                }
+                cta_sync();
+                if (tid < n) {
+                    float t = 0.f;
+                    for (int w = 0; w < kConsumerWarps; ++w) t += sm.red[rb][w][tid];
+                    __stcg(p.t_buf + row0 + tid, t);
+                }
+                rb ^= 1;
+            }
+            if (!ok) break;
+            // round 0 of the first expert's U strip lands during the barrier
+            if (warp == 0 && ns > 0) stage_u(sm.exl[l & 1][0], 0, min(ns, ucap));
+            staged_early = pending = ns > 0;
+            if (!grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
+            for (int k = tid; k < ntop * r; k += kThreads) put_t(k, __ldcg(p.t_buf + k), ntop * r);
+        }
+        for (int e = 0; e < ntop; ++e)
+            for (int i = tid; i < ns; i += kThreads)
+                sm.cbuf[e][i] = __ldg(sm.exl[l & 1][e].c + s0 + i);
+        cta_sync();
+        cyc_a = clock64() - ca0;
+        prof_put(p, li, 1, gtimer());
+
+        // ---------------- z = U t - c over the strip, compaction -------------
+        const long long cb0 = clock64();
+        {
+            bool ok = true;
+            for (int e = 0; e < ntop && ok; ++e) {
+                // fp32 predictor: this lane's t values (the columns of its U vectors)
+                float tu[PF == kF32 ? kMaxU * EPVP : 1];
+                if constexpr (PF == kF32) {
+#pragma unroll
+                    for (int k = 0; k < kMaxU; ++k) {
+                        const int v = lane + 32 * k;
+#pragma unroll
+                        for (int i = 0; i < EPVP; i += 4) {
+                            float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+                            if (v < nvecU) q = *reinterpret_cast<const float4 *>(sm.tsm + e * r + v * EPVP + i);
+                            tu[k * EPVP + i] = q.x; tu[k * EPVP + i + 1] = q.y;
+                            tu[k * EPVP + i + 2] = q.z; tu[k * EPVP + i + 3] = q.w;
+                        }
+                    }
+                }
+                for (int row0 = 0; row0 < ns && ok; row0 += ucap) {
+                    const int n = min(ucap, ns - row0);
+                    if (!(staged_early && row0 == 0)) {
+                        if (warp == 0) stage_u(sm.exl[l & 1][e], row0, n);
+                    }
+                    staged_early = false;
+                    pending = true;
+                    if (!stage_wait(&sm, p, spar, bci, &cyc_b)) { ok = false; break; }
+                    pending = false;
+                    if constexpr (PF == kF32) {
+                        // each warp takes rows warp, warp + 16, ...; four rows at a time,
+                        // each with its own accumulators, to keep the dependent FMA and
+                        // shuffle chains of different rows overlapped
+                        constexpr int kZR = 4;
+                        for (int rr0 = warp; rr0 < n; rr0 += kConsumerWarps * kZR) {
+                            float a[kZR][2];
+    #pragma unroll
+                            for (int j = 0; j < kZR; ++j) {
+                                a[j][0] = 0.f;
+                                a[j][1] = 0.f;
+                                const int rr = rr0 + j * kConsumerWarps;
+                                if (rr < n) {
+                                    const uint8_t *urow = stg + size_t(rr) * p.urow;
+    #pragma unroll
+                                    for (int k = 0; k < kMaxU; ++k) {
+                                        const int v = lane + 32 * k;
+                                        if (v < nvecU) {
+                                            float w[EPVP];
+                                            cvt<PF>(*reinterpret_cast<const VP *>(urow + v * VBP), w);
+    #pragma unroll
+                                            for (int i = 0; i < EPVP; ++i)
+                                                a[j][i & 1] = fmaf(w[i], tu[k * EPVP + i], a[j][i & 1]);
+                                        }
+                                    }
+                                }
+                            }
+    #pragma unroll
+                            for (int j = 0; j < kZR; ++j) a[j][0] += a[j][1];
+    #pragma unroll
+                            for (int o = 16; o > 0; o >>= 1)
+    #pragma unroll
+                                for (int j = 0; j < kZR; ++j) a[j][0] += __shfl_xor_sync(0xffffffffu, a[j][0], o);
+                            if (lane == 0) {
+    #pragma unroll
+                                for (int j = 0; j < kZR; ++j) {
+                                    const int rr = rr0 + j * kConsumerWarps;
+                                    if (rr < n) {
+                                        const int loc = row0 + rr;
+                                        const float z = a[j][0] - sm.cbuf[e][loc];
+                                        sm.zbuf[e][loc] = z;
+                                        if (predict && p.z_out) p.z_out[s0 + loc] = z;
+                                    }
+                                }
+                            }
+                        }
+                    } else {
+                        // tensor-core dots: A = 16 staged U rows x 16 columns
+                        // (ldmatrix; rows stored chunk-permuted by row mod 8
+                        // when u_swz), B = the matching 16 entries of t as
+                        // 16-bit parts (part g in column g), fp32
+                        // accumulators; warp w takes k-steps w, w + 16, ...
+                        constexpr int kParts = PF == kBF16 ? 3 : 2;
+                        const int ntr = ntop * r;
+                        const int nparts = (PF == kBF16 && 3 * ntr <= 2 * kMaxRankTotal) ? 3 : 2;
+                        const int nks = r / 16, nmt = (n + 15) / 16;
+                        const int g = lane >> 2, tq = lane & 3;
+                        float c[kZRows / 16][4];
+#pragma unroll
+                        for (int mt = 0; mt < kZRows / 16; ++mt)
+                            c[mt][0] = c[mt][1] = c[mt][2] = c[mt][3] = 0.f;
+                        const int arow = lane & 15;                       // row within an m-tile
+                        const int akey = p.u_swz ? (arow & 7) : 0;        // m-tiles start at multiples of 16
+                        const uint8_t *abase = stg + size_t(arow) * p.urow;
+                        const uint16_t *bpart = tpart + g * ntr + e * r + 2 * tq;
+                        for (int ks = warp; ks < nks; ks += kConsumerWarps) {
+                            uint32_t b0 = 0u, b1 = 0u;
+                            if (g < nparts) {
+                                b0 = *reinterpret_cast<const uint32_t *>(bpart + ks * 16);
+                                b1 = *reinterpret_cast<const uint32_t *>(bpart + ks * 16 + 8);
+                            }
+                            const int chunk = 2 * ks + (lane >> 4);            // 16-byte chunk of the row
+                            const uint8_t *arow_p = abase + ((chunk & ~7) | ((chunk ^ akey) & 7)) * 16;
+#pragma unroll
+                            for (int mt = 0; mt < kZRows / 16; ++mt) {
+                                if (mt < nmt) {
+                                    uint32_t a0, a1, a2, a3;
+                                    ldsm_x4(arow_p + size_t(mt) * 16 * p.urow, a0, a1, a2, a3);
+                                    mma16816<PF>(c[mt], a0, a1, a2, a3, b0, b1);
+                                }
+                            }
+                        }
+                        // sum over the parts: columns 0 and 1 sit in lane 4g, column 2 in lane 4g + 1
+#pragma unroll
+                        for (int mt = 0; mt < kZRows / 16; ++mt) {
+                            float z0 = c[mt][0] + c[mt][1], z1 = c[mt][2] + c[mt][3];
+                            if constexpr (kParts == 3) {
+                                z0 += __shfl_down_sync(0xffffffffu, c[mt][0], 1);
+                                z1 += __shfl_down_sync(0xffffffffu, c[mt][2], 1);
+                            }
+                            if (tq == 0 && mt < nmt) {
+                                sm.zred[warp][mt * 16 + g] = z0;
+                                sm.zred[warp][mt * 16 + g + 8] = z1;
+                            }
+                        }
+                        cta_sync();
+                        // across warps in fixed order
+                        const int nw = min(kConsumerWarps, nks);
+                        for (int rr = tid; rr < n; rr += kThreads) {
+                            float a = 0.f;
+                            for (int w = 0; w < nw; ++w) a += sm.zred[w][rr];
+                            const int loc = row0 + rr;
+                            const float z = a - sm.cbuf[e][loc];
+                            sm.zbuf[e][loc] = z;
+                            if (predict && p.z_out) p.z_out[s0 + loc] = z;
+                        }
+                    }
+                    cta_sync();   // the staging buffer is reused by the next round
+                }
+            }
+            if (!ok) break;
+        }
+        prof_put(p, li, 9, gtimer());
+        // compaction in ascending strip order: warp e builds expert slot e's list
+        if (warp < ntop) {
+            const int e = warp;
+            int cnt = 0;
+            const int off = e == 0 ? 0 : kMaxStrip;
+            for (int base = 0; base < ns; base += 32) {
+                const int loc = base + lane;
+                const bool act = loc < ns && sm.zbuf[e][loc] > p.threshold;
+                const unsigned msk = __ballot_sync(0xffffffffu, act);
+                if (act) {
+                    const int pos = cnt + __popc(msk & ((1u << lane) - 1u));
+                    sm.lst[off + pos] = int16_t((e << 12) | loc);
+                    if (predict) p.lists[size_t(b) * kMaxStrip + pos] = s0 + loc;
+                    if (p.masks) {
+                        const int gp = s0 + loc;
+                        const int words = (p.F + 31) / 32;
+                        atomicOr(p.masks + (size_t(li) * ntop + e) * words + (gp >> 5), 1u << (gp & 31));
+                    }
+                }
+                cnt += __popc(msk);
+            }
+            if (lane == 0) {
+                sm.lst_n[e] = cnt;
+                if (predict) p.counts[b] = cnt;
+                if (p.stats && !predict) atomicAdd(p.stats + li * 4 + 0, cnt);
+            }
+        }
+        if (tid == 0) sm.nz_n = 0;
+        cta_sync();
+        (void)cb0;
+        prof_put(p, li, 2, gtimer());
+
+        if (predict) {
+            // global ascending list: prefix of the strip counts, then copy
+            if (!grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
+            int pre = 0;
+            for (int i = tid; i < b; i += kThreads) pre += __ldcg(p.counts + i);
+            pre = __reduce_add_sync(0xffffffffu, pre);
+            if (lane == 0) sm.red[rb][warp][0] = __int_as_float(pre);
+            cta_sync();
+            int base = 0;
+            for (int w = 0; w < kConsumerWarps; ++w) base += __float_as_int(sm.red[rb][w][0]);
+            const int cnt = sm.lst_n[0];
+            for (int i = tid; i < cnt; i += kThreads) p.idx_out[base + i] = s0 + (sm.lst[i] & 0xfff);
+            if (b == S - 1 && tid == 0) p.count_out[0] = base + cnt;
+            break;
+        }
+
+        // ---------------- gather rows of active neurons ----------------------
+        // Rounds of up to kRound neurons: one bulk-copy round brings their
+        // W_gate/W_up records (and, when speculative, their W_down rows) into
+        // shared memory; the dots of all of them are reduced at once.
+        const long long cc0 = clock64();
+        const int m0 = sm.lst_n[0];
+        const int m = m0 + (ntop > 1 ? sm.lst_n[1] : 0);
+        auto entry = [&](int j) -> int { return j < m0 ? sm.lst[j] : sm.lst[kMaxStrip + (j - m0)]; };
+        const ExpertDev *exs[kMaxTopK] = {&sm.exl[l & 1][0], &sm.exl[l & 1][ntop > 1 ? 1 : 0]};
+        const int per_n = p.gu_bytes + (kSpec ? p.wrow : 0);   // bytes per neuron in a round
+        const int cap_n = min(kRound, kStageBytes / per_n);
+        // rows beyond the first round, and the next layer's V block and
+        // biases, start moving towards L2 now
+        for (int j = cap_n + tid; j < m; j += kThreads) {
+            const int en = entry(j), e = en >> 12, loc = en & 0xfff;
+            prefetch_l2(exs[e]->Wgu + size_t(s0 + loc) * p.gu_bytes, uint32_t(p.gu_bytes));
+            if (kSpec) prefetch_l2(exs[e]->Wd + size_t(s0 + loc) * p.wrow, uint32_t(p.wrow));
+        }
+        if (tid == kThreads - 1 && !moe && l + 1 < l1) {
+            if (ncol > 0) prefetch_l2(vblk(l + 1), uint32_t(r) * vbrow);
+            if (ns > 0) {
+                const int c_lo = s0 & ~3, c_hi = (s0 + ns + 3) & ~3;   // 16-byte aligned, padded
+                prefetch_l2(sm.exl[(l + 1) & 1][0].c + c_lo, uint32_t(c_hi - c_lo) * 4);
+            }
+        }
+
+        float acc[MAXVW * EPVW];
+#pragma unroll
+        for (int i = 0; i < MAXVW * EPVW; ++i) acc[i] = 0.f;
+        // acc += h * (a W_down row in shared memory)
+        auto axpy_smem = [&](const uint8_t *row, float h) {
+#pragma unroll
+            for (int k = 0; k < MAXVW; ++k) {
+                const int v = tid + kThreads * k;
+                if (v < nvecW) {
+                    float w[EPVW];
+                    cvt<WF>(*reinterpret_cast<const VW *>(row + v * VBW), w);
+                    float hs = h;
+                    if constexpr (WF == kI4) hs = h * __half2float(*reinterpret_cast<const __half *>(row + d / 2 + (v >> 1) * 2));
+#pragma unroll
+                    for (int i = 0; i < EPVW; ++i) acc[k * EPVW + i] = fmaf(hs, w[i], acc[k * EPVW + i]);
+                }
+            }
+        };
+        // dot of a row in shared memory with this thread's x columns
+        auto dot_smem = [&](const uint8_t *row) -> float {
+            float a = 0.f;
+#pragma unroll
+            for (int k = 0; k < MAXVW; ++k) {
+                const int v = tid + kThreads * k;
+                if (v < nvecW) {
+                    float w[EPVW];
+                    cvt<WF>(*reinterpret_cast<const VW *>(row + v * VBW), w);
+                    float c = 0.f;
+#pragma unroll
+                    for (int i = 0; i < EPVW; ++i) c = fmaf(w[i], xw[k * EPVW + i], c);
+                    if constexpr (WF == kI4) c *= __half2float(*reinterpret_cast<const __half *>(row + d / 2 + (v >> 1) * 2));
+                    a += c;
+                }
+            }
+            return a;
+        };
+
+        prof_put(p, li, 8, gtimer());
+        bool gok = true;
+        int nz_total = 0;            // neurons with h != 0 so far (list order)
+        for (int j0 = 0; j0 < m && gok; j0 += cap_n) {
+            const int k = min(cap_n, m - j0);
+            if (warp == 0) {
+                // lane 0 announces the round's bytes, then lane n copies neuron n
+                if (lane == 0) mbar_arrive_tx(&sm.stage_bar, uint32_t(k) * per_n);
+                __syncwarp();
+                if (lane < k) {
+                    const int en = entry(j0 + lane), e = en >> 12, loc = en & 0xfff;
+                    uint8_t *slot = stg + size_t(lane) * per_n;
+                    stage_copy(slot, exs[e]->Wgu + size_t(s0 + loc) * p.gu_bytes, uint32_t(p.gu_bytes),
+                               &sm.stage_bar);
+                    if (kSpec)
+                        stage_copy(slot + p.gu_bytes, exs[e]->Wd + size_t(s0 + loc) * p.wrow, uint32_t(p.wrow),
+                                   &sm.stage_bar);
+                }
+            }
+            if (j0 == 0) prof_put(p, li, 14, gtimer());
+            pending = true;
+            if (!stage_wait(&sm, p, spar, bci, &cyc_c)) { gok = false; break; }
+            pending = false;
+            if (j0 == 0) prof_put(p, li, 15, gtimer());
+            // dots of the round's neurons, four at a time: values 2n (gate) and
+            // 2n + 1 (up); after the reduction lanes 4q .. 4q + 3 hold value q
+#pragma unroll 1
+            for (int g0 = 0; g0 < k; g0 += 4) {
+                float v[8];
+#pragma unroll
+                for (int n = 0; n < 4; ++n) {
+                    v[2 * n] = 0.f;
+                    v[2 * n + 1] = 0.f;
+                    if (g0 + n < k) {
+                        const uint8_t *slot = stg + size_t(g0 + n) * per_n;
+                        v[2 * n] = dot_smem(slot);
+                        if (kGated) v[2 * n + 1] = dot_smem(slot + p.wrow);
+                    }
+                }
+                const float ws = warp_transpose_sum(v);
+                const int q = 2 * g0 + (lane >> 2);
+                if ((lane & 3) == 0 && q < 2 * k) sm.red[rb][warp][q] = ws;
+            }
+            if (j0 == 0) prof_put(p, li, 16, gtimer());
+            cta_sync();
+            if (j0 == 0) prof_put(p, li, 17, gtimer());
+            if (tid < 2 * k) {
+                float a = 0.f;
+                for (int w = 0; w < kConsumerWarps; ++w) a += sm.red[rb][w][tid];
+                sm.rsum[tid] = a;
+            }
+            rb ^= 1;
+            cta_sync();
+            if (j0 == 0) prof_put(p, li, 18, gtimer());
+            if (tid < k) {
+                const int en = entry(j0 + tid), e = en >> 12, loc = en & 0xfff;
+                sm.rh[tid] = act_h(p.act, sm.rsum[2 * tid] - sm.cbuf[e][loc], sm.rsum[2 * tid + 1]) *
+                             sm.route_w[e];
+            }
+            cta_sync();
+            if (j0 == 0) prof_put(p, li, 19, gtimer());
+            // neurons with h != 0, in list order
+            int nz_round = 0;
+            for (int n = 0; n < k; ++n) {
+                const float h = sm.rh[n];
+                if (h == 0.f) continue;
+                if (tid == 0) {
+                    sm.nz[nz_total + nz_round] = int16_t(entry(j0 + n));
+                    sm.hz[nz_total + nz_round] = h;
+                }
+                ++nz_round;
+                if (kSpec) axpy_smem(stg + size_t(n) * per_n + p.gu_bytes, h);
+            }
+            nz_total += nz_round;
+            if (j0 == 0) prof_put(p, li, 20, gtimer());
+            cta_sync();   // the staging buffer is reused by the next round
+            if (j0 == 0) prof_put(p, li, 21, gtimer());
+        }
+        prof_put(p, li, 22, gtimer());
+        // not speculative: the W_down rows of the neurons with h != 0, in rounds
+        if (gok && !kSpec) {
+            const int cap_d = min(kMaxTopK * kMaxStrip, kStageBytes / p.wrow);
+            for (int q0 = 0; q0 < nz_total && gok; q0 += cap_d) {
+                const int k = min(cap_d, nz_total - q0);
+                if (warp == 0) {
+                    if (lane == 0) mbar_arrive_tx(&sm.stage_bar, uint32_t(k) * p.wrow);
+                    __syncwarp();
+                    for (int n = lane; n < k; n += 32) {
+                        const int en = sm.nz[q0 + n], e = en >> 12, loc = en & 0xfff;
+                        stage_copy(stg + size_t(n) * p.wrow, exs[e]->Wd + size_t(s0 + loc) * p.wrow,
+                                   uint32_t(p.wrow), &sm.stage_bar);
+                    }
+                }
+                pending = true;
+                if (!stage_wait(&sm, p, spar, bci, &cyc_c)) { gok = false; break; }
+                pending = false;
+                for (int n = 0; n < k; ++n) axpy_smem(stg + size_t(n) * p.wrow, sm.hz[q0 + n]);
+                cta_sync();
+            }
+        }
+        if (!gok) break;
+        if (tid == 0 && p.stats) atomicAdd(p.stats + li * 4 + 1, nz_total);
+        // the next layer's predictor slice starts moving: U strip straight
+        // into shared memory (free until then), the rest of it into L2
+        if (!moe && l + 1 < l1 && ns > 0 && warp == 0) {
+            stage_u(sm.exl[(l + 1) & 1][0], 0, min(ns, ucap));
+            if (lane == 0 && ns > ucap)
+                prefetch_l2(sm.exl[(l + 1) & 1][0].U + size_t(s0 + ucap) * p.urow, uint32_t(ns - ucap) * p.urow);
+        }
+        staged_early = !moe && l + 1 < l1 && ns > 0;
+        if (staged_early) pending = true;
+        // the fixed-point buffer of layer l - 1 (read before two barriers ago)
+        // is cleared for layer l + 1
+        if (b == S - 1) {
+            long long *fz = p.fix + size_t((li + 1) & 1) * kFixStride;
+            for (int i = tid; i < kFixStride; i += kThreads) fz[i] = 0;
+        }
+        // per-CTA partial of y
+#pragma unroll
+        for (int k = 0; k < MAXVW; ++k) {
+            const int v = tid + kThreads * k;
+            if (v < nvecW) {
+#pragma unroll
+                for (int i = 0; i < EPVW; i += 4)
+                    __stcg(reinterpret_cast<float4 *>(p.partials + size_t(b) * d + v * EPVW + i),
+                           make_float4(acc[k * EPVW + i], acc[k * EPVW + i + 1],
+                                       acc[k * EPVW + i + 2], acc[k * EPVW + i + 3]));
+            }
+        }
+        (void)cc0;
+        prof_put(p, li, 23, gtimer());
+        prof_put(p, li, 3, gtimer());
+        if (!grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
+        prof_put(p, li, 4, gtimer());
+
+        // ---------------- reduction + next layer's column products -----------
+        const bool next = l + 1 < l1;
+        column_phase(li + 1, true, next, l + 1, li);
+        prof_put(p, li, 5, gtimer());
+        if (next && !grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
+        prof_put(p, li, 6, gtimer());
+        prof_put(p, li, 10, cyc_a);
+        prof_put(p, li, 11, cyc_b);
+        prof_put(p, li, 12, cyc_c);
+        prof_put(p, li, 13, cyc_bar);
+    }
+    // an early exit may leave one staging round in flight: let it land
+    // (bounded) so no bulk copy writes this CTA's shared memory after exit
+    if (pending && tid == 0) {
+        const long long t0 = gtimer();
+        while (!mbar_test(&sm.stage_bar, spar) && gtimer() - t0 < p.wait_ns) {
+        }
+    }
+#undef XP
+}
+
+// One instantiation per (weight format, predictor format, d_model class,
+// layer kind); each per-format translation unit instantiates its own set.
+template <int WF, int PF, int DMAX, int MODE>
+cudaError_t launch_one(const DecodeParams &p, cudaStream_t st, bool query, int *blocks)
+{
+    void *fn = (void *)decode_kernel<WF, PF, DMAX, MODE>;
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kStageBytes);
+    if (e != cudaSuccess) return e;
+    if (query) return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, fn, kThreads, kStageBytes);
+    void *args[] = {const_cast<DecodeParams *>(&p)};
+    return cudaLaunchCooperativeKernel(fn, dim3(p.S), dim3(kThreads), args, kStageBytes, st);
+}
+
+template <int WF, int PF, int DMAX>
+cudaError_t launch_mode(int mode, const DecodeParams &p, cudaStream_t st, bool query, int *blocks)
+{
+    switch (mode) {
+    case kModeSpec: return launch_one<WF, PF, DMAX, kModeSpec>(p, st, query, blocks);
+    case kModeGated | kModeSpec: return launch_one<WF, PF, DMAX, kModeGated | kModeSpec>(p, st, query, blocks);
+    case kModeGated: return launch_one<WF, PF, DMAX, kModeGated>(p, st, query, blocks);
+    case kModeMoE | kModeSpec: return launch_one<WF, PF, DMAX, kModeMoE | kModeSpec>(p, st, query, blocks);
+    case kModeMoE | kModeGated | kModeSpec:
+        return launch_one<WF, PF, DMAX, kModeMoE | kModeGated | kModeSpec>(p, st, query, blocks);
+    case kModeMoE | kModeGated: return launch_one<WF, PF, DMAX, kModeMoE | kModeGated>(p, st, query, blocks);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+// d_model classes: the register arrays of x hold ceil(d / (elements per
+// vector * threads)) vectors per thread, so two classes cover d <= 8192
+// (d <= 4096 for fp32).
+template <int WF, int PF>
+cudaError_t launch_fmt(int d, int mode, const DecodeParams &p, cudaStream_t st, bool query, int *blocks)
+{
+    constexpr int kSmall = (WF == kF32 || PF == kF32) ? 2048 : 4096;
+    if (d <= kSmall) return launch_mode<WF, PF, kSmall>(mode, p, st, query, blocks);
+    if (d <= 2 * kSmall) return launch_mode<WF, PF, 2 * kSmall>(mode, p, st, query, blocks);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+}  // namespace pi

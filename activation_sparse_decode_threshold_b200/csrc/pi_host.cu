@@ -71,6 +71,7 @@ struct pi_ffn {
     int S = 0;                       // strips = CTAs of the decode kernel
     int wfmt = 0, pfmt = 0, gated = 0;
     int vrow = 0, urow = 0, wrow = 0;
+    int u_swz = 0;
     std::vector<int32_t> strip_off;
     std::vector<int32_t> grp_off;              // column slices in 8-column groups
     std::vector<std::vector<int32_t>> perm;   // [layer * E + e]
@@ -123,9 +124,8 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
                     "supported (w_dtype, pred_dtype): (F32,F32) (F16,F16) (BF16,BF16) "
                     "(INT4G32,F16) (INT4G32,BF16)");
     const int pb = elem_bytes(D.pred_dtype);
-    if (D.rank < 1 || (D.rank * pb) % 16 != 0 || D.rank > 128 * (16 / pb))
-        return fail(PI_ERR_INVALID_ARG, "rank*bytes must be a multiple of 16 and rank <= %d",
-                    128 * (16 / pb));
+    if (D.rank < 1 || D.rank % 16 != 0 || D.rank > 128 * (16 / pb))
+        return fail(PI_ERR_INVALID_ARG, "rank must be a multiple of 16 and <= %d", 128 * (16 / pb));
     if (D.n_experts == 1) {
         if (D.top_k != 1) return fail(PI_ERR_INVALID_ARG, "a dense FFN needs top_k = 1");
     } else if (D.n_experts >= 2 && D.n_experts <= pi::kMaxExperts) {
@@ -158,6 +158,10 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
     h->gated = D.act != PI_ACT_RELU;
     h->vrow = D.d_model * pb;
     h->urow = D.rank * pb;
+    // 16-bit predictors feed tensor-core dots through 8-row matrix loads; rows
+    // of whole 128-byte groups are stored chunk-permuted so those loads do not
+    // collide in shared-memory banks
+    h->u_swz = D.pred_dtype != PI_F32 && h->urow % 128 == 0;
     h->wrow = D.w_dtype == PI_INT4G32 ? D.d_model / 2 + D.d_model / 16
                                       : D.d_model * elem_bytes(D.w_dtype);
     h->S = D.n_strips > 0 ? D.n_strips : prop.multiProcessorCount;
@@ -343,7 +347,10 @@ pi_status pi_ffn_load_layer(pi_ffn_t h, int layer, const pi_expert_weights *expe
                                         elem_bytes(D.pred_dtype), st), "repack V");
         else
             PI_CUDA(cudaMemcpyAsync(m + o_V, w.V, size_t(r) * h->vrow, cudaMemcpyDeviceToDevice, st), "copy V");
-        {
+        if (h->u_swz) {
+            PI_CUDA(pi::repack_u_swizzled(m + o_U, d_perm, F, static_cast<const uint8_t *>(w.U), h->urow,
+                                          h->d_strip_off, h->S, st), "repack U");
+        } else {
             const uint8_t *src[1] = {static_cast<const uint8_t *>(w.U)};
             const int rb[1] = {h->urow};
             PI_CUDA(pi::repack_rows(m + o_U, d_perm, F, 1, src, rb, st), "repack U");
@@ -431,6 +438,7 @@ static pi::DecodeParams base_params(pi_ffn_t h)
     p.wrow = h->wrow;
     p.gu_bytes = (h->gated ? 2 : 1) * h->wrow;
     p.spec_down = D.act != PI_ACT_DRELU;
+    p.u_swz = h->u_swz;
     p.t_buf = h->t_buf;
     p.partials = h->partials;
     p.lists = h->lists;

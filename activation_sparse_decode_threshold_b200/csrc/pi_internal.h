@@ -49,6 +49,7 @@ struct DecodeParams {
     int vrow, urow, wrow;           // row bytes: V (pred fmt), U (pred fmt), W (weight fmt)
     int gu_bytes;                   // bytes of a neuron's input record (2 * wrow gated)
     int spec_down;                  // prefetch down rows of all predicted-active neurons
+    int u_swz;                      // U rows stored chunk-permuted (repack_u_swizzled)
     int mode, pred_expert;
     // inputs / outputs
     float *resid;                   // [d] decode: in/out residual
@@ -72,7 +73,9 @@ struct DecodeParams {
 };
 
 // Phase timestamps recorded per layer and CTA when DecodeParams::prof is set.
-constexpr int kProfPoints = 14;   // 7 timestamps, 3 unused, 4 cycle counters
+// layer kinds (bits of the decode kernel's MODE parameter)
+constexpr int kModeMoE = 1, kModeGated = 2, kModeSpec = 4;
+constexpr int kProfPoints = 24;   // timestamps and cycle counters per layer and CTA
 
 cudaError_t launch_decode(int wfmt, int pfmt, const DecodeParams &p, cudaStream_t stream);
 int decode_max_blocks_per_sm(int wfmt, int pfmt, int d);
@@ -86,6 +89,10 @@ cudaError_t repack_rows(uint8_t *dst, const int32_t *perm, int rows, int n_src,
 cudaError_t repack_v_blocks(const uint8_t *V, uint8_t *dst, const int32_t *grp_off, int S, int r,
                             int d, int elem_bytes, cudaStream_t s);
 cudaError_t repack_bias(const float *src, float *dst, const int32_t *perm, int n, cudaStream_t s);
+// U rows in table order, 16-byte chunks permuted inside each 128-byte group by
+// (row - strip start) mod 8 (row_bytes a multiple of 128); strip_off on the device.
+cudaError_t repack_u_swizzled(uint8_t *dst, const int32_t *perm, int rows, const uint8_t *src, int row_bytes,
+                              const int32_t *strip_off, int S, cudaStream_t s);
 cudaError_t repack_down_transpose(const uint8_t *w_down, uint8_t *dst, const int32_t *perm,
                                   int d, int F, int elem_bytes, cudaStream_t s);
 

@@ -98,8 +98,8 @@ extern "C" PI_API pi_status pi_predict_noalloc(int d_model, int d_ff, int rank, 
     const int pb = pred_dtype == PI_F32 ? 4 : 2;
     if (d_model < 256 || d_model % 256 != 0 || d_model > (pb == 4 ? 4096 : 8192))
         return na_fail(PI_ERR_INVALID_ARG, "d_model must be a multiple of 256, <= 8192 (<= 4096 for F32)");
-    if (rank < 1 || (rank * pb) % 16 != 0 || rank > 128 * (16 / pb))
-        return na_fail(PI_ERR_INVALID_ARG, "rank * bytes must be a multiple of 16 and rank <= 1024 (512 for F32)");
+    if (rank < 1 || rank % 16 != 0 || rank > 128 * (16 / pb))
+        return na_fail(PI_ERR_INVALID_ARG, "rank must be a multiple of 16 and <= 1024 (512 for F32)");
     if (!std::isfinite(threshold)) return na_fail(PI_ERR_INVALID_ARG, "threshold must be finite");
     const void *ptrs[] = {V_dev, U_dev, x_dev};
     for (const void *q : ptrs)
@@ -164,6 +164,7 @@ extern "C" PI_API pi_status pi_predict_noalloc(int d_model, int d_ff, int rank, 
     p.wrow = d_model * pb;
     p.gu_bytes = 2 * p.wrow;
     p.spec_down = 0;
+    p.u_swz = 0;          // the caller's U rows as they are
     p.mode = pi::kModePredict;
     p.pred_expert = 0;
     p.x_in = x_dev;

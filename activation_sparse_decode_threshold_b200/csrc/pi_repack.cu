@@ -38,6 +38,29 @@ __global__ void k_repack_rows(uint8_t *__restrict__ dst, const int32_t *__restri
     }
 }
 
+// Predictor U rows in table order with the 16-byte chunks of each row permuted
+// inside every 128-byte group by the row's position in its strip modulo 8:
+// chunk j goes to (j & ~7) | ((j ^ key) & 7), key = (p - strip start) & 7.
+// Staged contiguously, the rows then let an 8-row matrix load hit eight
+// different shared-memory bank groups.
+__global__ void k_repack_u_swz(uint8_t *__restrict__ dst, const int32_t *__restrict__ perm, int rows,
+                               const uint8_t *__restrict__ src, int row_bytes,
+                               const int32_t *__restrict__ strip_off, int S)
+{
+    const int p = blockIdx.x;
+    if (p >= rows) return;
+    int lo = 0, hi = S - 1;                 // strip b with strip_off[b] <= p < strip_off[b + 1]
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) / 2;
+        if (strip_off[mid] <= p) lo = mid;
+        else hi = mid - 1;
+    }
+    const int key = (p - strip_off[lo]) & 7;
+    const uint4 *s = reinterpret_cast<const uint4 *>(src + (long long)perm[p] * row_bytes);
+    uint4 *t = reinterpret_cast<uint4 *>(dst + (long long)p * row_bytes);
+    for (int j = threadIdx.x; j < row_bytes / 16; j += blockDim.x) t[(j & ~7) | ((j ^ key) & 7)] = s[j];
+}
+
 __global__ void k_repack_bias(const float *__restrict__ src, float *__restrict__ dst,
                               const int32_t *__restrict__ perm, int n)
 {
@@ -113,6 +136,15 @@ cudaError_t repack_rows(uint8_t *dst, const int32_t *perm, int rows, int n_src,
         rs.bytes[i] = row_bytes[i];
     }
     k_repack_rows<<<rows, 128, 0, s>>>(dst, perm, rows, rs);
+    return cudaGetLastError();
+}
+
+cudaError_t repack_u_swizzled(uint8_t *dst, const int32_t *perm, int rows, const uint8_t *src, int row_bytes,
+                              const int32_t *strip_off, int S, cudaStream_t s)
+{
+    if (rows <= 0) return cudaSuccess;
+    if (row_bytes % 128 != 0) return cudaErrorInvalidValue;
+    k_repack_u_swz<<<rows, 128, 0, s>>>(dst, perm, rows, src, row_bytes, strip_off, S);
     return cudaGetLastError();
 }
 

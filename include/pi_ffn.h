@@ -81,7 +81,8 @@ typedef struct {
     int n_layers;        /* layers in the stack, >= 1 */
     int d_model;         /* d: multiple of 256, <= 8192 (<= 4096 for F32) */
     int d_ff;            /* F: neurons per FFN (per expert), <= 256 * n_strips */
-    int rank;            /* predictor rank r: r * bytes(pred_dtype) a multiple of 16,
+    int rank;            /* predictor rank r: a multiple of 16 (the tensor-core
+                            predictor dots take 16 columns per step),
                             r <= 1024 (<= 512 for F32) */
     int n_experts;       /* 1 = dense FFN; 2..16 = MoE with top-2 routing */
     int top_k;           /* 1 for a dense FFN, 2 for MoE */
@@ -205,14 +206,20 @@ PI_API void pi_ffn_destroy(pi_ffn_t h);
 PI_API pi_status pi_debug_set(pi_ffn_t h, int flags, double wait_limit_s);
 
 /* Testing aid: when `times_dev` is non-NULL, each later pi_sparse_ffn_decode
- * call records %globaltimer (ns) at ten points of every layer in every CTA:
- * times_dev[((l - layer_begin) * 14 + k) * n_strips + cta], k = 0 layer start,
- * 1 input ready, 2 t rows done, 3 after barrier 1, 4 logits done, 5 active
- * list published, 6 gather done, 7 after barrier 2, 8 reduction done,
- * 9 after barrier 3; k = 10..13 hold clock cycles thread 0 spent waiting for
- * predictor data, logit data, gathered rows and grid barriers.  The buffer
- * (caller-owned, device, 8-byte aligned) must
- * hold (l1 - l0) * 14 * n_strips values.  NULL turns recording off. */
+ * call records, per layer and CTA, %globaltimer (ns) at these points k:
+ *   0 layer start, 1 layer input and t ready, 9 predictor logits done,
+ *   2 active list done, 8 gather start, 14 first gather round's copies
+ *   issued, 15 its rows landed, 16 its dots done, 17 its warp sums stored,
+ *   18 its row sums, 19 its h, 20 its W_down accumulation, 21 its end,
+ *   22 all gather rounds done, 23 partial stored, 3 gather done, 4 after the
+ *   gather barrier, 7 partials reduced, 5 column phase done, 6 after the
+ *   column barrier;
+ * and k = 10..13 the clock cycles thread 0 spent obtaining the layer input,
+ * waiting for predictor rows, waiting for gathered rows and waiting in grid
+ * barriers.  Value (layer - layer_begin, k, cta) sits at
+ * times_dev[((layer - layer_begin) * 24 + k) * n_strips + cta].  The buffer
+ * (caller-owned, device, 8-byte aligned) must hold (l1 - l0) * 24 * n_strips
+ * values.  NULL turns recording off. */
 PI_API pi_status pi_debug_phase_times(pi_ffn_t h, long long *times_dev);
 
 /* The low-rank predictor on caller-owned weights, with no device allocation
