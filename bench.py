@@ -229,6 +229,20 @@ def run_reference(args, cfg, active, rank: int, world: int):
     return 0
 
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """Largest value of x over all ranks (identity when not distributed)."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: int, world: int, max_ms: float) -> float:
+    """Whole-job units per second: every rank's units over the slowest rank's time."""
+    return units_per_rank * world / (max_ms / 1e3)
+
+
 def workload_config(cfg, active, measured_active):
     return {"workload": cfg.name, "layers": cfg.n_layers, "d_model": cfg.d, "d_ff": cfg.F,
             "rank": cfg.rank, "act": cfg.act, "weights": cfg.wdtype, "predictor": cfg.pdtype,
@@ -309,13 +323,9 @@ def main() -> int:
         dist.barrier()
     if B.pi_sync(h) != B.PI_OK:
         raise RuntimeError(B.pi_last_error())
-    total_ms = t_start.elapsed_time(t_end)
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), dist, "cuda")
     launch_ms = [a.elapsed_time(b) for a, b in ev]
-    if dist is not None:
-        tt = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
-    value = K * world / (total_ms / 1e3)
+    value = job_throughput(K, world, total_ms)
 
     st = stats[W:].cpu().numpy()
     bytes_per_token = [algorithmic_bytes(cfg, st[s]) for s in range(K)]
@@ -343,12 +353,8 @@ def main() -> int:
             B.pi_sparse_ffn_decode_host(h, 0, L, hin[s], hout[s])
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1)
-        if dist is not None:
-            tt = torch.tensor([e2e_ms], device="cuda")
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
-        e2e = {"value": K * world / (e2e_ms / 1e3), "unit": "tok/s",
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, "cuda")
+        e2e = {"value": job_throughput(K, world, e2e_ms), "unit": "tok/s",
                "h2d_bytes_per_step": 4 * cfg.d, "d2h_bytes_per_step": 4 * cfg.d}
 
     torch.cuda.synchronize()
