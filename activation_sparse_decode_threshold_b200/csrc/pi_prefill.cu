@@ -37,8 +37,10 @@
 namespace pi {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, NSTAGE = 3;
-constexpr int kGemmThreads = 256;
+constexpr int BM = 128, BN = 256, BK = 64, NSTAGE = 4;
+constexpr int kProducerWarps = 8, kProducers = 32 * kProducerWarps;
+constexpr int kGemmThreads = kProducers + 32;    // + the MMA warp
+constexpr int kLag = 2;                          // stages between issuing a stage's copies and publishing it
 constexpr int kATileBytes = BM * BK * 2;          // 16 KB
 constexpr int kBTileBytes = BN * BK * 2;          // 32 KB
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
@@ -181,32 +183,55 @@ __device__ __forceinline__ uint32_t mnmaj_off(int ng, int k)
     return uint32_t(ng * (BK / 8 * 128) + (k >> 3) * 128 + (k & 7) * 16);
 }
 
-// 16 INT4 weights (8 bytes of nibbles, one group scale) -> 16 fp16 values
-__device__ __forceinline__ void dequant16(uint2 q, float s, uint4 &lo, uint4 &hi)
+// 16 INT4 weights (8 bytes of nibbles, low nibble = even element) with their
+// group scale -> 16 fp16 values s * (n - 8), on the half-precision pipe: a
+// nibble n placed in the fraction of the half 1024.0 gives 1024 + n exactly,
+// subtracting 1032 gives n - 8 exactly, and the product with s is rounded
+// once, as a rounding of the exact s * (n - 8) to fp16.
+__device__ __forceinline__ void dequant16(uint2 q, __half s, uint4 &lo, uint4 &hi)
 {
-    __half2 h[8];
+    const __half2 s2 = __halves2half2(s, s);
+    const __half2 off = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));   // 1032
+    uint32_t o[8];
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
         const uint32_t w = i == 0 ? q.x : q.y;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float a = float(int((w >> (8 * j)) & 0xf) - 8) * s;
-            const float b = float(int((w >> (8 * j + 4)) & 0xf) - 8) * s;
-            h[4 * i + j] = __floats2half2_rn(a, b);
+        for (int m = 0; m < 4; ++m) {
+            const uint32_t t = w >> (8 * m);
+            const uint32_t bits = (t & 0xFu) | ((t & 0xF0u) << 12) | 0x64006400u;
+            __half2 h = *reinterpret_cast<const __half2 *>(&bits);
+            h = __hmul2(__hsub2(h, off), s2);
+            o[4 * i + m] = *reinterpret_cast<const uint32_t *>(&h);
         }
     }
-    lo = *reinterpret_cast<uint4 *>(&h[0]);
-    hi = *reinterpret_cast<uint4 *>(&h[4]);
+    lo = make_uint4(o[0], o[1], o[2], o[3]);
+    hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
 // ---------------------------------------------------------------------------
-// GEMM kernel
+// GEMM kernel.  Warps 0-7 produce stages (cp.async for 16-bit operands, INT4
+// weights through registers one stage ahead and dequantised into the tile),
+// warp 8 issues the MMAs from one thread, and warps 0-7 run the epilogue
+// once the accumulator is complete.  Stage s is published on full[s] (every
+// producer thread arrives after its copies landed and a proxy fence) and
+// freed on empty[s] by tcgen05.commit.
 // ---------------------------------------------------------------------------
 template <int W> struct Elem { using T = __half; };
 template <> struct Elem<1> { using T = __nv_bfloat16; };
 template <typename T> __device__ __forceinline__ T from_f(float x);
 template <> __device__ __forceinline__ __half from_f<__half>(float x) { return __float2half_rn(x); }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+struct RawI4 {
+    uint2 q[4];
+    unsigned short sc[4];
+};
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *b)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(s2u(b)) : "memory");
+}
 
 template <int KIND, int W>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant__ GemmParams p)
@@ -217,9 +242,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     AT *Hbuf = reinterpret_cast<AT *>(p.H);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t bars[NSTAGE];
+    __shared__ uint64_t full[NSTAGE], empty[NSTAGE], done;
     __shared__ uint32_t tmem_base_sh;
-    __shared__ int abort_sh;
+    __shared__ volatile int abort_sh;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int d = p.d, F = p.F;
@@ -246,14 +271,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     const int nk_all = K / BK;
     const int ksplit = KIND == kGU ? 1 : kSplitK;
     const int kt0 = int((long long)blockIdx.z * nk_all / ksplit), kt1 = int((long long)(blockIdx.z + 1) * nk_all / ksplit);
+    const int nk = kt1 - kt0;
     const int n0 = blockIdx.x * BN;   // GU: B-row 2j/2j+1 = gate/up of neuron n0/2 + j
 
     if (tid == 0) {
-        for (int s = 0; s < NSTAGE; ++s) mbar_init(&bars[s], 1);
+        for (int s = 0; s < NSTAGE; ++s) {
+            mbar_init(&full[s], kProducers);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(&done, 1);
         abort_sh = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 0) {
+    if (warp == kProducerWarps) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      ::"r"(s2u(&tmem_base_sh)), "r"(BN) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -263,160 +293,196 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = tmem_base_sh;
 
-    // ---- stage loader: A (activations, K-major) and B (weights) ------------
-    auto load_stage = [&](int kt, int s) {
-        uint8_t *A = smem + s * kStageBytes;
-        uint8_t *B = A + kATileBytes;
-        const int k0 = kt * BK;
-        // A: 128 rows x 8 chunks of 16 bytes
-        for (int c = tid; c < BM * (BK / 8); c += kGemmThreads) {
-            const int row = c >> 3, kc = c & 7;
-            const int lr = mrow0 + row;
-            const bool ok = lr < mrow_end;
-            const AT *src;
-            if (KIND == kGU) src = X16 + size_t(ok ? p.e_tok[lr] : 0) * d + k0 + kc * 8;
-            else src = Hbuf + size_t(ok ? lr : 0) * F + k0 + kc * 8;
-            cp_async16(A + kmaj_off(row, kc), src, ok);
-        }
-        if constexpr (KIND == kGU) {
-            // B: 256 rows (neuron n0/2 + row/2; gate for even rows, up for odd) x 64 k, K-major
+    if (warp < kProducerWarps) {
+        // ------------------------------ producers ------------------------------
+        const int pt = tid;   // 0 .. 255
+        auto issue_async = [&](int kt, int s) {
+            uint8_t *A = smem + s * kStageBytes;
+            uint8_t *B = A + kATileBytes;
+            const int k0 = kt * BK;
+#pragma unroll
+            for (int i = 0; i < BM * (BK / 8) / kProducers; ++i) {   // A: 128 rows x 8 chunks
+                const int c = pt + kProducers * i, row = c >> 3, kc = c & 7;
+                const int lr = mrow0 + row;
+                const bool ok = lr < mrow_end;
+                const AT *src;
+                if (KIND == kGU) src = X16 + size_t(ok ? p.e_tok[lr] : 0) * d + k0 + kc * 8;
+                else src = Hbuf + size_t(ok ? lr : 0) * F + k0 + kc * 8;
+                cp_async16(A + kmaj_off(row, kc), src, ok);
+            }
             if constexpr (!I4) {
-                for (int c = tid; c < BN * (BK / 8); c += kGemmThreads) {
-                    const int row = c >> 3, kc = c & 7;
-                    const int nn = n0 / 2 + (row >> 1);
-                    const bool ok = nn < F && (p.gated || (row & 1) == 0);
-                    const uint8_t *rec = ex.Wgu + size_t(ok ? nn : 0) * p.gu_bytes + ((row & 1) ? p.wrow : 0);
-                    cp_async16(B + kmaj_off(row, kc), rec + (k0 + kc * 8) * 2, ok);
+                if constexpr (KIND == kGU) {
+#pragma unroll
+                    for (int i = 0; i < BN * (BK / 8) / kProducers; ++i) {   // 256 rows x 8 chunks, K-major
+                        const int c = pt + kProducers * i, row = c >> 3, kc = c & 7;
+                        const int nn = n0 / 2 + (row >> 1);
+                        const bool ok = nn < F && (p.gated || (row & 1) == 0);
+                        const uint8_t *rec = ex.Wgu + size_t(ok ? nn : 0) * p.gu_bytes + ((row & 1) ? p.wrow : 0);
+                        cp_async16(B + kmaj_off(row, kc), rec + (k0 + kc * 8) * 2, ok);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < BK * (BN / 8) / kProducers; ++i) {   // 64 k-rows x 32 chunks, MN-major
+                        const int c = pt + kProducers * i, k = c / (BN / 8), ng = c % (BN / 8);
+                        const uint8_t *row = ex.Wd + size_t(k0 + k) * p.wrow + (n0 + ng * 8) * 2;
+                        cp_async16(B + mnmaj_off(ng, k), row, true);
+                    }
                 }
-            } else {
-                // one thread per (row, 16-element half of the 64-wide stage)... 4 per row
-                for (int c = tid; c < BN * 4; c += kGemmThreads) {
+            }
+            cp_async_commit();
+        };
+        // INT4: the raw nibbles and scales of a stage, loaded into registers
+        auto load_raw = [&](int kt, RawI4 &r) {
+            const int k0 = kt * BK;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int c = pt + kProducers * i;
+                if constexpr (KIND == kGU) {
                     const int row = c >> 2, q16 = c & 3;       // elements k0 + 16 q16 .. +15
                     const int nn = n0 / 2 + (row >> 1);
                     const bool ok = nn < F && (p.gated || (row & 1) == 0);
-                    uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
+                    r.q[i] = make_uint2(0u, 0u);
+                    r.sc[i] = 0;
                     if (ok) {
                         const uint8_t *rec = ex.Wgu + size_t(nn) * p.gu_bytes + ((row & 1) ? p.wrow : 0);
                         const int kk = k0 + 16 * q16;
-                        const uint2 q = *reinterpret_cast<const uint2 *>(rec + kk / 2);
-                        const float sc = __half2float(*reinterpret_cast<const __half *>(rec + d / 2 + (kk / 32) * 2));
-                        dequant16(q, sc, lo, hi);
+                        r.q[i] = __ldg(reinterpret_cast<const uint2 *>(rec + kk / 2));
+                        r.sc[i] = __ldg(reinterpret_cast<const unsigned short *>(rec + d / 2) + kk / 32);
                     }
-                    *reinterpret_cast<uint4 *>(B + kmaj_off(row, 2 * q16)) = lo;
-                    *reinterpret_cast<uint4 *>(B + kmaj_off(row, 2 * q16 + 1)) = hi;
-                }
-            }
-        } else {
-            // B (down): n = output column j in [n0, n0 + 256), k = neuron i in [k0, k0 + 64):
-            // W_down neuron-major rows give 8 consecutive n per 16 bytes (MN-major)
-            if constexpr (!I4) {
-                for (int c = tid; c < BK * (BN / 8); c += kGemmThreads) {
-                    const int k = c / (BN / 8), ng = c % (BN / 8);
-                    const uint8_t *row = ex.Wd + size_t(k0 + k) * p.wrow + (n0 + ng * 8) * 2;
-                    cp_async16(B + mnmaj_off(ng, k), row, true);
-                }
-            } else {
-                for (int c = tid; c < BK * (BN / 16); c += kGemmThreads) {
-                    const int k = c / (BN / 16), g16 = c % (BN / 16);   // 16 n-values
+                } else {
+                    const int k = c / (BN / 16), g16 = c % (BN / 16);   // 16 n-values of W_down row k0 + k
                     const uint8_t *row = ex.Wd + size_t(k0 + k) * p.wrow;
                     const int nn = n0 + 16 * g16;
-                    const uint2 q = *reinterpret_cast<const uint2 *>(row + nn / 2);
-                    const float sc = __half2float(*reinterpret_cast<const __half *>(row + d / 2 + (nn / 32) * 2));
-                    uint4 lo, hi;
-                    dequant16(q, sc, lo, hi);
+                    r.q[i] = __ldg(reinterpret_cast<const uint2 *>(row + nn / 2));
+                    r.sc[i] = __ldg(reinterpret_cast<const unsigned short *>(row + d / 2) + nn / 32);
+                }
+            }
+        };
+        auto store_raw = [&](const RawI4 &r, int s) {
+            uint8_t *B = smem + s * kStageBytes + kATileBytes;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int c = pt + kProducers * i;
+                uint4 lo, hi;
+                dequant16(r.q[i], __ushort_as_half(r.sc[i]), lo, hi);
+                if constexpr (KIND == kGU) {
+                    const int row = c >> 2, q16 = c & 3;
+                    *reinterpret_cast<uint4 *>(B + kmaj_off(row, 2 * q16)) = lo;
+                    *reinterpret_cast<uint4 *>(B + kmaj_off(row, 2 * q16 + 1)) = hi;
+                } else {
+                    const int k = c / (BN / 16), g16 = c % (BN / 16);
                     *reinterpret_cast<uint4 *>(B + mnmaj_off(2 * g16, k)) = lo;
                     *reinterpret_cast<uint4 *>(B + mnmaj_off(2 * g16 + 1, k)) = hi;
                 }
             }
+        };
+        // publish stage `j`: its copies have landed (cp.async group), make
+        // them and the dequantised stores visible to the tensor core, arrive
+        auto publish = [&](int j) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            mbar_arrive(&full[j % NSTAGE]);
+        };
+        RawI4 raw_cur{}, raw_next{};
+        if constexpr (I4) {
+            if (nk > 0) load_raw(kt0, raw_cur);
         }
-        cp_async_commit();
-    };
-
-    const uint32_t idesc = make_idesc(KIND == kDOWN, W == 1);
-    const int nk = kt1 - kt0;
-    bool ok = true;
-    int j_issued = 0;   // last step whose MMAs were issued and committed
-    // prologue: stages 0 and 1 in flight
-    for (int j = 0; j < 2 && j < nk; ++j) load_stage(kt0 + j, j);
-    for (int j = 0; j < nk; ++j) {
-        const int s = j % NSTAGE;
-        if (j + 1 < nk) cp_async_wait<1>();
-        else cp_async_wait<0>();
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncthreads();
-        if (tid == 0) {
-            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            const uint32_t a0 = s2u(smem + s * kStageBytes), b0 = a0 + kATileBytes;
-#pragma unroll
-            for (int ks = 0; ks < BK / 16; ++ks) {
-                const uint64_t ad = make_sdesc(a0 + ks * 256, 128, BK / 8 * 128);
-                const uint64_t bd = make_sdesc(b0 + ks * 256, 128, BK / 8 * 128);
-                umma(tmem, ad, bd, idesc, j > 0 || ks > 0);
+        int j = 0;
+        for (; j < nk; ++j) {
+            const int s = j % NSTAGE;
+            if (j >= NSTAGE) {
+                // the MMAs of step j - NSTAGE read this stage
+                if (!mbar_wait(&empty[s], uint32_t(((j - NSTAGE) / NSTAGE) & 1), p.err)) abort_sh = 1;
             }
-            umma_commit(&bars[s]);
-        }
-        j_issued = j;
-        // refill the stage freed by the MMAs of step j - 1
-        if (j + 2 < nk) {
-            const int sn = (j + 2) % NSTAGE;
-            if (j + 2 >= NSTAGE) {
-                // that stage was last read by the MMAs of step j + 2 - NSTAGE
-                const uint32_t par = uint32_t(((j + 2 - NSTAGE) / NSTAGE) & 1);
-                if (tid == 0 && !mbar_wait(&bars[sn], par, p.err)) abort_sh = 1;
-                __syncthreads();
-                if (abort_sh) { ok = false; break; }
+            if (abort_sh) break;
+            issue_async(kt0 + j, s);
+            if constexpr (I4) {
+                if (j + 1 < nk) load_raw(kt0 + j + 1, raw_next);
+                store_raw(raw_cur, s);
+                raw_cur = raw_next;
             }
-            load_stage(kt0 + j + 2, sn);
+            if (j >= kLag) {
+                cp_async_wait<kLag>();
+                publish(j - kLag);
+            }
         }
-    }
-    // all MMAs done: the last commit covers every earlier MMA of this thread.
-    // After a timed-out wait this is the (again bounded) drain of the MMAs in
-    // flight before TMEM is released.
-    cp_async_wait<0>();
-    if (nk > 0 && tid == 0) {
-        const int last = ok ? nk - 1 : j_issued;
-        if (!mbar_wait(&bars[last % NSTAGE], uint32_t((last / NSTAGE) & 1), p.err)) abort_sh = 1;
-    }
-    __syncthreads();
-    ok = ok && !abort_sh;
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-
-    // ---- epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31, columns half (w / 4)
-    if (ok && nk > 0) {
+        // drain: publish the stages still in flight (all of them on abort too,
+        // so that no copy is outstanding at exit)
+        cp_async_wait<0>();
+        for (int q = max(0, j - kLag); q < j; ++q) publish(q);
+        // epilogue: wait for the accumulator
+        if (nk > 0 && !abort_sh && !mbar_wait(&done, 0u, p.err)) abort_sh = 1;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const int row = 32 * (warp & 3) + lane;
         const int lr = mrow0 + row;
-        const bool valid = lr < mrow_end;
+        const bool valid = lr < mrow_end && !abort_sh;
         const int col0 = 128 * (warp >> 2);
-        for (int cc = 0; cc < 128; cc += 16) {
-            float v[16];
-            tmem_ld16(tmem + (uint32_t(32 * (warp & 3)) << 16) + uint32_t(col0 + cc), v);
-            if (!valid) continue;
-            if constexpr (KIND == kGU) {
-                // columns 2j, 2j+1 = gate, up of neuron n0/2 + (col0 + cc)/2 + j
-                const int nb = n0 / 2 + (col0 + cc) / 2;
-                AT hv[8];
+        if (KIND == kDOWN && nk == 0) {
+            // an empty K range still owns its partial: zeros
+            if (valid) {
+                float *dst = p.Ypart + (size_t(blockIdx.z) * p.rows_cap + lr) * d + n0 + col0;
+                for (int j2 = 0; j2 < 128; j2 += 4) *reinterpret_cast<float4 *>(dst + j2) = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        } else if (!abort_sh) {
+            for (int cc = 0; cc < 128; cc += 16) {
+                float v[16];
+                tmem_ld16(tmem + (uint32_t(32 * (warp & 3)) << 16) + uint32_t(col0 + cc), v);
+                if (!valid) continue;
+                if constexpr (KIND == kGU) {
+                    // columns 2j, 2j+1 = gate, up of neuron n0/2 + (col0 + cc)/2 + j
+                    const int nb = n0 / 2 + (col0 + cc) / 2;
+                    AT hv[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int nn = nb + j;
-                    float g = v[2 * j] - (nn < F ? __ldg(ex.c + nn) : 0.f);
-                    float u = v[2 * j + 1];
-                    const float gp = g > 0.f ? g : 0.f;
-                    float h = p.act == 0 ? gp : (p.act == 1 ? gp * u : gp * (u > 0.f ? u : 0.f));
-                    hv[j] = from_f<AT>(h);
+                    for (int j2 = 0; j2 < 8; ++j2) {
+                        const int nn = nb + j2;
+                        const float g = v[2 * j2] - (nn < F ? __ldg(ex.c + nn) : 0.f);
+                        const float u = v[2 * j2 + 1];
+                        const float gp = g > 0.f ? g : 0.f;
+                        const float h = p.act == 0 ? gp : (p.act == 1 ? gp * u : gp * (u > 0.f ? u : 0.f));
+                        hv[j2] = from_f<AT>(h);
+                    }
+                    if (nb + 8 <= F)
+                        *reinterpret_cast<uint4 *>(Hbuf + size_t(lr) * F + nb) = *reinterpret_cast<uint4 *>(hv);
+                } else {
+                    float *dst = p.Ypart + (size_t(blockIdx.z) * p.rows_cap + lr) * d + n0 + col0 + cc;
+#pragma unroll
+                    for (int j2 = 0; j2 < 16; j2 += 4)
+                        *reinterpret_cast<float4 *>(dst + j2) = make_float4(v[j2], v[j2 + 1], v[j2 + 2], v[j2 + 3]);
                 }
-                if (nb + 8 <= F)
-                    *reinterpret_cast<uint4 *>(Hbuf + size_t(lr) * F + nb) = *reinterpret_cast<uint4 *>(hv);
-            } else {
-                float *dst = p.Ypart + (size_t(blockIdx.z) * p.rows_cap + lr) * d + n0 + col0 + cc;
-#pragma unroll
-                for (int j = 0; j < 16; j += 4)
-                    *reinterpret_cast<float4 *>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
             }
         }
+    } else if (warp == kProducerWarps && nk > 0) {
+        // ------------------------------ MMA issue ------------------------------
+        if (lane == 0) {
+            const uint32_t idesc = make_idesc(KIND == kDOWN, W == 1);
+            int issued = 0;
+            for (int j = 0; j < nk; ++j) {
+                const int s = j % NSTAGE;
+                if (!mbar_wait(&full[s], uint32_t((j / NSTAGE) & 1), p.err)) { abort_sh = 1; break; }
+                if (abort_sh) break;
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                const uint32_t a0 = s2u(smem + s * kStageBytes), b0 = a0 + kATileBytes;
+#pragma unroll
+                for (int ks = 0; ks < BK / 16; ++ks) {
+                    const uint64_t ad = make_sdesc(a0 + ks * 256, 128, BK / 8 * 128);
+                    const uint64_t bd = make_sdesc(b0 + ks * 256, 128, BK / 8 * 128);
+                    umma(tmem, ad, bd, idesc, j > 0 || ks > 0);
+                }
+                umma_commit(&empty[s]);
+                issued = j + 1;
+            }
+            // the accumulator is complete when every issued MMA is: one more
+            // commit (it tracks all earlier MMAs of this thread)
+            umma_commit(&done);
+            if (issued < nk) {
+                // aborted: let the issued MMAs finish (bounded) before TMEM is freed
+                mbar_wait(&done, 0u, p.err);
+            }
+        }
+        __syncwarp();
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
-    if (warp == 0)
+    if (warp == kProducerWarps)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BN) : "memory");
 }
 
