@@ -296,25 +296,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     if (warp < kProducerWarps) {
         // ------------------------------ producers ------------------------------
         const int pt = tid;   // 0 .. 255
+        // Chunk-to-lane mapping: a warp covers 8 consecutive rows x 4
+        // consecutive 16-byte chunks, so its global reads are whole 32-byte
+        // sectors and its shared stores are four 128-byte runs (no bank
+        // conflicts beyond the minimum).  Item i of this thread: rows from
+        // (c >> 5) and c & 7, chunks from (c >> 3) & 3, with c = pt + 256 i.
+        // Source rows do not change across K steps: resolved once here.
+        constexpr int kAI = BM * (BK / 8) / kProducers;    // 4 A chunks per thread per stage
+        const uint8_t *a_src[kAI];
+        uint32_t a_dst[kAI];
+        bool a_ok[kAI];
+#pragma unroll
+        for (int i = 0; i < kAI; ++i) {
+            const int c = pt + kProducers * i, rest = c >> 5;
+            const int row = (rest & 15) * 8 + (c & 7), kc = (rest >> 4) * 4 + ((c >> 3) & 3);
+            const int lr = mrow0 + row;
+            a_ok[i] = lr < mrow_end;
+            const AT *src = KIND == kGU ? X16 + size_t(a_ok[i] ? p.e_tok[lr] : 0) * d
+                                        : Hbuf + size_t(a_ok[i] ? lr : 0) * F;
+            a_src[i] = reinterpret_cast<const uint8_t *>(src) + kc * 16;
+            a_dst[i] = kmaj_off(row, kc);
+        }
         auto issue_async = [&](int kt, int s) {
             uint8_t *A = smem + s * kStageBytes;
             uint8_t *B = A + kATileBytes;
             const int k0 = kt * BK;
 #pragma unroll
-            for (int i = 0; i < BM * (BK / 8) / kProducers; ++i) {   // A: 128 rows x 8 chunks
-                const int c = pt + kProducers * i, row = c >> 3, kc = c & 7;
-                const int lr = mrow0 + row;
-                const bool ok = lr < mrow_end;
-                const AT *src;
-                if (KIND == kGU) src = X16 + size_t(ok ? p.e_tok[lr] : 0) * d + k0 + kc * 8;
-                else src = Hbuf + size_t(ok ? lr : 0) * F + k0 + kc * 8;
-                cp_async16(A + kmaj_off(row, kc), src, ok);
-            }
+            for (int i = 0; i < kAI; ++i) cp_async16(A + a_dst[i], a_src[i] + k0 * 2, a_ok[i]);
             if constexpr (!I4) {
                 if constexpr (KIND == kGU) {
 #pragma unroll
                     for (int i = 0; i < BN * (BK / 8) / kProducers; ++i) {   // 256 rows x 8 chunks, K-major
-                        const int c = pt + kProducers * i, row = c >> 3, kc = c & 7;
+                        const int c = pt + kProducers * i, rest = c >> 5;
+                        const int row = (rest & 31) * 8 + (c & 7), kc = (rest >> 5) * 4 + ((c >> 3) & 3);
                         const int nn = n0 / 2 + (row >> 1);
                         const bool ok = nn < F && (p.gated || (row & 1) == 0);
                         const uint8_t *rec = ex.Wgu + size_t(ok ? nn : 0) * p.gu_bytes + ((row & 1) ? p.wrow : 0);
@@ -323,7 +337,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
                 } else {
 #pragma unroll
                     for (int i = 0; i < BK * (BN / 8) / kProducers; ++i) {   // 64 k-rows x 32 chunks, MN-major
-                        const int c = pt + kProducers * i, k = c / (BN / 8), ng = c % (BN / 8);
+                        const int c = pt + kProducers * i, rest = c >> 5;
+                        const int k = (rest & 7) * 8 + (c & 7), ng = (rest >> 3) * 4 + ((c >> 3) & 3);
                         const uint8_t *row = ex.Wd + size_t(k0 + k) * p.wrow + (n0 + ng * 8) * 2;
                         cp_async16(B + mnmaj_off(ng, k), row, true);
                     }
@@ -331,7 +346,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
             }
             cp_async_commit();
         };
-        // INT4: the raw nibbles and scales of a stage, loaded into registers
+        // INT4: the raw nibbles and scales of a stage, loaded into registers.
+        // GU item: row c >> 2, 16 elements at chunk pair c & 3 (a warp: 8 rows
+        // x 32 contiguous bytes).  Down item: W_down row k (8 per warp) and 16
+        // output columns (4 consecutive groups per row).
         auto load_raw = [&](int kt, RawI4 &r) {
             const int k0 = kt * BK;
 #pragma unroll
@@ -350,7 +368,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
                         r.sc[i] = __ldg(reinterpret_cast<const unsigned short *>(rec + d / 2) + kk / 32);
                     }
                 } else {
-                    const int k = c / (BN / 16), g16 = c % (BN / 16);   // 16 n-values of W_down row k0 + k
+                    const int rest = c >> 5;
+                    const int k = (rest & 7) * 8 + (c & 7), g16 = (rest >> 3) * 4 + ((c >> 3) & 3);
                     const uint8_t *row = ex.Wd + size_t(k0 + k) * p.wrow;
                     const int nn = n0 + 16 * g16;
                     r.q[i] = __ldg(reinterpret_cast<const uint2 *>(row + nn / 2));
@@ -370,7 +389,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
                     *reinterpret_cast<uint4 *>(B + kmaj_off(row, 2 * q16)) = lo;
                     *reinterpret_cast<uint4 *>(B + kmaj_off(row, 2 * q16 + 1)) = hi;
                 } else {
-                    const int k = c / (BN / 16), g16 = c % (BN / 16);
+                    const int rest = c >> 5;
+                    const int k = (rest & 7) * 8 + (c & 7), g16 = (rest >> 3) * 4 + ((c >> 3) & 3);
                     *reinterpret_cast<uint4 *>(B + mnmaj_off(2 * g16, k)) = lo;
                     *reinterpret_cast<uint4 *>(B + mnmaj_off(2 * g16 + 1, k)) = hi;
                 }
