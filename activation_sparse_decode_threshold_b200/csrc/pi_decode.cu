@@ -28,6 +28,7 @@ cudaError_t dispatch(int wfmt, int pfmt, int d, int mode, const DecodeParams &p,
 
 int decode_mode(const DecodeParams &p)
 {
+    if (p.mode == kModePredict) return kModePred | (p.E > 1 ? kModeMoE : 0);
     return (p.E > 1 ? kModeMoE : 0) | (p.gated ? kModeGated : 0) | (p.spec_down ? kModeSpec : 0);
 }
 

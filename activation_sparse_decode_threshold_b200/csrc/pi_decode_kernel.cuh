@@ -272,6 +272,7 @@ constexpr int kRA = 16;           // V rows per staging round at most
 constexpr int kZRows = 96;        // U rows per staging round at most (a multiple of 16)
 constexpr int kMaxU = 4;          // U vectors per lane (rank <= 128 * EPV)
 constexpr int kRound = 16;        // neurons per gather round at most
+static_assert(kRound <= 32, "a round's neurons are tracked in one warp ballot");
 constexpr int kRed = 2 * kRound;  // values reduced per warp at most
 
 struct Smem {
@@ -412,11 +413,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     const int b = blockIdx.x, S = gridDim.x;
     const int d = p.d, r = p.r;
     const int s0 = p.strip_off[b], ns = p.strip_off[b + 1] - s0;
-    const bool predict = p.mode == kModePredict;
     // layer kind, fixed per instantiation so each kernel holds only its path
     constexpr bool moe = (MODE & kModeMoE) != 0;
     constexpr bool kGated = (MODE & kModeGated) != 0;
     constexpr bool kSpec = (MODE & kModeSpec) != 0;
+    constexpr bool predict = (MODE & kModePred) != 0;   // pi_predict: one layer, stop after the list
     const int ntop = predict ? 1 : p.top_k;
     const int nvecW = (WF == kI4 ? d / 2 : d * (WF == kF32 ? 4 : 2)) / VBW;
     const int nvecP = p.vrow / VBP;
@@ -1014,7 +1015,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             return a;
         };
 
-        prof_put(p, li, 8, gtimer());
         bool gok = true;
         int nz_total = 0;            // neurons with h != 0 so far (list order)
         for (int j0 = 0; j0 < m && gok; j0 += cap_n) {
@@ -1033,11 +1033,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                                    &sm.stage_bar);
                 }
             }
-            if (j0 == 0) prof_put(p, li, 14, gtimer());
             pending = true;
             if (!stage_wait(&sm, p, spar, bci, &cyc_c)) { gok = false; break; }
             pending = false;
-            if (j0 == 0) prof_put(p, li, 15, gtimer());
             // dots of the round's neurons, four at a time: values 2n (gate) and
             // 2n + 1 (up); after the reduction lanes 4q .. 4q + 3 hold value q
 #pragma unroll 1
@@ -1057,9 +1055,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 const int q = 2 * g0 + (lane >> 2);
                 if ((lane & 3) == 0 && q < 2 * k) sm.red[rb][warp][q] = ws;
             }
-            if (j0 == 0) prof_put(p, li, 16, gtimer());
             cta_sync();
-            if (j0 == 0) prof_put(p, li, 17, gtimer());
             if (tid < 2 * k) {
                 float a = 0.f;
                 for (int w = 0; w < kConsumerWarps; ++w) a += sm.red[rb][w][tid];
@@ -1067,32 +1063,63 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             }
             rb ^= 1;
             cta_sync();
-            if (j0 == 0) prof_put(p, li, 18, gtimer());
             if (tid < k) {
                 const int en = entry(j0 + tid), e = en >> 12, loc = en & 0xfff;
                 sm.rh[tid] = act_h(p.act, sm.rsum[2 * tid] - sm.cbuf[e][loc], sm.rsum[2 * tid + 1]) *
                              sm.route_w[e];
             }
             cta_sync();
-            if (j0 == 0) prof_put(p, li, 19, gtimer());
-            // neurons with h != 0, in list order
-            int nz_round = 0;
-            for (int n = 0; n < k; ++n) {
-                const float h = sm.rh[n];
-                if (h == 0.f) continue;
-                if (tid == 0) {
-                    sm.nz[nz_total + nz_round] = int16_t(entry(j0 + n));
-                    sm.hz[nz_total + nz_round] = h;
+            // neurons with h != 0, in list order (every warp forms the same
+            // ballot; warp 0 records them)
+            const bool nzv = lane < k && sm.rh[lane] != 0.f;
+            const unsigned nzm = __ballot_sync(0xffffffffu, nzv);
+            if (warp == 0 && nzv) {
+                const int pos = nz_total + __popc(nzm & ((1u << lane) - 1u));
+                sm.nz[pos] = int16_t(entry(j0 + lane));
+                sm.hz[pos] = sm.rh[lane];
+            }
+            const int nz_round = __popc(nzm);
+            if constexpr (kSpec) {
+                // acc += h * W_down row, kAG neurons at a time: their row
+                // vectors are loaded before any of them is accumulated
+                constexpr int kAG = MAXVW > 1 ? 2 : 4;
+#pragma unroll 1
+                for (int g0 = 0; g0 < k; g0 += kAG) {
+                    float hv[kAG];
+                    VW q[kAG][MAXVW];
+#pragma unroll
+                    for (int j = 0; j < kAG; ++j) {
+                        hv[j] = g0 + j < k ? sm.rh[g0 + j] : 0.f;
+                        const uint8_t *row = stg + size_t(g0 + j) * per_n + p.gu_bytes;
+#pragma unroll
+                        for (int kk = 0; kk < MAXVW; ++kk) {
+                            const int v = tid + kThreads * kk;
+                            if (hv[j] != 0.f && v < nvecW) q[j][kk] = *reinterpret_cast<const VW *>(row + v * VBW);
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < kAG; ++j) {
+                        if (hv[j] == 0.f) continue;
+                        const uint8_t *row = stg + size_t(g0 + j) * per_n + p.gu_bytes;
+#pragma unroll
+                        for (int kk = 0; kk < MAXVW; ++kk) {
+                            const int v = tid + kThreads * kk;
+                            if (v < nvecW) {
+                                float w[EPVW];
+                                cvt<WF>(q[j][kk], w);
+                                float hs = hv[j];
+                                if constexpr (WF == kI4)
+                                    hs *= __half2float(*reinterpret_cast<const __half *>(row + d / 2 + (v >> 1) * 2));
+#pragma unroll
+                                for (int i = 0; i < EPVW; ++i) acc[kk * EPVW + i] = fmaf(hs, w[i], acc[kk * EPVW + i]);
+                            }
+                        }
+                    }
                 }
-                ++nz_round;
-                if (kSpec) axpy_smem(stg + size_t(n) * per_n + p.gu_bytes, h);
             }
             nz_total += nz_round;
-            if (j0 == 0) prof_put(p, li, 20, gtimer());
             cta_sync();   // the staging buffer is reused by the next round
-            if (j0 == 0) prof_put(p, li, 21, gtimer());
         }
-        prof_put(p, li, 22, gtimer());
         // not speculative: the W_down rows of the neurons with h != 0, in rounds
         if (gok && !kSpec) {
             const int cap_d = min(kMaxTopK * kMaxStrip, kStageBytes / p.wrow);
@@ -1144,7 +1171,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             }
         }
         (void)cc0;
-        prof_put(p, li, 23, gtimer());
         prof_put(p, li, 3, gtimer());
         if (!grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
         prof_put(p, li, 4, gtimer());
@@ -1194,6 +1220,8 @@ cudaError_t launch_mode(int mode, const DecodeParams &p, cudaStream_t st, bool q
     case kModeMoE | kModeGated | kModeSpec:
         return launch_one<WF, PF, DMAX, kModeMoE | kModeGated | kModeSpec>(p, st, query, blocks);
     case kModeMoE | kModeGated: return launch_one<WF, PF, DMAX, kModeMoE | kModeGated>(p, st, query, blocks);
+    case kModePred: return launch_one<WF, PF, DMAX, kModePred>(p, st, query, blocks);
+    case kModePred | kModeMoE: return launch_one<WF, PF, DMAX, kModePred | kModeMoE>(p, st, query, blocks);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -74,8 +74,8 @@ struct DecodeParams {
 
 // Phase timestamps recorded per layer and CTA when DecodeParams::prof is set.
 // layer kinds (bits of the decode kernel's MODE parameter)
-constexpr int kModeMoE = 1, kModeGated = 2, kModeSpec = 4;
-constexpr int kProfPoints = 24;   // timestamps and cycle counters per layer and CTA
+constexpr int kModeMoE = 1, kModeGated = 2, kModeSpec = 4, kModePred = 8;
+constexpr int kProfPoints = 14;   // timestamps and cycle counters per layer and CTA
 
 cudaError_t launch_decode(int wfmt, int pfmt, const DecodeParams &p, cudaStream_t stream);
 int decode_max_blocks_per_sm(int wfmt, int pfmt, int d);

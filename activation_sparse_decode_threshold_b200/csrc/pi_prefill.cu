@@ -402,28 +402,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             mbar_arrive(&full[j % NSTAGE]);
         };
-        RawI4 raw_cur{}, raw_next{};
+        // INT4 raw data of stage j is loaded three steps ahead, rotating
+        // through four register sets (no dynamic indexing)
+        RawI4 ra{}, rb{}, rc{}, rd{};
         if constexpr (I4) {
-            if (nk > 0) load_raw(kt0, raw_cur);
+            if (nk > 0) load_raw(kt0, ra);
+            if (nk > 1) load_raw(kt0 + 1, rb);
+            if (nk > 2) load_raw(kt0 + 2, rc);
         }
         int j = 0;
-        for (; j < nk; ++j) {
+        bool stop = nk == 0;
+        auto step = [&](RawI4 &cur, RawI4 &nxt) {
+            if (stop) return;
             const int s = j % NSTAGE;
             if (j >= NSTAGE) {
                 // the MMAs of step j - NSTAGE read this stage
                 if (!mbar_wait(&empty[s], uint32_t(((j - NSTAGE) / NSTAGE) & 1), p.err)) abort_sh = 1;
             }
-            if (abort_sh) break;
+            if (abort_sh) { stop = true; return; }
             issue_async(kt0 + j, s);
             if constexpr (I4) {
-                if (j + 1 < nk) load_raw(kt0 + j + 1, raw_next);
-                store_raw(raw_cur, s);
-                raw_cur = raw_next;
+                if (j + 3 < nk) load_raw(kt0 + j + 3, nxt);
+                store_raw(cur, s);
             }
             if (j >= kLag) {
                 cp_async_wait<kLag>();
                 publish(j - kLag);
             }
+            if (++j >= nk) stop = true;
+        };
+        while (!stop) {
+            step(ra, rd);
+            step(rb, ra);
+            step(rc, rb);
+            step(rd, rc);
         }
         // drain: publish the stages still in flight (all of them on abort too,
         // so that no copy is outstanding at exit)

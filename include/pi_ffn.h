@@ -208,17 +208,14 @@ PI_API pi_status pi_debug_set(pi_ffn_t h, int flags, double wait_limit_s);
 /* Testing aid: when `times_dev` is non-NULL, each later pi_sparse_ffn_decode
  * call records, per layer and CTA, %globaltimer (ns) at these points k:
  *   0 layer start, 1 layer input and t ready, 9 predictor logits done,
- *   2 active list done, 8 gather start, 14 first gather round's copies
- *   issued, 15 its rows landed, 16 its dots done, 17 its warp sums stored,
- *   18 its row sums, 19 its h, 20 its W_down accumulation, 21 its end,
- *   22 all gather rounds done, 23 partial stored, 3 gather done, 4 after the
- *   gather barrier, 7 partials reduced, 5 column phase done, 6 after the
- *   column barrier;
+ *   2 active list done, 3 gather done, 4 after the gather barrier,
+ *   7 partials reduced, 5 column phase done, 6 after the column barrier
+ *   (8 unused);
  * and k = 10..13 the clock cycles thread 0 spent obtaining the layer input,
  * waiting for predictor rows, waiting for gathered rows and waiting in grid
  * barriers.  Value (layer - layer_begin, k, cta) sits at
- * times_dev[((layer - layer_begin) * 24 + k) * n_strips + cta].  The buffer
- * (caller-owned, device, 8-byte aligned) must hold (l1 - l0) * 24 * n_strips
+ * times_dev[((layer - layer_begin) * 14 + k) * n_strips + cta].  The buffer
+ * (caller-owned, device, 8-byte aligned) must hold (l1 - l0) * 14 * n_strips
  * values.  NULL turns recording off. */
 PI_API pi_status pi_debug_phase_times(pi_ffn_t h, long long *times_dev);
 
