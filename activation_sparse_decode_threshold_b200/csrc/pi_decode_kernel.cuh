@@ -319,33 +319,43 @@ __device__ __forceinline__ void fix_add(long long *dst, float v, float scale)
 constexpr float kFixT = 4294967296.0f;    // 2^32
 constexpr float kFixSS = 16777216.0f;     // 2^24
 
-// Grid-wide barrier of all CTAs of the cooperative launch: arrivals are
-// fire-and-forget releases on one counter (never reset within a launch);
-// thread 0 of each CTA polls it with acquire loads, bounded by wait_ns.  The
-// outcome is broadcast through shared memory so the whole CTA agrees.
+// Grid-wide barrier of all CTAs of the cooperative launch.  Arrivals are
+// spread over kBarLanes counters, one 128-byte line each (CTA b arrives on
+// counter b mod kBarLanes), so that they do not serialise on one L2 line;
+// the counters are never reset within a launch.  Thread 0 arrives with a
+// release (after the block barrier, so it carries the whole CTA's writes);
+// warp 0 then polls all counters at once, lane i reading counter i with an
+// acquire, bounded by wait_ns, and the verdict is broadcast through shared
+// memory so the whole CTA agrees.
 __device__ bool grid_sync(Smem *sm, const DecodeParams &p, unsigned &epoch, int &bci, long long *cyc)
 {
     cta_sync();
-    if (threadIdx.x == 0) {
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
         const long long c0 = clock64();
-        bool ok = true;
         epoch += 1;
-        unsigned target = epoch * gridDim.x;
-        if ((p.debug_flags & 1) && epoch == 1) target += 1;   // PI_DEBUG_STALL_BARRIER
-        __threadfence();
-        red_release_gpu(p.bar, 1u);
+        if (lane == 0) red_release_gpu(p.bar + (blockIdx.x % kBarLanes) * kBarStride, 1u);
+        // CTAs per counter: S / kBarLanes, one more for the first S % kBarLanes
+        const unsigned S = gridDim.x;
+        unsigned target = lane < kBarLanes ? epoch * (S / kBarLanes + (unsigned(lane) < S % kBarLanes ? 1u : 0u)) : 0u;
+        if ((p.debug_flags & 1) && epoch == 1 && lane == 0) target += 1;   // PI_DEBUG_STALL_BARRIER
+        const unsigned *ctr = p.bar + (lane < kBarLanes ? lane : 0) * kBarStride;
+        bool ok = true;
         const long long t0 = gtimer();
-        unsigned it = 0;
-        while (ld_acquire_gpu(p.bar) < target) {
-            if ((++it & 31) == 0 && gtimer() - t0 > p.wait_ns) {
-                set_error(p.err, kDevTimeout);
+        for (unsigned it = 1;; ++it) {
+            const bool mine = lane >= kBarLanes || ld_acquire_gpu(ctr) >= target;
+            if (__all_sync(0xffffffffu, mine)) break;
+            // the timeout verdict is taken warp-wide so every lane leaves together
+            if ((it & 63) == 0 && __any_sync(0xffffffffu, gtimer() - t0 > p.wait_ns)) {
+                if (lane == 0) set_error(p.err, kDevTimeout);
                 ok = false;
                 break;
             }
         }
-        __threadfence();
-        st_vol(&sm->bc[bci], ok ? 1 : 0);
-        if (cyc) *cyc += clock64() - c0;
+        if (lane == 0) {
+            st_vol(&sm->bc[bci], ok ? 1 : 0);
+            if (cyc) *cyc += clock64() - c0;
+        }
     }
     cta_sync();
     const bool ok = ld_vol(&sm->bc[bci]) != 0;

@@ -211,7 +211,7 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
     const size_t o_lists = up256(o_io + sizeof(float) * D.d_model);
     const size_t o_counts = up256(o_lists + sizeof(int32_t) * size_t(h->S) * pi::kMaxStrip);
     const size_t o_bar = up256(o_counts + sizeof(int32_t) * h->S);
-    const size_t o_err = o_bar + 256;
+    const size_t o_err = up256(o_bar + sizeof(unsigned) * pi::kBarWords);
     const size_t o_fix = o_err + 256;
     const size_t total = up256(o_fix + sizeof(long long) * 2 * pi::kFixStride);
     cudaError_t e = cudaMalloc(&h->scratch, total);
@@ -471,7 +471,7 @@ pi_status pi_predict(pi_ffn_t h, int layer, int expert, const float *x_dev, int3
     p.z_out = z_dev;
     p.idx_out = idx_dev;
     p.count_out = count_dev;
-    PI_CUDA(cudaMemsetAsync(h->bar, 0, 2 * sizeof(unsigned), st), "memset barrier");
+    PI_CUDA(cudaMemsetAsync(h->bar, 0, sizeof(unsigned) * pi::kBarWords, st), "memset barrier");
     PI_CUDA(cudaMemsetAsync(h->fix, 0, sizeof(long long) * 2 * pi::kFixStride, st), "memset accumulators");
     PI_CUDA(pi::launch_decode(h->wfmt, h->pfmt, p, st), "launch predict");
     return PI_OK;
@@ -500,7 +500,7 @@ pi_status pi_sparse_ffn_decode(pi_ffn_t h, int layer_begin, int layer_end, float
     p.trace = trace_dev;
     p.stats = stats_dev;
     p.masks = mask_dev;
-    PI_CUDA(cudaMemsetAsync(h->bar, 0, 2 * sizeof(unsigned), st), "memset barrier");
+    PI_CUDA(cudaMemsetAsync(h->bar, 0, sizeof(unsigned) * pi::kBarWords, st), "memset barrier");
     PI_CUDA(cudaMemsetAsync(h->fix, 0, sizeof(long long) * 2 * pi::kFixStride, st), "memset accumulators");
     if (stats_dev) PI_CUDA(cudaMemsetAsync(stats_dev, 0, sizeof(int32_t) * 4 * nl, st), "memset stats");
     if (mask_dev)

@@ -75,6 +75,9 @@ struct DecodeParams {
 // Phase timestamps recorded per layer and CTA when DecodeParams::prof is set.
 // layer kinds (bits of the decode kernel's MODE parameter)
 constexpr int kModeMoE = 1, kModeGated = 2, kModeSpec = 4, kModePred = 8;
+// grid barrier: arrival counters, each on its own 128-byte line
+constexpr int kBarLanes = 16, kBarStride = 32;
+constexpr int kBarWords = kBarLanes * kBarStride;
 constexpr int kProfPoints = 14;   // timestamps and cycle counters per layer and CTA
 
 cudaError_t launch_decode(int wfmt, int pfmt, const DecodeParams &p, cudaStream_t stream);

@@ -24,7 +24,7 @@ namespace {
 //   lists    kMaxStrips * kMaxStrip ints  per-strip active lists
 //   counts   kMaxStrips ints              per-strip active counts
 //   fix      2 * kFixStride int64         fixed-point accumulators (zeroed per call)
-//   bar      2 unsigned                   grid barrier words (zeroed per call)
+//   bar      kBarWords unsigned           grid barrier counters (zeroed per call)
 //   err      1 int                        device error word (zeroed per call)
 //   experts  2 ExpertDev                  weight pointers of this call
 //   strips   kMaxStrips + 1 ints          strip offsets
@@ -34,7 +34,7 @@ constexpr size_t kOffLists = kOffT + sizeof(float) * pi::kMaxRankTotal;
 constexpr size_t kOffCounts = kOffLists + sizeof(int32_t) * pi::kMaxStrips * pi::kMaxStrip;
 constexpr size_t kOffFix = (kOffCounts + sizeof(int32_t) * pi::kMaxStrips + 255) & ~size_t(255);
 constexpr size_t kOffBar = kOffFix + sizeof(long long) * 2 * pi::kFixStride;
-constexpr size_t kOffErr = kOffBar + 2 * sizeof(unsigned);
+constexpr size_t kOffErr = kOffBar + sizeof(unsigned) * pi::kBarWords;
 constexpr size_t kOffEx = (kOffErr + sizeof(int) + 255) & ~size_t(255);
 constexpr size_t kOffStrips = kOffEx + 2 * sizeof(pi::ExpertDev);
 constexpr size_t kOffGroups = kOffStrips + sizeof(int32_t) * (pi::kMaxStrips + 1);
