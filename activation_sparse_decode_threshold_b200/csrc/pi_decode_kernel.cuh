@@ -493,6 +493,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     auto column_phase = [&](int li_in, bool from_partials, bool next_exists, int l_next, int prow) {
         const float *src = predict ? p.x_in : p.resid;
         long long *fx = p.fix + size_t(li_in & 1) * kFixStride;
+        // dense: this thread's V-block rows (k = tid and tid + 512; r <= 1024)
+        // for the next layer's t partial start loading now, so their round
+        // trip overlaps the partial reduction's; the first kVP vectors of each
+        constexpr int kVP = 4;
+        const bool tpart = !moe && next_exists && ncol > 0;
+        const int nv = vbrow / VBP;
+        const int kr0 = tid, kr1 = tid + kThreads;
+        const uint8_t *vrow0 = nullptr, *vrow1 = nullptr;
+        VP va[kVP], vb2[kVP];
+        if (tpart) {
+            const uint8_t *vb = vblk(l_next);
+            vrow0 = vb + size_t(kr0 < r ? kr0 : 0) * vbrow;
+            vrow1 = vb + size_t(kr1 < r ? kr1 : 0) * vbrow;
+#pragma unroll
+            for (int j = 0; j < kVP; ++j) {
+                if (j < nv && kr0 < r) va[j] = ldvec<PF>(vrow0 + j * VBP);
+                if (j < nv && kr1 < r) vb2[j] = ldvec<PF>(vrow1 + j * VBP);
+            }
+        }
         if (from_partials) {
             const int q0 = c0 / 4, nq = ncol / 4;
             for (int qq = warp; qq < nq; qq += kConsumerWarps) {
@@ -540,43 +559,32 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             if (lane == 0 && ncol > 0) fix_add(fx + kMaxRankTotal, ss, kFixSS);
         }
         if (!moe) {
-            // t partial: row k of the V block dotted with this CTA's columns
-            const uint8_t *vb = vblk(l_next);
-            const int nv = vbrow / VBP;
-            // rows k and k + 512 together; four vectors of each in flight
-            for (int k = tid; k < r && ncol > 0; k += 2 * kThreads) {
-                const bool two = k + kThreads < r;
-                const uint8_t *row0 = vb + size_t(k) * vbrow;
-                const uint8_t *row1 = vb + size_t(two ? k + kThreads : k) * vbrow;
+            // t partial: rows kr0, kr1 of the V block dotted with this CTA's columns
+            if (tpart && kr0 < r) {
                 float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-                for (int v0 = 0; v0 < nv; v0 += 4) {
-                    VP q0[4], q1[4];
+                auto acc_vec = [&](const VP &q0, const VP &q1, int v) {
+                    float w0[EPVP], w1[EPVP];
+                    cvt<PF>(q0, w0);
+                    cvt<PF>(q1, w1);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        if (v0 + j < nv) {
-                            q0[j] = ldvec<PF>(row0 + (v0 + j) * VBP);
-                            q1[j] = ldvec<PF>(row1 + (v0 + j) * VBP);
-                        }
+                    for (int i = 0; i < EPVP; i += 2) {
+                        const float x0 = sm.rsl[v * EPVP + i], x1 = sm.rsl[v * EPVP + i + 1];
+                        a0 = fmaf(w0[i], x0, a0);
+                        a1 = fmaf(w0[i + 1], x1, a1);
+                        b0 = fmaf(w1[i], x0, b0);
+                        b1 = fmaf(w1[i + 1], x1, b1);
                     }
+                };
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        if (v0 + j < nv) {
-                            float w0[EPVP], w1[EPVP];
-                            cvt<PF>(q0[j], w0);
-                            cvt<PF>(q1[j], w1);
-#pragma unroll
-                            for (int i = 0; i < EPVP; i += 2) {
-                                const float x0 = sm.rsl[(v0 + j) * EPVP + i], x1 = sm.rsl[(v0 + j) * EPVP + i + 1];
-                                a0 = fmaf(w0[i], x0, a0);
-                                a1 = fmaf(w0[i + 1], x1, a1);
-                                b0 = fmaf(w1[i], x0, b0);
-                                b1 = fmaf(w1[i + 1], x1, b1);
-                            }
-                        }
-                    }
+                for (int j = 0; j < kVP; ++j)
+                    if (j < nv) acc_vec(va[j], kr1 < r ? vb2[j] : va[j], j);
+                for (int v = kVP; v < nv; ++v) {
+                    const VP q0 = ldvec<PF>(vrow0 + v * VBP);
+                    const VP q1 = kr1 < r ? ldvec<PF>(vrow1 + v * VBP) : q0;
+                    acc_vec(q0, q1, v);
                 }
-                fix_add(fx + k, a0 + a1, kFixT);
-                if (two) fix_add(fx + k + kThreads, b0 + b1, kFixT);
+                fix_add(fx + kr0, a0 + a1, kFixT);
+                if (kr1 < r) fix_add(fx + kr1, b0 + b1, kFixT);
             }
         } else if (!predict) {
             // router logit partials: W_r[e, cols] . r[cols]
@@ -651,6 +659,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     if (k < r) put_t(k, float(double(tq[j]) * (1.0 / 4294967296.0)) * inv, r);
                 }
             }
+            // this strip's biases, in the same round trip as t and x
+            for (int i = tid; i < ns; i += kThreads) sm.cbuf[0][i] = __ldg(sm.exl[l & 1][0].c + s0 + i);
             // the next layer's weight pointers, for its prefetches during this layer
             if (tid == kThreads - 1 && l + 1 < l1) sm.exl[(l + 1) & 1][0] = p.ex[size_t(l + 1) * p.E];
             if (tid == 0) {
@@ -765,10 +775,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             if (!grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
             for (int k = tid; k < ntop * r; k += kThreads) put_t(k, __ldcg(p.t_buf + k), ntop * r);
         }
-        for (int e = 0; e < ntop; ++e)
-            for (int i = tid; i < ns; i += kThreads)
-                sm.cbuf[e][i] = __ldg(sm.exl[l & 1][e].c + s0 + i);
-        cta_sync();
+        if constexpr (moe) {
+            for (int e = 0; e < ntop; ++e)
+                for (int i = tid; i < ns; i += kThreads)
+                    sm.cbuf[e][i] = __ldg(sm.exl[l & 1][e].c + s0 + i);
+            cta_sync();
+        }
         cyc_a = clock64() - ca0;
         prof_put(p, li, 1, gtimer());
 
