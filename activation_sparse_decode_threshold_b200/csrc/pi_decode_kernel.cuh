@@ -277,7 +277,14 @@ constexpr int kRed = 2 * kRound;  // values reduced per warp at most
 
 struct Smem {
     float red[2][kConsumerWarps][kRed];
-    float zred[kConsumerWarps][kZRows];    // per-warp partial logits of a U round
+    union {
+        float zred[kConsumerWarps][kZRows];    // per-warp partial logits of a U round (logit phase)
+        struct {                               // this CTA's share of the active list (gather phase)
+            int32_t glst[kMaxTopK * kMaxStrip];  // (slot << 24) | table position
+            float gc[kMaxTopK * kMaxStrip];      // their biases
+        };
+    };
+    int scan[kMaxStrips + 1];              // exclusive prefix of the strip counts
     alignas(16) float tsm[kMaxRankTotal];  // t (fp32 predictor) or its 16-bit parts (split_parts)
     alignas(16) float rsl[kMaxSliceCols];  // this CTA's columns of the new residual
     float cbuf[kMaxTopK][kMaxStrip];
@@ -285,9 +292,9 @@ struct Smem {
     ExpertDev exl[2][kMaxTopK];            // weight pointers of the layer's expert slots, by layer parity
     int16_t lst[kMaxTopK * kMaxStrip];     // active neurons: (slot << 12) | local
     int lst_n[kMaxTopK];
-    int16_t nz[kMaxTopK * kMaxStrip];      // neurons with h != 0, same encoding
+    int32_t nz[kMaxTopK * kMaxStrip];      // neurons with h != 0, encoded as glst
     float hz[kMaxTopK * kMaxStrip];        // their h (routing weight folded in)
-    int nz_n;
+    int share_n;                           // size of this CTA's share of the active list
     float rsum[kRed];                      // CTA-wide dot products of a gather round
     float rh[kRound];                      // h of each neuron of a gather round
     int route_e[kMaxTopK];
@@ -953,7 +960,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 if (p.stats && !predict) atomicAdd(p.stats + li * 4 + 0, cnt);
             }
         }
-        if (tid == 0) sm.nz_n = 0;
         cta_sync();
         (void)cb0;
         prof_put(p, li, 2, gtimer());
@@ -974,24 +980,71 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             break;
         }
 
+        // ---------------- balance: equal shares of the active list -----------
+        // Each strip publishes its active neurons (with their biases) and
+        // starts their rows moving towards L2; after a grid barrier every CTA
+        // takes an equal share [lo, hi) of the lists concatenated in strip
+        // order.  The share depends only on the active set, so the per-CTA
+        // partials and their fixed-order reduction stay deterministic.
+        const ExpertDev *exs[kMaxTopK] = {&sm.exl[l & 1][0], &sm.exl[l & 1][ntop > 1 ? 1 : 0]};
+        {
+            const int n0 = sm.lst_n[0], nl = n0 + (ntop > 1 ? sm.lst_n[1] : 0);
+            unsigned long long *pb = p.pub + size_t(b) * (kMaxTopK * kMaxStrip);
+            for (int j = tid; j < nl; j += kThreads) {
+                const int en = j < n0 ? sm.lst[j] : sm.lst[kMaxStrip + (j - n0)];
+                const int e = en >> 12, loc = en & 0xfff, pos = s0 + loc;
+                __stcg(pb + j, (unsigned long long)(unsigned(e << 24) | unsigned(pos)) |
+                                   ((unsigned long long)__float_as_uint(sm.cbuf[e][loc]) << 32));
+                prefetch_l2(exs[e]->Wgu + size_t(pos) * p.gu_bytes, uint32_t(p.gu_bytes));
+                if (kSpec) prefetch_l2(exs[e]->Wd + size_t(pos) * p.wrow, uint32_t(p.wrow));
+            }
+            if (tid == 0) __stcg(p.counts + b, nl);
+        }
+        if (!grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
+        {
+            // exclusive prefix of the strip counts (S <= 256: warps 0..7)
+            const int cnt = tid < S ? __ldcg(p.counts + tid) : 0;
+            int inc = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += v;
+            }
+            if (lane == 31) sm.red[rb][warp][0] = __int_as_float(inc);
+            cta_sync();
+            if (tid <= S) {
+                int pre = inc - cnt;
+                for (int w = 0; w < warp; ++w) pre += __float_as_int(sm.red[rb][w][0]);
+                sm.scan[tid] = pre;
+            }
+            rb ^= 1;
+            cta_sync();
+            const int ntot = sm.scan[S];
+            const int lo = int((long long)b * ntot / S), hi = int((long long)(b + 1) * ntot / S);
+            for (int j = lo + tid; j < hi; j += kThreads) {
+                int q0 = 0, q1 = S;   // strip q with scan[q] <= j < scan[q + 1]
+                while (q1 - q0 > 1) {
+                    const int mid = (q0 + q1) >> 1;
+                    if (sm.scan[mid] <= j) q0 = mid;
+                    else q1 = mid;
+                }
+                const unsigned long long w = __ldcg(p.pub + size_t(q0) * (kMaxTopK * kMaxStrip) + (j - sm.scan[q0]));
+                sm.glst[j - lo] = int(unsigned(w));
+                sm.gc[j - lo] = __uint_as_float(unsigned(w >> 32));
+            }
+            if (tid == 0) sm.share_n = hi - lo;
+            cta_sync();
+        }
+
         // ---------------- gather rows of active neurons ----------------------
         // Rounds of up to kRound neurons: one bulk-copy round brings their
         // W_gate/W_up records (and, when speculative, their W_down rows) into
         // shared memory; the dots of all of them are reduced at once.
         const long long cc0 = clock64();
-        const int m0 = sm.lst_n[0];
-        const int m = m0 + (ntop > 1 ? sm.lst_n[1] : 0);
-        auto entry = [&](int j) -> int { return j < m0 ? sm.lst[j] : sm.lst[kMaxStrip + (j - m0)]; };
-        const ExpertDev *exs[kMaxTopK] = {&sm.exl[l & 1][0], &sm.exl[l & 1][ntop > 1 ? 1 : 0]};
+        const int m = sm.share_n;
         const int per_n = p.gu_bytes + (kSpec ? p.wrow : 0);   // bytes per neuron in a round
         const int cap_n = min(kRound, kStageBytes / per_n);
-        // rows beyond the first round, and the next layer's V block and
-        // biases, start moving towards L2 now
-        for (int j = cap_n + tid; j < m; j += kThreads) {
-            const int en = entry(j), e = en >> 12, loc = en & 0xfff;
-            prefetch_l2(exs[e]->Wgu + size_t(s0 + loc) * p.gu_bytes, uint32_t(p.gu_bytes));
-            if (kSpec) prefetch_l2(exs[e]->Wd + size_t(s0 + loc) * p.wrow, uint32_t(p.wrow));
-        }
+        // the next layer's V block and biases start moving towards L2 now
         if (tid == kThreads - 1 && !moe && l + 1 < l1) {
             if (ncol > 0) prefetch_l2(vblk(l + 1), uint32_t(r) * vbrow);
             if (ns > 0) {
@@ -1046,12 +1099,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 if (lane == 0) mbar_arrive_tx(&sm.stage_bar, uint32_t(k) * per_n);
                 __syncwarp();
                 if (lane < k) {
-                    const int en = entry(j0 + lane), e = en >> 12, loc = en & 0xfff;
+                    const int en = sm.glst[j0 + lane], e = en >> 24, pos = en & 0xffffff;
                     uint8_t *slot = stg + size_t(lane) * per_n;
-                    stage_copy(slot, exs[e]->Wgu + size_t(s0 + loc) * p.gu_bytes, uint32_t(p.gu_bytes),
-                               &sm.stage_bar);
+                    stage_copy(slot, exs[e]->Wgu + size_t(pos) * p.gu_bytes, uint32_t(p.gu_bytes), &sm.stage_bar);
                     if (kSpec)
-                        stage_copy(slot + p.gu_bytes, exs[e]->Wd + size_t(s0 + loc) * p.wrow, uint32_t(p.wrow),
+                        stage_copy(slot + p.gu_bytes, exs[e]->Wd + size_t(pos) * p.wrow, uint32_t(p.wrow),
                                    &sm.stage_bar);
                 }
             }
@@ -1086,9 +1138,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             rb ^= 1;
             cta_sync();
             if (tid < k) {
-                const int en = entry(j0 + tid), e = en >> 12, loc = en & 0xfff;
-                sm.rh[tid] = act_h(p.act, sm.rsum[2 * tid] - sm.cbuf[e][loc], sm.rsum[2 * tid + 1]) *
-                             sm.route_w[e];
+                const int e = sm.glst[j0 + tid] >> 24;
+                sm.rh[tid] = act_h(p.act, sm.rsum[2 * tid] - sm.gc[j0 + tid], sm.rsum[2 * tid + 1]) * sm.route_w[e];
             }
             cta_sync();
             // neurons with h != 0, in list order (every warp forms the same
@@ -1097,7 +1148,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             const unsigned nzm = __ballot_sync(0xffffffffu, nzv);
             if (warp == 0 && nzv) {
                 const int pos = nz_total + __popc(nzm & ((1u << lane) - 1u));
-                sm.nz[pos] = int16_t(entry(j0 + lane));
+                sm.nz[pos] = sm.glst[j0 + lane];
                 sm.hz[pos] = sm.rh[lane];
             }
             const int nz_round = __popc(nzm);
@@ -1151,8 +1202,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     if (lane == 0) mbar_arrive_tx(&sm.stage_bar, uint32_t(k) * p.wrow);
                     __syncwarp();
                     for (int n = lane; n < k; n += 32) {
-                        const int en = sm.nz[q0 + n], e = en >> 12, loc = en & 0xfff;
-                        stage_copy(stg + size_t(n) * p.wrow, exs[e]->Wd + size_t(s0 + loc) * p.wrow,
+                        const int en = sm.nz[q0 + n], e = en >> 24, pos = en & 0xffffff;
+                        stage_copy(stg + size_t(n) * p.wrow, exs[e]->Wd + size_t(pos) * p.wrow,
                                    uint32_t(p.wrow), &sm.stage_bar);
                     }
                 }

@@ -88,6 +88,7 @@ struct pi_ffn {
     uint8_t *scratch = nullptr;
     float *t_buf = nullptr, *partials = nullptr, *io = nullptr;
     int32_t *lists = nullptr, *counts = nullptr;
+    unsigned long long *pub = nullptr;
     unsigned *bar = nullptr;
     int *err = nullptr;
     long long wait_ns = 2000000000LL;
@@ -210,7 +211,8 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
     const size_t o_io = up256(o_part + sizeof(float) * size_t(h->S) * D.d_model);
     const size_t o_lists = up256(o_io + sizeof(float) * D.d_model);
     const size_t o_counts = up256(o_lists + sizeof(int32_t) * size_t(h->S) * pi::kMaxStrip);
-    const size_t o_bar = up256(o_counts + sizeof(int32_t) * h->S);
+    const size_t o_pub = up256(o_counts + sizeof(int32_t) * h->S);
+    const size_t o_bar = up256(o_pub + sizeof(unsigned long long) * size_t(h->S) * pi::kMaxTopK * pi::kMaxStrip);
     const size_t o_err = up256(o_bar + sizeof(unsigned) * pi::kBarWords);
     const size_t o_fix = o_err + 256;
     const size_t total = up256(o_fix + sizeof(long long) * 2 * pi::kFixStride);
@@ -237,6 +239,7 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
     h->io = reinterpret_cast<float *>(h->scratch + o_io);
     h->lists = reinterpret_cast<int32_t *>(h->scratch + o_lists);
     h->counts = reinterpret_cast<int32_t *>(h->scratch + o_counts);
+    h->pub = reinterpret_cast<unsigned long long *>(h->scratch + o_pub);
     h->bar = reinterpret_cast<unsigned *>(h->scratch + o_bar);
     h->err = reinterpret_cast<int *>(h->scratch + o_err);
     h->fix = reinterpret_cast<long long *>(h->scratch + o_fix);
@@ -443,6 +446,7 @@ static pi::DecodeParams base_params(pi_ffn_t h)
     p.partials = h->partials;
     p.lists = h->lists;
     p.counts = h->counts;
+    p.pub = h->pub;
     p.bar = h->bar;
     p.err = h->err;
     p.wait_ns = h->wait_ns;

@@ -64,7 +64,9 @@ struct DecodeParams {
     long long *fix;                 // [2 * kFixStride] fixed-point accumulators, zeroed
     float *partials;                // [S * d]
     int32_t *lists;                 // [S * kMaxStrip]  (predict)
-    int32_t *counts;                // [S]              (predict)
+    int32_t *counts;                // [S] active count of each strip
+    unsigned long long *pub;        // [S * kMaxTopK * kMaxStrip] published active entries (decode):
+                                    // low word (slot << 24) | table position, high word the bias bits
     unsigned *bar;                  // [2] grid barrier: arrivals, generation; zeroed before launch
     int *err;                       // device error word (0 = ok)
     long long wait_ns;              // bound on every device-side wait
