@@ -33,7 +33,7 @@ from activation_sparse_decode_threshold_b200 import synth  # noqa: E402
 
 METRIC = "decode tok/s (FFN stack, batch 1) and achieved HBM GB/s on touched bytes vs peak"
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SRC = os.path.join(ROOT, "activation_sparse_decode_threshold_b200", "csrc", "pi_decode.cu")
+KERNEL_SRC = os.path.join(ROOT, "activation_sparse_decode_threshold_b200", "csrc", "pi_decode_kernel.cuh")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_dram_traffic.txt")
 PB = {"f32": 4, "f16": 2, "bf16": 2}
 
