@@ -269,7 +269,7 @@ __device__ __forceinline__ float act_h(int act, float g, float u)
 }
 
 constexpr int kRA = 16;           // V rows per staging round at most
-constexpr int kZRows = 96;        // U rows per staging round at most (a multiple of 16)
+constexpr int kZRows = 112;       // U rows per staging round at most (a multiple of 16)
 constexpr int kMaxU = 4;          // U vectors per lane (rank <= 128 * EPV)
 constexpr int kRound = 16;        // neurons per gather round at most
 static_assert(kRound <= 32, "a round's neurons are tracked in one warp ballot");
@@ -285,15 +285,23 @@ struct Smem {
         };
     };
     int scan[kMaxStrips + 1];              // exclusive prefix of the strip counts
-    alignas(16) float tsm[kMaxRankTotal];  // t (fp32 predictor) or its 16-bit parts (split_parts)
-    alignas(16) float rsl[kMaxSliceCols];  // this CTA's columns of the new residual
-    float cbuf[kMaxTopK][kMaxStrip];
-    float zbuf[kMaxTopK][kMaxStrip];
+    union {                                // layer start .. logits / gather
+        alignas(16) float tsm[kMaxRankTotal];  // t (fp32 predictor) or its 16-bit parts (split_parts)
+        struct {
+            int32_t nz[kMaxTopK * kMaxStrip];  // neurons with h != 0, encoded as glst
+            float hz[kMaxTopK * kMaxStrip];    // their h (routing weight folded in)
+        };
+    };
+    union {                                // column phase / layer start .. active list
+        alignas(16) float rsl[kMaxSliceCols];  // this CTA's columns of the new residual
+        struct {
+            float cbuf[kMaxTopK][kMaxStrip];
+            float zbuf[kMaxTopK][kMaxStrip];
+        };
+    };
     ExpertDev exl[2][kMaxTopK];            // weight pointers of the layer's expert slots, by layer parity
     int16_t lst[kMaxTopK * kMaxStrip];     // active neurons: (slot << 12) | local
     int lst_n[kMaxTopK];
-    int32_t nz[kMaxTopK * kMaxStrip];      // neurons with h != 0, encoded as glst
-    float hz[kMaxTopK * kMaxStrip];        // their h (routing weight folded in)
     int share_n;                           // size of this CTA's share of the active list
     float rsum[kRed];                      // CTA-wide dot products of a gather round
     float rh[kRound];                      // h of each neuron of a gather round
@@ -446,7 +454,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // this CTA's rows of t (row-split form, MoE)
     const int rows_total = ntop * r;
     const int a0 = int((long long)b * rows_total / S), a1 = int((long long)(b + 1) * rows_total / S);
-    const int ucap = min(kZRows, kStageBytes / p.urow) & ~15;   // U rows per staging round (a multiple of 16)
+    // U rows per staging round: the whole strip when it fits, else rounds of a
+    // multiple of 8 rows (chunk permutation keys are row mod 8)
+    const int ucap_rows = min(kZRows, kStageBytes / p.urow);
+    const int ucap = ns <= ucap_rows ? max(ns, 1) : (ucap_rows & ~7);
 
     // V block of this CTA (dense): rows of t restricted to this CTA's columns
     auto vblk = [&](int l) -> const uint8_t * {
@@ -877,42 +888,48 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                         const int nparts = (PF == kBF16 && 3 * ntr <= 2 * kMaxRankTotal) ? 3 : 2;
                         const int nks = r / 16, nmt = (n + 15) / 16;
                         const int g = lane >> 2, tq = lane & 3;
-                        float c[kZRows / 16][4];
-#pragma unroll
-                        for (int mt = 0; mt < kZRows / 16; ++mt)
-                            c[mt][0] = c[mt][1] = c[mt][2] = c[mt][3] = 0.f;
                         const int arow = lane & 15;                       // row within an m-tile
-                        const int akey = p.u_swz ? (arow & 7) : 0;        // m-tiles start at multiples of 16
-                        const uint8_t *abase = stg + size_t(arow) * p.urow;
                         const uint16_t *bpart = tpart + g * ntr + e * r + 2 * tq;
-                        for (int ks = warp; ks < nks; ks += kConsumerWarps) {
-                            uint32_t b0 = 0u, b1 = 0u;
-                            if (g < nparts) {
-                                b0 = *reinterpret_cast<const uint32_t *>(bpart + ks * 16);
-                                b1 = *reinterpret_cast<const uint32_t *>(bpart + ks * 16 + 8);
-                            }
-                            const int chunk = 2 * ks + (lane >> 4);            // 16-byte chunk of the row
-                            const uint8_t *arow_p = abase + ((chunk & ~7) | ((chunk ^ akey) & 7)) * 16;
+                        // m-tiles in passes of kZT (bounded accumulator registers)
+                        constexpr int kZT = MAXVW > 1 ? 4 : 6;
+                        for (int mt0 = 0; mt0 < nmt; mt0 += kZT) {
+                            float c[kZT][4];
 #pragma unroll
-                            for (int mt = 0; mt < kZRows / 16; ++mt) {
-                                if (mt < nmt) {
-                                    uint32_t a0, a1, a2, a3;
-                                    ldsm_x4(arow_p + size_t(mt) * 16 * p.urow, a0, a1, a2, a3);
-                                    mma16816<PF>(c[mt], a0, a1, a2, a3, b0, b1);
+                            for (int t = 0; t < kZT; ++t) c[t][0] = c[t][1] = c[t][2] = c[t][3] = 0.f;
+                            for (int ks = warp; ks < nks; ks += kConsumerWarps) {
+                                uint32_t b0 = 0u, b1 = 0u;
+                                if (g < nparts) {
+                                    b0 = *reinterpret_cast<const uint32_t *>(bpart + ks * 16);
+                                    b1 = *reinterpret_cast<const uint32_t *>(bpart + ks * 16 + 8);
+                                }
+                                const int chunk = 2 * ks + (lane >> 4);            // 16-byte chunk of the row
+#pragma unroll
+                                for (int t = 0; t < kZT; ++t) {
+                                    if (mt0 + t < nmt) {
+                                        // rows past the round's last are read as its last row
+                                        // (their results are never used); the chunk permutation
+                                        // key is the staged row mod 8 (rounds start at multiples of 8)
+                                        const int row = min((mt0 + t) * 16 + arow, n - 1);
+                                        const int key = p.u_swz ? (row & 7) : 0;
+                                        uint32_t a0, a1, a2, a3;
+                                        ldsm_x4(stg + size_t(row) * p.urow + ((chunk & ~7) | ((chunk ^ key) & 7)) * 16,
+                                                a0, a1, a2, a3);
+                                        mma16816<PF>(c[t], a0, a1, a2, a3, b0, b1);
+                                    }
                                 }
                             }
-                        }
-                        // sum over the parts: columns 0 and 1 sit in lane 4g, column 2 in lane 4g + 1
+                            // sum over the parts: columns 0 and 1 sit in lane 4g, column 2 in lane 4g + 1
 #pragma unroll
-                        for (int mt = 0; mt < kZRows / 16; ++mt) {
-                            float z0 = c[mt][0] + c[mt][1], z1 = c[mt][2] + c[mt][3];
-                            if constexpr (kParts == 3) {
-                                z0 += __shfl_down_sync(0xffffffffu, c[mt][0], 1);
-                                z1 += __shfl_down_sync(0xffffffffu, c[mt][2], 1);
-                            }
-                            if (tq == 0 && mt < nmt) {
-                                sm.zred[warp][mt * 16 + g] = z0;
-                                sm.zred[warp][mt * 16 + g + 8] = z1;
+                            for (int t = 0; t < kZT; ++t) {
+                                float z0 = c[t][0] + c[t][1], z1 = c[t][2] + c[t][3];
+                                if constexpr (kParts == 3) {
+                                    z0 += __shfl_down_sync(0xffffffffu, c[t][0], 1);
+                                    z1 += __shfl_down_sync(0xffffffffu, c[t][2], 1);
+                                }
+                                if (tq == 0 && mt0 + t < nmt) {
+                                    sm.zred[warp][(mt0 + t) * 16 + g] = z0;
+                                    sm.zred[warp][(mt0 + t) * 16 + g + 8] = z1;
+                                }
                             }
                         }
                         cta_sync();

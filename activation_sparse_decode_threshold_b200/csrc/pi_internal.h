@@ -16,7 +16,7 @@ constexpr int kMaxStrips = 256;       // strips (CTAs) at most
 constexpr int kMaxTopK = 2;
 constexpr int kMaxExperts = 16;
 constexpr int kMaxRankTotal = 2048;   // top_k * rank
-constexpr int kStageBytes = 192 * 1024;   // shared-memory staging of V rows / U strips
+constexpr int kStageBytes = 200 * 1024;   // shared-memory staging of V rows / U strips / gathered rows
 constexpr int kMaxSliceCols = 1024;       // residual columns per CTA at most
 constexpr int kFixStride = kMaxRankTotal + 1 + kMaxExperts;   // t, sum r^2, logits
 

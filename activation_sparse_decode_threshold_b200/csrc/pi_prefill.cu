@@ -347,16 +347,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
             cp_async_commit();
         };
         // INT4: the raw nibbles and scales of a stage, loaded into registers.
-        // GU item: row c >> 2, 16 elements at chunk pair c & 3 (a warp: 8 rows
-        // x 32 contiguous bytes).  Down item: W_down row k (8 per warp) and 16
-        // output columns (4 consecutive groups per row).
+        // GU item: 16 elements (chunk pair q16) of one row; the 8 lanes of each
+        // quarter-warp take 8 consecutive rows, so each of the four phases of
+        // a 16-byte shared store touches 8 different bank groups, and a row's
+        // 32 bytes come from 4 lanes.  Down item: W_down row k (8 per warp) and
+        // 16 output columns (4 consecutive groups per row).
         auto load_raw = [&](int kt, RawI4 &r) {
             const int k0 = kt * BK;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int c = pt + kProducers * i;
                 if constexpr (KIND == kGU) {
-                    const int row = c >> 2, q16 = c & 3;       // elements k0 + 16 q16 .. +15
+                    const int row = (c >> 5) * 8 + (c & 7), q16 = (c >> 3) & 3;   // elements k0 + 16 q16 .. +15
                     const int nn = n0 / 2 + (row >> 1);
                     const bool ok = nn < F && (p.gated || (row & 1) == 0);
                     r.q[i] = make_uint2(0u, 0u);
@@ -385,7 +387,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
                 uint4 lo, hi;
                 dequant16(r.q[i], __ushort_as_half(r.sc[i]), lo, hi);
                 if constexpr (KIND == kGU) {
-                    const int row = c >> 2, q16 = c & 3;
+                    const int row = (c >> 5) * 8 + (c & 7), q16 = (c >> 3) & 3;
                     *reinterpret_cast<uint4 *>(B + kmaj_off(row, 2 * q16)) = lo;
                     *reinterpret_cast<uint4 *>(B + kmaj_off(row, 2 * q16 + 1)) = hi;
                 } else {

@@ -243,6 +243,65 @@ def job_throughput(units_per_rank: int, world: int, max_ms: float) -> float:
     return units_per_rank * world / (max_ms / 1e3)
 
 
+def measured_tensor_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, fp16 same rate)"
+    return 1590.0, "fallback 1.59 PFLOP/s"
+
+
+def run_prefill(args, cfg, rank: int, world: int) -> int:
+    """Dense prefill of the workload's prompt (T tokens) through the stack on the
+    tcgen05 path: one step = the whole prompt through every layer."""
+    from activation_sparse_decode_threshold_b200 import binding as B
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    T = cfg.prefill_tokens or 512
+    h = build_handle(cfg, B, local, None)
+    L = cfg.n_layers
+    R = synth.prefill_input(cfg, T, "cuda")
+    r = torch.empty_like(R)
+    for _ in range(args.warmup):
+        r.copy_(R)
+        B.pi_dense_ffn_prefill(h, 0, L, T, r)
+    if B.pi_sync(h) != B.PI_OK:
+        raise RuntimeError(B.pi_last_error())
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for s in range(args.steps):
+            r.copy_(R)                      # the copy sits outside the events
+            ev[s][0].record(stream)
+            B.pi_dense_ffn_prefill(h, 0, L, T, r)
+            ev[s][1].record(stream)
+        torch.cuda.synchronize()
+    if B.pi_sync(h) != B.PI_OK:
+        raise RuntimeError(B.pi_last_error())
+    ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = sum(ms)
+    B.pi_ffn_destroy(h)
+    if rank != 0:
+        return 0
+    flop = 2.0 * T * cfg.top_k * cfg.d * cfg.F * (3 if cfg.gated else 2) * L
+    tflops = flop / (total_ms / args.steps / 1e3) / 1e12
+    peak, kind = measured_tensor_peak()
+    print(json.dumps({
+        "metric": "dense prefill TFLOP/s (tcgen05 path)", "value": tflops, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16 MMA, f32 accumulate", "data": "synthetic",
+        "config": dict(workload_config(cfg, None, None), workload=f"{cfg.name}-prefill{T}", tokens=T),
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": tflops / peak, "traffic": None, "peak_source": kind,
+                     "flop_per_step": flop},
+        "gpu_launches": 5 * L * args.steps,
+        "clocks": clk.summary(),
+    }), flush=True)
+    return 0
+
+
 def workload_config(cfg, active, measured_active):
     return {"workload": cfg.name, "layers": cfg.n_layers, "d_model": cfg.d, "d_ff": cfg.F,
             "rank": cfg.rank, "act": cfg.act, "weights": cfg.wdtype, "predictor": cfg.pdtype,
@@ -265,6 +324,8 @@ def main() -> int:
     ap.add_argument("--layers", type=int, default=None, help="override layer count (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--prefill", action="store_true",
+                    help="time the dense tensor-core prefill of the workload's prompt instead of decode")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -279,6 +340,8 @@ def main() -> int:
 
     if args.impl == "reference":
         return run_reference(args, cfg, active, rank, world)
+    if args.prefill:
+        return run_prefill(args, cfg, rank, world)
 
     from activation_sparse_decode_threshold_b200 import binding as B
     torch.cuda.set_device(local)
