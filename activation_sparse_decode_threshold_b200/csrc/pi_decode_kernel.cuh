@@ -310,6 +310,8 @@ struct Smem {
     float inv_rms;
     int bc[2];
     uint64_t stage_bar;                    // completion of a staging round
+    uint64_t gbar[kRound / 4];             // completion of each group of four neurons of a gather round
+    int gfail;                             // a warp's bounded wait on a group ran out
 };
 
 __device__ void set_error(int *err, int code)
@@ -467,6 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 
     unsigned epoch = 0;
     uint32_t spar = 0;
+    uint32_t gpar = 0, gpend = 0;   // gather group barriers: phase parities, groups in flight
     int bci = 0, rb = 0;
     bool staged_early = false;   // round 0 of the next U strip is already in flight
     bool pending = false;        // a staging round was issued and not yet waited for
@@ -482,6 +485,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 
     if (tid == 0) {
         mbar_init(&sm.stage_bar, 1);
+        for (int g = 0; g < kRound / 4; ++g) mbar_init(&sm.gbar[g], 1);
+        sm.gfail = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         if (!moe) sm.exl[l0 & 1][0] = p.ex[size_t(l0) * p.E];
     }
@@ -1111,26 +1116,49 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         int nz_total = 0;            // neurons with h != 0 so far (list order)
         for (int j0 = 0; j0 < m && gok; j0 += cap_n) {
             const int k = min(cap_n, m - j0);
+            const int ngr = (k + 3) / 4;   // groups of four neurons, one barrier each
             if (warp == 0) {
-                // lane 0 announces the round's bytes, then lane n copies neuron n
-                if (lane == 0) mbar_arrive_tx(&sm.stage_bar, uint32_t(k) * per_n);
+                // lane 0 announces each group's bytes, then lane n copies neuron n
+                // onto its group's barrier
+                if (lane < ngr) mbar_arrive_tx(&sm.gbar[lane], uint32_t(min(4, k - 4 * lane)) * per_n);
                 __syncwarp();
                 if (lane < k) {
                     const int en = sm.glst[j0 + lane], e = en >> 24, pos = en & 0xffffff;
                     uint8_t *slot = stg + size_t(lane) * per_n;
-                    stage_copy(slot, exs[e]->Wgu + size_t(pos) * p.gu_bytes, uint32_t(p.gu_bytes), &sm.stage_bar);
-                    if (kSpec)
-                        stage_copy(slot + p.gu_bytes, exs[e]->Wd + size_t(pos) * p.wrow, uint32_t(p.wrow),
-                                   &sm.stage_bar);
+                    uint64_t *gb = &sm.gbar[lane >> 2];
+                    stage_copy(slot, exs[e]->Wgu + size_t(pos) * p.gu_bytes, uint32_t(p.gu_bytes), gb);
+                    if (kSpec) stage_copy(slot + p.gu_bytes, exs[e]->Wd + size_t(pos) * p.wrow, uint32_t(p.wrow), gb);
                 }
             }
-            pending = true;
-            if (!stage_wait(&sm, p, spar, bci, &cyc_c)) { gok = false; break; }
-            pending = false;
-            // dots of the round's neurons, four at a time: values 2n (gate) and
-            // 2n + 1 (up); after the reduction lanes 4q .. 4q + 3 hold value q
+            gpend = (1u << ngr) - 1u;
+            // dots of the round's neurons, four at a time as each group lands:
+            // values 2n (gate) and 2n + 1 (up); after the reduction lanes
+            // 4q .. 4q + 3 hold value q
 #pragma unroll 1
             for (int g0 = 0; g0 < k; g0 += 4) {
+                {
+                    // this warp waits (bounded) for the group; every lane then
+                    // observes the completed phase itself
+                    const int g = g0 >> 2;
+                    const uint32_t par = (gpar >> g) & 1u;
+                    bool ok = true;
+                    if (lane == 0 && !mbar_test(&sm.gbar[g], par)) {
+                        const long long t0 = gtimer();
+                        for (unsigned it = 1;; ++it) {
+                            if (mbar_test(&sm.gbar[g], par)) break;
+                            if ((it & 15) == 0 && gtimer() - t0 > p.wait_ns) { ok = false; break; }
+                        }
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) {
+                        if (lane == 0) {
+                            set_error(p.err, kDevTimeout);
+                            sm.gfail = 1;
+                        }
+                        break;
+                    }
+                    mbar_test(&sm.gbar[g], par);   // acquire for this lane
+                }
                 float v[8];
 #pragma unroll
                 for (int n = 0; n < 4; ++n) {
@@ -1147,6 +1175,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 if ((lane & 3) == 0 && q < 2 * k) sm.red[rb][warp][q] = ws;
             }
             cta_sync();
+            if (sm.gfail) { gok = false; break; }
+            gpar ^= gpend;   // every group of the round completed one phase
+            gpend = 0u;
             if (tid < 2 * k) {
                 float a = 0.f;
                 for (int w = 0; w < kConsumerWarps; ++w) a += sm.red[rb][w][tid];
@@ -1278,10 +1309,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     }
     // an early exit may leave one staging round in flight: let it land
     // (bounded) so no bulk copy writes this CTA's shared memory after exit
-    if (pending && tid == 0) {
+    if (tid == 0) {
         const long long t0 = gtimer();
-        while (!mbar_test(&sm.stage_bar, spar) && gtimer() - t0 < p.wait_ns) {
-        }
+        if (pending)
+            while (!mbar_test(&sm.stage_bar, spar) && gtimer() - t0 < p.wait_ns) {
+            }
+        for (int g = 0; g < kRound / 4; ++g)
+            if ((gpend >> g) & 1u)
+                while (!mbar_test(&sm.gbar[g], (gpar >> g) & 1u) && gtimer() - t0 < p.wait_ns) {
+                }
     }
 #undef XP
 }
