@@ -1017,8 +1017,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 const int e = en >> 12, loc = en & 0xfff, pos = s0 + loc;
                 __stcg(pb + j, (unsigned long long)(unsigned(e << 24) | unsigned(pos)) |
                                    ((unsigned long long)__float_as_uint(sm.cbuf[e][loc]) << 32));
-                prefetch_l2(exs[e]->Wgu + size_t(pos) * p.gu_bytes, uint32_t(p.gu_bytes));
-                if (kSpec) prefetch_l2(exs[e]->Wd + size_t(pos) * p.wrow, uint32_t(p.wrow));
+                prefetch_l2(exs[e]->Wgu + size_t(pos) * p.rec_bytes, uint32_t(kSpec ? p.rec_bytes : p.gu_bytes));
             }
             if (tid == 0) __stcg(p.counts + b, nl);
         }
@@ -1064,7 +1063,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         // shared memory; the dots of all of them are reduced at once.
         const long long cc0 = clock64();
         const int m = sm.share_n;
-        const int per_n = p.gu_bytes + (kSpec ? p.wrow : 0);   // bytes per neuron in a round
+        const int per_n = kSpec ? p.rec_bytes : p.gu_bytes;   // bytes per neuron in a round (its record)
         const int cap_n = min(kRound, kStageBytes / per_n);
         // the next layer's V block and biases start moving towards L2 now
         if (tid == kThreads - 1 && !moe && l + 1 < l1) {
@@ -1126,8 +1125,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     const int en = sm.glst[j0 + lane], e = en >> 24, pos = en & 0xffffff;
                     uint8_t *slot = stg + size_t(lane) * per_n;
                     uint64_t *gb = &sm.gbar[lane >> 2];
-                    stage_copy(slot, exs[e]->Wgu + size_t(pos) * p.gu_bytes, uint32_t(p.gu_bytes), gb);
-                    if (kSpec) stage_copy(slot + p.gu_bytes, exs[e]->Wd + size_t(pos) * p.wrow, uint32_t(p.wrow), gb);
+                    stage_copy(slot, exs[e]->Wgu + size_t(pos) * p.rec_bytes, uint32_t(per_n), gb);
                 }
             }
             gpend = (1u << ngr) - 1u;
@@ -1251,7 +1249,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     __syncwarp();
                     for (int n = lane; n < k; n += 32) {
                         const int en = sm.nz[q0 + n], e = en >> 24, pos = en & 0xffffff;
-                        stage_copy(stg + size_t(n) * p.wrow, exs[e]->Wd + size_t(pos) * p.wrow,
+                        stage_copy(stg + size_t(n) * p.wrow, exs[e]->Wd + size_t(pos) * p.wd_stride,
                                    uint32_t(p.wrow), &sm.stage_bar);
                     }
                 }

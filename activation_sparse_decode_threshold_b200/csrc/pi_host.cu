@@ -72,6 +72,7 @@ struct pi_ffn {
     int wfmt = 0, pfmt = 0, gated = 0;
     int vrow = 0, urow = 0, wrow = 0;
     int u_swz = 0;
+    bool spec = false;
     std::vector<int32_t> strip_off;
     std::vector<int32_t> grp_off;              // column slices in 8-column groups
     std::vector<std::vector<int32_t>> perm;   // [layer * E + e]
@@ -157,6 +158,9 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
     h->wfmt = fmt_of(D.w_dtype);
     h->pfmt = fmt_of(D.pred_dtype);
     h->gated = D.act != PI_ACT_RELU;
+    // ReLU / ReGLU: z > 0 nearly always means h != 0, so a predicted neuron's
+    // W_down row is fetched with its input rows (speculatively)
+    h->spec = D.act != PI_ACT_DRELU;
     h->vrow = D.d_model * pb;
     h->urow = D.rank * pb;
     // 16-bit predictors feed tensor-core dots through 8-row matrix loads; rows
@@ -328,13 +332,17 @@ pi_status pi_ffn_load_layer(pi_ffn_t h, int layer, const pi_expert_weights *expe
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     PI_CUDA(cudaSetDevice(D.device), "cudaSetDevice");
+    // neuron records: gate row (+ up row); for the speculative kinds the W_down
+    // row joins the record, so one copy fetches everything a neuron needs
     const int gu_bytes = (h->gated ? 2 : 1) * h->wrow;
+    const bool spec = h->spec;
+    const int rec_bytes = gu_bytes + (spec ? h->wrow : 0);
     const size_t o_V = 0;
     const size_t o_U = up256(o_V + size_t(r) * h->vrow);
     const size_t o_c = up256(o_U + size_t(F) * h->urow);
     const size_t o_g = up256(o_c + sizeof(float) * F);
-    const size_t o_d = up256(o_g + size_t(F) * gu_bytes);
-    const size_t total = up256(o_d + size_t(F) * h->wrow);
+    const size_t o_d = up256(o_g + size_t(F) * rec_bytes);
+    const size_t total = spec ? o_d : up256(o_d + size_t(F) * h->wrow);
     int32_t *d_perm = nullptr;
     PI_CUDA(cudaMallocAsync(&d_perm, sizeof(int32_t) * F, st), "cudaMallocAsync(perm)");
     for (int e = 0; e < E; ++e) {
@@ -365,26 +373,33 @@ pi_status pi_ffn_load_layer(pi_ffn_t h, int layer, const pi_expert_weights *expe
             const int qb = d / 2, sb = d / 16;
             const uint8_t *sg8 = static_cast<const uint8_t *>(w.s_gate);
             const uint8_t *su8 = static_cast<const uint8_t *>(w.s_up);
-            const uint8_t *src[4] = {g8, sg8, u8, su8};
-            const int rb[4] = {qb, sb, qb, sb};
-            PI_CUDA(pi::repack_rows(m + o_g, d_perm, F, h->gated ? 4 : 2, src, rb, st), "repack gate/up");
-            const uint8_t *dsrc[2] = {static_cast<const uint8_t *>(w.w_down),
-                                      static_cast<const uint8_t *>(w.s_down)};
-            const int drb[2] = {qb, sb};
-            PI_CUDA(pi::repack_rows(m + o_d, d_perm, F, 2, dsrc, drb, st), "repack down");
+            const uint8_t *qd8 = static_cast<const uint8_t *>(w.w_down);
+            const uint8_t *sd8 = static_cast<const uint8_t *>(w.s_down);
+            const uint8_t *src[6] = {g8, sg8, u8, su8, qd8, sd8};
+            const int rb[6] = {qb, sb, qb, sb, qb, sb};
+            if (spec) {
+                // gate (, up), down in one record
+                const uint8_t *rs[6] = {g8, sg8, h->gated ? u8 : qd8, h->gated ? su8 : sd8, qd8, sd8};
+                PI_CUDA(pi::repack_rows(m + o_g, d_perm, F, h->gated ? 6 : 4, rs, rb, st), "repack records");
+            } else {
+                PI_CUDA(pi::repack_rows(m + o_g, d_perm, F, h->gated ? 4 : 2, src, rb, st), "repack gate/up");
+                PI_CUDA(pi::repack_rows(m + o_d, d_perm, F, 2, src + 4, rb + 4, st), "repack down");
+            }
         } else {
             const uint8_t *src[2] = {g8, u8};
             const int rb[2] = {h->wrow, h->wrow};
-            PI_CUDA(pi::repack_rows(m + o_g, d_perm, F, h->gated ? 2 : 1, src, rb, st), "repack gate/up");
-            PI_CUDA(pi::repack_down_transpose(static_cast<const uint8_t *>(w.w_down), m + o_d, d_perm, d,
-                                              F, elem_bytes(D.w_dtype), st), "transpose down");
+            PI_CUDA(pi::repack_rows(m + o_g, d_perm, F, h->gated ? 2 : 1, src, rb, st, rec_bytes),
+                    "repack gate/up");
+            PI_CUDA(pi::repack_down_transpose(static_cast<const uint8_t *>(w.w_down), spec ? m + o_g + gu_bytes : m + o_d,
+                                              d_perm, d, F, elem_bytes(D.w_dtype), st, spec ? rec_bytes : 0),
+                    "transpose down");
         }
         pi::ExpertDev &x = h->h_ex[idx];
         x.V = m + o_V;
         x.U = m + o_U;
         x.c = reinterpret_cast<const float *>(m + o_c);
         x.Wgu = m + o_g;
-        x.Wd = m + o_d;
+        x.Wd = spec ? m + o_g + gu_bytes : m + o_d;
         // the table is reused for the next expert: finish this one first
         PI_CUDA(cudaStreamSynchronize(st), "load_layer sync");
     }
@@ -440,7 +455,9 @@ static pi::DecodeParams base_params(pi_ffn_t h)
     p.urow = h->urow;
     p.wrow = h->wrow;
     p.gu_bytes = (h->gated ? 2 : 1) * h->wrow;
-    p.spec_down = D.act != PI_ACT_DRELU;
+    p.spec_down = h->spec;
+    p.rec_bytes = p.gu_bytes + (h->spec ? h->wrow : 0);
+    p.wd_stride = h->spec ? p.rec_bytes : h->wrow;
     p.u_swz = h->u_swz;
     p.t_buf = h->t_buf;
     p.partials = h->partials;
@@ -583,6 +600,8 @@ pi_status pi_dense_ffn_prefill(pi_ffn_t h, int layer_begin, int layer_end, int n
     v.gated = h->gated;
     v.wfmt = h->wfmt;
     v.wrow = h->wrow;
+    v.rec_bytes = (h->gated ? 2 : 1) * h->wrow + (h->spec ? h->wrow : 0);
+    v.wd_stride = h->spec ? v.rec_bytes : h->wrow;
     v.eps = D.eps;
     v.ex = h->h_ex.data();
     v.router = h->router_mem.data();

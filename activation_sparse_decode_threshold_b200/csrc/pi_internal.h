@@ -32,8 +32,10 @@ struct ExpertDev {
                          // columns); MoE: r rows of vrow bytes (rank is not permuted)
     const uint8_t *U;    // F rows of urow bytes, table order
     const float *c;      // F biases, table order
-    const uint8_t *Wgu;  // F input records of gu_bytes, table order
-    const uint8_t *Wd;   // F rows of wrow bytes: W_down columns, neuron-major
+    const uint8_t *Wgu;  // F neuron records, table order, rec_bytes apart: gate row (+ up row)
+                         // (+ the W_down row for the speculative kinds)
+    const uint8_t *Wd;   // F rows of wrow bytes, wd_stride apart: W_down columns, neuron-major
+                         // (inside the records for the speculative kinds)
 };
 
 enum Mode { kModeDecode = 0, kModePredict = 1 };
@@ -49,6 +51,8 @@ struct DecodeParams {
     int vrow, urow, wrow;           // row bytes: V (pred fmt), U (pred fmt), W (weight fmt)
     int gu_bytes;                   // bytes of a neuron's input record (2 * wrow gated)
     int spec_down;                  // prefetch down rows of all predicted-active neurons
+    int rec_bytes;                  // bytes between neuron records (gate|up, plus the down row when spec_down)
+    int wd_stride;                  // bytes between W_down rows (rec_bytes when spec_down, else wrow)
     int u_swz;                      // U rows stored chunk-permuted (repack_u_swizzled)
     int mode, pred_expert;
     // inputs / outputs
@@ -88,9 +92,11 @@ int decode_max_blocks_per_sm(int wfmt, int pfmt, int d);
 // Load-time repack kernels (pi_repack.cu).  repack_rows: dst record p is the
 // concatenation of row perm[p] of each of the n_src sources (row bytes each a
 // multiple of 16).
-constexpr int kMaxRepackSrc = 4;
+constexpr int kMaxRepackSrc = 6;
+// dst_stride: bytes between records (0 = the records' own size).
 cudaError_t repack_rows(uint8_t *dst, const int32_t *perm, int rows, int n_src,
-                        const uint8_t *const *src, const int *row_bytes, cudaStream_t s);
+                        const uint8_t *const *src, const int *row_bytes, cudaStream_t s,
+                        long long dst_stride = 0);
 cudaError_t repack_v_blocks(const uint8_t *V, uint8_t *dst, const int32_t *grp_off, int S, int r,
                             int d, int elem_bytes, cudaStream_t s);
 cudaError_t repack_bias(const float *src, float *dst, const int32_t *perm, int n, cudaStream_t s);
@@ -98,8 +104,9 @@ cudaError_t repack_bias(const float *src, float *dst, const int32_t *perm, int n
 // (row - strip start) mod 8 (row_bytes a multiple of 128); strip_off on the device.
 cudaError_t repack_u_swizzled(uint8_t *dst, const int32_t *perm, int rows, const uint8_t *src, int row_bytes,
                               const int32_t *strip_off, int S, cudaStream_t s);
+// dst_stride_bytes: bytes between neuron rows (0 = d * elem_bytes).
 cudaError_t repack_down_transpose(const uint8_t *w_down, uint8_t *dst, const int32_t *perm,
-                                  int d, int F, int elem_bytes, cudaStream_t s);
+                                  int d, int F, int elem_bytes, cudaStream_t s, long long dst_stride_bytes = 0);
 
 // Sets the message returned by pi_last_error on this host thread.
 void set_last_error(const char *msg);

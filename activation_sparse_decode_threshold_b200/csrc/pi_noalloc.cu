@@ -164,6 +164,8 @@ extern "C" PI_API pi_status pi_predict_noalloc(int d_model, int d_ff, int rank, 
     p.wrow = d_model * pb;
     p.gu_bytes = 2 * p.wrow;
     p.spec_down = 0;
+    p.rec_bytes = p.gu_bytes;
+    p.wd_stride = p.wrow;
     p.u_swz = 0;          // the caller's U rows as they are
     p.mode = pi::kModePredict;
     p.pred_expert = 0;

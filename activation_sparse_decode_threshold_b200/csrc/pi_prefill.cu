@@ -51,14 +51,14 @@ constexpr long long kWaitNs = 2000000000LL;
 enum GemmKind { kGU = 0, kDOWN = 1 };
 
 struct PrefillExpert {
-    const uint8_t *Wgu;   // F records of gu_bytes (gate row, then up row when gated)
+    const uint8_t *Wgu;   // F neuron records rec_bytes apart (gate row, then up row when gated)
     const uint8_t *Wd;    // F rows of wrow bytes (W_down columns)
     const float *c;       // F biases
 };
 
 struct GemmParams {
     PrefillExpert ex[kMaxExperts];
-    int E, d, F, gated, act, wrow, gu_bytes;
+    int E, d, F, gated, act, wrow, rec_bytes, wd_stride;
     const int32_t *e_off;     // [E + 1] first list position of each expert
     const int32_t *e_tok;     // [2T] token of each list position
     const void *X16;          // [T x d] normalised inputs (element type of the MMA)
@@ -184,10 +184,11 @@ __device__ __forceinline__ uint32_t mnmaj_off(int ng, int k)
 }
 
 // 16 INT4 weights (8 bytes of nibbles, low nibble = even element) with their
-// group scale -> 16 fp16 values s * (n - 8), on the half-precision pipe: a
-// nibble n placed in the fraction of the half 1024.0 gives 1024 + n exactly,
-// subtracting 1032 gives n - 8 exactly, and the product with s is rounded
-// once, as a rounding of the exact s * (n - 8) to fp16.
+// group scale -> 16 fp16 values s * (n - 8), on the integer and half pipes: a
+// nibble n placed in the fraction of the half 1024.0 (byte permutes put each
+// nibble under a 0x64 exponent byte) gives 1024 + n exactly, subtracting
+// 1032 gives n - 8 exactly, and the product with s is rounded once, as a
+// rounding of the exact s * (n - 8) to fp16.
 __device__ __forceinline__ void dequant16(uint2 q, __half s, uint4 &lo, uint4 &hi)
 {
     const __half2 s2 = __halves2half2(s, s);
@@ -196,11 +197,13 @@ __device__ __forceinline__ void dequant16(uint2 q, __half s, uint4 &lo, uint4 &h
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
         const uint32_t w = i == 0 ? q.x : q.y;
+        const uint32_t ev = w & 0x0F0F0F0Fu, od = (w >> 4) & 0x0F0F0F0Fu;   // even / odd elements
+        const uint32_t p01 = __byte_perm(ev, od, 0x5140), p23 = __byte_perm(ev, od, 0x7362);
+        const uint32_t bits[4] = {__byte_perm(p01, 0x64646464u, 0x4140), __byte_perm(p01, 0x64646464u, 0x4342),
+                                  __byte_perm(p23, 0x64646464u, 0x4140), __byte_perm(p23, 0x64646464u, 0x4342)};
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-            const uint32_t t = w >> (8 * m);
-            const uint32_t bits = (t & 0xFu) | ((t & 0xF0u) << 12) | 0x64006400u;
-            __half2 h = *reinterpret_cast<const __half2 *>(&bits);
+            __half2 h = *reinterpret_cast<const __half2 *>(&bits[m]);
             h = __hmul2(__hsub2(h, off), s2);
             o[4 * i + m] = *reinterpret_cast<const uint32_t *>(&h);
         }
@@ -331,7 +334,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
                         const int row = (rest & 31) * 8 + (c & 7), kc = (rest >> 5) * 4 + ((c >> 3) & 3);
                         const int nn = n0 / 2 + (row >> 1);
                         const bool ok = nn < F && (p.gated || (row & 1) == 0);
-                        const uint8_t *rec = ex.Wgu + size_t(ok ? nn : 0) * p.gu_bytes + ((row & 1) ? p.wrow : 0);
+                        const uint8_t *rec = ex.Wgu + size_t(ok ? nn : 0) * p.rec_bytes + ((row & 1) ? p.wrow : 0);
                         cp_async16(B + kmaj_off(row, kc), rec + (k0 + kc * 8) * 2, ok);
                     }
                 } else {
@@ -339,7 +342,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
                     for (int i = 0; i < BK * (BN / 8) / kProducers; ++i) {   // 64 k-rows x 32 chunks, MN-major
                         const int c = pt + kProducers * i, rest = c >> 5;
                         const int k = (rest & 7) * 8 + (c & 7), ng = (rest >> 3) * 4 + ((c >> 3) & 3);
-                        const uint8_t *row = ex.Wd + size_t(k0 + k) * p.wrow + (n0 + ng * 8) * 2;
+                        const uint8_t *row = ex.Wd + size_t(k0 + k) * p.wd_stride + (n0 + ng * 8) * 2;
                         cp_async16(B + mnmaj_off(ng, k), row, true);
                     }
                 }
@@ -352,28 +355,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         // a 16-byte shared store touches 8 different bank groups, and a row's
         // 32 bytes come from 4 lanes.  Down item: W_down row k (8 per warp) and
         // 16 output columns (4 consecutive groups per row).
+        // source rows of this thread's INT4 items (fixed across K steps)
+        const uint8_t *r_src[4];
+        int r_off[4];    // element offset of the item inside a K step (GU) or column offset (down)
+        bool r_ok[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int c = pt + kProducers * i;
+            if constexpr (KIND == kGU) {
+                const int row = (c >> 5) * 8 + (c & 7), q16 = (c >> 3) & 3;
+                const int nn = n0 / 2 + (row >> 1);
+                r_ok[i] = nn < F && (p.gated || (row & 1) == 0);
+                r_src[i] = ex.Wgu + size_t(r_ok[i] ? nn : 0) * p.rec_bytes + ((row & 1) ? p.wrow : 0);
+                r_off[i] = 16 * q16;
+            } else {
+                const int rest = c >> 5;
+                const int k = (rest & 7) * 8 + (c & 7), g16 = (rest >> 3) * 4 + ((c >> 3) & 3);
+                r_ok[i] = true;
+                r_src[i] = ex.Wd + size_t(k) * p.wd_stride;    // + k0 rows per step
+                r_off[i] = n0 + 16 * g16;
+            }
+        }
         auto load_raw = [&](int kt, RawI4 &r) {
             const int k0 = kt * BK;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const int c = pt + kProducers * i;
                 if constexpr (KIND == kGU) {
-                    const int row = (c >> 5) * 8 + (c & 7), q16 = (c >> 3) & 3;   // elements k0 + 16 q16 .. +15
-                    const int nn = n0 / 2 + (row >> 1);
-                    const bool ok = nn < F && (p.gated || (row & 1) == 0);
                     r.q[i] = make_uint2(0u, 0u);
                     r.sc[i] = 0;
-                    if (ok) {
-                        const uint8_t *rec = ex.Wgu + size_t(nn) * p.gu_bytes + ((row & 1) ? p.wrow : 0);
-                        const int kk = k0 + 16 * q16;
-                        r.q[i] = __ldg(reinterpret_cast<const uint2 *>(rec + kk / 2));
-                        r.sc[i] = __ldg(reinterpret_cast<const unsigned short *>(rec + d / 2) + kk / 32);
+                    if (r_ok[i]) {
+                        const int kk = k0 + r_off[i];
+                        r.q[i] = __ldg(reinterpret_cast<const uint2 *>(r_src[i] + kk / 2));
+                        r.sc[i] = __ldg(reinterpret_cast<const unsigned short *>(r_src[i] + d / 2) + kk / 32);
                     }
                 } else {
-                    const int rest = c >> 5;
-                    const int k = (rest & 7) * 8 + (c & 7), g16 = (rest >> 3) * 4 + ((c >> 3) & 3);
-                    const uint8_t *row = ex.Wd + size_t(k0 + k) * p.wrow;
-                    const int nn = n0 + 16 * g16;
+                    const uint8_t *row = r_src[i] + size_t(k0) * p.wd_stride;
+                    const int nn = r_off[i];
                     r.q[i] = __ldg(reinterpret_cast<const uint2 *>(row + nn / 2));
                     r.sc[i] = __ldg(reinterpret_cast<const unsigned short *>(row + d / 2) + nn / 32);
                 }
@@ -756,7 +773,8 @@ int prefill_run(PrefillState **state, const PrefillView &v, int l0, int l1, int 
     gp.gated = v.gated;
     gp.act = v.act;
     gp.wrow = v.wrow;
-    gp.gu_bytes = (v.gated ? 2 : 1) * v.wrow;
+    gp.rec_bytes = v.rec_bytes;
+    gp.wd_stride = v.wd_stride;
     gp.e_off = tp.e_off;
     gp.e_tok = tp.e_tok;
     gp.X16 = tp.X16;

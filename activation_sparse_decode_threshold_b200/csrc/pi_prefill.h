@@ -13,6 +13,7 @@ struct PrefillState;
 // What the prefill needs from a handle (weights in neuron-table order).
 struct PrefillView {
     int d, F, E, top_k, act, gated, wfmt, wrow;
+    int rec_bytes, wd_stride;                   // neuron record stride, W_down row stride (bytes)
     float eps;
     const ExpertDev *ex;                        // host copy [n_layers * E]
     uint8_t *const *router;                     // host copy [n_layers] device pointers

@@ -22,14 +22,12 @@ struct RepackSrc {
 };
 
 __global__ void k_repack_rows(uint8_t *__restrict__ dst, const int32_t *__restrict__ perm, int rows,
-                              RepackSrc rs)
+                              RepackSrc rs, long long dst_stride)
 {
     const int p = blockIdx.x;
     if (p >= rows) return;
     const long long o = perm[p];
-    int out_rb = 0;
-    for (int i = 0; i < rs.n; ++i) out_rb += rs.bytes[i];
-    uint8_t *t = dst + (long long)p * out_rb;
+    uint8_t *t = dst + (long long)p * dst_stride;
     for (int i = 0; i < rs.n; ++i) {
         const uint4 *s = reinterpret_cast<const uint4 *>(rs.src[i] + o * rs.bytes[i]);
         uint4 *tt = reinterpret_cast<uint4 *>(t);
@@ -70,7 +68,7 @@ __global__ void k_repack_bias(const float *__restrict__ src, float *__restrict__
 
 template <typename T>
 __global__ void k_down_transpose(const T *__restrict__ w, T *__restrict__ dst,
-                                 const int32_t *__restrict__ inv, int d, int F)
+                                 const int32_t *__restrict__ inv, int d, int F, long long dst_stride)
 {
     __shared__ T tile[32][33];
     const int i0 = blockIdx.x * 32, j0 = blockIdx.y * 32;
@@ -82,7 +80,7 @@ __global__ void k_down_transpose(const T *__restrict__ w, T *__restrict__ dst,
     __syncthreads();
     for (int yy = ty; yy < 32; yy += 8) {
         const int i = i0 + yy, j = j0 + tx;
-        if (i < F && j < d) dst[(long long)inv[i] * d + j] = tile[tx][yy];
+        if (i < F && j < d) dst[(long long)inv[i] * dst_stride + j] = tile[tx][yy];
     }
 }
 
@@ -125,7 +123,7 @@ cudaError_t repack_v_blocks(const uint8_t *V, uint8_t *dst, const int32_t *grp_o
 }
 
 cudaError_t repack_rows(uint8_t *dst, const int32_t *perm, int rows, int n_src,
-                        const uint8_t *const *src, const int *row_bytes, cudaStream_t s)
+                        const uint8_t *const *src, const int *row_bytes, cudaStream_t s, long long dst_stride)
 {
     if (rows <= 0) return cudaSuccess;
     if (n_src < 1 || n_src > kMaxRepackSrc) return cudaErrorInvalidValue;
@@ -135,7 +133,11 @@ cudaError_t repack_rows(uint8_t *dst, const int32_t *perm, int rows, int n_src,
         rs.src[i] = src[i];
         rs.bytes[i] = row_bytes[i];
     }
-    k_repack_rows<<<rows, 128, 0, s>>>(dst, perm, rows, rs);
+    long long packed = 0;
+    for (int i = 0; i < n_src; ++i) packed += row_bytes[i];
+    if (dst_stride == 0) dst_stride = packed;
+    if (dst_stride < packed || dst_stride % 16 != 0) return cudaErrorInvalidValue;
+    k_repack_rows<<<rows, 128, 0, s>>>(dst, perm, rows, rs, dst_stride);
     return cudaGetLastError();
 }
 
@@ -158,8 +160,11 @@ cudaError_t repack_bias(const float *src, float *dst, const int32_t *perm, int n
 // `perm` is the table (device).  The inverse table lives in a temporary
 // stream-ordered allocation for the duration of the transpose (load time only).
 cudaError_t repack_down_transpose(const uint8_t *w_down, uint8_t *dst, const int32_t *perm,
-                                  int d, int F, int elem_bytes, cudaStream_t s)
+                                  int d, int F, int elem_bytes, cudaStream_t s, long long dst_stride_bytes)
 {
+    if (dst_stride_bytes == 0) dst_stride_bytes = (long long)d * elem_bytes;
+    if (dst_stride_bytes % elem_bytes != 0) return cudaErrorInvalidValue;
+    const long long stride = dst_stride_bytes / elem_bytes;
     int32_t *inv = nullptr;
     cudaError_t e = cudaMallocAsync(&inv, sizeof(int32_t) * size_t(F), s);
     if (e != cudaSuccess) return e;
@@ -167,10 +172,10 @@ cudaError_t repack_down_transpose(const uint8_t *w_down, uint8_t *dst, const int
     dim3 grid((F + 31) / 32, (d + 31) / 32), block(32, 8);
     if (elem_bytes == 4)
         k_down_transpose<uint32_t><<<grid, block, 0, s>>>(
-            reinterpret_cast<const uint32_t *>(w_down), reinterpret_cast<uint32_t *>(dst), inv, d, F);
+            reinterpret_cast<const uint32_t *>(w_down), reinterpret_cast<uint32_t *>(dst), inv, d, F, stride);
     else
         k_down_transpose<uint16_t><<<grid, block, 0, s>>>(
-            reinterpret_cast<const uint16_t *>(w_down), reinterpret_cast<uint16_t *>(dst), inv, d, F);
+            reinterpret_cast<const uint16_t *>(w_down), reinterpret_cast<uint16_t *>(dst), inv, d, F, stride);
     e = cudaGetLastError();
     cudaError_t e2 = cudaFreeAsync(inv, s);
     return e != cudaSuccess ? e : e2;

@@ -25,6 +25,11 @@ SMALL = {
                                   n_experts=4),
     "fewer-neurons-than-strips": synth.small(synth.CONFIGS["llama7b"], n_layers=2, d=256, F=100,
                                              rank=32),
+    # INT4 experts with the speculative kinds (gate|up|down records)
+    "reglu-int4": synth.small(synth.CONFIGS["llama7b"], n_layers=2, d=512, F=1200, rank=64,
+                              wdtype="int4g32"),
+    "relu-int4-nongated": synth.small(synth.CONFIGS["falcon40b"], n_layers=2, d=512, F=1500, rank=64,
+                                      wdtype="int4g32"),
 }
 
 

@@ -22,6 +22,8 @@ SMALL = {
     "relu-f16-nongated": synth.small(synth.CONFIGS["falcon40b"], n_layers=2, d=512, F=2048, rank=64),
     "moe-int4-drelu": synth.small(synth.CONFIGS["mixtral47b"], n_layers=2, d=512, F=1024, rank=64,
                                   n_experts=4),
+    "reglu-int4": synth.small(synth.CONFIGS["llama7b"], n_layers=2, d=512, F=1024, rank=64,
+                              wdtype="int4g32"),
 }
 
 # logits closer than this between the 2nd and 3rd expert make the choice of
