@@ -38,7 +38,9 @@ namespace pi {
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64, NSTAGE = 4;
-constexpr int kProducerWarps = 8, kProducers = 32 * kProducerWarps;
+constexpr int kProducerWarps = 16, kProducers = 32 * kProducerWarps;
+constexpr int kRI = BN * 4 / kProducers;          // INT4 items (16 weights) per producer thread per stage
+constexpr int kEpiCols = BN / (kProducerWarps / 4); // accumulator columns per epilogue warp
 constexpr int kGemmThreads = kProducers + 32;    // + the MMA warp
 constexpr int kLag = 2;                          // stages between issuing a stage's copies and publishing it
 constexpr int kATileBytes = BM * BK * 2;          // 16 KB
@@ -213,9 +215,9 @@ __device__ __forceinline__ void dequant16(uint2 q, __half s, uint4 &lo, uint4 &h
 }
 
 // ---------------------------------------------------------------------------
-// GEMM kernel.  Warps 0-7 produce stages (cp.async for 16-bit operands, INT4
-// weights through registers one stage ahead and dequantised into the tile),
-// warp 8 issues the MMAs from one thread, and warps 0-7 run the epilogue
+// GEMM kernel.  Warps 0-15 produce stages (cp.async for 16-bit operands, INT4
+// weights through registers three stages ahead and dequantised into the tile),
+// warp 16 issues the MMAs from one thread, and warps 0-15 run the epilogue
 // once the accumulator is complete.  Stage s is published on full[s] (every
 // producer thread arrives after its copies landed and a proxy fence) and
 // freed on empty[s] by tcgen05.commit.
@@ -227,8 +229,8 @@ template <> __device__ __forceinline__ __half from_f<__half>(float x) { return _
 template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
 struct RawI4 {
-    uint2 q[4];
-    unsigned short sc[4];
+    uint2 q[kRI];
+    unsigned short sc[kRI];
 };
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *b)
@@ -356,11 +358,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         // 32 bytes come from 4 lanes.  Down item: W_down row k (8 per warp) and
         // 16 output columns (4 consecutive groups per row).
         // source rows of this thread's INT4 items (fixed across K steps)
-        const uint8_t *r_src[4];
-        int r_off[4];    // element offset of the item inside a K step (GU) or column offset (down)
-        bool r_ok[4];
+        const uint8_t *r_src[kRI];
+        int r_off[kRI];    // element offset of the item inside a K step (GU) or column offset (down)
+        bool r_ok[kRI];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < kRI; ++i) {
             const int c = pt + kProducers * i;
             if constexpr (KIND == kGU) {
                 const int row = (c >> 5) * 8 + (c & 7), q16 = (c >> 3) & 3;
@@ -379,7 +381,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         auto load_raw = [&](int kt, RawI4 &r) {
             const int k0 = kt * BK;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < kRI; ++i) {
                 if constexpr (KIND == kGU) {
                     r.q[i] = make_uint2(0u, 0u);
                     r.sc[i] = 0;
@@ -399,7 +401,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         auto store_raw = [&](const RawI4 &r, int s) {
             uint8_t *B = smem + s * kStageBytes + kATileBytes;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < kRI; ++i) {
                 const int c = pt + kProducers * i;
                 uint4 lo, hi;
                 dequant16(r.q[i], __ushort_as_half(r.sc[i]), lo, hi);
@@ -466,15 +468,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         const int row = 32 * (warp & 3) + lane;
         const int lr = mrow0 + row;
         const bool valid = lr < mrow_end && !abort_sh;
-        const int col0 = 128 * (warp >> 2);
+        const int col0 = kEpiCols * (warp >> 2);
         if (KIND == kDOWN && nk == 0) {
             // an empty K range still owns its partial: zeros
             if (valid) {
                 float *dst = p.Ypart + (size_t(blockIdx.z) * p.rows_cap + lr) * d + n0 + col0;
-                for (int j2 = 0; j2 < 128; j2 += 4) *reinterpret_cast<float4 *>(dst + j2) = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int j2 = 0; j2 < kEpiCols; j2 += 4) *reinterpret_cast<float4 *>(dst + j2) = make_float4(0.f, 0.f, 0.f, 0.f);
             }
         } else if (!abort_sh) {
-            for (int cc = 0; cc < 128; cc += 16) {
+            for (int cc = 0; cc < kEpiCols; cc += 16) {
                 float v[16];
                 tmem_ld16(tmem + (uint32_t(32 * (warp & 3)) << 16) + uint32_t(col0 + cc), v);
                 if (!valid) continue;
