@@ -68,7 +68,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     with ThreadPoolExecutor(max_workers=min(os.cpu_count() or 4, max(1, len(jobs)))) as ex:
         list(ex.map(run, jobs))
     if force or jobs or not os.path.exists(OUT):
-        cmd = [nvcc, *ARCH, "-shared", "-o", OUT + ".tmp", *objs, "-lcudart", "-lcuda"]
+        cmd = [nvcc, *ARCH, "-shared", "-o", OUT + ".tmp", *objs, "-lcudart"]
         run(cmd)
         os.replace(OUT + ".tmp", OUT)
     return OUT

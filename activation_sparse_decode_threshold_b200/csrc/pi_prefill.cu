@@ -25,6 +25,7 @@
 // one elected thread issues tcgen05.mma (kind::f16, fp32 accumulators in
 // TMEM) four K=16 steps per stage, and tcgen05.commit on a per-stage
 // mbarrier frees the stage.  Three stages.  Every wait is bounded.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -42,7 +43,7 @@ constexpr int kProducerWarps = 16, kProducers = 32 * kProducerWarps;
 constexpr int kRI = BN * 4 / kProducers;          // INT4 items (16 weights) per producer thread per stage
 constexpr int kEpiCols = BN / (kProducerWarps / 4); // accumulator columns per epilogue warp
 constexpr int kGemmThreads = kProducers + 32;    // + the MMA warp
-constexpr int kLag = 2;                          // stages between issuing a stage's copies and publishing it
+constexpr int kLag = 1;                          // stages between issuing a stage's copies and publishing it
 constexpr int kATileBytes = BM * BK * 2;          // 16 KB
 constexpr int kBTileBytes = BN * BK * 2;          // 32 KB
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
@@ -63,11 +64,13 @@ struct GemmParams {
     int E, d, F, gated, act, wrow, rec_bytes, wd_stride;
     const int32_t *e_off;     // [E + 1] first list position of each expert
     const int32_t *e_tok;     // [2T] token of each list position
-    const void *X16;          // [T x d] normalised inputs (element type of the MMA)
     void *H;                  // [2T x F] activations per list position (same type)
     float *Ypart;             // [kSplitK x 2T x d] down partials
     int rows_cap;             // 2T
     int *err;
+    // A operand: rows of list positions (normalised inputs sorted by expert for
+    // the gate/up GEMM, H for the down GEMM), 64 x 128 boxes with 128-byte swizzle
+    alignas(64) CUtensorMap tmA;
 };
 
 // ---------------------------------------------------------------------------
@@ -121,6 +124,31 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
+__device__ __forceinline__ void mbar_arrive_tx(uint64_t *b, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(s2u(b)), "r"(bytes) : "memory");
+}
+// 2-D tiled TMA load of box (x, y) into shared memory, completion on `bar`
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(s2u(dst)), "l"(map), "r"(x), "r"(y), "r"(s2u(bar))
+        : "memory");
+}
+// shared-memory matrix descriptor of a K-major tile with 128-byte swizzle (rows
+// of 128 bytes, 8-row groups 1024 bytes apart, as the tensor-map load writes
+// them); the start address moves by 32 bytes per 16-element K step
+__device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t saddr)
+{
+    uint64_t d = 0;
+    d |= uint64_t((saddr >> 4) & 0x3fff);
+    d |= uint64_t(1) << 16;             // leading byte offset (unused with this layout)
+    d |= uint64_t(1024 >> 4) << 32;     // stride byte offset: 8 rows x 128 bytes
+    d |= uint64_t(1) << 46;             // descriptor version
+    d |= uint64_t(2) << 61;             // 128-byte swizzle
+    return d;
+}
 // shared-memory matrix descriptor: canonical layout without swizzle; start,
 // leading (K direction) and stride (M/N direction) byte offsets in 16-byte
 // units; descriptor version 1
@@ -243,11 +271,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
 {
     constexpr bool I4 = W == 2;
     using AT = typename Elem<W>::T;
-    const AT *X16 = reinterpret_cast<const AT *>(p.X16);
     AT *Hbuf = reinterpret_cast<AT *>(p.H);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t full[NSTAGE], empty[NSTAGE], done;
+    __shared__ uint64_t full[NSTAGE], afull[NSTAGE], empty[NSTAGE], done;
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
 
@@ -282,6 +309,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     if (tid == 0) {
         for (int s = 0; s < NSTAGE; ++s) {
             mbar_init(&full[s], kProducers);
+            mbar_init(&afull[s], 1);
             mbar_init(&empty[s], 1);
         }
         mbar_init(&done, 1);
@@ -301,33 +329,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     if (warp < kProducerWarps) {
         // ------------------------------ producers ------------------------------
         const int pt = tid;   // 0 .. 255
-        // Chunk-to-lane mapping: a warp covers 8 consecutive rows x 4
-        // consecutive 16-byte chunks, so its global reads are whole 32-byte
-        // sectors and its shared stores are four 128-byte runs (no bank
-        // conflicts beyond the minimum).  Item i of this thread: rows from
-        // (c >> 5) and c & 7, chunks from (c >> 3) & 3, with c = pt + 256 i.
-        // Source rows do not change across K steps: resolved once here.
-        constexpr int kAI = BM * (BK / 8) / kProducers;    // 4 A chunks per thread per stage
-        const uint8_t *a_src[kAI];
-        uint32_t a_dst[kAI];
-        bool a_ok[kAI];
-#pragma unroll
-        for (int i = 0; i < kAI; ++i) {
-            const int c = pt + kProducers * i, rest = c >> 5;
-            const int row = (rest & 15) * 8 + (c & 7), kc = (rest >> 4) * 4 + ((c >> 3) & 3);
-            const int lr = mrow0 + row;
-            a_ok[i] = lr < mrow_end;
-            const AT *src = KIND == kGU ? X16 + size_t(a_ok[i] ? p.e_tok[lr] : 0) * d
-                                        : Hbuf + size_t(a_ok[i] ? lr : 0) * F;
-            a_src[i] = reinterpret_cast<const uint8_t *>(src) + kc * 16;
-            a_dst[i] = kmaj_off(row, kc);
-        }
+        // Chunk-to-lane mapping of the B tile: a warp covers 8 consecutive
+        // rows x 4 consecutive 16-byte chunks, so its global reads are whole
+        // 32-byte sectors and its shared stores are four 128-byte runs (no bank
+        // conflicts beyond the minimum).  The A tile comes by tensor-map load.
         auto issue_async = [&](int kt, int s) {
             uint8_t *A = smem + s * kStageBytes;
             uint8_t *B = A + kATileBytes;
             const int k0 = kt * BK;
-#pragma unroll
-            for (int i = 0; i < kAI; ++i) cp_async16(A + a_dst[i], a_src[i] + k0 * 2, a_ok[i]);
+            if (pt == 0) {
+                // A: 128 list positions x 64 elements; rows past the expert's are
+                // loaded too and their results discarded, rows past the buffer read 0
+                mbar_arrive_tx(&afull[s], uint32_t(kATileBytes));
+                tma_load_2d(A, &p.tmA, k0, mrow0, &afull[s]);
+            }
             if constexpr (!I4) {
                 if constexpr (KIND == kGU) {
 #pragma unroll
@@ -349,7 +364,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
                     }
                 }
             }
-            cp_async_commit();
+            if constexpr (!I4) cp_async_commit();
         };
         // INT4: the raw nibbles and scales of a stage, loaded into registers.
         // GU item: 16 elements (chunk pair q16) of one row; the 8 lanes of each
@@ -443,10 +458,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
             if (abort_sh) { stop = true; return; }
             issue_async(kt0 + j, s);
             if constexpr (I4) {
+                // dequantised synchronously: the stage is published at once
                 if (j + 3 < nk) load_raw(kt0 + j + 3, nxt);
                 store_raw(cur, s);
-            }
-            if (j >= kLag) {
+                publish(j);
+            } else if (j >= kLag) {
                 cp_async_wait<kLag>();
                 publish(j - kLag);
             }
@@ -460,8 +476,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         }
         // drain: publish the stages still in flight (all of them on abort too,
         // so that no copy is outstanding at exit)
-        cp_async_wait<0>();
-        for (int q = max(0, j - kLag); q < j; ++q) publish(q);
+        if constexpr (!I4) {
+            cp_async_wait<0>();
+            for (int q = max(0, j - kLag); q < j; ++q) publish(q);
+        }
+        // no tensor-map load may still be writing this CTA's shared memory at
+        // exit: the issuing thread waits (bounded) for the last loads it issued
+        if (pt == 0)
+            for (int q = max(0, j - NSTAGE); q < j; ++q)
+                mbar_wait(&afull[q % NSTAGE], uint32_t((q / NSTAGE) & 1), p.err);
         // epilogue: wait for the accumulator
         if (nk > 0 && !abort_sh && !mbar_wait(&done, 0u, p.err)) abort_sh = 1;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -510,13 +533,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
             int issued = 0;
             for (int j = 0; j < nk; ++j) {
                 const int s = j % NSTAGE;
-                if (!mbar_wait(&full[s], uint32_t((j / NSTAGE) & 1), p.err)) { abort_sh = 1; break; }
+                if (!mbar_wait(&full[s], uint32_t((j / NSTAGE) & 1), p.err) ||
+                    !mbar_wait(&afull[s], uint32_t((j / NSTAGE) & 1), p.err)) { abort_sh = 1; break; }
                 if (abort_sh) break;
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                 const uint32_t a0 = s2u(smem + s * kStageBytes), b0 = a0 + kATileBytes;
 #pragma unroll
                 for (int ks = 0; ks < BK / 16; ++ks) {
-                    const uint64_t ad = make_sdesc(a0 + ks * 256, 128, BK / 8 * 128);
+                    const uint64_t ad = make_sdesc_sw128(a0 + ks * 32);
                     const uint64_t bd = make_sdesc(b0 + ks * 256, 128, BK / 8 * 128);
                     umma(tmem, ad, bd, idesc, j > 0 || ks > 0);
                 }
@@ -675,6 +699,17 @@ __global__ void __launch_bounds__(kSortThreads) k_sort(TokenParams p)
     }
 }
 
+// The normalised inputs in list order (rows of each expert's tokens
+// contiguous), for the tensor-map loads of the gate/up GEMM.  16-bit elements.
+__global__ void k_gather_x(TokenParams p, uint8_t *__restrict__ xs)
+{
+    const int q = blockIdx.x;
+    if (q >= p.e_off[p.E]) return;
+    const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(p.X16) + size_t(p.e_tok[q]) * p.d * 2);
+    uint4 *dst = reinterpret_cast<uint4 *>(xs + size_t(q) * p.d * 2);
+    for (int i = threadIdx.x; i < p.d / 8; i += blockDim.x) dst[i] = src[i];
+}
+
 // r += sum over the token's experts (ascending index) of w * (sum of the
 // K-split partials in split order)
 __global__ void k_combine(TokenParams p)
@@ -697,6 +732,24 @@ __global__ void k_combine(TokenParams p)
 // ---------------------------------------------------------------------------
 // Host
 // ---------------------------------------------------------------------------
+// The tensor-map encoder is a driver entry point, looked up through the
+// runtime so that the library has no link-time dependency on the driver.
+typedef CUresult (*TensorMapEncodeFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                      const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                      CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                      CUtensorMapFloatOOBfill);
+static TensorMapEncodeFn tensor_map_encoder()
+{
+    static TensorMapEncodeFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<TensorMapEncodeFn>(ptr);
+    }
+    return fn;
+}
 struct PrefillState {
     int T = 0, d = 0, F = 0;
     uint8_t *buf = nullptr;
@@ -718,7 +771,8 @@ int prefill_run(PrefillState **state, const PrefillView &v, int l0, int l1, int 
     }
     const int rows_cap = 2 * T;
     const size_t o_x16 = 0;
-    const size_t o_h = up256(o_x16 + sizeof(__half) * size_t(T) * v.d);
+    const size_t o_xs = up256(o_x16 + sizeof(__half) * size_t(T) * v.d);
+    const size_t o_h = up256(o_xs + sizeof(__half) * size_t(rows_cap) * v.d);
     const size_t o_y = up256(o_h + sizeof(__half) * size_t(rows_cap) * v.F);
     const size_t o_re = up256(o_y + sizeof(float) * size_t(kSplitK) * rows_cap * v.d);
     const size_t o_rw = up256(o_re + sizeof(int32_t) * 2 * T);
@@ -779,12 +833,35 @@ int prefill_run(PrefillState **state, const PrefillView &v, int l0, int l1, int 
     gp.wd_stride = v.wd_stride;
     gp.e_off = tp.e_off;
     gp.e_tok = tp.e_tok;
-    gp.X16 = tp.X16;
     gp.H = B + o_h;
     gp.Ypart = reinterpret_cast<float *>(B + o_y);
     gp.rows_cap = rows_cap;
     gp.err = v.err;
     const int mtiles = (rows_cap + BM - 1) / BM + v.E;   // upper bound over experts
+    // tensor maps of the A operands: rows_cap rows of K 16-bit elements,
+    // boxes of 64 elements (128 bytes) x 128 rows, 128-byte swizzle
+    CUtensorMap tm_gu, tm_dn;
+    {
+        const CUtensorMapDataType dt = W == 1 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+        const TensorMapEncodeFn enc = tensor_map_encoder();
+        if (!enc) {
+            snprintf(msg, msg_len, "prefill: the driver offers no cuTensorMapEncodeTiled");
+            return 2;
+        }
+        auto encode = [&](CUtensorMap *m, void *base, int K) -> CUresult {
+            const cuuint64_t gdim[2] = {cuuint64_t(K), cuuint64_t(rows_cap)};
+            const cuuint64_t gstride[1] = {cuuint64_t(K) * 2};
+            const cuuint32_t box[2] = {BK, BM};
+            const cuuint32_t estr[2] = {1, 1};
+            return enc(m, dt, 2, base, gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        };
+        if (encode(&tm_gu, B + o_xs, v.d) != CUDA_SUCCESS || encode(&tm_dn, B + o_h, v.F) != CUDA_SUCCESS) {
+            snprintf(msg, msg_len, "prefill: cuTensorMapEncodeTiled failed");
+            return 2;
+        }
+    }
 
     for (int l = l0; l < l1; ++l) {
         tp.router = v.E > 1 ? reinterpret_cast<const __half *>(v.router[l]) : nullptr;
@@ -794,9 +871,12 @@ int prefill_run(PrefillState **state, const PrefillView &v, int l0, int l1, int 
         }
         k_norm_route<<<T, 256, 0, stream>>>(tp);
         k_sort<<<1, kSortThreads, 0, stream>>>(tp);
+        k_gather_x<<<rows_cap, 128, 0, stream>>>(tp, B + o_xs);
         dim3 g1(2 * v.F / BN, mtiles, 1);
+        gp.tmA = tm_gu;
         gu<<<g1, kGemmThreads, kGemmSmem, stream>>>(gp);
         dim3 g2(v.d / BN, mtiles, kSplitK);
+        gp.tmA = tm_dn;
         dn<<<g2, kGemmThreads, kGemmSmem, stream>>>(gp);
         k_combine<<<T, 256, 0, stream>>>(tp);
         const cudaError_t e = cudaGetLastError();
