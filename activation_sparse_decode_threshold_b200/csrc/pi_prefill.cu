@@ -582,43 +582,56 @@ struct TokenParams {
     int rows_cap;
 };
 
-__global__ void k_norm_route(TokenParams p)
+constexpr int kNormThreads = 256;
+constexpr int kMaxD = 8192;
+__global__ void __launch_bounds__(kNormThreads) k_norm_route(TokenParams p)
 {
-    const int t = blockIdx.x, tid = threadIdx.x;
+    const int t = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const float *r = p.resid + size_t(t) * p.d;
     __shared__ float red[32];
     __shared__ float lg[kMaxExperts];
+    __shared__ float xs[kMaxD];
+    // sum of squares (vectorised, fixed order: threads, then warps)
     float ss = 0.f;
-    for (int j = tid; j < p.d; j += blockDim.x) ss = fmaf(r[j], r[j], ss);
+    for (int j = 4 * tid; j < p.d; j += 4 * kNormThreads) {
+        const float4 v = *reinterpret_cast<const float4 *>(r + j);
+        *reinterpret_cast<float4 *>(xs + j) = v;
+        ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+    }
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if ((tid & 31) == 0) red[tid >> 5] = ss;
+    if (lane == 0) red[warp] = ss;
     __syncthreads();
     if (tid == 0) {
         float a = 0.f;
-        for (int w = 0; w < int(blockDim.x >> 5); ++w) a += red[w];
+        for (int w = 0; w < kNormThreads / 32; ++w) a += red[w];
         red[31] = 1.f / sqrtf(a / float(p.d) + p.eps);
     }
     __syncthreads();
     const float inv = red[31];
-    for (int j = tid; j < p.d; j += blockDim.x) {
-        if (p.x_bf16) reinterpret_cast<__nv_bfloat16 *>(p.X16)[size_t(t) * p.d + j] = __float2bfloat16_rn(r[j] * inv);
-        else reinterpret_cast<__half *>(p.X16)[size_t(t) * p.d + j] = __float2half_rn(r[j] * inv);
+    for (int j = tid; j < p.d; j += kNormThreads) {
+        const float x = xs[j] * inv;
+        xs[j] = x;
+        if (p.x_bf16) reinterpret_cast<__nv_bfloat16 *>(p.X16)[size_t(t) * p.d + j] = __float2bfloat16_rn(x);
+        else reinterpret_cast<__half *>(p.X16)[size_t(t) * p.d + j] = __float2half_rn(x);
     }
     if (p.E > 1) {
-        // router logits in fp32 from the fp32 input
-        for (int e = 0; e < p.E; ++e) {
+        __syncthreads();
+        // router logits in fp32: warp w takes experts w, w + 8, ...; lanes run
+        // over 8-element pieces of the router row
+        for (int e = warp; e < p.E; e += kNormThreads / 32) {
+            const __half *row = p.router + size_t(e) * p.d;
             float a = 0.f;
-            for (int j = tid; j < p.d; j += blockDim.x)
-                a = fmaf(__half2float(p.router[size_t(e) * p.d + j]), r[j] * inv, a);
-            for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-            __syncthreads();
-            if ((tid & 31) == 0) red[tid >> 5] = a;
-            __syncthreads();
-            if (tid == 0) {
-                float s = 0.f;
-                for (int w = 0; w < int(blockDim.x >> 5); ++w) s += red[w];
-                lg[e] = s;
+            for (int j = 8 * lane; j < p.d; j += 8 * 32) {
+                const uint4 q = *reinterpret_cast<const uint4 *>(row + j);
+                const __half2 *h2 = reinterpret_cast<const __half2 *>(&q);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = __half22float2(h2[i]);
+                    a = fmaf(f.x, xs[j + 2 * i], fmaf(f.y, xs[j + 2 * i + 1], a));
+                }
             }
+            for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+            if (lane == 0) lg[e] = a;
         }
         __syncthreads();
         if (tid == 0) {
@@ -715,15 +728,22 @@ __global__ void k_gather_x(TokenParams p, uint8_t *__restrict__ xs)
 __global__ void k_combine(TokenParams p)
 {
     const int t = blockIdx.x;
-    for (int j = threadIdx.x; j < p.d; j += blockDim.x) {
-        float y = 0.f;
+    for (int j = 4 * threadIdx.x; j < p.d; j += 4 * blockDim.x) {
+        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int k = 0; k < p.top_k; ++k) {
             const int q = p.pos[2 * t + k];
-            float s = 0.f;
-            for (int sp = 0; sp < kSplitK; ++sp) s += p.Ypart[(size_t(sp) * p.rows_cap + q) * p.d + j];
-            y = fmaf(p.route_w[2 * t + k], s, y);
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int sp = 0; sp < kSplitK; ++sp) {
+                const float4 v = *reinterpret_cast<const float4 *>(p.Ypart + (size_t(sp) * p.rows_cap + q) * p.d + j);
+                a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
+            }
+            const float w = p.route_w[2 * t + k];
+            y.x = fmaf(w, a.x, y.x); y.y = fmaf(w, a.y, y.y); y.z = fmaf(w, a.z, y.z); y.w = fmaf(w, a.w, y.w);
         }
-        p.resid[size_t(t) * p.d + j] += y;
+        float4 *rr = reinterpret_cast<float4 *>(p.resid + size_t(t) * p.d + j);
+        float4 r = *rr;
+        r.x += y.x; r.y += y.y; r.z += y.z; r.w += y.w;
+        *rr = r;
     }
 }
 
@@ -869,7 +889,7 @@ int prefill_run(PrefillState **state, const PrefillView &v, int l0, int l1, int 
             const ExpertDev &x = v.ex[size_t(l) * v.E + e];
             gp.ex[e] = PrefillExpert{x.Wgu, x.Wd, x.c};
         }
-        k_norm_route<<<T, 256, 0, stream>>>(tp);
+        k_norm_route<<<T, kNormThreads, 0, stream>>>(tp);
         k_sort<<<1, kSortThreads, 0, stream>>>(tp);
         k_gather_x<<<rows_cap, 128, 0, stream>>>(tp, B + o_xs);
         dim3 g1(2 * v.F / BN, mtiles, 1);
