@@ -19,12 +19,15 @@
 //   k_combine      y = sum over the token's experts in ascending expert index
 //                  of w * (sum of the K-split partials, fixed order); r += y
 //
-// GEMM tiles: 128 x 256 x 64; operands are written into shared memory by the
-// CTA's threads in the canonical no-swizzle core-matrix layout (8 rows x 16
-// bytes per core matrix; INT4 weights are dequantised to fp16 on the way),
-// one elected thread issues tcgen05.mma (kind::f16, fp32 accumulators in
-// TMEM) four K=16 steps per stage, and tcgen05.commit on a per-stage
-// mbarrier frees the stage.  Three stages.  Every wait is bounded.
+// GEMM tiles: up to 256 list positions (two 128-row halves) x 256 weight rows
+// x 64 per stage.  The activation halves arrive by 2-D tensor-map loads; the
+// weight tile is written into shared memory by the CTA's threads in the
+// canonical no-swizzle core-matrix layout (8 rows x 16 bytes per core matrix;
+// INT4 weights are dequantised to fp16 on the way) once and feeds both
+// halves.  One elected thread issues tcgen05.mma (kind::f16, M = 128,
+// N = 256, fp32 accumulators in TMEM, one per half) four K=16 steps per stage
+// and half, and tcgen05.commit on a per-stage mbarrier frees the stage.
+// Three stages.  Every wait is bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -38,7 +41,9 @@
 namespace pi {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, NSTAGE = 4;
+constexpr int BM = 128, BN = 256, BK = 64, NSTAGE = 3;
+constexpr int kHalves = 2;                        // 128-row halves of a CTA's rows (one accumulator each)
+constexpr int kTileRows = kHalves * BM;
 constexpr int kProducerWarps = 16, kProducers = 32 * kProducerWarps;
 constexpr int kRI = BN * 4 / kProducers;          // INT4 items (16 weights) per producer thread per stage
 constexpr int kEpiCols = BN / (kProducerWarps / 4); // accumulator columns per epilogue warp
@@ -46,8 +51,9 @@ constexpr int kGemmThreads = kProducers + 32;    // + the MMA warp
 constexpr int kLag = 1;                          // stages between issuing a stage's copies and publishing it
 constexpr int kATileBytes = BM * BK * 2;          // 16 KB
 constexpr int kBTileBytes = BN * BK * 2;          // 32 KB
-constexpr int kStageBytes = kATileBytes + kBTileBytes;
+constexpr int kStageBytes = kHalves * kATileBytes + kBTileBytes;   // 64 KB
 constexpr int kGemmSmem = NSTAGE * kStageBytes + 1024;
+constexpr int kTmemCols = kHalves * BN;           // 512: the whole tensor memory (one CTA per SM)
 constexpr int kSplitK = 4;                        // K splits of the down GEMM
 constexpr long long kWaitNs = 2000000000LL;
 
@@ -280,17 +286,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int d = p.d, F = p.F;
-    // tile coordinates: blockIdx.x = N tile, blockIdx.y = M tile over all experts,
-    // blockIdx.z = K split (down GEMM)
+    // tile coordinates: blockIdx.x = N tile, blockIdx.y = M tile (up to 256
+    // list positions of one expert) over all experts, blockIdx.z = K split
+    // (down GEMM)
     int e = -1, mrow0 = 0;
     {
         int acc = 0;
         for (int x = 0; x < p.E; ++x) {
             const int cnt = p.e_off[x + 1] - p.e_off[x];
-            const int tiles = (cnt + BM - 1) / BM;
+            const int tiles = (cnt + kTileRows - 1) / kTileRows;
             if (int(blockIdx.y) < acc + tiles) {
                 e = x;
-                mrow0 = p.e_off[x] + (int(blockIdx.y) - acc) * BM;
+                mrow0 = p.e_off[x] + (int(blockIdx.y) - acc) * kTileRows;
                 break;
             }
             acc += tiles;
@@ -298,6 +305,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     }
     if (e < 0) return;   // uniform: no tile for this CTA
     const int mrow_end = p.e_off[e + 1];
+    const int nh = mrow_end - mrow0 > BM ? 2 : 1;   // halves holding rows of this expert
     const PrefillExpert ex = p.ex[e];
     const int K = KIND == kGU ? d : F;
     const int nk_all = K / BK;
@@ -318,7 +326,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     }
     if (warp == kProducerWarps) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     ::"r"(s2u(&tmem_base_sh)), "r"(BN) : "memory");
+                     ::"r"(s2u(&tmem_base_sh)), "r"(kTmemCols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -335,13 +343,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         // conflicts beyond the minimum).  The A tile comes by tensor-map load.
         auto issue_async = [&](int kt, int s) {
             uint8_t *A = smem + s * kStageBytes;
-            uint8_t *B = A + kATileBytes;
+            uint8_t *B = A + kHalves * kATileBytes;
             const int k0 = kt * BK;
             if (pt == 0) {
-                // A: 128 list positions x 64 elements; rows past the expert's are
-                // loaded too and their results discarded, rows past the buffer read 0
-                mbar_arrive_tx(&afull[s], uint32_t(kATileBytes));
+                // A: one or two halves of 128 list positions x 64 elements; rows
+                // past the expert's are loaded too and their results discarded,
+                // rows past the buffer read 0
+                mbar_arrive_tx(&afull[s], uint32_t(nh * kATileBytes));
                 tma_load_2d(A, &p.tmA, k0, mrow0, &afull[s]);
+                if (nh > 1) tma_load_2d(A + kATileBytes, &p.tmA, k0, mrow0 + BM, &afull[s]);
             }
             if constexpr (!I4) {
                 if constexpr (KIND == kGU) {
@@ -414,7 +424,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
             }
         };
         auto store_raw = [&](const RawI4 &r, int s) {
-            uint8_t *B = smem + s * kStageBytes + kATileBytes;
+            uint8_t *B = smem + s * kStageBytes + kHalves * kATileBytes;
 #pragma unroll
             for (int i = 0; i < kRI; ++i) {
                 const int c = pt + kProducers * i;
@@ -488,20 +498,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         // epilogue: wait for the accumulator
         if (nk > 0 && !abort_sh && !mbar_wait(&done, 0u, p.err)) abort_sh = 1;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const int row = 32 * (warp & 3) + lane;
-        const int lr = mrow0 + row;
-        const bool valid = lr < mrow_end && !abort_sh;
         const int col0 = kEpiCols * (warp >> 2);
-        if (KIND == kDOWN && nk == 0) {
-            // an empty K range still owns its partial: zeros
-            if (valid) {
-                float *dst = p.Ypart + (size_t(blockIdx.z) * p.rows_cap + lr) * d + n0 + col0;
-                for (int j2 = 0; j2 < kEpiCols; j2 += 4) *reinterpret_cast<float4 *>(dst + j2) = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int h = 0; h < nh; ++h) {
+            const int lr = mrow0 + h * BM + 32 * (warp & 3) + lane;
+            const bool valid = lr < mrow_end && !abort_sh;
+            if (KIND == kDOWN && nk == 0) {
+                // an empty K range still owns its partial: zeros
+                if (valid) {
+                    float *dst = p.Ypart + (size_t(blockIdx.z) * p.rows_cap + lr) * d + n0 + col0;
+                    for (int j2 = 0; j2 < kEpiCols; j2 += 4) *reinterpret_cast<float4 *>(dst + j2) = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+                continue;
             }
-        } else if (!abort_sh) {
+            if (abort_sh) break;
             for (int cc = 0; cc < kEpiCols; cc += 16) {
                 float v[16];
-                tmem_ld16(tmem + (uint32_t(32 * (warp & 3)) << 16) + uint32_t(col0 + cc), v);
+                tmem_ld16(tmem + (uint32_t(32 * (warp & 3)) << 16) + uint32_t(h * BN + col0 + cc), v);
                 if (!valid) continue;
                 if constexpr (KIND == kGU) {
                     // columns 2j, 2j+1 = gate, up of neuron n0/2 + (col0 + cc)/2 + j
@@ -513,8 +525,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
                         const float g = v[2 * j2] - (nn < F ? __ldg(ex.c + nn) : 0.f);
                         const float u = v[2 * j2 + 1];
                         const float gp = g > 0.f ? g : 0.f;
-                        const float h = p.act == 0 ? gp : (p.act == 1 ? gp * u : gp * (u > 0.f ? u : 0.f));
-                        hv[j2] = from_f<AT>(h);
+                        const float hh = p.act == 0 ? gp : (p.act == 1 ? gp * u : gp * (u > 0.f ? u : 0.f));
+                        hv[j2] = from_f<AT>(hh);
                     }
                     if (nb + 8 <= F)
                         *reinterpret_cast<uint4 *>(Hbuf + size_t(lr) * F + nb) = *reinterpret_cast<uint4 *>(hv);
@@ -537,12 +549,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
                     !mbar_wait(&afull[s], uint32_t((j / NSTAGE) & 1), p.err)) { abort_sh = 1; break; }
                 if (abort_sh) break;
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                const uint32_t a0 = s2u(smem + s * kStageBytes), b0 = a0 + kATileBytes;
+                const uint32_t a0 = s2u(smem + s * kStageBytes), b0 = a0 + kHalves * kATileBytes;
 #pragma unroll
                 for (int ks = 0; ks < BK / 16; ++ks) {
-                    const uint64_t ad = make_sdesc_sw128(a0 + ks * 32);
+                    // the weight tile's K step feeds each half's accumulator
                     const uint64_t bd = make_sdesc(b0 + ks * 256, 128, BK / 8 * 128);
-                    umma(tmem, ad, bd, idesc, j > 0 || ks > 0);
+                    umma(tmem, make_sdesc_sw128(a0 + ks * 32), bd, idesc, j > 0 || ks > 0);
+                    if (nh > 1)
+                        umma(tmem + uint32_t(BN), make_sdesc_sw128(a0 + kATileBytes + ks * 32), bd, idesc, j > 0 || ks > 0);
                 }
                 umma_commit(&empty[s]);
                 issued = j + 1;
@@ -560,7 +574,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     if (warp == kProducerWarps)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BN) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -857,7 +871,7 @@ int prefill_run(PrefillState **state, const PrefillView &v, int l0, int l1, int 
     gp.Ypart = reinterpret_cast<float *>(B + o_y);
     gp.rows_cap = rows_cap;
     gp.err = v.err;
-    const int mtiles = (rows_cap + BM - 1) / BM + v.E;   // upper bound over experts
+    const int mtiles = (rows_cap + kTileRows - 1) / kTileRows + v.E;   // upper bound over experts
     // tensor maps of the A operands: rows_cap rows of K 16-bit elements,
     // boxes of 64 elements (128 bytes) x 128 rows, 128-byte swizzle
     CUtensorMap tm_gu, tm_dn;
