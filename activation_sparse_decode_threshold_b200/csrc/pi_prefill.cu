@@ -20,14 +20,15 @@
 //                  of w * (sum of the K-split partials, fixed order); r += y
 //
 // GEMM tiles: up to 256 list positions (two 128-row halves) x 256 weight rows
-// x 64 per stage.  The activation halves arrive by 2-D tensor-map loads; the
-// weight tile is written into shared memory by the CTA's threads in the
-// canonical no-swizzle core-matrix layout (8 rows x 16 bytes per core matrix;
-// INT4 weights are dequantised to fp16 on the way) once and feeds both
-// halves.  One elected thread issues tcgen05.mma (kind::f16, M = 128,
-// N = 256, fp32 accumulators in TMEM, one per half) four K=16 steps per stage
-// and half, and tcgen05.commit on a per-stage mbarrier frees the stage.
-// Three stages.  Every wait is bounded.
+// x 64 per stage.  The activation halves arrive by 2-D tensor-map loads in
+// the 128-byte swizzle; the weight tile is written into shared memory by the
+// CTA's threads (INT4 weights dequantised to fp16 on the way), in the same
+// swizzle for the K-major gate/up weights and in the canonical no-swizzle
+// core-matrix layout (8 k-rows x 16 bytes) for the MN-major W_down, once per
+// stage for both halves.  One elected thread issues tcgen05.mma (kind::f16,
+// M = 128, N = 256, fp32 accumulators in TMEM, one per half) four K=16 steps
+// per stage and half, and tcgen05.commit on a per-stage mbarrier frees the
+// stage.  Three stages.  Every wait is bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -167,8 +168,8 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uin
     d |= uint64_t(1) << 46;
     return d;
 }
-// instruction descriptor: f16 A and B, f32 accumulate, M = 128, N = 256
-__device__ __forceinline__ uint32_t make_idesc(bool b_mn_major, bool bf16)
+// instruction descriptor: f16 A and B, f32 accumulate, M = m (128 or 64), N = 256
+__device__ __forceinline__ uint32_t make_idesc(bool b_mn_major, bool bf16, int m = BM)
 {
     uint32_t i = 0;
     i |= 1u << 4;                        // D format: f32
@@ -177,7 +178,7 @@ __device__ __forceinline__ uint32_t make_idesc(bool b_mn_major, bool bf16)
     i |= 0u << 15;                       // A K-major
     i |= (b_mn_major ? 1u : 0u) << 16;   // B K-major / MN-major
     i |= uint32_t(BN >> 3) << 17;
-    i |= uint32_t(BM >> 4) << 24;
+    i |= uint32_t(m >> 4) << 24;
     return i;
 }
 __device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, bool acc)
@@ -207,10 +208,14 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v)
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// byte offset of element (row, k) of a K-major tile with BK columns
-__device__ __forceinline__ uint32_t kmaj_off(int row, int kchunk)
+// byte offset of 16-byte chunk `kc` (0..7) of row `row` of a K-major tile
+// with 128-byte rows in the 128-byte swizzle (the chunk index XOR the row
+// mod 8, 8-row groups 1024 bytes apart), the layout a SWIZZLE_128B
+// tensor-map load writes; 8 consecutive rows of one chunk fall in 8
+// different bank groups
+__device__ __forceinline__ uint32_t sw128_off(int row, int kc)
 {
-    return uint32_t((row >> 3) * (BK / 8 * 128) + kchunk * 128 + (row & 7) * 16);
+    return uint32_t((row >> 3) * 1024 + (row & 7) * 128 + ((kc ^ (row & 7)) << 4));
 }
 // byte offset of the 16-byte chunk holding n = 8*ng .. 8*ng+7 of k-row `k`
 // in an MN-major tile (core matrices: 8 k-rows x 8 n-values)
@@ -306,6 +311,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     if (e < 0) return;   // uniform: no tile for this CTA
     const int mrow_end = p.e_off[e + 1];
     const int nh = mrow_end - mrow0 > BM ? 2 : 1;   // halves holding rows of this expert
+    // a second half of at most 64 rows takes an M = 64 MMA: its accumulator
+    // row 16 q + i sits in TMEM lane 32 q + i (i < 16) of the half's columns
+    const bool h1_m64 = nh == 2 && mrow_end - mrow0 <= BM + 64;
     const PrefillExpert ex = p.ex[e];
     const int K = KIND == kGU ? d : F;
     const int nk_all = K / BK;
@@ -362,7 +370,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
                         const int nn = n0 / 2 + (row >> 1);
                         const bool ok = nn < F && (p.gated || (row & 1) == 0);
                         const uint8_t *rec = ex.Wgu + size_t(ok ? nn : 0) * p.rec_bytes + ((row & 1) ? p.wrow : 0);
-                        cp_async16(B + kmaj_off(row, kc), rec + (k0 + kc * 8) * 2, ok);
+                        cp_async16(B + sw128_off(row, kc), rec + (k0 + kc * 8) * 2, ok);
                     }
                 } else {
 #pragma unroll
@@ -432,8 +440,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
                 dequant16(r.q[i], __ushort_as_half(r.sc[i]), lo, hi);
                 if constexpr (KIND == kGU) {
                     const int row = (c >> 5) * 8 + (c & 7), q16 = (c >> 3) & 3;
-                    *reinterpret_cast<uint4 *>(B + kmaj_off(row, 2 * q16)) = lo;
-                    *reinterpret_cast<uint4 *>(B + kmaj_off(row, 2 * q16 + 1)) = hi;
+                    *reinterpret_cast<uint4 *>(B + sw128_off(row, 2 * q16)) = lo;
+                    *reinterpret_cast<uint4 *>(B + sw128_off(row, 2 * q16 + 1)) = hi;
                 } else {
                     const int rest = c >> 5;
                     const int k = (rest & 7) * 8 + (c & 7), g16 = (rest >> 3) * 4 + ((c >> 3) & 3);
@@ -500,8 +508,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const int col0 = kEpiCols * (warp >> 2);
         for (int h = 0; h < nh; ++h) {
-            const int lr = mrow0 + h * BM + 32 * (warp & 3) + lane;
-            const bool valid = lr < mrow_end && !abort_sh;
+            const bool m64 = h == 1 && h1_m64;
+            const int lr = mrow0 + h * BM + (m64 ? 16 : 32) * (warp & 3) + lane;
+            const bool valid = (!m64 || lane < 16) && lr < mrow_end && !abort_sh;
             if (KIND == kDOWN && nk == 0) {
                 // an empty K range still owns its partial: zeros
                 if (valid) {
@@ -542,6 +551,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         // ------------------------------ MMA issue ------------------------------
         if (lane == 0) {
             const uint32_t idesc = make_idesc(KIND == kDOWN, W == 1);
+            const uint32_t idesc1 = h1_m64 ? make_idesc(KIND == kDOWN, W == 1, 64) : idesc;
             int issued = 0;
             for (int j = 0; j < nk; ++j) {
                 const int s = j % NSTAGE;
@@ -553,10 +563,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
 #pragma unroll
                 for (int ks = 0; ks < BK / 16; ++ks) {
                     // the weight tile's K step feeds each half's accumulator
-                    const uint64_t bd = make_sdesc(b0 + ks * 256, 128, BK / 8 * 128);
+                    const uint64_t bd = KIND == kGU ? make_sdesc_sw128(b0 + ks * 32)
+                                                    : make_sdesc(b0 + ks * 256, 128, BK / 8 * 128);
                     umma(tmem, make_sdesc_sw128(a0 + ks * 32), bd, idesc, j > 0 || ks > 0);
                     if (nh > 1)
-                        umma(tmem + uint32_t(BN), make_sdesc_sw128(a0 + kATileBytes + ks * 32), bd, idesc, j > 0 || ks > 0);
+                        umma(tmem + uint32_t(BN), make_sdesc_sw128(a0 + kATileBytes + ks * 32), bd, idesc1, j > 0 || ks > 0);
                 }
                 umma_commit(&empty[s]);
                 issued = j + 1;
