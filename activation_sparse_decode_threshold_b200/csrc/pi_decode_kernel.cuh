@@ -83,6 +83,14 @@ __device__ __forceinline__ void mbar_arrive_tx(uint64_t *b, uint32_t bytes)
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(s2u(b)), "r"(bytes)
                  : "memory");
 }
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes)
+{
+    asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(s2u(b)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *b)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(s2u(b)) : "memory");
+}
 __device__ __forceinline__ bool mbar_test(uint64_t *b, uint32_t parity)
 {
     uint32_t ok;
@@ -272,6 +280,7 @@ constexpr int kRA = 16;           // V rows per staging round at most
 constexpr int kZRows = 112;       // U rows per staging round at most (a multiple of 16)
 constexpr int kMaxU = 4;          // U vectors per lane (rank <= 128 * EPV)
 constexpr int kRound = 16;        // neurons per gather round at most
+constexpr int kVsmMax = 64 * 1024;  // largest V block staged in shared memory for the column phase
 static_assert(kRound <= 32, "a round's neurons are tracked in one warp ballot");
 constexpr int kRed = 2 * kRound;  // values reduced per warp at most
 
@@ -310,6 +319,7 @@ struct Smem {
     float inv_rms;
     int bc[2];
     uint64_t stage_bar;                    // completion of a staging round
+    uint64_t vbar;                         // completion of the V block staged for the column phase
     uint64_t gbar[kRound / 4];             // completion of each group of four neurons of a gather round
     int gfail;                             // a warp's bounded wait on a group ran out
 };
@@ -380,18 +390,19 @@ __device__ bool grid_sync(Smem *sm, const DecodeParams &p, unsigned &epoch, int 
     return ok;
 }
 
-// Staging round: thread 0 has issued bulk copies onto sm->stage_bar; it waits
-// (bounded) and the whole CTA adopts its verdict.
+// Staging round: thread 0 has issued bulk copies onto sm->stage_bar (or
+// `bar`); it waits (bounded) and the whole CTA adopts its verdict.
 __device__ bool stage_wait(Smem *sm, const DecodeParams &p, uint32_t &par, int &bci,
-                           long long *cyc = nullptr)
+                           long long *cyc = nullptr, uint64_t *bar = nullptr)
 {
+    if (!bar) bar = &sm->stage_bar;
     if (threadIdx.x == 0) {
         const long long c0 = clock64();
-        bool ok = mbar_test(&sm->stage_bar, par);
+        bool ok = mbar_test(bar, par);
         if (!ok) {
             const long long t0 = gtimer();
             for (unsigned it = 1; !ok; ++it) {
-                ok = mbar_test(&sm->stage_bar, par);
+                ok = mbar_test(bar, par);
                 if (!ok && (it & 15) == 0 && gtimer() - t0 > p.wait_ns) {
                     set_error(p.err, kDevTimeout);
                     break;
@@ -405,7 +416,7 @@ __device__ bool stage_wait(Smem *sm, const DecodeParams &p, uint32_t &par, int &
     const bool ok = ld_vol(&sm->bc[bci]) != 0;
     bci ^= 1;
     if (ok) {
-        mbar_test(&sm->stage_bar, par);   // acquire for this thread (phase complete)
+        mbar_test(bar, par);   // acquire for this thread (phase complete)
         par ^= 1;                         // a failed round keeps its phase for the drain
     }
     return ok;
@@ -466,6 +477,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         return sm.exl[l & 1][0].V + size_t(r) * c0 * (p.vrow / d);
     };
     const int vbrow = ncol * (p.vrow / d);   // bytes of one V-block row
+    // dense decode: after the gather the next layer's V block is bulk-copied
+    // into the top of the staging buffer, beside the first `ufirst` rows of
+    // the next U strip's first round; the rest of that round follows once the
+    // column phase has read the V block
+    const int vbytes = r * vbrow;
+    const int voff = (kStageBytes - vbytes) & ~127;
+    const bool vsm = !moe && !predict && ncol > 0 && vbytes <= kVsmMax;
+    const int u_round0 = min(ns, ucap);
+    const int ufirst = vsm ? min(u_round0, voff / p.urow) : u_round0;
 
     unsigned epoch = 0;
     uint32_t spar = 0;
@@ -473,18 +493,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     int bci = 0, rb = 0;
     bool staged_early = false;   // round 0 of the next U strip is already in flight
     bool pending = false;        // a staging round was issued and not yet waited for
+    uint32_t vpar = 0;
+    bool vpend = false;          // a V block was issued and not yet waited for
+    bool upart2 = false;         // the staged U round still misses its second piece
 
-    // stage rows [row0, row0 + n) of an expert's U strip, contiguous (lane 0
-    // of warp 0 issues the copies)
-    auto stage_u = [&](const ExpertDev &ex, int row0, int n) {
+    // stage rows [row0, row0 + n) of an expert's U strip, contiguous, at
+    // staged row `at` (lane 0 of warp 0 issues the copies); a round staged in
+    // two pieces announces the first piece's bytes without arriving, and its
+    // second piece arrives (`last`)
+    auto stage_u_at = [&](const ExpertDev &ex, int row0, int n, int at, bool last) {
         if (lane == 0) {
-            mbar_arrive_tx(&sm.stage_bar, uint32_t(n) * p.urow);
-            stage_copy(stg, ex.U + size_t(s0 + row0) * p.urow, uint32_t(n) * p.urow, &sm.stage_bar);
+            if (last) mbar_arrive_tx(&sm.stage_bar, uint32_t(n) * p.urow);
+            else mbar_expect_tx(&sm.stage_bar, uint32_t(n) * p.urow);
+            if (n > 0)
+                stage_copy(stg + size_t(at) * p.urow, ex.U + size_t(s0 + row0) * p.urow, uint32_t(n) * p.urow,
+                           &sm.stage_bar);
         }
     };
+    auto stage_u = [&](const ExpertDev &ex, int row0, int n) { stage_u_at(ex, row0, n, 0, true); };
 
     if (tid == 0) {
         mbar_init(&sm.stage_bar, 1);
+        mbar_init(&sm.vbar, 1);
         for (int g = 0; g < kRound / 4; ++g) mbar_init(&sm.gbar[g], 1);
         sm.gfail = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -513,19 +543,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // all added in fixed point.  `from_partials`: r = r_old + sum of the
     // per-CTA partials of y in fixed CTA order; otherwise r is the input.
     // -----------------------------------------------------------------------
-    auto column_phase = [&](int li_in, bool from_partials, bool next_exists, int l_next, int prow) {
+    // vs: the V block of l_next is being staged in shared memory (vbar)
+    auto column_phase = [&](int li_in, bool from_partials, bool next_exists, int l_next, int prow,
+                            bool vs) -> bool {
         const float *src = predict ? p.x_in : p.resid;
         long long *fx = p.fix + size_t(li_in & 1) * kFixStride;
         // dense: this thread's V-block rows (k = tid and tid + 512; r <= 1024)
-        // for the next layer's t partial start loading now, so their round
-        // trip overlaps the partial reduction's; the first kVP vectors of each
+        // for the next layer's t partial; from global memory they start
+        // loading now, so their round trip overlaps the partial reduction's
+        // (the first kVP vectors of each)
         constexpr int kVP = 4;
         const bool tpart = !moe && next_exists && ncol > 0;
         const int nv = vbrow / VBP;
         const int kr0 = tid, kr1 = tid + kThreads;
         const uint8_t *vrow0 = nullptr, *vrow1 = nullptr;
         VP va[kVP], vb2[kVP];
-        if (tpart) {
+        if (tpart && !vs) {
             const uint8_t *vb = vblk(l_next);
             vrow0 = vb + size_t(kr0 < r ? kr0 : 0) * vbrow;
             vrow1 = vb + size_t(kr1 < r ? kr1 : 0) * vbrow;
@@ -573,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         if (prow >= 0) prof_put(p, prow, 7, gtimer());
         if (!predict && p.trace && li_in < l1 - l0)
             for (int j = tid; j < ncol; j += kThreads) __stcg(p.trace + size_t(li_in) * d + c0 + j, sm.rsl[j]);
-        if (!next_exists) return;
+        if (!next_exists) return true;
         // sum of squares of this CTA's columns (fixed order: lanes, then tree)
         if (warp == 0 && !predict) {
             float ss = 0.f;
@@ -583,21 +616,46 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
         if (!moe) {
             // t partial: rows kr0, kr1 of the V block dotted with this CTA's columns
-            if (tpart && kr0 < r) {
-                float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-                auto acc_vec = [&](const VP &q0, const VP &q1, int v) {
-                    float w0[EPVP], w1[EPVP];
-                    cvt<PF>(q0, w0);
-                    cvt<PF>(q1, w1);
+            float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+            auto acc_vec = [&](const VP &q0, const VP &q1, int v) {
+                float w0[EPVP], w1[EPVP];
+                cvt<PF>(q0, w0);
+                cvt<PF>(q1, w1);
 #pragma unroll
-                    for (int i = 0; i < EPVP; i += 2) {
-                        const float x0 = sm.rsl[v * EPVP + i], x1 = sm.rsl[v * EPVP + i + 1];
-                        a0 = fmaf(w0[i], x0, a0);
-                        a1 = fmaf(w0[i + 1], x1, a1);
-                        b0 = fmaf(w1[i], x0, b0);
-                        b1 = fmaf(w1[i + 1], x1, b1);
+                for (int i = 0; i < EPVP; i += 2) {
+                    const float x0 = sm.rsl[v * EPVP + i], x1 = sm.rsl[v * EPVP + i + 1];
+                    a0 = fmaf(w0[i], x0, a0);
+                    a1 = fmaf(w0[i + 1], x1, a1);
+                    b0 = fmaf(w1[i], x0, b0);
+                    b1 = fmaf(w1[i + 1], x1, b1);
+                }
+            };
+            if (tpart && vs) {
+                if (!stage_wait(&sm, p, vpar, bci, nullptr, &sm.vbar)) return false;
+                vpend = false;
+                if (kr0 < r) {
+                    // each thread walks its rows' vectors from `rot` on, so the
+                    // eight rows of a quarter-warp fall in eight different
+                    // 16-byte bank groups (rows are nv vectors apart)
+                    const int lowbit = nv & -nv;
+                    const int rot = (lane & 7) / (8 / (lowbit < 8 ? lowbit : 8));
+                    const uint8_t *vs0 = stg + voff + size_t(kr0) * vbrow;
+                    const uint8_t *vs1 = stg + voff + size_t(kr1 < r ? kr1 : kr0) * vbrow;
+                    for (int j = 0; j < nv; ++j) {
+                        int jj = j + rot;
+                        if (jj >= nv) jj -= nv;
+                        acc_vec(*reinterpret_cast<const VP *>(vs0 + jj * VBP),
+                                *reinterpret_cast<const VP *>(vs1 + jj * VBP), jj);
                     }
-                };
+                    fix_add(fx + kr0, a0 + a1, kFixT);
+                    if (kr1 < r) fix_add(fx + kr1, b0 + b1, kFixT);
+                }
+                // the V block is read: the rest of the next U round lands there
+                cta_sync();
+                if (upart2 && warp == 0)
+                    stage_u_at(sm.exl[l_next & 1][0], ufirst, u_round0 - ufirst, ufirst, true);
+                upart2 = false;
+            } else if (tpart && kr0 < r) {
 #pragma unroll
                 for (int j = 0; j < kVP; ++j)
                     if (j < nv) acc_vec(va[j], kr1 < r ? vb2[j] : va[j], j);
@@ -618,6 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 fix_add(fx + kMaxRankTotal + 1 + tid, a, kFixT);
             }
         }
+        return true;
     };
 
     float xw[MAXVW * EPVW];
@@ -625,7 +684,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 #define XP(i) (kSameX ? xw[(i)] : xp_own[(i)])
 
     // prologue: the first layer's input columns
-    column_phase(0, false, true, l0, -1);
+    column_phase(0, false, true, l0, -1, false);
     long long cyc0 = 0;
     const bool started = grid_sync(&sm, p, epoch, bci, &cyc0);
 
@@ -1264,13 +1323,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         if (tid == 0 && p.stats) atomicAdd(p.stats + li * 4 + 1, nz_total);
         // the next layer's predictor slice starts moving: U strip straight
         // into shared memory (free until then), the rest of it into L2
-        if (!moe && l + 1 < l1 && ns > 0 && warp == 0) {
-            stage_u(sm.exl[(l + 1) & 1][0], 0, min(ns, ucap));
-            if (lane == 0 && ns > ucap)
-                prefetch_l2(sm.exl[(l + 1) & 1][0].U + size_t(s0 + ucap) * p.urow, uint32_t(ns - ucap) * p.urow);
+        // (dense decode: with the V block for the column phase in the top of
+        // the buffer and the U round's first piece below it)
+        const bool vnext = vsm && l + 1 < l1;
+        if (!moe && l + 1 < l1 && warp == 0) {
+            const ExpertDev &nx = sm.exl[(l + 1) & 1][0];
+            if (vnext && lane == 0) {
+                mbar_arrive_tx(&sm.vbar, uint32_t(vbytes));
+                stage_copy(stg + voff, vblk(l + 1), uint32_t(vbytes), &sm.vbar);
+            }
+            if (ns > 0) {
+                const int n1 = vnext ? ufirst : u_round0;
+                stage_u_at(nx, 0, n1, 0, n1 == u_round0);
+                if (lane == 0 && ns > ucap)
+                    prefetch_l2(nx.U + size_t(s0 + ucap) * p.urow, uint32_t(ns - ucap) * p.urow);
+            }
         }
         staged_early = !moe && l + 1 < l1 && ns > 0;
         if (staged_early) pending = true;
+        vpend = vnext;
+        upart2 = staged_early && vnext && ufirst < u_round0;
         // the fixed-point buffer of layer l - 1 (read before two barriers ago)
         // is cleared for layer l + 1
         if (b == S - 1) {
@@ -1296,7 +1368,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 
         // ---------------- reduction + next layer's column products -----------
         const bool next = l + 1 < l1;
-        column_phase(li + 1, true, next, l + 1, li);
+        if (!column_phase(li + 1, true, next, l + 1, li, vsm && next)) break;
         prof_put(p, li, 5, gtimer());
         if (next && !grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
         prof_put(p, li, 6, gtimer());
@@ -1309,8 +1381,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // (bounded) so no bulk copy writes this CTA's shared memory after exit
     if (tid == 0) {
         const long long t0 = gtimer();
+        // a U round staged in two pieces whose second piece was never issued:
+        // arrive for it, so the phase completes when the first piece lands
+        if (upart2) mbar_arrive(&sm.stage_bar);
         if (pending)
             while (!mbar_test(&sm.stage_bar, spar) && gtimer() - t0 < p.wait_ns) {
+            }
+        if (vpend)
+            while (!mbar_test(&sm.vbar, vpar) && gtimer() - t0 < p.wait_ns) {
             }
         for (int g = 0; g < kRound / 4; ++g)
             if ((gpend >> g) & 1u)
