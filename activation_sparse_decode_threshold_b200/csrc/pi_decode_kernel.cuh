@@ -280,7 +280,7 @@ constexpr int kRA = 16;           // V rows per staging round at most
 constexpr int kZRows = 112;       // U rows per staging round at most (a multiple of 16)
 constexpr int kMaxU = 4;          // U vectors per lane (rank <= 128 * EPV)
 constexpr int kRound = 16;        // neurons per gather round at most
-constexpr int kVsmMax = 64 * 1024;  // largest V block staged in shared memory for the column phase
+constexpr int kVsmMax = 128 * 1024;  // largest V block staged in shared memory for the column phase
 static_assert(kRound <= 32, "a round's neurons are tracked in one warp ballot");
 constexpr int kRed = 2 * kRound;  // values reduced per warp at most
 
