@@ -6,10 +6,16 @@
 // columns.  Per layer l (dense FFN):
 //
 //   [B] t = V x (from the column phase below), x = RMSNorm(r);
-//       z = U t - c over the strip, active iff z > threshold, the active list
-//       compacted in ascending table order with warp ballots (PowerInfer
-//       (unite.ai), "Adaptive sparse predictor").
-//   [C] for active neurons only: the neuron's W_gate / W_up rows -> h =
+//       z = U t - c over the strip (tensor-core dots of the staged U rows),
+//       active iff z > threshold, the active list compacted in ascending
+//       table order with warp ballots (PowerInfer (unite.ai), "Adaptive
+//       sparse predictor").
+//   [balance] every strip publishes its active list; after a grid barrier
+//       each CTA takes an equal share of the lists concatenated in strip
+//       order (depends only on the active set: deterministic).
+//   [C] for the active neurons of its share: the neuron's record (W_gate /
+//       W_up rows, plus its W_down row for ReLU / ReGLU, where h != 0 almost
+//       always follows z > 0) by bulk copy into shared memory -> h =
 //       act(g, u); for h != 0 its W_down column (stored as a row) accumulates
 //       into a per-CTA fp32 partial of y ("Neuron-aware operators": rows of
 //       the input matrices, columns of the output matrix).
@@ -21,19 +27,19 @@
 //       64-bit fixed point so the totals do not depend on arrival order.
 //   --- grid barrier ---
 //
-// Two grid barriers per layer.  The MoE layer adds routing (from fixed-point
-// router logits, identical in every CTA), t computed by rows of the two
-// chosen experts, and a third barrier.
+// Three grid barriers per dense layer.  The MoE layer adds routing (from
+// fixed-point router logits, identical in every CTA), t computed by rows of
+// the two chosen experts, and a fourth barrier.
 //
 // Memory: weight bytes are pulled towards the SM as soon as their addresses
-// are known -- the next layer's U strip is bulk-copied straight into shared
-// memory when the gather ends (it lands during the barriers), its V block is
-// prefetched into L2, and a strip's active neuron records (plus, for ReLU /
-// ReGLU, where h != 0 almost always follows z > 0, their W_down rows) are
-// prefetched into L2 the moment the active list exists; the 16 warps read
-// them with batched 128-bit loads, the W_down rows of one batch together with
-// the W_gate/W_up records of the next.  All waits are bounded (%globaltimer);
-// a wait that runs out records an error word and every CTA returns.
+// are known.  A strip's active records are prefetched into L2 the moment its
+// list is published; the next layer's V block and biases are prefetched into
+// L2 when the gather starts; when it ends, the next layer's V block (dense)
+// and the first U round are bulk-copied into shared memory, where they land
+// during the barriers (the V block in the top of the staging buffer, the U
+// rows below it, and the U rows that do not fit yet once the column phase has
+// read the V block).  All waits are bounded (%globaltimer); a wait that runs
+// out records an error word and every CTA returns.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -346,7 +352,8 @@ __device__ __forceinline__ void fix_add(long long *dst, float v, float scale)
 constexpr float kFixT = 4294967296.0f;    // 2^32
 constexpr float kFixSS = 16777216.0f;     // 2^24
 
-// Grid-wide barrier of all CTAs of the cooperative launch.  Arrivals are
+// Grid-wide barrier of all CTAs of the cooperative launch, in two halves so
+// that a CTA can issue work between its arrival and its wait.  Arrivals are
 // spread over kBarLanes counters, one 128-byte line each (CTA b arrives on
 // counter b mod kBarLanes), so that they do not serialise on one L2 line;
 // the counters are never reset within a launch.  Thread 0 arrives with a
@@ -354,14 +361,19 @@ constexpr float kFixSS = 16777216.0f;     // 2^24
 // warp 0 then polls all counters at once, lane i reading counter i with an
 // acquire, bounded by wait_ns, and the verdict is broadcast through shared
 // memory so the whole CTA agrees.
-__device__ bool grid_sync(Smem *sm, const DecodeParams &p, unsigned &epoch, int &bci, long long *cyc)
+__device__ __forceinline__ void grid_arrive(const DecodeParams &p, unsigned &epoch)
 {
     cta_sync();
     if (threadIdx.x < 32) {
+        epoch += 1;
+        if (threadIdx.x == 0) red_release_gpu(p.bar + (blockIdx.x % kBarLanes) * kBarStride, 1u);
+    }
+}
+__device__ bool grid_wait(Smem *sm, const DecodeParams &p, unsigned epoch, int &bci, long long *cyc)
+{
+    if (threadIdx.x < 32) {
         const int lane = threadIdx.x;
         const long long c0 = clock64();
-        epoch += 1;
-        if (lane == 0) red_release_gpu(p.bar + (blockIdx.x % kBarLanes) * kBarStride, 1u);
         // CTAs per counter: S / kBarLanes, one more for the first S % kBarLanes
         const unsigned S = gridDim.x;
         unsigned target = lane < kBarLanes ? epoch * (S / kBarLanes + (unsigned(lane) < S % kBarLanes ? 1u : 0u)) : 0u;
@@ -388,6 +400,11 @@ __device__ bool grid_sync(Smem *sm, const DecodeParams &p, unsigned &epoch, int 
     const bool ok = ld_vol(&sm->bc[bci]) != 0;
     bci ^= 1;
     return ok;
+}
+__device__ __forceinline__ bool grid_sync(Smem *sm, const DecodeParams &p, unsigned &epoch, int &bci, long long *cyc)
+{
+    grid_arrive(p, epoch);
+    return grid_wait(sm, p, epoch, bci, cyc);
 }
 
 // Staging round: thread 0 has issued bulk copies onto sm->stage_bar (or
@@ -650,11 +667,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     fix_add(fx + kr0, a0 + a1, kFixT);
                     if (kr1 < r) fix_add(fx + kr1, b0 + b1, kFixT);
                 }
-                // the V block is read: the rest of the next U round lands there
-                cta_sync();
-                if (upart2 && warp == 0)
-                    stage_u_at(sm.exl[l_next & 1][0], ufirst, u_round0 - ufirst, ufirst, true);
-                upart2 = false;
             } else if (tpart && kr0 < r) {
 #pragma unroll
                 for (int j = 0; j < kVP; ++j)
@@ -852,9 +864,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             }
             if (!ok) break;
             // round 0 of the first expert's U strip lands during the barrier
+            // (issued after the arrival, whose release would wait for it)
+            grid_arrive(p, epoch);
             if (warp == 0 && ns > 0) stage_u(sm.exl[l & 1][0], 0, min(ns, ucap));
             staged_early = pending = ns > 0;
-            if (!grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
+            if (!grid_wait(&sm, p, epoch, bci, &cyc_bar)) break;
             for (int k = tid; k < ntop * r; k += kThreads) put_t(k, __ldcg(p.t_buf + k), ntop * r);
         }
         if constexpr (moe) {
@@ -1062,11 +1076,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
 
         // ---------------- balance: equal shares of the active list -----------
-        // Each strip publishes its active neurons (with their biases) and
-        // starts their rows moving towards L2; after a grid barrier every CTA
-        // takes an equal share [lo, hi) of the lists concatenated in strip
-        // order.  The share depends only on the active set, so the per-CTA
-        // partials and their fixed-order reduction stay deterministic.
+        // Each strip publishes its active neurons (with their biases), arrives
+        // at a grid barrier and starts their rows moving towards L2; after the
+        // barrier every CTA takes an equal share [lo, hi) of the lists
+        // concatenated in strip order.  The share depends only on the active
+        // set, so the per-CTA partials and their fixed-order reduction stay
+        // deterministic.
         const ExpertDev *exs[kMaxTopK] = {&sm.exl[l & 1][0], &sm.exl[l & 1][ntop > 1 ? 1 : 0]};
         {
             const int n0 = sm.lst_n[0], nl = n0 + (ntop > 1 ? sm.lst_n[1] : 0);
@@ -1076,11 +1091,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 const int e = en >> 12, loc = en & 0xfff, pos = s0 + loc;
                 __stcg(pb + j, (unsigned long long)(unsigned(e << 24) | unsigned(pos)) |
                                    ((unsigned long long)__float_as_uint(sm.cbuf[e][loc]) << 32));
-                prefetch_l2(exs[e]->Wgu + size_t(pos) * p.rec_bytes, uint32_t(kSpec ? p.rec_bytes : p.gu_bytes));
             }
             if (tid == 0) __stcg(p.counts + b, nl);
+            // the rows start moving towards L2 once this CTA has arrived, so
+            // that the arrival's release does not wait for them
+            grid_arrive(p, epoch);
+            for (int j = tid; j < nl; j += kThreads) {
+                const int en = j < n0 ? sm.lst[j] : sm.lst[kMaxStrip + (j - n0)];
+                const int e = en >> 12, pos = s0 + (en & 0xfff);
+                prefetch_l2(exs[e]->Wgu + size_t(pos) * p.rec_bytes, uint32_t(kSpec ? p.rec_bytes : p.gu_bytes));
+            }
         }
-        if (!grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
+        if (!grid_wait(&sm, p, epoch, bci, &cyc_bar)) break;
         {
             // exclusive prefix of the strip counts (S <= 256: warps 0..7)
             const int cnt = tid < S ? __ldcg(p.counts + tid) : 0;
@@ -1120,6 +1142,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         // Rounds of up to kRound neurons: one bulk-copy round brings their
         // W_gate/W_up records (and, when speculative, their W_down rows) into
         // shared memory; the dots of all of them are reduced at once.
+        prof_put(p, li, 8, gtimer());
         const long long cc0 = clock64();
         const int m = sm.share_n;
         const int per_n = kSpec ? p.rec_bytes : p.gu_bytes;   // bytes per neuron in a round (its record)
@@ -1321,28 +1344,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
         if (!gok) break;
         if (tid == 0 && p.stats) atomicAdd(p.stats + li * 4 + 1, nz_total);
-        // the next layer's predictor slice starts moving: U strip straight
-        // into shared memory (free until then), the rest of it into L2
-        // (dense decode: with the V block for the column phase in the top of
-        // the buffer and the U round's first piece below it)
-        const bool vnext = vsm && l + 1 < l1;
-        if (!moe && l + 1 < l1 && warp == 0) {
-            const ExpertDev &nx = sm.exl[(l + 1) & 1][0];
-            if (vnext && lane == 0) {
-                mbar_arrive_tx(&sm.vbar, uint32_t(vbytes));
-                stage_copy(stg + voff, vblk(l + 1), uint32_t(vbytes), &sm.vbar);
-            }
-            if (ns > 0) {
-                const int n1 = vnext ? ufirst : u_round0;
-                stage_u_at(nx, 0, n1, 0, n1 == u_round0);
-                if (lane == 0 && ns > ucap)
-                    prefetch_l2(nx.U + size_t(s0 + ucap) * p.urow, uint32_t(ns - ucap) * p.urow);
-            }
-        }
-        staged_early = !moe && l + 1 < l1 && ns > 0;
-        if (staged_early) pending = true;
-        vpend = vnext;
-        upart2 = staged_early && vnext && ufirst < u_round0;
         // the fixed-point buffer of layer l - 1 (read before two barriers ago)
         // is cleared for layer l + 1
         if (b == S - 1) {
@@ -1363,14 +1364,45 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
         (void)cc0;
         prof_put(p, li, 3, gtimer());
-        if (!grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
+        grid_arrive(p, epoch);
+        // the next layer's predictor slice starts moving once this CTA has
+        // arrived (the arrival's release would otherwise wait for these
+        // copies): the first U round straight into shared memory (free until
+        // then), the rest of the strip into L2; dense decode puts the V block
+        // for the column phase in the top of the buffer and the U round's
+        // first piece below it
+        const bool vnext = vsm && l + 1 < l1;
+        if (!moe && l + 1 < l1 && warp == 0) {
+            const ExpertDev &nx = sm.exl[(l + 1) & 1][0];
+            if (vnext && lane == 0) {
+                mbar_arrive_tx(&sm.vbar, uint32_t(vbytes));
+                stage_copy(stg + voff, vblk(l + 1), uint32_t(vbytes), &sm.vbar);
+            }
+            if (ns > 0) {
+                const int n1 = vnext ? ufirst : u_round0;
+                stage_u_at(nx, 0, n1, 0, n1 == u_round0);
+                if (lane == 0 && ns > ucap)
+                    prefetch_l2(nx.U + size_t(s0 + ucap) * p.urow, uint32_t(ns - ucap) * p.urow);
+            }
+        }
+        staged_early = !moe && l + 1 < l1 && ns > 0;
+        if (staged_early) pending = true;
+        vpend = vnext;
+        upart2 = staged_early && vnext && ufirst < u_round0;
+        if (!grid_wait(&sm, p, epoch, bci, &cyc_bar)) break;
         prof_put(p, li, 4, gtimer());
 
         // ---------------- reduction + next layer's column products -----------
         const bool next = l + 1 < l1;
         if (!column_phase(li + 1, true, next, l + 1, li, vsm && next)) break;
         prof_put(p, li, 5, gtimer());
-        if (next && !grid_sync(&sm, p, epoch, bci, &cyc_bar)) break;
+        if (next) {
+            grid_arrive(p, epoch);
+            // the V block has been read: the rest of the next U round lands there
+            if (upart2 && warp == 0) stage_u_at(sm.exl[(l + 1) & 1][0], ufirst, u_round0 - ufirst, ufirst, true);
+            upart2 = false;
+            if (!grid_wait(&sm, p, epoch, bci, &cyc_bar)) break;
+        }
         prof_put(p, li, 6, gtimer());
         prof_put(p, li, 10, cyc_a);
         prof_put(p, li, 11, cyc_b);

@@ -15,6 +15,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -71,8 +72,15 @@ def measured_peaks():
 
 
 def kernel_hash() -> str:
-    with open(KERNEL_SRC, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """sha256/16 of the kernel's code: the source with its comments and
+    blank space removed, so that editing a comment keeps the recorded
+    counters valid while any change of code voids them."""
+    with open(KERNEL_SRC, encoding="utf-8") as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    code = " ".join(src.split())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def recorded_traffic(workload: str):

@@ -208,9 +208,9 @@ PI_API pi_status pi_debug_set(pi_ffn_t h, int flags, double wait_limit_s);
 /* Testing aid: when `times_dev` is non-NULL, each later pi_sparse_ffn_decode
  * call records, per layer and CTA, %globaltimer (ns) at these points k:
  *   0 layer start, 1 layer input and t ready, 9 predictor logits done,
- *   2 active list done, 3 gather done, 4 after the gather barrier,
- *   7 partials reduced, 5 column phase done, 6 after the column barrier
- *   (8 unused);
+ *   2 active list done, 8 this CTA's share of the active list known,
+ *   3 gather done, 4 after the gather barrier, 7 partials reduced,
+ *   5 column phase done, 6 after the column barrier;
  * and k = 10..13 the clock cycles thread 0 spent obtaining the layer input,
  * waiting for predictor rows, waiting for gathered rows and waiting in grid
  * barriers.  Value (layer - layer_begin, k, cta) sits at
