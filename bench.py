@@ -71,16 +71,18 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_hash() -> str:
-    """sha256/16 of the kernel's code: the source with its comments and
-    blank space removed, so that editing a comment keeps the recorded
-    counters valid while any change of code voids them."""
-    with open(KERNEL_SRC, encoding="utf-8") as f:
-        src = f.read()
+def code_hash(src: str) -> str:
+    """sha256/16 of C/C++ source with its comments and blank space removed,
+    so that editing a comment keeps recorded counters valid while any change
+    of code voids them."""
     src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
     src = re.sub(r"//[^\n]*", " ", src)
-    code = " ".join(src.split())
-    return hashlib.sha256(code.encode()).hexdigest()[:16]
+    return hashlib.sha256(" ".join(src.split()).encode()).hexdigest()[:16]
+
+
+def kernel_hash() -> str:
+    with open(KERNEL_SRC, encoding="utf-8") as f:
+        return code_hash(f.read())
 
 
 def recorded_traffic(workload: str):

@@ -73,3 +73,12 @@ def test_reference_arm_rank0_prints_other_ranks_exit_quietly():
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["cpu_baseline"]["kind"] == "oracle" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_code_hash_ignores_comments_and_blank_space_only():
+    base = "int f(int a) {\n    return a + 1;   // one more\n}\n"
+    same = "/* header */\nint f(int a)\n{ return a + 1; }\n// trailing note\n"
+    changed = "int f(int a) {\n    return a + 2;   // one more\n}\n"
+    assert bench.code_hash(base) == bench.code_hash(same)
+    assert bench.code_hash(base) != bench.code_hash(changed)
+    assert len(bench.kernel_hash()) == 16
