@@ -184,7 +184,15 @@ PI_API pi_status pi_sparse_ffn_decode_host(pi_ffn_t h, int layer_begin, int laye
  * computing").  resid_dev is n_tokens x d float, in/out.  Per layer every
  * token is normalised, routed (MoE), and passed through the full FFN of its
  * expert(s) with no predictor; outputs are combined in ascending expert index
- * and added to the residual. */
+ * and added to the residual.  resid_dev is 16-byte aligned and caller-owned;
+ * the library owns a workspace that grows to the largest n_tokens seen (about
+ * n_tokens x (4 d_ff + 38 d_model) bytes).  Work is asynchronous on
+ * `stream`; pi_sync reports device-side errors.  The result is deterministic
+ * and each token's row depends only on that token.
+ * Errors: PI_ERR_INVALID_ARG (null pointer, bad layer range, n_tokens < 1,
+ * misaligned resid_dev), PI_ERR_NOT_LOADED (a layer of the range not loaded),
+ * PI_ERR_UNSUPPORTED (weights other than F16/BF16/INT4G32, or d_ff not a
+ * multiple of 128), PI_ERR_OOM (workspace), PI_ERR_CUDA. */
 PI_API pi_status pi_dense_ffn_prefill(pi_ffn_t h, int layer_begin, int layer_end, int n_tokens,
                                float *resid_dev, void *stream);
 
