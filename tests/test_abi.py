@@ -43,6 +43,11 @@ def _desc(**kw):
     (dict(n_experts=40, top_k=2), B.PI_ERR_INVALID_ARG),
     (dict(eps=0.0), B.PI_ERR_INVALID_ARG),
     (dict(threshold=float("inf")), B.PI_ERR_INVALID_ARG),
+    (dict(d_model=128), B.PI_ERR_INVALID_ARG),
+    (dict(rank=0), B.PI_ERR_INVALID_ARG),
+    (dict(w_dtype=0, pred_dtype=0, rank=1024), B.PI_ERR_INVALID_ARG),   # fp32 rows hold <= 512
+    (dict(w_dtype=3, pred_dtype=0), B.PI_ERR_UNSUPPORTED),              # INT4 with an fp32 predictor
+    (dict(n_experts=8, top_k=2, w_dtype=0, pred_dtype=0, rank=256), B.PI_ERR_UNSUPPORTED),
 ])
 def test_create_rejects_bad_descriptors_on_host(bad, status):
     h = ctypes.c_void_p()
