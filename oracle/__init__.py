@@ -31,7 +31,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
-DTYPES = {"f32": 0, "f16": 1, "bf16": 2, "int4g32": 3}
+DTYPES = {"f32": 0, "f16": 1, "bf16": 2, "int4g32": 3, "i8row": 4}
 ACTS = {"relu": 0, "reglu": 1, "drelu": 2}
 EPS = 1e-6
 
@@ -63,11 +63,12 @@ def lib():
         L.or_load_row.argtypes = [ip, vp, vp, ctypes.c_long, ip, vp]
         L.or_rmsnorm.argtypes = [vp, ip, dp, vp]
         L.or_predict.argtypes = [ip, ip, ip, ip, vp, vp, vp, dp, vp, vp, vp, vp]
+        L.or_predict_q.argtypes = [ip, ip, ip, ip, vp, vp, vp, vp, vp, dp, vp, vp, vp, vp]
         L.or_ffn_masked.argtypes = [ip, ip, ip, ip, vp, vp, vp, vp, vp, vp, ip, vp, vp, vp, vp, vp]
         L.or_route_top2.argtypes = [ip, ip, ip, vp, vp, vp, vp, vp]
         L.or_strip_offsets.argtypes = [ip, ip, vp]
         L.or_neuron_table.argtypes = [ip, ip, vp, vp]
-        for f in ("or_dequant_int4_g32", "or_load_row", "or_rmsnorm", "or_predict",
+        for f in ("or_dequant_int4_g32", "or_load_row", "or_rmsnorm", "or_predict", "or_predict_q",
                   "or_ffn_masked", "or_route_top2", "or_strip_offsets", "or_neuron_table"):
             getattr(L, f).restype = None
         _lib = L
@@ -125,19 +126,25 @@ def rmsnorm(r: np.ndarray, eps: float = EPS) -> np.ndarray:
     return x
 
 
-def predict(x, V, U, c, pdtype: str, threshold: float = 0.0):
-    """t = V x, z = U t - c, mask = z > threshold.  Returns (t, z, mask)."""
+def predict(x, V, U, c, pdtype: str, threshold: float = 0.0, sV=None, sU=None):
+    """t = V x, z = U t - c, mask = z > threshold.  Returns (t, z, mask).
+    For the "i8row" format V and U are signed bytes and sV, sU their per-row
+    fp32 scales."""
     x = _c(x, np.float64)
     c = _c(c, np.float64)
     V = _c(V)
     U = _c(U)
     rank, d = V.shape
     F = U.shape[0]
+    if pdtype == "i8row":
+        assert sV is not None and sU is not None, "the i8row predictor needs row scales"
+        sV, sU = _c(sV, np.float32), _c(sU, np.float32)
+        assert sV.shape == (rank,) and sU.shape == (F,)
     t = np.empty(rank, np.float64)
     z = np.empty(F, np.float64)
     mask = np.empty(F, np.uint8)
-    lib().or_predict(d, F, rank, DTYPES[pdtype], _p(V), _p(U), _p(c), float(threshold),
-                     _p(x), _p(t), _p(z), _p(mask))
+    lib().or_predict_q(d, F, rank, DTYPES[pdtype], _p(V), _p(sV), _p(U), _p(sU), _p(c),
+                       float(threshold), _p(x), _p(t), _p(z), _p(mask))
     return t, z, mask
 
 
@@ -156,6 +163,8 @@ class Expert:
     s_gate: np.ndarray | None = None   # INT4 scales, F x d/32 fp16
     s_up: np.ndarray | None = None
     s_down: np.ndarray | None = None   # F x d/32 (per neuron column)
+    sU: np.ndarray | None = None       # i8row predictor: fp32 scale per row of U (F)
+    sV: np.ndarray | None = None       # and of V (rank)
 
     @property
     def d(self) -> int:
@@ -237,7 +246,7 @@ def decode_layer(r, experts: list, router=None, threshold: float = 0.0, eps: flo
     zs, masks, hs = [], [], []
     for e_id, w_e in zip(use, wts):
         e = experts[e_id]
-        _, z, mask = predict(x, e.V, e.U, e.c, e.pdtype, threshold)
+        _, z, mask = predict(x, e.V, e.U, e.c, e.pdtype, threshold, e.sV, e.sU)
         h, y_e = ffn_masked(e, x, mask)
         if router is None:
             y = y_e

@@ -31,7 +31,8 @@
  * symmetric group-32 (nibble n = q + 8, low nibble = even element, fp16 scale
  * per 32 consecutive elements of a neuron vector); MoE routing is softmax over
  * the experts, top-2 (ties to the lower index), weights renormalised over the
- * two.
+ * two.  The cheaper predictor format (I8ROW) is symmetric 8-bit with one fp32
+ * scale per row: element k of row i is s_i * q_ik, q_ik a signed byte.
  *
  * Parity status: every function below is pinned by tests/test_oracle_pins.py
  * (closed forms, brute force on 8-neuron layers, the Fig. 8 merge, independent
@@ -42,7 +43,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-enum { OR_F32 = 0, OR_F16 = 1, OR_BF16 = 2, OR_INT4G32 = 3 };
+enum { OR_F32 = 0, OR_F16 = 1, OR_BF16 = 2, OR_INT4G32 = 3, OR_I8ROW = 4 };
 enum { OR_RELU = 0, OR_REGLU = 1, OR_DRELU = 2 };
 
 /* ---------------------------------------------------------------------------
@@ -100,10 +101,18 @@ void or_dequant_int4_g32(const uint8_t *q, const uint16_t *scales, int n,
 }
 
 /* Row `row` of a stored matrix with n columns, as doubles.  For INT4 the
- * matrix is `rows x n/2` bytes of nibbles plus `rows x n/32` fp16 scales. */
+ * matrix is `rows x n/2` bytes of nibbles plus `rows x n/32` fp16 scales; for
+ * I8ROW it is `rows x n` signed bytes plus one fp32 scale per row. */
 void or_load_row(int dtype, const void *base, const void *scales, long row,
                  int n, double *out)
 {
+    if (dtype == OR_I8ROW) {
+        const int8_t *q = (const int8_t *)base + row * (long)n;
+        double s = (double)((const float *)scales)[row];
+        for (int k = 0; k < n; ++k)
+            out[k] = s * (double)q[k];
+        return;
+    }
     if (dtype == OR_INT4G32) {
         or_dequant_int4_g32((const uint8_t *)base + row * (long)(n / 2),
                             (const uint16_t *)scales + row * (long)(n / 32), n,
@@ -133,14 +142,15 @@ void or_rmsnorm(const double *r, int d, double eps, double *x)
  * Low-rank form: t = V x (V is rank x d), z_i = U_i . t - c_i (U is F x rank),
  * neuron i predicted active iff z_i > threshold (threshold 0 by default).
  * ------------------------------------------------------------------------- */
-void or_predict(int d, int F, int rank, int pdtype, const void *V,
-                const void *U, const double *c, double threshold,
-                const double *x, double *t, double *z, uint8_t *mask)
+void or_predict_q(int d, int F, int rank, int pdtype, const void *V,
+                  const void *V_s, const void *U, const void *U_s,
+                  const double *c, double threshold, const double *x,
+                  double *t, double *z, uint8_t *mask)
 {
     #pragma omp parallel for schedule(static)
     for (int k = 0; k < rank; ++k) {
         double *row = (double *)malloc(sizeof(double) * d);
-        or_load_row(pdtype, V, NULL, k, d, row);
+        or_load_row(pdtype, V, V_s, k, d, row);
         double acc = 0.0;
         for (int j = 0; j < d; ++j)
             acc += row[j] * x[j];
@@ -150,7 +160,7 @@ void or_predict(int d, int F, int rank, int pdtype, const void *V,
     #pragma omp parallel for schedule(static)
     for (int i = 0; i < F; ++i) {
         double *row = (double *)malloc(sizeof(double) * rank);
-        or_load_row(pdtype, U, NULL, i, rank, row);
+        or_load_row(pdtype, U, U_s, i, rank, row);
         double acc = 0.0;
         for (int k = 0; k < rank; ++k)
             acc += row[k] * t[k];
@@ -158,6 +168,15 @@ void or_predict(int d, int F, int rank, int pdtype, const void *V,
         mask[i] = z[i] > threshold ? 1 : 0;
         free(row);
     }
+}
+
+/* The float-format predictor (no scales). */
+void or_predict(int d, int F, int rank, int pdtype, const void *V,
+                const void *U, const double *c, double threshold,
+                const double *x, double *t, double *z, uint8_t *mask)
+{
+    or_predict_q(d, F, rank, pdtype, V, NULL, U, NULL, c, threshold, x, t, z,
+                 mask);
 }
 
 /* ---------------------------------------------------------------------------

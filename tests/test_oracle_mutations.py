@@ -38,6 +38,10 @@ MUTATIONS = {
     "router no renorm": ("    weights[0] = p[lo] / (p[lo] + p[hi]);", "    weights[0] = p[lo];"),
     "predictor drops V": ("            acc += row[j] * x[j];\n        t[k] = acc;",
                           "            acc += x[j];\n        t[k] = acc;"),
+    "int8 read unsigned": ("const int8_t *q = (const int8_t *)base + row * (long)n;",
+                           "const uint8_t *q = (const uint8_t *)base + row * (long)n;"),
+    "int8 scale of the wrong row": ("double s = (double)((const float *)scales)[row];",
+                                    "double s = (double)((const float *)scales)[0];"),
     "down skips last neuron": ("        for (int i = 0; i < F; ++i) {\n                if (h[i] == 0.0)",
                                "        for (int i = 0; i < F - 1; ++i) {\n                if (h[i] == 0.0)"),
 }

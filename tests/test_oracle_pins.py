@@ -314,6 +314,41 @@ def test_threshold_minus_infinity_gives_dense(oracle_mod):
     assert np.array_equal(oracle_mod.ffn_masked(e, x, mask)[1], oracle_mod.ffn_masked(e, x)[1])
 
 
+def test_int8_row_predictor_fixture(oracle_mod):
+    """Hand-derived fixture of the 8-bit per-row predictor format (signed bytes
+    in two's complement, -128 and -127 included, one fp32 scale per row)."""
+    g = gold("int8_row_predict.json")
+    V = np.array(g["V_bytes"], np.uint8).view(np.int8)
+    U = np.array(g["U_bytes"], np.uint8).view(np.int8)
+    t, z, mask = oracle_mod.predict(np.array(g["x"]), V, U, f32(g["c"]), "i8row", 0.0,
+                                    f32(g["V_scales"]), f32(g["U_scales"]))
+    assert np.array_equal(t, np.array(g["t"]))
+    assert np.array_equal(z, np.array(g["z"]))
+    assert np.array_equal(mask, np.array(g["mask"], np.uint8))
+
+
+def test_int8_row_predictor_equals_float_predictor_on_its_values(oracle_mod):
+    """With power-of-two scales every dequantised element s * q is exact in
+    fp32, so the 8-bit predictor must give the float predictor's t, z and mask
+    on those fp32 values bit for bit (an independent route to the same
+    numbers: numpy forms s * q, the float path reads it back)."""
+    rng = np.random.default_rng(21)
+    d, F, r = 96, 150, 16
+    qV = rng.integers(-128, 128, (r, d)).astype(np.int8)
+    qU = rng.integers(-128, 128, (F, r)).astype(np.int8)
+    sV = (2.0 ** rng.integers(-9, -4, r)).astype(np.float32)
+    sU = (2.0 ** rng.integers(-9, -4, F)).astype(np.float32)
+    c = rng.standard_normal(F).astype(np.float32) * 0.1
+    x = rng.standard_normal(d)
+    Vf = f32(sV[:, None] * qV.astype(np.float32))
+    Uf = f32(sU[:, None] * qU.astype(np.float32))
+    t1, z1, m1 = oracle_mod.predict(x, qV, qU, c, "i8row", 0.0, sV, sU)
+    t2, z2, m2 = oracle_mod.predict(x, Vf, Uf, c, "f32", 0.0)
+    assert np.array_equal(t1, t2) and np.array_equal(z1, z2) and np.array_equal(m1, m2)
+    # and the numbers are the low-rank predictor of the dequantised matrices
+    assert np.allclose(z1, Uf.astype(np.float64) @ (Vf.astype(np.float64) @ x) - c, rtol=1e-12, atol=1e-12)
+
+
 # ---------------------------------------------------------------------------
 # Neuron table
 # ---------------------------------------------------------------------------
