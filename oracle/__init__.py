@@ -259,6 +259,54 @@ def decode_layer(r, experts: list, router=None, threshold: float = 0.0, eps: flo
                        weights=wts, logits=logits)
 
 
+def decode_layer_batch(R, experts: list, router=None, threshold: float = 0.0,
+                       eps: float = EPS):
+    """One layer of small-batch decode (B independent tokens, rows of R).
+
+    Each token is normalised, routed and predicted on its own.  The rows that
+    are read are those of the union of the tokens' predicted sets (per expert),
+    each read once for the whole batch; token b keeps its own set: its h is
+    computed over the union and set to exactly 0 outside its own predicted set,
+    so its output is its batch-1 output (nearauto.com PowerInfer article,
+    "Experiments", Fig. 14: the sparse path keeps its gains at small batch
+    sizes).  Returns (per-token LayerResults, per-expert union masks)."""
+    R = np.atleast_2d(_c(R, np.float64))
+    Bn = R.shape[0]
+    X = [rmsnorm(R[b], eps) for b in range(Bn)]
+    plans = []
+    for b in range(Bn):
+        if router is None:
+            plans.append(([0], [1.0], None))
+        else:
+            lg, ex, w = route_top2(X[b], router)
+            plans.append(([int(ex[0]), int(ex[1])], [float(w[0]), float(w[1])], lg))
+    preds = {}
+    union = {}
+    for b, (use, _, _) in enumerate(plans):
+        for e_id in use:
+            e = experts[e_id]
+            _, z, m = predict(X[b], e.V, e.U, e.c, e.pdtype, threshold, e.sV, e.sU)
+            preds[(b, e_id)] = (z, m)
+            union[e_id] = m.copy() if e_id not in union else (union[e_id] | m)
+    out = []
+    for b, (use, wts, lg) in enumerate(plans):
+        y = np.zeros_like(R[b])
+        zs, masks, hs = [], [], []
+        for e_id, w_e in zip(use, wts):
+            e = experts[e_id]
+            z, m = preds[(b, e_id)]
+            h_u, _ = ffn_masked(e, X[b], union[e_id])     # h over the rows read for the batch
+            h = np.where(m.astype(bool), h_u, 0.0)          # the token's own set
+            _, y_e = ffn_masked(e, X[b], (h != 0).astype(np.uint8))
+            y = y_e if router is None else y + w_e * y_e
+            zs.append(z)
+            masks.append(m)
+            hs.append(h)
+        out.append(LayerResult(x=X[b], y=y, r_out=R[b] + y, z=zs, mask=masks, h=hs,
+                               experts=use, weights=wts, logits=lg))
+    return out, union
+
+
 def decode_stack(r, layers: list, routers=None, threshold: float = 0.0):
     """Free-running stack: r_{l+1} = r_l + FFN_l(RMSNorm(r_l)).  `layers[l]` is a
     list of experts (one for a dense FFN).  Returns (r_final, [LayerResult])."""

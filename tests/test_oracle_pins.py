@@ -349,6 +349,45 @@ def test_int8_row_predictor_equals_float_predictor_on_its_values(oracle_mod):
     assert np.allclose(z1, Uf.astype(np.float64) @ (Vf.astype(np.float64) @ x) - c, rtol=1e-12, atol=1e-12)
 
 
+@pytest.mark.parametrize("moe", [False, True])
+def test_batch_decode_is_per_token_decode_over_the_union(oracle_mod, moe):
+    """Small-batch decode reads the union of the tokens' predicted rows once,
+    but each token keeps its own set, so its output is its batch-1 output bit
+    for bit.  The case is built so that the rule matters: some token has a
+    neuron in the union, outside its own set, whose gate fires."""
+    rng = np.random.default_rng(31)
+    d, F, r, Bn = 24, 64, 6, 5
+    E = 3 if moe else 1
+    experts = []
+    for _ in range(E):
+        wg = rng.standard_normal((F, d))
+        U, V = rng.standard_normal((F, r)), rng.standard_normal((r, d))
+        experts.append(expert_from(oracle_mod, "reglu", wg, rng.standard_normal((F, d)),
+                                   rng.standard_normal((d, F)), rng.standard_normal(F) * 0.5, U=U, V=V))
+    router = rng.standard_normal((E, d)).astype(np.float16) if moe else None
+    R = rng.standard_normal((Bn, d))
+    res, union = oracle_mod.decode_layer_batch(R, experts, router)
+    matters = False
+    for b in range(Bn):
+        one = oracle_mod.decode_layer(R[b], experts, router)
+        assert one.experts == res[b].experts
+        assert np.array_equal(one.y, res[b].y)
+        for k, e_id in enumerate(one.experts):
+            assert np.array_equal(one.mask[k], res[b].mask[k])
+            assert np.array_equal(one.h[k], res[b].h[k])
+            h_all, _ = oracle_mod.ffn_masked(experts[e_id], one.x)
+            extra = union[e_id].astype(bool) & ~one.mask[k].astype(bool)
+            matters |= bool(np.any(h_all[extra] != 0))
+    for e_id, u in union.items():
+        ref = np.zeros(F, bool)
+        for b in range(Bn):
+            for k, e2 in enumerate(res[b].experts):
+                if e2 == e_id:
+                    ref |= res[b].mask[k].astype(bool)
+        assert np.array_equal(u.astype(bool), ref)
+    assert matters
+
+
 # ---------------------------------------------------------------------------
 # Neuron table
 # ---------------------------------------------------------------------------
