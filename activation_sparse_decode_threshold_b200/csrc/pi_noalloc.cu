@@ -70,6 +70,8 @@ __global__ void na_setup(unsigned char *base, const uint8_t *V, const uint8_t *U
         ex[t].c = c;
         ex[t].Wgu = nullptr;
         ex[t].Wd = nullptr;
+        ex[t].sU = nullptr;
+        ex[t].sV = nullptr;
     }
     int32_t *strips = reinterpret_cast<int32_t *>(base + kOffStrips);
     int32_t *groups = reinterpret_cast<int32_t *>(base + kOffGroups);
@@ -81,6 +83,13 @@ __global__ void na_setup(unsigned char *base, const uint8_t *V, const uint8_t *U
     for (size_t i = t; i < (kOffEx - kOffFix) / 4; i += blockDim.x)
         reinterpret_cast<int *>(base + kOffFix)[i] = 0;
     if (t == 0) *count = -1;
+}
+
+// Runs after the predictor kernel on the same stream: a bounded wait that ran
+// out in any CTA shows as *count = -1, whatever that CTA's peers wrote.
+__global__ void na_finish(const int *err, int32_t *count)
+{
+    if (*reinterpret_cast<const volatile int *>(err) != 0) *count = -1;
 }
 
 }  // namespace
@@ -107,8 +116,9 @@ extern "C" PI_API pi_status pi_predict_noalloc(int d_model, int d_ff, int rank, 
             return na_fail(PI_ERR_INVALID_ARG, "V, U and x must be 16-byte aligned");
 
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
-        return na_fail(PI_ERR_CUDA, "no current CUDA device");
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return na_fail(PI_ERR_CUDA, "no current CUDA device");
+    if (dev >= kMaxDevices)
+        return na_fail(PI_ERR_UNSUPPORTED, "the current device index is 64 or more (devices 0..63 supported)");
     int nsm = 0;
     if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return na_fail(PI_ERR_CUDA, "cudaDeviceGetAttribute failed");
@@ -184,6 +194,9 @@ extern "C" PI_API pi_status pi_predict_noalloc(int d_model, int d_ff, int rank, 
     p.debug_flags = 0;
     p.prof = nullptr;
     e = pi::launch_decode(fmt, fmt, p, st);
+    if (e != cudaSuccess) return na_fail(PI_ERR_CUDA, cudaGetErrorString(e));
+    na_finish<<<1, 1, 0, st>>>(p.err, count_dev);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return na_fail(PI_ERR_CUDA, cudaGetErrorString(e));
     return PI_OK;
 }
