@@ -56,7 +56,6 @@ constexpr int kStageBytes = kHalves * kATileBytes + kBTileBytes;   // 64 KB
 constexpr int kGemmSmem = NSTAGE * kStageBytes + 1024;
 constexpr int kTmemCols = kHalves * BN;           // 512: the whole tensor memory (one CTA per SM)
 constexpr int kSplitK = 4;                        // K splits of the down GEMM
-constexpr long long kWaitNs = 2000000000LL;
 
 enum GemmKind { kGU = 0, kDOWN = 1 };
 
@@ -75,6 +74,8 @@ struct GemmParams {
     float *Ypart;             // [kSplitK x 2T x d] down partials
     int rows_cap;             // 2T
     int *err;
+    long long wait_ns;        // bound on every mbarrier wait
+    int debug_flags;          // PI_DEBUG_STALL_PREFILL: one producer withholds its first arrival
     // A operand: rows of list positions (normalised inputs sorted by expert for
     // the gate/up GEMM, H for the down GEMM), 64 x 128 boxes with 128-byte swizzle
     alignas(64) CUtensorMap tmA;
@@ -110,13 +111,13 @@ __device__ __forceinline__ long long gtimer()
     return t;
 }
 // bounded wait; false (and the error word set) when it runs out
-__device__ bool mbar_wait(uint64_t *b, uint32_t parity, int *err)
+__device__ bool mbar_wait(uint64_t *b, uint32_t parity, int *err, long long wait_ns)
 {
     if (mbar_test(b, parity)) return true;
     const long long t0 = gtimer();
     for (unsigned it = 1;; ++it) {
         if (mbar_test(b, parity)) return true;
-        if ((it & 15) == 0 && gtimer() - t0 > kWaitNs) {
+        if ((it & 15) == 0 && gtimer() - t0 > wait_ns) {
             atomicCAS(err, 0, int(kDevTimeout));
             return false;
         }
@@ -452,9 +453,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         };
         // publish stage `j`: its copies have landed (cp.async group), make
         // them and the dequantised stores visible to the tensor core, arrive
+        // (testing aid: with PI_DEBUG_STALL_PREFILL, producer 0 of the first
+        // gate/up CTA never arrives for its first stage, so the MMA warp's
+        // bounded wait runs out before any MMA is issued)
+        const bool withhold = (p.debug_flags & 2) && KIND == kGU && pt == 0 &&
+                              blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
         auto publish = [&](int j) {
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            mbar_arrive(&full[j % NSTAGE]);
+            if (!(withhold && j == 0)) mbar_arrive(&full[j % NSTAGE]);
         };
         // INT4 raw data of stage j is loaded three steps ahead, rotating
         // through four register sets (no dynamic indexing)
@@ -471,7 +477,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
             const int s = j % NSTAGE;
             if (j >= NSTAGE) {
                 // the MMAs of step j - NSTAGE read this stage
-                if (!mbar_wait(&empty[s], uint32_t(((j - NSTAGE) / NSTAGE) & 1), p.err)) abort_sh = 1;
+                if (!mbar_wait(&empty[s], uint32_t(((j - NSTAGE) / NSTAGE) & 1), p.err, p.wait_ns)) abort_sh = 1;
             }
             if (abort_sh) { stop = true; return; }
             issue_async(kt0 + j, s);
@@ -502,9 +508,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         // exit: the issuing thread waits (bounded) for the last loads it issued
         if (pt == 0)
             for (int q = max(0, j - NSTAGE); q < j; ++q)
-                mbar_wait(&afull[q % NSTAGE], uint32_t((q / NSTAGE) & 1), p.err);
+                mbar_wait(&afull[q % NSTAGE], uint32_t((q / NSTAGE) & 1), p.err, p.wait_ns);
         // epilogue: wait for the accumulator
-        if (nk > 0 && !abort_sh && !mbar_wait(&done, 0u, p.err)) abort_sh = 1;
+        if (nk > 0 && !abort_sh && !mbar_wait(&done, 0u, p.err, p.wait_ns)) abort_sh = 1;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const int col0 = kEpiCols * (warp >> 2);
         for (int h = 0; h < nh; ++h) {
@@ -555,8 +561,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
             int issued = 0;
             for (int j = 0; j < nk; ++j) {
                 const int s = j % NSTAGE;
-                if (!mbar_wait(&full[s], uint32_t((j / NSTAGE) & 1), p.err) ||
-                    !mbar_wait(&afull[s], uint32_t((j / NSTAGE) & 1), p.err)) { abort_sh = 1; break; }
+                if (!mbar_wait(&full[s], uint32_t((j / NSTAGE) & 1), p.err, p.wait_ns) ||
+                    !mbar_wait(&afull[s], uint32_t((j / NSTAGE) & 1), p.err, p.wait_ns)) { abort_sh = 1; break; }
                 if (abort_sh) break;
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                 const uint32_t a0 = s2u(smem + s * kStageBytes), b0 = a0 + kHalves * kATileBytes;
@@ -577,7 +583,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
             umma_commit(&done);
             if (issued < nk) {
                 // aborted: let the issued MMAs finish (bounded) before TMEM is freed
-                mbar_wait(&done, 0u, p.err);
+                mbar_wait(&done, 0u, p.err, p.wait_ns);
             }
         }
         __syncwarp();
@@ -882,6 +888,8 @@ int prefill_run(PrefillState **state, const PrefillView &v, int l0, int l1, int 
     gp.Ypart = reinterpret_cast<float *>(B + o_y);
     gp.rows_cap = rows_cap;
     gp.err = v.err;
+    gp.wait_ns = v.wait_ns;
+    gp.debug_flags = v.debug_flags;
     const int mtiles = (rows_cap + kTileRows - 1) / kTileRows + v.E;   // upper bound over experts
     // tensor maps of the A operands: rows_cap rows of K 16-bit elements,
     // boxes of 64 elements (128 bytes) x 128 rows, 128-byte swizzle

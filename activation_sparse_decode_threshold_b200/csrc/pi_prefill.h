@@ -19,6 +19,8 @@ struct PrefillView {
     uint8_t *const *router;                     // host copy [n_layers] device pointers
     const std::vector<std::vector<int32_t>> *perm;
     int *err;                                   // the handle's device error word
+    long long wait_ns;                          // bound on every device-side wait
+    int debug_flags;                            // PI_DEBUG_* testing aids
 };
 
 // Returns 0 on success, 1 unsupported, 2 CUDA error, 3 out of memory; `msg`

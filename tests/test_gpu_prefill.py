@@ -65,10 +65,13 @@ def _routable(res) -> np.ndarray:
     return (s[:, 1] - s[:, 2]) > ROUTE_MARGIN
 
 
-def _check(y_gpu, res):
+def _check(y_gpu, res, case=None):
     ok = _routable(res)
     assert ok.mean() > 0.9
-    return G.check_output(y_gpu[ok].ravel(), res.y[ok].ravel())
+    rl, ma = G.check_output(y_gpu[ok].ravel(), res.y[ok].ravel())
+    if case:
+        G.record_error(case, rel_l2=rl, max_abs=ma)
+    return rl, ma
 
 
 @pytest.mark.parametrize("name", sorted(SMALL))
@@ -83,7 +86,7 @@ def test_prefill_single_layer(handles, name, T):
     res = oracle.prefill_layer(Rn, ex, router)
     y_gpu = out.double().cpu().numpy() - Rn
     assert np.all(np.isfinite(y_gpu))
-    _check(y_gpu, res)
+    _check(y_gpu, res, f"prefill/small/{name}")
 
 
 def test_prefill_two_layer_stack(handles):
@@ -133,10 +136,26 @@ def test_prefill_rejects_unsupported_shapes(handles):
     assert ei.value.status == B.PI_ERR_UNSUPPORTED
 
 
+def _tile_rows(Rn: np.ndarray, router: np.ndarray) -> np.ndarray:
+    """Tokens that cover every 128-row tile half of every expert's GEMM rows:
+    the first, middle and last list position of each half, the list of an
+    expert being its tokens in ascending order (the kernel's sort order)."""
+    ex = np.array([oracle.route_top2(oracle.rmsnorm(row), router)[1] for row in Rn])
+    rows = set()
+    for e in range(router.shape[0]):
+        toks = np.nonzero((ex == e).any(axis=1))[0]
+        for h0 in range(0, toks.size, 128):
+            half = toks[h0:h0 + 128]
+            rows.update(int(half[i]) for i in (0, half.size // 2, half.size - 1))
+    return np.array(sorted(rows))
+
+
 def test_prefill_full_size_moe_512_tokens(handles):
     """The 47B MoE shape, INT4 experts, one 512-token prompt through layer 0
-    and the last layer; sampled tokens of each layer against the oracle,
-    teacher-forced on the GPU's own layer input."""
+    and the last layer; teacher-forced on the GPU's own layer input, each
+    layer checked against the oracle on tokens that cover every 128-row tile
+    half of every expert (first, middle and last list position of each half,
+    so each expert's ragged last tile is covered too)."""
     cfg = synth.CONFIGS["mixtral47b"]
     T = cfg.prefill_tokens
     h = G.create(cfg, 2)
@@ -149,13 +168,36 @@ def test_prefill_full_size_moe_512_tokens(handles):
     out = _prefill(h, mid, 1, 2)
     assert torch.isfinite(out).all()
     assert torch.equal(_prefill(h, R, 0, 2), out)      # the stack call is the same arithmetic
-    rows = np.array([0, 1, 77, 255, 256, 511])
     for slot, (rin, rout) in enumerate([(R, mid), (mid, out)]):
         lw = synth.make_layer(cfg, layers[slot], "cuda")
         ex, router = G.oracle_layer(cfg, lw)
         del lw
-        Rn = rin.double().cpu().numpy()[rows]
+        Rall = rin.double().cpu().numpy()
+        rows = _tile_rows(Rall, router)
+        assert rows.size >= 2 * cfg.n_experts
+        Rn = Rall[rows]
         res = oracle.prefill_layer(Rn, ex, router)
         y_gpu = rout.double().cpu().numpy()[rows] - Rn
         ok = _routable(res)
-        G.check_output(y_gpu[ok].ravel(), res.y[ok].ravel())
+        rl, ma = G.check_output(y_gpu[ok].ravel(), res.y[ok].ravel())
+        G.record_error("prefill/full/mixtral47b-512tok", rel_l2=rl, max_abs=ma, rows=int(ok.sum()))
+
+
+def test_prefill_bounded_wait_reports_timeout_and_handle_survives(handles):
+    """A prefill whose tensor-core issuer never sees its first stage published
+    (PI_DEBUG_STALL_PREFILL) gives up after the handle's wait limit, releases
+    its tensor memory and reports PI_ERR_TIMEOUT; the next prefill on the same
+    handle is correct."""
+    cfg = SMALL["moe-int4-drelu"]
+    h, lws = _build(cfg, handles, n_layers=1)
+    R = synth.prefill_input(cfg, 200, "cuda")
+    B.pi_debug_set(h, B.PI_DEBUG_STALL_PREFILL, 0.05)
+    r = R.clone()
+    B.pi_dense_ffn_prefill(h, 0, 1, 200, r)
+    assert B.pi_sync(h) == B.PI_ERR_TIMEOUT
+    B.pi_debug_set(h, 0, 2.0)
+    out = _prefill(h, R, 0, 1)
+    ex, router = G.oracle_layer(cfg, lws[0])
+    Rn = R.double().cpu().numpy()
+    res = oracle.prefill_layer(Rn, ex, router)
+    _check(out.double().cpu().numpy() - Rn, res)
