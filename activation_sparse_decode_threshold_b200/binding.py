@@ -21,8 +21,9 @@ PI_ERR_CUDA, PI_ERR_TIMEOUT, PI_ERR_DEVICE_CHECK, PI_ERR_NOT_LOADED = 4, 5, 6, 7
 STATUS = {0: "PI_OK", 1: "PI_ERR_INVALID_ARG", 2: "PI_ERR_UNSUPPORTED", 3: "PI_ERR_OOM",
           4: "PI_ERR_CUDA", 5: "PI_ERR_TIMEOUT", 6: "PI_ERR_DEVICE_CHECK", 7: "PI_ERR_NOT_LOADED"}
 ACT = {"relu": 0, "reglu": 1, "drelu": 2}
-DTYPE = {"f32": 0, "f16": 1, "bf16": 2, "int4g32": 3}
+DTYPE = {"f32": 0, "f16": 1, "bf16": 2, "int4g32": 3, "i8row": 4}
 PI_DEBUG_STALL_BARRIER = 1
+PI_DEBUG_STALL_PREFILL = 2
 
 
 class PiError(RuntimeError):
@@ -42,7 +43,8 @@ class pi_ffn_desc(ctypes.Structure):
 class pi_expert_weights(ctypes.Structure):
     _fields_ = [("w_gate", ctypes.c_void_p), ("w_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p),
                 ("s_gate", ctypes.c_void_p), ("s_up", ctypes.c_void_p), ("s_down", ctypes.c_void_p),
-                ("bias", ctypes.c_void_p), ("U", ctypes.c_void_p), ("V", ctypes.c_void_p)]
+                ("bias", ctypes.c_void_p), ("U", ctypes.c_void_p), ("V", ctypes.c_void_p),
+                ("s_U", ctypes.c_void_p), ("s_V", ctypes.c_void_p)]
 
 
 _lib = None
@@ -65,6 +67,7 @@ def lib() -> ctypes.CDLL:
             "pi_predict": [vp, ip, ip, vp, vp, vp, vp, vp],
             "pi_sparse_ffn_decode": [vp, ip, ip, vp, vp, vp, vp, vp],
             "pi_sparse_ffn_decode_host": [vp, ip, ip, vp, vp, vp],
+            "pi_sparse_ffn_decode_batch": [vp, ip, ip, ip, vp, vp, vp, vp, vp],
             "pi_dense_ffn_prefill": [vp, ip, ip, ip, vp, vp],
             "pi_sync": [vp, vp],
             "pi_debug_set": [vp, ip, ctypes.c_double],
@@ -134,14 +137,15 @@ def pi_ffn_destroy(h: int):
 
 def pi_ffn_load_layer(h, layer, experts, router=None, freq=None, stream=None):
     """`experts`: list of objects with attributes w_gate, w_up, w_down, s_gate,
-    s_up, s_down, c (bias), U, V (device tensors, None where absent).
+    s_up, s_down, c (bias), U, V, sU, sV (device tensors, None where absent).
     `freq`: host float32 array (n_experts x F) or None."""
     import numpy as np
     arr = (pi_expert_weights * len(experts))()
     for i, e in enumerate(experts):
         arr[i] = pi_expert_weights(_ptr(e.w_gate), _ptr(e.w_up), _ptr(e.w_down),
                                    _ptr(getattr(e, "s_gate", None)), _ptr(getattr(e, "s_up", None)),
-                                   _ptr(getattr(e, "s_down", None)), _ptr(e.c), _ptr(e.U), _ptr(e.V))
+                                   _ptr(getattr(e, "s_down", None)), _ptr(e.c), _ptr(e.U), _ptr(e.V),
+                                   _ptr(getattr(e, "sU", None)), _ptr(getattr(e, "sV", None)))
     fq = None
     if freq is not None:
         fq = np.ascontiguousarray(np.asarray(freq, np.float32))
@@ -176,6 +180,14 @@ def pi_sparse_ffn_decode(h, layer_begin, layer_end, resid, trace=None, stats=Non
     _check(lib().pi_sparse_ffn_decode(h, layer_begin, layer_end, _ptr(resid), _ptr(trace),
                                       _ptr(stats), _ptr(masks), _stream(stream)),
            "pi_sparse_ffn_decode")
+
+
+def pi_sparse_ffn_decode_batch(h, layer_begin, layer_end, resid, trace=None, stats=None, masks=None,
+                               stream=None):
+    """`resid`: device float32 tensor [n_tokens x d] (n_tokens = resid.shape[0])."""
+    _check(lib().pi_sparse_ffn_decode_batch(h, layer_begin, layer_end, int(resid.shape[0]), _ptr(resid),
+                                            _ptr(trace), _ptr(stats), _ptr(masks), _stream(stream)),
+           "pi_sparse_ffn_decode_batch")
 
 
 def pi_sparse_ffn_decode_host(h, layer_begin, layer_end, resid_in, resid_out, stream=None):

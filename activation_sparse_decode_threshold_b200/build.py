@@ -16,7 +16,8 @@ CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libpi_ffn.so")
 OBJ = os.path.join(ROOT, "_build")
 SOURCES = ["pi_decode_f16.cu", "pi_decode_bf16.cu", "pi_decode_i4f16.cu", "pi_decode_i4bf16.cu",
-           "pi_decode_f32.cu", "pi_host.cu", "pi_decode.cu", "pi_repack.cu", "pi_prefill.cu", "pi_noalloc.cu"]
+           "pi_decode_f16i8.cu", "pi_decode_bf16i8.cu", "pi_decode_i4i8.cu",
+           "pi_decode_f32.cu", "pi_host.cu", "pi_decode.cu", "pi_repack.cu", "pi_prefill.cu", "pi_noalloc.cu", "pi_batch.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-Xcompiler", "-fvisibility=hidden"]

@@ -10,6 +10,9 @@ cudaError_t decode_launch_bf16(int d, int mode, const DecodeParams &p, cudaStrea
 cudaError_t decode_launch_i4f16(int d, int mode, const DecodeParams &p, cudaStream_t st, bool query, int *blocks);
 cudaError_t decode_launch_i4bf16(int d, int mode, const DecodeParams &p, cudaStream_t st, bool query,
                                  int *blocks);
+cudaError_t decode_launch_f16i8(int d, int mode, const DecodeParams &p, cudaStream_t st, bool query, int *blocks);
+cudaError_t decode_launch_bf16i8(int d, int mode, const DecodeParams &p, cudaStream_t st, bool query, int *blocks);
+cudaError_t decode_launch_i4i8(int d, int mode, const DecodeParams &p, cudaStream_t st, bool query, int *blocks);
 
 namespace {
 
@@ -21,6 +24,9 @@ cudaError_t dispatch(int wfmt, int pfmt, int d, int mode, const DecodeParams &p,
     if (wfmt == kBF16 && pfmt == kBF16) return decode_launch_bf16(d, mode, p, st, query, blocks);
     if (wfmt == kI4 && pfmt == kF16) return decode_launch_i4f16(d, mode, p, st, query, blocks);
     if (wfmt == kI4 && pfmt == kBF16) return decode_launch_i4bf16(d, mode, p, st, query, blocks);
+    if (wfmt == kF16 && pfmt == kI8) return decode_launch_f16i8(d, mode, p, st, query, blocks);
+    if (wfmt == kBF16 && pfmt == kI8) return decode_launch_bf16i8(d, mode, p, st, query, blocks);
+    if (wfmt == kI4 && pfmt == kI8) return decode_launch_i4i8(d, mode, p, st, query, blocks);
     return cudaErrorInvalidValue;
 }
 

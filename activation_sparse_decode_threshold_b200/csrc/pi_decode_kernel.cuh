@@ -155,11 +155,12 @@ template <> struct Fm<kF32>  { static constexpr int VB = 16, EPV = 4;  using V =
 template <> struct Fm<kF16>  { static constexpr int VB = 16, EPV = 8;  using V = uint4; };
 template <> struct Fm<kBF16> { static constexpr int VB = 16, EPV = 8;  using V = uint4; };
 template <> struct Fm<kI4>   { static constexpr int VB = 8,  EPV = 16; using V = uint2; };
+template <> struct Fm<kI8>   { static constexpr int VB = 8,  EPV = 8;  using V = uint2; };   // signed bytes (row scale apart)
 
 template <int F>
 __device__ __forceinline__ typename Fm<F>::V ldvec(const uint8_t *p)
 {
-    if constexpr (F == kI4) return ldw2(p);
+    if constexpr (F == kI4 || F == kI8) return ldw2(p);
     else return ldw4(p);
 }
 
@@ -184,6 +185,12 @@ __device__ __forceinline__ void cvt(const typename Fm<F>::V &v, float *o)
             o[2 * i] = __uint_as_float(w[i] << 16);
             o[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
         }
+    } else if constexpr (F == kI8) {
+        const uint32_t w[2] = {v.x, v.y};
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) o[4 * i + j] = float(int8_t(uint8_t(w[i] >> (8 * j))));
     } else {
         // element 2j sits in the low nibble of byte j; n - 8 is formed exactly
         // by placing n in the mantissa of 2^23 and subtracting 2^23 + 8
@@ -274,6 +281,21 @@ __device__ __forceinline__ void split_parts(float x, int nparts, uint16_t *out, 
     }
 }
 
+// Four signed bytes (byte j = element j) as two f16x2 values, exactly: each
+// byte is biased to unsigned, placed in the mantissa of 1024 (0x6400 | u is
+// 1024 + u in binary16) and 1024 + 128 is subtracted.
+__device__ __forceinline__ void i8x4_to_h2(uint32_t w, uint32_t &lo, uint32_t &hi)
+{
+    const uint32_t u = w ^ 0x80808080u;
+    const uint32_t a = __byte_perm(u, 0x64646464u, 0x7170);
+    const uint32_t b = __byte_perm(u, 0x64646464u, 0x7372);
+    const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));   // 1152
+    const __half2 ha = __hsub2(*reinterpret_cast<const __half2 *>(&a), bias);
+    const __half2 hb = __hsub2(*reinterpret_cast<const __half2 *>(&b), bias);
+    lo = *reinterpret_cast<const uint32_t *>(&ha);
+    hi = *reinterpret_cast<const uint32_t *>(&hb);
+}
+
 __device__ __forceinline__ float act_h(int act, float g, float u)
 {
     const float gp = g > 0.f ? g : 0.f;
@@ -342,59 +364,59 @@ __device__ __forceinline__ void prof_put(const DecodeParams &p, int li, int poin
 }
 
 // Fixed-point accumulation (exact, so the result does not depend on the
-// order in which CTAs arrive): values are rounded to multiples of 2^-32 (2^-24
-// for sums of squares) and added as 64-bit integers.
-__device__ __forceinline__ void fix_add(long long *dst, float v, float scale)
+// order in which CTAs arrive): values are rounded to multiples of 2^-32 and
+// added as 64-bit integers.  A scaled value of magnitude 2^55 or more (or not
+// finite) could make the sum over up to 256 CTAs leave the int64 range: it is
+// recorded as a failed device check (the caller's pi_sync reports
+// PI_ERR_DEVICE_CHECK) instead of wrapping silently.
+constexpr float kFixT = 4294967296.0f;    // 2^32
+constexpr float kFixMax = 36028797018963968.0f;   // 2^55
+__device__ __forceinline__ void fix_add(long long *dst, float v, float scale, int *err)
 {
-    const long long q = __float2ll_rn(v * scale);
+    const float sv = v * scale;
+    if (!(fabsf(sv) < kFixMax)) {
+        set_error(err, kDevCheck);
+        return;
+    }
+    const long long q = __float2ll_rn(sv);
     atomicAdd(reinterpret_cast<unsigned long long *>(dst), static_cast<unsigned long long>(q));
 }
-constexpr float kFixT = 4294967296.0f;    // 2^32
-constexpr float kFixSS = 16777216.0f;     // 2^24
 
 // Grid-wide barrier of all CTAs of the cooperative launch, in two halves so
-// that a CTA can issue work between its arrival and its wait.  Arrivals are
-// spread over kBarLanes counters, one 128-byte line each (CTA b arrives on
-// counter b mod kBarLanes), so that they do not serialise on one L2 line;
-// the counters are never reset within a launch.  Thread 0 arrives with a
-// release (after the block barrier, so it carries the whole CTA's writes);
-// warp 0 then polls all counters at once, lane i reading counter i with an
-// acquire, bounded by wait_ns, and the verdict is broadcast through shared
-// memory so the whole CTA agrees.
+// that a CTA can issue work between its arrival and its wait.  Thread 0
+// arrives with a release on one counter (after the block barrier, so it
+// carries the whole CTA's writes) and then polls it with acquires until all
+// S CTAs of this barrier's epoch have arrived, bounded by wait_ns; the
+// verdict is broadcast through shared memory so the whole CTA agrees.  The
+// counter is never reset within a launch.  (Measured on the B200: one counter
+// polled by one thread per CTA completes a barrier of 148 CTAs in about 1.3
+// us, against 1.7 us for arrivals spread over 16 counters polled by a warp.)
 __device__ __forceinline__ void grid_arrive(const DecodeParams &p, unsigned &epoch)
 {
     cta_sync();
-    if (threadIdx.x < 32) {
-        epoch += 1;
-        if (threadIdx.x == 0) red_release_gpu(p.bar + (blockIdx.x % kBarLanes) * kBarStride, 1u);
-    }
+    epoch += 1;
+    if (threadIdx.x == 0) red_release_gpu(p.bar, 1u);
 }
 __device__ bool grid_wait(Smem *sm, const DecodeParams &p, unsigned epoch, int &bci, long long *cyc)
 {
-    if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
+    if (threadIdx.x == 0) {
         const long long c0 = clock64();
-        // CTAs per counter: S / kBarLanes, one more for the first S % kBarLanes
-        const unsigned S = gridDim.x;
-        unsigned target = lane < kBarLanes ? epoch * (S / kBarLanes + (unsigned(lane) < S % kBarLanes ? 1u : 0u)) : 0u;
-        if ((p.debug_flags & 1) && epoch == 1 && lane == 0) target += 1;   // PI_DEBUG_STALL_BARRIER
-        const unsigned *ctr = p.bar + (lane < kBarLanes ? lane : 0) * kBarStride;
+        unsigned target = epoch * gridDim.x;
+        if ((p.debug_flags & 1) && epoch == 1) target += 1;   // PI_DEBUG_STALL_BARRIER
         bool ok = true;
-        const long long t0 = gtimer();
-        for (unsigned it = 1;; ++it) {
-            const bool mine = lane >= kBarLanes || ld_acquire_gpu(ctr) >= target;
-            if (__all_sync(0xffffffffu, mine)) break;
-            // the timeout verdict is taken warp-wide so every lane leaves together
-            if ((it & 63) == 0 && __any_sync(0xffffffffu, gtimer() - t0 > p.wait_ns)) {
-                if (lane == 0) set_error(p.err, kDevTimeout);
-                ok = false;
-                break;
+        if (ld_acquire_gpu(p.bar) < target) {
+            const long long t0 = gtimer();
+            for (unsigned it = 1;; ++it) {
+                if (ld_acquire_gpu(p.bar) >= target) break;
+                if ((it & 31) == 0 && gtimer() - t0 > p.wait_ns) {
+                    set_error(p.err, kDevTimeout);
+                    ok = false;
+                    break;
+                }
             }
         }
-        if (lane == 0) {
-            st_vol(&sm->bc[bci], ok ? 1 : 0);
-            if (cyc) *cyc += clock64() - c0;
-        }
+        st_vol(&sm->bc[bci], ok ? 1 : 0);
+        if (cyc) *cyc += clock64() - c0;
     }
     cta_sync();
     const bool ok = ld_vol(&sm->bc[bci]) != 0;
@@ -550,6 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     uint16_t *const tpart = reinterpret_cast<uint16_t *>(sm.tsm);
     auto put_t = [&](int k, float tv, int ntr) {
         if constexpr (PF == kF32) sm.tsm[k] = tv;
+        else if constexpr (PF == kI8) split_parts<kF16>(tv, 2, tpart + k, ntr);
         else split_parts<PF>(tv, (PF == kBF16 && 3 * ntr <= 2 * kMaxRankTotal) ? 3 : 2, tpart + k, ntr);
     };
 
@@ -624,16 +647,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         if (!predict && p.trace && li_in < l1 - l0)
             for (int j = tid; j < ncol; j += kThreads) __stcg(p.trace + size_t(li_in) * d + c0 + j, sm.rsl[j]);
         if (!next_exists) return true;
-        // sum of squares of this CTA's columns (fixed order: lanes, then tree)
+        // sum of squares of this CTA's columns (fixed order: lanes, then tree),
+        // one float per CTA; the layer start sums the CTAs' values in CTA order
         if (warp == 0 && !predict) {
             float ss = 0.f;
             for (int j = lane; j < ncol; j += 32) ss = fmaf(sm.rsl[j], sm.rsl[j], ss);
             ss = warp_sum(ss);
-            if (lane == 0 && ncol > 0) fix_add(fx + kMaxRankTotal, ss, kFixSS);
+            if (lane == 0) __stcg(p.ssq + size_t(li_in & 1) * kMaxStrips + b, ss);
         }
         if (!moe) {
             // t partial: rows kr0, kr1 of the V block dotted with this CTA's columns
+            // (8-bit predictor: times the rows' scales)
             float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+            float sv0 = 1.f, sv1 = 1.f;
+            if constexpr (PF == kI8) {
+                if (tpart && kr0 < r) sv0 = __ldg(sm.exl[l_next & 1][0].sV + kr0);
+                if (tpart && kr1 < r) sv1 = __ldg(sm.exl[l_next & 1][0].sV + kr1);
+            }
             auto acc_vec = [&](const VP &q0, const VP &q1, int v) {
                 float w0[EPVP], w1[EPVP];
                 cvt<PF>(q0, w0);
@@ -664,8 +694,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                         acc_vec(*reinterpret_cast<const VP *>(vs0 + jj * VBP),
                                 *reinterpret_cast<const VP *>(vs1 + jj * VBP), jj);
                     }
-                    fix_add(fx + kr0, a0 + a1, kFixT);
-                    if (kr1 < r) fix_add(fx + kr1, b0 + b1, kFixT);
+                    fix_add(fx + kr0, (a0 + a1) * sv0, kFixT, p.err);
+                    if (kr1 < r) fix_add(fx + kr1, (b0 + b1) * sv1, kFixT, p.err);
                 }
             } else if (tpart && kr0 < r) {
 #pragma unroll
@@ -676,8 +706,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     const VP q1 = kr1 < r ? ldvec<PF>(vrow1 + v * VBP) : q0;
                     acc_vec(q0, q1, v);
                 }
-                fix_add(fx + kr0, a0 + a1, kFixT);
-                if (kr1 < r) fix_add(fx + kr1, b0 + b1, kFixT);
+                fix_add(fx + kr0, (a0 + a1) * sv0, kFixT, p.err);
+                if (kr1 < r) fix_add(fx + kr1, (b0 + b1) * sv1, kFixT, p.err);
             }
         } else if (!predict) {
             // router logit partials: W_r[e, cols] . r[cols]
@@ -685,7 +715,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             if (tid < p.E && ncol > 0) {
                 float a = 0.f;
                 for (int j = 0; j < ncol; ++j) a = fmaf(__half2float(R[size_t(tid) * d + c0 + j]), sm.rsl[j], a);
-                fix_add(fx + kMaxRankTotal + 1 + tid, a, kFixT);
+                fix_add(fx + kMaxRankTotal + 1 + tid, a, kFixT, p.err);
             }
         }
         return true;
@@ -709,11 +739,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 
         // ---------------- layer input x, [MoE] routing and t rows ------------
         const float *src = predict ? p.x_in : p.resid;
-        float inv = 1.f;
-        if (!predict) {
-            const long long ssq = __ldcg(fx + kMaxRankTotal);
-            inv = 1.f / sqrtf(float(double(ssq) * (1.0 / 16777216.0)) / float(d) + p.eps);
-        }
+        // every global load of the layer start is issued before the sum of
+        // squares is known (one round trip): this thread's columns of r (or
+        // x), t's fixed-point values (dense) and the strip's biases
 #pragma unroll
         for (int k = 0; k < MAXVW; ++k) {
             const int v = tid + kThreads * k;
@@ -721,8 +749,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             for (int i = 0; i < EPVW; i += 4) {
                 float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (v < nvecW) q = __ldcg(reinterpret_cast<const float4 *>(src + v * EPVW + i));
-                xw[k * EPVW + i] = q.x * inv; xw[k * EPVW + i + 1] = q.y * inv;
-                xw[k * EPVW + i + 2] = q.z * inv; xw[k * EPVW + i + 3] = q.w * inv;
+                xw[k * EPVW + i] = q.x; xw[k * EPVW + i + 1] = q.y;
+                xw[k * EPVW + i + 2] = q.z; xw[k * EPVW + i + 3] = q.w;
             }
         }
         if constexpr (!kSameX) {
@@ -733,28 +761,47 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 for (int i = 0; i < EPVP; i += 4) {
                     float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
                     if (v < nvecP) q = __ldcg(reinterpret_cast<const float4 *>(src + v * EPVP + i));
-                    xp_own[k * EPVP + i] = q.x * inv; xp_own[k * EPVP + i + 1] = q.y * inv;
-                    xp_own[k * EPVP + i + 2] = q.z * inv; xp_own[k * EPVP + i + 3] = q.w * inv;
+                    xp_own[k * EPVP + i] = q.x; xp_own[k * EPVP + i + 1] = q.y;
+                    xp_own[k * EPVP + i + 2] = q.z; xp_own[k * EPVP + i + 3] = q.w;
                 }
+            }
+        }
+        long long tq[kMaxRankTotal / kThreads];
+        if (!moe) {
+#pragma unroll
+            for (int j = 0; j < kMaxRankTotal / kThreads; ++j) {
+                const int k = tid + kThreads * j;
+                tq[j] = k < r ? __ldcg(fx + k) : 0;
+            }
+            for (int i = tid; i < ns; i += kThreads) sm.cbuf[0][i] = __ldg(sm.exl[l & 1][0].c + s0 + i);
+        }
+        float inv = 1.f;
+        if (!predict) {
+            // sum of squares: the CTAs' values in CTA order (warp 0; lane j takes
+            // CTAs j, j + 32, ..., then a fixed tree), broadcast through shared memory
+            if (warp == 0) {
+                const float *sq = p.ssq + size_t(li & 1) * kMaxStrips;
+                float ss = 0.f;
+                for (int c = lane; c < S; c += 32) ss += __ldcg(sq + c);
+                ss = warp_sum(ss);
+                if (lane == 0) sm.inv_rms = 1.f / sqrtf(ss / float(d) + p.eps);
+            }
+            cta_sync();
+            inv = sm.inv_rms;
+#pragma unroll
+            for (int i = 0; i < MAXVW * EPVW; ++i) xw[i] *= inv;
+            if constexpr (!kSameX) {
+#pragma unroll
+                for (int i = 0; i < MAXVP * EPVP; ++i) xp_own[i] *= inv;
             }
         }
         if (!moe) {
             // t from the fixed-point column partials
-            {
-                long long tq[kMaxRankTotal / kThreads];
 #pragma unroll
-                for (int j = 0; j < kMaxRankTotal / kThreads; ++j) {
-                    const int k = tid + kThreads * j;
-                    tq[j] = k < r ? __ldcg(fx + k) : 0;
-                }
-#pragma unroll
-                for (int j = 0; j < kMaxRankTotal / kThreads; ++j) {
-                    const int k = tid + kThreads * j;
-                    if (k < r) put_t(k, float(double(tq[j]) * (1.0 / 4294967296.0)) * inv, r);
-                }
+            for (int j = 0; j < kMaxRankTotal / kThreads; ++j) {
+                const int k = tid + kThreads * j;
+                if (k < r) put_t(k, float(double(tq[j]) * (1.0 / 4294967296.0)) * inv, r);
             }
-            // this strip's biases, in the same round trip as t and x
-            for (int i = tid; i < ns; i += kThreads) sm.cbuf[0][i] = __ldg(sm.exl[l & 1][0].c + s0 + i);
             // the next layer's weight pointers, for its prefetches during this layer
             if (tid == kThreads - 1 && l + 1 < l1) sm.exl[(l + 1) & 1][0] = p.ex[size_t(l + 1) * p.E];
             if (tid == 0) {
@@ -801,35 +848,51 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 sm.route_e[1] = hi;
                 sm.route_w[0] = wlo;
                 sm.route_w[1] = whi;
-                // the experts' V rows and U strips start moving now
+                for (int e = 0; e < ntop; ++e) sm.exl[l & 1][e] = p.ex[size_t(l) * p.E + (e == 0 ? lo : hi)];
+            }
+            // the first round of this CTA's V rows is on the critical path: its
+            // copies are issued at once (thread 0), and only then do the
+            // experts' U strips start moving towards L2 (needed after the
+            // t barrier), so that they queue behind the V rows
+            const int per = min(kRA, kStageBytes / p.vrow);
+            auto issue_vrows = [&](int row0, int n) {
+                mbar_arrive_tx(&sm.stage_bar, uint32_t(n) * p.vrow);
+                for (int rr = 0; rr < n;) {
+                    const int row = row0 + rr, e = row / r;
+                    const int cnt = min(n - rr, (e + 1) * r - row);
+                    const uint8_t *vrow = sm.exl[l & 1][e].V + size_t(row - e * r) * p.vrow;
+                    stage_copy(stg + size_t(rr) * p.vrow, vrow, uint32_t(cnt) * p.vrow, &sm.stage_bar);
+                    rr += cnt;
+                }
+            };
+            // the experts' U strips (needed after the t barrier) start moving
+            // towards L2 once the first V round has landed, so that they do not
+            // compete with it
+            auto prefetch_u = [&]() {
+                for (int e = 0; e < ntop; ++e)
+                    if (ns > 0) prefetch_l2(sm.exl[l & 1][e].U + size_t(s0) * p.urow, uint32_t(ns) * p.urow);
+            };
+            if (tid == 0) {
+                if (a1 > a0) issue_vrows(a0, min(per, a1 - a0));
                 for (int e = 0; e < ntop; ++e) {
-                    const ExpertDev ex = p.ex[size_t(l) * p.E + (e == 0 ? lo : hi)];
-                    sm.exl[l & 1][e] = ex;
-                    const int lo_r = max(a0, e * r), hi_r = min(a1, (e + 1) * r);
+                    const ExpertDev &ex = sm.exl[l & 1][e];
+                    const int lo_r = max(a0 + per, e * r), hi_r = min(a1, (e + 1) * r);
                     if (hi_r > lo_r)
                         prefetch_l2(ex.V + size_t(lo_r - e * r) * p.vrow, uint32_t(hi_r - lo_r) * p.vrow);
-                    if (ns > 0) prefetch_l2(ex.U + size_t(s0) * p.urow, uint32_t(ns) * p.urow);
                 }
+                if (a1 <= a0) prefetch_u();
             }
+            pending = a1 > a0;
             cta_sync();
             // t rows [a0, a1) of the two experts, staged in rounds of kRA rows
-            const int per = min(kRA, kStageBytes / p.vrow);
             bool ok = true;
             for (int row0 = a0; row0 < a1 && ok; row0 += per) {
                 const int n = min(per, a1 - row0);
-                if (tid == 0) {
-                    mbar_arrive_tx(&sm.stage_bar, uint32_t(n) * p.vrow);
-                    for (int rr = 0; rr < n;) {
-                        const int row = row0 + rr, e = row / r;
-                        const int cnt = min(n - rr, (e + 1) * r - row);
-                        const uint8_t *vrow = sm.exl[l & 1][e].V + size_t(row - e * r) * p.vrow;
-                        stage_copy(stg + size_t(rr) * p.vrow, vrow, uint32_t(cnt) * p.vrow, &sm.stage_bar);
-                        rr += cnt;
-                    }
-                }
+                if (tid == 0 && row0 > a0) issue_vrows(row0, n);
                 pending = true;
                 if (!stage_wait(&sm, p, spar, bci)) { ok = false; break; }
                 pending = false;
+                if (tid == 0 && row0 == a0) prefetch_u();
                 float part[kRA];
 #pragma unroll
                 for (int rr = 0; rr < kRA; ++rr) {
@@ -858,6 +921,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 if (tid < n) {
                     float t = 0.f;
                     for (int w = 0; w < kConsumerWarps; ++w) t += sm.red[rb][w][tid];
+                    if constexpr (PF == kI8) {
+                        const int row = row0 + tid, e = row / r;
+                        t *= __ldg(sm.exl[l & 1][e].sV + (row - e * r));
+                    }
                     __stcg(p.t_buf + row0 + tid, t);
                 }
                 rb ^= 1;
@@ -954,6 +1021,63 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                                     }
                                 }
                             }
+                        }
+                    } else if constexpr (PF == kI8) {
+                        // tensor-core dots of signed-byte U rows: A from 32-bit shared loads
+                        // (bytes 4tq..4tq+3 of the step's 16-byte chunk, made f16 exactly);
+                        // the mma's logical columns 2tq, 2tq+1, 2tq+8, 2tq+9 stand for the
+                        // row elements 4tq .. 4tq+3, and B takes t's parts in the same order
+                        const int ntr = ntop * r;
+                        const int nks = r / 16, nmt = (n + 15) / 16;
+                        const int g = lane >> 2, tq = lane & 3;
+                        const uint16_t *bpart = tpart + g * ntr + e * r + 4 * tq;
+                        constexpr int kZT = MAXVW > 1 ? 4 : 6;
+                        for (int mt0 = 0; mt0 < nmt; mt0 += kZT) {
+                            float c[kZT][4];
+#pragma unroll
+                            for (int t = 0; t < kZT; ++t) c[t][0] = c[t][1] = c[t][2] = c[t][3] = 0.f;
+                            for (int ks = warp; ks < nks; ks += kConsumerWarps) {
+                                uint32_t b0 = 0u, b1 = 0u;
+                                if (g < 2) {
+                                    b0 = *reinterpret_cast<const uint32_t *>(bpart + ks * 16);
+                                    b1 = *reinterpret_cast<const uint32_t *>(bpart + ks * 16 + 2);
+                                }
+#pragma unroll
+                                for (int t = 0; t < kZT; ++t) {
+                                    if (mt0 + t < nmt) {
+                                        const int r0 = min((mt0 + t) * 16 + g, n - 1);
+                                        const int r1 = min((mt0 + t) * 16 + g + 8, n - 1);
+                                        const int k0 = p.u_swz ? (r0 & 7) : 0, k1 = p.u_swz ? (r1 & 7) : 0;
+                                        const uint32_t w0 = *reinterpret_cast<const uint32_t *>(
+                                            stg + size_t(r0) * p.urow + ((ks & ~7) | ((ks ^ k0) & 7)) * 16 + 4 * tq);
+                                        const uint32_t w1 = *reinterpret_cast<const uint32_t *>(
+                                            stg + size_t(r1) * p.urow + ((ks & ~7) | ((ks ^ k1) & 7)) * 16 + 4 * tq);
+                                        uint32_t a0, a1, a2, a3;
+                                        i8x4_to_h2(w0, a0, a2);
+                                        i8x4_to_h2(w1, a1, a3);
+                                        mma16816<kF16>(c[t], a0, a1, a2, a3, b0, b1);
+                                    }
+                                }
+                            }
+                            // the two parts sit in columns 0 and 1 (lane 4g)
+#pragma unroll
+                            for (int t = 0; t < kZT; ++t) {
+                                if (tq == 0 && mt0 + t < nmt) {
+                                    sm.zred[warp][(mt0 + t) * 16 + g] = c[t][0] + c[t][1];
+                                    sm.zred[warp][(mt0 + t) * 16 + g + 8] = c[t][2] + c[t][3];
+                                }
+                            }
+                        }
+                        cta_sync();
+                        const int nw = min(kConsumerWarps, nks);
+                        const float *su = sm.exl[l & 1][e].sU + s0 + row0;
+                        for (int rr = tid; rr < n; rr += kThreads) {
+                            float a = 0.f;
+                            for (int w = 0; w < nw; ++w) a += sm.zred[w][rr];
+                            const int loc = row0 + rr;
+                            const float z = a * __ldg(su + rr) - sm.cbuf[e][loc];
+                            sm.zbuf[e][loc] = z;
+                            if (predict && p.z_out) p.z_out[s0 + loc] = z;
                         }
                     } else {
                         // tensor-core dots: A = 16 staged U rows x 16 columns
@@ -1083,6 +1207,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         // set, so the per-CTA partials and their fixed-order reduction stay
         // deterministic.
         const ExpertDev *exs[kMaxTopK] = {&sm.exl[l & 1][0], &sm.exl[l & 1][ntop > 1 ? 1 : 0]};
+        if (p.local_gather) {
+            // each CTA gathers its own strip's active neurons (the snake-dealt
+            // table balances their expected number): no exchange, no barrier;
+            // records past the first round start moving towards L2 at once
+            const int n0 = sm.lst_n[0], nl = n0 + (ntop > 1 ? sm.lst_n[1] : 0);
+            const int cap1 = min(kRound, kStageBytes / (kSpec ? p.rec_bytes : p.gu_bytes));
+            for (int j = tid; j < nl; j += kThreads) {
+                const int en = j < n0 ? sm.lst[j] : sm.lst[kMaxStrip + (j - n0)];
+                const int e = en >> 12, loc = en & 0xfff, pos = s0 + loc;
+                sm.glst[j] = int(unsigned(e << 24) | unsigned(pos));
+                sm.gc[j] = sm.cbuf[e][loc];
+                if (j >= cap1)
+                    prefetch_l2(exs[e]->Wgu + size_t(pos) * p.rec_bytes, uint32_t(kSpec ? p.rec_bytes : p.gu_bytes));
+            }
+            if (tid == 0) sm.share_n = nl;
+            cta_sync();
+        } else {
         {
             const int n0 = sm.lst_n[0], nl = n0 + (ntop > 1 ? sm.lst_n[1] : 0);
             unsigned long long *pb = p.pub + size_t(b) * (kMaxTopK * kMaxStrip);
@@ -1136,6 +1277,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             }
             if (tid == 0) sm.share_n = hi - lo;
             cta_sync();
+        }
         }
 
         // ---------------- gather rows of active neurons ----------------------

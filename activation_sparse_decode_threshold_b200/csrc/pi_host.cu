@@ -49,11 +49,12 @@ int fmt_of(pi_dtype t)
     case PI_F16: return pi::kF16;
     case PI_BF16: return pi::kBF16;
     case PI_INT4G32: return pi::kI4;
+    case PI_I8: return pi::kI8;
     }
     return -1;
 }
 
-int elem_bytes(pi_dtype t) { return t == PI_F32 ? 4 : 2; }
+int elem_bytes(pi_dtype t) { return t == PI_F32 ? 4 : (t == PI_I8 ? 1 : 2); }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -85,6 +86,7 @@ struct pi_ffn {
     int32_t *d_strip_off = nullptr;
     int32_t *d_grp_off = nullptr;
     long long *fix = nullptr;
+    float *ssq = nullptr;
     // scratch
     uint8_t *scratch = nullptr;
     float *t_buf = nullptr, *partials = nullptr, *io = nullptr;
@@ -96,6 +98,12 @@ struct pi_ffn {
     int debug_flags = 0;
     long long *prof = nullptr;
     pi::PrefillState *prefill = nullptr;
+    // small-batch decode: workspace and row-major V per layer, made on first use
+    uint8_t *bscratch = nullptr;
+    std::vector<uint8_t *> vrm;               // [layer]
+    std::vector<char> vrm_ok;                 // [layer]
+    const uint8_t **d_vrm = nullptr;
+    int batch_fits = -1;                      // batch kernel co-resident with S CTAs (-1 unknown)
 };
 
 extern "C" {
@@ -114,20 +122,21 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
         return fail(PI_ERR_UNSUPPORTED, "F32 weights need d_model <= 4096");
     if (D.d_ff < 1) return fail(PI_ERR_INVALID_ARG, "d_ff must be >= 1");
     if (D.act < PI_ACT_RELU || D.act > PI_ACT_DRELU) return fail(PI_ERR_INVALID_ARG, "bad act");
-    if (fmt_of(D.w_dtype) < 0) return fail(PI_ERR_INVALID_ARG, "bad w_dtype");
-    if (D.pred_dtype != PI_F32 && D.pred_dtype != PI_F16 && D.pred_dtype != PI_BF16)
-        return fail(PI_ERR_INVALID_ARG, "pred_dtype must be F32, F16 or BF16");
+    if (fmt_of(D.w_dtype) < 0 || D.w_dtype == PI_I8) return fail(PI_ERR_INVALID_ARG, "bad w_dtype");
+    if (fmt_of(D.pred_dtype) < 0 || D.pred_dtype == PI_INT4G32)
+        return fail(PI_ERR_INVALID_ARG, "pred_dtype must be F32, F16, BF16 or I8");
     const bool pair_ok = (D.w_dtype == PI_F32 && D.pred_dtype == PI_F32) ||
-                         (D.w_dtype == PI_F16 && D.pred_dtype == PI_F16) ||
-                         (D.w_dtype == PI_BF16 && D.pred_dtype == PI_BF16) ||
+                         (D.w_dtype == PI_F16 && (D.pred_dtype == PI_F16 || D.pred_dtype == PI_I8)) ||
+                         (D.w_dtype == PI_BF16 && (D.pred_dtype == PI_BF16 || D.pred_dtype == PI_I8)) ||
                          (D.w_dtype == PI_INT4G32 && D.pred_dtype != PI_F32);
     if (!pair_ok)
         return fail(PI_ERR_UNSUPPORTED,
-                    "supported (w_dtype, pred_dtype): (F32,F32) (F16,F16) (BF16,BF16) "
-                    "(INT4G32,F16) (INT4G32,BF16)");
+                    "supported (w_dtype, pred_dtype): (F32,F32) (F16,F16) (BF16,BF16) (F16,I8) (BF16,I8) "
+                    "(INT4G32,F16) (INT4G32,BF16) (INT4G32,I8)");
     const int pb = elem_bytes(D.pred_dtype);
-    if (D.rank < 1 || D.rank % 16 != 0 || D.rank > 128 * (16 / pb))
-        return fail(PI_ERR_INVALID_ARG, "rank must be a multiple of 16 and <= %d", 128 * (16 / pb));
+    const int max_rank = D.pred_dtype == PI_F32 ? 512 : 1024;
+    if (D.rank < 1 || D.rank % 16 != 0 || D.rank > max_rank)
+        return fail(PI_ERR_INVALID_ARG, "rank must be a multiple of 16 and <= %d", max_rank);
     if (D.n_experts == 1) {
         if (D.top_k != 1) return fail(PI_ERR_INVALID_ARG, "a dense FFN needs top_k = 1");
     } else if (D.n_experts >= 2 && D.n_experts <= pi::kMaxExperts) {
@@ -219,7 +228,8 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
     const size_t o_bar = up256(o_pub + sizeof(unsigned long long) * size_t(h->S) * pi::kMaxTopK * pi::kMaxStrip);
     const size_t o_err = up256(o_bar + sizeof(unsigned) * pi::kBarWords);
     const size_t o_fix = o_err + 256;
-    const size_t total = up256(o_fix + sizeof(long long) * 2 * pi::kFixStride);
+    const size_t o_ssq = up256(o_fix + sizeof(long long) * 2 * pi::kFixStride);
+    const size_t total = up256(o_ssq + sizeof(float) * 2 * pi::kMaxStrips);
     cudaError_t e = cudaMalloc(&h->scratch, total);
     if (e == cudaSuccess) e = cudaMemset(h->scratch, 0, total);
     if (e == cudaSuccess) e = cudaMalloc(&h->d_ex, sizeof(pi::ExpertDev) * size_t(L) * E);
@@ -247,6 +257,7 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
     h->bar = reinterpret_cast<unsigned *>(h->scratch + o_bar);
     h->err = reinterpret_cast<int *>(h->scratch + o_err);
     h->fix = reinterpret_cast<long long *>(h->scratch + o_fix);
+    h->ssq = reinterpret_cast<float *>(h->scratch + o_ssq);
     *out = h;
     return PI_OK;
 }
@@ -262,6 +273,9 @@ void pi_ffn_destroy(pi_ffn_t h)
     cudaFree(h->d_strip_off);
     cudaFree(h->d_grp_off);
     cudaFree(h->scratch);
+    cudaFree(h->bscratch);
+    for (uint8_t *p : h->vrm) cudaFree(p);
+    cudaFree(h->d_vrm);
     pi::prefill_destroy(h->prefill);
     delete h;
 }
@@ -318,7 +332,9 @@ pi_status pi_ffn_load_layer(pi_ffn_t h, int layer, const pi_expert_weights *expe
         if (!h->gated && w.w_up) return fail(PI_ERR_INVALID_ARG, "expert %d: non-gated FFN takes no w_up", e);
         if (int4 && (!w.s_gate || !w.s_down || (h->gated && !w.s_up)))
             return fail(PI_ERR_INVALID_ARG, "expert %d: INT4 weights need scales", e);
-        const void *ptrs[] = {w.w_gate, w.w_up, w.w_down, w.s_gate, w.s_up, w.s_down, w.U, w.V};
+        if (D.pred_dtype == PI_I8 && (!w.s_U || !w.s_V))
+            return fail(PI_ERR_INVALID_ARG, "expert %d: an I8 predictor needs s_U and s_V", e);
+        const void *ptrs[] = {w.w_gate, w.w_up, w.w_down, w.s_gate, w.s_up, w.s_down, w.U, w.V, w.s_U, w.s_V};
         for (const void *q : ptrs)
             if (q && !aligned16(q))
                 return fail(PI_ERR_INVALID_ARG, "expert %d: weight pointers must be 16-byte aligned", e);
@@ -342,7 +358,10 @@ pi_status pi_ffn_load_layer(pi_ffn_t h, int layer, const pi_expert_weights *expe
     const size_t o_c = up256(o_U + size_t(F) * h->urow);
     const size_t o_g = up256(o_c + sizeof(float) * F);
     const size_t o_d = up256(o_g + size_t(F) * rec_bytes);
-    const size_t total = spec ? o_d : up256(o_d + size_t(F) * h->wrow);
+    const size_t o_s = spec ? o_d : up256(o_d + size_t(F) * h->wrow);   // I8 predictor scales
+    const bool i8 = D.pred_dtype == PI_I8;
+    const size_t o_sV = up256(o_s + (i8 ? sizeof(float) * F : 0));
+    const size_t total = i8 ? up256(o_sV + sizeof(float) * r) : o_s;
     int32_t *d_perm = nullptr;
     PI_CUDA(cudaMallocAsync(&d_perm, sizeof(int32_t) * F, st), "cudaMallocAsync(perm)");
     for (int e = 0; e < E; ++e) {
@@ -367,6 +386,10 @@ pi_status pi_ffn_load_layer(pi_ffn_t h, int layer, const pi_expert_weights *expe
             PI_CUDA(pi::repack_rows(m + o_U, d_perm, F, 1, src, rb, st), "repack U");
         }
         PI_CUDA(pi::repack_bias(w.bias, reinterpret_cast<float *>(m + o_c), d_perm, F, st), "repack c");
+        if (i8) {
+            PI_CUDA(pi::repack_bias(w.s_U, reinterpret_cast<float *>(m + o_s), d_perm, F, st), "repack U scales");
+            PI_CUDA(cudaMemcpyAsync(m + o_sV, w.s_V, sizeof(float) * r, cudaMemcpyDeviceToDevice, st), "copy V scales");
+        }
         const uint8_t *g8 = static_cast<const uint8_t *>(w.w_gate);
         const uint8_t *u8 = static_cast<const uint8_t *>(w.w_up);
         if (int4) {
@@ -400,6 +423,8 @@ pi_status pi_ffn_load_layer(pi_ffn_t h, int layer, const pi_expert_weights *expe
         x.c = reinterpret_cast<const float *>(m + o_c);
         x.Wgu = m + o_g;
         x.Wd = spec ? m + o_g + gu_bytes : m + o_d;
+        x.sU = i8 ? reinterpret_cast<const float *>(m + o_s) : nullptr;
+        x.sV = i8 ? reinterpret_cast<const float *>(m + o_sV) : nullptr;
         // the table is reused for the next expert: finish this one first
         PI_CUDA(cudaStreamSynchronize(st), "load_layer sync");
     }
@@ -418,6 +443,7 @@ pi_status pi_ffn_load_layer(pi_ffn_t h, int layer, const pi_expert_weights *expe
     PI_CUDA(cudaStreamSynchronize(st), "load_layer sync");
     h->loaded[layer] = 1;
     if (h->prefill) pi::prefill_invalidate(h->prefill, layer);
+    if (!h->vrm_ok.empty()) h->vrm_ok[layer] = 0;
     return PI_OK;
 }
 
@@ -441,6 +467,7 @@ static pi::DecodeParams base_params(pi_ffn_t h)
     p.strip_off = h->d_strip_off;
     p.grp_off = h->d_grp_off;
     p.fix = h->fix;
+    p.ssq = h->ssq;
     p.d = D.d_model;
     p.F = D.d_ff;
     p.r = D.rank;
@@ -468,6 +495,7 @@ static pi::DecodeParams base_params(pi_ffn_t h)
     p.err = h->err;
     p.wait_ns = h->wait_ns;
     p.debug_flags = h->debug_flags;
+    p.local_gather = (h->debug_flags & 4) ? 1 : 0;
     p.prof = h->prof;
     return p;
 }
@@ -528,6 +556,107 @@ pi_status pi_sparse_ffn_decode(pi_ffn_t h, int layer_begin, int layer_end, float
         PI_CUDA(cudaMemsetAsync(mask_dev, 0, sizeof(uint32_t) * size_t(nl) * D.top_k * ((D.d_ff + 31) / 32), st),
                 "memset masks");
     PI_CUDA(pi::launch_decode(h->wfmt, h->pfmt, p, st), "launch decode");
+    return PI_OK;
+}
+
+pi_status pi_sparse_ffn_decode_batch(pi_ffn_t h, int layer_begin, int layer_end, int n_tokens,
+                                     float *resid_dev, float *trace_dev, int32_t *stats_dev,
+                                     uint32_t *mask_dev, void *stream)
+{
+    if (!h || !resid_dev) return fail(PI_ERR_INVALID_ARG, "pi_sparse_ffn_decode_batch: null argument");
+    const pi_ffn_desc &D = h->desc;
+    if (layer_begin < 0 || layer_end > D.n_layers || layer_begin >= layer_end)
+        return fail(PI_ERR_INVALID_ARG, "layer range [%d, %d) invalid for %d layers", layer_begin,
+                    layer_end, D.n_layers);
+    if (n_tokens < 1 || n_tokens > 4 * pi::batch_max_tokens())
+        return fail(PI_ERR_INVALID_ARG, "n_tokens must be in [1, %d]", 4 * pi::batch_max_tokens());
+    for (int l = layer_begin; l < layer_end; ++l)
+        if (!h->loaded[l]) return fail(PI_ERR_NOT_LOADED, "layer %d not loaded", l);
+    if (!aligned16(resid_dev) || (trace_dev && !aligned16(trace_dev)))
+        return fail(PI_ERR_INVALID_ARG, "resid_dev and trace_dev must be 16-byte aligned");
+    if (D.n_experts != 1) return fail(PI_ERR_UNSUPPORTED, "small-batch decode takes dense FFN layers");
+    if (!((D.w_dtype == PI_F16 && D.pred_dtype == PI_F16) || (D.w_dtype == PI_BF16 && D.pred_dtype == PI_BF16)))
+        return fail(PI_ERR_UNSUPPORTED, "small-batch decode takes F16 or BF16 weights with a predictor of the same format");
+    if (D.d_model > pi::batch_max_d())
+        return fail(PI_ERR_UNSUPPORTED, "small-batch decode takes d_model <= %d", pi::batch_max_d());
+    if ((D.d_model / 8 + h->S - 1) / h->S * 8 > 256)
+        return fail(PI_ERR_UNSUPPORTED, "small-batch decode needs d_model / n_strips <= 256 columns");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    PI_CUDA(cudaSetDevice(D.device), "cudaSetDevice");
+    if (h->batch_fits < 0) {   // co-residency of the batch kernel, checked once per handle
+        int nsm = 0;
+        PI_CUDA(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, D.device), "cudaDeviceGetAttribute");
+        const int per_sm = pi::batch_max_blocks_per_sm(h->wfmt);
+        h->batch_fits = per_sm >= 1 && h->S <= per_sm * nsm ? 1 : 0;
+    }
+    if (!h->batch_fits)
+        return fail(PI_ERR_UNSUPPORTED, "small-batch kernel: %d strips exceed co-resident CTAs", h->S);
+    const int L = D.n_layers, S = h->S, d = D.d_model, r = D.rank, nbmax = pi::batch_max_tokens();
+    const int tpl = pi::batch_tokens_per_launch(h->wfmt);
+    // workspace: t [8 r] | ss [S 8] | partials [S 8 d] | counts [S] | pub [S kMaxStrip] | bar
+    const size_t o_t = 0;
+    const size_t o_ss = up256(o_t + sizeof(float) * size_t(nbmax) * r);
+    const size_t o_part = up256(o_ss + sizeof(float) * size_t(S) * 8);
+    const size_t o_cnt = up256(o_part + sizeof(float) * size_t(S) * nbmax * d);
+    const size_t o_pub = up256(o_cnt + sizeof(int32_t) * S);
+    const size_t o_bar = up256(o_pub + sizeof(unsigned long long) * size_t(S) * pi::kMaxStrip);
+    const size_t total = up256(o_bar + sizeof(unsigned) * pi::kBarWords);
+    if (!h->bscratch) {
+        PI_CUDA(cudaMalloc(&h->bscratch, total), "cudaMalloc(batch workspace)");
+        PI_CUDA(cudaMemset(h->bscratch, 0, total), "memset(batch workspace)");
+        h->vrm.assign(L, nullptr);
+        h->vrm_ok.assign(L, 0);
+        PI_CUDA(cudaMalloc(&h->d_vrm, sizeof(uint8_t *) * L), "cudaMalloc(V table)");
+        PI_CUDA(cudaMemset(h->d_vrm, 0, sizeof(uint8_t *) * L), "memset(V table)");
+    }
+    // row-major V of each layer of the range (made from the column blocks)
+    for (int l = layer_begin; l < layer_end; ++l) {
+        if (h->vrm_ok[l]) continue;
+        if (!h->vrm[l]) PI_CUDA(cudaMalloc(&h->vrm[l], size_t(r) * h->vrow), "cudaMalloc(V rows)");
+        PI_CUDA(pi::unblock_v(h->h_ex[l].V, h->vrm[l], h->d_grp_off, S, r, d, elem_bytes(D.pred_dtype), st),
+                "unblock V");
+        const uint8_t *vp = h->vrm[l];
+        PI_CUDA(cudaMemcpyAsync(h->d_vrm + l, &vp, sizeof(vp), cudaMemcpyHostToDevice, st), "V table");
+        PI_CUDA(cudaStreamSynchronize(st), "V rows sync");
+        h->vrm_ok[l] = 1;
+    }
+    const int nl = layer_end - layer_begin;
+    pi::BatchLaunch B{};
+    B.ex = h->d_ex;
+    B.vrm = h->d_vrm;
+    B.strip_off = h->d_strip_off;
+    B.grp_off = h->d_grp_off;
+    B.d = d; B.F = D.d_ff; B.r = r; B.act = int(D.act); B.gated = h->gated; B.S = S; B.nb = n_tokens;
+    B.layer_begin = layer_begin; B.layer_end = layer_end;
+    B.threshold = D.threshold; B.eps = D.eps;
+    B.vrow = h->vrow; B.urow = h->urow; B.wrow = h->wrow;
+    B.gu_bytes = (h->gated ? 2 : 1) * h->wrow;
+    B.spec = h->spec;
+    B.rec_bytes = B.gu_bytes + (h->spec ? h->wrow : 0);
+    B.wd_stride = h->spec ? B.rec_bytes : h->wrow;
+    B.u_swz = h->u_swz;
+    B.trace = trace_dev; B.stats = stats_dev; B.masks = mask_dev;
+    B.ntok = n_tokens;
+    B.t_buf = reinterpret_cast<float *>(h->bscratch + o_t);
+    B.ss = reinterpret_cast<float *>(h->bscratch + o_ss);
+    B.partials = reinterpret_cast<float *>(h->bscratch + o_part);
+    B.counts = reinterpret_cast<int32_t *>(h->bscratch + o_cnt);
+    B.pub = reinterpret_cast<unsigned long long *>(h->bscratch + o_pub);
+    B.bar = reinterpret_cast<unsigned *>(h->bscratch + o_bar);
+    B.err = h->err;
+    B.wait_ns = h->wait_ns;
+    if (stats_dev) PI_CUDA(cudaMemsetAsync(stats_dev, 0, sizeof(int32_t) * 4 * nl, st), "memset stats");
+    if (mask_dev)
+        PI_CUDA(cudaMemsetAsync(mask_dev, 0, sizeof(uint32_t) * size_t(nl) * n_tokens * ((D.d_ff + 31) / 32), st),
+                "memset masks");
+    // groups of up to eight (F16) or four (BF16) tokens, one launch each
+    for (int t0 = 0; t0 < n_tokens; t0 += tpl) {
+        B.tok0 = t0;
+        B.nb = std::min(tpl, n_tokens - t0);
+        B.resid = resid_dev + size_t(t0) * d;
+        PI_CUDA(cudaMemsetAsync(B.bar, 0, sizeof(unsigned) * pi::kBarWords, st), "memset barrier");
+        PI_CUDA(pi::launch_batch(h->wfmt, B, st), "launch batch decode");
+    }
     return PI_OK;
 }
 
@@ -607,6 +736,8 @@ pi_status pi_dense_ffn_prefill(pi_ffn_t h, int layer_begin, int layer_end, int n
     v.router = h->router_mem.data();
     v.perm = &h->perm;
     v.err = h->err;
+    v.wait_ns = h->wait_ns;
+    v.debug_flags = h->debug_flags;
     char msg[256] = "";
     const int rc = pi::prefill_run(&h->prefill, v, layer_begin, layer_end, n_tokens, resid_dev,
                                    static_cast<cudaStream_t>(stream), msg, sizeof msg);

@@ -18,9 +18,9 @@ constexpr int kMaxExperts = 16;
 constexpr int kMaxRankTotal = 2048;   // top_k * rank
 constexpr int kStageBytes = 200 * 1024;   // shared-memory staging of V rows / U strips / gathered rows
 constexpr int kMaxSliceCols = 1024;       // residual columns per CTA at most
-constexpr int kFixStride = kMaxRankTotal + 1 + kMaxExperts;   // t, sum r^2, logits
+constexpr int kFixStride = kMaxRankTotal + 1 + kMaxExperts;   // t, (unused), router logits
 
-enum Fmt { kF32 = 0, kF16 = 1, kBF16 = 2, kI4 = 3 };
+enum Fmt { kF32 = 0, kF16 = 1, kBF16 = 2, kI4 = 3, kI8 = 4 };   // kI8: predictor only
 
 // One expert (or dense FFN) of one layer, in table order, library-owned.
 // A neuron's input record holds its W_gate row followed by its W_up row when
@@ -36,6 +36,8 @@ struct ExpertDev {
                          // (+ the W_down row for the speculative kinds)
     const uint8_t *Wd;   // F rows of wrow bytes, wd_stride apart: W_down columns, neuron-major
                          // (inside the records for the speculative kinds)
+    const float *sU;     // 8-bit predictor: scale of each U row (table order); else null
+    const float *sV;     // 8-bit predictor: scale of each V row (r); else null
 };
 
 enum Mode { kModeDecode = 0, kModePredict = 1 };
@@ -66,6 +68,7 @@ struct DecodeParams {
     // scratch (library-owned or caller-provided, see pi_host.cu)
     float *t_buf;                   // [top_k * r]
     long long *fix;                 // [2 * kFixStride] fixed-point accumulators, zeroed
+    float *ssq;                     // [2 * kMaxStrips] per-CTA sums of squares of r, by layer parity
     float *partials;                // [S * d]
     int32_t *lists;                 // [S * kMaxStrip]  (predict)
     int32_t *counts;                // [S] active count of each strip
@@ -75,19 +78,48 @@ struct DecodeParams {
     int *err;                       // device error word (0 = ok)
     long long wait_ns;              // bound on every device-side wait
     int debug_flags;
+    int local_gather;               // each CTA gathers its own strip's active neurons (no balance step)
     long long *prof;                // [(l1-l0) * kProfPoints * S] phase timestamps, or null
 };
 
 // Phase timestamps recorded per layer and CTA when DecodeParams::prof is set.
 // layer kinds (bits of the decode kernel's MODE parameter)
 constexpr int kModeMoE = 1, kModeGated = 2, kModeSpec = 4, kModePred = 8;
-// grid barrier: arrival counters, each on its own 128-byte line
-constexpr int kBarLanes = 16, kBarStride = 32;
-constexpr int kBarWords = kBarLanes * kBarStride;
+// grid barrier: one arrival counter at word 0 of a zeroed area of kBarWords words
+constexpr int kBarWords = 512;
 constexpr int kProfPoints = 14;   // timestamps and cycle counters per layer and CTA
 
 cudaError_t launch_decode(int wfmt, int pfmt, const DecodeParams &p, cudaStream_t stream);
 int decode_max_blocks_per_sm(int wfmt, int pfmt, int d);
+
+// Small-batch decode (pi_batch.cu): up to batch_max_tokens() tokens per launch.
+struct BatchLaunch {
+    const ExpertDev *ex;                 // [n_layers]
+    const uint8_t *const *vrm;           // [n_layers] V row-major
+    const int32_t *strip_off, *grp_off;  // [S + 1]
+    int d, F, r, act, gated, S, nb;
+    int layer_begin, layer_end;
+    float threshold, eps;
+    int vrow, urow, wrow, gu_bytes, rec_bytes, wd_stride, spec, u_swz;
+    float *resid, *trace;                // resid: this launch's nb rows; trace: all ntok rows per layer
+    int32_t *stats;
+    uint32_t *masks;                     // all ntok rows per layer
+    int ntok, tok0;                      // tokens of the call, first token of this launch
+    float *t_buf, *ss, *partials;        // [nb x r], [S x 8], [S x nb x d]
+    int32_t *counts;                     // [S]
+    unsigned long long *pub;             // [S x kMaxStrip]
+    unsigned *bar;                       // [kBarWords], zeroed before launch
+    int *err;
+    long long wait_ns;
+};
+cudaError_t launch_batch(int wfmt, const BatchLaunch &L, cudaStream_t st);
+int batch_max_blocks_per_sm(int wfmt);
+int batch_max_tokens();
+int batch_tokens_per_launch(int wfmt);   // 8 (F16), 4 (BF16: x and h as two bf16 parts)
+int batch_max_d();
+// V column blocks (the dense decode layout) back to row-major.
+cudaError_t unblock_v(const uint8_t *blk, uint8_t *vrm, const int32_t *grp_off_dev, int S, int r, int d, int eb,
+                      cudaStream_t st);
 
 // Load-time repack kernels (pi_repack.cu).  repack_rows: dst record p is the
 // concatenation of row perm[p] of each of the n_src sources (row bytes each a

@@ -101,6 +101,10 @@ __global__ void k_v_blocks(const uint8_t *__restrict__ V, uint8_t *__restrict__ 
     }
     const int b = lo, g0 = grp_off[b], nb = grp_off[b + 1] - g0;
     const long long o = (long long)r * 8 * g0 + (long long)k * 8 * nb + 8LL * (g - g0);
+    if (eb == 1) {   // 8 signed bytes: one 8-byte word
+        *reinterpret_cast<uint2 *>(dst + o) = *reinterpret_cast<const uint2 *>(V + (long long)k * d + 8LL * g);
+        return;
+    }
     const uint4 *s = reinterpret_cast<const uint4 *>(V + ((long long)k * d + 8LL * g) * eb);
     uint4 *t = reinterpret_cast<uint4 *>(dst + o * eb);
     for (int i = 0; i < eb / 2; ++i) t[i] = s[i];   // 8 elements = eb/2 16-byte words

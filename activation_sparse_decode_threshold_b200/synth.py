@@ -28,6 +28,9 @@ Workload recipe (all draws from ``torch.Generator`` seeded per tensor):
   low nibble first.  This is how the synthetic INT4 model file is written;
   the hot path only ever reads it.
 * Router (MoE) ~ N(0, 0.02^2), fp16.  Token inputs ``r_t ~ N(0, 1)``, seed 99 + t.
+* 8-bit predictor (``pdtype = "i8row"``): each row of U and of V gets
+  ``s = fp32(max|w| / 127)`` and ``q = clamp(round_half_even(w / s), -127, 127)``
+  as a signed byte (an all-zero row gets s = 0, q = 0).
 """
 from __future__ import annotations
 
@@ -87,6 +90,12 @@ CONFIGS = {
     "mixtral47b": FFNConfig("turbosparse-mixtral-47b-moe8top2-drelu-32x4096x14336-int4g32", 32,
                             4096, 14336, 1024, "drelu", "int4g32", "f16", 0.10, 256,
                             n_experts=8, top_k=2, prefill_tokens=512),
+    # the same two shapes with the cheaper 8-bit per-row predictor
+    "llama7b-i8pred": FFNConfig("llama2-7b-reglu-32x4096x11008-f16-i8pred", 32, 4096, 11008, 1024,
+                                "reglu", "f16", "i8row", 0.10, 256),
+    "mixtral47b-i8pred": FFNConfig("turbosparse-mixtral-47b-moe8top2-drelu-32x4096x14336-int4g32-i8pred",
+                                   32, 4096, 14336, 1024, "drelu", "int4g32", "i8row", 0.10, 256,
+                                   n_experts=8, top_k=2, prefill_tokens=512),
 }
 
 
@@ -170,6 +179,15 @@ def quantize_int4_g32(w: torch.Tensor):
     return packed.contiguous(), s16.contiguous()
 
 
+def quantize_i8_rows(w: torch.Tensor):
+    """Rows of w (n x k) -> (signed bytes int8 n x k, fp32 scales n)."""
+    w = w.float()
+    s = (w.abs().amax(dim=1) / 127.0).float()
+    q = torch.where(s[:, None] > 0, torch.round(w / torch.where(s > 0, s, torch.ones_like(s))[:, None]),
+                    torch.zeros_like(w))
+    return q.clamp_(-127, 127).to(torch.int8).contiguous(), s.contiguous()
+
+
 # ---------------------------------------------------------------------------
 # Layers
 # ---------------------------------------------------------------------------
@@ -191,6 +209,8 @@ class ExpertWeights:
     s_gate: torch.Tensor | None = None
     s_up: torch.Tensor | None = None
     s_down: torch.Tensor | None = None
+    sU: torch.Tensor | None = None      # 8-bit predictor: fp32 scale per row of U
+    sV: torch.Tensor | None = None      # and of V
 
 
 @dataclass
@@ -217,18 +237,21 @@ def make_expert(cfg: FFNConfig, layer: int, expert: int, device="cpu",
     c = torch.from_numpy(bias_for(norms, p, shift_to).astype(np.float32)).to(device)
     # profiled frequency = firing probability under the (possibly shifted) bias
     freq = p if shift_to is None else 1.0 - _ndtr(c.cpu().double().numpy() / norms)
-    pdt = _TORCH_DT[cfg.pdtype]
+    if cfg.pdtype == "i8row":
+        Up, sU = quantize_i8_rows(U)
+        Vp, sV = quantize_i8_rows(V)
+    else:
+        pdt = _TORCH_DT[cfg.pdtype]
+        Up, Vp, sU, sV = U.to(pdt).contiguous(), V.to(pdt).contiguous(), None, None
     if cfg.wdtype == "int4g32":
         qg, sg = quantize_int4_g32(wg)
         qu, su = quantize_int4_g32(wu) if wu is not None else (None, None)
         qd, sd = quantize_int4_g32(wd.t().contiguous())
-        return ExpertWeights(qg, qu, qd, c, U.to(pdt).contiguous(), V.to(pdt).contiguous(),
-                             freq, sg, su, sd)
+        return ExpertWeights(qg, qu, qd, c, Up, Vp, freq, sg, su, sd, sU, sV)
     wdt = _TORCH_DT[cfg.wdtype]
     return ExpertWeights(wg.to(wdt).contiguous(),
                          None if wu is None else wu.to(wdt).contiguous(),
-                         wd.to(wdt).contiguous(), c, U.to(pdt).contiguous(),
-                         V.to(pdt).contiguous(), freq)
+                         wd.to(wdt).contiguous(), c, Up, Vp, freq, sU=sU, sV=sV)
 
 
 def make_layer(cfg: FFNConfig, layer: int, device="cpu", active: float | None = None) -> LayerWeights:

@@ -36,7 +36,7 @@ METRIC = "decode tok/s (FFN stack, batch 1) and achieved HBM GB/s on touched byt
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SRC = os.path.join(ROOT, "activation_sparse_decode_threshold_b200", "csrc", "pi_decode_kernel.cuh")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_dram_traffic.txt")
-PB = {"f32": 4, "f16": 2, "bf16": 2}
+PB = {"f32": 4, "f16": 2, "bf16": 2, "i8row": 1}
 
 
 def wrow_bytes(cfg) -> float:
@@ -52,6 +52,8 @@ def algorithmic_bytes(cfg, stats: np.ndarray) -> float:
     neuron, and the router for MoE."""
     pb = PB[cfg.pdtype]
     per_expert = pb * cfg.rank * (cfg.d + cfg.F) + 4 * cfg.F
+    if cfg.pdtype == "i8row":
+        per_expert += 4 * (cfg.rank + cfg.F)      # one fp32 scale per row of U and of V
     rows_in = 2 if cfg.gated else 1
     w = wrow_bytes(cfg)
     tot = 0.0
@@ -183,7 +185,8 @@ def oracle_sample_layers(cfg, n_layers: int, active):
         n = synth.to_numpy
         ex = [oracle.Expert(act=cfg.act, wdtype=cfg.wdtype, pdtype=cfg.pdtype, w_gate=n(e.w_gate),
                             w_up=n(e.w_up), w_down=n(e.w_down), c=n(e.c), U=n(e.U), V=n(e.V),
-                            s_gate=n(e.s_gate), s_up=n(e.s_up), s_down=n(e.s_down))
+                            s_gate=n(e.s_gate), s_up=n(e.s_up), s_down=n(e.s_down),
+                            sU=n(e.sU), sV=n(e.sV))
               for e in lw.experts]
         out.append((ex, None if lw.router is None else n(lw.router)))
         del lw
@@ -211,7 +214,8 @@ def cpu_baseline(cfg, active, budget_s: float = 15.0, n_layers: int = 2):
     per_token = secs / n * cfg.n_layers
     return {"value": 1.0 / per_token, "unit": "tok/s", "cores": oracle_threads(), "kind": "oracle",
             "sample": f"{n} token-layers ({n_layers} distinct layers of {cfg.n_layers}), "
-                      f"fp64 oracle, time scaled by {cfg.n_layers} layers per token"}
+                      f"fp64 oracle, time scaled by {cfg.n_layers} layers per token",
+            "projected_from": f"{n} token-layers timed, scaled to {cfg.n_layers}-layer tokens"}
 
 
 def run_reference(args, cfg, active, rank: int, world: int):
@@ -228,6 +232,8 @@ def run_reference(args, cfg, active, rank: int, world: int):
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_token * 1e3,
+        "projected_from": f"{args.steps} token-layers timed ({secs:.2f} s of oracle time), "
+                          f"each scaled by {cfg.n_layers} layers: ms_per_step is a projection",
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(cfg, active, None),
         "cpu_baseline": {"value": value, "unit": "tok/s", "cores": oracle_threads(), "kind": "oracle",
@@ -323,6 +329,101 @@ def workload_config(cfg, active, measured_active):
 
 
 # ---------------------------------------------------------------------------
+# Further workloads, each on its own handle (reported beside the headline)
+# ---------------------------------------------------------------------------
+def decode_rate(cfg, B, local: int, active, steps: int, warmup: int, h=None) -> dict:
+    """Decode tok/s and achieved GB/s of one workload: `steps` tokens timed with
+    CUDA events after `warmup`, inputs resident, clocks sampled meanwhile."""
+    own = h is None
+    if own:
+        h = build_handle(cfg, B, local, active)
+    L = cfg.n_layers
+    inputs = synth.token_inputs(cfg, steps + warmup, "cuda", 1000)
+    resid = inputs.clone()
+    stats = torch.zeros((steps + warmup, L, 4), device="cuda", dtype=torch.int32)
+    for s in range(warmup):
+        B.pi_sparse_ffn_decode(h, 0, L, resid[s], None, stats[s])
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        time.sleep(0.2)
+        for s in range(steps):
+            ev[s][0].record(stream)
+            B.pi_sparse_ffn_decode(h, 0, L, resid[warmup + s], None, stats[warmup + s])
+            ev[s][1].record(stream)
+        torch.cuda.synchronize()
+    if B.pi_sync(h) != B.PI_OK:
+        raise RuntimeError(B.pi_last_error())
+    if own:
+        B.pi_ffn_destroy(h)
+    ms = [a.elapsed_time(b) for a, b in ev]
+    st = stats[warmup:].cpu().numpy()
+    avg_bytes = float(np.mean([algorithmic_bytes(cfg, st[s]) for s in range(steps)]))
+    mean_s = float(np.mean(ms)) / 1e3
+    peak, kind = measured_peaks()
+    gbs = avg_bytes / mean_s / 1e9
+    return {"tok_s": 1.0 / mean_s, "ms_per_token": mean_s * 1e3, "achieved_gbs": gbs,
+            "roofline_frac": gbs / peak, "peak_gbs": peak, "peak_source": kind,
+            "algorithmic_bytes_per_token": avg_bytes,
+            "measured_active": float(st[:, :, 0].mean() / (cfg.F * cfg.top_k)),
+            "nonzero_h_fraction": float(st[:, :, 1].mean() / (cfg.F * cfg.top_k)),
+            "tokens_timed": steps, "warmup": warmup, "clocks": clk.summary()}
+
+
+def prefill_rate(cfg, B, local: int, h, steps: int = 3, warmup: int = 2) -> dict:
+    """Dense prefill of the workload's prompt through every layer (tcgen05)."""
+    T = cfg.prefill_tokens or 512
+    L = cfg.n_layers
+    R = synth.prefill_input(cfg, T, "cuda")
+    r = torch.empty_like(R)
+    for _ in range(warmup):
+        r.copy_(R)
+        B.pi_dense_ffn_prefill(h, 0, L, T, r)
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for s in range(steps):
+            r.copy_(R)
+            ev[s][0].record(stream)
+            B.pi_dense_ffn_prefill(h, 0, L, T, r)
+            ev[s][1].record(stream)
+        torch.cuda.synchronize()
+    if B.pi_sync(h) != B.PI_OK:
+        raise RuntimeError(B.pi_last_error())
+    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    flop = 2.0 * T * cfg.top_k * cfg.d * cfg.F * (3 if cfg.gated else 2) * L
+    peak, kind = measured_tensor_peak()
+    tf = flop / (ms / 1e3) / 1e12
+    return {"tokens": T, "ms_per_prompt": ms, "tflops": tf, "roofline_frac": tf / peak,
+            "peak_tflops": peak, "peak_source": kind, "prompts_timed": steps, "clocks": clk.summary()}
+
+
+def run_extras(B, local: int, steps: int) -> dict:
+    """The other workloads of the method's measurement plan, each on its own
+    handle: the mistral7b sparsity sweep, falcon40b, mixtral47b decode and the
+    512-token dense prefill of the mixtral47b shape."""
+    out = {}
+    m = synth.CONFIGS["mistral7b"]
+    for a in m.sweep:
+        out[f"mistral7b@active{a}"] = decode_rate(m, B, local, a, steps, 8)
+        torch.cuda.empty_cache()
+    out["falcon40b"] = decode_rate(synth.CONFIGS["falcon40b"], B, local, None, max(16, steps // 2), 8)
+    torch.cuda.empty_cache()
+    mx = synth.CONFIGS["mixtral47b"]
+    h = build_handle(mx, B, local, None)
+    try:
+        out["mixtral47b"] = decode_rate(mx, B, local, None, steps, 8, h)
+        out["mixtral47b-prefill512"] = prefill_rate(mx, B, local, h)
+    finally:
+        torch.cuda.synchronize()
+        B.pi_ffn_destroy(h)
+    torch.cuda.empty_cache()
+    return out
+
+
+# ---------------------------------------------------------------------------
 def main() -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -334,6 +435,8 @@ def main() -> int:
     ap.add_argument("--layers", type=int, default=None, help="override layer count (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other workloads (sweep, falcon40b, mixtral47b, prefill)")
     ap.add_argument("--prefill", action="store_true",
                     help="time the dense tensor-core prefill of the workload's prompt instead of decode")
     args = ap.parse_args()
@@ -438,6 +541,10 @@ def main() -> int:
     if rank != 0:
         return 0
 
+    extra = None
+    if world == 1 and not args.no_extra and not args.layers and args.config == "llama7b" and active is None:
+        extra = run_extras(B, local, 64)
+
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(cfg, active)
@@ -461,6 +568,7 @@ def main() -> int:
         "e2e": e2e,
         "gpu_launches": K,
         "clocks": clk.summary(),
+        "extra": extra,
     }
     print(json.dumps(line), flush=True)
     return 0

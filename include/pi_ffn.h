@@ -74,8 +74,12 @@ typedef enum { PI_ACT_RELU = 0, PI_ACT_REGLU = 1, PI_ACT_DRELU = 2 } pi_act;
 
 /* Stored formats.  INT4G32: symmetric 4-bit, value = s * (n - 8) with n the
  * nibble (low nibble = even element) and s one fp16 scale per 32 consecutive
- * elements of a neuron vector (a W_gate/W_up row or a W_down column). */
-typedef enum { PI_F32 = 0, PI_F16 = 1, PI_BF16 = 2, PI_INT4G32 = 3 } pi_dtype;
+ * elements of a neuron vector (a W_gate/W_up row or a W_down column).
+ * I8 (predictor only): symmetric 8-bit, value = s * q with q a signed byte and
+ * s one fp32 scale per row of U and of V -- the cheaper predictor (predictors
+ * are costly in memory: PowerInfer (unite.ai), "Adaptive sparse predictor"),
+ * half the bytes of a 16-bit one. */
+typedef enum { PI_F32 = 0, PI_F16 = 1, PI_BF16 = 2, PI_INT4G32 = 3, PI_I8 = 4 } pi_dtype;
 
 typedef struct {
     int n_layers;        /* layers in the stack, >= 1 */
@@ -88,7 +92,8 @@ typedef struct {
     int top_k;           /* 1 for a dense FFN, 2 for MoE */
     pi_act act;
     pi_dtype w_dtype;    /* F32, F16, BF16 or INT4G32 */
-    pi_dtype pred_dtype; /* F32, F16 or BF16 (F32 weights need F32 here) */
+    pi_dtype pred_dtype; /* F32, F16, BF16 or I8 (F32 weights need F32 here; I8 goes
+                            with F16, BF16 or INT4G32 weights) */
     int n_strips;        /* neuron strips per FFN = CTAs of the decode kernel;
                             0 = number of SMs of the device */
     float threshold;     /* predictor threshold, normally 0 (active iff z > threshold) */
@@ -107,12 +112,15 @@ typedef struct {
  *           INT4 matrices are F x d/2 bytes of nibbles.
  *   bias    c, F floats (the gate bias enters as -c)
  *   U       F x r row-major [pred_dtype];  V  r x d row-major [pred_dtype]
+ *   s_U, s_V  I8 predictor only: fp32 scale of each row of U (F) and of V (r);
+ *           NULL otherwise.
  */
 typedef struct {
     const void *w_gate, *w_up, *w_down;
     const void *s_gate, *s_up, *s_down;
     const float *bias;
     const void *U, *V;
+    const float *s_U, *s_V;
 } pi_expert_weights;
 
 /* Create a handle: validates `desc`, reserves per-handle scratch on
@@ -170,6 +178,37 @@ PI_API pi_status pi_sparse_ffn_decode(pi_ffn_t h, int layer_begin, int layer_end
                                float *trace_dev, int32_t *stats_dev, uint32_t *mask_dev,
                                void *stream);
 
+/* Small-batch sparse decode of layers [layer_begin, layer_end) on n_tokens
+ * independent tokens (1 <= n_tokens <= 32), one persistent launch per group
+ * of up to 8 tokens (F16 weights) or 4 tokens (BF16 weights).  The
+ * sparse path keeps its gains at small batch sizes (nearauto.com PowerInfer
+ * article, "Experiments", Fig. 14): per layer each token is normalised and
+ * predicted on its own, the rows read are those of the UNION of the tokens'
+ * predicted sets (each union neuron's W_gate / W_up / W_down rows fetched once
+ * for the batch), and token b keeps its own predicted set (h exactly 0
+ * outside it), so its output is its batch-1 output up to rounding.
+ *   resid_dev  [n_tokens x d] float, in/out (row b = token b's residual).
+ *   trace_dev  [(l1-l0) x n_tokens x d] float or NULL: each layer's input.
+ *   stats_dev  [(l1-l0) x 4] int32 or NULL: per layer {union size, sum over the
+ *              tokens of their predicted-active counts, union neurons with
+ *              h != 0 for some token, 0}; with more tokens than one launch
+ *              takes, the union figures are summed over the launches.
+ *   mask_dev   [(l1-l0) x n_tokens x ceil(F/32)] uint32 or NULL: each token's
+ *              predicted-active bits in table order.
+ * Gate/up/down products run on the tensor cores with x and h rounded to fp16
+ * for F16 weights (as in the dense prefill) and carried as two bf16 parts for
+ * BF16 weights; the predictor keeps t and x to fp32 accuracy (16-bit parts).  Deterministic.  Supported: dense FFN layers
+ * (n_experts = 1) with F16 or BF16 weights and a predictor of the same format,
+ * d_model <= 4096 and d_model / n_strips <= 256; otherwise
+ * PI_ERR_UNSUPPORTED.  The first call on a handle allocates a workspace
+ * (about n_strips x 8 x d_model x 4 bytes) and a row-major copy of each used
+ * layer's V (rank x d_model), kept until pi_ffn_destroy (a reloaded layer's
+ * copy is remade).  Errors as pi_sparse_ffn_decode, plus PI_ERR_INVALID_ARG
+ * for n_tokens outside [1, 32]. */
+PI_API pi_status pi_sparse_ffn_decode_batch(pi_ffn_t h, int layer_begin, int layer_end, int n_tokens,
+                                            float *resid_dev, float *trace_dev, int32_t *stats_dev,
+                                            uint32_t *mask_dev, void *stream);
+
 /* Same as pi_sparse_ffn_decode on HOST buffers: copies resid_in_host (d
  * floats) to the device, decodes, copies the result to resid_out_host, and
  * synchronises `stream` before returning.  Host buffers should be pinned for
@@ -206,11 +245,17 @@ PI_API const char *pi_last_error(void);
 /* Release the handle and all device memory it owns (after its work is done). */
 PI_API void pi_ffn_destroy(pi_ffn_t h);
 
-/* Testing aid: bound every device-side wait of this handle by `wait_limit_s`
- * seconds (default 2.0) and, with flags & PI_DEBUG_STALL_BARRIER, make the
- * decode kernel's first grid barrier wait for one arrival that never comes,
- * so that the bounded wait runs out and pi_sync reports PI_ERR_TIMEOUT. */
+/* Testing aid: bound every device-side wait of this handle (decode and
+ * prefill kernels) by `wait_limit_s` seconds (default 2.0).  With flags &
+ * PI_DEBUG_STALL_BARRIER, the decode kernel's first grid barrier waits for one
+ * arrival that never comes; with flags & PI_DEBUG_STALL_PREFILL, one producer
+ * thread of the first prefill gate/up GEMM tile never publishes its first
+ * stage, so the tensor-core issuer's bounded wait runs out before it issues
+ * any MMA.  Either way the wait runs out, the kernel releases what it holds
+ * (in-flight copies, tensor memory) and returns, and pi_sync reports
+ * PI_ERR_TIMEOUT; the handle stays usable. */
 #define PI_DEBUG_STALL_BARRIER 1
+#define PI_DEBUG_STALL_PREFILL 2
 PI_API pi_status pi_debug_set(pi_ffn_t h, int flags, double wait_limit_s);
 
 /* Testing aid: when `times_dev` is non-NULL, each later pi_sparse_ffn_decode
@@ -241,12 +286,16 @@ PI_API pi_status pi_debug_phase_times(pi_ffn_t h, long long *times_dev);
  * pi_ffn_desc; d_ff <= 256 * min(SM count, 256); larger sizes return
  * PI_ERR_INVALID_ARG.  Scratch: one file-scope __device__ array of about 300 KB
  * that every device loading the library holds until exit.
- * Runs on the current device.  Its first call on a device looks up the
+ * Runs on the current device, which must be one of devices 0..63 (a higher
+ * index returns PI_ERR_UNSUPPORTED).  Its first call on a device looks up the
  * array's device address (cudaGetSymbolAddress) and must come before any
- * stream capture on that device.  Every call shares the array and leaves its
+ * stream capture on that device; the address is kept for the life of the
+ * process, so cudaDeviceReset must not be called on a device after this entry
+ * point has been used there.  Every call shares the array and leaves its
  * contents behind (each call clears what must start at zero), so calls that
  * overlap on the GPU -- on two streams, or from two threads -- race and must
- * not be issued.  *count_dev reads -1 if the kernel gave up on a bounded wait.
+ * not be issued.  *count_dev reads -1 if any bounded wait of the call ran out
+ * (a second, one-thread kernel on `stream` writes it after the predictor).
  * Asynchronous on `stream`. */
 PI_API pi_status pi_predict_noalloc(int d_model, int d_ff, int rank, pi_dtype pred_dtype,
                                     float threshold, const void *V_dev, const void *U_dev,

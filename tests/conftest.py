@@ -18,3 +18,9 @@ def oracle_mod():
     import oracle
     oracle.build()
     return oracle
+
+
+def pytest_sessionfinish(session, exitstatus):
+    mod = sys.modules.get("gpu_util")
+    if mod is not None:
+        mod.write_errors()

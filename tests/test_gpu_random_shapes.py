@@ -68,7 +68,8 @@ def test_random_shape_decode(handles, act, wd, pd, d, F, rank, strips, active, E
         outs = list(trace[1:]) + [rL]
         for l in range(cfg.n_layers):
             ex, router = olayers[l]
-            G.check_layer(cfg, ex, router, perms[l], trace[l], outs[l], stats[l], masks[l])
+            G.check_layer(cfg, ex, router, perms[l], trace[l], outs[l], stats[l], masks[l],
+                          case="decode/random-shapes")
     # the dense prefill of the same layer where its shape allows it
     if wd != "f32" and d % 256 == 0 and F % 128 == 0:
         R = synth.prefill_input(cfg, 96, "cuda")
