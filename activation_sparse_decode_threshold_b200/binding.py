@@ -68,6 +68,9 @@ def lib() -> ctypes.CDLL:
             "pi_sparse_ffn_decode": [vp, ip, ip, vp, vp, vp, vp, vp],
             "pi_sparse_ffn_decode_host": [vp, ip, ip, vp, vp, vp],
             "pi_sparse_ffn_decode_batch": [vp, ip, ip, ip, vp, vp, vp, vp, vp],
+            "pi_sparse_ffn_decode_partial": [vp, ip, vp, vp, vp, vp, vp],
+            "pi_residual_add": [vp, vp, vp, vp],
+            "pi_ffn_set_hot_neurons": [vp, ip],
             "pi_dense_ffn_prefill": [vp, ip, ip, ip, vp, vp],
             "pi_sync": [vp, vp],
             "pi_debug_set": [vp, ip, ctypes.c_double],
@@ -154,6 +157,10 @@ def pi_ffn_load_layer(h, layer, experts, router=None, freq=None, stream=None):
            "pi_ffn_load_layer")
 
 
+def pi_ffn_set_hot_neurons(h, hot_per_strip: int):
+    _check(lib().pi_ffn_set_hot_neurons(h, hot_per_strip), "pi_ffn_set_hot_neurons")
+
+
 def pi_neuron_table(h, layer, expert, F):
     import numpy as np
     perm = np.empty(F, np.int32)
@@ -188,6 +195,15 @@ def pi_sparse_ffn_decode_batch(h, layer_begin, layer_end, resid, trace=None, sta
     _check(lib().pi_sparse_ffn_decode_batch(h, layer_begin, layer_end, int(resid.shape[0]), _ptr(resid),
                                             _ptr(trace), _ptr(stats), _ptr(masks), _stream(stream)),
            "pi_sparse_ffn_decode_batch")
+
+
+def pi_sparse_ffn_decode_partial(h, layer, resid, y, stats=None, masks=None, stream=None):
+    _check(lib().pi_sparse_ffn_decode_partial(h, layer, _ptr(resid), _ptr(y), _ptr(stats), _ptr(masks),
+                                              _stream(stream)), "pi_sparse_ffn_decode_partial")
+
+
+def pi_residual_add(h, resid, y, stream=None):
+    _check(lib().pi_residual_add(h, _ptr(resid), _ptr(y), _stream(stream)), "pi_residual_add")
 
 
 def pi_sparse_ffn_decode_host(h, layer_begin, layer_end, resid_in, resid_out, stream=None):

@@ -242,6 +242,12 @@ __device__ __forceinline__ void ldsm_x4(const void *p, uint32_t &r0, uint32_t &r
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                  : "r"(s2u(p)));
 }
+__device__ __forceinline__ void ldsm_x4_a(uint32_t saddr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(saddr));
+}
 // D += A (16x16, row) * B (16x8, col), 16-bit inputs of format F, fp32 accumulate.
 template <int F>
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -294,6 +300,27 @@ __device__ __forceinline__ void i8x4_to_h2(uint32_t w, uint32_t &lo, uint32_t &h
     const __half2 hb = __hsub2(*reinterpret_cast<const __half2 *>(&b), bias);
     lo = *reinterpret_cast<const uint32_t *>(&ha);
     hi = *reinterpret_cast<const uint32_t *>(&hb);
+}
+
+// Where a neuron's record lives.  Without a VRAM budget (hot_k = 0) every
+// record is in HBM at its table position.  With one, the first hot_k
+// positions of each strip stay in HBM, packed strip by strip (index
+// b * hot_k + loc), and the others live in pinned host memory, packed in
+// table order (index pos - (b + 1) * hot_k).  The code is the index, with bit
+// 23 set for a record in host memory.
+constexpr unsigned kColdBit = 1u << 23;
+__device__ __forceinline__ unsigned rec_code(int hot_k, int b, int loc, int pos)
+{
+    if (hot_k == 0) return unsigned(pos);
+    if (loc < hot_k) return unsigned(b * hot_k + loc);
+    return kColdBit | unsigned(pos - (b + 1) * hot_k);
+}
+// 16-byte pieces [lo, hi) of a record in host memory into shared memory, by
+// the calling threads (plain loads: the bytes cross the host link)
+__device__ __forceinline__ void copy_host_rec(uint8_t *dst, const uint8_t *src, int bytes, int t0, int nt)
+{
+    for (int i = t0; i < bytes / 16; i += nt)
+        reinterpret_cast<uint4 *>(dst)[i] = *reinterpret_cast<const uint4 *>(src + 16 * size_t(i));
 }
 
 __device__ __forceinline__ float act_h(int act, float g, float u)
@@ -634,9 +661,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     sacc.w += __shfl_xor_sync(0xffffffffu, sacc.w, o);
                 }
                 if (lane == 0) {
-                    rv.x += sacc.x; rv.y += sacc.y; rv.z += sacc.z; rv.w += sacc.w;
-                    __stcg(reinterpret_cast<float4 *>(p.resid) + q, rv);
-                    *reinterpret_cast<float4 *>(sm.rsl + 4 * qq) = rv;
+                    if (p.y_out) {
+                        // one-layer call on a shard of the neurons: this shard's y,
+                        // the residual left as it is (the caller sums the shards)
+                        __stcg(reinterpret_cast<float4 *>(p.y_out) + q, sacc);
+                    } else {
+                        rv.x += sacc.x; rv.y += sacc.y; rv.z += sacc.z; rv.w += sacc.w;
+                        __stcg(reinterpret_cast<float4 *>(p.resid) + q, rv);
+                        *reinterpret_cast<float4 *>(sm.rsl + 4 * qq) = rv;
+                    }
                 }
             }
         } else {
@@ -884,6 +917,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             }
             pending = a1 > a0;
             cta_sync();
+            prof_put(p, li, 18, gtimer());
             // t rows [a0, a1) of the two experts, staged in rounds of kRA rows
             bool ok = true;
             for (int row0 = a0; row0 < a1 && ok; row0 += per) {
@@ -892,6 +926,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 pending = true;
                 if (!stage_wait(&sm, p, spar, bci)) { ok = false; break; }
                 pending = false;
+                if (row0 == a0) prof_put(p, li, 19, gtimer());
                 if (tid == 0 && row0 == a0) prefetch_u();
                 float part[kRA];
 #pragma unroll
@@ -930,12 +965,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 rb ^= 1;
             }
             if (!ok) break;
+            prof_put(p, li, 20, gtimer());
             // round 0 of the first expert's U strip lands during the barrier
             // (issued after the arrival, whose release would wait for it)
             grid_arrive(p, epoch);
             if (warp == 0 && ns > 0) stage_u(sm.exl[l & 1][0], 0, min(ns, ucap));
             staged_early = pending = ns > 0;
             if (!grid_wait(&sm, p, epoch, bci, &cyc_bar)) break;
+            prof_put(p, li, 21, gtimer());
             for (int k = tid; k < ntop * r; k += kThreads) put_t(k, __ldcg(p.t_buf + k), ntop * r);
         }
         if constexpr (moe) {
@@ -976,6 +1013,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     pending = true;
                     if (!stage_wait(&sm, p, spar, bci, &cyc_b)) { ok = false; break; }
                     pending = false;
+                    if (e == 0 && row0 == 0) prof_put(p, li, 14, gtimer());
                     if constexpr (PF == kF32) {
                         // each warp takes rows warp, warp + 16, ...; four rows at a time,
                         // each with its own accumulators, to keep the dependent FMA and
@@ -1042,19 +1080,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                                     b0 = *reinterpret_cast<const uint32_t *>(bpart + ks * 16);
                                     b1 = *reinterpret_cast<const uint32_t *>(bpart + ks * 16 + 2);
                                 }
+                                // every shared load of the step first, then conversions and MMAs
+                                uint32_t w[kZT][2];
 #pragma unroll
                                 for (int t = 0; t < kZT; ++t) {
                                     if (mt0 + t < nmt) {
                                         const int r0 = min((mt0 + t) * 16 + g, n - 1);
                                         const int r1 = min((mt0 + t) * 16 + g + 8, n - 1);
                                         const int k0 = p.u_swz ? (r0 & 7) : 0, k1 = p.u_swz ? (r1 & 7) : 0;
-                                        const uint32_t w0 = *reinterpret_cast<const uint32_t *>(
+                                        w[t][0] = *reinterpret_cast<const uint32_t *>(
                                             stg + size_t(r0) * p.urow + ((ks & ~7) | ((ks ^ k0) & 7)) * 16 + 4 * tq);
-                                        const uint32_t w1 = *reinterpret_cast<const uint32_t *>(
+                                        w[t][1] = *reinterpret_cast<const uint32_t *>(
                                             stg + size_t(r1) * p.urow + ((ks & ~7) | ((ks ^ k1) & 7)) * 16 + 4 * tq);
+                                    }
+                                }
+#pragma unroll
+                                for (int t = 0; t < kZT; ++t) {
+                                    if (mt0 + t < nmt) {
                                         uint32_t a0, a1, a2, a3;
-                                        i8x4_to_h2(w0, a0, a2);
-                                        i8x4_to_h2(w1, a1, a3);
+                                        i8x4_to_h2(w[t][0], a0, a2);
+                                        i8x4_to_h2(w[t][1], a1, a3);
                                         mma16816<kF16>(c[t], a0, a1, a2, a3, b0, b1);
                                     }
                                 }
@@ -1072,8 +1117,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                         const int nw = min(kConsumerWarps, nks);
                         const float *su = sm.exl[l & 1][e].sU + s0 + row0;
                         for (int rr = tid; rr < n; rr += kThreads) {
-                            float a = 0.f;
-                            for (int w = 0; w < nw; ++w) a += sm.zred[w][rr];
+                            float q[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                            for (int w = 0; w < kConsumerWarps; ++w)
+                                if (w < nw) q[w & 3] += sm.zred[w][rr];
+                            const float a = (q[0] + q[1]) + (q[2] + q[3]);
                             const int loc = row0 + rr;
                             const float z = a * __ldg(su + rr) - sm.cbuf[e][loc];
                             sm.zbuf[e][loc] = z;
@@ -1098,6 +1146,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                             float c[kZT][4];
 #pragma unroll
                             for (int t = 0; t < kZT; ++t) c[t][0] = c[t][1] = c[t][2] = c[t][3] = 0.f;
+                            // this lane's row in each m-tile (rows past the round's last are
+                            // read as its last row; their results are never used); its chunk
+                            // permutation key is the staged row mod 8 (rounds start at
+                            // multiples of 8)
+                            int arw[kZT];
+#pragma unroll
+                            for (int t = 0; t < kZT; ++t) arw[t] = min((mt0 + t) * 16 + arow, n - 1);
+                            const uint32_t sbase = s2u(stg);
                             for (int ks = warp; ks < nks; ks += kConsumerWarps) {
                                 uint32_t b0 = 0u, b1 = 0u;
                                 if (g < nparts) {
@@ -1105,19 +1161,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                                     b1 = *reinterpret_cast<const uint32_t *>(bpart + ks * 16 + 8);
                                 }
                                 const int chunk = 2 * ks + (lane >> 4);            // 16-byte chunk of the row
+                                // the matrix loads of three m-tiles first, then their MMAs,
+                                // so that the loads' latencies overlap
 #pragma unroll
-                                for (int t = 0; t < kZT; ++t) {
-                                    if (mt0 + t < nmt) {
-                                        // rows past the round's last are read as its last row
-                                        // (their results are never used); the chunk permutation
-                                        // key is the staged row mod 8 (rounds start at multiples of 8)
-                                        const int row = min((mt0 + t) * 16 + arow, n - 1);
-                                        const int key = p.u_swz ? (row & 7) : 0;
-                                        uint32_t a0, a1, a2, a3;
-                                        ldsm_x4(stg + size_t(row) * p.urow + ((chunk & ~7) | ((chunk ^ key) & 7)) * 16,
-                                                a0, a1, a2, a3);
-                                        mma16816<PF>(c[t], a0, a1, a2, a3, b0, b1);
+                                for (int t0 = 0; t0 < kZT; t0 += 3) {
+                                    uint32_t a[3][4];
+#pragma unroll
+                                    for (int t = t0; t < t0 + 3; ++t) {
+                                        if (t < kZT && mt0 + t < nmt) {
+                                            const int key = p.u_swz ? (arw[t] & 7) : 0;
+                                            ldsm_x4_a(sbase + uint32_t(arw[t]) * uint32_t(p.urow) +
+                                                          uint32_t(((chunk & ~7) | ((chunk ^ key) & 7)) << 4),
+                                                      a[t - t0]);
+                                        }
                                     }
+#pragma unroll
+                                    for (int t = t0; t < t0 + 3; ++t)
+                                        if (t < kZT && mt0 + t < nmt)
+                                            mma16816<PF>(c[t], a[t - t0][0], a[t - t0][1], a[t - t0][2], a[t - t0][3], b0, b1);
                                 }
                             }
                             // sum over the parts: columns 0 and 1 sit in lane 4g, column 2 in lane 4g + 1
@@ -1135,11 +1196,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                             }
                         }
                         cta_sync();
-                        // across warps in fixed order
+                        if (e == 0 && row0 == 0) prof_put(p, li, 15, gtimer());
+                        // across warps in fixed order: four interleaved partial sums
+                        // (warps w, w + 4, ...), then those four in order
                         const int nw = min(kConsumerWarps, nks);
                         for (int rr = tid; rr < n; rr += kThreads) {
-                            float a = 0.f;
-                            for (int w = 0; w < nw; ++w) a += sm.zred[w][rr];
+                            float q[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                            for (int w = 0; w < kConsumerWarps; ++w)
+                                if (w < nw) q[w & 3] += sm.zred[w][rr];
+                            const float a = (q[0] + q[1]) + (q[2] + q[3]);
                             const int loc = row0 + rr;
                             const float z = a - sm.cbuf[e][loc];
                             sm.zbuf[e][loc] = z;
@@ -1216,10 +1282,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             for (int j = tid; j < nl; j += kThreads) {
                 const int en = j < n0 ? sm.lst[j] : sm.lst[kMaxStrip + (j - n0)];
                 const int e = en >> 12, loc = en & 0xfff, pos = s0 + loc;
-                sm.glst[j] = int(unsigned(e << 24) | unsigned(pos));
+                const unsigned code = rec_code(p.hot_k, b, loc, pos);
+                sm.glst[j] = int(unsigned(e << 24) | code);
                 sm.gc[j] = sm.cbuf[e][loc];
-                if (j >= cap1)
-                    prefetch_l2(exs[e]->Wgu + size_t(pos) * p.rec_bytes, uint32_t(kSpec ? p.rec_bytes : p.gu_bytes));
+                if (j >= cap1 && !(code & kColdBit))
+                    prefetch_l2(exs[e]->Wgu + size_t(code) * p.rec_bytes, uint32_t(kSpec ? p.rec_bytes : p.gu_bytes));
             }
             if (tid == 0) sm.share_n = nl;
             cta_sync();
@@ -1230,7 +1297,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             for (int j = tid; j < nl; j += kThreads) {
                 const int en = j < n0 ? sm.lst[j] : sm.lst[kMaxStrip + (j - n0)];
                 const int e = en >> 12, loc = en & 0xfff, pos = s0 + loc;
-                __stcg(pb + j, (unsigned long long)(unsigned(e << 24) | unsigned(pos)) |
+                __stcg(pb + j, (unsigned long long)(unsigned(e << 24) | rec_code(p.hot_k, b, loc, pos)) |
                                    ((unsigned long long)__float_as_uint(sm.cbuf[e][loc]) << 32));
             }
             if (tid == 0) __stcg(p.counts + b, nl);
@@ -1239,11 +1306,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             grid_arrive(p, epoch);
             for (int j = tid; j < nl; j += kThreads) {
                 const int en = j < n0 ? sm.lst[j] : sm.lst[kMaxStrip + (j - n0)];
-                const int e = en >> 12, pos = s0 + (en & 0xfff);
-                prefetch_l2(exs[e]->Wgu + size_t(pos) * p.rec_bytes, uint32_t(kSpec ? p.rec_bytes : p.gu_bytes));
+                const int e = en >> 12, loc = en & 0xfff;
+                const unsigned code = rec_code(p.hot_k, b, loc, s0 + loc);
+                if (!(code & kColdBit))
+                    prefetch_l2(exs[e]->Wgu + size_t(code) * p.rec_bytes, uint32_t(kSpec ? p.rec_bytes : p.gu_bytes));
             }
         }
         if (!grid_wait(&sm, p, epoch, bci, &cyc_bar)) break;
+        prof_put(p, li, 16, gtimer());
         {
             // exclusive prefix of the strip counts (S <= 256: warps 0..7)
             const int cnt = tid < S ? __ldcg(p.counts + tid) : 0;
@@ -1341,16 +1411,31 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             const int k = min(cap_n, m - j0);
             const int ngr = (k + 3) / 4;   // groups of four neurons, one barrier each
             if (warp == 0) {
-                // lane 0 announces each group's bytes, then lane n copies neuron n
-                // onto its group's barrier
-                if (lane < ngr) mbar_arrive_tx(&sm.gbar[lane], uint32_t(min(4, k - 4 * lane)) * per_n);
+                // lane 0 announces each group's bytes (records in HBM only), then
+                // lane n copies neuron n onto its group's barrier
+                const int en_l = lane < k ? sm.glst[j0 + lane] : 0;
+                const bool hot_l = lane < k && !(unsigned(en_l) & kColdBit);
+                const unsigned hot_m = __ballot_sync(0xffffffffu, hot_l);
+                if (lane < ngr) mbar_arrive_tx(&sm.gbar[lane], uint32_t(__popc((hot_m >> (4 * lane)) & 0xfu)) * per_n);
                 __syncwarp();
-                if (lane < k) {
-                    const int en = sm.glst[j0 + lane], e = en >> 24, pos = en & 0xffffff;
+                if (hot_l) {
+                    const int e = en_l >> 24;
+                    const unsigned code = unsigned(en_l) & 0xffffffu;
                     uint8_t *slot = stg + size_t(lane) * per_n;
                     uint64_t *gb = &sm.gbar[lane >> 2];
-                    stage_copy(slot, exs[e]->Wgu + size_t(pos) * p.rec_bytes, uint32_t(per_n), gb);
+                    stage_copy(slot, exs[e]->Wgu + size_t(code) * p.rec_bytes, uint32_t(per_n), gb);
                 }
+            }
+            if (p.hot_k) {
+                // records in host memory: every thread copies pieces of them
+                for (int n = 0; n < k; ++n) {
+                    const int en = sm.glst[j0 + n];
+                    if (!(unsigned(en) & kColdBit)) continue;
+                    const unsigned idx = unsigned(en) & (kColdBit - 1u);
+                    copy_host_rec(stg + size_t(n) * per_n, exs[en >> 24]->Wgu_cold + size_t(idx) * p.rec_bytes, per_n,
+                                  tid, kThreads);
+                }
+                cta_sync();
             }
             gpend = (1u << ngr) - 1u;
             // dots of the round's neurons, four at a time as each group lands:
@@ -1372,6 +1457,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                         }
                     }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (j0 == 0 && g0 == 0 && warp == 0) prof_put(p, li, 17, gtimer());
                     if (!ok) {
                         if (lane == 0) {
                             set_error(p.err, kDevTimeout);
@@ -1469,13 +1555,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             for (int q0 = 0; q0 < nz_total && gok; q0 += cap_d) {
                 const int k = min(cap_d, nz_total - q0);
                 if (warp == 0) {
-                    if (lane == 0) mbar_arrive_tx(&sm.stage_bar, uint32_t(k) * p.wrow);
+                    int nhot = 0;
+                    for (int n = lane; n < k; n += 32)
+                        nhot += (unsigned(sm.nz[q0 + n]) & kColdBit) ? 0 : 1;
+                    nhot = __reduce_add_sync(0xffffffffu, nhot);
+                    if (lane == 0) mbar_arrive_tx(&sm.stage_bar, uint32_t(nhot) * p.wrow);
                     __syncwarp();
                     for (int n = lane; n < k; n += 32) {
-                        const int en = sm.nz[q0 + n], e = en >> 24, pos = en & 0xffffff;
-                        stage_copy(stg + size_t(n) * p.wrow, exs[e]->Wd + size_t(pos) * p.wd_stride,
+                        const int en = sm.nz[q0 + n], e = en >> 24;
+                        if (unsigned(en) & kColdBit) continue;
+                        const unsigned code = unsigned(en) & 0xffffffu;
+                        stage_copy(stg + size_t(n) * p.wrow, exs[e]->Wd + size_t(code) * p.wd_stride,
                                    uint32_t(p.wrow), &sm.stage_bar);
                     }
+                }
+                if (p.hot_k) {
+                    for (int n = 0; n < k; ++n) {
+                        const int en = sm.nz[q0 + n];
+                        if (!(unsigned(en) & kColdBit)) continue;
+                        const unsigned idx = unsigned(en) & (kColdBit - 1u);
+                        copy_host_rec(stg + size_t(n) * p.wrow, exs[en >> 24]->Wd_cold + size_t(idx) * p.wd_stride,
+                                      p.wrow, tid, kThreads);
+                    }
+                    cta_sync();
                 }
                 pending = true;
                 if (!stage_wait(&sm, p, spar, bci, &cyc_c)) { gok = false; break; }

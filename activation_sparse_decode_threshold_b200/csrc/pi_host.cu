@@ -104,6 +104,8 @@ struct pi_ffn {
     std::vector<char> vrm_ok;                 // [layer]
     const uint8_t **d_vrm = nullptr;
     int batch_fits = -1;                      // batch kernel co-resident with S CTAs (-1 unknown)
+    int hot_k = 0;                            // records kept in HBM per strip (0 = all)
+    std::vector<uint8_t *> host_mem;          // [layer * E + e] pinned cold records
 };
 
 extern "C" {
@@ -214,6 +216,7 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
     const int L = D.n_layers, E = D.n_experts;
     h->perm.assign(size_t(L) * E, {});
     h->mem.assign(size_t(L) * E, nullptr);
+    h->host_mem.assign(size_t(L) * E, nullptr);
     h->router_mem.assign(L, nullptr);
     h->loaded.assign(L, 0);
     h->h_ex.assign(size_t(L) * E, pi::ExpertDev{});
@@ -267,6 +270,7 @@ void pi_ffn_destroy(pi_ffn_t h)
     if (!h) return;
     cudaSetDevice(h->desc.device);
     for (uint8_t *p : h->mem) cudaFree(p);
+    for (uint8_t *p : h->host_mem) cudaFreeHost(p);
     for (uint8_t *p : h->router_mem) cudaFree(p);
     cudaFree(h->d_ex);
     cudaFree(h->d_router);
@@ -353,23 +357,36 @@ pi_status pi_ffn_load_layer(pi_ffn_t h, int layer, const pi_expert_weights *expe
     const int gu_bytes = (h->gated ? 2 : 1) * h->wrow;
     const bool spec = h->spec;
     const int rec_bytes = gu_bytes + (spec ? h->wrow : 0);
+    // with a VRAM budget the layer memory keeps S * hot_k records (and down
+    // rows); the rest go to pinned host memory (see pi_ffn_set_hot_neurons)
+    const int hk = h->hot_k;
+    const size_t n_dev = hk ? size_t(h->S) * hk : size_t(F);
+    const size_t n_host = size_t(F) - n_dev;
     const size_t o_V = 0;
     const size_t o_U = up256(o_V + size_t(r) * h->vrow);
     const size_t o_c = up256(o_U + size_t(F) * h->urow);
     const size_t o_g = up256(o_c + sizeof(float) * F);
-    const size_t o_d = up256(o_g + size_t(F) * rec_bytes);
-    const size_t o_s = spec ? o_d : up256(o_d + size_t(F) * h->wrow);   // I8 predictor scales
+    const size_t o_d = up256(o_g + n_dev * rec_bytes);
+    const size_t o_s = spec ? o_d : up256(o_d + n_dev * h->wrow);   // I8 predictor scales
     const bool i8 = D.pred_dtype == PI_I8;
     const size_t o_sV = up256(o_s + (i8 ? sizeof(float) * F : 0));
     const size_t total = i8 ? up256(o_sV + sizeof(float) * r) : o_s;
     int32_t *d_perm = nullptr;
     PI_CUDA(cudaMallocAsync(&d_perm, sizeof(int32_t) * F, st), "cudaMallocAsync(perm)");
+    // every record (and down row) in table order, split afterwards when budgeted
+    uint8_t *full_g = nullptr, *full_d = nullptr;
+    if (hk) {
+        PI_CUDA(cudaMallocAsync(&full_g, size_t(F) * rec_bytes, st), "cudaMallocAsync(records)");
+        if (!spec) PI_CUDA(cudaMallocAsync(&full_d, size_t(F) * h->wrow, st), "cudaMallocAsync(down rows)");
+    }
     for (int e = 0; e < E; ++e) {
         const size_t idx = size_t(layer) * E + e;
         const pi_expert_weights &w = experts[e];
         build_table(freq_host ? freq_host + size_t(e) * F : nullptr, F, h->strip_off, h->perm[idx]);
         if (!h->mem[idx]) PI_CUDA(cudaMalloc(&h->mem[idx], total), "cudaMalloc(layer)");
         uint8_t *m = h->mem[idx];
+        uint8_t *rec_dst = hk ? full_g : m + o_g;
+        uint8_t *down_dst = hk ? full_d : m + o_d;
         PI_CUDA(cudaMemcpyAsync(d_perm, h->perm[idx].data(), sizeof(int32_t) * F,
                                 cudaMemcpyHostToDevice, st), "copy perm");
         if (E == 1)   // dense: column blocks, one per strip (see pi_decode.cu)
@@ -403,17 +420,17 @@ pi_status pi_ffn_load_layer(pi_ffn_t h, int layer, const pi_expert_weights *expe
             if (spec) {
                 // gate (, up), down in one record
                 const uint8_t *rs[6] = {g8, sg8, h->gated ? u8 : qd8, h->gated ? su8 : sd8, qd8, sd8};
-                PI_CUDA(pi::repack_rows(m + o_g, d_perm, F, h->gated ? 6 : 4, rs, rb, st), "repack records");
+                PI_CUDA(pi::repack_rows(rec_dst, d_perm, F, h->gated ? 6 : 4, rs, rb, st), "repack records");
             } else {
-                PI_CUDA(pi::repack_rows(m + o_g, d_perm, F, h->gated ? 4 : 2, src, rb, st), "repack gate/up");
-                PI_CUDA(pi::repack_rows(m + o_d, d_perm, F, 2, src + 4, rb + 4, st), "repack down");
+                PI_CUDA(pi::repack_rows(rec_dst, d_perm, F, h->gated ? 4 : 2, src, rb, st), "repack gate/up");
+                PI_CUDA(pi::repack_rows(down_dst, d_perm, F, 2, src + 4, rb + 4, st), "repack down");
             }
         } else {
             const uint8_t *src[2] = {g8, u8};
             const int rb[2] = {h->wrow, h->wrow};
-            PI_CUDA(pi::repack_rows(m + o_g, d_perm, F, h->gated ? 2 : 1, src, rb, st, rec_bytes),
+            PI_CUDA(pi::repack_rows(rec_dst, d_perm, F, h->gated ? 2 : 1, src, rb, st, rec_bytes),
                     "repack gate/up");
-            PI_CUDA(pi::repack_down_transpose(static_cast<const uint8_t *>(w.w_down), spec ? m + o_g + gu_bytes : m + o_d,
+            PI_CUDA(pi::repack_down_transpose(static_cast<const uint8_t *>(w.w_down), spec ? rec_dst + gu_bytes : down_dst,
                                               d_perm, d, F, elem_bytes(D.w_dtype), st, spec ? rec_bytes : 0),
                     "transpose down");
         }
@@ -423,12 +440,34 @@ pi_status pi_ffn_load_layer(pi_ffn_t h, int layer, const pi_expert_weights *expe
         x.c = reinterpret_cast<const float *>(m + o_c);
         x.Wgu = m + o_g;
         x.Wd = spec ? m + o_g + gu_bytes : m + o_d;
+        x.Wgu_cold = nullptr;
+        x.Wd_cold = nullptr;
+        if (hk) {
+            // hot records to the layer memory, the rest to pinned host memory
+            const size_t host_bytes = n_host * (rec_bytes + (spec ? 0 : h->wrow));
+            if (!h->host_mem[idx] && host_bytes > 0)
+                PI_CUDA(cudaHostAlloc(reinterpret_cast<void **>(&h->host_mem[idx]), host_bytes, cudaHostAllocMapped),
+                        "cudaHostAlloc(cold records)");
+            uint8_t *hdev = nullptr;
+            if (host_bytes > 0)
+                PI_CUDA(cudaHostGetDevicePointer(reinterpret_cast<void **>(&hdev), h->host_mem[idx], 0),
+                        "cudaHostGetDevicePointer");
+            PI_CUDA(pi::split_records(full_g, m + o_g, hdev, F, rec_bytes, h->d_strip_off, h->S, hk, st),
+                    "split records");
+            if (!spec)
+                PI_CUDA(pi::split_records(full_d, m + o_d, hdev + n_host * rec_bytes, F, h->wrow, h->d_strip_off,
+                                          h->S, hk, st), "split down rows");
+            x.Wgu_cold = hdev;
+            x.Wd_cold = spec ? hdev + gu_bytes : hdev + n_host * rec_bytes;
+        }
         x.sU = i8 ? reinterpret_cast<const float *>(m + o_s) : nullptr;
         x.sV = i8 ? reinterpret_cast<const float *>(m + o_sV) : nullptr;
         // the table is reused for the next expert: finish this one first
         PI_CUDA(cudaStreamSynchronize(st), "load_layer sync");
     }
     PI_CUDA(cudaFreeAsync(d_perm, st), "cudaFreeAsync(perm)");
+    if (full_g) PI_CUDA(cudaFreeAsync(full_g, st), "cudaFreeAsync(records)");
+    if (full_d) PI_CUDA(cudaFreeAsync(full_d, st), "cudaFreeAsync(down rows)");
     if (E > 1) {
         if (!h->router_mem[layer])
             PI_CUDA(cudaMalloc(&h->router_mem[layer], size_t(E) * d * 2), "cudaMalloc(router)");
@@ -444,6 +483,18 @@ pi_status pi_ffn_load_layer(pi_ffn_t h, int layer, const pi_expert_weights *expe
     h->loaded[layer] = 1;
     if (h->prefill) pi::prefill_invalidate(h->prefill, layer);
     if (!h->vrm_ok.empty()) h->vrm_ok[layer] = 0;
+    return PI_OK;
+}
+
+pi_status pi_ffn_set_hot_neurons(pi_ffn_t h, int hot_per_strip)
+{
+    if (!h) return fail(PI_ERR_INVALID_ARG, "null handle");
+    for (char c : h->loaded)
+        if (c) return fail(PI_ERR_INVALID_ARG, "set the VRAM budget before loading any layer");
+    const int min_strip = h->desc.d_ff / h->S;
+    if (hot_per_strip < 0 || hot_per_strip > min_strip)
+        return fail(PI_ERR_INVALID_ARG, "hot_per_strip must be in [0, %d] (the smallest strip)", min_strip);
+    h->hot_k = hot_per_strip;
     return PI_OK;
 }
 
@@ -496,6 +547,7 @@ static pi::DecodeParams base_params(pi_ffn_t h)
     p.wait_ns = h->wait_ns;
     p.debug_flags = h->debug_flags;
     p.local_gather = (h->debug_flags & 4) ? 1 : 0;
+    p.hot_k = h->hot_k;
     p.prof = h->prof;
     return p;
 }
@@ -575,6 +627,7 @@ pi_status pi_sparse_ffn_decode_batch(pi_ffn_t h, int layer_begin, int layer_end,
     if (!aligned16(resid_dev) || (trace_dev && !aligned16(trace_dev)))
         return fail(PI_ERR_INVALID_ARG, "resid_dev and trace_dev must be 16-byte aligned");
     if (D.n_experts != 1) return fail(PI_ERR_UNSUPPORTED, "small-batch decode takes dense FFN layers");
+    if (h->hot_k) return fail(PI_ERR_UNSUPPORTED, "small-batch decode needs every record in HBM (no VRAM budget)");
     if (!((D.w_dtype == PI_F16 && D.pred_dtype == PI_F16) || (D.w_dtype == PI_BF16 && D.pred_dtype == PI_BF16)))
         return fail(PI_ERR_UNSUPPORTED, "small-batch decode takes F16 or BF16 weights with a predictor of the same format");
     if (D.d_model > pi::batch_max_d())
@@ -660,6 +713,53 @@ pi_status pi_sparse_ffn_decode_batch(pi_ffn_t h, int layer_begin, int layer_end,
     return PI_OK;
 }
 
+namespace {
+__global__ void k_residual_add(float *__restrict__ r, const float *__restrict__ y, int d)
+{
+    const int j = blockIdx.x * blockDim.x + threadIdx.x;
+    if (j < d) r[j] += y[j];
+}
+}  // namespace
+
+pi_status pi_sparse_ffn_decode_partial(pi_ffn_t h, int layer, const float *resid_dev, float *y_dev,
+                                       int32_t *stats_dev, uint32_t *mask_dev, void *stream)
+{
+    if (!h || !resid_dev || !y_dev) return fail(PI_ERR_INVALID_ARG, "pi_sparse_ffn_decode_partial: null argument");
+    const pi_ffn_desc &D = h->desc;
+    if (layer < 0 || layer >= D.n_layers) return fail(PI_ERR_INVALID_ARG, "layer %d out of range", layer);
+    if (!h->loaded[layer]) return fail(PI_ERR_NOT_LOADED, "layer %d not loaded", layer);
+    if (!aligned16(resid_dev) || !aligned16(y_dev))
+        return fail(PI_ERR_INVALID_ARG, "resid_dev and y_dev must be 16-byte aligned");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    PI_CUDA(cudaSetDevice(D.device), "cudaSetDevice");
+    pi::DecodeParams p = base_params(h);
+    p.mode = pi::kModeDecode;
+    p.layer_begin = layer;
+    p.layer_end = layer + 1;
+    p.resid = const_cast<float *>(resid_dev);   // read only: y goes to y_out
+    p.y_out = y_dev;
+    p.stats = stats_dev;
+    p.masks = mask_dev;
+    PI_CUDA(cudaMemsetAsync(h->bar, 0, sizeof(unsigned) * pi::kBarWords, st), "memset barrier");
+    PI_CUDA(cudaMemsetAsync(h->fix, 0, sizeof(long long) * 2 * pi::kFixStride, st), "memset accumulators");
+    if (stats_dev) PI_CUDA(cudaMemsetAsync(stats_dev, 0, sizeof(int32_t) * 4, st), "memset stats");
+    if (mask_dev)
+        PI_CUDA(cudaMemsetAsync(mask_dev, 0, sizeof(uint32_t) * D.top_k * ((D.d_ff + 31) / 32), st), "memset masks");
+    PI_CUDA(pi::launch_decode(h->wfmt, h->pfmt, p, st), "launch partial decode");
+    return PI_OK;
+}
+
+pi_status pi_residual_add(pi_ffn_t h, float *resid_dev, const float *y_dev, void *stream)
+{
+    if (!h || !resid_dev || !y_dev) return fail(PI_ERR_INVALID_ARG, "pi_residual_add: null argument");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    PI_CUDA(cudaSetDevice(h->desc.device), "cudaSetDevice");
+    const int d = h->desc.d_model;
+    k_residual_add<<<(d + 255) / 256, 256, 0, st>>>(resid_dev, y_dev, d);
+    PI_CUDA(cudaGetLastError(), "launch residual add");
+    return PI_OK;
+}
+
 pi_status pi_sparse_ffn_decode_host(pi_ffn_t h, int layer_begin, int layer_end,
                                     const float *resid_in_host, float *resid_out_host, void *stream)
 {
@@ -719,6 +819,7 @@ pi_status pi_dense_ffn_prefill(pi_ffn_t h, int layer_begin, int layer_end, int n
     for (int l = layer_begin; l < layer_end; ++l)
         if (!h->loaded[l]) return fail(PI_ERR_NOT_LOADED, "layer %d not loaded", l);
     if (!aligned16(resid_dev)) return fail(PI_ERR_INVALID_ARG, "resid_dev must be 16-byte aligned");
+    if (h->hot_k) return fail(PI_ERR_UNSUPPORTED, "dense prefill needs every record in HBM (no VRAM budget)");
     PI_CUDA(cudaSetDevice(D.device), "cudaSetDevice");
     pi::PrefillView v{};
     v.d = D.d_model;

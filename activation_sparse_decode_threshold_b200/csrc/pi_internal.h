@@ -38,6 +38,11 @@ struct ExpertDev {
                          // (inside the records for the speculative kinds)
     const float *sU;     // 8-bit predictor: scale of each U row (table order); else null
     const float *sV;     // 8-bit predictor: scale of each V row (r); else null
+    // With a VRAM budget (DecodeParams::hot_k > 0) Wgu / Wd hold only the first
+    // hot_k records of each strip (index b * hot_k + loc) and the others sit in
+    // pinned host memory at these device-visible addresses (index pos - (b+1) hot_k).
+    const uint8_t *Wgu_cold;
+    const uint8_t *Wd_cold;
 };
 
 enum Mode { kModeDecode = 0, kModePredict = 1 };
@@ -59,6 +64,7 @@ struct DecodeParams {
     int mode, pred_expert;
     // inputs / outputs
     float *resid;                   // [d] decode: in/out residual
+    float *y_out;                   // [d] or null: one-layer call that emits y (the residual unchanged)
     const float *x_in;              // [d] predict: layer input
     float *trace;                   // [(l1-l0) * d] or null
     int32_t *stats;                 // [(l1-l0) * 4] or null (zeroed by the host)
@@ -79,6 +85,7 @@ struct DecodeParams {
     long long wait_ns;              // bound on every device-side wait
     int debug_flags;
     int local_gather;               // each CTA gathers its own strip's active neurons (no balance step)
+    int hot_k;                      // records in HBM per strip (0 = all; others in host memory)
     long long *prof;                // [(l1-l0) * kProfPoints * S] phase timestamps, or null
 };
 
@@ -87,7 +94,7 @@ struct DecodeParams {
 constexpr int kModeMoE = 1, kModeGated = 2, kModeSpec = 4, kModePred = 8;
 // grid barrier: one arrival counter at word 0 of a zeroed area of kBarWords words
 constexpr int kBarWords = 512;
-constexpr int kProfPoints = 14;   // timestamps and cycle counters per layer and CTA
+constexpr int kProfPoints = 22;   // timestamps and cycle counters per layer and CTA
 
 cudaError_t launch_decode(int wfmt, int pfmt, const DecodeParams &p, cudaStream_t stream);
 int decode_max_blocks_per_sm(int wfmt, int pfmt, int d);
@@ -132,6 +139,10 @@ cudaError_t repack_rows(uint8_t *dst, const int32_t *perm, int rows, int n_src,
 cudaError_t repack_v_blocks(const uint8_t *V, uint8_t *dst, const int32_t *grp_off, int S, int r,
                             int d, int elem_bytes, cudaStream_t s);
 cudaError_t repack_bias(const float *src, float *dst, const int32_t *perm, int n, cudaStream_t s);
+// Records (`bytes` each, table order) split by strip position: the first hot_k
+// of each strip to `hot`, the others to `cold` (a device-visible host buffer).
+cudaError_t split_records(const uint8_t *src, uint8_t *hot, uint8_t *cold, int F, int bytes,
+                          const int32_t *strip_off, int S, int hot_k, cudaStream_t s);
 // U rows in table order, 16-byte chunks permuted inside each 128-byte group by
 // (row - strip start) mod 8 (row_bytes a multiple of 128); strip_off on the device.
 cudaError_t repack_u_swizzled(uint8_t *dst, const int32_t *perm, int rows, const uint8_t *src, int row_bytes,

@@ -116,7 +116,35 @@ __global__ void k_invert(const int32_t *__restrict__ perm, int32_t *__restrict__
     if (p < n) inv[perm[p]] = p;
 }
 
+// Records in table order -> the first hot_k of each strip to `hot` (index
+// b * hot_k + loc) and the rest to `cold` (index p - (b + 1) * hot_k).
+__global__ void k_split_records(const uint8_t *__restrict__ src, uint8_t *__restrict__ hot, uint8_t *__restrict__ cold,
+                                int F, int bytes, const int32_t *__restrict__ strip_off, int S, int hot_k)
+{
+    const int p = blockIdx.x;
+    if (p >= F) return;
+    int lo = 0, hi = S - 1;                 // strip b with strip_off[b] <= p < strip_off[b + 1]
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) / 2;
+        if (strip_off[mid] <= p) lo = mid;
+        else hi = mid - 1;
+    }
+    const int loc = p - strip_off[lo];
+    uint8_t *dst = loc < hot_k ? hot + (size_t(lo) * hot_k + loc) * bytes
+                               : cold + (size_t(p) - size_t(lo + 1) * hot_k) * bytes;
+    const uint4 *s4 = reinterpret_cast<const uint4 *>(src + size_t(p) * bytes);
+    for (int j = threadIdx.x; j < bytes / 16; j += blockDim.x) reinterpret_cast<uint4 *>(dst)[j] = s4[j];
+}
+
 }  // namespace
+
+cudaError_t split_records(const uint8_t *src, uint8_t *hot, uint8_t *cold, int F, int bytes,
+                          const int32_t *strip_off, int S, int hot_k, cudaStream_t s)
+{
+    if (F <= 0) return cudaSuccess;
+    k_split_records<<<F, 128, 0, s>>>(src, hot, cold, F, bytes, strip_off, S, hot_k);
+    return cudaGetLastError();
+}
 
 cudaError_t repack_v_blocks(const uint8_t *V, uint8_t *dst, const int32_t *grp_off, int S, int r,
                             int d, int elem_bytes, cudaStream_t s)

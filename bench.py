@@ -400,14 +400,93 @@ def prefill_rate(cfg, B, local: int, h, steps: int = 3, warmup: int = 2) -> dict
             "peak_tflops": peak, "peak_source": kind, "prompts_timed": steps, "clocks": clk.summary()}
 
 
+def batch_rate(cfg, B, local: int, h, nb: int, steps: int = 8, warmup: int = 3) -> dict:
+    """Small-batch decode: `nb` tokens per step through pi_sparse_ffn_decode_batch,
+    `steps` steps timed with CUDA events after `warmup`, inputs resident."""
+    L = cfg.n_layers
+    R = synth.token_inputs(cfg, nb * (steps + warmup), "cuda", 2000)
+    stats = torch.zeros((steps + warmup, L, 4), device="cuda", dtype=torch.int32)
+    bufs = [R[i * nb:(i + 1) * nb].clone() for i in range(steps + warmup)]
+    for i in range(warmup):
+        B.pi_sparse_ffn_decode_batch(h, 0, L, bufs[i], None, stats[i])
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for i in range(warmup, warmup + steps):
+            B.pi_sparse_ffn_decode_batch(h, 0, L, bufs[i], None, stats[i])
+        e1.record(stream)
+        torch.cuda.synchronize()
+    if B.pi_sync(h) != B.PI_OK:
+        raise RuntimeError(B.pi_last_error())
+    ms = e0.elapsed_time(e1) / steps
+    st = stats[warmup:].cpu().numpy()
+    # touched bytes per step: predictor once per launch group, the union's gate/up
+    # rows, the down rows of union neurons with some h != 0, index + mask entries
+    pb = PB[cfg.pdtype]
+    groups = -(-nb // (4 if cfg.wdtype == "bf16" else 8))
+    w = wrow_bytes(cfg)
+    per_layer = [groups * (pb * cfg.rank * (cfg.d + cfg.F) + 4 * cfg.F) + (2 if cfg.gated else 1) * u * w
+                 + uh * w + 8 * u for s_ in st for (u, _, uh, _) in s_]
+    byts = float(np.sum(per_layer)) / steps
+    peak, kind = measured_peaks()
+    return {"tokens_per_step": nb, "tok_s": nb / (ms / 1e3), "ms_per_step": ms,
+            "achieved_gbs": byts / (ms / 1e3) / 1e9, "roofline_frac": byts / (ms / 1e3) / 1e9 / peak,
+            "peak_source": kind, "union_per_layer": float(st[:, :, 0].mean()),
+            "predicted_per_layer_summed_over_tokens": float(st[:, :, 1].mean()),
+            "launch_groups": groups, "steps_timed": steps, "clocks": clk.summary()}
+
+
+def tp_rate(cfg, B, local: int, h, steps: int = 32, warmup: int = 4) -> dict:
+    """The tensor-parallel layer sequence on one rank holding every neuron: per
+    layer pi_sparse_ffn_decode_partial, (the all-reduce of y, an identity on
+    one rank) and pi_residual_add -- the fused decode's work in 2 L launches."""
+    L = cfg.n_layers
+    R = synth.token_inputs(cfg, steps + warmup, "cuda", 3000)
+    y = torch.empty(cfg.d, device="cuda")
+
+    def token(r):
+        for l in range(L):
+            B.pi_sparse_ffn_decode_partial(h, l, r, y)
+            B.pi_residual_add(h, r, y)
+    for i in range(warmup):
+        token(R[i])
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(warmup, warmup + steps):
+        token(R[i])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if B.pi_sync(h) != B.PI_OK:
+        raise RuntimeError(B.pi_last_error())
+    ms = e0.elapsed_time(e1) / steps
+    return {"tok_s": 1e3 / ms, "ms_per_token": ms, "launches_per_token": 2 * L, "ranks": 1,
+            "note": "per-layer launches of the sharded path with one rank; the all-reduce is an identity"}
+
+
 def run_extras(B, local: int, steps: int) -> dict:
     """The other workloads of the method's measurement plan, each on its own
     handle: the mistral7b sparsity sweep, falcon40b, mixtral47b decode and the
-    512-token dense prefill of the mixtral47b shape."""
+    512-token dense prefill of the mixtral47b shape, small-batch decode of
+    mistral7b, and the llama7b and mixtral47b shapes with the 8-bit per-row
+    predictor.  (Small-batch decode of llama7b runs on the headline's handle.)"""
     out = {}
     m = synth.CONFIGS["mistral7b"]
     for a in m.sweep:
-        out[f"mistral7b@active{a}"] = decode_rate(m, B, local, a, steps, 8)
+        if a == m.mean_active:
+            h = build_handle(m, B, local, None)
+            try:
+                out[f"mistral7b@active{a}"] = decode_rate(m, B, local, None, steps, 8, h)
+                out["mistral7b-batch4"] = batch_rate(m, B, local, h, 4)
+                out["mistral7b-batch8"] = batch_rate(m, B, local, h, 8)
+            finally:
+                torch.cuda.synchronize()
+                B.pi_ffn_destroy(h)
+        else:
+            out[f"mistral7b@active{a}"] = decode_rate(m, B, local, a, steps, 8)
         torch.cuda.empty_cache()
     out["falcon40b"] = decode_rate(synth.CONFIGS["falcon40b"], B, local, None, max(16, steps // 2), 8)
     torch.cuda.empty_cache()
@@ -420,6 +499,9 @@ def run_extras(B, local: int, steps: int) -> dict:
         torch.cuda.synchronize()
         B.pi_ffn_destroy(h)
     torch.cuda.empty_cache()
+    for name in ("llama7b-i8pred", "mixtral47b-i8pred"):
+        out[name] = decode_rate(synth.CONFIGS[name], B, local, None, steps, 8)
+        torch.cuda.empty_cache()
     return out
 
 
@@ -533,17 +615,21 @@ def main() -> int:
         e2e = {"value": job_throughput(K, world, e2e_ms), "unit": "tok/s",
                "h2d_bytes_per_step": 4 * cfg.d, "d2h_bytes_per_step": 4 * cfg.d}
 
+    extra = None
+    if world == 1 and not args.no_extra and not args.layers and args.config == "llama7b" and active is None:
+        extra = {f"llama7b-batch{nb}": batch_rate(cfg, B, local, h, nb) for nb in (4, 8, 16)}
+        extra["llama7b-tp1-per-layer"] = tp_rate(cfg, B, local, h)
     torch.cuda.synchronize()
     B.pi_ffn_destroy(h)
+    torch.cuda.empty_cache()
+    if extra is not None:
+        extra.update(run_extras(B, local, 64))
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return 0
 
-    extra = None
-    if world == 1 and not args.no_extra and not args.layers and args.config == "llama7b" and active is None:
-        extra = run_extras(B, local, 64)
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:

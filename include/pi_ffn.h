@@ -139,6 +139,21 @@ PI_API pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out);
 PI_API pi_status pi_ffn_load_layer(pi_ffn_t h, int layer, const pi_expert_weights *experts,
                             const void *router_dev, const float *freq_host, void *stream);
 
+/* VRAM budget (the survey's "next" row f4; PowerInfer (unite.ai), "Neuron
+ * placement and management": hot neurons on the GPU, cold ones in host memory).
+ * Keep only the first `hot_per_strip` neuron records of every strip in device
+ * memory -- the strip's hottest neurons, since the table orders each strip
+ * hottest first -- and the others in pinned, device-mapped host memory, read
+ * by the decode kernel over the host link when predicted active.  The
+ * predictor (V, U, c) and INT4 scales stay in device memory.  0 (the default)
+ * keeps every record in device memory.  Must be called before any layer is
+ * loaded; 0 <= hot_per_strip <= floor(d_ff / n_strips), else
+ * PI_ERR_INVALID_ARG.  Decode results are bit-identical to a handle without a
+ * budget; pi_dense_ffn_prefill and pi_sparse_ffn_decode_batch return
+ * PI_ERR_UNSUPPORTED on a budgeted handle.  Device memory per layer and expert
+ * drops by (d_ff - n_strips * hot_per_strip) records. */
+PI_API pi_status pi_ffn_set_hot_neurons(pi_ffn_t h, int hot_per_strip);
+
 /* Neuron table of (layer, expert): perm_host[p] = original index of the
  * neuron stored at table position p (F entries).  Strip b of the table holds
  * positions [off[b], off[b+1]) with off from pi_strip_offsets.  Table rule:
@@ -209,6 +224,26 @@ PI_API pi_status pi_sparse_ffn_decode_batch(pi_ffn_t h, int layer_begin, int lay
                                             float *resid_dev, float *trace_dev, int32_t *stats_dev,
                                             uint32_t *mask_dev, void *stream);
 
+/* Tensor-parallel neuron sharding (the survey's "next" row f3; the pages name
+ * no collective).  A handle may hold a SHARD of each layer's neurons: its
+ * d_ff is the shard's neuron count and pi_ffn_load_layer receives that
+ * shard's rows of W_gate / W_up / U / c and columns of W_down, with the full
+ * V (replicated), so each shard predicts exactly its own neurons of the full
+ * predictor.  The layer's output y is the sum over the shards.
+ *
+ * pi_sparse_ffn_decode_partial runs one layer on resid_dev (the residual
+ * entering the layer, [d] float, read only) and writes this handle's share of
+ * y to y_dev ([d] float): RMSNorm, prediction, gather and the fixed-order
+ * reduction as in pi_sparse_ffn_decode, without the residual add.  The caller
+ * sums y over the shards (an all-reduce across ranks, e.g. NCCL) and adds it
+ * with pi_residual_add (resid_dev[j] += y_dev[j], j < d).  A handle holding
+ * all neurons gives exactly y of pi_sparse_ffn_decode's layer.  stats_dev
+ * ([4]) and mask_dev (top_k x ceil(d_ff/32)) as in pi_sparse_ffn_decode, for
+ * this shard.  Asynchronous on `stream`; errors as pi_sparse_ffn_decode. */
+PI_API pi_status pi_sparse_ffn_decode_partial(pi_ffn_t h, int layer, const float *resid_dev, float *y_dev,
+                                              int32_t *stats_dev, uint32_t *mask_dev, void *stream);
+PI_API pi_status pi_residual_add(pi_ffn_t h, float *resid_dev, const float *y_dev, void *stream);
+
 /* Same as pi_sparse_ffn_decode on HOST buffers: copies resid_in_host (d
  * floats) to the device, decodes, copies the result to resid_out_host, and
  * synchronises `stream` before returning.  Host buffers should be pinned for
@@ -260,15 +295,19 @@ PI_API pi_status pi_debug_set(pi_ffn_t h, int flags, double wait_limit_s);
 
 /* Testing aid: when `times_dev` is non-NULL, each later pi_sparse_ffn_decode
  * call records, per layer and CTA, %globaltimer (ns) at these points k:
- *   0 layer start, 1 layer input and t ready, 9 predictor logits done,
- *   2 active list done, 8 this CTA's share of the active list known,
- *   3 gather done, 4 after the gather barrier, 7 partials reduced,
- *   5 column phase done, 6 after the column barrier;
+ *   0 layer start, 1 layer input and t ready, 14 first predictor rows in
+ *   shared memory, 15 first tensor-core logits done, 9 predictor logits done,
+ *   2 active list done, 16 after the balance barrier, 8 this CTA's share of
+ *   the active list known, 17 first gathered rows landed, 3 gather done,
+ *   4 after the gather barrier, 7 partials reduced, 5 column phase done,
+ *   6 after the column barrier; for routed (MoE) layers also 18 experts
+ *   chosen, 19 first V rows in shared memory, 20 t rows written, 21 after the
+ *   t barrier;
  * and k = 10..13 the clock cycles thread 0 spent obtaining the layer input,
  * waiting for predictor rows, waiting for gathered rows and waiting in grid
  * barriers.  Value (layer - layer_begin, k, cta) sits at
- * times_dev[((layer - layer_begin) * 14 + k) * n_strips + cta].  The buffer
- * (caller-owned, device, 8-byte aligned) must hold (l1 - l0) * 14 * n_strips
+ * times_dev[((layer - layer_begin) * 22 + k) * n_strips + cta].  The buffer
+ * (caller-owned, device, 8-byte aligned) must hold (l1 - l0) * 22 * n_strips
  * values.  NULL turns recording off. */
 PI_API pi_status pi_debug_phase_times(pi_ffn_t h, long long *times_dev);
 

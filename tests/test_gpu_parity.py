@@ -279,3 +279,57 @@ def test_residual_out_of_fixed_point_range_reports_device_check(handles):
     B.pi_sparse_ffn_decode(h, 0, 1, r2)
     assert B.pi_sync(h) == B.PI_OK
     assert torch.isfinite(r2).all()
+
+
+# ---------------------------------------------------------------------------
+# VRAM budget: cold records in pinned host memory
+# ---------------------------------------------------------------------------
+BUDGET = {
+    "reglu-f16": (SMALL["reglu-f16"], 2),
+    "drelu-bf16": (SMALL["drelu-bf16"], 3),
+    "moe-int4-drelu": (SMALL["moe-int4-drelu"], 1),
+    "relu-f16-nongated": (SMALL["relu-f16-nongated"], 5),
+}
+
+
+@pytest.mark.parametrize("name", sorted(BUDGET))
+def test_vram_budget_gives_the_same_bits_and_matches_oracle(handles, name):
+    """Most records live in pinned host memory (only the hottest few of each
+    strip stay in HBM); decode gives the same bits as the all-HBM handle and
+    matches the oracle layer by layer."""
+    cfg, hot = BUDGET[name]
+    h0, lws = _build(cfg, handles)
+    h1 = G.create(cfg)
+    handles.append(h1)
+    B.pi_ffn_set_hot_neurons(h1, hot)
+    for l, lw in enumerate(lws):
+        G.load(h1, l, lw)
+    olayers = [G.oracle_layer(cfg, lw) for lw in lws]
+    perms = [G.tables(h1, lw, l, cfg.F) for l, lw in enumerate(lws)]
+    for t in range(3):
+        r0 = synth.token_input(cfg, t)
+        a, trace, stats, masks = G.decode_traced(h1, cfg, 0, cfg.n_layers, r0)
+        b, _, _, _ = G.decode_traced(h0, cfg, 0, cfg.n_layers, r0)
+        assert np.array_equal(a, b)
+        outs = list(trace[1:]) + [a]
+        for l in range(cfg.n_layers):
+            ex, router = olayers[l]
+            G.check_layer(cfg, ex, router, perms[l], trace[l], outs[l], stats[l], masks[l],
+                          case=f"decode/vram-budget/{name}")
+
+
+def test_vram_budget_rejections(handles):
+    cfg = SMALL["reglu-f16"]
+    h, _ = _build(cfg, handles, n_layers=1)
+    with pytest.raises(B.PiError):             # after a layer is loaded
+        B.pi_ffn_set_hot_neurons(h, 1)
+    h2 = G.create(cfg, 1)
+    handles.append(h2)
+    with pytest.raises(B.PiError):             # more than the smallest strip
+        B.pi_ffn_set_hot_neurons(h2, cfg.F)
+    B.pi_ffn_set_hot_neurons(h2, 1)
+    G.load(h2, 0, synth.make_layer(cfg, 0, "cuda"))
+    R = synth.prefill_input(cfg, 4, "cuda")
+    with pytest.raises(B.PiError) as ei:
+        B.pi_dense_ffn_prefill(h2, 0, 1, 4, R)
+    assert ei.value.status == B.PI_ERR_UNSUPPORTED
