@@ -347,6 +347,7 @@ struct Smem {
             int32_t glst[kMaxTopK * kMaxStrip];  // (slot << 24) | table position
             float gc[kMaxTopK * kMaxStrip];      // their biases
         };
+        ExpertDev exall[kMaxExperts];          // every expert's weight pointers (MoE layer start)
     };
     int scan[kMaxStrips + 1];              // exclusive prefix of the strip counts
     union {                                // layer start .. logits / gather
@@ -808,6 +809,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             }
             for (int i = tid; i < ns; i += kThreads) sm.cbuf[0][i] = __ldg(sm.exl[l & 1][0].c + s0 + i);
         }
+        // MoE: every expert's weight pointers move to shared memory beside the
+        // sum of squares, so the routed experts' come without a round trip
+        if (moe && !predict && warp == 1 && lane < p.E) sm.exall[lane] = p.ex[size_t(l) * p.E + lane];
         float inv = 1.f;
         if (!predict) {
             // sum of squares: the CTAs' values in CTA order (warp 0; lane j takes
@@ -856,10 +860,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 float wlo = 1.f, whi = 0.f;
                 if (!predict) {
                     float logit[kMaxExperts], pr[kMaxExperts];
+                    // every logit's load first (one round trip), then the arithmetic
+                    long long raw[kMaxExperts];
+#pragma unroll
+                    for (int e = 0; e < kMaxExperts; ++e) raw[e] = e < p.E ? __ldcg(fx + kMaxRankTotal + 1 + e) : 0;
                     float mx = -INFINITY;
-                    for (int e = 0; e < p.E; ++e) {
-                        logit[e] = float(double(__ldcg(fx + kMaxRankTotal + 1 + e)) * (1.0 / 4294967296.0)) * inv;
-                        mx = fmaxf(mx, logit[e]);
+#pragma unroll
+                    for (int e = 0; e < kMaxExperts; ++e) {
+                        logit[e] = float(double(raw[e]) * (1.0 / 4294967296.0)) * inv;
+                        if (e < p.E) mx = fmaxf(mx, logit[e]);
                     }
                     float den = 0.f;
                     for (int e = 0; e < p.E; ++e) { pr[e] = expf(logit[e] - mx); den += pr[e]; }
@@ -881,7 +890,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 sm.route_e[1] = hi;
                 sm.route_w[0] = wlo;
                 sm.route_w[1] = whi;
-                for (int e = 0; e < ntop; ++e) sm.exl[l & 1][e] = p.ex[size_t(l) * p.E + (e == 0 ? lo : hi)];
+                for (int e = 0; e < ntop; ++e)
+                    sm.exl[l & 1][e] = predict ? p.ex[size_t(l) * p.E + lo] : sm.exall[e == 0 ? lo : hi];
             }
             // the first round of this CTA's V rows is on the critical path: its
             // copies are issued at once (thread 0), and only then do the
