@@ -675,32 +675,11 @@ __global__ void __launch_bounds__(kThreads, 1) batch_kernel(const __grid_constan
     }
 }
 
-// V column blocks (block b: r rows of its ncol_b columns) back to row-major.
-__global__ void k_unblock_v(const uint8_t *__restrict__ blk, uint8_t *__restrict__ vrm, const int32_t *__restrict__ grp_off,
-                            int S, int r, int d, int eb)
-{
-    const int k = blockIdx.x;           // row of V
-    for (int b = 0; b < S; ++b) {
-        const int c0 = 8 * grp_off[b], nc = 8 * (grp_off[b + 1] - grp_off[b]);
-        const uint8_t *src = blk + (size_t(r) * c0 + size_t(k) * nc) * eb;
-        uint8_t *dst = vrm + (size_t(k) * d + c0) * eb;
-        for (int j = threadIdx.x; j < nc * eb / 16; j += blockDim.x)
-            reinterpret_cast<uint4 *>(dst)[j] = reinterpret_cast<const uint4 *>(src)[j];
-    }
-}
-
 }  // namespace
 
 int batch_max_tokens() { return kNB; }
 int batch_tokens_per_launch(int wfmt) { return wfmt == kBF16 ? kNB / 2 : kNB; }
 int batch_max_d() { return kBD; }
-
-cudaError_t unblock_v(const uint8_t *blk, uint8_t *vrm, const int32_t *grp_off_dev, int S, int r, int d, int eb,
-                      cudaStream_t st)
-{
-    k_unblock_v<<<r, 128, 0, st>>>(blk, vrm, grp_off_dev, S, r, d, eb);
-    return cudaGetLastError();
-}
 
 cudaError_t launch_batch(int wfmt, const BatchLaunch &L, cudaStream_t st)
 {

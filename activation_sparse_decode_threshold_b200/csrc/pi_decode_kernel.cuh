@@ -2,11 +2,10 @@
 //
 // One cooperative launch runs a range of layers for one token.  Each CTA owns
 // one strip of the neuron table (a contiguous run of table positions holding
-// a balanced share of hot neurons, hottest first) and one slice of the d_model
-// columns.  Per layer l (dense FFN):
+// a balanced share of hot neurons, hottest first), a few rows of t and one
+// slice of the d_model columns.  Per layer l (dense FFN):
 //
-//   [B] t = V x (from the column phase below), x = RMSNorm(r);
-//       z = U t - c over the strip (tensor-core dots of the staged U rows),
+//   [B] z = U t - c over the strip (tensor-core dots of the staged U rows),
 //       active iff z > threshold, the active list compacted in ascending
 //       table order with warp ballots (PowerInfer (unite.ai), "Adaptive
 //       sparse predictor").
@@ -19,27 +18,30 @@
 //       act(g, u); for h != 0 its W_down column (stored as a row) accumulates
 //       into a per-CTA fp32 partial of y ("Neuron-aware operators": rows of
 //       the input matrices, columns of the output matrix).
+//   [merge] each CTA's partial, rounded to 64-bit fixed point, is added into
+//       the layer's total by one bulk reduction in L2 (integer adds: the total
+//       does not depend on arrival order; the merge of partial results,
+//       nearauto.com PowerInfer article, Fig. 8).
 //   --- grid barrier ---
-//   [column phase] r <- r + sum of the per-CTA partials, for this CTA's
-//       columns, in fixed CTA order (the merge of partial results, nearauto.com
-//       PowerInfer article, Fig. 8); then, for layer l + 1, this CTA's share of
-//       sum(r^2) and of t = V r (V stored column-blocked per CTA), added in
-//       64-bit fixed point so the totals do not depend on arrival order.
+//   [next input] every CTA reads the whole total and forms the whole next
+//       input r + y, its sum of squares and x = RMSNorm(r + y) in the same
+//       order (so every CTA holds the same x); its own rows of t = V x for
+//       layer l + 1 go to global memory, its columns of r + y to the next
+//       input buffer.
 //   --- grid barrier ---
 //
-// Three grid barriers per dense layer.  The MoE layer adds routing (from
-// fixed-point router logits, identical in every CTA), t computed by rows of
-// the two chosen experts, and a fourth barrier.
+// Three grid barriers per layer.  A routed (MoE) layer picks its two experts
+// in the [next input] step from router logits every CTA computes from its own
+// copy of x, and its rows of t then come from the chosen experts' V.
 //
 // Memory: weight bytes are pulled towards the SM as soon as their addresses
 // are known.  A strip's active records are prefetched into L2 the moment its
-// list is published; the next layer's V block and biases are prefetched into
-// L2 when the gather starts; when it ends, the next layer's V block (dense)
-// and the first U round are bulk-copied into shared memory, where they land
-// during the barriers (the V block in the top of the staging buffer, the U
-// rows below it, and the U rows that do not fit yet once the column phase has
-// read the V block).  All waits are bounded (%globaltimer); a wait that runs
-// out records an error word and every CTA returns.
+// list is published; the next layer's V rows of this CTA and biases (router
+// rows when routed) are prefetched into L2 when the gather starts; when it
+// ends, they are bulk-copied into shared memory with the first rows of the
+// next U strip, and land during the merge and its barrier.  All waits are
+// bounded (%globaltimer); a wait that runs out records an error word and
+// every CTA returns.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -335,7 +337,6 @@ constexpr int kRA = 16;           // V rows per staging round at most
 constexpr int kZRows = 112;       // U rows per staging round at most (a multiple of 16)
 constexpr int kMaxU = 4;          // U vectors per lane (rank <= 128 * EPV)
 constexpr int kRound = 16;        // neurons per gather round at most
-constexpr int kVsmMax = 128 * 1024;  // largest V block staged in shared memory for the column phase
 static_assert(kRound <= 32, "a round's neurons are tracked in one warp ballot");
 constexpr int kRed = 2 * kRound;  // values reduced per warp at most
 
@@ -372,7 +373,6 @@ struct Smem {
     float rh[kRound];                      // h of each neuron of a gather round
     int route_e[kMaxTopK];
     float route_w[kMaxTopK];
-    float inv_rms;
     int bc[2];
     uint64_t stage_bar;                    // completion of a staging round
     uint64_t vbar;                         // completion of the V block staged for the column phase
@@ -399,15 +399,42 @@ __device__ __forceinline__ void prof_put(const DecodeParams &p, int li, int poin
 // PI_ERR_DEVICE_CHECK) instead of wrapping silently.
 constexpr float kFixT = 4294967296.0f;    // 2^32
 constexpr float kFixMax = 36028797018963968.0f;   // 2^55
-__device__ __forceinline__ void fix_add(long long *dst, float v, float scale, int *err)
+__device__ __forceinline__ unsigned long long fix_q(float v, int *err)
 {
-    const float sv = v * scale;
+    const float sv = v * kFixT;
     if (!(fabsf(sv) < kFixMax)) {
         set_error(err, kDevCheck);
-        return;
+        return 0ull;
     }
-    const long long q = __float2ll_rn(sv);
-    atomicAdd(reinterpret_cast<unsigned long long *>(dst), static_cast<unsigned long long>(q));
+    return static_cast<unsigned long long>(__float2ll_rn(sv));
+}
+
+// Shared-memory writes made visible to the bulk-copy (async) proxy, and the
+// executing thread's generic and async views of global memory ordered.
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// dst[i] += src[i] for `bytes` of 64-bit integers, by bulk reductions from
+// this CTA's shared memory (32 KB pieces), committed as one bulk group.
+__device__ __forceinline__ void bulk_reduce_add_u64(unsigned long long *dst, const void *src, uint32_t bytes)
+{
+    for (uint32_t o = 0; o < bytes; o += 32768u) {
+        const uint32_t n = bytes - o < 32768u ? bytes - o : 32768u;
+        asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.u64 [%0], [%1], %2;"
+                     ::"l"(reinterpret_cast<uint8_t *>(dst) + o), "r"(s2u(src) + o), "r"(n)
+                     : "memory");
+    }
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until this thread's bulk groups have completed (their writes performed).
+__device__ __forceinline__ void bulk_wait_all()
+{
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // Grid-wide barrier of all CTAs of the cooperative launch, in two halves so
@@ -506,9 +533,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 {
     constexpr int EPVW = Fm<WF>::EPV, EPVP = Fm<PF>::EPV, VBW = Fm<WF>::VB, VBP = Fm<PF>::VB;
     constexpr int MAXVW = (DMAX / EPVW + kThreads - 1) / kThreads;
-    constexpr int MAXVP = (DMAX / EPVP + kThreads - 1) / kThreads;
-    // when both formats share the vector layout, x is cached once
-    constexpr bool kSameX = (WF == PF);
     using VW = typename Fm<WF>::V;
     using VP = typename Fm<PF>::V;
 
@@ -525,32 +549,34 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     constexpr bool predict = (MODE & kModePred) != 0;   // pi_predict: one layer, stop after the list
     const int ntop = predict ? 1 : p.top_k;
     const int nvecW = (WF == kI4 ? d / 2 : d * (WF == kF32 ? 4 : 2)) / VBW;
-    const int nvecP = p.vrow / VBP;
     const int nvecU = p.urow / VBP;
     const int l0 = p.layer_begin;
     const int l1 = predict ? p.layer_begin + 1 : p.layer_end;
     // this CTA's columns of the residual (8-column groups)
     const int c0 = 8 * p.grp_off[b], ncol = 8 * (p.grp_off[b + 1] - p.grp_off[b]);
-    // this CTA's rows of t (row-split form, MoE)
+    // this CTA's rows of t (rows [a0, a1) of the layer's experts' ranks together)
     const int rows_total = ntop * r;
     const int a0 = int((long long)b * rows_total / S), a1 = int((long long)(b + 1) * rows_total / S);
+    const int nrows = a1 - a0;
     // U rows per staging round: the whole strip when it fits, else rounds of a
     // multiple of 8 rows (chunk permutation keys are row mod 8)
     const int ucap_rows = min(kZRows, kStageBytes / p.urow);
     const int ucap = ns <= ucap_rows ? max(ns, 1) : (ucap_rows & ~7);
 
-    // V block of this CTA (dense): rows of t restricted to this CTA's columns
-    auto vblk = [&](int l) -> const uint8_t * {
-        return sm.exl[l & 1][0].V + size_t(r) * c0 * (p.vrow / d);
-    };
-    const int vbrow = ncol * (p.vrow / d);   // bytes of one V-block row
-    // dense decode: after the gather the next layer's V block is bulk-copied
-    // into the top of the staging buffer, beside the first `ufirst` rows of
-    // the next U strip's first round; the rest of that round follows once the
-    // column phase has read the V block
-    const int vbytes = r * vbrow;
-    const int voff = (kStageBytes - vbytes) & ~127;
-    const bool vsm = !moe && !predict && ncol > 0 && vbytes <= kVsmMax;
+    // Staging buffer at the end of a layer (decode): this CTA's partial of y
+    // as fixed-point values at the top [yoff, end); below it the next layer's
+    // V rows of this CTA [voff, yoff) (dense, when they fit: issued when the
+    // gather ends, they land during the reduction and its barrier); below
+    // them the first `ufirst` rows of the next U strip's first round, whose
+    // other rows follow once the V rows have been read.  A routed layer
+    // stages the router's rows at offset 0 when the gather ends and its V
+    // rows from rt_off on once the experts are known.
+    const int yoff = predict ? kStageBytes : kStageBytes - d * 8;
+    const int voff = (yoff - nrows * p.vrow) & ~127;
+    const bool vsm = !moe && nrows > 0 && nrows <= kRA && voff >= 0;
+    const int rt_bytes = moe ? p.E * d * 2 : 0;
+    const bool rsm = moe && !predict && rt_bytes <= yoff;
+    const int rt_off = rsm ? (rt_bytes + 127) & ~127 : 0;
     const int u_round0 = min(ns, ucap);
     const int ufirst = vsm ? min(u_round0, voff / p.urow) : u_round0;
 
@@ -561,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     bool staged_early = false;   // round 0 of the next U strip is already in flight
     bool pending = false;        // a staging round was issued and not yet waited for
     uint32_t vpar = 0;
-    bool vpend = false;          // a V block was issued and not yet waited for
+    bool vpend = false;          // V rows (dense) or router rows (routed) issued on vbar, not yet waited for
     bool upart2 = false;         // the staged U round still misses its second piece
 
     // stage rows [row0, row0 + n) of an expert's U strip, contiguous, at
@@ -578,6 +604,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
     };
     auto stage_u = [&](const ExpertDev &ex, int row0, int n) { stage_u_at(ex, row0, n, 0, true); };
+    // dense, warp 0: layer ln's V rows of this CTA onto vbar and the first
+    // piece of its first U round onto stage_bar (the rest of the strip into L2)
+    auto stage_next_dense = [&](int ln) {
+        const ExpertDev &nx = sm.exl[ln & 1][0];
+        if (lane == 0) {
+            mbar_arrive_tx(&sm.vbar, uint32_t(nrows) * p.vrow);
+            stage_copy(stg + voff, nx.V + size_t(a0) * p.vrow, uint32_t(nrows) * p.vrow, &sm.vbar);
+        }
+        if (ns > 0) {
+            stage_u_at(nx, 0, ufirst, 0, ufirst == u_round0);
+            if (lane == 0 && ns > ucap)
+                prefetch_l2(nx.U + size_t(s0 + ucap) * p.urow, uint32_t(ns - ucap) * p.urow);
+        }
+    };
+    // routed, lane 0 of warp 0: layer ln's router rows onto vbar
+    auto stage_router = [&](int ln) {
+        if (lane == 0) {
+            mbar_arrive_tx(&sm.vbar, uint32_t(rt_bytes));
+            stage_copy(stg, p.router[ln], uint32_t(rt_bytes), &sm.vbar);
+        }
+    };
 
     if (tid == 0) {
         mbar_init(&sm.stage_bar, 1);
@@ -585,15 +632,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         for (int g = 0; g < kRound / 4; ++g) mbar_init(&sm.gbar[g], 1);
         sm.gfail = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        if (!moe) sm.exl[l0 & 1][0] = p.ex[size_t(l0) * p.E];
+        if (!moe) {
+            sm.exl[l0 & 1][0] = p.ex[size_t(l0) * p.E];
+            sm.route_e[0] = sm.route_e[1] = 0;
+            sm.route_w[0] = 1.f;
+            sm.route_w[1] = 0.f;
+        }
     }
     __syncwarp();
-    if (!moe && warp == 0 && ns > 0) {
-        const ExpertDev ex0 = sm.exl[l0 & 1][0];
-        stage_u(ex0, 0, min(ns, ucap));
-        if (lane == 0 && ns > ucap) prefetch_l2(ex0.U + size_t(s0 + ucap) * p.urow, uint32_t(ns - ucap) * p.urow);
+    if (warp == 0) {
+        if (vsm) stage_next_dense(l0);
+        if (rsm) stage_router(l0);
     }
-    if (!moe && ns > 0) staged_early = pending = true;
+    vpend = vsm || rsm;
+    if (vsm && ns > 0) {
+        staged_early = pending = true;
+        upart2 = ufirst < u_round0;
+    }
     cta_sync();
 
     // t value k of `ntr` (the layer's experts' ranks together) into shared memory
@@ -604,271 +659,163 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         else split_parts<PF>(tv, (PF == kBF16 && 3 * ntr <= 2 * kMaxRankTotal) ? 3 : 2, tpart + k, ntr);
     };
 
-    // -----------------------------------------------------------------------
-    // Column phase: this CTA's columns of r (the layer input `li_in`), its
-    // sum of squares, and its partial products for the next layer: the t
-    // partial V[:, cols] r[cols] (dense) or the router logit partials (MoE),
-    // all added in fixed point.  `from_partials`: r = r_old + sum of the
-    // per-CTA partials of y in fixed CTA order; otherwise r is the input.
-    // -----------------------------------------------------------------------
-    // vs: the V block of l_next is being staged in shared memory (vbar)
-    auto column_phase = [&](int li_in, bool from_partials, bool next_exists, int l_next, int prow,
-                            bool vs) -> bool {
-        const float *src = predict ? p.x_in : p.resid;
-        long long *fx = p.fix + size_t(li_in & 1) * kFixStride;
-        // dense: this thread's V-block rows (k = tid and tid + 512; r <= 1024)
-        // for the next layer's t partial; from global memory they start
-        // loading now, so their round trip overlaps the partial reduction's
-        // (the first kVP vectors of each)
-        constexpr int kVP = 4;
-        const bool tpart = !moe && next_exists && ncol > 0;
-        const int nv = vbrow / VBP;
-        const int kr0 = tid, kr1 = tid + kThreads;
-        const uint8_t *vrow0 = nullptr, *vrow1 = nullptr;
-        VP va[kVP], vb2[kVP];
-        if (tpart && !vs) {
-            const uint8_t *vb = vblk(l_next);
-            vrow0 = vb + size_t(kr0 < r ? kr0 : 0) * vbrow;
-            vrow1 = vb + size_t(kr1 < r ? kr1 : 0) * vbrow;
+    // x of the current layer: this thread's vectors v = tid + kThreads k of
+    // EPVW elements (the weight format's vector layout)
+    float xw[MAXVW * EPVW];
+    // EPVW elements of a predictor-format row from element e0 on, as floats
+    static_assert(EPVW % EPVP == 0, "a weight vector spans whole predictor vectors");
+    auto ld_pf = [&](const uint8_t *row, int e0, float *w) {
+        constexpr int PB = PF == kF32 ? 4 : (PF == kI8 ? 1 : 2);
 #pragma unroll
-            for (int j = 0; j < kVP; ++j) {
-                if (j < nv && kr0 < r) va[j] = ldvec<PF>(vrow0 + j * VBP);
-                if (j < nv && kr1 < r) vb2[j] = ldvec<PF>(vrow1 + j * VBP);
-            }
+        for (int j = 0; j < EPVW / EPVP; ++j)
+            cvt<PF>(*reinterpret_cast<const VP *>(row + size_t(e0 + j * EPVP) * PB), w + j * EPVP);
+    };
+    // rows [row0, row0 + n) of layer ln's experts' V (rows of t) at staging
+    // offset rt_off, in one round on stage_bar (thread 0)
+    auto issue_vrows = [&](int ln, int row0, int n) {
+        mbar_arrive_tx(&sm.stage_bar, uint32_t(n) * p.vrow);
+        for (int rr = 0; rr < n;) {
+            const int row = row0 + rr, e = row / r;
+            const int cnt = min(n - rr, (e + 1) * r - row);
+            stage_copy(stg + rt_off + size_t(rr) * p.vrow, sm.exl[ln & 1][e].V + size_t(row - e * r) * p.vrow,
+                       uint32_t(cnt) * p.vrow, &sm.stage_bar);
+            rr += cnt;
         }
-        if (from_partials) {
-            const int q0 = c0 / 4, nq = ncol / 4;
-            for (int qq = warp; qq < nq; qq += kConsumerWarps) {
-                const int q = q0 + qq;
-                float4 pv[kMaxStrips / 32];
-#pragma unroll
-                for (int j = 0; j < kMaxStrips / 32; ++j) {
-                    const int c = lane + 32 * j;
-                    pv[j] = c < S ? __ldcg(reinterpret_cast<const float4 *>(p.partials + size_t(c) * d) + q)
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-                float4 rv = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (lane == 0) rv = __ldcg(reinterpret_cast<const float4 *>(p.resid) + q);
-                float4 sacc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int j = 0; j < kMaxStrips / 32; ++j) {
-                    sacc.x += pv[j].x; sacc.y += pv[j].y; sacc.z += pv[j].z; sacc.w += pv[j].w;
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    sacc.x += __shfl_xor_sync(0xffffffffu, sacc.x, o);
-                    sacc.y += __shfl_xor_sync(0xffffffffu, sacc.y, o);
-                    sacc.z += __shfl_xor_sync(0xffffffffu, sacc.z, o);
-                    sacc.w += __shfl_xor_sync(0xffffffffu, sacc.w, o);
-                }
-                if (lane == 0) {
-                    if (p.y_out) {
-                        // one-layer call on a shard of the neurons: this shard's y,
-                        // the residual left as it is (the caller sums the shards)
-                        __stcg(reinterpret_cast<float4 *>(p.y_out) + q, sacc);
-                    } else {
-                        rv.x += sacc.x; rv.y += sacc.y; rv.z += sacc.z; rv.w += sacc.w;
-                        __stcg(reinterpret_cast<float4 *>(p.resid) + q, rv);
-                        *reinterpret_cast<float4 *>(sm.rsl + 4 * qq) = rv;
-                    }
-                }
-            }
-        } else {
-            for (int j = tid; j < ncol; j += kThreads) sm.rsl[j] = __ldcg(src + c0 + j);
-        }
-        cta_sync();
-        if (prow >= 0) prof_put(p, prow, 7, gtimer());
-        if (!predict && p.trace && li_in < l1 - l0)
-            for (int j = tid; j < ncol; j += kThreads) __stcg(p.trace + size_t(li_in) * d + c0 + j, sm.rsl[j]);
-        if (!next_exists) return true;
-        // sum of squares of this CTA's columns (fixed order: lanes, then tree),
-        // one float per CTA; the layer start sums the CTAs' values in CTA order
-        if (warp == 0 && !predict) {
-            float ss = 0.f;
-            for (int j = lane; j < ncol; j += 32) ss = fmaf(sm.rsl[j], sm.rsl[j], ss);
-            ss = warp_sum(ss);
-            if (lane == 0) __stcg(p.ssq + size_t(li_in & 1) * kMaxStrips + b, ss);
-        }
-        if (!moe) {
-            // t partial: rows kr0, kr1 of the V block dotted with this CTA's columns
-            // (8-bit predictor: times the rows' scales)
-            float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-            float sv0 = 1.f, sv1 = 1.f;
-            if constexpr (PF == kI8) {
-                if (tpart && kr0 < r) sv0 = __ldg(sm.exl[l_next & 1][0].sV + kr0);
-                if (tpart && kr1 < r) sv1 = __ldg(sm.exl[l_next & 1][0].sV + kr1);
-            }
-            auto acc_vec = [&](const VP &q0, const VP &q1, int v) {
-                float w0[EPVP], w1[EPVP];
-                cvt<PF>(q0, w0);
-                cvt<PF>(q1, w1);
-#pragma unroll
-                for (int i = 0; i < EPVP; i += 2) {
-                    const float x0 = sm.rsl[v * EPVP + i], x1 = sm.rsl[v * EPVP + i + 1];
-                    a0 = fmaf(w0[i], x0, a0);
-                    a1 = fmaf(w0[i + 1], x1, a1);
-                    b0 = fmaf(w1[i], x0, b0);
-                    b1 = fmaf(w1[i + 1], x1, b1);
-                }
-            };
-            if (tpart && vs) {
-                if (!stage_wait(&sm, p, vpar, bci, nullptr, &sm.vbar)) return false;
-                vpend = false;
-                if (kr0 < r) {
-                    // each thread walks its rows' vectors from `rot` on, so the
-                    // eight rows of a quarter-warp fall in eight different
-                    // 16-byte bank groups (rows are nv vectors apart)
-                    const int lowbit = nv & -nv;
-                    const int rot = (lane & 7) / (8 / (lowbit < 8 ? lowbit : 8));
-                    const uint8_t *vs0 = stg + voff + size_t(kr0) * vbrow;
-                    const uint8_t *vs1 = stg + voff + size_t(kr1 < r ? kr1 : kr0) * vbrow;
-                    for (int j = 0; j < nv; ++j) {
-                        int jj = j + rot;
-                        if (jj >= nv) jj -= nv;
-                        acc_vec(*reinterpret_cast<const VP *>(vs0 + jj * VBP),
-                                *reinterpret_cast<const VP *>(vs1 + jj * VBP), jj);
-                    }
-                    fix_add(fx + kr0, (a0 + a1) * sv0, kFixT, p.err);
-                    if (kr1 < r) fix_add(fx + kr1, (b0 + b1) * sv1, kFixT, p.err);
-                }
-            } else if (tpart && kr0 < r) {
-#pragma unroll
-                for (int j = 0; j < kVP; ++j)
-                    if (j < nv) acc_vec(va[j], kr1 < r ? vb2[j] : va[j], j);
-                for (int v = kVP; v < nv; ++v) {
-                    const VP q0 = ldvec<PF>(vrow0 + v * VBP);
-                    const VP q1 = kr1 < r ? ldvec<PF>(vrow1 + v * VBP) : q0;
-                    acc_vec(q0, q1, v);
-                }
-                fix_add(fx + kr0, (a0 + a1) * sv0, kFixT, p.err);
-                if (kr1 < r) fix_add(fx + kr1, (b0 + b1) * sv1, kFixT, p.err);
-            }
-        } else if (!predict) {
-            // router logit partials: W_r[e, cols] . r[cols]
-            const __half *R = reinterpret_cast<const __half *>(p.router[l_next]);
-            if (tid < p.E && ncol > 0) {
-                float a = 0.f;
-                for (int j = 0; j < ncol; ++j) a = fmaf(__half2float(R[size_t(tid) * d + c0 + j]), sm.rsl[j], a);
-                fix_add(fx + kMaxRankTotal + 1 + tid, a, kFixT, p.err);
-            }
-        }
-        return true;
     };
 
-    float xw[MAXVW * EPVW];
-    float xp_own[kSameX ? 1 : MAXVP * EPVP];
-#define XP(i) (kSameX ? xw[(i)] : xp_own[(i)])
-
-    // prologue: the first layer's input columns
-    column_phase(0, false, true, l0, -1, false);
-    long long cyc0 = 0;
-    const bool started = grid_sync(&sm, p, epoch, bci, &cyc0);
-
-    for (int l = l0; started && l < l1; ++l) {
-        const int li = l - l0;
-        long long cyc_a = 0, cyc_b = 0, cyc_c = 0, cyc_bar = 0;
-        prof_put(p, li, 0, gtimer());
-        const long long ca0 = clock64();
-        const long long *fx = p.fix + size_t(li & 1) * kFixStride;
-
-        // ---------------- layer input x, [MoE] routing and t rows ------------
-        const float *src = predict ? p.x_in : p.resid;
-        // every global load of the layer start is issued before the sum of
-        // squares is known (one round trip): this thread's columns of r (or
-        // x), t's fixed-point values (dense) and the strip's biases
+    // -----------------------------------------------------------------------
+    // Input of layer ln.  In the prologue (lp < l0) r is the caller's input;
+    // otherwise it is the input of layer lp plus the fixed-point total of lp's
+    // y, and every CTA forms all of it.  This CTA's columns are written out
+    // (the next input buffer, the trace, or the caller's residual after the
+    // last layer); x = RMSNorm(r) goes to xw (the predictor call takes x as
+    // given); a routed layer picks its experts; this CTA's rows of t = V x go
+    // to t_buf; a grid barrier follows, after which every CTA reads t.  The
+    // last layer stops after writing the residual, and a one-layer call that
+    // emits y stops after writing y.  False if a bounded wait ran out.
+    // -----------------------------------------------------------------------
+    auto form_input = [&](int lp, int ln, long long *cycb) -> bool {
+        const bool first = lp < l0;
+        const bool emit = !first && p.y_out != nullptr;
+        const bool last = ln >= l1;
+        const int lip = lp - l0;   // profiling row (the layer whose tail this is)
+        if (moe && !predict && !emit && !last && warp == 1 && lane < p.E)
+            sm.exall[lane] = p.ex[size_t(ln) * p.E + lane];
+        float rv[MAXVW * EPVW];
+        {
+            const float *rin = first ? (predict ? p.x_in : p.resid) : p.rbuf + size_t(lp & 1) * d;
+            const unsigned long long *yt = first ? nullptr : p.yfix + size_t(lp & 1) * d;
+            unsigned long long yq[MAXVW * EPVW];
+            // every load first (one round trip), then the arithmetic
 #pragma unroll
-        for (int k = 0; k < MAXVW; ++k) {
-            const int v = tid + kThreads * k;
-#pragma unroll
-            for (int i = 0; i < EPVW; i += 4) {
-                float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (v < nvecW) q = __ldcg(reinterpret_cast<const float4 *>(src + v * EPVW + i));
-                xw[k * EPVW + i] = q.x; xw[k * EPVW + i + 1] = q.y;
-                xw[k * EPVW + i + 2] = q.z; xw[k * EPVW + i + 3] = q.w;
-            }
-        }
-        if constexpr (!kSameX) {
-#pragma unroll
-            for (int k = 0; k < MAXVP; ++k) {
+            for (int k = 0; k < MAXVW; ++k) {
                 const int v = tid + kThreads * k;
 #pragma unroll
-                for (int i = 0; i < EPVP; i += 4) {
+                for (int i = 0; i < EPVW; i += 4) {
                     float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (v < nvecP) q = __ldcg(reinterpret_cast<const float4 *>(src + v * EPVP + i));
-                    xp_own[k * EPVP + i] = q.x; xp_own[k * EPVP + i + 1] = q.y;
-                    xp_own[k * EPVP + i + 2] = q.z; xp_own[k * EPVP + i + 3] = q.w;
+                    if (v < nvecW && !emit) q = __ldcg(reinterpret_cast<const float4 *>(rin + v * EPVW + i));
+                    rv[k * EPVW + i] = q.x; rv[k * EPVW + i + 1] = q.y;
+                    rv[k * EPVW + i + 2] = q.z; rv[k * EPVW + i + 3] = q.w;
+                }
+                if (!first) {
+#pragma unroll
+                    for (int i = 0; i < EPVW; i += 2) {
+                        ulonglong2 q = make_ulonglong2(0ull, 0ull);
+                        if (v < nvecW) q = __ldcg(reinterpret_cast<const ulonglong2 *>(yt + v * EPVW + i));
+                        yq[k * EPVW + i] = q.x;
+                        yq[k * EPVW + i + 1] = q.y;
+                    }
+                }
+            }
+            if (!first) {
+#pragma unroll
+                for (int j = 0; j < MAXVW * EPVW; ++j)
+                    rv[j] += float(double(static_cast<long long>(yq[j])) * (1.0 / 4294967296.0));
+            }
+        }
+        // this CTA's columns [c0, c0 + ncol)
+        if (!predict) {
+            float *dst = emit ? p.y_out : (last ? p.resid : p.rbuf + size_t(ln & 1) * d);
+            float *trc = (!emit && !last && p.trace) ? p.trace + size_t(ln - l0) * d : nullptr;
+            unsigned long long *yz = first ? p.yfix + size_t(l0 & 1) * d : nullptr;
+#pragma unroll
+            for (int k = 0; k < MAXVW; ++k) {
+                const int v = tid + kThreads * k;
+#pragma unroll
+                for (int i = 0; i < EPVW; ++i) {
+                    const int e = v * EPVW + i;
+                    if (v < nvecW && e >= c0 && e < c0 + ncol) {
+                        __stcg(dst + e, rv[k * EPVW + i]);
+                        if (trc) __stcg(trc + e, rv[k * EPVW + i]);
+                        if (yz) yz[e] = 0ull;   // layer l0's fixed-point total starts at zero
+                    }
                 }
             }
         }
-        long long tq[kMaxRankTotal / kThreads];
-        if (!moe) {
-#pragma unroll
-            for (int j = 0; j < kMaxRankTotal / kThreads; ++j) {
-                const int k = tid + kThreads * j;
-                tq[j] = k < r ? __ldcg(fx + k) : 0;
-            }
-            for (int i = tid; i < ns; i += kThreads) sm.cbuf[0][i] = __ldg(sm.exl[l & 1][0].c + s0 + i);
-        }
-        // MoE: every expert's weight pointers move to shared memory beside the
-        // sum of squares, so the routed experts' come without a round trip
-        if (moe && !predict && warp == 1 && lane < p.E) sm.exall[lane] = p.ex[size_t(l) * p.E + lane];
+        if (emit || last) return true;
+        // x = RMSNorm(r): every CTA sums the same squares in the same order
         float inv = 1.f;
         if (!predict) {
-            // sum of squares: the CTAs' values in CTA order (warp 0; lane j takes
-            // CTAs j, j + 32, ..., then a fixed tree), broadcast through shared memory
-            if (warp == 0) {
-                const float *sq = p.ssq + size_t(li & 1) * kMaxStrips;
-                float ss = 0.f;
-                for (int c = lane; c < S; c += 32) ss += __ldcg(sq + c);
-                ss = warp_sum(ss);
-                if (lane == 0) sm.inv_rms = 1.f / sqrtf(ss / float(d) + p.eps);
-            }
+            float ss = 0.f;
+#pragma unroll
+            for (int j = 0; j < MAXVW * EPVW; ++j) ss = fmaf(rv[j], rv[j], ss);
+            ss = warp_sum(ss);
+            if (lane == 0) sm.red[rb][warp][0] = ss;
             cta_sync();
-            inv = sm.inv_rms;
+            float tot = 0.f;
 #pragma unroll
-            for (int i = 0; i < MAXVW * EPVW; ++i) xw[i] *= inv;
-            if constexpr (!kSameX) {
-#pragma unroll
-                for (int i = 0; i < MAXVP * EPVP; ++i) xp_own[i] *= inv;
-            }
+            for (int w = 0; w < kConsumerWarps; ++w) tot += sm.red[rb][w][0];
+            rb ^= 1;
+            if (tid == 0 && !(tot <= 3.0e38f)) set_error(p.err, kDevCheck);   // sum of squares out of range
+            inv = 1.f / sqrtf(tot / float(d) + p.eps);
         }
-        if (!moe) {
-            // t from the fixed-point column partials
 #pragma unroll
-            for (int j = 0; j < kMaxRankTotal / kThreads; ++j) {
-                const int k = tid + kThreads * j;
-                if (k < r) put_t(k, float(double(tq[j]) * (1.0 / 4294967296.0)) * inv, r);
-            }
-            // the next layer's weight pointers, for its prefetches during this layer
-            if (tid == kThreads - 1 && l + 1 < l1) sm.exl[(l + 1) & 1][0] = p.ex[size_t(l + 1) * p.E];
-            if (tid == 0) {
-                sm.route_e[0] = predict ? p.pred_expert : 0;
-                sm.route_e[1] = 0;
-                sm.route_w[0] = 1.f;
-                sm.route_w[1] = 0.f;
-                if (p.stats && b == 0 && !predict) {
-                    p.stats[li * 4 + 2] = -1;
-                    p.stats[li * 4 + 3] = -1;
+        for (int j = 0; j < MAXVW * EPVW; ++j) xw[j] = rv[j] * inv;
+        if (lip >= 0) prof_put(p, lip, 7, gtimer());
+
+        if constexpr (moe) {
+            if (!predict) {
+                // router logits W_r x, every CTA the same in the same order;
+                // softmax over E, the two largest (ties: lower index), renormalised
+                if (rsm) {
+                    if (!stage_wait(&sm, p, vpar, bci, nullptr, &sm.vbar)) return false;
+                    vpend = false;
                 }
-            }
-            cta_sync();
-        } else {
-            // routing from the fixed-point logits, identical in every CTA:
-            // softmax over E, two largest (ties: lower index), renormalised
-            if (tid == 0) {
-                int lo = p.pred_expert, hi = 0;
-                float wlo = 1.f, whi = 0.f;
-                if (!predict) {
+                const uint8_t *R = rsm ? stg : p.router[ln];
+                float q[kMaxExperts];
+#pragma unroll
+                for (int e = 0; e < kMaxExperts; ++e) {
+                    q[e] = 0.f;
+                    if (e < p.E) {
+#pragma unroll
+                        for (int k = 0; k < MAXVW; ++k) {
+                            const int v = tid + kThreads * k;
+                            if (v < nvecW) {
+#pragma unroll
+                                for (int i = 0; i < EPVW; i += 4) {
+                                    const uint2 h = *reinterpret_cast<const uint2 *>(R + (size_t(e) * d + v * EPVW + i) * 2);
+                                    const float2 f0 = __half22float2(*reinterpret_cast<const __half2 *>(&h.x));
+                                    const float2 f1 = __half22float2(*reinterpret_cast<const __half2 *>(&h.y));
+                                    q[e] = fmaf(f0.x, xw[k * EPVW + i], q[e]);
+                                    q[e] = fmaf(f0.y, xw[k * EPVW + i + 1], q[e]);
+                                    q[e] = fmaf(f1.x, xw[k * EPVW + i + 2], q[e]);
+                                    q[e] = fmaf(f1.y, xw[k * EPVW + i + 3], q[e]);
+                                }
+                            }
+                        }
+                    }
+                }
+                const float s = warp_transpose_sum<kMaxExperts>(q);   // lane L: logit L / 2
+                if ((lane & 1) == 0 && (lane >> 1) < p.E) sm.red[rb][warp][lane >> 1] = s;
+                cta_sync();
+                if (tid == 0) {
                     float logit[kMaxExperts], pr[kMaxExperts];
-                    // every logit's load first (one round trip), then the arithmetic
-                    long long raw[kMaxExperts];
-#pragma unroll
-                    for (int e = 0; e < kMaxExperts; ++e) raw[e] = e < p.E ? __ldcg(fx + kMaxRankTotal + 1 + e) : 0;
                     float mx = -INFINITY;
-#pragma unroll
-                    for (int e = 0; e < kMaxExperts; ++e) {
-                        logit[e] = float(double(raw[e]) * (1.0 / 4294967296.0)) * inv;
-                        if (e < p.E) mx = fmaxf(mx, logit[e]);
+                    for (int e = 0; e < p.E; ++e) {
+                        float a = 0.f;
+                        for (int w = 0; w < kConsumerWarps; ++w) a += sm.red[rb][w][e];
+                        logit[e] = a;
+                        mx = fmaxf(mx, a);
                     }
                     float den = 0.f;
                     for (int e = 0; e < p.E; ++e) { pr[e] = expf(logit[e] - mx); den += pr[e]; }
@@ -877,120 +824,129 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     for (int e = 1; e < p.E; ++e) if (pr[e] > pr[ea]) ea = e;
                     int eb = ea == 0 ? 1 : 0;
                     for (int e = 0; e < p.E; ++e) if (e != ea && pr[e] > pr[eb]) eb = e;
-                    lo = min(ea, eb);
-                    hi = max(ea, eb);
-                    wlo = pr[lo] / (pr[lo] + pr[hi]);
-                    whi = pr[hi] / (pr[lo] + pr[hi]);
+                    const int lo = min(ea, eb), hi = max(ea, eb);
+                    sm.route_e[0] = lo;
+                    sm.route_e[1] = hi;
+                    sm.route_w[0] = pr[lo] / (pr[lo] + pr[hi]);
+                    sm.route_w[1] = pr[hi] / (pr[lo] + pr[hi]);
+                    sm.exl[ln & 1][0] = sm.exall[lo];
+                    sm.exl[ln & 1][1] = sm.exall[hi];
                     if (p.stats && b == 0) {
-                        p.stats[li * 4 + 2] = lo;
-                        p.stats[li * 4 + 3] = hi;
+                        p.stats[(ln - l0) * 4 + 2] = lo;
+                        p.stats[(ln - l0) * 4 + 3] = hi;
                     }
                 }
-                sm.route_e[0] = lo;
-                sm.route_e[1] = hi;
-                sm.route_w[0] = wlo;
-                sm.route_w[1] = whi;
-                for (int e = 0; e < ntop; ++e)
-                    sm.exl[l & 1][e] = predict ? p.ex[size_t(l) * p.E + lo] : sm.exall[e == 0 ? lo : hi];
+                rb ^= 1;
+            } else if (tid == 0) {
+                // the predictor call: the caller's expert
+                sm.route_e[0] = p.pred_expert;
+                sm.route_w[0] = 1.f;
+                sm.exl[ln & 1][0] = p.ex[size_t(ln) * p.E + p.pred_expert];
             }
-            // the first round of this CTA's V rows is on the critical path: its
-            // copies are issued at once (thread 0), and only then do the
-            // experts' U strips start moving towards L2 (needed after the
-            // t barrier), so that they queue behind the V rows
-            const int per = min(kRA, kStageBytes / p.vrow);
-            auto issue_vrows = [&](int row0, int n) {
-                mbar_arrive_tx(&sm.stage_bar, uint32_t(n) * p.vrow);
-                for (int rr = 0; rr < n;) {
-                    const int row = row0 + rr, e = row / r;
-                    const int cnt = min(n - rr, (e + 1) * r - row);
-                    const uint8_t *vrow = sm.exl[l & 1][e].V + size_t(row - e * r) * p.vrow;
-                    stage_copy(stg + size_t(rr) * p.vrow, vrow, uint32_t(cnt) * p.vrow, &sm.stage_bar);
-                    rr += cnt;
-                }
-            };
-            // the experts' U strips (needed after the t barrier) start moving
-            // towards L2 once the first V round has landed, so that they do not
-            // compete with it
-            auto prefetch_u = [&]() {
-                for (int e = 0; e < ntop; ++e)
-                    if (ns > 0) prefetch_l2(sm.exl[l & 1][e].U + size_t(s0) * p.urow, uint32_t(ns) * p.urow);
-            };
-            if (tid == 0) {
-                if (a1 > a0) issue_vrows(a0, min(per, a1 - a0));
-                for (int e = 0; e < ntop; ++e) {
-                    const ExpertDev &ex = sm.exl[l & 1][e];
-                    const int lo_r = max(a0 + per, e * r), hi_r = min(a1, (e + 1) * r);
-                    if (hi_r > lo_r)
-                        prefetch_l2(ex.V + size_t(lo_r - e * r) * p.vrow, uint32_t(hi_r - lo_r) * p.vrow);
-                }
-                if (a1 <= a0) prefetch_u();
-            }
-            pending = a1 > a0;
             cta_sync();
-            prof_put(p, li, 18, gtimer());
-            // t rows [a0, a1) of the two experts, staged in rounds of kRA rows
-            bool ok = true;
-            for (int row0 = a0; row0 < a1 && ok; row0 += per) {
-                const int n = min(per, a1 - row0);
-                if (tid == 0 && row0 > a0) issue_vrows(row0, n);
+            if (lip >= 0) prof_put(p, lip, 18, gtimer());
+        }
+
+        // this CTA's rows of t = V x: each thread dots its x elements with the
+        // staged rows' same elements; one transposing warp reduction per round
+        const int per = vsm ? nrows : min(kRA, (kStageBytes - rt_off) / p.vrow);
+        const int vb = vsm ? voff : rt_off;
+        for (int row0 = a0; row0 < a1; row0 += per) {
+            const int n = min(per, a1 - row0);
+            if (vsm) {
+                if (!stage_wait(&sm, p, vpar, bci, nullptr, &sm.vbar)) return false;
+                vpend = false;
+            } else {
+                if (tid == 0) issue_vrows(ln, row0, n);
                 pending = true;
-                if (!stage_wait(&sm, p, spar, bci)) { ok = false; break; }
+                if (!stage_wait(&sm, p, spar, bci)) return false;
                 pending = false;
-                if (row0 == a0) prof_put(p, li, 19, gtimer());
-                if (tid == 0 && row0 == a0) prefetch_u();
-                float part[kRA];
+                // routed: the experts' U strips (needed after the barrier) move
+                // towards L2 once the first V rows have landed
+                if (moe && row0 == a0 && tid == 0)
+                    for (int e = 0; e < ntop; ++e)
+                        if (ns > 0) prefetch_l2(sm.exl[ln & 1][e].U + size_t(s0) * p.urow, uint32_t(ns) * p.urow);
+            }
+            if (row0 == a0 && lip >= 0) prof_put(p, lip, 19, gtimer());
+            float part[kRA];
 #pragma unroll
-                for (int rr = 0; rr < kRA; ++rr) {
-                    part[rr] = 0.f;
-                    if (rr < n) {
+            for (int rr = 0; rr < kRA; ++rr) {
+                part[rr] = 0.f;
+                if (rr < n) {
+                    const uint8_t *row = stg + vb + size_t(rr) * p.vrow;
 #pragma unroll
-                        for (int k = 0; k < MAXVP; ++k) {
-                            const int v = tid + kThreads * k;
-                            if (v < nvecP) {
-                                float w[EPVP];
-                                cvt<PF>(*reinterpret_cast<const VP *>(stg + size_t(rr) * p.vrow + v * VBP), w);
+                    for (int k = 0; k < MAXVW; ++k) {
+                        const int v = tid + kThreads * k;
+                        if (v < nvecW) {
+                            float w[EPVW];
+                            ld_pf(row, v * EPVW, w);
 #pragma unroll
-                                for (int i = 0; i < EPVP; ++i) part[rr] = fmaf(w[i], XP(k * EPVP + i), part[rr]);
-                            }
+                            for (int i = 0; i < EPVW; ++i) part[rr] = fmaf(w[i], xw[k * EPVW + i], part[rr]);
                         }
                     }
                 }
-#pragma unroll
-                for (int rr = 0; rr < kRA; ++rr) {
-                    if (rr < n) {
-                        const float v = warp_sum(part[rr]);
-                        if (lane == 0) sm.red[rb][warp][rr] = v;
-                    }
-                }
-                cta_sync();
-                if (tid < n) {
-                    float t = 0.f;
-                    for (int w = 0; w < kConsumerWarps; ++w) t += sm.red[rb][w][tid];
-                    if constexpr (PF == kI8) {
-                        const int row = row0 + tid, e = row / r;
-                        t *= __ldg(sm.exl[l & 1][e].sV + (row - e * r));
-                    }
-                    __stcg(p.t_buf + row0 + tid, t);
-                }
-                rb ^= 1;
             }
-            if (!ok) break;
-            prof_put(p, li, 20, gtimer());
-            // round 0 of the first expert's U strip lands during the barrier
-            // (issued after the arrival, whose release would wait for it)
-            grid_arrive(p, epoch);
-            if (warp == 0 && ns > 0) stage_u(sm.exl[l & 1][0], 0, min(ns, ucap));
-            staged_early = pending = ns > 0;
-            if (!grid_wait(&sm, p, epoch, bci, &cyc_bar)) break;
-            prof_put(p, li, 21, gtimer());
-            for (int k = tid; k < ntop * r; k += kThreads) put_t(k, __ldcg(p.t_buf + k), ntop * r);
-        }
-        if constexpr (moe) {
-            for (int e = 0; e < ntop; ++e)
-                for (int i = tid; i < ns; i += kThreads)
-                    sm.cbuf[e][i] = __ldg(sm.exl[l & 1][e].c + s0 + i);
+            const float s = warp_transpose_sum<kRA>(part);   // lane L: row L / 2 of the round
+            if ((lane & 1) == 0 && (lane >> 1) < n) sm.red[rb][warp][lane >> 1] = s;
             cta_sync();
+            if (tid < n) {
+                float t = 0.f;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) t += sm.red[rb][w][tid];
+                if constexpr (PF == kI8) {
+                    const int row = row0 + tid, e = row / r;
+                    t *= __ldg(sm.exl[ln & 1][e].sV + (row - e * r));
+                }
+                __stcg(p.t_buf + row0 + tid, t);
+            }
+            rb ^= 1;
         }
+        if (lip >= 0) prof_put(p, lip, 5, gtimer());
+        // the first U round of layer ln (or the piece of it that waited for
+        // the V rows' space) lands during the barrier; issued after the
+        // arrival, whose release would otherwise wait for the copies
+        grid_arrive(p, epoch);
+        if (ns > 0 && warp == 0) {
+            if (vsm) {
+                if (upart2) stage_u_at(sm.exl[ln & 1][0], ufirst, u_round0 - ufirst, ufirst, true);
+            } else {
+                stage_u(sm.exl[ln & 1][0], 0, min(ns, ucap));
+                if (!moe && lane == 0 && ns > ucap)
+                    prefetch_l2(sm.exl[ln & 1][0].U + size_t(s0 + ucap) * p.urow, uint32_t(ns - ucap) * p.urow);
+            }
+        }
+        if (vsm) upart2 = false;
+        else if (ns > 0) staged_early = pending = true;
+        return grid_wait(&sm, p, epoch, bci, cycb);
+    };
+
+    // prologue: the first layer's input, routing and t
+    long long cyc0 = 0;
+    const bool started = form_input(l0 - 1, l0, &cyc0);
+
+    for (int l = l0; started && l < l1; ++l) {
+        const int li = l - l0;
+        long long cyc_a = 0, cyc_b = 0, cyc_c = 0, cyc_bar = 0;
+        prof_put(p, li, 0, gtimer());
+        const long long ca0 = clock64();
+
+        // ---------------- the layer's t and biases ---------------------------
+        for (int k = tid; k < ntop * r; k += kThreads) put_t(k, __ldcg(p.t_buf + k), ntop * r);
+        for (int e = 0; e < ntop; ++e)
+            for (int i = tid; i < ns; i += kThreads) sm.cbuf[e][i] = __ldg(sm.exl[l & 1][e].c + s0 + i);
+        // the next layer's weight pointers (dense), for its prefetches during this layer
+        if (!moe && tid == kThreads - 1 && l + 1 < l1) sm.exl[(l + 1) & 1][0] = p.ex[size_t(l + 1) * p.E];
+        // layer l - 1's fixed-point total (read before the last barrier) is
+        // cleared for layer l + 1
+        if (!predict && l + 1 < l1) {
+            unsigned long long *yz = p.yfix + size_t((l + 1) & 1) * d;
+            for (int e = c0 + tid; e < c0 + ncol; e += kThreads) yz[e] = 0ull;
+        }
+        if (!moe && tid == 0 && p.stats && b == 0 && !predict) {
+            p.stats[li * 4 + 2] = -1;
+            p.stats[li * 4 + 3] = -1;
+        }
+        cta_sync();
         cyc_a = clock64() - ca0;
         prof_put(p, li, 1, gtimer());
 
@@ -1369,12 +1325,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         const int m = sm.share_n;
         const int per_n = kSpec ? p.rec_bytes : p.gu_bytes;   // bytes per neuron in a round (its record)
         const int cap_n = min(kRound, kStageBytes / per_n);
-        // the next layer's V block and biases start moving towards L2 now
-        if (tid == kThreads - 1 && !moe && l + 1 < l1) {
-            if (ncol > 0) prefetch_l2(vblk(l + 1), uint32_t(r) * vbrow);
-            if (ns > 0) {
-                const int c_lo = s0 & ~3, c_hi = (s0 + ns + 3) & ~3;   // 16-byte aligned, padded
-                prefetch_l2(sm.exl[(l + 1) & 1][0].c + c_lo, uint32_t(c_hi - c_lo) * 4);
+        // the next layer's V rows of this CTA and biases (dense) or router
+        // rows (routed) start moving towards L2 now
+        if (tid == kThreads - 1 && l + 1 < l1) {
+            if (!moe) {
+                if (nrows > 0) prefetch_l2(sm.exl[(l + 1) & 1][0].V + size_t(a0) * p.vrow, uint32_t(nrows) * p.vrow);
+                if (ns > 0) {
+                    const int c_lo = s0 & ~3, c_hi = (s0 + ns + 3) & ~3;   // 16-byte aligned, padded
+                    prefetch_l2(sm.exl[(l + 1) & 1][0].c + c_lo, uint32_t(c_hi - c_lo) * 4);
+                }
+            } else {
+                prefetch_l2(p.router[l + 1], uint32_t(rt_bytes));
             }
         }
 
@@ -1598,65 +1559,54 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
         if (!gok) break;
         if (tid == 0 && p.stats) atomicAdd(p.stats + li * 4 + 1, nz_total);
-        // the fixed-point buffer of layer l - 1 (read before two barriers ago)
-        // is cleared for layer l + 1
-        if (b == S - 1) {
-            long long *fz = p.fix + size_t((li + 1) & 1) * kFixStride;
-            for (int i = tid; i < kFixStride; i += kThreads) fz[i] = 0;
-        }
-        // per-CTA partial of y
-#pragma unroll
-        for (int k = 0; k < MAXVW; ++k) {
-            const int v = tid + kThreads * k;
-            if (v < nvecW) {
-#pragma unroll
-                for (int i = 0; i < EPVW; i += 4)
-                    __stcg(reinterpret_cast<float4 *>(p.partials + size_t(b) * d + v * EPVW + i),
-                           make_float4(acc[k * EPVW + i], acc[k * EPVW + i + 1],
-                                       acc[k * EPVW + i + 2], acc[k * EPVW + i + 3]));
-            }
-        }
         (void)cc0;
+
+        // ---------------- y: the CTAs' partials summed in fixed point --------
+        // This CTA's partial of y as 64-bit fixed-point values at the top of
+        // the staging buffer, added into layer l's total by one bulk reduction
+        // (integer adds, so the total does not depend on their order); the
+        // arrival follows its completion.
+        {
+            unsigned long long *ys = reinterpret_cast<unsigned long long *>(stg + yoff);
+#pragma unroll
+            for (int k = 0; k < MAXVW; ++k) {
+                const int v = tid + kThreads * k;
+                if (v < nvecW) {
+#pragma unroll
+                    for (int i = 0; i < EPVW; i += 2)
+                        *reinterpret_cast<ulonglong2 *>(ys + v * EPVW + i) =
+                            make_ulonglong2(fix_q(acc[k * EPVW + i], p.err), fix_q(acc[k * EPVW + i + 1], p.err));
+                }
+            }
+            fence_proxy_async_smem();
+        }
+        cta_sync();
+        if (tid == 0) {
+            fence_proxy_async_global();
+            bulk_reduce_add_u64(p.yfix + size_t(l & 1) * d, stg + yoff, uint32_t(d) * 8u);
+            bulk_wait_all();
+            fence_proxy_async_global();
+        }
         prof_put(p, li, 3, gtimer());
         grid_arrive(p, epoch);
-        // the next layer's predictor slice starts moving once this CTA has
-        // arrived (the arrival's release would otherwise wait for these
-        // copies): the first U round straight into shared memory (free until
-        // then), the rest of the strip into L2; dense decode puts the V block
-        // for the column phase in the top of the buffer and the U round's
-        // first piece below it
-        const bool vnext = vsm && l + 1 < l1;
-        if (!moe && l + 1 < l1 && warp == 0) {
-            const ExpertDev &nx = sm.exl[(l + 1) & 1][0];
-            if (vnext && lane == 0) {
-                mbar_arrive_tx(&sm.vbar, uint32_t(vbytes));
-                stage_copy(stg + voff, vblk(l + 1), uint32_t(vbytes), &sm.vbar);
-            }
-            if (ns > 0) {
-                const int n1 = vnext ? ufirst : u_round0;
-                stage_u_at(nx, 0, n1, 0, n1 == u_round0);
-                if (lane == 0 && ns > ucap)
-                    prefetch_l2(nx.U + size_t(s0 + ucap) * p.urow, uint32_t(ns - ucap) * p.urow);
-            }
+        // the next layer's V rows and first U piece (dense) or router rows
+        // (routed) start moving once this CTA has arrived (the arrival's
+        // release would otherwise wait for these copies)
+        const bool next = l + 1 < l1;
+        if (next && warp == 0) {
+            if (vsm) stage_next_dense(l + 1);
+            if (rsm) stage_router(l + 1);
         }
-        staged_early = !moe && l + 1 < l1 && ns > 0;
-        if (staged_early) pending = true;
-        vpend = vnext;
-        upart2 = staged_early && vnext && ufirst < u_round0;
+        if (next && (vsm || rsm)) vpend = true;
+        if (next && vsm && ns > 0) {
+            staged_early = pending = true;
+            upart2 = ufirst < u_round0;
+        }
         if (!grid_wait(&sm, p, epoch, bci, &cyc_bar)) break;
         prof_put(p, li, 4, gtimer());
 
-        // ---------------- reduction + next layer's column products -----------
-        const bool next = l + 1 < l1;
-        if (!column_phase(li + 1, true, next, l + 1, li, vsm && next)) break;
-        prof_put(p, li, 5, gtimer());
-        if (next) {
-            grid_arrive(p, epoch);
-            // the V block has been read: the rest of the next U round lands there
-            if (upart2 && warp == 0) stage_u_at(sm.exl[(l + 1) & 1][0], ufirst, u_round0 - ufirst, ufirst, true);
-            upart2 = false;
-            if (!grid_wait(&sm, p, epoch, bci, &cyc_bar)) break;
-        }
+        // ---------------- the next layer's input, routing and t --------------
+        if (!form_input(l, l + 1, &cyc_bar)) break;
         prof_put(p, li, 6, gtimer());
         prof_put(p, li, 10, cyc_a);
         prof_put(p, li, 11, cyc_b);
@@ -1681,7 +1631,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 while (!mbar_test(&sm.gbar[g], (gpar >> g) & 1u) && gtimer() - t0 < p.wait_ns) {
                 }
     }
-#undef XP
 }
 
 // One instantiation per (weight format, predictor format, d_model class,

@@ -85,11 +85,11 @@ struct pi_ffn {
     const uint8_t **d_router = nullptr;
     int32_t *d_strip_off = nullptr;
     int32_t *d_grp_off = nullptr;
-    long long *fix = nullptr;
-    float *ssq = nullptr;
     // scratch
     uint8_t *scratch = nullptr;
-    float *t_buf = nullptr, *partials = nullptr, *io = nullptr;
+    float *t_buf = nullptr, *io = nullptr;
+    unsigned long long *yfix = nullptr;       // [2 d] each layer's y in fixed point, by layer parity
+    float *rbuf = nullptr;                    // [2 d] each layer's input, by layer parity
     int32_t *lists = nullptr, *counts = nullptr;
     unsigned long long *pub = nullptr;
     unsigned *bar = nullptr;
@@ -98,11 +98,10 @@ struct pi_ffn {
     int debug_flags = 0;
     long long *prof = nullptr;
     pi::PrefillState *prefill = nullptr;
-    // small-batch decode: workspace and row-major V per layer, made on first use
+    // small-batch decode: workspace and a table of the layers' V, made on first use
     uint8_t *bscratch = nullptr;
-    std::vector<uint8_t *> vrm;               // [layer]
-    std::vector<char> vrm_ok;                 // [layer]
-    const uint8_t **d_vrm = nullptr;
+    std::vector<char> vrm_ok;                 // [layer] the V table's entry is current
+    const uint8_t **d_vrm = nullptr;          // [layer] each layer's V rows
     int batch_fits = -1;                      // batch kernel co-resident with S CTAs (-1 unknown)
     int hot_k = 0;                            // records kept in HBM per strip (0 = all)
     std::vector<uint8_t *> host_mem;          // [layer * E + e] pinned cold records
@@ -221,18 +220,17 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
     h->loaded.assign(L, 0);
     h->h_ex.assign(size_t(L) * E, pi::ExpertDev{});
 
-    // scratch: t [2r] | partials [S d] | io [d] | lists [S kMaxStrip] | counts [S] | bar | err
+    // scratch: t [2r] | yfix [2d] | rbuf [2d] | io [d] | lists [S kMaxStrip] | counts [S] | pub | bar | err
     const size_t o_t = 0;
-    const size_t o_part = up256(o_t + sizeof(float) * 2 * D.rank);
-    const size_t o_io = up256(o_part + sizeof(float) * size_t(h->S) * D.d_model);
+    const size_t o_yfix = up256(o_t + sizeof(float) * 2 * D.rank);
+    const size_t o_rbuf = up256(o_yfix + sizeof(unsigned long long) * 2 * D.d_model);
+    const size_t o_io = up256(o_rbuf + sizeof(float) * 2 * D.d_model);
     const size_t o_lists = up256(o_io + sizeof(float) * D.d_model);
     const size_t o_counts = up256(o_lists + sizeof(int32_t) * size_t(h->S) * pi::kMaxStrip);
     const size_t o_pub = up256(o_counts + sizeof(int32_t) * h->S);
     const size_t o_bar = up256(o_pub + sizeof(unsigned long long) * size_t(h->S) * pi::kMaxTopK * pi::kMaxStrip);
     const size_t o_err = up256(o_bar + sizeof(unsigned) * pi::kBarWords);
-    const size_t o_fix = o_err + 256;
-    const size_t o_ssq = up256(o_fix + sizeof(long long) * 2 * pi::kFixStride);
-    const size_t total = up256(o_ssq + sizeof(float) * 2 * pi::kMaxStrips);
+    const size_t total = o_err + 256;
     cudaError_t e = cudaMalloc(&h->scratch, total);
     if (e == cudaSuccess) e = cudaMemset(h->scratch, 0, total);
     if (e == cudaSuccess) e = cudaMalloc(&h->d_ex, sizeof(pi::ExpertDev) * size_t(L) * E);
@@ -252,15 +250,14 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
         return st;
     }
     h->t_buf = reinterpret_cast<float *>(h->scratch + o_t);
-    h->partials = reinterpret_cast<float *>(h->scratch + o_part);
+    h->yfix = reinterpret_cast<unsigned long long *>(h->scratch + o_yfix);
+    h->rbuf = reinterpret_cast<float *>(h->scratch + o_rbuf);
     h->io = reinterpret_cast<float *>(h->scratch + o_io);
     h->lists = reinterpret_cast<int32_t *>(h->scratch + o_lists);
     h->counts = reinterpret_cast<int32_t *>(h->scratch + o_counts);
     h->pub = reinterpret_cast<unsigned long long *>(h->scratch + o_pub);
     h->bar = reinterpret_cast<unsigned *>(h->scratch + o_bar);
     h->err = reinterpret_cast<int *>(h->scratch + o_err);
-    h->fix = reinterpret_cast<long long *>(h->scratch + o_fix);
-    h->ssq = reinterpret_cast<float *>(h->scratch + o_ssq);
     *out = h;
     return PI_OK;
 }
@@ -278,7 +275,6 @@ void pi_ffn_destroy(pi_ffn_t h)
     cudaFree(h->d_grp_off);
     cudaFree(h->scratch);
     cudaFree(h->bscratch);
-    for (uint8_t *p : h->vrm) cudaFree(p);
     cudaFree(h->d_vrm);
     pi::prefill_destroy(h->prefill);
     delete h;
@@ -389,11 +385,8 @@ pi_status pi_ffn_load_layer(pi_ffn_t h, int layer, const pi_expert_weights *expe
         uint8_t *down_dst = hk ? full_d : m + o_d;
         PI_CUDA(cudaMemcpyAsync(d_perm, h->perm[idx].data(), sizeof(int32_t) * F,
                                 cudaMemcpyHostToDevice, st), "copy perm");
-        if (E == 1)   // dense: column blocks, one per strip (see pi_decode.cu)
-            PI_CUDA(pi::repack_v_blocks(static_cast<const uint8_t *>(w.V), m + o_V, h->d_grp_off, h->S, r, d,
-                                        elem_bytes(D.pred_dtype), st), "repack V");
-        else
-            PI_CUDA(cudaMemcpyAsync(m + o_V, w.V, size_t(r) * h->vrow, cudaMemcpyDeviceToDevice, st), "copy V");
+        // V row-major: each CTA reads its rows of t
+        PI_CUDA(cudaMemcpyAsync(m + o_V, w.V, size_t(r) * h->vrow, cudaMemcpyDeviceToDevice, st), "copy V");
         if (h->u_swz) {
             PI_CUDA(pi::repack_u_swizzled(m + o_U, d_perm, F, static_cast<const uint8_t *>(w.U), h->urow,
                                           h->d_strip_off, h->S, st), "repack U");
@@ -517,8 +510,6 @@ static pi::DecodeParams base_params(pi_ffn_t h)
     p.router = h->d_router;
     p.strip_off = h->d_strip_off;
     p.grp_off = h->d_grp_off;
-    p.fix = h->fix;
-    p.ssq = h->ssq;
     p.d = D.d_model;
     p.F = D.d_ff;
     p.r = D.rank;
@@ -538,7 +529,8 @@ static pi::DecodeParams base_params(pi_ffn_t h)
     p.wd_stride = h->spec ? p.rec_bytes : h->wrow;
     p.u_swz = h->u_swz;
     p.t_buf = h->t_buf;
-    p.partials = h->partials;
+    p.yfix = h->yfix;
+    p.rbuf = h->rbuf;
     p.lists = h->lists;
     p.counts = h->counts;
     p.pub = h->pub;
@@ -573,7 +565,6 @@ pi_status pi_predict(pi_ffn_t h, int layer, int expert, const float *x_dev, int3
     p.idx_out = idx_dev;
     p.count_out = count_dev;
     PI_CUDA(cudaMemsetAsync(h->bar, 0, sizeof(unsigned) * pi::kBarWords, st), "memset barrier");
-    PI_CUDA(cudaMemsetAsync(h->fix, 0, sizeof(long long) * 2 * pi::kFixStride, st), "memset accumulators");
     PI_CUDA(pi::launch_decode(h->wfmt, h->pfmt, p, st), "launch predict");
     return PI_OK;
 }
@@ -602,7 +593,6 @@ pi_status pi_sparse_ffn_decode(pi_ffn_t h, int layer_begin, int layer_end, float
     p.stats = stats_dev;
     p.masks = mask_dev;
     PI_CUDA(cudaMemsetAsync(h->bar, 0, sizeof(unsigned) * pi::kBarWords, st), "memset barrier");
-    PI_CUDA(cudaMemsetAsync(h->fix, 0, sizeof(long long) * 2 * pi::kFixStride, st), "memset accumulators");
     if (stats_dev) PI_CUDA(cudaMemsetAsync(stats_dev, 0, sizeof(int32_t) * 4 * nl, st), "memset stats");
     if (mask_dev)
         PI_CUDA(cudaMemsetAsync(mask_dev, 0, sizeof(uint32_t) * size_t(nl) * D.top_k * ((D.d_ff + 31) / 32), st),
@@ -657,20 +647,16 @@ pi_status pi_sparse_ffn_decode_batch(pi_ffn_t h, int layer_begin, int layer_end,
     if (!h->bscratch) {
         PI_CUDA(cudaMalloc(&h->bscratch, total), "cudaMalloc(batch workspace)");
         PI_CUDA(cudaMemset(h->bscratch, 0, total), "memset(batch workspace)");
-        h->vrm.assign(L, nullptr);
         h->vrm_ok.assign(L, 0);
         PI_CUDA(cudaMalloc(&h->d_vrm, sizeof(uint8_t *) * L), "cudaMalloc(V table)");
         PI_CUDA(cudaMemset(h->d_vrm, 0, sizeof(uint8_t *) * L), "memset(V table)");
     }
-    // row-major V of each layer of the range (made from the column blocks)
+    // the V table: each layer's V (row-major) for the range
     for (int l = layer_begin; l < layer_end; ++l) {
         if (h->vrm_ok[l]) continue;
-        if (!h->vrm[l]) PI_CUDA(cudaMalloc(&h->vrm[l], size_t(r) * h->vrow), "cudaMalloc(V rows)");
-        PI_CUDA(pi::unblock_v(h->h_ex[l].V, h->vrm[l], h->d_grp_off, S, r, d, elem_bytes(D.pred_dtype), st),
-                "unblock V");
-        const uint8_t *vp = h->vrm[l];
+        const uint8_t *vp = h->h_ex[size_t(l) * D.n_experts].V;
         PI_CUDA(cudaMemcpyAsync(h->d_vrm + l, &vp, sizeof(vp), cudaMemcpyHostToDevice, st), "V table");
-        PI_CUDA(cudaStreamSynchronize(st), "V rows sync");
+        PI_CUDA(cudaStreamSynchronize(st), "V table sync");
         h->vrm_ok[l] = 1;
     }
     const int nl = layer_end - layer_begin;
@@ -741,7 +727,6 @@ pi_status pi_sparse_ffn_decode_partial(pi_ffn_t h, int layer, const float *resid
     p.stats = stats_dev;
     p.masks = mask_dev;
     PI_CUDA(cudaMemsetAsync(h->bar, 0, sizeof(unsigned) * pi::kBarWords, st), "memset barrier");
-    PI_CUDA(cudaMemsetAsync(h->fix, 0, sizeof(long long) * 2 * pi::kFixStride, st), "memset accumulators");
     if (stats_dev) PI_CUDA(cudaMemsetAsync(stats_dev, 0, sizeof(int32_t) * 4, st), "memset stats");
     if (mask_dev)
         PI_CUDA(cudaMemsetAsync(mask_dev, 0, sizeof(uint32_t) * D.top_k * ((D.d_ff + 31) / 32), st), "memset masks");

@@ -18,7 +18,6 @@ constexpr int kMaxExperts = 16;
 constexpr int kMaxRankTotal = 2048;   // top_k * rank
 constexpr int kStageBytes = 200 * 1024;   // shared-memory staging of V rows / U strips / gathered rows
 constexpr int kMaxSliceCols = 1024;       // residual columns per CTA at most
-constexpr int kFixStride = kMaxRankTotal + 1 + kMaxExperts;   // t, (unused), router logits
 
 enum Fmt { kF32 = 0, kF16 = 1, kBF16 = 2, kI4 = 3, kI8 = 4 };   // kI8: predictor only
 
@@ -51,7 +50,8 @@ struct DecodeParams {
     const ExpertDev *ex;            // [n_layers * E]
     const uint8_t *const *router;   // [n_layers] E x d fp16, or null entries
     const int32_t *strip_off;       // [S + 1]
-    const int32_t *grp_off;         // [S + 1] column slices, in 8-column groups
+    const int32_t *grp_off;         // [S + 1] column slices, in 8-column groups (the columns
+                                    // of r, y and the trace each CTA writes)
     int d, F, r, E, top_k, act, gated, S;
     int layer_begin, layer_end;
     float threshold, eps;
@@ -72,10 +72,10 @@ struct DecodeParams {
     float *z_out;                   // predict: [F] or null
     int32_t *idx_out, *count_out;   // predict
     // scratch (library-owned or caller-provided, see pi_host.cu)
-    float *t_buf;                   // [top_k * r]
-    long long *fix;                 // [2 * kFixStride] fixed-point accumulators, zeroed
-    float *ssq;                     // [2 * kMaxStrips] per-CTA sums of squares of r, by layer parity
-    float *partials;                // [S * d]
+    float *t_buf;                   // [top_k * r] t of the next layer (each CTA writes its rows)
+    unsigned long long *yfix;       // [2 * d] decode: each layer's y summed in 64-bit fixed point
+                                    // (2^-32 units), by layer parity; the kernel clears them itself
+    float *rbuf;                    // [2 * d] decode: each layer's input r, by layer parity
     int32_t *lists;                 // [S * kMaxStrip]  (predict)
     int32_t *counts;                // [S] active count of each strip
     unsigned long long *pub;        // [S * kMaxTopK * kMaxStrip] published active entries (decode):
@@ -124,10 +124,6 @@ int batch_max_blocks_per_sm(int wfmt);
 int batch_max_tokens();
 int batch_tokens_per_launch(int wfmt);   // 8 (F16), 4 (BF16: x and h as two bf16 parts)
 int batch_max_d();
-// V column blocks (the dense decode layout) back to row-major.
-cudaError_t unblock_v(const uint8_t *blk, uint8_t *vrm, const int32_t *grp_off_dev, int S, int r, int d, int eb,
-                      cudaStream_t st);
-
 // Load-time repack kernels (pi_repack.cu).  repack_rows: dst record p is the
 // concatenation of row perm[p] of each of the n_src sources (row bytes each a
 // multiple of 16).
@@ -136,8 +132,6 @@ constexpr int kMaxRepackSrc = 6;
 cudaError_t repack_rows(uint8_t *dst, const int32_t *perm, int rows, int n_src,
                         const uint8_t *const *src, const int *row_bytes, cudaStream_t s,
                         long long dst_stride = 0);
-cudaError_t repack_v_blocks(const uint8_t *V, uint8_t *dst, const int32_t *grp_off, int S, int r,
-                            int d, int elem_bytes, cudaStream_t s);
 cudaError_t repack_bias(const float *src, float *dst, const int32_t *perm, int n, cudaStream_t s);
 // Records (`bytes` each, table order) split by strip position: the first hot_k
 // of each strip to `hot`, the others to `cold` (a device-visible host buffer).

@@ -23,20 +23,18 @@ namespace {
 //   t        kMaxRankTotal floats         rows of t = V x
 //   lists    kMaxStrips * kMaxStrip ints  per-strip active lists
 //   counts   kMaxStrips ints              per-strip active counts
-//   fix      2 * kFixStride int64         fixed-point accumulators (zeroed per call)
 //   bar      kBarWords unsigned           grid barrier counters (zeroed per call)
 //   err      1 int                        device error word (zeroed per call)
-//   experts  2 ExpertDev                  weight pointers of this call
+//   experts  1 ExpertDev                  weight pointers of this call
 //   strips   kMaxStrips + 1 ints          strip offsets
 //   groups   kMaxStrips + 1 ints          column-slice offsets
 constexpr size_t kOffT = 0;
 constexpr size_t kOffLists = kOffT + sizeof(float) * pi::kMaxRankTotal;
 constexpr size_t kOffCounts = kOffLists + sizeof(int32_t) * pi::kMaxStrips * pi::kMaxStrip;
-constexpr size_t kOffFix = (kOffCounts + sizeof(int32_t) * pi::kMaxStrips + 255) & ~size_t(255);
-constexpr size_t kOffBar = kOffFix + sizeof(long long) * 2 * pi::kFixStride;
+constexpr size_t kOffBar = (kOffCounts + sizeof(int32_t) * pi::kMaxStrips + 255) & ~size_t(255);
 constexpr size_t kOffErr = kOffBar + sizeof(unsigned) * pi::kBarWords;
 constexpr size_t kOffEx = (kOffErr + sizeof(int) + 255) & ~size_t(255);
-constexpr size_t kOffStrips = kOffEx + 2 * sizeof(pi::ExpertDev);
+constexpr size_t kOffStrips = kOffEx + sizeof(pi::ExpertDev);
 constexpr size_t kOffGroups = kOffStrips + sizeof(int32_t) * (pi::kMaxStrips + 1);
 constexpr size_t kNoAllocBytes = (kOffGroups + sizeof(int32_t) * (pi::kMaxStrips + 1) + 255) & ~size_t(255);
 
@@ -57,21 +55,23 @@ pi_status na_fail(pi_status st, const char *msg)
 }
 
 // Writes the call's tables into the array and clears what must start at zero
-// (accumulators, barrier words, error word); the count reads -1 until the
+// (barrier words, error word); the count reads -1 until the
 // predictor kernel completes.
 __global__ void na_setup(unsigned char *base, const uint8_t *V, const uint8_t *U, const float *c,
                          int F, int S, int ng, int32_t *count)
 {
     const int t = threadIdx.x;
-    if (t < 2) {
+    if (t == 0) {
         pi::ExpertDev *ex = reinterpret_cast<pi::ExpertDev *>(base + kOffEx);
-        ex[t].V = V;
-        ex[t].U = U;
-        ex[t].c = c;
-        ex[t].Wgu = nullptr;
-        ex[t].Wd = nullptr;
-        ex[t].sU = nullptr;
-        ex[t].sV = nullptr;
+        ex->V = V;
+        ex->U = U;
+        ex->c = c;
+        ex->Wgu = nullptr;
+        ex->Wd = nullptr;
+        ex->sU = nullptr;
+        ex->sV = nullptr;
+        ex->Wgu_cold = nullptr;
+        ex->Wd_cold = nullptr;
     }
     int32_t *strips = reinterpret_cast<int32_t *>(base + kOffStrips);
     int32_t *groups = reinterpret_cast<int32_t *>(base + kOffGroups);
@@ -80,8 +80,8 @@ __global__ void na_setup(unsigned char *base, const uint8_t *V, const uint8_t *U
         strips[b] = b * q + (b < rem ? b : rem);
         groups[b] = int((long long)b * ng / S);
     }
-    for (size_t i = t; i < (kOffEx - kOffFix) / 4; i += blockDim.x)
-        reinterpret_cast<int *>(base + kOffFix)[i] = 0;
+    for (size_t i = t; i < (kOffEx - kOffBar) / 4; i += blockDim.x)
+        reinterpret_cast<int *>(base + kOffBar)[i] = 0;
     if (t == 0) *count = -1;
 }
 
@@ -150,9 +150,8 @@ extern "C" PI_API pi_status pi_predict_noalloc(int d_model, int d_ff, int rank, 
     if (e != cudaSuccess) return na_fail(PI_ERR_CUDA, cudaGetErrorString(e));
 
     pi::DecodeParams p{};
-    // The predictor's row-split path (V row-major) is the one the decode
-    // kernel takes for routed layers, so the call presents a two-expert layer
-    // whose experts are both this predictor, and predicts expert 0.
+    // One dense layer whose predictor is the caller's (V row-major, as the
+    // decode kernel stores it); its FFN weights are never read.
     p.ex = reinterpret_cast<const pi::ExpertDev *>(base + kOffEx);
     p.router = nullptr;
     p.strip_off = reinterpret_cast<const int32_t *>(base + kOffStrips);
@@ -160,8 +159,8 @@ extern "C" PI_API pi_status pi_predict_noalloc(int d_model, int d_ff, int rank, 
     p.d = d_model;
     p.F = d_ff;
     p.r = rank;
-    p.E = 2;
-    p.top_k = 2;
+    p.E = 1;
+    p.top_k = 1;
     p.act = PI_ACT_REGLU;
     p.gated = 1;
     p.S = S;
@@ -184,10 +183,8 @@ extern "C" PI_API pi_status pi_predict_noalloc(int d_model, int d_ff, int rank, 
     p.idx_out = idx_dev;
     p.count_out = count_dev;
     p.t_buf = reinterpret_cast<float *>(base + kOffT);
-    p.partials = nullptr;   // not touched in predictor mode
     p.lists = reinterpret_cast<int32_t *>(base + kOffLists);
     p.counts = reinterpret_cast<int32_t *>(base + kOffCounts);
-    p.fix = reinterpret_cast<long long *>(base + kOffFix);
     p.bar = reinterpret_cast<unsigned *>(base + kOffBar);
     p.err = reinterpret_cast<int *>(base + kOffErr);
     p.wait_ns = 2000000000LL;

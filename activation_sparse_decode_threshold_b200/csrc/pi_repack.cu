@@ -84,32 +84,6 @@ __global__ void k_down_transpose(const T *__restrict__ w, T *__restrict__ dst,
     }
 }
 
-// V (r x d, row-major) -> column blocks: block b holds rows 0..r-1 of the
-// columns [8 grp_off[b], 8 grp_off[b+1]) and starts at element r * 8 grp_off[b].
-__global__ void k_v_blocks(const uint8_t *__restrict__ V, uint8_t *__restrict__ dst,
-                           const int32_t *__restrict__ grp_off, int S, int r, int d, int eb)
-{
-    const int ng = d / 8;
-    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= (long long)r * ng) return;
-    const int k = int(idx / ng), g = int(idx % ng);
-    int lo = 0, hi = S - 1;                 // owner: last b with grp_off[b] <= g
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) / 2;
-        if (grp_off[mid] <= g) lo = mid;
-        else hi = mid - 1;
-    }
-    const int b = lo, g0 = grp_off[b], nb = grp_off[b + 1] - g0;
-    const long long o = (long long)r * 8 * g0 + (long long)k * 8 * nb + 8LL * (g - g0);
-    if (eb == 1) {   // 8 signed bytes: one 8-byte word
-        *reinterpret_cast<uint2 *>(dst + o) = *reinterpret_cast<const uint2 *>(V + (long long)k * d + 8LL * g);
-        return;
-    }
-    const uint4 *s = reinterpret_cast<const uint4 *>(V + ((long long)k * d + 8LL * g) * eb);
-    uint4 *t = reinterpret_cast<uint4 *>(dst + o * eb);
-    for (int i = 0; i < eb / 2; ++i) t[i] = s[i];   // 8 elements = eb/2 16-byte words
-}
-
 __global__ void k_invert(const int32_t *__restrict__ perm, int32_t *__restrict__ inv, int n)
 {
     const int p = blockIdx.x * blockDim.x + threadIdx.x;
@@ -143,14 +117,6 @@ cudaError_t split_records(const uint8_t *src, uint8_t *hot, uint8_t *cold, int F
 {
     if (F <= 0) return cudaSuccess;
     k_split_records<<<F, 128, 0, s>>>(src, hot, cold, F, bytes, strip_off, S, hot_k);
-    return cudaGetLastError();
-}
-
-cudaError_t repack_v_blocks(const uint8_t *V, uint8_t *dst, const int32_t *grp_off, int S, int r,
-                            int d, int elem_bytes, cudaStream_t s)
-{
-    const long long n = (long long)r * (d / 8);
-    k_v_blocks<<<int((n + 255) / 256), 256, 0, s>>>(V, dst, grp_off, S, r, d, elem_bytes);
     return cudaGetLastError();
 }
 

@@ -233,8 +233,9 @@ PI_API pi_status pi_sparse_ffn_decode_batch(pi_ffn_t h, int layer_begin, int lay
  *
  * pi_sparse_ffn_decode_partial runs one layer on resid_dev (the residual
  * entering the layer, [d] float, read only) and writes this handle's share of
- * y to y_dev ([d] float): RMSNorm, prediction, gather and the fixed-order
- * reduction as in pi_sparse_ffn_decode, without the residual add.  The caller
+ * y to y_dev ([d] float): RMSNorm, prediction, gather and the fixed-point
+ * merge of the CTAs' partials as in pi_sparse_ffn_decode, without the
+ * residual add.  The caller
  * sums y over the shards (an all-reduce across ranks, e.g. NCCL) and adds it
  * with pi_residual_add (resid_dev[j] += y_dev[j], j < d).  A handle holding
  * all neurons gives exactly y of pi_sparse_ffn_decode's layer.  stats_dev

@@ -243,10 +243,11 @@ def test_full_size_sampled_layers(handles, name, active):
 @pytest.mark.parametrize("scale", [1e-3, 1e3])
 def test_residual_scale_matches_oracle(handles, scale):
     """RMSNorm makes each layer's input scale-free: residuals scaled by 1e-3
-    or 1e3 still match the oracle layer by layer (the sums of squares are
-    per-CTA floats, and the predictor's fixed-point sums stay in range).
-    Far larger residuals keep the right layer inputs too, but the fp32
-    residual's own rounding then swamps a layer's increment y."""
+    or 1e3 still match the oracle layer by layer (every CTA forms the sum of
+    squares of the whole input in fp32, t comes from x, and y's fixed-point
+    total depends on x alone).  Far larger residuals keep the right layer
+    inputs too, but the fp32 residual's own rounding then swamps a layer's
+    increment y."""
     cfg = SMALL["reglu-f16"]
     h, lws = _build(cfg, handles)
     olayers = [G.oracle_layer(cfg, lw) for lw in lws]
@@ -265,13 +266,13 @@ def test_residual_scale_matches_oracle(handles, scale):
         G.record_error(f"decode/scale{scale:g}", rel_l2=rl, max_abs=ma, band=band)
 
 
-def test_residual_out_of_fixed_point_range_reports_device_check(handles):
-    """A residual so large (|r| ~ 1e12) that the predictor's fixed-point
-    partial sums could leave the int64 range is reported as a failed device
-    check, not returned as a silently wrong answer; the handle stays usable."""
+def test_residual_out_of_range_reports_device_check(handles):
+    """A residual so large (|r| ~ 1e20) that its sum of squares leaves the
+    fp32 range is reported as a failed device check, not returned as a
+    silently wrong answer; the handle stays usable."""
     cfg = SMALL["reglu-f16"]
     h, _ = _build(cfg, handles, n_layers=1)
-    r0 = (synth.token_input(cfg, 9) * 1e12).cuda()
+    r0 = (synth.token_input(cfg, 9) * 1e20).cuda()
     r = r0.clone()
     B.pi_sparse_ffn_decode(h, 0, 1, r)
     assert B.pi_sync(h) == B.PI_ERR_DEVICE_CHECK

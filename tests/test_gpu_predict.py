@@ -3,8 +3,8 @@ every predictor format and both d_model classes of the kernel, through the C
 ABI.
 
 pi_predict runs its own instantiations of the decode kernel (predictor-only
-kinds, a dense one with V in column blocks and a MoE one with V rows split
-over the CTAs), so each is checked here on its own: the active set must equal
+kinds, a dense one and a MoE one, both with the rows of t split over the
+CTAs), so each is checked here on its own: the active set must equal
 the oracle's outside the |z| < 1e-3 band and the logits must agree element by
 element.  Full-size cases use the workloads' real layer shapes in the launch
 configuration of the benchmark (one CTA per SM)."""
