@@ -72,6 +72,12 @@ __device__ __forceinline__ uint4 ldw4(const uint8_t *p)
                  : "l"(p));
     return v;
 }
+__device__ __forceinline__ uint32_t ldw1(const uint8_t *p)
+{
+    uint32_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
 __device__ __forceinline__ uint2 ldw2(const uint8_t *p)
 {
     uint2 v;
@@ -135,6 +141,10 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p)
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+__device__ __forceinline__ void red_add_u64(unsigned long long *p, unsigned long long v)
+{
+    asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
 __device__ __forceinline__ void red_release_gpu(unsigned *p, unsigned v)
 {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
@@ -149,20 +159,21 @@ __device__ __forceinline__ void st_vol(int *p, int v)
 }
 
 // ---------------------------------------------------------------------------
-// Stored formats.  A vector is 16 bytes of a row (8 bytes for INT4: 16
-// nibbles, half of a 32-element scale group).
+// Stored formats.  A vector is 16 bytes of a row (4 bytes for INT4: 8
+// nibbles, a quarter of a 32-element scale group; 8 bytes for INT8).
 // ---------------------------------------------------------------------------
 template <int F> struct Fm;
 template <> struct Fm<kF32>  { static constexpr int VB = 16, EPV = 4;  using V = uint4; };
 template <> struct Fm<kF16>  { static constexpr int VB = 16, EPV = 8;  using V = uint4; };
 template <> struct Fm<kBF16> { static constexpr int VB = 16, EPV = 8;  using V = uint4; };
-template <> struct Fm<kI4>   { static constexpr int VB = 8,  EPV = 16; using V = uint2; };
+template <> struct Fm<kI4>   { static constexpr int VB = 4,  EPV = 8;  using V = uint32_t; };   // 8 nibbles
 template <> struct Fm<kI8>   { static constexpr int VB = 8,  EPV = 8;  using V = uint2; };   // signed bytes (row scale apart)
 
 template <int F>
 __device__ __forceinline__ typename Fm<F>::V ldvec(const uint8_t *p)
 {
-    if constexpr (F == kI4 || F == kI8) return ldw2(p);
+    if constexpr (F == kI4) return ldw1(p);
+    else if constexpr (F == kI8) return ldw2(p);
     else return ldw4(p);
 }
 
@@ -196,12 +207,8 @@ __device__ __forceinline__ void cvt(const typename Fm<F>::V &v, float *o)
     } else {
         // element 2j sits in the low nibble of byte j; n - 8 is formed exactly
         // by placing n in the mantissa of 2^23 and subtracting 2^23 + 8
-        const uint32_t w[2] = {v.x, v.y};
 #pragma unroll
-        for (int i = 0; i < 2; ++i)
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                o[8 * i + j] = __uint_as_float(0x4b000000u | ((w[i] >> (4 * j)) & 0xfu)) - 8388616.0f;
+        for (int j = 0; j < 8; ++j) o[j] = __uint_as_float(0x4b000000u | ((v >> (4 * j)) & 0xfu)) - 8388616.0f;
     }
 }
 
@@ -337,6 +344,7 @@ constexpr int kRA = 16;           // V rows per staging round at most
 constexpr int kZRows = 112;       // U rows per staging round at most (a multiple of 16)
 constexpr int kMaxU = 4;          // U vectors per lane (rank <= 128 * EPV)
 constexpr int kRound = 16;        // neurons per gather round at most
+constexpr int kIssue = 32;        // neurons whose records are in flight at once at most
 static_assert(kRound <= 32, "a round's neurons are tracked in one warp ballot");
 constexpr int kRed = 2 * kRound;  // values reduced per warp at most
 
@@ -376,7 +384,7 @@ struct Smem {
     int bc[2];
     uint64_t stage_bar;                    // completion of a staging round
     uint64_t vbar;                         // completion of the V block staged for the column phase
-    uint64_t gbar[kRound / 4];             // completion of each group of four neurons of a gather round
+    uint64_t gbar[kIssue / 4];             // completion of each group of four neurons of a gather batch
     int gfail;                             // a warp's bounded wait on a group ran out
 };
 
@@ -569,14 +577,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // gather ends, they land during the reduction and its barrier); below
     // them the first `ufirst` rows of the next U strip's first round, whose
     // other rows follow once the V rows have been read.  A routed layer
-    // stages the router's rows at offset 0 when the gather ends and its V
-    // rows from rt_off on once the experts are known.
+    // stages its V rows in rounds from offset 0 once the experts are known.
     const int yoff = predict ? kStageBytes : kStageBytes - d * 8;
     const int voff = (yoff - nrows * p.vrow) & ~127;
     const bool vsm = !moe && nrows > 0 && nrows <= kRA && voff >= 0;
-    const int rt_bytes = moe ? p.E * d * 2 : 0;
-    const bool rsm = moe && !predict && rt_bytes <= yoff;
-    const int rt_off = rsm ? (rt_bytes + 127) & ~127 : 0;
     const int u_round0 = min(ns, ucap);
     const int ufirst = vsm ? min(u_round0, voff / p.urow) : u_round0;
 
@@ -587,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     bool staged_early = false;   // round 0 of the next U strip is already in flight
     bool pending = false;        // a staging round was issued and not yet waited for
     uint32_t vpar = 0;
-    bool vpend = false;          // V rows (dense) or router rows (routed) issued on vbar, not yet waited for
+    bool vpend = false;          // V rows (dense) issued on vbar, not yet waited for
     bool upart2 = false;         // the staged U round still misses its second piece
 
     // stage rows [row0, row0 + n) of an expert's U strip, contiguous, at
@@ -618,18 +622,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 prefetch_l2(nx.U + size_t(s0 + ucap) * p.urow, uint32_t(ns - ucap) * p.urow);
         }
     };
-    // routed, lane 0 of warp 0: layer ln's router rows onto vbar
-    auto stage_router = [&](int ln) {
-        if (lane == 0) {
-            mbar_arrive_tx(&sm.vbar, uint32_t(rt_bytes));
-            stage_copy(stg, p.router[ln], uint32_t(rt_bytes), &sm.vbar);
-        }
-    };
 
     if (tid == 0) {
         mbar_init(&sm.stage_bar, 1);
         mbar_init(&sm.vbar, 1);
-        for (int g = 0; g < kRound / 4; ++g) mbar_init(&sm.gbar[g], 1);
+        for (int g = 0; g < kIssue / 4; ++g) mbar_init(&sm.gbar[g], 1);
         sm.gfail = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         if (!moe) {
@@ -640,11 +637,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
     }
     __syncwarp();
-    if (warp == 0) {
-        if (vsm) stage_next_dense(l0);
-        if (rsm) stage_router(l0);
-    }
-    vpend = vsm || rsm;
+    // routed decode, warp 1: layer ln's router columns of this CTA into shared
+    // memory as floats (t's space, free between the gather and the next t)
+    const bool rts_ok = moe && !predict && p.E * ncol <= kMaxRankTotal;
+    auto load_router_cols = [&](int ln) {
+        const __half *R = reinterpret_cast<const __half *>(p.router[ln]);
+        for (int i = lane; i < p.E * ncol; i += 32) {
+            const int e = i / ncol, j = i - e * ncol;
+            sm.tsm[i] = __half2float(R[size_t(e) * d + c0 + j]);
+        }
+    };
+    if (rts_ok && warp == 1) load_router_cols(l0);
+    if (warp == 0 && vsm) stage_next_dense(l0);
+    vpend = vsm;
     if (vsm && ns > 0) {
         staged_early = pending = true;
         upart2 = ufirst < u_round0;
@@ -670,14 +675,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         for (int j = 0; j < EPVW / EPVP; ++j)
             cvt<PF>(*reinterpret_cast<const VP *>(row + size_t(e0 + j * EPVP) * PB), w + j * EPVP);
     };
-    // rows [row0, row0 + n) of layer ln's experts' V (rows of t) at staging
-    // offset rt_off, in one round on stage_bar (thread 0)
+    // rows [row0, row0 + n) of layer ln's experts' V (rows of t) at the
+    // start of the staging buffer, in one round on stage_bar (thread 0)
     auto issue_vrows = [&](int ln, int row0, int n) {
         mbar_arrive_tx(&sm.stage_bar, uint32_t(n) * p.vrow);
         for (int rr = 0; rr < n;) {
             const int row = row0 + rr, e = row / r;
             const int cnt = min(n - rr, (e + 1) * r - row);
-            stage_copy(stg + rt_off + size_t(rr) * p.vrow, sm.exl[ln & 1][e].V + size_t(row - e * r) * p.vrow,
+            stage_copy(stg + size_t(rr) * p.vrow, sm.exl[ln & 1][e].V + size_t(row - e * r) * p.vrow,
                        uint32_t(cnt) * p.vrow, &sm.stage_bar);
             rr += cnt;
         }
@@ -733,6 +738,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     rv[j] += float(double(static_cast<long long>(yq[j])) * (1.0 / 4294967296.0));
             }
         }
+        if (lip >= 0) prof_put(p, lip, 20, gtimer());
         // this CTA's columns [c0, c0 + ncol)
         if (!predict) {
             float *dst = emit ? p.y_out : (last ? p.resid : p.rbuf + size_t(ln & 1) * d);
@@ -746,6 +752,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     const int e = v * EPVW + i;
                     if (v < nvecW && e >= c0 && e < c0 + ncol) {
                         __stcg(dst + e, rv[k * EPVW + i]);
+                        if (moe) sm.rsl[e - c0] = rv[k * EPVW + i];   // for the router's share
                         if (trc) __stcg(trc + e, rv[k * EPVW + i]);
                         if (yz) yz[e] = 0ull;   // layer l0's fixed-point total starts at zero
                     }
@@ -775,68 +782,83 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 
         if constexpr (moe) {
             if (!predict) {
-                // router logits W_r x, every CTA the same in the same order;
-                // softmax over E, the two largest (ties: lower index), renormalised
-                if (rsm) {
-                    if (!stage_wait(&sm, p, vpar, bci, nullptr, &sm.vbar)) return false;
-                    vpend = false;
-                }
-                const uint8_t *R = rsm ? stg : p.router[ln];
-                float q[kMaxExperts];
+                // router logits W_r x: each CTA adds its columns' share in 64-bit
+                // fixed point (integer adds: the totals do not depend on their
+                // order); after a grid barrier every CTA reads the E totals and
+                // takes the same decision: softmax over E, the two largest
+                // (ties: lower index), renormalised
+                unsigned long long *rl = reinterpret_cast<unsigned long long *>(p.bar + kRouterWord) +
+                                         size_t(ln & 1) * kMaxExperts;
+                if (warp == 0 && ncol > 0) {
+                    const __half *R = reinterpret_cast<const __half *>(p.router[ln]);
+                    const bool staged = rts_ok;   // this CTA's router columns already in shared memory
+                    // four experts at a time; after the reduction lanes 8q .. 8q + 7
+                    // hold expert e0 + q's value
+#pragma unroll 1
+                    for (int e0 = 0; e0 < p.E; e0 += 4) {
+                        float q[4];
 #pragma unroll
-                for (int e = 0; e < kMaxExperts; ++e) {
-                    q[e] = 0.f;
-                    if (e < p.E) {
-#pragma unroll
-                        for (int k = 0; k < MAXVW; ++k) {
-                            const int v = tid + kThreads * k;
-                            if (v < nvecW) {
-#pragma unroll
-                                for (int i = 0; i < EPVW; i += 4) {
-                                    const uint2 h = *reinterpret_cast<const uint2 *>(R + (size_t(e) * d + v * EPVW + i) * 2);
-                                    const float2 f0 = __half22float2(*reinterpret_cast<const __half2 *>(&h.x));
-                                    const float2 f1 = __half22float2(*reinterpret_cast<const __half2 *>(&h.y));
-                                    q[e] = fmaf(f0.x, xw[k * EPVW + i], q[e]);
-                                    q[e] = fmaf(f0.y, xw[k * EPVW + i + 1], q[e]);
-                                    q[e] = fmaf(f1.x, xw[k * EPVW + i + 2], q[e]);
-                                    q[e] = fmaf(f1.y, xw[k * EPVW + i + 3], q[e]);
+                        for (int e = 0; e < 4; ++e) {
+                            q[e] = 0.f;
+                            if (e0 + e < p.E)
+                                for (int j = lane; j < ncol; j += 32) {
+                                    const float w = staged ? sm.tsm[(e0 + e) * ncol + j]
+                                                           : __half2float(R[size_t(e0 + e) * d + c0 + j]);
+                                    q[e] = fmaf(w, sm.rsl[j], q[e]);
                                 }
-                            }
+                        }
+                        const float s = warp_transpose_sum<4>(q);
+                        if ((lane & 7) == 0 && e0 + (lane >> 3) < p.E)
+                            red_add_u64(rl + e0 + (lane >> 3), fix_q(s * inv, p.err));
+                    }
+                }
+                if (lip >= 0) prof_put(p, lip, 22, gtimer());
+                grid_arrive(p, epoch);
+                if (!grid_wait(&sm, p, epoch, bci, cycb)) return false;
+                if (lip >= 0) prof_put(p, lip, 23, gtimer());
+                if (warp == 0) {
+                    // lane e holds expert e; the max, the sum and the two
+                    // largest probabilities (ties: lower index) by shuffles in
+                    // a fixed order, so every CTA decides the same
+                    const bool live = lane < p.E;
+                    const float lg = live ? float(double(static_cast<long long>(__ldcg(rl + lane))) * (1.0 / 4294967296.0))
+                                          : -INFINITY;
+                    float mx = lg;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                    const float ex = live ? expf(lg - mx) : 0.f;
+                    const float den = warp_sum(ex);
+                    const float pr = live ? ex / den : -1.f;
+                    auto top = [&](float v) {   // (value, lane) of the largest v, ties to the lower lane
+                        int at = lane;
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) {
+                            const float v2 = __shfl_xor_sync(0xffffffffu, v, o);
+                            const int a2 = __shfl_xor_sync(0xffffffffu, at, o);
+                            if (v2 > v || (v2 == v && a2 < at)) { v = v2; at = a2; }
+                        }
+                        return at;
+                    };
+                    const int ea = top(pr);
+                    const int eb = top(lane == ea ? -2.f : pr);
+                    const int lo = min(ea, eb), hi = max(ea, eb);
+                    const float plo = __shfl_sync(0xffffffffu, pr, lo), phi = __shfl_sync(0xffffffffu, pr, hi);
+                    if (lane == 0) {
+                        sm.route_e[0] = lo;
+                        sm.route_e[1] = hi;
+                        sm.route_w[0] = plo / (plo + phi);
+                        sm.route_w[1] = phi / (plo + phi);
+                        if (p.stats && b == 0) {
+                            p.stats[(ln - l0) * 4 + 2] = lo;
+                            p.stats[(ln - l0) * 4 + 3] = hi;
                         }
                     }
+                    // the two experts' weight pointers, one 8-byte word per lane
+                    constexpr int kW = int(sizeof(ExpertDev) / 8);
+                    if (lane < 2 * kW)
+                        reinterpret_cast<unsigned long long *>(&sm.exl[ln & 1][lane / kW])[lane % kW] =
+                            reinterpret_cast<const unsigned long long *>(&sm.exall[lane < kW ? lo : hi])[lane % kW];
                 }
-                const float s = warp_transpose_sum<kMaxExperts>(q);   // lane L: logit L / 2
-                if ((lane & 1) == 0 && (lane >> 1) < p.E) sm.red[rb][warp][lane >> 1] = s;
-                cta_sync();
-                if (tid == 0) {
-                    float logit[kMaxExperts], pr[kMaxExperts];
-                    float mx = -INFINITY;
-                    for (int e = 0; e < p.E; ++e) {
-                        float a = 0.f;
-                        for (int w = 0; w < kConsumerWarps; ++w) a += sm.red[rb][w][e];
-                        logit[e] = a;
-                        mx = fmaxf(mx, a);
-                    }
-                    float den = 0.f;
-                    for (int e = 0; e < p.E; ++e) { pr[e] = expf(logit[e] - mx); den += pr[e]; }
-                    for (int e = 0; e < p.E; ++e) pr[e] /= den;
-                    int ea = 0;
-                    for (int e = 1; e < p.E; ++e) if (pr[e] > pr[ea]) ea = e;
-                    int eb = ea == 0 ? 1 : 0;
-                    for (int e = 0; e < p.E; ++e) if (e != ea && pr[e] > pr[eb]) eb = e;
-                    const int lo = min(ea, eb), hi = max(ea, eb);
-                    sm.route_e[0] = lo;
-                    sm.route_e[1] = hi;
-                    sm.route_w[0] = pr[lo] / (pr[lo] + pr[hi]);
-                    sm.route_w[1] = pr[hi] / (pr[lo] + pr[hi]);
-                    sm.exl[ln & 1][0] = sm.exall[lo];
-                    sm.exl[ln & 1][1] = sm.exall[hi];
-                    if (p.stats && b == 0) {
-                        p.stats[(ln - l0) * 4 + 2] = lo;
-                        p.stats[(ln - l0) * 4 + 3] = hi;
-                    }
-                }
-                rb ^= 1;
             } else if (tid == 0) {
                 // the predictor call: the caller's expert
                 sm.route_e[0] = p.pred_expert;
@@ -849,8 +871,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 
         // this CTA's rows of t = V x: each thread dots its x elements with the
         // staged rows' same elements; one transposing warp reduction per round
-        const int per = vsm ? nrows : min(kRA, (kStageBytes - rt_off) / p.vrow);
-        const int vb = vsm ? voff : rt_off;
+        const int per = vsm ? nrows : min(kRA, kStageBytes / p.vrow);
+        const int vb = vsm ? voff : 0;
         for (int row0 = a0; row0 < a1; row0 += per) {
             const int n = min(per, a1 - row0);
             if (vsm) {
@@ -861,33 +883,39 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 pending = true;
                 if (!stage_wait(&sm, p, spar, bci)) return false;
                 pending = false;
-                // routed: the experts' U strips (needed after the barrier) move
-                // towards L2 once the first V rows have landed
-                if (moe && row0 == a0 && tid == 0)
-                    for (int e = 0; e < ntop; ++e)
-                        if (ns > 0) prefetch_l2(sm.exl[ln & 1][e].U + size_t(s0) * p.urow, uint32_t(ns) * p.urow);
             }
             if (row0 == a0 && lip >= 0) prof_put(p, lip, 19, gtimer());
-            float part[kRA];
+            // routed: the experts' U strips (needed after the barrier) start
+            // moving towards L2 once the first V rows have landed, issued by a
+            // thread that neither polls nor releases a grid barrier
+            if (moe && row0 == a0 && tid == kThreads - 32 && ns > 0)
+                for (int e = 0; e < ntop; ++e)
+                    prefetch_l2(sm.exl[ln & 1][e].U + size_t(s0) * p.urow, uint32_t(ns) * p.urow);
+            // four rows at a time; after the reduction lanes 8q .. 8q + 7 hold
+            // row g + q of the round
+#pragma unroll 1
+            for (int g = 0; g < n; g += 4) {
+                float part[4];
 #pragma unroll
-            for (int rr = 0; rr < kRA; ++rr) {
-                part[rr] = 0.f;
-                if (rr < n) {
-                    const uint8_t *row = stg + vb + size_t(rr) * p.vrow;
+                for (int rr = 0; rr < 4; ++rr) {
+                    part[rr] = 0.f;
+                    if (g + rr < n) {
+                        const uint8_t *row = stg + vb + size_t(g + rr) * p.vrow;
 #pragma unroll
-                    for (int k = 0; k < MAXVW; ++k) {
-                        const int v = tid + kThreads * k;
-                        if (v < nvecW) {
-                            float w[EPVW];
-                            ld_pf(row, v * EPVW, w);
+                        for (int k = 0; k < MAXVW; ++k) {
+                            const int v = tid + kThreads * k;
+                            if (v < nvecW) {
+                                float w[EPVW];
+                                ld_pf(row, v * EPVW, w);
 #pragma unroll
-                            for (int i = 0; i < EPVW; ++i) part[rr] = fmaf(w[i], xw[k * EPVW + i], part[rr]);
+                                for (int i = 0; i < EPVW; ++i) part[rr] = fmaf(w[i], xw[k * EPVW + i], part[rr]);
+                            }
                         }
                     }
                 }
+                const float s = warp_transpose_sum<4>(part);
+                if ((lane & 7) == 0 && g + (lane >> 3) < n) sm.red[rb][warp][g + (lane >> 3)] = s;
             }
-            const float s = warp_transpose_sum<kRA>(part);   // lane L: row L / 2 of the round
-            if ((lane & 1) == 0 && (lane >> 1) < n) sm.red[rb][warp][lane >> 1] = s;
             cta_sync();
             if (tid < n) {
                 float t = 0.f;
@@ -920,13 +948,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         return grid_wait(&sm, p, epoch, bci, cycb);
     };
 
-    // prologue: the first layer's input, routing and t
-    long long cyc0 = 0;
-    const bool started = form_input(l0 - 1, l0, &cyc0);
-
-    for (int l = l0; started && l < l1; ++l) {
+    // Each pass forms the input of layer l + 1 and then runs that layer; the
+    // first pass (l = l0 - 1) is the prologue.  One call site keeps one copy
+    // of the input step's code.
+    long long cyc_a = 0, cyc_b = 0, cyc_c = 0, cyc_bar = 0;
+    for (int l = l0 - 1;;) {
+        // ---------------- the next layer's input, routing and t --------------
+        if (!form_input(l, l + 1, &cyc_bar)) break;
+        if (l >= l0) {
+            prof_put(p, l - l0, 6, gtimer());
+            prof_put(p, l - l0, 10, cyc_a);
+            prof_put(p, l - l0, 11, cyc_b);
+            prof_put(p, l - l0, 12, cyc_c);
+            prof_put(p, l - l0, 13, cyc_bar);
+        }
+        if (++l >= l1) break;
         const int li = l - l0;
-        long long cyc_a = 0, cyc_b = 0, cyc_c = 0, cyc_bar = 0;
+        cyc_a = cyc_b = cyc_c = cyc_bar = 0;
         prof_put(p, li, 0, gtimer());
         const long long ca0 = clock64();
 
@@ -942,6 +980,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             unsigned long long *yz = p.yfix + size_t((l + 1) & 1) * d;
             for (int e = c0 + tid; e < c0 + ncol; e += kThreads) yz[e] = 0ull;
         }
+        // routed: layer l - 1's router totals (read before the last barrier)
+        // are cleared for layer l + 1
+        if (moe && !predict && b == 0 && tid < kMaxExperts && l + 1 < l1)
+            reinterpret_cast<unsigned long long *>(p.bar + kRouterWord)[size_t((l + 1) & 1) * kMaxExperts + tid] = 0ull;
         if (!moe && tid == 0 && p.stats && b == 0 && !predict) {
             p.stats[li * 4 + 2] = -1;
             p.stats[li * 4 + 3] = -1;
@@ -1324,7 +1366,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         const long long cc0 = clock64();
         const int m = sm.share_n;
         const int per_n = kSpec ? p.rec_bytes : p.gu_bytes;   // bytes per neuron in a round (its record)
-        const int cap_n = min(kRound, kStageBytes / per_n);
+        // records are issued in batches of up to kIssue (as many as the
+        // staging buffer holds) and consumed in rounds of up to kRound, so a
+        // round's dots overlap the later rounds' copies
+        const int cap_all = min(kIssue, kStageBytes / per_n);
+        const int cap_n = min(kRound, cap_all);
+        int jb = 0, je = 0;   // the batch in shared memory: neurons [jb, je) in slots 0 ..
+
         // the next layer's V rows of this CTA and biases (dense) or router
         // rows (routed) start moving towards L2 now
         if (tid == kThreads - 1 && l + 1 < l1) {
@@ -1334,8 +1382,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     const int c_lo = s0 & ~3, c_hi = (s0 + ns + 3) & ~3;   // 16-byte aligned, padded
                     prefetch_l2(sm.exl[(l + 1) & 1][0].c + c_lo, uint32_t(c_hi - c_lo) * 4);
                 }
-            } else {
-                prefetch_l2(p.router[l + 1], uint32_t(rt_bytes));
+            } else if (ncol > 0) {
+                // this CTA's columns of each router row (its share of the logits)
+                for (int e = 0; e < p.E; ++e)
+                    prefetch_l2(p.router[l + 1] + (size_t(e) * d + c0) * 2, uint32_t(ncol) * 2);
             }
         }
 
@@ -1351,7 +1401,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     float w[EPVW];
                     cvt<WF>(*reinterpret_cast<const VW *>(row + v * VBW), w);
                     float hs = h;
-                    if constexpr (WF == kI4) hs = h * __half2float(*reinterpret_cast<const __half *>(row + d / 2 + (v >> 1) * 2));
+                    if constexpr (WF == kI4) hs = h * __half2float(*reinterpret_cast<const __half *>(row + d / 2 + (v >> 2) * 2));
 #pragma unroll
                     for (int i = 0; i < EPVW; ++i) acc[k * EPVW + i] = fmaf(hs, w[i], acc[k * EPVW + i]);
                 }
@@ -1369,7 +1419,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     float c = 0.f;
 #pragma unroll
                     for (int i = 0; i < EPVW; ++i) c = fmaf(w[i], xw[k * EPVW + i], c);
-                    if constexpr (WF == kI4) c *= __half2float(*reinterpret_cast<const __half *>(row + d / 2 + (v >> 1) * 2));
+                    if constexpr (WF == kI4) c *= __half2float(*reinterpret_cast<const __half *>(row + d / 2 + (v >> 2) * 2));
                     a += c;
                 }
             }
@@ -1378,37 +1428,46 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 
         bool gok = true;
         int nz_total = 0;            // neurons with h != 0 so far (list order)
-        for (int j0 = 0; j0 < m && gok; j0 += cap_n) {
-            const int k = min(cap_n, m - j0);
-            const int ngr = (k + 3) / 4;   // groups of four neurons, one barrier each
-            if (warp == 0) {
-                // lane 0 announces each group's bytes (records in HBM only), then
-                // lane n copies neuron n onto its group's barrier
-                const int en_l = lane < k ? sm.glst[j0 + lane] : 0;
-                const bool hot_l = lane < k && !(unsigned(en_l) & kColdBit);
-                const unsigned hot_m = __ballot_sync(0xffffffffu, hot_l);
-                if (lane < ngr) mbar_arrive_tx(&sm.gbar[lane], uint32_t(__popc((hot_m >> (4 * lane)) & 0xfu)) * per_n);
-                __syncwarp();
-                if (hot_l) {
-                    const int e = en_l >> 24;
-                    const unsigned code = unsigned(en_l) & 0xffffffu;
-                    uint8_t *slot = stg + size_t(lane) * per_n;
-                    uint64_t *gb = &sm.gbar[lane >> 2];
-                    stage_copy(slot, exs[e]->Wgu + size_t(code) * p.rec_bytes, uint32_t(per_n), gb);
+        for (int j0 = 0, k = 0; j0 < m && gok; j0 += k) {
+            if (j0 == je) {
+                // the next batch: neurons [j0, je) into slots 0 .. je - j0 - 1
+                jb = j0;
+                je = min(m, j0 + cap_all);
+                const int kb = je - jb;
+                const int ngb = (kb + 3) / 4;   // groups of four neurons, one barrier each
+                if (warp == 0) {
+                    // lane 0 announces each group's bytes (records in HBM only), then
+                    // lane n copies neuron n onto its group's barrier
+                    const int en_l = lane < kb ? sm.glst[jb + lane] : 0;
+                    const bool hot_l = lane < kb && !(unsigned(en_l) & kColdBit);
+                    const unsigned hot_m = __ballot_sync(0xffffffffu, hot_l);
+                    if (lane < ngb)
+                        mbar_arrive_tx(&sm.gbar[lane], uint32_t(__popc((hot_m >> (4 * lane)) & 0xfu)) * per_n);
+                    __syncwarp();
+                    if (hot_l) {
+                        const int e = en_l >> 24;
+                        const unsigned code = unsigned(en_l) & 0xffffffu;
+                        uint8_t *slot = stg + size_t(lane) * per_n;
+                        uint64_t *gb = &sm.gbar[lane >> 2];
+                        stage_copy(slot, exs[e]->Wgu + size_t(code) * p.rec_bytes, uint32_t(per_n), gb);
+                    }
                 }
-            }
-            if (p.hot_k) {
-                // records in host memory: every thread copies pieces of them
-                for (int n = 0; n < k; ++n) {
-                    const int en = sm.glst[j0 + n];
-                    if (!(unsigned(en) & kColdBit)) continue;
-                    const unsigned idx = unsigned(en) & (kColdBit - 1u);
-                    copy_host_rec(stg + size_t(n) * per_n, exs[en >> 24]->Wgu_cold + size_t(idx) * p.rec_bytes, per_n,
-                                  tid, kThreads);
+                if (p.hot_k) {
+                    // records in host memory: every thread copies pieces of them
+                    for (int n = 0; n < kb; ++n) {
+                        const int en = sm.glst[jb + n];
+                        if (!(unsigned(en) & kColdBit)) continue;
+                        const unsigned idx = unsigned(en) & (kColdBit - 1u);
+                        copy_host_rec(stg + size_t(n) * per_n, exs[en >> 24]->Wgu_cold + size_t(idx) * p.rec_bytes,
+                                      per_n, tid, kThreads);
+                    }
+                    cta_sync();
                 }
-                cta_sync();
+                gpend = (1u << ngb) - 1u;
             }
-            gpend = (1u << ngr) - 1u;
+            k = min(cap_n, je - j0);
+            const int sb = j0 - jb;                                         // this round's first slot
+            const unsigned rmask = ((1u << ((k + 3) / 4)) - 1u) << (sb >> 2);   // its groups
             // dots of the round's neurons, four at a time as each group lands:
             // values 2n (gate) and 2n + 1 (up); after the reduction lanes
             // 4q .. 4q + 3 hold value q
@@ -1417,7 +1476,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 {
                     // this warp waits (bounded) for the group; every lane then
                     // observes the completed phase itself
-                    const int g = g0 >> 2;
+                    const int g = (sb + g0) >> 2;
                     const uint32_t par = (gpar >> g) & 1u;
                     bool ok = true;
                     if (lane == 0 && !mbar_test(&sm.gbar[g], par)) {
@@ -1444,7 +1503,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     v[2 * n] = 0.f;
                     v[2 * n + 1] = 0.f;
                     if (g0 + n < k) {
-                        const uint8_t *slot = stg + size_t(g0 + n) * per_n;
+                        const uint8_t *slot = stg + size_t(sb + g0 + n) * per_n;
                         v[2 * n] = dot_smem(slot);
                         if (kGated) v[2 * n + 1] = dot_smem(slot + p.wrow);
                     }
@@ -1455,8 +1514,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             }
             cta_sync();
             if (sm.gfail) { gok = false; break; }
-            gpar ^= gpend;   // every group of the round completed one phase
-            gpend = 0u;
+            gpar ^= rmask;   // every group of the round completed one phase
+            gpend &= ~rmask;
             if (tid < 2 * k) {
                 float a = 0.f;
                 for (int w = 0; w < kConsumerWarps; ++w) a += sm.red[rb][w][tid];
@@ -1490,7 +1549,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 #pragma unroll
                     for (int j = 0; j < kAG; ++j) {
                         hv[j] = g0 + j < k ? sm.rh[g0 + j] : 0.f;
-                        const uint8_t *row = stg + size_t(g0 + j) * per_n + p.gu_bytes;
+                        const uint8_t *row = stg + size_t(sb + g0 + j) * per_n + p.gu_bytes;
 #pragma unroll
                         for (int kk = 0; kk < MAXVW; ++kk) {
                             const int v = tid + kThreads * kk;
@@ -1500,7 +1559,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 #pragma unroll
                     for (int j = 0; j < kAG; ++j) {
                         if (hv[j] == 0.f) continue;
-                        const uint8_t *row = stg + size_t(g0 + j) * per_n + p.gu_bytes;
+                        const uint8_t *row = stg + size_t(sb + g0 + j) * per_n + p.gu_bytes;
 #pragma unroll
                         for (int kk = 0; kk < MAXVW; ++kk) {
                             const int v = tid + kThreads * kk;
@@ -1509,7 +1568,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                                 cvt<WF>(q[j][kk], w);
                                 float hs = hv[j];
                                 if constexpr (WF == kI4)
-                                    hs *= __half2float(*reinterpret_cast<const __half *>(row + d / 2 + (v >> 1) * 2));
+                                    hs *= __half2float(*reinterpret_cast<const __half *>(row + d / 2 + (v >> 2) * 2));
 #pragma unroll
                                 for (int i = 0; i < EPVW; ++i) acc[kk * EPVW + i] = fmaf(hs, w[i], acc[kk * EPVW + i]);
                             }
@@ -1518,8 +1577,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 }
             }
             nz_total += nz_round;
-            cta_sync();   // the staging buffer is reused by the next round
+            cta_sync();   // the round's slots are reused by the next batch
         }
+        prof_put(p, li, 25, gtimer());
         // not speculative: the W_down rows of the neurons with h != 0, in rounds
         if (gok && !kSpec) {
             const int cap_d = min(kMaxTopK * kMaxStrip, kStageBytes / p.wrow);
@@ -1558,6 +1618,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             }
         }
         if (!gok) break;
+        prof_put(p, li, 26, gtimer());
+        if (rts_ok && warp == 1 && l + 1 < l1) load_router_cols(l + 1);
         if (tid == 0 && p.stats) atomicAdd(p.stats + li * 4 + 1, nz_total);
         (void)cc0;
 
@@ -1589,29 +1651,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
         prof_put(p, li, 3, gtimer());
         grid_arrive(p, epoch);
-        // the next layer's V rows and first U piece (dense) or router rows
-        // (routed) start moving once this CTA has arrived (the arrival's
-        // release would otherwise wait for these copies)
+        // the next layer's V rows and first U piece (dense) start moving once
+        // this CTA has arrived (the arrival's release would otherwise wait
+        // for these copies)
         const bool next = l + 1 < l1;
-        if (next && warp == 0) {
-            if (vsm) stage_next_dense(l + 1);
-            if (rsm) stage_router(l + 1);
-        }
-        if (next && (vsm || rsm)) vpend = true;
+        if (next && warp == 0 && vsm) stage_next_dense(l + 1);
+        if (next && vsm) vpend = true;
         if (next && vsm && ns > 0) {
             staged_early = pending = true;
             upart2 = ufirst < u_round0;
         }
         if (!grid_wait(&sm, p, epoch, bci, &cyc_bar)) break;
         prof_put(p, li, 4, gtimer());
-
-        // ---------------- the next layer's input, routing and t --------------
-        if (!form_input(l, l + 1, &cyc_bar)) break;
-        prof_put(p, li, 6, gtimer());
-        prof_put(p, li, 10, cyc_a);
-        prof_put(p, li, 11, cyc_b);
-        prof_put(p, li, 12, cyc_c);
-        prof_put(p, li, 13, cyc_bar);
     }
     // an early exit may leave one staging round in flight: let it land
     // (bounded) so no bulk copy writes this CTA's shared memory after exit
@@ -1626,7 +1677,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         if (vpend)
             while (!mbar_test(&sm.vbar, vpar) && gtimer() - t0 < p.wait_ns) {
             }
-        for (int g = 0; g < kRound / 4; ++g)
+        for (int g = 0; g < kIssue / 4; ++g)
             if ((gpend >> g) & 1u)
                 while (!mbar_test(&sm.gbar[g], (gpar >> g) & 1u) && gtimer() - t0 < p.wait_ns) {
                 }

@@ -92,9 +92,13 @@ struct DecodeParams {
 // Phase timestamps recorded per layer and CTA when DecodeParams::prof is set.
 // layer kinds (bits of the decode kernel's MODE parameter)
 constexpr int kModeMoE = 1, kModeGated = 2, kModeSpec = 4, kModePred = 8;
-// grid barrier: one arrival counter at word 0 of a zeroed area of kBarWords words
+// grid barrier: one arrival counter at word 0 of a zeroed area of kBarWords
+// words; words kRouterWord on hold the routed layers' router-logit totals
+// (2 x kMaxExperts 64-bit fixed-point values, by layer parity)
 constexpr int kBarWords = 512;
-constexpr int kProfPoints = 22;   // timestamps and cycle counters per layer and CTA
+constexpr int kRouterWord = 256;
+static_assert(kRouterWord + 4 * kMaxExperts <= kBarWords, "router totals inside the zeroed barrier area");
+constexpr int kProfPoints = 32;   // timestamps and cycle counters per layer and CTA
 
 cudaError_t launch_decode(int wfmt, int pfmt, const DecodeParams &p, cudaStream_t stream);
 int decode_max_blocks_per_sm(int wfmt, int pfmt, int d);
