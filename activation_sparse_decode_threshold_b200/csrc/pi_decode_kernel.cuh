@@ -380,6 +380,7 @@ struct Smem {
     float rsum[kRed];                      // CTA-wide dot products of a gather round
     float rh[kRound];                      // h of each neuron of a gather round
     int route_e[kMaxTopK];
+    float rlg[kMaxExperts];                // router logits of the next layer (routed)
     float route_w[kMaxTopK];
     int bc[2];
     uint64_t stage_bar;                    // completion of a staging round
@@ -817,47 +818,39 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 if (!grid_wait(&sm, p, epoch, bci, cycb)) return false;
                 if (lip >= 0) prof_put(p, lip, 23, gtimer());
                 if (warp == 0) {
-                    // lane e holds expert e; the max, the sum and the two
-                    // largest probabilities (ties: lower index) by shuffles in
-                    // a fixed order, so every CTA decides the same
-                    const bool live = lane < p.E;
-                    const float lg = live ? float(double(static_cast<long long>(__ldcg(rl + lane))) * (1.0 / 4294967296.0))
-                                          : -INFINITY;
-                    float mx = lg;
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                    const float ex = live ? expf(lg - mx) : 0.f;
-                    const float den = warp_sum(ex);
-                    const float pr = live ? ex / den : -1.f;
-                    auto top = [&](float v) {   // (value, lane) of the largest v, ties to the lower lane
-                        int at = lane;
-#pragma unroll
-                        for (int o = 16; o > 0; o >>= 1) {
-                            const float v2 = __shfl_xor_sync(0xffffffffu, v, o);
-                            const int a2 = __shfl_xor_sync(0xffffffffu, at, o);
-                            if (v2 > v || (v2 == v && a2 < at)) { v = v2; at = a2; }
-                        }
-                        return at;
-                    };
-                    const int ea = top(pr);
-                    const int eb = top(lane == ea ? -2.f : pr);
-                    const int lo = min(ea, eb), hi = max(ea, eb);
-                    const float plo = __shfl_sync(0xffffffffu, pr, lo), phi = __shfl_sync(0xffffffffu, pr, hi);
+                    // lane e reads expert e's total; lane 0 then decides in
+                    // compact loops (this code runs once per layer on one
+                    // thread, where straight-line code costs instruction fetches)
+                    if (lane < p.E)
+                        sm.rlg[lane] = float(double(static_cast<long long>(__ldcg(rl + lane))) * (1.0 / 4294967296.0));
+                    __syncwarp();
                     if (lane == 0) {
+                        float pr[kMaxExperts];
+                        float mx = -INFINITY;
+#pragma unroll 1
+                        for (int e = 0; e < p.E; ++e) mx = fmaxf(mx, sm.rlg[e]);
+                        float den = 0.f;
+#pragma unroll 1
+                        for (int e = 0; e < p.E; ++e) { pr[e] = expf(sm.rlg[e] - mx); den += pr[e]; }
+                        int ea = 0;
+#pragma unroll 1
+                        for (int e = 1; e < p.E; ++e) if (pr[e] > pr[ea]) ea = e;
+                        int eb = ea == 0 ? 1 : 0;
+#pragma unroll 1
+                        for (int e = 0; e < p.E; ++e) if (e != ea && pr[e] > pr[eb]) eb = e;
+                        const int lo = min(ea, eb), hi = max(ea, eb);
+                        const float plo = pr[lo] / den, phi = pr[hi] / den;
                         sm.route_e[0] = lo;
                         sm.route_e[1] = hi;
                         sm.route_w[0] = plo / (plo + phi);
                         sm.route_w[1] = phi / (plo + phi);
+                        sm.exl[ln & 1][0] = sm.exall[lo];
+                        sm.exl[ln & 1][1] = sm.exall[hi];
                         if (p.stats && b == 0) {
                             p.stats[(ln - l0) * 4 + 2] = lo;
                             p.stats[(ln - l0) * 4 + 3] = hi;
                         }
                     }
-                    // the two experts' weight pointers, one 8-byte word per lane
-                    constexpr int kW = int(sizeof(ExpertDev) / 8);
-                    if (lane < 2 * kW)
-                        reinterpret_cast<unsigned long long *>(&sm.exl[ln & 1][lane / kW])[lane % kW] =
-                            reinterpret_cast<const unsigned long long *>(&sm.exall[lane < kW ? lo : hi])[lane % kW];
                 }
             } else if (tid == 0) {
                 // the predictor call: the caller's expert
