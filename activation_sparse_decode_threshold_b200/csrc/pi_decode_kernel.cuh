@@ -639,13 +639,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     }
     __syncwarp();
     // routed decode, warp 1: layer ln's router columns of this CTA into shared
-    // memory as floats (t's space, free between the gather and the next t)
-    const bool rts_ok = moe && !predict && p.E * ncol <= kMaxRankTotal;
+    // memory as floats, in the upper half of the column-slice space (free from
+    // the share until the next layer's biases; the lower half takes the
+    // slice of r + y); every load is issued before any is stored
+    constexpr int kRtsOff = kMaxSliceCols / 2;
+    const bool rts_ok = moe && !predict && p.E * ncol <= kRtsOff && ncol <= kRtsOff;
     auto load_router_cols = [&](int ln) {
         const __half *R = reinterpret_cast<const __half *>(p.router[ln]);
-        for (int i = lane; i < p.E * ncol; i += 32) {
-            const int e = i / ncol, j = i - e * ncol;
-            sm.tsm[i] = __half2float(R[size_t(e) * d + c0 + j]);
+        const int n = p.E * ncol;
+        for (int i0 = 0; i0 < n; i0 += 32 * 8) {
+            __half v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = i0 + 32 * u + lane;
+                const int e = i / ncol, j = i - e * ncol;
+                v[u] = i < n ? R[size_t(e) * d + c0 + j] : __float2half(0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = i0 + 32 * u + lane;
+                if (i < n) sm.rsl[kRtsOff + i] = __half2float(v[u]);
+            }
         }
     };
     if (rts_ok && warp == 1) load_router_cols(l0);
@@ -803,7 +817,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                             q[e] = 0.f;
                             if (e0 + e < p.E)
                                 for (int j = lane; j < ncol; j += 32) {
-                                    const float w = staged ? sm.tsm[(e0 + e) * ncol + j]
+                                    const float w = staged ? sm.rsl[kRtsOff + (e0 + e) * ncol + j]
                                                            : __half2float(R[size_t(e0 + e) * d + c0 + j]);
                                     q[e] = fmaf(w, sm.rsl[j], q[e]);
                                 }
@@ -1351,6 +1365,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
         }
 
+        // routed: the next layer's router columns land during the gather
+        if (rts_ok && warp == 1 && l + 1 < l1) load_router_cols(l + 1);
         // ---------------- gather rows of active neurons ----------------------
         // Rounds of up to kRound neurons: one bulk-copy round brings their
         // W_gate/W_up records (and, when speculative, their W_down rows) into
@@ -1612,7 +1628,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
         if (!gok) break;
         prof_put(p, li, 26, gtimer());
-        if (rts_ok && warp == 1 && l + 1 < l1) load_router_cols(l + 1);
         if (tid == 0 && p.stats) atomicAdd(p.stats + li * 4 + 1, nz_total);
         (void)cc0;
 
