@@ -807,6 +807,7 @@ pi_status pi_dense_ffn_prefill(pi_ffn_t h, int layer_begin, int layer_end, int n
     if (h->hot_k) return fail(PI_ERR_UNSUPPORTED, "dense prefill needs every record in HBM (no VRAM budget)");
     PI_CUDA(cudaSetDevice(D.device), "cudaSetDevice");
     pi::PrefillView v{};
+    v.n_layers = D.n_layers;
     v.d = D.d_model;
     v.F = D.d_ff;
     v.E = D.n_experts;

@@ -48,14 +48,21 @@ constexpr int kTileRows = kHalves * BM;
 constexpr int kProducerWarps = 16, kProducers = 32 * kProducerWarps;
 constexpr int kRI = BN * 4 / kProducers;          // INT4 items (16 weights) per producer thread per stage
 constexpr int kEpiCols = BN / (kProducerWarps / 4); // accumulator columns per epilogue warp
-constexpr int kGemmThreads = kProducers + 32;    // + the MMA warp
+constexpr int kGemmThreads = kProducers + 64;    // + the MMA warp + the INT4 raw loader warp
 constexpr int kLag = 1;                          // stages between issuing a stage's copies and publishing it
-constexpr int kAhead = 7;                        // K steps between loading INT4 weights and dequantising them
-                                                 // (measured: 3 -> 474, 5 -> 497, 7 -> 500 TFLOP/s)
 constexpr int kATileBytes = BM * BK * 2;          // 16 KB
 constexpr int kBTileBytes = BN * BK * 2;          // 32 KB
 constexpr int kStageBytes = kHalves * kATileBytes + kBTileBytes;   // 64 KB
 constexpr int kGemmSmem = NSTAGE * kStageBytes + 1024;
+// INT4 weights reach shared memory by tensor-map loads, raw, kRawSlots K steps
+// ahead of their dequantisation: a gate/up stage is 256 rows x 32 bytes of
+// nibbles, a down stage 64 k-rows x 128 bytes; the gate/up scales come in
+// chunks of four K steps (256 rows x 16 bytes), the down scales per step
+// (64 k-rows x 16 bytes)
+constexpr int kRawSlots = 3;
+constexpr int kRawBytes = 8192;
+constexpr int kScaleChunk = 4096;
+constexpr int kGemmSmemI4 = kGemmSmem + kRawSlots * kRawBytes + 2 * kScaleChunk;
 constexpr int kTmemCols = kHalves * BN;           // 512: the whole tensor memory (one CTA per SM)
 constexpr int kSplitK = 4;                        // K splits of the down GEMM
 
@@ -81,6 +88,11 @@ struct GemmParams {
     // A operand: rows of list positions (normalised inputs sorted by expert for
     // the gate/up GEMM, H for the down GEMM), 64 x 128 boxes with 128-byte swizzle
     alignas(64) CUtensorMap tmA;
+    // INT4 weights of each expert, as bytes: gate/up nibbles (boxes of 32 bytes
+    // x {gate, up} x 128 neurons) and scales (16 bytes x {gate, up} x 128), or
+    // down nibbles (128 bytes x 64 k-rows, 128-byte swizzle) and scales (16 x 64)
+    alignas(64) CUtensorMap tmW[kMaxExperts];
+    alignas(64) CUtensorMap tmS[kMaxExperts];
 };
 
 // ---------------------------------------------------------------------------
@@ -144,6 +156,14 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
         ::"r"(s2u(dst)), "l"(map), "r"(x), "r"(y), "r"(s2u(bar))
+        : "memory");
+}
+// 3-D tiled TMA load of box (x, y, z) into shared memory, completion on `bar`
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int x, int y, int z, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(s2u(dst)), "l"(map), "r"(x), "r"(y), "r"(z), "r"(s2u(bar))
         : "memory");
 }
 // shared-memory matrix descriptor of a K-major tile with 128-byte swizzle (rows
@@ -270,11 +290,6 @@ template <typename T> __device__ __forceinline__ T from_f(float x);
 template <> __device__ __forceinline__ __half from_f<__half>(float x) { return __float2half_rn(x); }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
-struct RawI4 {
-    uint2 q[kRI];
-    unsigned short sc[kRI];
-};
-
 __device__ __forceinline__ void mbar_arrive(uint64_t *b)
 {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(s2u(b)) : "memory");
@@ -289,6 +304,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t full[NSTAGE], afull[NSTAGE], empty[NSTAGE], done;
+    __shared__ uint64_t rbar[kRawSlots], rfree[kRawSlots];   // INT4 raw ring: landed / consumed
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
 
@@ -331,6 +347,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
             mbar_init(&afull[s], 1);
             mbar_init(&empty[s], 1);
         }
+        for (int s = 0; s < kRawSlots; ++s) {
+            mbar_init(&rbar[s], 1);
+            mbar_init(&rfree[s], kProducers);
+        }
         mbar_init(&done, 1);
         abort_sh = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -344,6 +364,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = tmem_base_sh;
+
+    uint8_t *const raw = smem + NSTAGE * kStageBytes;
+    uint8_t *const scl = raw + kRawSlots * kRawBytes;
+    auto issue_raw = [&](int q) {   // the loader warp: stage q of this CTA's K range
+        const int slot = q % kRawSlots, kt = kt0 + q;
+        uint8_t *dst = raw + slot * kRawBytes;
+        if constexpr (KIND == kGU) {
+            const int G = p.gated ? 2 : 1;
+            const bool sc = q == 0 || (kt & 3) == 0;
+            mbar_arrive_tx(&rbar[slot], uint32_t(G * (BN / 2) * (BK / 2) + (sc ? G * (BN / 2) * 16 : 0)));
+            tma_load_3d(dst, &p.tmW[e], kt * (BK / 2), 0, n0 / 2, &rbar[slot]);
+            if (sc)
+                tma_load_3d(scl + ((kt >> 2) & 1) * kScaleChunk, &p.tmS[e], d / 2 + (kt >> 2) * 16, 0, n0 / 2,
+                            &rbar[slot]);
+        } else {
+            mbar_arrive_tx(&rbar[slot], uint32_t(kRawBytes + BK * 16));
+            tma_load_2d(dst, &p.tmW[e], n0 / 2, kt * BK, &rbar[slot]);
+            tma_load_2d(scl + slot * (BK * 16), &p.tmS[e], d / 2 + n0 / 16, kt * BK, &rbar[slot]);
+        }
+    };
 
     if (warp < kProducerWarps) {
         // ------------------------------ producers ------------------------------
@@ -387,67 +427,44 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
             }
             if constexpr (!I4) cp_async_commit();
         };
-        // INT4: the raw nibbles and scales of a stage, loaded into registers.
-        // GU item: 16 elements (chunk pair q16) of one row; the 8 lanes of each
-        // quarter-warp take 8 consecutive rows, so each of the four phases of
-        // a 16-byte shared store touches 8 different bank groups, and a row's
-        // 32 bytes come from 4 lanes.  Down item: W_down row k (8 per warp) and
-        // 16 output columns (4 consecutive groups per row).
-        // source rows of this thread's INT4 items (fixed across K steps)
-        const uint8_t *r_src[kRI];
-        int r_off[kRI];    // element offset of the item inside a K step (GU) or column offset (down)
-        bool r_ok[kRI];
-#pragma unroll
-        for (int i = 0; i < kRI; ++i) {
-            const int c = pt + kProducers * i;
-            if constexpr (KIND == kGU) {
-                const int row = (c >> 5) * 8 + (c & 7), q16 = (c >> 3) & 3;
-                const int nn = n0 / 2 + (row >> 1);
-                r_ok[i] = nn < F && (p.gated || (row & 1) == 0);
-                r_src[i] = ex.Wgu + size_t(r_ok[i] ? nn : 0) * p.rec_bytes + ((row & 1) ? p.wrow : 0);
-                r_off[i] = 16 * q16;
-            } else {
-                const int rest = c >> 5;
-                const int k = (rest & 7) * 8 + (c & 7), g16 = (rest >> 3) * 4 + ((c >> 3) & 3);
-                r_ok[i] = true;
-                r_src[i] = ex.Wd + size_t(k) * p.wd_stride;    // + k0 rows per step
-                r_off[i] = n0 + 16 * g16;
-            }
-        }
-        auto load_raw = [&](int kt, RawI4 &r) {
-            const int k0 = kt * BK;
-#pragma unroll
-            for (int i = 0; i < kRI; ++i) {
-                if constexpr (KIND == kGU) {
-                    r.q[i] = make_uint2(0u, 0u);
-                    r.sc[i] = 0;
-                    if (r_ok[i]) {
-                        const int kk = k0 + r_off[i];
-                        r.q[i] = __ldg(reinterpret_cast<const uint2 *>(r_src[i] + kk / 2));
-                        r.sc[i] = __ldg(reinterpret_cast<const unsigned short *>(r_src[i] + d / 2) + kk / 32);
-                    }
-                } else {
-                    const uint8_t *row = r_src[i] + size_t(k0) * p.wd_stride;
-                    const int nn = r_off[i];
-                    r.q[i] = __ldg(reinterpret_cast<const uint2 *>(row + nn / 2));
-                    r.sc[i] = __ldg(reinterpret_cast<const unsigned short *>(row + d / 2) + nn / 32);
-                }
-            }
-        };
-        auto store_raw = [&](const RawI4 &r, int s) {
+        // INT4: raw stages reach shared memory by tensor-map loads (the loader
+        // warp below), kRawSlots stages in flight: rbar[q % kRawSlots]
+        // completes stage q; every producer arrives on rfree[q % kRawSlots]
+        // once it has dequantised stage q, so the slot can take stage
+        // q + kRawSlots.  Gate/up item c: row c / 4 of the tile, 16 elements
+        // (c % 4) of the K step: a warp reads 256 contiguous raw bytes and
+        // writes four 128-byte runs.  Down item: W_down row k (8 per warp) and
+        // 16 output columns, the raw rows in 128-byte swizzle so 8 rows of one
+        // column chunk fall in 8 bank groups.
+        auto dequant_stage = [&](int q, int s) {
+            const int slot = q % kRawSlots, kt = kt0 + q;
+            const uint8_t *rw = raw + slot * kRawBytes;
             uint8_t *B = smem + s * kStageBytes + kHalves * kATileBytes;
 #pragma unroll
             for (int i = 0; i < kRI; ++i) {
                 const int c = pt + kProducers * i;
-                uint4 lo, hi;
-                dequant16(r.q[i], __ushort_as_half(r.sc[i]), lo, hi);
+                uint2 qv = make_uint2(0u, 0u);
+                unsigned short sv = 0;
                 if constexpr (KIND == kGU) {
-                    const int row = (c >> 5) * 8 + (c & 7), q16 = (c >> 3) & 3;
+                    const int row = c >> 2, q16 = c & 3;
+                    const bool ok = p.gated || (row & 1) == 0;
+                    const int rr = p.gated ? row : row >> 1;
+                    if (ok) {
+                        qv = *reinterpret_cast<const uint2 *>(rw + rr * (BK / 2) + q16 * 8);
+                        sv = *reinterpret_cast<const unsigned short *>(
+                            scl + ((kt >> 2) & 1) * kScaleChunk + rr * 16 + ((kt & 3) * 2 + (q16 >> 1)) * 2);
+                    }
+                    uint4 lo, hi;
+                    dequant16(qv, __ushort_as_half(sv), lo, hi);
                     *reinterpret_cast<uint4 *>(B + sw128_off(row, 2 * q16)) = lo;
                     *reinterpret_cast<uint4 *>(B + sw128_off(row, 2 * q16 + 1)) = hi;
                 } else {
                     const int rest = c >> 5;
                     const int k = (rest & 7) * 8 + (c & 7), g16 = (rest >> 3) * 4 + ((c >> 3) & 3);
+                    qv = *reinterpret_cast<const uint2 *>(rw + k * 128 + (((g16 >> 1) ^ (k & 7)) << 4) + (g16 & 1) * 8);
+                    sv = *reinterpret_cast<const unsigned short *>(scl + slot * (BK * 16) + k * 16 + (g16 >> 1) * 2);
+                    uint4 lo, hi;
+                    dequant16(qv, __ushort_as_half(sv), lo, hi);
                     *reinterpret_cast<uint4 *>(B + mnmaj_off(2 * g16, k)) = lo;
                     *reinterpret_cast<uint4 *>(B + mnmaj_off(2 * g16 + 1, k)) = hi;
                 }
@@ -464,40 +481,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             if (!(withhold && j == 0)) mbar_arrive(&full[j % NSTAGE]);
         };
-        // INT4 raw data of stage j is loaded kAhead steps ahead, rotating
-        // through kAhead + 1 register sets (constant indices: no dynamic indexing)
-        constexpr int kSets = kAhead + 1;
-        RawI4 rs[kSets];
-        if constexpr (I4) {
-#pragma unroll
-            for (int q = 0; q < kAhead; ++q)
-                if (q < nk) load_raw(kt0 + q, rs[q]);
-        }
         int j = 0;
         bool stop = nk == 0;
-        auto step = [&](RawI4 &cur, RawI4 &nxt) {
-            if (stop) return;
+        while (!stop) {
             const int s = j % NSTAGE;
             if (j >= NSTAGE) {
                 // the MMAs of step j - NSTAGE read this stage
                 if (!mbar_wait(&empty[s], uint32_t(((j - NSTAGE) / NSTAGE) & 1), p.err, p.wait_ns)) abort_sh = 1;
             }
-            if (abort_sh) { stop = true; return; }
+            if (abort_sh) break;
             issue_async(kt0 + j, s);
             if constexpr (I4) {
-                // dequantised synchronously: the stage is published at once
-                if (j + kAhead < nk) load_raw(kt0 + j + kAhead, nxt);
-                store_raw(cur, s);
+                if (!mbar_wait(&rbar[j % kRawSlots], uint32_t((j / kRawSlots) & 1), p.err, p.wait_ns)) {
+                    abort_sh = 1;
+                    break;
+                }
+                dequant_stage(j, s);
+                mbar_arrive(&rfree[j % kRawSlots]);
                 publish(j);
             } else if (j >= kLag) {
                 cp_async_wait<kLag>();
                 publish(j - kLag);
             }
             if (++j >= nk) stop = true;
-        };
-        while (!stop) {
-#pragma unroll
-            for (int q = 0; q < kSets; ++q) step(rs[q], rs[(q + kSets - 1) % kSets]);
         }
         // drain: publish the stages still in flight (all of them on abort too,
         // so that no copy is outstanding at exit)
@@ -507,9 +513,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
         }
         // no tensor-map load may still be writing this CTA's shared memory at
         // exit: the issuing thread waits (bounded) for the last loads it issued
-        if (pt == 0)
+        if (pt == 0) {
             for (int q = max(0, j - NSTAGE); q < j; ++q)
                 mbar_wait(&afull[q % NSTAGE], uint32_t((q / NSTAGE) & 1), p.err, p.wait_ns);
+        }
         // epilogue: wait for the accumulator
         if (nk > 0 && !abort_sh && !mbar_wait(&done, 0u, p.err, p.wait_ns)) abort_sh = 1;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -588,6 +595,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
             }
         }
         __syncwarp();
+    }
+    if (I4 && warp == kProducerWarps + 1 && lane == 0) {
+        // ------------------------------ INT4 raw loader ------------------------------
+        // stage q's nibbles and scales start moving as soon as its slot is free
+        int issued = 0;
+        for (int q = 0; q < nk && !abort_sh; ++q) {
+            if (q >= kRawSlots &&
+                !mbar_wait(&rfree[q % kRawSlots], uint32_t(((q - kRawSlots) / kRawSlots) & 1), p.err, p.wait_ns)) {
+                abort_sh = 1;
+                break;
+            }
+            issue_raw(q);
+            issued = q + 1;
+        }
+        // no tensor-map load may still be writing this CTA's shared memory at
+        // exit: the last loads issued land (bounded)
+        for (int q = max(0, issued - kRawSlots); q < issued; ++q)
+            mbar_wait(&rbar[q % kRawSlots], uint32_t((q / kRawSlots) & 1), p.err, p.wait_ns);
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
@@ -806,6 +831,11 @@ struct PrefillState {
     int T = 0, d = 0, F = 0;
     uint8_t *buf = nullptr;
     size_t bytes = 0;
+    // INT4 weight tensor maps per layer and expert: gate/up nibbles, gate/up
+    // scales, down nibbles, down scales (encoded on first use, dropped when the
+    // layer is reloaded)
+    std::vector<CUtensorMap> wmaps;
+    std::vector<char> wmaps_ok;
 };
 
 static size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -851,8 +881,9 @@ int prefill_run(PrefillState **state, const PrefillView &v, int l0, int l1, int 
     void (*gu)(GemmParams) = W == 0 ? k_gemm<kGU, 0> : (W == 1 ? k_gemm<kGU, 1> : k_gemm<kGU, 2>);
     void (*dn)(GemmParams) = W == 0 ? k_gemm<kDOWN, 0> : (W == 1 ? k_gemm<kDOWN, 1> : k_gemm<kDOWN, 2>);
     // per device and kernel; cheap enough to repeat per call
-    if (cudaFuncSetAttribute(gu, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) != cudaSuccess ||
-        cudaFuncSetAttribute(dn, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) != cudaSuccess) {
+    const int smem_bytes = W == 2 ? kGemmSmemI4 : kGemmSmem;
+    if (cudaFuncSetAttribute(gu, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess ||
+        cudaFuncSetAttribute(dn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess) {
         snprintf(msg, msg_len, "prefill: cudaFuncSetAttribute: %s", cudaGetErrorString(cudaGetLastError()));
         return 2;
     }
@@ -917,6 +948,50 @@ int prefill_run(PrefillState **state, const PrefillView &v, int l0, int l1, int 
         }
     }
 
+    if (W == 2) {
+        // INT4 weights as bytes: gate/up rows {wrow bytes} x {gate, up} x F
+        // neurons (rec_bytes apart), down rows {wrow bytes} x F (wd_stride apart)
+        const TensorMapEncodeFn enc = tensor_map_encoder();
+        const size_t nl = v.n_layers;
+        if (st->wmaps.size() != nl * v.E * 4) {
+            st->wmaps.assign(nl * v.E * 4, CUtensorMap{});
+            st->wmaps_ok.assign(nl, 0);
+        }
+        const int G = v.gated ? 2 : 1;
+        for (int l = l0; l < l1; ++l) {
+            if (st->wmaps_ok[l]) continue;
+            for (int e = 0; e < v.E; ++e) {
+                const ExpertDev &x = v.ex[size_t(l) * v.E + e];
+                CUtensorMap *m = &st->wmaps[(size_t(l) * v.E + e) * 4];
+                const cuuint64_t gdim3[3] = {cuuint64_t(v.wrow), cuuint64_t(G), cuuint64_t(v.F)};
+                const cuuint64_t gstr3[2] = {cuuint64_t(v.wrow), cuuint64_t(v.rec_bytes)};
+                const cuuint32_t boxw[3] = {BK / 2, cuuint32_t(G), BN / 2}, boxs[3] = {16, cuuint32_t(G), BN / 2};
+                const cuuint32_t es3[3] = {1, 1, 1};
+                const cuuint64_t gdim2[2] = {cuuint64_t(v.wrow), cuuint64_t(v.F)};
+                const cuuint64_t gstr2[1] = {cuuint64_t(v.wd_stride)};
+                const cuuint32_t boxdw[2] = {128, BK}, boxds[2] = {16, BK};
+                const cuuint32_t es2[2] = {1, 1};
+                const CUtensorMapDataType u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+                if (enc(&m[0], u8, 3, const_cast<uint8_t *>(x.Wgu), gdim3, gstr3, boxw, es3,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+                    enc(&m[1], u8, 3, const_cast<uint8_t *>(x.Wgu), gdim3, gstr3, boxs, es3,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+                    enc(&m[2], u8, 2, const_cast<uint8_t *>(x.Wd), gdim2, gstr2, boxdw, es2,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+                    enc(&m[3], u8, 2, const_cast<uint8_t *>(x.Wd), gdim2, gstr2, boxds, es2,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+                    snprintf(msg, msg_len, "prefill: cuTensorMapEncodeTiled failed for the INT4 weights");
+                    return 2;
+                }
+            }
+            st->wmaps_ok[l] = 1;
+        }
+    }
+
     for (int l = l0; l < l1; ++l) {
         tp.router = v.E > 1 ? reinterpret_cast<const __half *>(v.router[l]) : nullptr;
         for (int e = 0; e < v.E; ++e) {
@@ -928,10 +1003,20 @@ int prefill_run(PrefillState **state, const PrefillView &v, int l0, int l1, int 
         k_gather_x<<<rows_cap, 128, 0, stream>>>(tp, B + o_xs);
         dim3 g1(2 * v.F / BN, mtiles, 1);
         gp.tmA = tm_gu;
-        gu<<<g1, kGemmThreads, kGemmSmem, stream>>>(gp);
+        if (W == 2)
+            for (int e = 0; e < v.E; ++e) {
+                gp.tmW[e] = st->wmaps[(size_t(l) * v.E + e) * 4 + 0];
+                gp.tmS[e] = st->wmaps[(size_t(l) * v.E + e) * 4 + 1];
+            }
+        gu<<<g1, kGemmThreads, smem_bytes, stream>>>(gp);
         dim3 g2(v.d / BN, mtiles, kSplitK);
         gp.tmA = tm_dn;
-        dn<<<g2, kGemmThreads, kGemmSmem, stream>>>(gp);
+        if (W == 2)
+            for (int e = 0; e < v.E; ++e) {
+                gp.tmW[e] = st->wmaps[(size_t(l) * v.E + e) * 4 + 2];
+                gp.tmS[e] = st->wmaps[(size_t(l) * v.E + e) * 4 + 3];
+            }
+        dn<<<g2, kGemmThreads, smem_bytes, stream>>>(gp);
         k_combine<<<T, 256, 0, stream>>>(tp);
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) {
@@ -942,7 +1027,10 @@ int prefill_run(PrefillState **state, const PrefillView &v, int l0, int l1, int 
     return 0;
 }
 
-void prefill_invalidate(PrefillState *, int) {}
+void prefill_invalidate(PrefillState *st, int layer)
+{
+    if (st && layer >= 0 && layer < int(st->wmaps_ok.size())) st->wmaps_ok[layer] = 0;
+}
 
 void prefill_destroy(PrefillState *state)
 {

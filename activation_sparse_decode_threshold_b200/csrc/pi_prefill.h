@@ -12,6 +12,7 @@ struct PrefillState;
 
 // What the prefill needs from a handle (weights in neuron-table order).
 struct PrefillView {
+    int n_layers;
     int d, F, E, top_k, act, gated, wfmt, wrow;
     int rec_bytes, wd_stride;                   // neuron record stride, W_down row stride (bytes)
     float eps;
