@@ -1084,7 +1084,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                         const int nks = r / 16, nmt = (n + 15) / 16;
                         const int g = lane >> 2, tq = lane & 3;
                         const uint16_t *bpart = tpart + g * ntr + e * r + 4 * tq;
-                        constexpr int kZT = MAXVW > 1 ? 4 : 8;
+                        // m-tiles per pass: eight keep a 97-row strip (F = 14336 over 148
+                        // CTAs) in one pass; the fp16-weight kernels keep six, whose
+                        // register budget their 74-row strips (F = 11008) run faster in
+                        // (measured: 2.5% per layer)
+                        constexpr int kZT = MAXVW > 1 ? 4 : (WF == kF16 ? 6 : 8);
                         for (int mt0 = 0; mt0 < nmt; mt0 += kZT) {
                             float c[kZT][4];
 #pragma unroll
@@ -1156,7 +1160,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                         const int arow = lane & 15;                       // row within an m-tile
                         const uint16_t *bpart = tpart + g * ntr + e * r + 2 * tq;
                         // m-tiles in passes of kZT (bounded accumulator registers)
-                        constexpr int kZT = MAXVW > 1 ? 4 : 8;
+                        // m-tiles per pass: eight keep a 97-row strip (F = 14336 over 148
+                        // CTAs) in one pass; the fp16-weight kernels keep six, whose
+                        // register budget their 74-row strips (F = 11008) run faster in
+                        // (measured: 2.5% per layer)
+                        constexpr int kZT = MAXVW > 1 ? 4 : (WF == kF16 ? 6 : 8);
                         for (int mt0 = 0; mt0 < nmt; mt0 += kZT) {
                             float c[kZT][4];
 #pragma unroll
