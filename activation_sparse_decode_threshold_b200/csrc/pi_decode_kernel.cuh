@@ -571,6 +571,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // multiple of 8 rows (chunk permutation keys are row mod 8)
     const int ucap_rows = min(kZRows, kStageBytes / p.urow);
     const int ucap = ns <= ucap_rows ? max(ns, 1) : (ucap_rows & ~7);
+    // routed: when both experts' strips fit the staging buffer together (an
+    // 8-bit predictor's rows), both are staged before the t barrier, the
+    // second right after the first (chunk permutation keys are relative to
+    // each strip's own first row)
+    const int u2 = ns;
+    const bool both_u = moe && !predict && p.top_k == 2 && ns > 0 && ns <= ucap && 2 * ns * p.urow <= kStageBytes;
 
     // Staging buffer at the end of a layer (decode): this CTA's partial of y
     // as fixed-point values at the top [yoff, end); below it the next layer's
@@ -944,6 +950,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         if (ns > 0 && warp == 0) {
             if (vsm) {
                 if (upart2) stage_u_at(sm.exl[ln & 1][0], ufirst, u_round0 - ufirst, ufirst, true);
+            } else if (both_u) {
+                stage_u_at(sm.exl[ln & 1][0], 0, ns, 0, false);
+                stage_u_at(sm.exl[ln & 1][1], 0, ns, u2, true);
             } else {
                 stage_u(sm.exl[ln & 1][0], 0, min(ns, ucap));
                 if (!moe && lane == 0 && ns > ucap)
@@ -1021,13 +1030,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 }
                 for (int row0 = 0; row0 < ns && ok; row0 += ucap) {
                     const int n = min(ucap, ns - row0);
-                    if (!(staged_early && row0 == 0)) {
-                        if (warp == 0) stage_u(sm.exl[l & 1][e], row0, n);
+                    // the second expert's strip landed with the first's
+                    const bool second = both_u && e == 1;
+                    const uint8_t *ust = stg + (second ? size_t(u2) * p.urow : 0);
+                    if (!second) {
+                        if (!(staged_early && row0 == 0)) {
+                            if (warp == 0) stage_u(sm.exl[l & 1][e], row0, n);
+                        }
+                        staged_early = false;
+                        pending = true;
+                        if (!stage_wait(&sm, p, spar, bci, &cyc_b)) { ok = false; break; }
+                        pending = false;
                     }
-                    staged_early = false;
-                    pending = true;
-                    if (!stage_wait(&sm, p, spar, bci, &cyc_b)) { ok = false; break; }
-                    pending = false;
                     if (e == 0 && row0 == 0) prof_put(p, li, 14, gtimer());
                     if constexpr (PF == kF32) {
                         // each warp takes rows warp, warp + 16, ...; four rows at a time,
@@ -1042,7 +1056,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                                 a[j][1] = 0.f;
                                 const int rr = rr0 + j * kConsumerWarps;
                                 if (rr < n) {
-                                    const uint8_t *urow = stg + size_t(rr) * p.urow;
+                                    const uint8_t *urow = ust + size_t(rr) * p.urow;
     #pragma unroll
                                     for (int k = 0; k < kMaxU; ++k) {
                                         const int v = lane + 32 * k;
@@ -1108,9 +1122,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                                         const int r1 = min((mt0 + t) * 16 + g + 8, n - 1);
                                         const int k0 = p.u_swz ? (r0 & 7) : 0, k1 = p.u_swz ? (r1 & 7) : 0;
                                         w[t][0] = *reinterpret_cast<const uint32_t *>(
-                                            stg + size_t(r0) * p.urow + ((ks & ~7) | ((ks ^ k0) & 7)) * 16 + 4 * tq);
+                                            ust + size_t(r0) * p.urow + ((ks & ~7) | ((ks ^ k0) & 7)) * 16 + 4 * tq);
                                         w[t][1] = *reinterpret_cast<const uint32_t *>(
-                                            stg + size_t(r1) * p.urow + ((ks & ~7) | ((ks ^ k1) & 7)) * 16 + 4 * tq);
+                                            ust + size_t(r1) * p.urow + ((ks & ~7) | ((ks ^ k1) & 7)) * 16 + 4 * tq);
                                     }
                                 }
 #pragma unroll
@@ -1176,7 +1190,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                             int arw[kZT];
 #pragma unroll
                             for (int t = 0; t < kZT; ++t) arw[t] = min((mt0 + t) * 16 + arow, n - 1);
-                            const uint32_t sbase = s2u(stg);
+                            const uint32_t sbase = s2u(ust);
                             for (int ks = warp; ks < nks; ks += kConsumerWarps) {
                                 uint32_t b0 = 0u, b1 = 0u;
                                 if (g < nparts) {
