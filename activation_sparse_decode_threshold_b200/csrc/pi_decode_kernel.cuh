@@ -366,7 +366,7 @@ struct Smem {
             float hz[kMaxTopK * kMaxStrip];    // their h (routing weight folded in)
         };
     };
-    union {                                // column phase / layer start .. active list
+    union {                                // input forming / layer start .. active list
         alignas(16) float rsl[kMaxSliceCols];  // this CTA's columns of the new residual
         struct {
             float cbuf[kMaxTopK][kMaxStrip];
@@ -384,7 +384,7 @@ struct Smem {
     float route_w[kMaxTopK];
     int bc[2];
     uint64_t stage_bar;                    // completion of a staging round
-    uint64_t vbar;                         // completion of the V block staged for the column phase
+    uint64_t vbar;                         // completion of the next layer's V rows (dense), staged after the y arrival
     uint64_t gbar[kIssue / 4];             // completion of each group of four neurons of a gather batch
     int gfail;                             // a warp's bounded wait on a group ran out
 };

@@ -27,8 +27,8 @@ enum Fmt { kF32 = 0, kF16 = 1, kBF16 = 2, kI4 = 3, kI8 = 4 };   // kI8: predicto
 // bulk copy brings everything the neuron's activation needs.  An INT4 row is
 // its d/2 nibble bytes followed by its d/32 fp16 scales.
 struct ExpertDev {
-    const uint8_t *V;    // dense: column blocks, one per CTA (block b: r rows of its
-                         // columns); MoE: r rows of vrow bytes (rank is not permuted)
+    const uint8_t *V;    // r rows of vrow bytes, row-major (rank is not permuted); each
+                         // CTA reads its own run of rows for the t phase
     const uint8_t *U;    // F rows of urow bytes, table order
     const float *c;      // F biases, table order
     const uint8_t *Wgu;  // F neuron records, table order, rec_bytes apart: gate row (+ up row)
