@@ -141,6 +141,18 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p)
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+// Tagged 64-bit slots: one strong 64-bit access moves a 32-bit value and its
+// tag together, so a reader that sees the tag it expects also sees the value.
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long *p, unsigned long long v)
+{
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *p)
+{
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
 __device__ __forceinline__ void red_add_u64(unsigned long long *p, unsigned long long v)
 {
     asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
@@ -591,6 +603,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     const int u_round0 = min(ns, ucap);
     const int ufirst = vsm ? min(u_round0, voff / p.urow) : u_round0;
 
+    // the rows of t as tagged slots (tag: the layer's index in this launch + 1)
+    unsigned long long *const tslot = reinterpret_cast<unsigned long long *>(p.bar + kTagTWord);
     unsigned epoch = 0;
     uint32_t spar = 0;
     uint32_t gpar = 0, gpend = 0;   // gather group barriers: phase parities, groups in flight
@@ -938,15 +952,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     const int row = row0 + tid, e = row / r;
                     t *= __ldg(sm.exl[ln & 1][e].sV + (row - e * r));
                 }
-                __stcg(p.t_buf + row0 + tid, t);
+                st_relaxed_u64(tslot + row0 + tid, (static_cast<unsigned long long>(ln - l0 + 1) << 32) |
+                                                       __float_as_uint(t));
             }
             rb ^= 1;
         }
         if (lip >= 0) prof_put(p, lip, 5, gtimer());
-        // the first U round of layer ln (or the piece of it that waited for
-        // the V rows' space) lands during the barrier; issued after the
-        // arrival, whose release would otherwise wait for the copies
-        grid_arrive(p, epoch);
+        // The rows of t travel as tagged slots, which every CTA polls at the
+        // layer's start: no grid barrier.  The prologue alone keeps one, so
+        // that every CTA's zeroing of layer l0's fixed-point total is ordered
+        // before any CTA's reduction into it.  The first U round of layer ln
+        // (or the piece of it that waited for the V rows' space) lands during
+        // the wait; issued after the arrival, whose release would otherwise
+        // wait for the copies.
+        const bool pbar = first && !predict;
+        if (pbar) grid_arrive(p, epoch);
         if (ns > 0 && warp == 0) {
             if (vsm) {
                 if (upart2) stage_u_at(sm.exl[ln & 1][0], ufirst, u_round0 - ufirst, ufirst, true);
@@ -961,7 +981,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
         if (vsm) upart2 = false;
         else if (ns > 0) staged_early = pending = true;
-        return grid_wait(&sm, p, epoch, bci, cycb);
+        return pbar ? grid_wait(&sm, p, epoch, bci, cycb) : true;
     };
 
     // Each pass forms the input of layer l + 1 and then runs that layer; the
@@ -985,7 +1005,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         const long long ca0 = clock64();
 
         // ---------------- the layer's t and biases ---------------------------
-        for (int k = tid; k < ntop * r; k += kThreads) put_t(k, __ldcg(p.t_buf + k), ntop * r);
         for (int e = 0; e < ntop; ++e)
             for (int i = tid; i < ns; i += kThreads) sm.cbuf[e][i] = __ldg(sm.exl[l & 1][e].c + s0 + i);
         // the next layer's weight pointers (dense), for its prefetches during this layer
@@ -1004,7 +1023,46 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             p.stats[li * 4 + 2] = -1;
             p.stats[li * 4 + 3] = -1;
         }
-        cta_sync();
+        // the rows of t: each thread polls its slots until all of them carry
+        // this layer's tag (bounded by wait_ns), then keeps the values
+        bool tok = true;
+        {
+            constexpr int kTS = kMaxRankTotal / kThreads;
+            static_assert(kTS * kThreads == kMaxRankTotal && kTS <= 32, "whole slots per thread");
+            const int nt = ntop * r;
+            const unsigned tg = unsigned(l - l0 + 1);
+            unsigned long long w[kTS];
+            unsigned need = 0;
+#pragma unroll
+            for (int i = 0; i < kTS; ++i) {
+                const int k = tid + i * kThreads;
+                w[i] = k < nt ? ld_relaxed_u64(tslot + k) : 0ull;
+                if (k < nt && unsigned(w[i] >> 32) != tg) need |= 1u << i;
+            }
+            if (need) {
+                const long long t0 = gtimer();
+                for (unsigned it = 1;; ++it) {
+#pragma unroll
+                    for (int i = 0; i < kTS; ++i)
+                        if ((need >> i) & 1u) {
+                            w[i] = ld_relaxed_u64(tslot + tid + i * kThreads);
+                            if (unsigned(w[i] >> 32) == tg) need &= ~(1u << i);
+                        }
+                    if (!need) break;
+                    if ((it & 31) == 0 && gtimer() - t0 > p.wait_ns) {
+                        set_error(p.err, kDevTimeout);
+                        tok = false;
+                        break;
+                    }
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < kTS; ++i) {
+                const int k = tid + i * kThreads;
+                if (k < nt) put_t(k, __uint_as_float(unsigned(w[i])), nt);
+            }
+        }
+        if (!__syncthreads_and(tok)) break;
         cyc_a = clock64() - ca0;
         prof_put(p, li, 1, gtimer());
 

@@ -87,7 +87,7 @@ struct pi_ffn {
     int32_t *d_grp_off = nullptr;
     // scratch
     uint8_t *scratch = nullptr;
-    float *t_buf = nullptr, *io = nullptr;
+    float *io = nullptr;
     unsigned long long *yfix = nullptr;       // [2 d] each layer's y in fixed point, by layer parity
     float *rbuf = nullptr;                    // [2 d] each layer's input, by layer parity
     int32_t *lists = nullptr, *counts = nullptr;
@@ -220,9 +220,9 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
     h->loaded.assign(L, 0);
     h->h_ex.assign(size_t(L) * E, pi::ExpertDev{});
 
-    // scratch: t [2r] | yfix [2d] | rbuf [2d] | io [d] | lists [S kMaxStrip] | counts [S] | pub | bar | err
-    const size_t o_t = 0;
-    const size_t o_yfix = up256(o_t + sizeof(float) * 2 * D.rank);
+    // scratch: yfix [2d] | rbuf [2d] | io [d] | lists [S kMaxStrip] | counts [S] | pub | bar | err
+    // (the rows of t travel in the zeroed barrier area)
+    const size_t o_yfix = 0;
     const size_t o_rbuf = up256(o_yfix + sizeof(unsigned long long) * 2 * D.d_model);
     const size_t o_io = up256(o_rbuf + sizeof(float) * 2 * D.d_model);
     const size_t o_lists = up256(o_io + sizeof(float) * D.d_model);
@@ -249,7 +249,6 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
         pi_ffn_destroy(h);
         return st;
     }
-    h->t_buf = reinterpret_cast<float *>(h->scratch + o_t);
     h->yfix = reinterpret_cast<unsigned long long *>(h->scratch + o_yfix);
     h->rbuf = reinterpret_cast<float *>(h->scratch + o_rbuf);
     h->io = reinterpret_cast<float *>(h->scratch + o_io);
@@ -528,7 +527,6 @@ static pi::DecodeParams base_params(pi_ffn_t h)
     p.rec_bytes = p.gu_bytes + (h->spec ? h->wrow : 0);
     p.wd_stride = h->spec ? p.rec_bytes : h->wrow;
     p.u_swz = h->u_swz;
-    p.t_buf = h->t_buf;
     p.yfix = h->yfix;
     p.rbuf = h->rbuf;
     p.lists = h->lists;

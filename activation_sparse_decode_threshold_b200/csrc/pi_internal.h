@@ -72,7 +72,6 @@ struct DecodeParams {
     float *z_out;                   // predict: [F] or null
     int32_t *idx_out, *count_out;   // predict
     // scratch (library-owned or caller-provided, see pi_host.cu)
-    float *t_buf;                   // [top_k * r] t of the next layer (each CTA writes its rows)
     unsigned long long *yfix;       // [2 * d] decode: each layer's y summed in 64-bit fixed point
                                     // (2^-32 units), by layer parity; the kernel clears them itself
     float *rbuf;                    // [2 * d] decode: each layer's input r, by layer parity
@@ -92,12 +91,16 @@ struct DecodeParams {
 // Phase timestamps recorded per layer and CTA when DecodeParams::prof is set.
 // layer kinds (bits of the decode kernel's MODE parameter)
 constexpr int kModeMoE = 1, kModeGated = 2, kModeSpec = 4, kModePred = 8;
-// grid barrier: one arrival counter at word 0 of a zeroed area of kBarWords
-// words; words kRouterWord on hold the routed layers' router-logit totals
-// (2 x kMaxExperts 64-bit fixed-point values, by layer parity)
-constexpr int kBarWords = 512;
+// Synchronisation area, zeroed before every launch (kBarWords 32-bit words):
+// word 0 is the grid barrier's arrival counter; words kRouterWord on hold the
+// routed layers' router-logit totals (2 x kMaxExperts 64-bit fixed-point
+// values, by layer parity); words kTagTWord on hold the rows of t as tagged
+// 64-bit slots (the value's bits in the low half, the writing layer's tag in
+// the high half).
 constexpr int kRouterWord = 256;
-static_assert(kRouterWord + 4 * kMaxExperts <= kBarWords, "router totals inside the zeroed barrier area");
+constexpr int kTagTWord = 512;
+constexpr int kBarWords = kTagTWord + 2 * kMaxRankTotal;
+static_assert(kRouterWord + 4 * kMaxExperts <= kTagTWord, "router totals inside the zeroed barrier area");
 constexpr int kProfPoints = 32;   // timestamps and cycle counters per layer and CTA
 
 cudaError_t launch_decode(int wfmt, int pfmt, const DecodeParams &p, cudaStream_t stream);

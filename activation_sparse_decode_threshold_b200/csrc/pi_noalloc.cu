@@ -20,16 +20,14 @@
 namespace {
 
 // Scratch layout (bytes), for up to kMaxStrips strips:
-//   t        kMaxRankTotal floats         rows of t = V x
 //   lists    kMaxStrips * kMaxStrip ints  per-strip active lists
 //   counts   kMaxStrips ints              per-strip active counts
-//   bar      kBarWords unsigned           grid barrier counters (zeroed per call)
+//   bar      kBarWords unsigned           grid barrier counter, tagged slots of t (zeroed per call)
 //   err      1 int                        device error word (zeroed per call)
 //   experts  1 ExpertDev                  weight pointers of this call
 //   strips   kMaxStrips + 1 ints          strip offsets
 //   groups   kMaxStrips + 1 ints          column-slice offsets
-constexpr size_t kOffT = 0;
-constexpr size_t kOffLists = kOffT + sizeof(float) * pi::kMaxRankTotal;
+constexpr size_t kOffLists = 0;
 constexpr size_t kOffCounts = kOffLists + sizeof(int32_t) * pi::kMaxStrips * pi::kMaxStrip;
 constexpr size_t kOffBar = (kOffCounts + sizeof(int32_t) * pi::kMaxStrips + 255) & ~size_t(255);
 constexpr size_t kOffErr = kOffBar + sizeof(unsigned) * pi::kBarWords;
@@ -182,7 +180,6 @@ extern "C" PI_API pi_status pi_predict_noalloc(int d_model, int d_ff, int rank, 
     p.z_out = z_dev;
     p.idx_out = idx_dev;
     p.count_out = count_dev;
-    p.t_buf = reinterpret_cast<float *>(base + kOffT);
     p.lists = reinterpret_cast<int32_t *>(base + kOffLists);
     p.counts = reinterpret_cast<int32_t *>(base + kOffCounts);
     p.bar = reinterpret_cast<unsigned *>(base + kOffBar);
