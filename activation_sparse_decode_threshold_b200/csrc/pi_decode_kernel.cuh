@@ -323,6 +323,27 @@ __device__ __forceinline__ void i8x4_to_h2(uint32_t w, uint32_t &lo, uint32_t &h
     hi = *reinterpret_cast<const uint32_t *>(&hb);
 }
 
+// Eight INT4 codes (nibble i of w = element i, value n_i - 8) as four f16x2
+// values, exactly, paired (e0, e4), (e1, e5), (e2, e6), (e3, e7): a nibble
+// in the low four bits of a half is 1024 + n in binary16, and one in bits
+// 4..7 is 1024 + 16 n, scaled by 1/16 in the same fused multiply-add that
+// takes the offset away.
+__device__ __forceinline__ void i4x8_to_h2(uint32_t w, uint32_t (&o)[4])
+{
+    const __half2 off_lo = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));   // 1032
+    const __half2 scl_hi = __halves2half2(__ushort_as_half(0x2c00), __ushort_as_half(0x2c00));   // 1/16
+    const __half2 off_hi = __halves2half2(__ushort_as_half(0xd480), __ushort_as_half(0xd480));   // -72
+    const uint32_t w8 = w >> 8;
+    const uint32_t q[4] = {(w & 0x000f000fu) | 0x64006400u, (w & 0x00f000f0u) | 0x64006400u,
+                           (w8 & 0x000f000fu) | 0x64006400u, (w8 & 0x00f000f0u) | 0x64006400u};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __half2 h = *reinterpret_cast<const __half2 *>(&q[i]);
+        const __half2 r = (i & 1) ? __hfma2(h, scl_hi, off_hi) : __hsub2(h, off_lo);
+        o[i] = *reinterpret_cast<const uint32_t *>(&r);
+    }
+}
+
 // Where a neuron's record lives.  Without a VRAM budget (hot_k = 0) every
 // record is in HBM at its table position.  With one, the first hot_k
 // positions of each strip stay in HBM, packed strip by strip (index
@@ -598,6 +619,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // other rows follow once the V rows have been read.  A routed layer
     // stages its V rows in rounds from offset 0 once the experts are known.
     const int yoff = predict ? kStageBytes : kStageBytes - d * 8;
+    // INT4 weights: x as two fp16 parts in the tensor-core B layout of the
+    // gather's dots (4d bytes at the top of the staging buffer, written after
+    // the predictor's rounds and read until the last gather round)
+    const int xpoff = kStageBytes - 4 * d;
+    const uint8_t *xp = stg + xpoff;
     const int voff = (yoff - nrows * p.vrow) & ~127;
     const bool vsm = !moe && nrows > 0 && nrows <= kRA && voff >= 0;
     const int u_round0 = min(ns, ucap);
@@ -1313,6 +1339,32 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             if (!ok) break;
         }
         prof_put(p, li, 9, gtimer());
+        if constexpr (WF == kI4) {
+            // x in the gather dots' B layout: for k-group G (32 elements) and
+            // lane quad tq, part p's four f16x2 values hold x at elements
+            // 8 tq + (0, 4), (1, 5), (2, 6), (3, 7) of the group, the pairing
+            // of i4x8_to_h2; the thread holding vector v = 4 G + tq writes them
+            if (!predict) {
+#pragma unroll
+                for (int k = 0; k < MAXVW; ++k) {
+                    const int v = tid + kThreads * k;
+                    if (v < nvecW) {
+                        uint32_t hv[4], lv[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            uint16_t q0[2], q1[2];
+                            split_parts<kF16>(xw[k * EPVW + i], 2, q0, 1);
+                            split_parts<kF16>(xw[k * EPVW + i + 4], 2, q1, 1);
+                            hv[i] = uint32_t(q0[0]) | (uint32_t(q1[0]) << 16);
+                            lv[i] = uint32_t(q0[1]) | (uint32_t(q1[1]) << 16);
+                        }
+                        uint4 *dst = reinterpret_cast<uint4 *>(stg + xpoff) + (size_t(v >> 2) * 2) * 4 + (v & 3);
+                        dst[0] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+                        dst[4] = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+                    }
+                }
+            }
+        }
         // compaction in ascending strip order: warp e builds expert slot e's list
         if (warp < ntop) {
             const int e = warp;
@@ -1458,7 +1510,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         // records are issued in batches of up to kIssue (as many as the
         // staging buffer holds) and consumed in rounds of up to kRound, so a
         // round's dots overlap the later rounds' copies
-        const int cap_all = min(kIssue, kStageBytes / per_n);
+        // slots of a batch, sstr bytes apart: INT4 records get 16 bytes of
+        // padding, so that the tensor-core dots' eight rows per load fall in
+        // different shared-memory banks
+        const int sstr = WF == kI4 ? per_n + 16 : per_n;
+        const int cap_all = min(kIssue, (WF == kI4 ? xpoff : kStageBytes) / sstr);
         const int cap_n = min(kRound, cap_all);
         int jb = 0, je = 0;   // the batch in shared memory: neurons [jb, je) in slots 0 ..
 
@@ -1536,7 +1592,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     if (hot_l) {
                         const int e = en_l >> 24;
                         const unsigned code = unsigned(en_l) & 0xffffffu;
-                        uint8_t *slot = stg + size_t(lane) * per_n;
+                        uint8_t *slot = stg + size_t(lane) * sstr;
                         uint64_t *gb = &sm.gbar[lane >> 2];
                         stage_copy(slot, exs[e]->Wgu + size_t(code) * p.rec_bytes, uint32_t(per_n), gb);
                     }
@@ -1547,7 +1603,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                         const int en = sm.glst[jb + n];
                         if (!(unsigned(en) & kColdBit)) continue;
                         const unsigned idx = unsigned(en) & (kColdBit - 1u);
-                        copy_host_rec(stg + size_t(n) * per_n, exs[en >> 24]->Wgu_cold + size_t(idx) * p.rec_bytes,
+                        copy_host_rec(stg + size_t(n) * sstr, exs[en >> 24]->Wgu_cold + size_t(idx) * p.rec_bytes,
                                       per_n, tid, kThreads);
                     }
                     cta_sync();
@@ -1557,9 +1613,101 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             k = min(cap_n, je - j0);
             const int sb = j0 - jb;                                         // this round's first slot
             const unsigned rmask = ((1u << ((k + 3) / 4)) - 1u) << (sb >> 2);   // its groups
-            // dots of the round's neurons, four at a time as each group lands:
-            // values 2n (gate) and 2n + 1 (up); after the reduction lanes
-            // 4q .. 4q + 3 hold value q
+            // Dots of the round's neurons: values 2n (gate) and 2n + 1 (up),
+            // each warp's partial over its own x vectors to sm.red.
+            //
+            // INT4 weights: tensor-core dots, one m-tile of 16 rows at a time
+            // (gated: the gate rows of eight neurons over their up rows; else
+            // sixteen neurons' rows) once the groups holding them have landed.
+            // A holds the rows' codes as exact f16 values, B the two fp16 parts
+            // of x; warp w takes the 32-element k-groups of its own x vectors
+            // (G = 8 w + 128 kk + j), and each group's dot is scaled by the
+            // row's group scale in fp32.
+            if constexpr (WF == kI4) {
+                constexpr int kNT = kGated ? 8 : 16;   // neurons per m-tile
+                const int g = lane >> 2, tq = lane & 3;
+                bool tok = true;
+#pragma unroll 1
+                for (int n0 = 0; n0 < k && tok; n0 += kNT) {
+                    for (int g0 = n0; g0 < min(n0 + kNT, k); g0 += 4) {
+                        // this warp waits (bounded) for the group; every lane
+                        // then observes the completed phase itself
+                        const int gi = (sb + g0) >> 2;
+                        const uint32_t par = (gpar >> gi) & 1u;
+                        bool ok = true;
+                        if (lane == 0 && !mbar_test(&sm.gbar[gi], par)) {
+                            const long long t0 = gtimer();
+                            for (unsigned it = 1;; ++it) {
+                                if (mbar_test(&sm.gbar[gi], par)) break;
+                                if ((it & 15) == 0 && gtimer() - t0 > p.wait_ns) { ok = false; break; }
+                            }
+                        }
+                        ok = __shfl_sync(0xffffffffu, ok, 0);
+                        if (j0 == 0 && g0 == 0 && warp == 0) prof_put(p, li, 17, gtimer());
+                        if (!ok) {
+                            if (lane == 0) {
+                                set_error(p.err, kDevTimeout);
+                                sm.gfail = 1;
+                            }
+                            tok = false;
+                            break;
+                        }
+                        mbar_test(&sm.gbar[gi], par);   // acquire for this lane
+                    }
+                    if (!tok) break;
+                    // this lane's rows g and g + 8 of the tile (rows past the
+                    // round's last neuron read its last slot; never stored)
+                    const int na = n0 + g, nb = kGated ? na : n0 + g + 8;
+                    const uint8_t *ra = stg + size_t(sb + min(na, k - 1)) * sstr;
+                    const uint8_t *rbw = kGated ? ra + p.wrow : stg + size_t(sb + min(nb, k - 1)) * sstr;
+                    float accA = 0.f, accB = 0.f;
+#pragma unroll
+                    for (int kk = 0; kk < MAXVW; ++kk) {
+#pragma unroll 2
+                        for (int j = 0; j < 8; ++j) {
+                            const int G = 8 * warp + 128 * kk + j;
+                            if (G < d / 32) {
+                                const uint32_t wa = *reinterpret_cast<const uint32_t *>(ra + G * 16 + 4 * tq);
+                                const uint32_t wb = *reinterpret_cast<const uint32_t *>(rbw + G * 16 + 4 * tq);
+                                uint4 bx = make_uint4(0u, 0u, 0u, 0u);
+                                if (g < 2) bx = reinterpret_cast<const uint4 *>(xp)[(G * 2 + g) * 4 + tq];
+                                uint32_t fa[4], fb[4];
+                                i4x8_to_h2(wa, fa);
+                                i4x8_to_h2(wb, fb);
+                                float c[4] = {0.f, 0.f, 0.f, 0.f};
+                                mma16816<kF16>(c, fa[0], fb[0], fa[1], fb[1], bx.x, bx.y);
+                                mma16816<kF16>(c, fa[2], fb[2], fa[3], fb[3], bx.z, bx.w);
+                                // columns 0 and 1 (the parts) of rows g and g + 8 sit in lane 4g
+                                if (tq == 0) {
+                                    const float sa = __half2float(*reinterpret_cast<const __half *>(ra + d / 2 + 2 * G));
+                                    const float sbw = __half2float(*reinterpret_cast<const __half *>(rbw + d / 2 + 2 * G));
+                                    accA = fmaf(sa, c[0] + c[1], accA);
+                                    accB = fmaf(sbw, c[2] + c[3], accB);
+                                }
+                            }
+                        }
+                    }
+                    if (tq == 0) {
+                        if constexpr (kGated) {
+                            if (na < k) {
+                                sm.red[rb][warp][2 * na] = accA;
+                                sm.red[rb][warp][2 * na + 1] = accB;
+                            }
+                        } else {
+                            if (na < k) {
+                                sm.red[rb][warp][2 * na] = accA;
+                                sm.red[rb][warp][2 * na + 1] = 0.f;
+                            }
+                            if (nb < k) {
+                                sm.red[rb][warp][2 * nb] = accB;
+                                sm.red[rb][warp][2 * nb + 1] = 0.f;
+                            }
+                        }
+                    }
+                }
+            } else
+            // other formats: four neurons at a time as each group lands; after
+            // the reduction lanes 4q .. 4q + 3 hold value q
 #pragma unroll 1
             for (int g0 = 0; g0 < k; g0 += 4) {
                 {
@@ -1592,7 +1740,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     v[2 * n] = 0.f;
                     v[2 * n + 1] = 0.f;
                     if (g0 + n < k) {
-                        const uint8_t *slot = stg + size_t(sb + g0 + n) * per_n;
+                        const uint8_t *slot = stg + size_t(sb + g0 + n) * sstr;
                         v[2 * n] = dot_smem(slot);
                         if (kGated) v[2 * n + 1] = dot_smem(slot + p.wrow);
                     }
@@ -1638,7 +1786,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 #pragma unroll
                     for (int j = 0; j < kAG; ++j) {
                         hv[j] = g0 + j < k ? sm.rh[g0 + j] : 0.f;
-                        const uint8_t *row = stg + size_t(sb + g0 + j) * per_n + p.gu_bytes;
+                        const uint8_t *row = stg + size_t(sb + g0 + j) * sstr + p.gu_bytes;
 #pragma unroll
                         for (int kk = 0; kk < MAXVW; ++kk) {
                             const int v = tid + kThreads * kk;
@@ -1648,7 +1796,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 #pragma unroll
                     for (int j = 0; j < kAG; ++j) {
                         if (hv[j] == 0.f) continue;
-                        const uint8_t *row = stg + size_t(sb + g0 + j) * per_n + p.gu_bytes;
+                        const uint8_t *row = stg + size_t(sb + g0 + j) * sstr + p.gu_bytes;
 #pragma unroll
                         for (int kk = 0; kk < MAXVW; ++kk) {
                             const int v = tid + kThreads * kk;
