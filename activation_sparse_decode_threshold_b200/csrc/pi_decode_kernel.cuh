@@ -323,25 +323,30 @@ __device__ __forceinline__ void i8x4_to_h2(uint32_t w, uint32_t &lo, uint32_t &h
     hi = *reinterpret_cast<const uint32_t *>(&hb);
 }
 
-// Eight INT4 codes (nibble i of w = element i, value n_i - 8) as four f16x2
-// values, exactly, paired (e0, e4), (e1, e5), (e2, e6), (e3, e7): a nibble
-// in the low four bits of a half is 1024 + n in binary16, and one in bits
-// 4..7 is 1024 + 16 n, scaled by 1/16 in the same fused multiply-add that
-// takes the offset away.
-__device__ __forceinline__ void i4x8_to_h2(uint32_t w, uint32_t (&o)[4])
+// Eight INT4 codes (nibble i of w = element i, code n_i, value n_i - 8) as
+// signed bytes 16 (n_i - 8), exactly: flipping a nibble's top bit gives the
+// value in 4-bit two's complement, and moving it to the top of a byte scales
+// it by 16.  ev holds elements 0, 2, 4, 6 (byte j = element 2j), od holds
+// elements 1, 3, 5, 7.
+__device__ __forceinline__ void i4x8_to_s8(uint32_t w, uint32_t &ev, uint32_t &od)
 {
-    const __half2 off_lo = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));   // 1032
-    const __half2 scl_hi = __halves2half2(__ushort_as_half(0x2c00), __ushort_as_half(0x2c00));   // 1/16
-    const __half2 off_hi = __halves2half2(__ushort_as_half(0xd480), __ushort_as_half(0xd480));   // -72
-    const uint32_t w8 = w >> 8;
-    const uint32_t q[4] = {(w & 0x000f000fu) | 0x64006400u, (w & 0x00f000f0u) | 0x64006400u,
-                           (w8 & 0x000f000fu) | 0x64006400u, (w8 & 0x00f000f0u) | 0x64006400u};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const __half2 h = *reinterpret_cast<const __half2 *>(&q[i]);
-        const __half2 r = (i & 1) ? __hfma2(h, scl_hi, off_hi) : __hsub2(h, off_lo);
-        o[i] = *reinterpret_cast<const uint32_t *>(&r);
-    }
+    ev = ((w << 4) ^ 0x80808080u) & 0xf0f0f0f0u;
+    od = (w ^ 0x80808080u) & 0xf0f0f0f0u;
+}
+// D = A B of signed bytes, 32-bit integer result (exact), C = 0.
+__device__ __forceinline__ void imma16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1)
+{
+    asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                 "{%8, %9}, {%10, %10, %10, %10};"
+                 : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
+}
+// An integer of magnitude below 2^22 as fp32, exactly: placed in the mantissa
+// of 1.5 * 2^23, which is then subtracted.
+__device__ __forceinline__ float i22_to_f(int c)
+{
+    return __int_as_float(c + 0x4B400000) - 12582912.0f;
 }
 
 // Where a neuron's record lives.  Without a VRAM budget (hot_k = 0) every
@@ -619,11 +624,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // other rows follow once the V rows have been read.  A routed layer
     // stages its V rows in rounds from offset 0 once the experts are known.
     const int yoff = predict ? kStageBytes : kStageBytes - d * 8;
-    // INT4 weights: x as two fp16 parts in the tensor-core B layout of the
-    // gather's dots (4d bytes at the top of the staging buffer, written after
-    // the predictor's rounds and read until the last gather round)
-    const int xpoff = kStageBytes - 4 * d;
+    // INT4 weights: x as signed base-128 digits in the tensor-core B layout of
+    // the gather's dots (8d bytes at the top of the staging buffer, written
+    // after the predictor's rounds and read until the last gather round).
+    // |x_j| <= sqrt(d) after the RMSNorm, so x * xs with xs = 2^(6 - e),
+    // 4^e >= d, lies in [-64, 64]; digit 0 is its nearest integer and each
+    // further digit the nearest integer of 128 times the remainder, so that
+    // x = xs^-1 sum_{p<5} digit_p 128^-p up to 2^-29 xs^-1, every step exact.
+    const int xpoff = kStageBytes - 8 * d;
     const uint8_t *xp = stg + xpoff;
+    int xse = 0;
+    while ((1 << (2 * xse)) < d) ++xse;
+    const float xs = ldexpf(1.f, 6 - xse);
     const int voff = (yoff - nrows * p.vrow) & ~127;
     const bool vsm = !moe && nrows > 0 && nrows <= kRA && voff >= 0;
     const int u_round0 = min(ns, ucap);
@@ -1010,6 +1022,38 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         return pbar ? grid_wait(&sm, p, epoch, bci, cycb) : true;
     };
 
+    // INT4 weights: x's digits in the gather dots' B layout, for k-group G
+    // (32 elements), column p (digit p; columns 5..7 zero) and lane quad tq, 8
+    // bytes: digit p of elements 8 tq + 0, 2, 4, 6, then of 8 tq + 1, 3, 5, 7
+    // (the order of i4x8_to_s8).  The thread holding vector v = 4 G + tq
+    // writes them, while the CTA waits at the balance step.
+    auto write_digits = [&]() {
+        if constexpr (WF == kI4) {
+#pragma unroll
+            for (int k = 0; k < MAXVW; ++k) {
+                const int v = tid + kThreads * k;
+                if (v < nvecW) {
+                    uint32_t dg[5][2] = {};
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        float t = xw[k * EPVW + i] * xs;
+#pragma unroll
+                        for (int q = 0; q < 5; ++q) {
+                            const float r = rintf(t);
+                            dg[q][i & 1] |= (uint32_t(int(r)) & 0xffu) << (8 * (i >> 1));
+                            t = (t - r) * 128.f;
+                        }
+                    }
+                    uint2 *dst = reinterpret_cast<uint2 *>(stg + xpoff) + size_t(v >> 2) * 32 + (v & 3);
+#pragma unroll
+                    for (int q = 0; q < 5; ++q) dst[q * 4] = make_uint2(dg[q][0], dg[q][1]);
+#pragma unroll
+                    for (int q = 5; q < 8; ++q) dst[q * 4] = make_uint2(0u, 0u);
+                }
+            }
+        }
+    };
+
     // Each pass forms the input of layer l + 1 and then runs that layer; the
     // first pass (l = l0 - 1) is the prologue.  One call site keeps one copy
     // of the input step's code.
@@ -1339,32 +1383,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             if (!ok) break;
         }
         prof_put(p, li, 9, gtimer());
-        if constexpr (WF == kI4) {
-            // x in the gather dots' B layout: for k-group G (32 elements) and
-            // lane quad tq, part p's four f16x2 values hold x at elements
-            // 8 tq + (0, 4), (1, 5), (2, 6), (3, 7) of the group, the pairing
-            // of i4x8_to_h2; the thread holding vector v = 4 G + tq writes them
-            if (!predict) {
-#pragma unroll
-                for (int k = 0; k < MAXVW; ++k) {
-                    const int v = tid + kThreads * k;
-                    if (v < nvecW) {
-                        uint32_t hv[4], lv[4];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            uint16_t q0[2], q1[2];
-                            split_parts<kF16>(xw[k * EPVW + i], 2, q0, 1);
-                            split_parts<kF16>(xw[k * EPVW + i + 4], 2, q1, 1);
-                            hv[i] = uint32_t(q0[0]) | (uint32_t(q1[0]) << 16);
-                            lv[i] = uint32_t(q0[1]) | (uint32_t(q1[1]) << 16);
-                        }
-                        uint4 *dst = reinterpret_cast<uint4 *>(stg + xpoff) + (size_t(v >> 2) * 2) * 4 + (v & 3);
-                        dst[0] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-                        dst[4] = make_uint4(lv[0], lv[1], lv[2], lv[3]);
-                    }
-                }
-            }
-        }
         // compaction in ascending strip order: warp e builds expert slot e's list
         if (warp < ntop) {
             const int e = warp;
@@ -1436,6 +1454,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     prefetch_l2(exs[e]->Wgu + size_t(code) * p.rec_bytes, uint32_t(kSpec ? p.rec_bytes : p.gu_bytes));
             }
             if (tid == 0) sm.share_n = nl;
+            write_digits();
             cta_sync();
         } else {
         {
@@ -1458,6 +1477,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 if (!(code & kColdBit))
                     prefetch_l2(exs[e]->Wgu + size_t(code) * p.rec_bytes, uint32_t(kSpec ? p.rec_bytes : p.gu_bytes));
             }
+            write_digits();
         }
         if (!grid_wait(&sm, p, epoch, bci, &cyc_bar)) break;
         prof_put(p, li, 16, gtimer());
@@ -1616,13 +1636,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             // Dots of the round's neurons: values 2n (gate) and 2n + 1 (up),
             // each warp's partial over its own x vectors to sm.red.
             //
-            // INT4 weights: tensor-core dots, one m-tile of 16 rows at a time
-            // (gated: the gate rows of eight neurons over their up rows; else
-            // sixteen neurons' rows) once the groups holding them have landed.
-            // A holds the rows' codes as exact f16 values, B the two fp16 parts
-            // of x; warp w takes the 32-element k-groups of its own x vectors
-            // (G = 8 w + 128 kk + j), and each group's dot is scaled by the
-            // row's group scale in fp32.
+            // INT4 weights: integer tensor-core dots, one m-tile of 16 rows at
+            // a time (gated: the gate rows of eight neurons over their up rows;
+            // else sixteen neurons' rows) once the groups holding them have
+            // landed.  A holds 16 (n - 8) of the rows' codes, B x's digits
+            // (column p = digit p), so D = 16 * 2^(7p) * xs * (the group's dot
+            // with digit p of x), exact in int32; warp w takes the 32-element
+            // k-groups of its own x vectors (G = 8 w + 128 kk + j) and adds each
+            // group's digit columns, weighted, times the row's group scale.
             if constexpr (WF == kI4) {
                 constexpr int kNT = kGated ? 8 : 16;   // neurons per m-tile
                 const int g = lane >> 2, tq = lane & 3;
@@ -1660,6 +1681,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     const int na = n0 + g, nb = kGated ? na : n0 + g + 8;
                     const uint8_t *ra = stg + size_t(sb + min(na, k - 1)) * sstr;
                     const uint8_t *rbw = kGated ? ra + p.wrow : stg + size_t(sb + min(nb, k - 1)) * sstr;
+                    // this lane's digit columns 2 tq and 2 tq + 1: weights 2^-7p / (16 xs)
+                    const float dw0 = tq < 3 ? ldexpf(1.f, -14 * tq - 4) / xs : 0.f;
+                    const float dw1 = tq < 2 ? ldexpf(1.f, -14 * tq - 11) / xs : 0.f;
                     float accA = 0.f, accB = 0.f;
 #pragma unroll
                     for (int kk = 0; kk < MAXVW; ++kk) {
@@ -1669,24 +1693,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                             if (G < d / 32) {
                                 const uint32_t wa = *reinterpret_cast<const uint32_t *>(ra + G * 16 + 4 * tq);
                                 const uint32_t wb = *reinterpret_cast<const uint32_t *>(rbw + G * 16 + 4 * tq);
-                                uint4 bx = make_uint4(0u, 0u, 0u, 0u);
-                                if (g < 2) bx = reinterpret_cast<const uint4 *>(xp)[(G * 2 + g) * 4 + tq];
-                                uint32_t fa[4], fb[4];
-                                i4x8_to_h2(wa, fa);
-                                i4x8_to_h2(wb, fb);
-                                float c[4] = {0.f, 0.f, 0.f, 0.f};
-                                mma16816<kF16>(c, fa[0], fb[0], fa[1], fb[1], bx.x, bx.y);
-                                mma16816<kF16>(c, fa[2], fb[2], fa[3], fb[3], bx.z, bx.w);
-                                // columns 0 and 1 (the parts) of rows g and g + 8 sit in lane 4g
-                                if (tq == 0) {
-                                    const float sa = __half2float(*reinterpret_cast<const __half *>(ra + d / 2 + 2 * G));
-                                    const float sbw = __half2float(*reinterpret_cast<const __half *>(rbw + d / 2 + 2 * G));
-                                    accA = fmaf(sa, c[0] + c[1], accA);
-                                    accB = fmaf(sbw, c[2] + c[3], accB);
-                                }
+                                const uint2 bx = reinterpret_cast<const uint2 *>(xp)[(G * 8 + g) * 4 + tq];
+                                uint32_t ae, ao, be, bo;
+                                i4x8_to_s8(wa, ae, ao);
+                                i4x8_to_s8(wb, be, bo);
+                                int dd[4];
+                                imma16832(dd, ae, be, ao, bo, bx.x, bx.y);
+                                const float sa = __half2float(*reinterpret_cast<const __half *>(ra + d / 2 + 2 * G));
+                                const float sbw = __half2float(*reinterpret_cast<const __half *>(rbw + d / 2 + 2 * G));
+                                accA = fmaf(sa, fmaf(i22_to_f(dd[0]), dw0, i22_to_f(dd[1]) * dw1), accA);
+                                accB = fmaf(sbw, fmaf(i22_to_f(dd[2]), dw0, i22_to_f(dd[3]) * dw1), accB);
                             }
                         }
                     }
+                    // the digit columns sit in the four lanes of a quad
+                    accA += __shfl_xor_sync(0xffffffffu, accA, 1);
+                    accB += __shfl_xor_sync(0xffffffffu, accB, 1);
+                    accA += __shfl_xor_sync(0xffffffffu, accA, 2);
+                    accB += __shfl_xor_sync(0xffffffffu, accB, 2);
                     if (tq == 0) {
                         if constexpr (kGated) {
                             if (na < k) {

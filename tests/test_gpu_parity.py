@@ -30,6 +30,12 @@ SMALL = {
                               wdtype="int4g32"),
     "relu-int4-nongated": synth.small(synth.CONFIGS["falcon40b"], n_layers=2, d=512, F=1500, rank=64,
                                       wdtype="int4g32"),
+    # INT4 at d_model 8192: two x vectors per thread, so every warp's tensor-core
+    # gather dots take k-groups from both of its vector ranges
+    "relu-int4-d8192": synth.small(synth.CONFIGS["falcon40b"], n_layers=2, d=8192, F=1500, rank=64,
+                                   wdtype="int4g32"),
+    "moe-int4-drelu-d8192": synth.small(synth.CONFIGS["mixtral47b"], n_layers=2, d=8192, F=1024, rank=64,
+                                        n_experts=4),
     # the 8-bit per-row predictor with 16-bit and INT4 weights, dense and MoE
     "reglu-f16-i8pred": synth.small(synth.CONFIGS["llama7b-i8pred"], n_layers=3, d=512, F=1000, rank=128),
     "drelu-bf16-i8pred": synth.small(synth.CONFIGS["mistral7b"], n_layers=2, d=768, F=2100, rank=64,
