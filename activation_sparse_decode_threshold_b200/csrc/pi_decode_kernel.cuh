@@ -897,25 +897,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                         sm.rlg[lane] = float(double(static_cast<long long>(__ldcg(rl + lane))) * (1.0 / 4294967296.0));
                     __syncwarp();
                     if (lane == 0) {
-                        float pr[kMaxExperts];
-                        float mx = -INFINITY;
-#pragma unroll 1
-                        for (int e = 0; e < p.E; ++e) mx = fmaxf(mx, sm.rlg[e]);
-                        float den = 0.f;
-#pragma unroll 1
-                        for (int e = 0; e < p.E; ++e) { pr[e] = expf(sm.rlg[e] - mx); den += pr[e]; }
+                        // the softmax is increasing in the logit, so the two
+                        // largest probabilities are the two largest logits
+                        // (ties: lower index), and the renormalised pair
+                        // p_a / (p_a + p_b) = 1 / (1 + exp(l_b - l_a)) needs
+                        // one exponential, taken of a non-positive difference
                         int ea = 0;
 #pragma unroll 1
-                        for (int e = 1; e < p.E; ++e) if (pr[e] > pr[ea]) ea = e;
+                        for (int e = 1; e < p.E; ++e) if (sm.rlg[e] > sm.rlg[ea]) ea = e;
                         int eb = ea == 0 ? 1 : 0;
 #pragma unroll 1
-                        for (int e = 0; e < p.E; ++e) if (e != ea && pr[e] > pr[eb]) eb = e;
+                        for (int e = 0; e < p.E; ++e) if (e != ea && sm.rlg[e] > sm.rlg[eb]) eb = e;
+                        const float q = expf(sm.rlg[eb] - sm.rlg[ea]);   // p_b / p_a <= 1
+                        const float wa = 1.f / (1.f + q), wb = q / (1.f + q);
                         const int lo = min(ea, eb), hi = max(ea, eb);
-                        const float plo = pr[lo] / den, phi = pr[hi] / den;
                         sm.route_e[0] = lo;
                         sm.route_e[1] = hi;
-                        sm.route_w[0] = plo / (plo + phi);
-                        sm.route_w[1] = phi / (plo + phi);
+                        sm.route_w[0] = lo == ea ? wa : wb;
+                        sm.route_w[1] = lo == ea ? wb : wa;
                         sm.exl[ln & 1][0] = sm.exall[lo];
                         sm.exl[ln & 1][1] = sm.exall[hi];
                         if (p.stats && b == 0) {
