@@ -862,28 +862,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 // (ties: lower index), renormalised
                 unsigned long long *rl = reinterpret_cast<unsigned long long *>(p.bar + kRouterWord) +
                                          size_t(ln & 1) * kMaxExperts;
-                if (warp == 0 && ncol > 0) {
+                if (warp < p.E && ncol > 0) {
+                    // warp e: expert e's dot over this CTA's columns
                     const __half *R = reinterpret_cast<const __half *>(p.router[ln]);
                     const bool staged = rts_ok;   // this CTA's router columns already in shared memory
-                    // four experts at a time; after the reduction lanes 8q .. 8q + 7
-                    // hold expert e0 + q's value
-#pragma unroll 1
-                    for (int e0 = 0; e0 < p.E; e0 += 4) {
-                        float q[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            q[e] = 0.f;
-                            if (e0 + e < p.E)
-                                for (int j = lane; j < ncol; j += 32) {
-                                    const float w = staged ? sm.rsl[kRtsOff + (e0 + e) * ncol + j]
-                                                           : __half2float(R[size_t(e0 + e) * d + c0 + j]);
-                                    q[e] = fmaf(w, sm.rsl[j], q[e]);
-                                }
-                        }
-                        const float s = warp_transpose_sum<4>(q);
-                        if ((lane & 7) == 0 && e0 + (lane >> 3) < p.E)
-                            red_add_u64(rl + e0 + (lane >> 3), fix_q(s * inv, p.err));
+                    const int e = warp;
+                    float q = 0.f;
+                    for (int j = lane; j < ncol; j += 32) {
+                        const float w = staged ? sm.rsl[kRtsOff + e * ncol + j] : __half2float(R[size_t(e) * d + c0 + j]);
+                        q = fmaf(w, sm.rsl[j], q);
                     }
+                    q = warp_sum(q);
+                    if (lane == 0) red_add_u64(rl + e, fix_q(q * inv, p.err));
                 }
                 if (lip >= 0) prof_put(p, lip, 22, gtimer());
                 grid_arrive(p, epoch);
