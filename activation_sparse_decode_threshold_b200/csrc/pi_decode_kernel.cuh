@@ -418,7 +418,6 @@ struct Smem {
     float rsum[kRed];                      // CTA-wide dot products of a gather round
     float rh[kRound];                      // h of each neuron of a gather round
     int route_e[kMaxTopK];
-    float rlg[kMaxExperts];                // router logits of the next layer (routed)
     float route_w[kMaxTopK];
     int bc[2];
     uint64_t stage_bar;                    // completion of a staging round
@@ -880,25 +879,33 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 if (!grid_wait(&sm, p, epoch, bci, cycb)) return false;
                 if (lip >= 0) prof_put(p, lip, 23, gtimer());
                 if (warp == 0) {
-                    // lane e reads expert e's total; lane 0 then decides in
-                    // compact loops (this code runs once per layer on one
-                    // thread, where straight-line code costs instruction fetches)
-                    if (lane < p.E)
-                        sm.rlg[lane] = float(double(static_cast<long long>(__ldcg(rl + lane))) * (1.0 / 4294967296.0));
-                    __syncwarp();
+                    // lane e holds expert e's logit.  The softmax is increasing
+                    // in the logit, so the two largest probabilities are the two
+                    // largest logits (ties: lower index), found by two warp
+                    // argmax butterflies, and the renormalised pair
+                    // p_a / (p_a + p_b) = 1 / (1 + exp(l_b - l_a)) needs one
+                    // exponential, taken of a non-positive difference
+                    const float lg = lane < p.E ? float(double(static_cast<long long>(__ldcg(rl + lane))) *
+                                                        (1.0 / 4294967296.0))
+                                                : -INFINITY;
+                    auto argmax = [&](float v) -> int {
+                        int i = lane;
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) {
+                            const float vo = __shfl_xor_sync(0xffffffffu, v, o);
+                            const int io = __shfl_xor_sync(0xffffffffu, i, o);
+                            if (vo > v || (vo == v && io < i)) {
+                                v = vo;
+                                i = io;
+                            }
+                        }
+                        return i;
+                    };
+                    const int ea = argmax(lg);
+                    const int eb = argmax(lane == ea ? -INFINITY : lg);
+                    const float la = __shfl_sync(0xffffffffu, lg, ea), lb = __shfl_sync(0xffffffffu, lg, eb);
                     if (lane == 0) {
-                        // the softmax is increasing in the logit, so the two
-                        // largest probabilities are the two largest logits
-                        // (ties: lower index), and the renormalised pair
-                        // p_a / (p_a + p_b) = 1 / (1 + exp(l_b - l_a)) needs
-                        // one exponential, taken of a non-positive difference
-                        int ea = 0;
-#pragma unroll 1
-                        for (int e = 1; e < p.E; ++e) if (sm.rlg[e] > sm.rlg[ea]) ea = e;
-                        int eb = ea == 0 ? 1 : 0;
-#pragma unroll 1
-                        for (int e = 0; e < p.E; ++e) if (e != ea && sm.rlg[e] > sm.rlg[eb]) eb = e;
-                        const float q = expf(sm.rlg[eb] - sm.rlg[ea]);   // p_b / p_a <= 1
+                        const float q = expf(lb - la);   // p_b / p_a <= 1
                         const float wa = 1.f / (1.f + q), wb = q / (1.f + q);
                         const int lo = min(ea, eb), hi = max(ea, eb);
                         sm.route_e[0] = lo;
