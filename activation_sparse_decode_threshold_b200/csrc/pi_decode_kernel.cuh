@@ -609,9 +609,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     const int ucap_rows = min(kZRows, kStageBytes / p.urow);
     const int ucap = ns <= ucap_rows ? max(ns, 1) : (ucap_rows & ~7);
     // routed: when both experts' strips fit the staging buffer together (an
-    // 8-bit predictor's rows), both are staged before the t barrier, the
-    // second right after the first (chunk permutation keys are relative to
-    // each strip's own first row)
+    // 8-bit predictor's rows), both are staged right after this CTA's rows
+    // of t, the second right after the first (chunk permutation keys are
+    // relative to each strip's own first row)
     const int u2 = ns;
     const bool both_u = moe && !predict && p.top_k == 2 && ns > 0 && ns <= ucap && 2 * ns * p.urow <= kStageBytes;
 
@@ -767,7 +767,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // (the next input buffer, the trace, or the caller's residual after the
     // last layer); x = RMSNorm(r) goes to xw (the predictor call takes x as
     // given); a routed layer picks its experts; this CTA's rows of t = V x go
-    // to t_buf; a grid barrier follows, after which every CTA reads t.  The
+    // out as tagged slots, which every CTA polls at the layer's start.  The
     // last layer stops after writing the residual, and a one-layer call that
     // emits y stops after writing y.  False if a bounded wait ran out.
     // -----------------------------------------------------------------------
@@ -1075,14 +1075,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             for (int i = tid; i < ns; i += kThreads) sm.cbuf[e][i] = __ldg(sm.exl[l & 1][e].c + s0 + i);
         // the next layer's weight pointers (dense), for its prefetches during this layer
         if (!moe && tid == kThreads - 1 && l + 1 < l1) sm.exl[(l + 1) & 1][0] = p.ex[size_t(l + 1) * p.E];
-        // layer l - 1's fixed-point total (read before the last barrier) is
-        // cleared for layer l + 1
+        // layer l - 1's fixed-point total (read before the last merge barrier)
+        // is cleared for layer l + 1
         if (!predict && l + 1 < l1) {
             unsigned long long *yz = p.yfix + size_t((l + 1) & 1) * d;
             for (int e = c0 + tid; e < c0 + ncol; e += kThreads) yz[e] = 0ull;
         }
-        // routed: layer l - 1's router totals (read before the last barrier)
-        // are cleared for layer l + 1
+        // routed: layer l - 1's router totals (read before the last merge
+        // barrier) are cleared for layer l + 1
         if (moe && !predict && b == 0 && tid < kMaxExperts && l + 1 < l1)
             reinterpret_cast<unsigned long long *>(p.bar + kRouterWord)[size_t((l + 1) & 1) * kMaxExperts + tid] = 0ull;
         if (!moe && tid == 0 && p.stats && b == 0 && !predict) {

@@ -296,15 +296,16 @@ PI_API pi_status pi_debug_set(pi_ffn_t h, int flags, double wait_limit_s);
 
 /* Testing aid: when `times_dev` is non-NULL, each later pi_sparse_ffn_decode
  * call records, per layer and CTA, %globaltimer (ns) at these points k:
- *   0 layer start, 1 layer t and biases ready, 14 first predictor rows in
+ *   0 layer start, 1 layer t polled and biases ready, 14 first predictor rows in
  *   shared memory, 15 first tensor-core logits done, 9 predictor logits done,
  *   2 active list done, 16 after the balance barrier, 8 this CTA's share of
  *   the active list known, 17 first gathered rows landed, 25 gather rounds
  *   done, 26 down rows done (the CTA's partial of y complete), 3 partial
  *   merged into the layer's total, 4 after the merge barrier, 20 next input
- *   summed, 7 next x formed, 5 this CTA's rows of t written, 6 after the t
- *   barrier; for routed (MoE) layers also 22 router share added, 23 after
- *   the router barrier, 18 experts chosen, 19 first V rows in shared memory;
+ *   summed, 7 next x formed, 5 this CTA's rows of t written, 6 the input
+ *   step done (the prologue's grid barrier included); for routed (MoE)
+ *   layers also 22 router share added, 23 after the router barrier, 18
+ *   experts chosen, 19 first V rows in shared memory;
  * and k = 10..13 the clock cycles thread 0 spent obtaining the layer input,
  * waiting for predictor rows, waiting for gathered rows and waiting in grid
  * barriers.  Points 20, 7, 22, 23, 18, 19, 5 and 6 belong to the step that
