@@ -342,6 +342,15 @@ __device__ __forceinline__ void imma16832(int (&d)[4], uint32_t a0, uint32_t a1,
                  : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
                  : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
 }
+// D += A B of signed bytes, 32-bit integer accumulators (exact).
+__device__ __forceinline__ void imma16832_acc(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1)
+{
+    asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                 "{%8, %9}, {%0, %1, %2, %3};"
+                 : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 // An integer of magnitude below 2^22 as fp32, exactly: placed in the mantissa
 // of 1.5 * 2^23, which is then subtracted.
 __device__ __forceinline__ float i22_to_f(int c)
@@ -640,6 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     const int u_round0 = min(ns, ucap);
     const int ufirst = vsm ? min(u_round0, voff / p.urow) : u_round0;
 
+    float tsc = 1.f;   // 8-bit predictor: the scale of t's digits in this layer
     // the rows of t as tagged slots (tag: the layer's index in this launch + 1)
     unsigned long long *const tslot = reinterpret_cast<unsigned long long *>(p.bar + kTagTWord);
     unsigned epoch = 0;
@@ -732,7 +742,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     uint16_t *const tpart = reinterpret_cast<uint16_t *>(sm.tsm);
     auto put_t = [&](int k, float tv, int ntr) {
         if constexpr (PF == kF32) sm.tsm[k] = tv;
-        else if constexpr (PF == kI8) split_parts<kF16>(tv, 2, tpart + k, ntr);
+        else if constexpr (PF == kI8) (void)tv;   // t goes in as digits, written after the poll
         else split_parts<PF>(tv, (PF == kBF16 && 3 * ntr <= 2 * kMaxRankTotal) ? 3 : 2, tpart + k, ntr);
     };
 
@@ -1127,6 +1137,59 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 const int k = tid + i * kThreads;
                 if (k < nt) put_t(k, __uint_as_float(unsigned(w[i])), nt);
             }
+            if constexpr (PF == kI8) {
+                // 8-bit predictor: t as signed base-128 digits for the integer
+                // logits.  The bound of |t| over the layer (the same in every
+                // CTA) gives ts = 2^(6 - e), max |t| < 2^e, so t * ts lies in
+                // (-64, 64); digit 0 is its nearest integer and each further
+                // digit the nearest integer of 128 times the remainder (every
+                // step exact; four digits leave below 2^-22 2^(e-6)).
+                float mx = 0.f;
+#pragma unroll
+                for (int i = 0; i < kTS; ++i)
+                    if (tid + i * kThreads < nt) mx = fmaxf(mx, fabsf(__uint_as_float(unsigned(w[i]))));
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                if (lane == 0) sm.red[rb][warp][0] = mx;
+                cta_sync();
+#pragma unroll
+                for (int w2 = 0; w2 < kConsumerWarps; ++w2) mx = fmaxf(mx, sm.red[rb][w2][0]);
+                rb ^= 1;
+                int ex = 0;
+                (void)frexpf(mx, &ex);
+                tsc = ldexpf(1.f, 6 - ex);
+                // the digits of four consecutive t values form one 32-bit word
+                // (byte j = element 4q + j): for expert slot e, k32 step s,
+                // digit p and lane quad tq, the word pair of elements 32 s +
+                // 4 tq .. + 3 and 32 s + 16 + 4 tq .. + 3 (the B fragment)
+                uint32_t *dw = reinterpret_cast<uint32_t *>(sm.tsm);
+                const int nk32 = r >> 5;
+#pragma unroll
+                for (int i = 0; i < kTS; ++i) {
+                    const int k = tid + i * kThreads;
+                    if (k < nt) {   // the same in every lane of a warp (nt is a multiple of 32)
+                        float v = __uint_as_float(unsigned(w[i])) * tsc;
+                        uint32_t db[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float rq = rintf(v);
+                            db[q] = (uint32_t(int(rq)) & 0xffu) << (8 * (lane & 3));
+                            v = (v - rq) * 128.f;
+                        }
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            db[q] |= __shfl_xor_sync(0xffffffffu, db[q], 1);
+                            db[q] |= __shfl_xor_sync(0xffffffffu, db[q], 2);
+                        }
+                        if ((lane & 3) == 0) {
+                            const int e = k / r, kk = k - e * r, st = kk >> 5, qd = (kk & 31) >> 2;
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                dw[(((e * nk32 + st) * 4 + q) * 4 + (qd & 3)) * 2 + (qd >> 2)] = db[q];
+                        }
+                    }
+                }
+            }
         }
         if (!__syncthreads_and(tok)) break;
         cyc_a = clock64() - ca0;
@@ -1214,59 +1277,65 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                             }
                         }
                     } else if constexpr (PF == kI8) {
-                        // tensor-core dots of signed-byte U rows: A from 32-bit shared loads
-                        // (bytes 4tq..4tq+3 of the step's 16-byte chunk, made f16 exactly);
-                        // the mma's logical columns 2tq, 2tq+1, 2tq+8, 2tq+9 stand for the
-                        // row elements 4tq .. 4tq+3, and B takes t's parts in the same order
-                        const int ntr = ntop * r;
-                        const int nks = r / 16, nmt = (n + 15) / 16;
+                        // integer tensor-core dots of signed-byte U rows: A = 16
+                        // staged rows x 32 bytes (ldmatrix; rows stored
+                        // chunk-permuted by row mod 8 when u_swz, as the 16-bit
+                        // rows), B = t's digits (column p = digit p), D exact in
+                        // int32 over the warp's k32 steps; warp w takes steps
+                        // w, w + 16, ...
+                        const int nks = r >> 5, nmt = (n + 15) / 16;
                         const int g = lane >> 2, tq = lane & 3;
-                        const uint16_t *bpart = tpart + g * ntr + e * r + 4 * tq;
+                        const int arow = lane & 15;
+                        const uint2 *bd = reinterpret_cast<const uint2 *>(sm.tsm) + size_t(e) * nks * 16 + tq;
+                        // this lane's digit columns 2 tq and 2 tq + 1: weights 2^-7p / ts
+                        const float dw0 = tq < 2 ? ldexpf(1.f, -14 * tq) / tsc : 0.f;
+                        const float dw1 = tq < 2 ? ldexpf(1.f, -14 * tq - 7) / tsc : 0.f;
                         // m-tiles per pass: eight keep a 97-row strip (F = 14336 over 148
-                        // CTAs) in one pass; the fp16-weight kernels keep six, whose
-                        // register budget their 74-row strips (F = 11008) run faster in
-                        // (measured: 2.5% per layer)
+                        // CTAs) in one pass; the fp16-weight kernels keep six
                         constexpr int kZT = MAXVW > 1 ? 4 : (WF == kF16 ? 6 : 8);
                         for (int mt0 = 0; mt0 < nmt; mt0 += kZT) {
-                            float c[kZT][4];
+                            int c[kZT][4];
 #pragma unroll
-                            for (int t = 0; t < kZT; ++t) c[t][0] = c[t][1] = c[t][2] = c[t][3] = 0.f;
+                            for (int t = 0; t < kZT; ++t) c[t][0] = c[t][1] = c[t][2] = c[t][3] = 0;
+                            int arw[kZT];
+#pragma unroll
+                            for (int t = 0; t < kZT; ++t) arw[t] = min((mt0 + t) * 16 + arow, n - 1);
+                            const uint32_t sbase = s2u(ust);
                             for (int ks = warp; ks < nks; ks += kConsumerWarps) {
-                                uint32_t b0 = 0u, b1 = 0u;
-                                if (g < 2) {
-                                    b0 = *reinterpret_cast<const uint32_t *>(bpart + ks * 16);
-                                    b1 = *reinterpret_cast<const uint32_t *>(bpart + ks * 16 + 2);
-                                }
-                                // every shared load of the step first, then conversions and MMAs
-                                uint32_t w[kZT][2];
+                                uint2 bx = make_uint2(0u, 0u);
+                                if (g < 4) bx = bd[(ks * 4 + g) * 4];
+                                const int chunk = 2 * ks + (lane >> 4);   // 16-byte chunk of the row
 #pragma unroll
-                                for (int t = 0; t < kZT; ++t) {
-                                    if (mt0 + t < nmt) {
-                                        const int r0 = min((mt0 + t) * 16 + g, n - 1);
-                                        const int r1 = min((mt0 + t) * 16 + g + 8, n - 1);
-                                        const int k0 = p.u_swz ? (r0 & 7) : 0, k1 = p.u_swz ? (r1 & 7) : 0;
-                                        w[t][0] = *reinterpret_cast<const uint32_t *>(
-                                            ust + size_t(r0) * p.urow + ((ks & ~7) | ((ks ^ k0) & 7)) * 16 + 4 * tq);
-                                        w[t][1] = *reinterpret_cast<const uint32_t *>(
-                                            ust + size_t(r1) * p.urow + ((ks & ~7) | ((ks ^ k1) & 7)) * 16 + 4 * tq);
-                                    }
-                                }
+                                for (int t0 = 0; t0 < kZT; t0 += 3) {
+                                    uint32_t a[3][4];
 #pragma unroll
-                                for (int t = 0; t < kZT; ++t) {
-                                    if (mt0 + t < nmt) {
-                                        uint32_t a0, a1, a2, a3;
-                                        i8x4_to_h2(w[t][0], a0, a2);
-                                        i8x4_to_h2(w[t][1], a1, a3);
-                                        mma16816<kF16>(c[t], a0, a1, a2, a3, b0, b1);
+                                    for (int t = t0; t < t0 + 3; ++t) {
+                                        if (t < kZT && mt0 + t < nmt) {
+                                            const int key = p.u_swz ? (arw[t] & 7) : 0;
+                                            ldsm_x4_a(sbase + uint32_t(arw[t]) * uint32_t(p.urow) +
+                                                          uint32_t(((chunk & ~7) | ((chunk ^ key) & 7)) << 4),
+                                                      a[t - t0]);
+                                        }
                                     }
+#pragma unroll
+                                    for (int t = t0; t < t0 + 3; ++t)
+                                        if (t < kZT && mt0 + t < nmt)
+                                            imma16832_acc(c[t], a[t - t0][0], a[t - t0][1], a[t - t0][2], a[t - t0][3],
+                                                          bx.x, bx.y);
                                 }
                             }
-                            // the two parts sit in columns 0 and 1 (lane 4g)
+                            // the digit columns sit in the four lanes of a quad
 #pragma unroll
                             for (int t = 0; t < kZT; ++t) {
+                                float z0 = fmaf(float(c[t][0]), dw0, float(c[t][1]) * dw1);
+                                float z1 = fmaf(float(c[t][2]), dw0, float(c[t][3]) * dw1);
+                                z0 += __shfl_xor_sync(0xffffffffu, z0, 1);
+                                z1 += __shfl_xor_sync(0xffffffffu, z1, 1);
+                                z0 += __shfl_xor_sync(0xffffffffu, z0, 2);
+                                z1 += __shfl_xor_sync(0xffffffffu, z1, 2);
                                 if (tq == 0 && mt0 + t < nmt) {
-                                    sm.zred[warp][(mt0 + t) * 16 + g] = c[t][0] + c[t][1];
-                                    sm.zred[warp][(mt0 + t) * 16 + g + 8] = c[t][2] + c[t][3];
+                                    sm.zred[warp][(mt0 + t) * 16 + g] = z0;
+                                    sm.zred[warp][(mt0 + t) * 16 + g + 8] = z1;
                                 }
                             }
                         }

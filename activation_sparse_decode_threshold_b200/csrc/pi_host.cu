@@ -138,6 +138,8 @@ pi_status pi_ffn_create(const pi_ffn_desc *desc, pi_ffn_t *out)
     const int max_rank = D.pred_dtype == PI_F32 ? 512 : 1024;
     if (D.rank < 1 || D.rank % 16 != 0 || D.rank > max_rank)
         return fail(PI_ERR_INVALID_ARG, "rank must be a multiple of 16 and <= %d", max_rank);
+    if (D.pred_dtype == PI_I8 && D.rank % 32 != 0)
+        return fail(PI_ERR_INVALID_ARG, "an I8 predictor needs rank a multiple of 32");
     if (D.n_experts == 1) {
         if (D.top_k != 1) return fail(PI_ERR_INVALID_ARG, "a dense FFN needs top_k = 1");
     } else if (D.n_experts >= 2 && D.n_experts <= pi::kMaxExperts) {

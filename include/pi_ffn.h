@@ -86,7 +86,8 @@ typedef struct {
     int d_model;         /* d: multiple of 256, <= 8192 (<= 4096 for F32) */
     int d_ff;            /* F: neurons per FFN (per expert), <= 256 * n_strips */
     int rank;            /* predictor rank r: a multiple of 16 (the tensor-core
-                            predictor dots take 16 columns per step),
+                            predictor dots take 16 columns per step; 32 for
+                            an I8 predictor, whose integer dots take 32),
                             r <= 1024 (<= 512 for F32) */
     int n_experts;       /* 1 = dense FFN; 2..16 = MoE with top-2 routing */
     int top_k;           /* 1 for a dense FFN, 2 for MoE */

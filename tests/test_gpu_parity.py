@@ -349,3 +349,12 @@ def test_vram_budget_rejections(handles):
     with pytest.raises(B.PiError) as ei:
         B.pi_dense_ffn_prefill(h2, 0, 1, 4, R)
     assert ei.value.status == B.PI_ERR_UNSUPPORTED
+
+
+def test_i8_predictor_rank_must_be_a_multiple_of_32():
+    # the 8-bit predictor's integer logits take 32 columns of U per step
+    with pytest.raises(B.PiError) as ei:
+        B.pi_ffn_create(1, 512, 1000, 48, act="reglu", w_dtype="f16", pred_dtype="i8row")
+    assert ei.value.status == B.PI_ERR_INVALID_ARG
+    h = B.pi_ffn_create(1, 512, 1000, 64, act="reglu", w_dtype="f16", pred_dtype="i8row")
+    B.pi_ffn_destroy(h)
