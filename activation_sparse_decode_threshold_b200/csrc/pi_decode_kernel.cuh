@@ -1138,12 +1138,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 if (k < nt) put_t(k, __uint_as_float(unsigned(w[i])), nt);
             }
             if constexpr (PF == kI8) {
-                // 8-bit predictor: t as signed base-128 digits for the integer
-                // logits.  The bound of |t| over the layer (the same in every
-                // CTA) gives ts = 2^(6 - e), max |t| < 2^e, so t * ts lies in
-                // (-64, 64); digit 0 is its nearest integer and each further
-                // digit the nearest integer of 128 times the remainder (every
-                // step exact; four digits leave below 2^-22 2^(e-6)).
+                // 8-bit predictor: each warp's bound of |t|, gathered through
+                // the block barrier below
                 float mx = 0.f;
 #pragma unroll
                 for (int i = 0; i < kTS; ++i)
@@ -1151,7 +1147,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
                 if (lane == 0) sm.red[rb][warp][0] = mx;
-                cta_sync();
+            }
+            if (!__syncthreads_and(tok)) break;
+            if constexpr (PF == kI8) {
+                // t as signed base-128 digits for the integer logits.  The
+                // bound of |t| over the layer (the same in every CTA) gives
+                // ts = 2^(6 - e), max |t| < 2^e, so t * ts lies in (-64, 64);
+                // digit 0 is its nearest integer and each further digit the
+                // nearest integer of 128 times the remainder (every step exact;
+                // four digits leave below 2^-22 2^(e-6)).  Adding 1.5 * 2^23
+                // rounds to the nearest integer and leaves it, two's
+                // complement, in the low byte of the sum's bits.
+                float mx = 0.f;
 #pragma unroll
                 for (int w2 = 0; w2 < kConsumerWarps; ++w2) mx = fmaxf(mx, sm.red[rb][w2][0]);
                 rb ^= 1;
@@ -1172,9 +1179,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                         uint32_t db[4];
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
-                            const float rq = rintf(v);
-                            db[q] = (uint32_t(int(rq)) & 0xffu) << (8 * (lane & 3));
-                            v = (v - rq) * 128.f;
+                            const float m = v + 12582912.f;
+                            db[q] = (__float_as_uint(m) & 0xffu) << (8 * (lane & 3));
+                            v = (v - (m - 12582912.f)) * 128.f;
                         }
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
@@ -1191,7 +1198,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 }
             }
         }
-        if (!__syncthreads_and(tok)) break;
+
         cyc_a = clock64() - ca0;
         prof_put(p, li, 1, gtimer());
 
