@@ -956,7 +956,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 pending = false;
             }
             if (row0 == a0 && lip >= 0) prof_put(p, lip, 19, gtimer());
-            // routed: the experts' U strips (needed after the barrier) start
+            // routed: the experts' U strips (needed at the layer's start) start
             // moving towards L2 once the first V rows have landed, issued by a
             // thread that neither polls nor releases a grid barrier
             if (moe && row0 == a0 && tid == kThreads - 32 && ns > 0)
