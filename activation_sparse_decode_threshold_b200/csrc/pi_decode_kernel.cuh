@@ -308,21 +308,6 @@ __device__ __forceinline__ void split_parts(float x, int nparts, uint16_t *out, 
     }
 }
 
-// Four signed bytes (byte j = element j) as two f16x2 values, exactly: each
-// byte is biased to unsigned, placed in the mantissa of 1024 (0x6400 | u is
-// 1024 + u in binary16) and 1024 + 128 is subtracted.
-__device__ __forceinline__ void i8x4_to_h2(uint32_t w, uint32_t &lo, uint32_t &hi)
-{
-    const uint32_t u = w ^ 0x80808080u;
-    const uint32_t a = __byte_perm(u, 0x64646464u, 0x7170);
-    const uint32_t b = __byte_perm(u, 0x64646464u, 0x7372);
-    const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));   // 1152
-    const __half2 ha = __hsub2(*reinterpret_cast<const __half2 *>(&a), bias);
-    const __half2 hb = __hsub2(*reinterpret_cast<const __half2 *>(&b), bias);
-    lo = *reinterpret_cast<const uint32_t *>(&ha);
-    hi = *reinterpret_cast<const uint32_t *>(&hb);
-}
-
 // Eight INT4 codes (nibble i of w = element i, code n_i, value n_i - 8) as
 // signed bytes 16 (n_i - 8), exactly: flipping a nibble's top bit gives the
 // value in 4-bit two's complement, and moving it to the top of a byte scales
