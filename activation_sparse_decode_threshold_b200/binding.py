@@ -24,6 +24,7 @@ ACT = {"relu": 0, "reglu": 1, "drelu": 2}
 DTYPE = {"f32": 0, "f16": 1, "bf16": 2, "int4g32": 3, "i8row": 4}
 PI_DEBUG_STALL_BARRIER = 1
 PI_DEBUG_STALL_PREFILL = 2
+PI_DEBUG_STALL_T_POLL = 8
 
 
 class PiError(RuntimeError):

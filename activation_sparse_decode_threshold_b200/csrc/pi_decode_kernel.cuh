@@ -1091,7 +1091,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             constexpr int kTS = kMaxRankTotal / kThreads;
             static_assert(kTS * kThreads == kMaxRankTotal && kTS <= 32, "whole slots per thread");
             const int nt = ntop * r;
-            const unsigned tg = unsigned(l - l0 + 1);
+            // (PI_DEBUG_STALL_T_POLL: a tag that no layer writes)
+            const unsigned tg = unsigned(l - l0 + 1) + ((p.debug_flags & 8) ? 0x40000000u : 0u);
             unsigned long long w[kTS];
             unsigned need = 0;
 #pragma unroll

@@ -285,14 +285,18 @@ PI_API void pi_ffn_destroy(pi_ffn_t h);
 /* Testing aid: bound every device-side wait of this handle (decode and
  * prefill kernels) by `wait_limit_s` seconds (default 2.0).  With flags &
  * PI_DEBUG_STALL_BARRIER, the decode kernel's first grid barrier waits for one
- * arrival that never comes; with flags & PI_DEBUG_STALL_PREFILL, one producer
- * thread of the first prefill gate/up GEMM tile never publishes its first
- * stage, so the tensor-core issuer's bounded wait runs out before it issues
- * any MMA.  Either way the wait runs out, the kernel releases what it holds
- * (in-flight copies, tensor memory) and returns, and pi_sync reports
- * PI_ERR_TIMEOUT; the handle stays usable. */
+ * arrival that never comes; with flags & PI_DEBUG_STALL_T_POLL, every CTA of
+ * the decode kernel polls the rows of t of its first layer for a tag that no
+ * CTA writes; with flags & PI_DEBUG_STALL_PREFILL, one producer thread of the
+ * first prefill gate/up GEMM tile never publishes its first stage, so the
+ * tensor-core issuer's bounded wait runs out before it issues any MMA.  Either
+ * way the wait runs out, the kernel releases what it holds (in-flight copies,
+ * tensor memory) and returns, and pi_sync reports PI_ERR_TIMEOUT; the handle
+ * stays usable.  (Flag 4 is taken: each CTA gathers its own strip's active
+ * neurons, without the balance step.) */
 #define PI_DEBUG_STALL_BARRIER 1
 #define PI_DEBUG_STALL_PREFILL 2
+#define PI_DEBUG_STALL_T_POLL 8
 PI_API pi_status pi_debug_set(pi_ffn_t h, int flags, double wait_limit_s);
 
 /* Testing aid: when `times_dev` is non-NULL, each later pi_sparse_ffn_decode

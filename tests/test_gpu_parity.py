@@ -205,11 +205,14 @@ def test_identity_table_gives_same_result_within_rounding(handles):
     G.check_output(a - r0.double().numpy(), b - r0.double().numpy())
 
 
-def test_bounded_wait_reports_timeout_and_context_survives(handles):
+@pytest.mark.parametrize("flag", ["PI_DEBUG_STALL_BARRIER", "PI_DEBUG_STALL_T_POLL"])
+def test_bounded_wait_reports_timeout_and_context_survives(handles, flag):
+    # a grid barrier that misses one arrival, or a poll of the rows of t for a
+    # tag that no CTA writes: the bounded wait runs out, the kernel returns
     cfg = SMALL["reglu-f16"]
     h, _ = _build(cfg, handles, n_layers=1)
     r = synth.token_input(cfg, 0).cuda()
-    B.pi_debug_set(h, B.PI_DEBUG_STALL_BARRIER, 0.05)
+    B.pi_debug_set(h, getattr(B, flag), 0.05)
     B.pi_sparse_ffn_decode(h, 0, 1, r.clone())
     assert B.pi_sync(h) == B.PI_ERR_TIMEOUT
     B.pi_debug_set(h, 0, 2.0)
