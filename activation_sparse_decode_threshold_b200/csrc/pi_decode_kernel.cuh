@@ -15,9 +15,10 @@
 //   [C] for the active neurons of its share: the neuron's record (W_gate /
 //       W_up rows, plus its W_down row for ReLU / ReGLU, where h != 0 almost
 //       always follows z > 0) by bulk copy into shared memory -> h =
-//       act(g, u); for h != 0 its W_down column (stored as a row) accumulates
-//       into a per-CTA fp32 partial of y ("Neuron-aware operators": rows of
-//       the input matrices, columns of the output matrix).
+//       act(g, u) (INT4 records: dots on the integer tensor cores with x as
+//       base-128 digits); for h != 0 its W_down column (stored as a row)
+//       accumulates into a per-CTA fp32 partial of y ("Neuron-aware
+//       operators": rows of the input matrices, columns of the output matrix).
 //   [merge] each CTA's partial, rounded to 64-bit fixed point, is added into
 //       the layer's total by one bulk reduction in L2 (integer adds: the total
 //       does not depend on arrival order; the merge of partial results,
@@ -25,14 +26,15 @@
 //   --- grid barrier ---
 //   [next input] every CTA reads the whole total and forms the whole next
 //       input r + y, its sum of squares and x = RMSNorm(r + y) in the same
-//       order (so every CTA holds the same x); its own rows of t = V x for
-//       layer l + 1 go to global memory, its columns of r + y to the next
-//       input buffer.
-//   --- grid barrier ---
+//       order (so every CTA holds the same x); its columns of r + y go to the
+//       next input buffer, its own rows of t = V x for layer l + 1 to every
+//       CTA as tagged 64-bit slots (value and layer tag in one store), which
+//       the next layer's start polls instead of a grid barrier.
 //
-// Three grid barriers per layer.  A routed (MoE) layer picks its two experts
-// in the [next input] step from router logits every CTA computes from its own
-// copy of x, and its rows of t then come from the chosen experts' V.
+// Two grid barriers per layer.  A routed (MoE) layer adds each CTA's column
+// share of the router logits into 64-bit fixed-point totals in the [next
+// input] step, passes a third grid barrier, picks its two experts the same
+// way in every CTA, and takes its rows of t from the chosen experts' V.
 //
 // Memory: weight bytes are pulled towards the SM as soon as their addresses
 // are known.  A strip's active records are prefetched into L2 the moment its
