@@ -48,6 +48,7 @@ def _desc(**kw):
     (dict(w_dtype=0, pred_dtype=0, rank=1024), B.PI_ERR_INVALID_ARG),   # fp32 rows hold <= 512
     (dict(w_dtype=3, pred_dtype=0), B.PI_ERR_UNSUPPORTED),              # INT4 with an fp32 predictor
     (dict(n_experts=8, top_k=2, w_dtype=0, pred_dtype=0, rank=256), B.PI_ERR_UNSUPPORTED),
+    (dict(pred_dtype=4, rank=1008), B.PI_ERR_INVALID_ARG),   # the 8-bit predictor takes 32 columns per step
 ])
 def test_create_rejects_bad_descriptors_on_host(bad, status):
     h = ctypes.c_void_p()
