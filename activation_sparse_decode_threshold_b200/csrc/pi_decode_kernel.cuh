@@ -1285,9 +1285,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                         // this lane's digit columns 2 tq and 2 tq + 1: weights 2^-7p / ts
                         const float dw0 = tq < 2 ? ldexpf(1.f, -14 * tq) / tsc : 0.f;
                         const float dw1 = tq < 2 ? ldexpf(1.f, -14 * tq - 7) / tsc : 0.f;
-                        // m-tiles per pass: eight keep a 97-row strip (F = 14336 over 148
-                        // CTAs) in one pass; the fp16-weight kernels keep six
-                        constexpr int kZT = MAXVW > 1 ? 4 : (WF == kF16 ? 6 : 8);
+                        // m-tiles per pass: seven keep a 97-row strip (F = 14336 over 148
+                        // CTAs) in one pass; the fp16-weight kernels keep five (74-row
+                        // strips, F = 11008)
+                        constexpr int kZT = MAXVW > 1 ? 4 : (WF == kF16 ? 5 : 7);
                         for (int mt0 = 0; mt0 < nmt; mt0 += kZT) {
                             int c[kZT][4];
 #pragma unroll
@@ -1362,11 +1363,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                         const int arow = lane & 15;                       // row within an m-tile
                         const uint16_t *bpart = tpart + g * ntr + e * r + 2 * tq;
                         // m-tiles in passes of kZT (bounded accumulator registers)
-                        // m-tiles per pass: eight keep a 97-row strip (F = 14336 over 148
-                        // CTAs) in one pass; the fp16-weight kernels keep six, whose
-                        // register budget their 74-row strips (F = 11008) run faster in
-                        // (measured: 2.5% per layer)
-                        constexpr int kZT = MAXVW > 1 ? 4 : (WF == kF16 ? 6 : 8);
+                        // m-tiles per pass: seven keep a 97-row strip (F = 14336 over 148
+                        // CTAs) in one pass; the fp16-weight kernels keep five, exactly
+                        // their 74-row strips (F = 11008): accumulators for tiles a strip
+                        // does not have cost registers (measured: 0.5-0.8% per layer
+                        // against eight and six)
+                        constexpr int kZT = MAXVW > 1 ? 4 : (WF == kF16 ? 5 : 7);
                         for (int mt0 = 0; mt0 < nmt; mt0 += kZT) {
                             float c[kZT][4];
 #pragma unroll
