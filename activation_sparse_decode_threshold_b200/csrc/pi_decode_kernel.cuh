@@ -377,7 +377,7 @@ __device__ __forceinline__ float act_h(int act, float g, float u)
 constexpr int kRA = 16;           // V rows per staging round at most
 constexpr int kZRows = 112;       // U rows per staging round at most (a multiple of 16)
 constexpr int kMaxU = 4;          // U vectors per lane (rank <= 128 * EPV)
-constexpr int kRound = 16;        // neurons per gather round at most
+constexpr int kRound = 20;        // neurons per gather round at most (a routed strip share of ~19 in one round)
 constexpr int kIssue = 32;        // neurons whose records are in flight at once at most
 static_assert(kRound <= 32, "a round's neurons are tracked in one warp ballot");
 constexpr int kRed = 2 * kRound;  // values reduced per warp at most
