@@ -949,9 +949,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             if (moe && row0 == a0 && tid == kThreads - 32 && ns > 0)
                 for (int e = 0; e < ntop; ++e)
                     prefetch_l2(sm.exl[ln & 1][e].U + size_t(s0) * p.urow, uint32_t(ns) * p.urow);
-            // four rows at a time; after the reduction lanes 8q .. 8q + 7 hold
-            // row g + q of the round
-#pragma unroll 1
+            // four rows at a time, two groups of four in flight; after the
+            // reduction lanes 8q .. 8q + 7 hold row g + q of the round
+#pragma unroll 2
             for (int g = 0; g < n; g += 4) {
                 float part[4];
 #pragma unroll
